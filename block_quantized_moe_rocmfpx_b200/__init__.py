@@ -1,0 +1,219 @@
+"""B200 (sm_100a) block-quantised MoE FFN: thin Python binding of ``librfx.so``.
+
+Argument marshalling only: every step of the hot path runs in the library's
+CUDA kernels (``csrc/``); PyTorch supplies device memory and streams.  The
+binding keeps the C ABI's names (``include/rfx.h``).  There is no CPU fallback:
+importing fails if the library is missing and every call raises on a non-OK
+status.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librfx.so")
+
+RFX_OK, RFX_EINVAL, RFX_EUNSUPPORTED, RFX_ECUDA, RFX_EDEVICE, RFX_ERANGE = 0, -1, -2, -3, -4, -5
+RFX_FP2, RFX_FP3, RFX_FP4 = 2, 3, 4
+MAX_T = 8
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m block_quantized_moe_rocmfpx_b200.build` "
+                      "(nvcc, sm_100a); there is no fallback implementation")
+
+_lib = ctypes.CDLL(LIB_PATH)
+_i32, _i64, _sz, _vp = ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p
+
+
+class moe_layer_desc(ctypes.Structure):
+    _fields_ = [("H", _i32), ("I", _i32), ("E", _i32), ("k", _i32),
+                ("f_gate", _i32), ("f_up", _i32), ("f_down", _i32),
+                ("gate", _vp), ("up", _vp), ("down", _vp),
+                ("stride_gate", _sz), ("stride_up", _sz), ("stride_down", _sz),
+                ("has_shared", _i32),
+                ("f_sh_gate", _i32), ("f_sh_up", _i32), ("f_sh_down", _i32),
+                ("sh_gate", _vp), ("sh_up", _vp), ("sh_down", _vp)]
+
+
+def _proto(name, res, args):
+    f = getattr(_lib, name)
+    f.restype = res
+    f.argtypes = args
+    return f
+
+
+_lib_last_error = _proto("rfx_last_error", ctypes.c_char_p, [])
+_packed_bytes = _proto("rfx_packed_bytes", _sz, [_i32, _i64, _i64])
+_pack = _proto("rfx_pack", _i32, [_i32, _vp, _vp, _i64, _i64, _vp, _sz])
+_unpack = _proto("rfx_unpack", _i32, [_i32, _vp, _i64, _i64, _vp, _vp])
+_pack_device = _proto("rfx_pack_device", _i32, [_i32, _vp, _vp, _i64, _i64, _vp, _vp])
+_router = _proto("moe_router_topk", _i32, [_vp, _i32, _i32, _i32, _vp, _vp, _vp])
+_gemv = _proto("rfx_gemv_q", _i32, [_i32, _vp, _i64, _i64, _vp, _i32, _i32, _vp, _vp])
+_layer_create = _proto("moe_layer_create", _i32, [ctypes.POINTER(moe_layer_desc), ctypes.POINTER(_vp)])
+_layer_destroy = _proto("moe_layer_destroy", None, [_vp])
+_ws_bytes = _proto("moe_ffn_workspace_bytes", _sz, [_vp, _i32])
+_ws_init = _proto("rfx_ws_init", _i32, [_vp, _sz, _vp])
+_ws_status = _proto("rfx_ws_status", _i32, [_vp, _vp])
+_forward = _proto("moe_ffn_forward", _i32, [_vp, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp])
+
+EXPORTED = ["rfx_last_error", "rfx_packed_bytes", "rfx_pack", "rfx_unpack", "rfx_pack_device", "moe_router_topk",
+            "rfx_gemv_q", "moe_layer_create", "moe_layer_destroy", "moe_ffn_workspace_bytes", "rfx_ws_init",
+            "rfx_ws_status", "moe_ffn_forward"]
+
+
+class RfxError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"rfx status {code}: {msg}")
+        self.code = code
+
+
+def rfx_last_error() -> str:
+    return _lib_last_error().decode()
+
+
+def _check(rc: int):
+    if rc != RFX_OK:
+        raise RfxError(rc, rfx_last_error())
+
+
+def _ptr(t) -> int | None:
+    """Device pointer of a torch tensor, host pointer of a numpy array, or an int."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if isinstance(t, np.ndarray):
+        return t.ctypes.data
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+# ------------------------------------------------------------------ format ---
+
+def rfx_packed_bytes(fmt: int, rows: int, cols: int) -> int:
+    return int(_packed_bytes(fmt, rows, cols))
+
+
+def rfx_pack(fmt: int, codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    rows, cols = codes.shape
+    scales = np.ascontiguousarray(scales, dtype=np.uint8 if fmt == RFX_FP4 else np.uint16)
+    out = np.empty(rfx_packed_bytes(fmt, rows, cols), dtype=np.uint8)
+    _check(_pack(fmt, _ptr(codes), _ptr(scales), rows, cols, _ptr(out), out.nbytes))
+    return out
+
+
+def rfx_unpack(fmt: int, packed: np.ndarray, rows: int, cols: int):
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    codes = np.empty((rows, cols), dtype=np.uint8)
+    scales = np.empty((rows, cols // 32), dtype=np.uint8 if fmt == RFX_FP4 else np.uint16)
+    _check(_unpack(fmt, _ptr(packed), rows, cols, _ptr(codes), _ptr(scales)))
+    return codes, scales
+
+
+def rfx_pack_device(fmt: int, codes, scales, rows: int, cols: int, dst, stream=None):
+    """Pack device arrays (torch uint8 codes [rows][cols], scales) into device dst."""
+    _check(_pack_device(fmt, _ptr(codes), _ptr(scales), rows, cols, _ptr(dst), _stream(stream)))
+
+
+# ---------------------------------------------------------------- kernels ---
+
+def moe_router_topk(logits, k: int, idx, w, stream=None):
+    """logits fp32 [T][E] (device) -> idx int32 [T][k], w fp32 [T][k] (device, preallocated)."""
+    T, E = logits.shape
+    _check(_router(_ptr(logits), T, E, k, _ptr(idx), _ptr(w), _stream(stream)))
+
+
+def rfx_gemv_q(fmt: int, W, N: int, K: int, x, y, stream=None):
+    """y fp32 [q][N] = dequant(W) x for x bf16 [q][K] or fp32 [q][K] (device tensors)."""
+    import torch
+    q = x.shape[0]
+    x_is_fp32 = 1 if x.dtype == torch.float32 else 0
+    _check(_gemv(fmt, _ptr(W), N, K, _ptr(x), x_is_fp32, q, _ptr(y), _stream(stream)))
+
+
+def moe_layer_create(desc: moe_layer_desc) -> int:
+    h = _vp()
+    _check(_layer_create(ctypes.byref(desc), ctypes.byref(h)))
+    return h.value
+
+
+def moe_layer_destroy(handle: int):
+    _layer_destroy(handle)
+
+
+def moe_ffn_workspace_bytes(handle: int, T: int) -> int:
+    return int(_ws_bytes(handle, T))
+
+
+def rfx_ws_init(ws, stream=None):
+    _check(_ws_init(_ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def rfx_ws_status(ws, stream=None) -> int:
+    rc = int(_ws_status(_ptr(ws), _stream(stream)))
+    return rc
+
+
+def moe_ffn_forward(handle: int, x, T: int, idx, w, y, ws, stream=None):
+    _check(_forward(handle, _ptr(x), T, _ptr(idx), _ptr(w), _ptr(y), _ptr(ws), ws.numel() * ws.element_size(),
+                    _stream(stream)))
+
+
+# --------------------------------------------------------- convenience ---
+
+class MoeLayer:
+    """One MoE layer over caller-owned packed device buffers.
+
+    ``gate``/``up``/``down`` are uint8 device tensors holding E packed experts
+    at a fixed stride; ``shared`` is (gate, up, down) or None.  Creates the
+    host handle and a zeroed workspace for up to ``max_T`` token columns.
+    """
+
+    def __init__(self, H, I, E, k, fmts, gate, up, down, strides, shared=None, shared_fmts=(4, 4, 4), max_T=MAX_T):
+        import torch
+        self.H, self.I, self.E, self.k = H, I, E, k
+        self._keep = [gate, up, down] + (list(shared) if shared else [])
+        d = moe_layer_desc()
+        d.H, d.I, d.E, d.k = H, I, E, k
+        d.f_gate, d.f_up, d.f_down = fmts
+        d.gate, d.up, d.down = _ptr(gate), _ptr(up), _ptr(down)
+        d.stride_gate, d.stride_up, d.stride_down = strides
+        d.has_shared = 1 if shared else 0
+        if shared:
+            d.f_sh_gate, d.f_sh_up, d.f_sh_down = shared_fmts
+            d.sh_gate, d.sh_up, d.sh_down = (_ptr(s) for s in shared)
+        self.desc = d
+        self.handle = moe_layer_create(d)
+        self.max_T = max_T
+        nbytes = moe_ffn_workspace_bytes(self.handle, max_T)
+        self.ws = torch.empty(nbytes, dtype=torch.uint8, device=gate.device)
+        rfx_ws_init(self.ws)
+
+    def forward(self, x, idx, w, y, stream=None):
+        T = x.shape[0]
+        if T > self.max_T:
+            raise ValueError(f"T={T} > max_T={self.max_T}")
+        moe_ffn_forward(self.handle, x, T, idx, w, y, self.ws, stream)
+
+    def status(self, stream=None) -> int:
+        return rfx_ws_status(self.ws, stream)
+
+    def __del__(self):
+        try:
+            if getattr(self, "handle", None):
+                moe_layer_destroy(self.handle)
+                self.handle = None
+        except Exception:
+            pass

@@ -1,0 +1,199 @@
+// api.cu -- C ABI entry points (include/rfx.h): argument checks, workspace
+// layout and kernel launches.  No entry point allocates device memory.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstring>
+#include <new>
+#include <string>
+
+#include "../../include/rfx.h"
+#include "gemv.h"
+#include "moe_decode.h"
+#include "rfx_layout.h"
+
+int rfx_fail(int code, const std::string& msg);  // rfx_pack.cpp
+
+struct moe_layer {
+    moe_layer_desc d;
+};
+
+namespace {
+
+bool fmt_ok(int f) { return f == 2 || f == 3 || f == 4; }
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+int cuda_fail(const char* where, cudaError_t e) {
+    return rfx_fail(RFX_ECUDA, std::string(where) + ": " + cudaGetErrorString(e));
+}
+
+int device_props(int& sms, int& smem_optin) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail("cudaDeviceGetAttribute", e);
+    e = cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e != cudaSuccess) return cuda_fail("cudaDeviceGetAttribute", e);
+    return RFX_OK;
+}
+
+}  // namespace
+
+extern "C" int rfx_pack_device(rfx_format f, const uint8_t* codes, const void* scales, int64_t rows, int64_t cols,
+                               void* dst, void* stream) {
+    if (!fmt_ok(f)) return rfx_fail(RFX_EINVAL, "rfx_pack_device: bad format");
+    if (rows < 0 || cols <= 0 || cols % 32 != 0) return rfx_fail(RFX_EINVAL, "rfx_pack_device: bad shape");
+    if (rows > 65535LL * 16) return rfx_fail(RFX_EUNSUPPORTED, "rfx_pack_device: more than 1048560 rows");
+    if (rows == 0) return RFX_OK;
+    if (!codes || !scales || !dst) return rfx_fail(RFX_EINVAL, "rfx_pack_device: null pointer");
+    cudaError_t e = rfx::pack_device_launch(f, codes, scales, rows, cols, (uint8_t*)dst, (cudaStream_t)stream);
+    return e == cudaSuccess ? RFX_OK : cuda_fail("rfx_pack_device", e);
+}
+
+extern "C" int moe_router_topk(const float* logits, int T, int E, int k, int32_t* idx, float* w, void* stream) {
+    if (T < 0 || E < 1 || E > 1024 || k < 1 || k > E || k > 16)
+        return rfx_fail(RFX_EINVAL, "moe_router_topk: need T >= 0, 1 <= E <= 1024, 1 <= k <= min(E, 16)");
+    if (T == 0) return RFX_OK;
+    if (!logits || !idx || !w) return rfx_fail(RFX_EINVAL, "moe_router_topk: null pointer");
+    cudaError_t e = rfx::router_topk_launch(logits, T, E, k, idx, w, (cudaStream_t)stream);
+    return e == cudaSuccess ? RFX_OK : cuda_fail("moe_router_topk", e);
+}
+
+extern "C" int rfx_gemv_q(rfx_format f, const void* W, int64_t N, int64_t K, const void* x, int x_is_fp32, int q,
+                          float* y, void* stream) {
+    if (!fmt_ok(f)) return rfx_fail(RFX_EINVAL, "rfx_gemv_q: bad format");
+    if (N < 1 || K < 32 || K % 32 != 0) return rfx_fail(RFX_EINVAL, "rfx_gemv_q: need N >= 1 and K a positive multiple of 32");
+    if (q < 1 || q > 8) return rfx_fail(RFX_EUNSUPPORTED, "rfx_gemv_q: 1 <= q <= 8");
+    if (!W || !x || !y) return rfx_fail(RFX_EINVAL, "rfx_gemv_q: null pointer");
+    if (!aligned16(W)) return rfx_fail(RFX_EINVAL, "rfx_gemv_q: W must be 16-byte aligned");
+    if (((uintptr_t)x & 3u) != 0) return rfx_fail(RFX_EINVAL, "rfx_gemv_q: x must be 4-byte aligned");
+    int sms = 0, smem_optin = 0;
+    int rc = device_props(sms, smem_optin);
+    if (rc != RFX_OK) return rc;
+    if (rfx::gemv_smem_bytes(q, K, x_is_fp32 != 0) > (size_t)smem_optin)
+        return rfx_fail(RFX_EUNSUPPORTED, "rfx_gemv_q: q*K too large for the shared-memory copy of x");
+    if ((N + 15) / 16 > 2LL * 2147483647LL) return rfx_fail(RFX_EUNSUPPORTED, "rfx_gemv_q: N too large");
+    rfx::GemvParams p{(const uint8_t*)W, N, K, x, q, y};
+    cudaError_t e = rfx::gemv_launch(p, f, x_is_fp32 != 0, (cudaStream_t)stream);
+    return e == cudaSuccess ? RFX_OK : cuda_fail("rfx_gemv_q", e);
+}
+
+extern "C" int moe_layer_create(const moe_layer_desc* d, moe_layer** out) {
+    if (!d || !out) return rfx_fail(RFX_EINVAL, "moe_layer_create: null pointer");
+    *out = nullptr;
+    if (d->H < 32 || d->I < 32 || d->H % 32 || d->I % 32)
+        return rfx_fail(RFX_EINVAL, "moe_layer_create: H and I must be positive multiples of 32");
+    if (d->E < 1 || d->E > 1024 || d->k < 1 || d->k > d->E || d->k > MOE_MAXK)
+        return rfx_fail(RFX_EINVAL, "moe_layer_create: need 1 <= k <= min(E, 8), E <= 1024");
+    if (!fmt_ok(d->f_gate) || !fmt_ok(d->f_up) || !fmt_ok(d->f_down))
+        return rfx_fail(RFX_EINVAL, "moe_layer_create: bad routed format");
+    if (d->f_gate != d->f_up) return rfx_fail(RFX_EUNSUPPORTED, "moe_layer_create: gate and up must share a format");
+    if (!d->gate || !d->up || !d->down) return rfx_fail(RFX_EINVAL, "moe_layer_create: null routed pointer");
+    if (!aligned16(d->gate) || !aligned16(d->up) || !aligned16(d->down) || d->stride_gate % 16 ||
+        d->stride_up % 16 || d->stride_down % 16)
+        return rfx_fail(RFX_EINVAL, "moe_layer_create: routed bases and strides must be 16-byte aligned");
+    if (d->stride_gate < rfx_packed_bytes(d->f_gate, d->I, d->H) || d->stride_up < rfx_packed_bytes(d->f_up, d->I, d->H) ||
+        d->stride_down < rfx_packed_bytes(d->f_down, d->H, d->I))
+        return rfx_fail(RFX_EINVAL, "moe_layer_create: expert stride smaller than the packed matrix");
+    if (d->has_shared) {
+        if (!fmt_ok(d->f_sh_gate) || !fmt_ok(d->f_sh_up) || !fmt_ok(d->f_sh_down))
+            return rfx_fail(RFX_EINVAL, "moe_layer_create: bad shared format");
+        if (d->f_sh_gate != d->f_sh_up)
+            return rfx_fail(RFX_EUNSUPPORTED, "moe_layer_create: shared gate and up must share a format");
+        if (!d->sh_gate || !d->sh_up || !d->sh_down) return rfx_fail(RFX_EINVAL, "moe_layer_create: null shared pointer");
+        if (!aligned16(d->sh_gate) || !aligned16(d->sh_up) || !aligned16(d->sh_down))
+            return rfx_fail(RFX_EINVAL, "moe_layer_create: shared pointers must be 16-byte aligned");
+    }
+    moe_layer* L = new (std::nothrow) moe_layer;
+    if (!L) return rfx_fail(RFX_EINVAL, "moe_layer_create: out of host memory");
+    L->d = *d;
+    *out = L;
+    return RFX_OK;
+}
+
+extern "C" void moe_layer_destroy(moe_layer* layer) { delete layer; }
+
+extern "C" size_t moe_ffn_workspace_bytes(const moe_layer* layer, int T) {
+    if (!layer || T < 1 || T > MOE_MAXT) return 0;
+    return rfx::moe_ws_layout(T, layer->d.k, layer->d.H, layer->d.I).total;
+}
+
+extern "C" int rfx_ws_init(void* ws, size_t ws_bytes, void* stream) {
+    if (!ws) return rfx_fail(RFX_EINVAL, "rfx_ws_init: null workspace");
+    cudaError_t e = cudaMemsetAsync(ws, 0, ws_bytes, (cudaStream_t)stream);
+    return e == cudaSuccess ? RFX_OK : cuda_fail("rfx_ws_init", e);
+}
+
+extern "C" int rfx_ws_status(void* ws, void* stream) {
+    if (!ws) return rfx_fail(RFX_EINVAL, "rfx_ws_status: null workspace");
+    uint32_t err = 0;
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail("rfx_ws_status", e);
+    e = cudaMemcpy(&err, (uint32_t*)ws + MOE_CTRL_ERR, 4, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail("rfx_ws_status", e);
+    if (err) {
+        uint32_t zero = 0;
+        e = cudaMemcpy((uint32_t*)ws + MOE_CTRL_ERR, &zero, 4, cudaMemcpyHostToDevice);
+        if (e != cudaSuccess) return cuda_fail("rfx_ws_status", e);
+    }
+    if (err & MOE_ERR_TIMEOUT) return rfx_fail(RFX_EDEVICE, "device: a bounded wait timed out");
+    if (err & (MOE_ERR_EXPERT | MOE_ERR_DUP))
+        return rfx_fail(RFX_EDEVICE, "device: expert id out of range or repeated within a token column");
+    if (err & MOE_ERR_RANGE) return rfx_fail(RFX_ERANGE, "device: SwiGLU output beyond the binary16 range");
+    return RFX_OK;
+}
+
+namespace rfx {
+
+// Fill launch parameters for T columns; returns RFX_OK or an error.
+int moe_prepare(const moe_layer* layer, const void* x, int T, const int32_t* idx, const float* w, float* y, void* ws,
+                size_t ws_bytes, MoeParams& p, int& grid, size_t& smem) {
+    if (!layer) return rfx_fail(RFX_EINVAL, "moe_ffn_forward: null layer");
+    const moe_layer_desc& d = layer->d;
+    if (T < 1 || T > MOE_MAXT) return rfx_fail(RFX_EUNSUPPORTED, "moe_ffn_forward: 1 <= T <= 8 token columns");
+    if (!x || !idx || !w || !y || !ws) return rfx_fail(RFX_EINVAL, "moe_ffn_forward: null pointer");
+    if (((uintptr_t)x & 3u) || ((uintptr_t)ws & 255u))
+        return rfx_fail(RFX_EINVAL, "moe_ffn_forward: x must be 4-byte and ws 256-byte aligned");
+    const MoeWs L = moe_ws_layout(T, d.k, d.H, d.I);
+    if (ws_bytes < L.total) return rfx_fail(RFX_EINVAL, "moe_ffn_forward: workspace smaller than moe_ffn_workspace_bytes");
+    int sms = 0, smem_optin = 0;
+    int rc = device_props(sms, smem_optin);
+    if (rc != RFX_OK) return rc;
+    p.H = d.H; p.I = d.I; p.E = d.E; p.k = d.k; p.T = T;
+    p.fA = d.f_gate; p.fB = d.f_down;
+    p.fsA = d.has_shared ? d.f_sh_gate : 2;
+    p.fsB = d.has_shared ? d.f_sh_down : 2;
+    p.gate = (const uint8_t*)d.gate; p.up = (const uint8_t*)d.up; p.down = (const uint8_t*)d.down;
+    p.sg = (long long)d.stride_gate; p.su = (long long)d.stride_up; p.sd = (long long)d.stride_down;
+    p.has_shared = d.has_shared ? 1 : 0;
+    p.shg = (const uint8_t*)d.sh_gate; p.shu = (const uint8_t*)d.sh_up; p.shd = (const uint8_t*)d.sh_down;
+    p.x = (const uint16_t*)x; p.idx = idx; p.wts = w; p.y = y;
+    uint8_t* wsb = (uint8_t*)ws;
+    p.ctrl = (uint32_t*)(wsb + L.ctrl_off);
+    p.hbuf = (uint16_t*)(wsb + L.h_off);
+    p.dpart = (float*)(wsb + L.d_off);
+    p.x_stride = d.H / 16 * 32 + 32;
+    const size_t xb = (size_t)T * p.x_stride, hb = 2 * (size_t)4 * T * d.I;
+    p.xh_bytes = (int)((std::max(xb, hb) + 127) / 128 * 128);
+    p.ns = 0;
+    for (int ns = MOE_MAX_STAGES; ns >= 2; --ns)
+        if (moe_decode_smem_bytes(ns, p.xh_bytes) <= (size_t)smem_optin) { p.ns = ns; break; }
+    if (!p.ns) return rfx_fail(RFX_EUNSUPPORTED, "moe_ffn_forward: shapes need more shared memory than the device has");
+    smem = moe_decode_smem_bytes(p.ns, p.xh_bytes);
+    grid = sms;
+    return RFX_OK;
+}
+
+}  // namespace rfx
+
+extern "C" int moe_ffn_forward(const moe_layer* layer, const void* x, int T, const int32_t* idx, const float* w,
+                               float* y, void* ws, size_t ws_bytes, void* stream) {
+    rfx::MoeParams p;
+    int grid = 0;
+    size_t smem = 0;
+    int rc = rfx::moe_prepare(layer, x, T, idx, w, y, ws, ws_bytes, p, grid, smem);
+    if (rc != RFX_OK) return rc;
+    cudaError_t e = rfx::moe_decode_launch(p, grid, (cudaStream_t)stream);
+    return e == cudaSuccess ? RFX_OK : cuda_fail("moe_ffn_forward", e);
+}

@@ -1,0 +1,71 @@
+// moe_decode.h -- launch parameters and workspace layout of the MoE decode /
+// verify kernel (moe_decode.cu).
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#define MOE_MAXT 8            // token columns per call (decode / verify)
+#define MOE_MAXK 8            // routed experts per token
+#define MOE_MAXS (MOE_MAXT * MOE_MAXK + 1)
+#define MOE_MAX_STAGES 6
+#define MOE_STAGE_BYTES 4352  // two full FP4 chunks (gate + up)
+
+// workspace control words (uint32)
+#define MOE_CTRL_TASK 0
+#define MOE_CTRL_EXIT 1
+#define MOE_CTRL_ERR 2
+#define MOE_CTRL_SLOT 8
+#define MOE_CTRL_ROWBLK (MOE_CTRL_SLOT + MOE_MAXS + 7)
+
+// device error bits
+#define MOE_ERR_EXPERT 1u
+#define MOE_ERR_DUP 2u
+#define MOE_ERR_TIMEOUT 4u
+#define MOE_ERR_RANGE 8u
+
+namespace rfx {
+
+struct MoeParams {
+    int H, I, E, k, T;
+    int fA, fB, fsA, fsB;  // routed gate/up, routed down, shared gate/up, shared down formats
+    const uint8_t* gate;
+    const uint8_t* up;
+    const uint8_t* down;
+    long long sg, su, sd;  // routed expert strides (bytes)
+    int has_shared;
+    const uint8_t* shg;
+    const uint8_t* shu;
+    const uint8_t* shd;
+    const uint16_t* x;     // bf16 [T][H]
+    const int32_t* idx;    // [T][k]
+    const float* wts;      // [T][k]
+    float* y;              // [T][H]
+    uint32_t* ctrl;
+    uint16_t* hbuf;        // fp16 [MAXS_T][2*T*I]
+    float* dpart;          // fp32 [MAXS_T][T][H]
+    int ns;                // stages per consumer warp
+    int x_stride;          // bytes per x column in shared memory
+    int xh_bytes;          // bytes of the x / h region
+};
+
+// Workspace layout for (T, k, H, I).
+struct MoeWs {
+    size_t ctrl_off, h_off, d_off, total;
+};
+
+inline MoeWs moe_ws_layout(int T, int k, int H, int I) {
+    MoeWs L;
+    const size_t ns = (size_t)T * k + 1;
+    const size_t ctrl_words = MOE_CTRL_ROWBLK + (size_t)H / 32;
+    L.ctrl_off = 0;
+    L.h_off = (ctrl_words * 4 + 255) / 256 * 256;
+    L.d_off = L.h_off + (ns * 4 * T * I + 255) / 256 * 256;
+    L.total = L.d_off + (ns * T * H * 4 + 255) / 256 * 256;
+    return L;
+}
+
+size_t moe_decode_smem_bytes(int ns, int xh_bytes);
+cudaError_t moe_decode_launch(const MoeParams& p, int grid, cudaStream_t stream);
+
+}  // namespace rfx

@@ -1,0 +1,203 @@
+/*
+ * rfx.h -- C ABI of the B200 (sm_100a) block-quantised MoE FFN library.
+ *
+ * The operation: the mixture-of-experts feed-forward step of a
+ * DeepSeek-V4-Flash-style model over ROCmFPX-style block-quantised weights,
+ * for decode (one token) and speculative verify (q <= 8 token columns), plus
+ * the router top-k.  Sources, cited by page title and section:
+ *
+ *  [TZ] taozi.news, "DeepSeek V4 Flash 在 128GB 锐龙 AI MAX+ 上跑到 32 tok/s",
+ *       section "ROCmFPX：把 284B 权重压进 128 GB" -- blocks of 32 weights with
+ *       low-bit codes and a scale; ROCmFP2 10 B/block (2.50 bit), ROCmFP3
+ *       3.50 bit, ROCmFP4 4.25 bit; routed gate/up in FP2, routed down in FP3,
+ *       sensitive projections FP4 or higher.
+ *  [AI] ainomam.com, "APU 实现 token 自由：AMD Ryzen AI MAX+ 395 跑 DeepSeek V4
+ *       Flash，284B 模型跑出 32 tok/s", section "Lucebox 的优化三板斧" -- 256
+ *       routed experts + 1 shared, 6 active per layer; in the q=4 verify path
+ *       every packed weight is decoded once and applied to all verify columns;
+ *       tuned TOP-K / ARGSORT routing kernels.
+ *  [MZ] m.mzlw.cn, "Lucebox专攻DeepSeek V4：DSpark草稿模型、MoE专家并行与
+ *       ROCmFPX量化达成42 tok/s", section "MoE 专家并行" -- 43 MoE layers, 256
+ *       routed experts, top-6 plus 1 shared expert; section "DSpark 草稿模型"
+ *       -- verify width q2..q5.
+ *
+ * Conventions
+ *  - Every function returns an rfx_status (0 = OK).  No exception crosses the
+ *    ABI.  rfx_last_error() gives a thread-local message for the last failure.
+ *  - "device" pointers are CUDA global-memory pointers of the current device;
+ *    "host" pointers are CPU memory.  All buffers are owned by the caller; the
+ *    library never allocates device memory (except rfx_layer_create, which
+ *    allocates only a small host struct).
+ *  - Device calls are asynchronous on `stream` (a cudaStream_t, NULL = legacy
+ *    default stream).  The return code covers argument validation and launch
+ *    errors.  Errors found on the device (expert id out of range, an
+ *    intermediate that overflows binary16, a bounded wait that timed out) set
+ *    a flag in the workspace that rfx_ws_status() reads after a sync.
+ *
+ * Packed weight format (this library's reading: the pages give only the block
+ * size and the bytes per block).  W[n][k] = scale[n][k/32] * level(code[n][k]):
+ *   RFX_FP2: 2-bit codes, level = c - 1.5  (-1.5 .. 1.5), binary16 scale, 10 B/block
+ *   RFX_FP3: 3-bit codes, level = c - 3.5  (-3.5 .. 3.5), binary16 scale, 14 B/block
+ *   RFX_FP4: 4-bit codes, level = c - 7.5  (-7.5 .. 7.5), E8M0 scale byte
+ *            (value 2^(e-127), 0xFF invalid), 17 B/block
+ * Blocks run along k (the reduction dimension) of one output row.  Packed
+ * layout: row-groups of 16 rows (rows padded to a multiple of 16 with zero
+ * codes and zero scales), each a contiguous stream of chunks of up to 8 tiles
+ * (tile = 16 rows x 1 block).  A chunk of nt tiles holds nt*16*codebytes of
+ * codes followed by nt*16*scalebytes of scales.  Codes are lane-major: lane
+ * L = 4g+t (g = 0..7, t = 0..3) owns nt*2b bytes at offset L*nt*2b.  Per tile
+ * the lane owns 8 "registers" r = 0..7, each two codes (low, high element):
+ *   m = r>>2, j = r&3, row = g + 8*(j&1), k0 = 16m + 2t + 8*(j>>1) inside the
+ *   block; low = code[row][k0], high = code[row][k0+1].
+ *   FP2: one 32-bit word per tile; r at bits [2r,2r+2) (low) and [16+2r,..) (high).
+ *   FP4: two 32-bit words per tile; word m holds r at bits [4j,4j+4) and [16+4j,..).
+ *   FP3: tiles are paired (96 bits per lane per pair, 3 words); pair register
+ *        R = 8*(tile&1) + r.  For R < 15: word R/5, field p = R%5 at bits
+ *        [3p,3p+3) (low) and [16+3p,..) (high).  R = 15: bit i of the low code
+ *        at bit 15 of word i, bit i of the high code at bit 31 of word i.  A
+ *        lone last tile of a chunk (odd nt) is a 48-bit little-endian stream of
+ *        its 16 codes, code 2r+e (e = 0 low, 1 high) at bits [3(2r+e), +3).
+ *   Scales of a chunk: [g][tile][row g, row g+8], binary16 or E8M0 bytes.
+ */
+#ifndef RFX_H
+#define RFX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    RFX_OK = 0,
+    RFX_EINVAL = -1,        /* bad argument (null pointer, size, format, code or scale value) */
+    RFX_EUNSUPPORTED = -2,  /* valid but outside what this build supports (e.g. q > 8) */
+    RFX_ECUDA = -3,         /* a CUDA runtime call or launch failed */
+    RFX_EDEVICE = -4,       /* device-side check failed (bad expert id, wait timeout) */
+    RFX_ERANGE = -5         /* an intermediate exceeded the binary16 range (|h| > 65504) */
+} rfx_status;
+
+typedef enum { RFX_FP2 = 2, RFX_FP3 = 3, RFX_FP4 = 4 } rfx_format;
+
+/* Thread-local text of the last non-OK status returned on this thread. */
+const char* rfx_last_error(void);
+
+/* ------------------------------------------------------------- format --- */
+
+/*
+ * Bytes of the packed form of a [rows][cols] matrix: rows padded up to a
+ * multiple of 16, times cols/32 blocks, times the block bytes of the format
+ * ([TZ] "ROCmFPX：把 284B 权重压进 128 GB": 32 weights per block, 10 B for
+ * ROCmFP2).  Returns 0 for an invalid format, rows < 0 or cols % 32 != 0.
+ */
+size_t rfx_packed_bytes(rfx_format f, int64_t rows, int64_t cols);
+
+/*
+ * Host packer.  codes: host uint8 [rows][cols], each < 2^f.  scales: host
+ * [rows][cols/32], uint16 binary16 bits for FP2/FP3 (finite values only),
+ * uint8 E8M0 for FP4 (0xFF rejected).  dst: host buffer of at least
+ * rfx_packed_bytes(f, rows, cols) bytes.  Returns RFX_EINVAL on any bad value;
+ * dst is then unspecified.
+ */
+int rfx_pack(rfx_format f, const uint8_t* codes, const void* scales, int64_t rows, int64_t cols,
+             void* dst, size_t dst_bytes);
+
+/* Host inverse of rfx_pack (codes [rows][cols], scales [rows][cols/32]). */
+int rfx_unpack(rfx_format f, const void* src, int64_t rows, int64_t cols, uint8_t* codes, void* scales);
+
+/*
+ * Device packer: same layout as rfx_pack with all pointers in device memory
+ * (codes [rows][cols] uint8, scales [rows][cols/32]).  Asynchronous on stream.
+ * Code and scale values are not checked on the device; a code >= 2^f is
+ * reduced modulo 2^f.
+ */
+int rfx_pack_device(rfx_format f, const uint8_t* codes, const void* scales, int64_t rows, int64_t cols,
+                    void* dst, void* stream);
+
+/* ------------------------------------------------------------- router --- */
+
+/*
+ * Router top-k with softmax over the selected logits ([AI] "Lucebox 的优化三板斧":
+ * TOP-K / ARGSORT routing; [MZ] "MoE 专家并行": top-6 of 256).
+ * logits: device fp32 [T][E] row-major (finite).  For each token t: idx[t][0..k)
+ * = the k largest logits in descending order, equal values ordered by the
+ * lower expert index; w[t][j] = exp(l_j - l_0) / sum_i exp(l_i - l_0) over the
+ * k selected.  idx: device int32 [T][k]; w: device fp32 [T][k].
+ * Limits: 1 <= E <= 1024, 1 <= k <= min(E, 16), T >= 0 (T = 0 is a no-op).
+ */
+int moe_router_topk(const float* logits, int T, int E, int k, int32_t* idx, float* w, void* stream);
+
+/* --------------------------------------------------------------- GEMV --- */
+
+/*
+ * y[c][n] = sum_k W[n][k] x[c][k] for c < q, n < N: the quantised mat-vec with
+ * in-kernel block dequantisation, every block decoded once for all q columns
+ * ([AI] "Lucebox 的优化三板斧": decode once, apply to all verify columns).
+ * W: device, packed (rfx_pack layout) [N][K].  x: device [q][K], bf16 bits
+ * (x_is_fp32 = 0) or fp32 (x_is_fp32 = 1; then |x| must be < 65504).
+ * y: device fp32 [q][N].  Limits: K % 32 == 0, 1 <= q <= 8, N >= 1.
+ */
+int rfx_gemv_q(rfx_format f, const void* W, int64_t N, int64_t K, const void* x, int x_is_fp32, int q,
+               float* y, void* stream);
+
+/* ------------------------------------------------------------ MoE FFN --- */
+
+/*
+ * One MoE layer ([MZ] "MoE 专家并行"): E routed experts, each with gate and up
+ * [I][H] and down [H][I] packed matrices, and an optional shared expert.  The
+ * routed matrices of expert e live at base + e * stride (bytes, multiple of
+ * 16, device memory); formats are per matrix kind ([TZ]: FP2 gate/up, FP3
+ * down, FP4 shared in the pages' assignment; any format is accepted).
+ */
+typedef struct {
+    int H, I, E, k;
+    rfx_format f_gate, f_up, f_down;
+    const void* gate; const void* up; const void* down;
+    size_t stride_gate, stride_up, stride_down;
+    int has_shared;
+    rfx_format f_sh_gate, f_sh_up, f_sh_down;
+    const void* sh_gate; const void* sh_up; const void* sh_down;
+} moe_layer_desc;
+
+typedef struct moe_layer moe_layer;
+
+/* Validate d and make a host-side handle (no device memory). */
+int moe_layer_create(const moe_layer_desc* d, moe_layer** out);
+void moe_layer_destroy(moe_layer* layer);
+
+/*
+ * Device workspace bytes moe_ffn_forward needs for T token columns.  The
+ * workspace holds counters, the SwiGLU intermediate and per-expert partial
+ * outputs; it must be zeroed once (rfx_ws_init) before its first use and may
+ * then be reused by successive calls on the same stream.  Calls that overlap
+ * on the GPU must use different workspaces.
+ */
+size_t moe_ffn_workspace_bytes(const moe_layer* layer, int T);
+int rfx_ws_init(void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Read and clear the device error flag of a workspace.  Synchronises stream.
+ * Returns RFX_OK, RFX_EDEVICE (bad expert id / duplicate id in a column /
+ * wait timeout) or RFX_ERANGE (|h| > 65504 met).
+ */
+int rfx_ws_status(void* ws, void* stream);
+
+/*
+ * MoE FFN for T token columns ([AI] "Lucebox 的优化三板斧"; [MZ] "MoE 专家并行"):
+ *   y[t] = sum_j w[t][j] * down_{e_tj}( silu(gate_{e_tj} x[t]) * up_{e_tj} x[t] )
+ *          + down_s( silu(gate_s x[t]) * up_s x[t] )      (shared weight 1)
+ * with e_tj = idx[t][j], silu(z) = z / (1 + e^-z).  The experts routed by any
+ * column are grouped: each packed block of each union expert is read from HBM
+ * and decoded once and applied to every column routed to that expert.
+ * x: device bf16 bits [T][H].  idx: device int32 [T][k], distinct per row,
+ * in [0, E).  w: device fp32 [T][k].  y: device fp32 [T][H].
+ * Limits: 1 <= T <= 8 (decode / verify), H % 32 == 0, I % 32 == 0, k <= 8.
+ */
+int moe_ffn_forward(const moe_layer* layer, const void* x, int T, const int32_t* idx, const float* w,
+                    float* y, void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* RFX_H */

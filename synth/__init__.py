@@ -159,3 +159,74 @@ class MatrixSpec:
     def scales(self, row0: int = 0, nrows: int | None = None) -> np.ndarray:
         n = self.rows - row0 if nrows is None else nrows
         return scales(self.scale_key, self.bits, n, self.cols, row0)
+
+
+# ------------------------------------------------ device twin (synth_dev.cu) ---
+
+_SRC_DEV = os.path.join(_HERE, "synth_dev.cu")
+_SO_DEV = os.path.join(_HERE, "libsynth_dev.so")
+_lib_dev = None
+_dev_tables = {}
+
+
+def build_dev(force: bool = False) -> str:
+    """Compile ``libsynth_dev.so`` (nvcc, sm_100a)."""
+    if force or not os.path.exists(_SO_DEV) or os.path.getmtime(_SO_DEV) < os.path.getmtime(_SRC_DEV):
+        tmp = _SO_DEV + f".tmp{os.getpid()}"
+        subprocess.check_call(["nvcc", "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-Xcompiler", "-fPIC",
+                               "-shared", "-o", tmp, _SRC_DEV])
+        os.replace(tmp, _SO_DEV)
+    return _SO_DEV
+
+
+def lib_dev():
+    global _lib_dev
+    with _lock:
+        if _lib_dev is None:
+            build_dev()
+            L = ctypes.CDLL(_SO_DEV)
+            u64, i64, i32, vp = ctypes.c_uint64, ctypes.c_int64, ctypes.c_int, ctypes.c_void_p
+            L.synth_codes_dev.restype = i32
+            L.synth_codes_dev.argtypes = [u64, i32, i64, i64, i64, vp, vp]
+            L.synth_scales_dev.restype = i32
+            L.synth_scales_dev.argtypes = [u64, i32, i64, i64, i64, vp, vp, vp, vp]
+            _lib_dev = L
+    return _lib_dev
+
+
+def scale_tables():
+    """Host copies of the 65536-entry binary16 and E8M0 scale tables."""
+    f16 = np.empty(65536, dtype=np.uint16)
+    e8 = np.empty(65536, dtype=np.uint8)
+    lib().synth_scale_tables.restype = None
+    lib().synth_scale_tables.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+    lib().synth_scale_tables(_p(f16), _p(e8))
+    return f16, e8
+
+
+def _tables_on(device):
+    import torch
+    key_ = str(device)
+    if key_ not in _dev_tables:
+        f16, e8 = scale_tables()
+        _dev_tables[key_] = (torch.from_numpy(f16.view(np.int16).copy()).to(device),
+                             torch.from_numpy(e8.copy()).to(device))
+    return _dev_tables[key_]
+
+
+def _stream_ptr(stream):
+    import torch
+    return (stream or torch.cuda.current_stream()).cuda_stream
+
+
+def codes_dev(k: int, bits: int, rows: int, cols: int, out, row0: int = 0, stream=None):
+    """Device codes into ``out`` (torch uint8, >= rows*cols bytes, 16-byte aligned)."""
+    if lib_dev().synth_codes_dev(k, bits, row0, rows, cols, out.data_ptr(), _stream_ptr(stream)) != 0:
+        raise RuntimeError("synth_codes_dev failed")
+
+
+def scales_dev(k: int, bits: int, rows: int, cols: int, out, row0: int = 0, stream=None):
+    tf16, te8 = _tables_on(out.device)
+    if lib_dev().synth_scales_dev(k, bits, row0, rows, cols, out.data_ptr(), tf16.data_ptr(), te8.data_ptr(),
+                                  _stream_ptr(stream)) != 0:
+        raise RuntimeError("synth_scales_dev failed")

@@ -97,6 +97,13 @@ static void build_tables(void) {
 
 void synth_init(void) { build_tables(); }
 
+/* Copy of the 65536-entry scale tables (for the device twin of this module). */
+void synth_scale_tables(uint16_t* f16, uint8_t* e8m0) {
+    build_tables();
+    memcpy(f16, g_scale_f16, sizeof(g_scale_f16));
+    memcpy(e8m0, g_scale_e8m0, sizeof(g_scale_e8m0));
+}
+
 /*
  * Codes of rows [row0, row0+nrows) of a [rows][cols] matrix (cols % 32 == 0),
  * one code per byte, row-major: out[(r - row0) * cols + k].

@@ -12,6 +12,12 @@ GOLDEN = os.path.join(ROOT, "tests", "golden")
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA B200 (sm_100a) device")
+    # build the in-tree libraries if a source changed (nvcc cross-compiles sm_100a on any host)
+    from block_quantized_moe_rocmfpx_b200 import build as _b
+    _b.build()
+    import synth
+    synth.build()
+    synth.build_dev()
 
 
 def pytest_collection_modifyitems(config, items):

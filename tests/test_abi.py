@@ -1,0 +1,160 @@
+"""C-ABI library on the host: symbols, packed layout, argument checks.
+
+No kernel is launched here (no GPU needed): the packer is host code and every
+argument error is detected before any CUDA call.
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import block_quantized_moe_rocmfpx_b200 as rfx
+import synth
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "rfx.h")
+
+
+def declared_functions():
+    txt = open(HEADER).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    names = re.findall(r"\b([a-z_][a-z0-9_]*)\s*\(", txt)
+    skip = {"if", "sizeof", "defined"}
+    return sorted({n for n in names if n not in skip and (n.startswith("rfx_") or n.startswith("moe_"))})
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_functions()
+    assert len(names) >= 12
+    lib = ctypes.CDLL(rfx.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(rfx.EXPORTED)
+
+
+@pytest.mark.parametrize("fmt", [2, 3, 4])
+def test_packed_bytes_is_block_bytes(fmt):
+    bb = {2: 10, 3: 14, 4: 17}[fmt]
+    assert rfx.rfx_packed_bytes(fmt, 2048, 4096) == 2048 * 128 * bb
+    assert rfx.rfx_packed_bytes(fmt, 17, 64) == 32 * 2 * bb        # rows padded to 16
+    assert rfx.rfx_packed_bytes(fmt, 16, 48) == 0                  # cols % 32 != 0
+    assert rfx.rfx_packed_bytes(7, 16, 64) == 0
+
+
+@pytest.mark.parametrize("fmt", [2, 3, 4])
+@pytest.mark.parametrize("rows,cols", [(16, 256), (48, 4096), (33, 352), (16, 160), (5, 32), (64, 96)])
+def test_pack_unpack_round_trip(fmt, rows, cols):
+    spec = synth.MatrixSpec(1, 0, 0, 0, fmt, rows, cols)
+    c, s = spec.codes(), spec.scales()
+    packed = rfx.rfx_pack(fmt, c, s)
+    assert packed.nbytes == rfx.rfx_packed_bytes(fmt, rows, cols)
+    c2, s2 = rfx.rfx_unpack(fmt, packed, rows, cols)
+    assert np.array_equal(c, c2) and np.array_equal(s, s2)
+
+
+@pytest.mark.parametrize("fmt", [2, 3, 4])
+def test_pack_extreme_codes(fmt):
+    rows, cols = 32, 512
+    for c0 in (0, (1 << fmt) - 1):
+        c = np.full((rows, cols), c0, np.uint8)
+        s = np.full((rows, cols // 32), 0x7BFF if fmt != 4 else 0xFE, np.uint16 if fmt != 4 else np.uint8)
+        c2, s2 = rfx.rfx_unpack(fmt, rfx.rfx_pack(fmt, c, s), rows, cols)
+        assert np.array_equal(c, c2) and np.array_equal(s, s2)
+
+
+def _reg_coords(g, t, r):
+    m, j = r >> 2, r & 3
+    return g + 8 * (j & 1), 16 * m + 2 * t + 8 * (j >> 1)
+
+
+def test_layout_matches_header_description():
+    """Rebuild the first chunk of a row-group from the bit positions rfx.h documents."""
+    rows, cols = 16, 256 + 96          # one full chunk and one partial chunk of 3 tiles
+    for fmt in (2, 3, 4):
+        spec = synth.MatrixSpec(4, 0, 1, 0, fmt, rows, cols)
+        c, s = spec.codes(), spec.scales()
+        packed = rfx.rfx_pack(fmt, c, s)
+        nt = 8
+        lane_bytes = nt * 2 * fmt
+        for L in (0, 5, 31):
+            g, t = L >> 2, L & 3
+            lane = packed[L * lane_bytes:(L + 1) * lane_bytes]
+            words = np.frombuffer(lane.tobytes(), dtype=np.uint32)
+            for b in range(nt):
+                for r in range(8):
+                    row, k = _reg_coords(g, t, r)
+                    lo, hi = int(c[row, 32 * b + k]), int(c[row, 32 * b + k + 1])
+                    if fmt == 2:
+                        w = int(words[b])
+                        assert (w >> (2 * r)) & 3 == lo and (w >> (16 + 2 * r)) & 3 == hi
+                    elif fmt == 4:
+                        w, j = int(words[2 * b + (r >> 2)]), r & 3
+                        assert (w >> (4 * j)) & 15 == lo and (w >> (16 + 4 * j)) & 15 == hi
+                    else:
+                        R = 8 * (b & 1) + r
+                        ws = [int(v) for v in words[3 * (b >> 1):3 * (b >> 1) + 3]]
+                        if R < 15:
+                            w, p = ws[R // 5], R % 5
+                            assert (w >> (3 * p)) & 7 == lo and (w >> (16 + 3 * p)) & 7 == hi
+                        else:
+                            assert sum(((ws[i] >> 15) & 1) << i for i in range(3)) == lo
+                            assert sum(((ws[i] >> 31) & 1) << i for i in range(3)) == hi
+        # scales of the first chunk: [g][tile][row g, row g+8]
+        sb = 1 if fmt == 4 else 2
+        sc = packed[8 * 16 * 4 * fmt: 8 * 16 * 4 * fmt + 8 * 8 * 2 * sb]
+        sc = np.frombuffer(sc.tobytes(), dtype=np.uint8 if fmt == 4 else np.uint16).reshape(8, 8, 2)
+        for g in range(8):
+            for b in range(8):
+                assert sc[g, b, 0] == s[g, b] and sc[g, b, 1] == s[g + 8, b]
+
+
+def test_pack_rejects_bad_values():
+    c = np.zeros((16, 64), np.uint8)
+    s16 = np.full((16, 2), 0x3C00, np.uint16)
+    with pytest.raises(rfx.RfxError) as e:
+        rfx.rfx_pack(2, np.full((16, 64), 4, np.uint8), s16)
+    assert e.value.code == rfx.RFX_EINVAL
+    with pytest.raises(rfx.RfxError):
+        rfx.rfx_pack(3, c, np.full((16, 2), 0x7C00, np.uint16))      # inf scale
+    with pytest.raises(rfx.RfxError):
+        rfx.rfx_pack(4, c, np.full((16, 2), 0xFF, np.uint8))          # E8M0 NaN
+    with pytest.raises(rfx.RfxError):
+        rfx.rfx_pack(5, c, s16)
+    assert "rfx_pack" in rfx.rfx_last_error()
+
+
+def test_device_calls_reject_bad_arguments_before_cuda():
+    lib = ctypes.CDLL(rfx.LIB_PATH)
+    assert lib.moe_router_topk(None, -1, 256, 6, None, None, None) == rfx.RFX_EINVAL
+    assert lib.moe_router_topk(None, 4, 256, 0, None, None, None) == rfx.RFX_EINVAL
+    assert lib.moe_router_topk(None, 4, 8, 9, None, None, None) == rfx.RFX_EINVAL
+    assert lib.moe_router_topk(None, 0, 256, 6, None, None, None) == rfx.RFX_OK       # T = 0: no-op
+    assert lib.rfx_gemv_q(2, None, 16, 64, None, 0, 9, None, None) == rfx.RFX_EUNSUPPORTED
+    assert lib.rfx_gemv_q(2, None, 16, 48, None, 0, 1, None, None) == rfx.RFX_EINVAL
+    assert lib.rfx_gemv_q(6, None, 16, 64, None, 0, 1, None, None) == rfx.RFX_EINVAL
+
+
+def test_layer_create_validation():
+    d = rfx.moe_layer_desc()
+    d.H, d.I, d.E, d.k = 4096, 2048, 256, 6
+    d.f_gate, d.f_up, d.f_down = 2, 2, 3
+    d.gate = d.up = d.down = 256
+    d.stride_gate = d.stride_up = rfx.rfx_packed_bytes(2, 2048, 4096)
+    d.stride_down = rfx.rfx_packed_bytes(3, 4096, 2048)
+    h = rfx.moe_layer_create(d)
+    assert h
+    assert rfx.moe_ffn_workspace_bytes(h, 4) > 0 and rfx.moe_ffn_workspace_bytes(h, 9) == 0
+    rfx.moe_layer_destroy(h)
+    for field, val in (("H", 100), ("k", 9), ("f_up", 3), ("stride_down", 16), ("gate", 8), ("E", 2000)):
+        bad = rfx.moe_layer_desc.from_buffer_copy(d)
+        setattr(bad, field, val)
+        with pytest.raises(rfx.RfxError):
+            rfx.moe_layer_create(bad)
+    bad = rfx.moe_layer_desc.from_buffer_copy(d)
+    bad.has_shared = 1
+    with pytest.raises(rfx.RfxError):          # shared pointers missing
+        rfx.moe_layer_create(bad)
+    lib = ctypes.CDLL(rfx.LIB_PATH)
+    assert lib.moe_ffn_forward(None, None, 1, None, None, None, None, 0, None) == rfx.RFX_EINVAL
