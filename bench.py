@@ -1,0 +1,419 @@
+"""Benchmark: MoE-FFN decode / verify tokens/s and achieved HBM GB/s on B200.
+
+Workload (default): one full-size MoE layer (H=4096, I=2048, 256 routed experts
+top-6 + 1 shared; routed gate/up ROCmFP2, down ROCmFP3, shared ROCmFP4, 2.3 GB
+packed) in decode at q=1 over 1000 seeded tokens with Zipf(s=1.1) routing
+bias.  A step is one pass of the whole hot path for one batch: router top-k +
+softmax, expert grouping, fused dequant gate/up GEMV + SwiGLU, down GEMV and
+weighted combine.  The same layer in speculative verify at q=4 is reported
+beside it.  Weights are synthetic (seeded) and stay resident in HBM; 8 copies
+of the layer are rotated so that every step reads its weights from DRAM
+(inputs larger than L2).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun) every rank runs an independent replica of the workload
+(the path is one GPU's work; nothing is exchanged) and rank 0 prints one JSON
+line with the whole-job throughput over the max-over-ranks device time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-FFN decode tokens/s & achieved HBM GB/s (% of ~8 TB/s) at q=1 and q=4"
+H, I, E, K_TOP = 4096, 2048, 256, 6
+ZIPF_S = 1.1
+NTOK = 1000
+COPIES = 8
+SEED = 0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            P = json.load(f)
+        return float(P["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ----------------------------------------------------------------- clocks ---
+
+class Clocks:
+    """nvidia-smi sampling during the timed region."""
+
+    def __init__(self, index: int):
+        import torch
+        try:
+            self.index = "GPU-" + str(torch.cuda.get_device_properties(index).uuid)
+        except Exception:
+            self.index = str(index)
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                    rows.append(parts)
+        except Exception:
+            pass
+        finally:
+            try:
+                os.unlink(self.path)
+            except Exception:
+                pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]), "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())
+                if any(r[3].replace(".", "").isdigit() for r in rows) else None}
+
+
+# ----------------------------------------------------------------- oracle ---
+
+def cpu_baseline(n_tokens: int, q: int, budget_s: float = 20.0):
+    """The fp64 oracle as it stands, on the host cores, on a bounded sample of
+    the same workload (tokens of the same layer and routing).  Codes are
+    regenerated outside the timed region."""
+    import numpy as np
+    import oracle
+    import synth
+
+    L = synth.logits(SEED, 0, 0, n_tokens * q, E, ZIPF_S)
+    xb = synth.x_bf16(SEED, 0, n_tokens * q, H)
+    idx, w = oracle.router_topk(L, K_TOP)
+    mats = {}
+
+    def get(kind, e, bits, r, c):
+        if (kind, e) not in mats:
+            s = synth.MatrixSpec(SEED, 0, kind, e, bits, r, c)
+            mats[(kind, e)] = oracle.Mat(bits, s.codes(), s.scales())
+        return mats[(kind, e)]
+
+    shared = tuple(get(k, 0, 4, r, c) for k, (r, c) in zip((3, 4, 5), ((I, H), (I, H), (H, I))))
+    xf = synth.bf16_to_f64(xb)
+    done, t_oracle = 0, 0.0
+    for t in range(n_tokens * q):
+        ex = [tuple(get(k, int(e), b, r, c) for k, b, (r, c) in zip((0, 1, 2), (2, 2, 3), ((I, H), (I, H), (H, I))))
+              for e in idx[t]]
+        t0 = time.perf_counter()
+        oracle.router_topk(L[t:t + 1], K_TOP)
+        oracle.moe_token(ex, w[t], shared, xf[t])
+        t_oracle += time.perf_counter() - t0
+        done += 1
+        if t_oracle > budget_s:
+            break
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return {"value": done / t_oracle, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{done} token columns of the q={q} workload (router + 6 routed experts + shared, fp64), "
+                      f"{t_oracle:.1f} s of oracle time"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    base = cpu_baseline(args.steps, 1, budget_s=max(10.0, min(60.0, 2.0 * args.steps)))
+    line = {"impl": "reference", "metric": METRIC, "value": base["value"], "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 / base["value"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "one full-size MoE layer decode q=1 (H=4096, I=2048, 256 experts top-6 + 1 shared, "
+                                   "FP2 gate/up, FP3 down, FP4 shared), Zipf(1.1) routing", "global_batch": 1,
+                       "seq_len": 1, "parallelism": "replicas"},
+            "cpu_baseline": base,
+            "e2e": {"value": base["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# -------------------------------------------------------------------- GPU ---
+
+class Workload:
+    """C rotating copies of one synthetic full-size layer plus seeded inputs."""
+
+    def __init__(self, q: int, ntok: int, dev):
+        import torch
+        import numpy as np
+        import synth
+        from synth.layers import SynthLayer
+        self.q, self.dev = q, dev
+        base = SynthLayer(SEED, 0, H, I, E, K_TOP, device=dev)
+        self.base = base
+        self.layers = [base.moe_layer(max_T=q)]
+        self._keep = [base]
+        for c in range(1, COPIES):
+            bufs = [b.clone() for b in base.bufs]
+            sh = [b.clone() for b in base.shared]
+            import block_quantized_moe_rocmfpx_b200 as rfx
+            ml = rfx.MoeLayer(H, I, E, K_TOP, base.fmts, *bufs, base.strides, shared=sh,
+                              shared_fmts=base.shared_fmts, max_T=q)
+            self._keep.append((bufs, sh))
+            self.layers.append(ml)
+        torch.cuda.synchronize()
+        self.ntok = ntok
+        nb = ntok * q
+        self.logits_h = synth.logits(SEED, 0, 0, nb, E, ZIPF_S)
+        self.x_h = synth.x_bf16(SEED, 0, nb, H)
+        self.logits = torch.from_numpy(self.logits_h).to(dev).view(ntok, q, E)
+        self.x = torch.from_numpy(self.x_h).view(torch.bfloat16).to(dev).view(ntok, q, H)
+        self.idx = torch.empty((ntok, q, K_TOP), dtype=torch.int32, device=dev)
+        self.w = torch.empty((ntok, q, K_TOP), dtype=torch.float32, device=dev)
+        self.y = torch.empty((COPIES, q, H), dtype=torch.float32, device=dev)
+
+    def step(self, t: int, route: bool = True, ffn: bool = True):
+        import block_quantized_moe_rocmfpx_b200 as rfx
+        s = t % self.ntok
+        if route:
+            rfx.moe_router_topk(self.logits[s], K_TOP, self.idx[s], self.w[s])
+        if ffn:
+            self.layers[t % COPIES].forward(self.x[s], self.idx[s], self.w[s], self.y[t % COPIES])
+
+    def algo_bytes(self, tokens) -> float:
+        """Bytes one pass must move: packed blocks of the union of routed
+        experts + the shared expert, plus activations in/out."""
+        import numpy as np
+        idx = self.idx.cpu().numpy()
+        tot = 0.0
+        for t in tokens:
+            s = t % self.ntok
+            tot += self.base.union_bytes(idx[s].ravel())
+            tot += self.q * (2 * H + 8 * K_TOP + 4 * H + 4 * E)
+        return tot
+
+
+def graph_of(fn, n, stream):
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for t in range(n):
+            fn(t)
+    return g
+
+
+def time_graph(g, stream):
+    """Device time of one replay: events recorded on the stream the graph is launched on."""
+    import torch
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def measure(q: int, steps: int, warmup: int, dev, rank, world, want_clocks: bool, want_e2e: bool):
+    import torch
+    import torch.distributed as dist
+    wl = Workload(q, NTOK, dev)
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        for t in range(3):            # eager warm-up (kernel attributes, lazy loading)
+            wl.step(t)
+        torch.cuda.synchronize()
+        off = warmup
+        g_warm = graph_of(lambda t: wl.step(t), warmup, stream)
+        g_main = graph_of(lambda t: wl.step(off + t), steps, stream)
+        g_ffn = graph_of(lambda t: wl.step(off + t, route=False), steps, stream)
+    # warm-up
+    with torch.cuda.stream(stream):
+        g_warm.replay()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = None
+    with (Clocks(torch.cuda.current_device()) if want_clocks else _Null()) as ck:
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        ms = time_graph(g_main, stream)
+        if world > 1:
+            dist.barrier()
+        clk = ck.summary() if want_clocks else None
+    # dominant kernel alone (routing already in HBM from the timed pass)
+    ms_ffn = time_graph(g_ffn, stream)
+    status = max(ml.status() for ml in wl.layers[:1])
+    abytes = wl.algo_bytes(range(off, off + steps))
+    res = {"ms": ms, "ms_ffn": ms_ffn, "bytes": abytes, "clocks": clk, "status": status}
+    if want_e2e:
+        res["e2e"] = e2e(wl, steps, stream)
+    del g_warm, g_main, g_ffn
+    return res
+
+
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        pass
+
+    def summary(self):
+        return None
+
+
+def e2e(wl, steps, stream):
+    """Same workload through the public API with host buffers: per step, the
+    token's x and router logits go host->device from pinned memory, the router
+    and the MoE FFN run, and y comes back device->host."""
+    import torch
+    import block_quantized_moe_rocmfpx_b200 as rfx
+    q = wl.q
+    n = min(steps, wl.ntok)
+    xh = torch.from_numpy(wl.x_h).view(torch.bfloat16).view(wl.ntok, q, H).pin_memory()
+    lh = torch.from_numpy(wl.logits_h).view(wl.ntok, q, E).pin_memory()
+    yh = torch.empty((n, q, H), dtype=torch.float32).pin_memory()
+    xd = torch.empty((q, H), dtype=torch.bfloat16, device=wl.dev)
+    ld = torch.empty((q, E), dtype=torch.float32, device=wl.dev)
+    idx = torch.empty((q, K_TOP), dtype=torch.int32, device=wl.dev)
+    w = torch.empty((q, K_TOP), dtype=torch.float32, device=wl.dev)
+    yd = torch.empty((q, H), dtype=torch.float32, device=wl.dev)
+
+    def one(t):
+        xd.copy_(xh[t], non_blocking=True)
+        ld.copy_(lh[t], non_blocking=True)
+        rfx.moe_router_topk(ld, K_TOP, idx, w)
+        wl.layers[t % COPIES].forward(xd, idx, w, yd)
+        yh[t].copy_(yd, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for t in range(5):
+            one(t)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for t in range(n):
+            one(t)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    return {"value": n * q / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": q * (2 * H + 4 * E),
+            "d2h_bytes_per_step": q * 4 * H, "steps": n}
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    import __graft_entry__
+    if rank == 0 or world == 1:
+        __graft_entry__.build()
+    if world > 1:
+        dist.barrier()
+    r1 = measure(1, args.steps, max(3, args.warmup), dev, rank, world, True, not args.no_e2e)
+    r4 = measure(4, args.steps, max(3, args.warmup), dev, rank, world, False, False)
+
+    def reduce_max(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    ms1, ms4 = reduce_max(r1["ms"]), reduce_max(r4["ms"])
+    ms1f, ms4f = reduce_max(r1["ms_ffn"]), reduce_max(r4["ms_ffn"])
+    e2e_v = None
+    if "e2e" in r1:
+        e2e_ms = reduce_max(r1["e2e"]["steps"] / r1["e2e"]["value"] * 1e3)
+        e2e_v = dict(r1["e2e"])
+        e2e_v["value"] = world * r1["e2e"]["steps"] / (e2e_ms / 1e3)
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        peak, peak_kind = peaks()
+        gbs1 = r1["bytes"] / (r1["ms_ffn"] / 1e3) / 1e9
+        gbs4 = r4["bytes"] / (r4["ms_ffn"] / 1e3) / 1e9
+        value = world * args.steps / (ms1 / 1e3)
+        base = None if args.no_cpu_baseline else cpu_baseline(3, 1, budget_s=15.0)
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": max(3, args.warmup), "ms_per_step": ms1 / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "one full-size MoE layer decode q=1 (H=4096, I=2048, 256 experts top-6 + 1 shared, "
+                                   "FP2 gate/up, FP3 down, FP4 shared; 2.30 GB packed), 1000 seeded tokens, "
+                                   "Zipf(1.1) routing", "global_batch": world, "seq_len": 1,
+                       "parallelism": "replicas" if world > 1 else "single",
+                       "l2": f"inputs larger than L2: {COPIES} rotating copies of the layer",
+                       "graph": "CUDA graph of all timed steps"},
+            "roofline": {"bound": "hbm", "achieved": gbs1, "peak": peak, "unit": "GB/s", "frac": gbs1 / peak,
+                         "traffic": None, "kernel": "moe_decode_kernel", "peak_kind": peak_kind,
+                         "algo_bytes_per_launch": r1["bytes"] / args.steps,
+                         "kernel_us": r1["ms_ffn"] * 1e3 / args.steps},
+            "q4": {"value": world * 4 * args.steps / (ms4 / 1e3), "unit": "tokens/s", "ms_per_step": ms4 / args.steps,
+                   "achieved_gbs": gbs4, "frac": gbs4 / peak, "kernel_us": r4["ms_ffn"] * 1e3 / args.steps,
+                   "algo_bytes_per_launch": r4["bytes"] / args.steps},
+            "cpu_baseline": base,
+            "e2e": e2e_v,
+            "gpu_launches": 2 * args.steps,
+            "clocks": r1["clocks"],
+            "device_status": {"q1": r1["status"], "q4": r4["status"]},
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

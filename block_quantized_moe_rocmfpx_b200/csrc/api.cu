@@ -27,14 +27,25 @@ int cuda_fail(const char* where, cudaError_t e) {
     return rfx_fail(RFX_ECUDA, std::string(where) + ": " + cudaGetErrorString(e));
 }
 
+// SM count and opt-in shared memory of the current device, queried once per device.
 int device_props(int& sms, int& smem_optin) {
+    static int cache_sms[64] = {0}, cache_smem[64] = {0};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+    if (dev < 64 && cache_sms[dev]) {
+        sms = cache_sms[dev];
+        smem_optin = cache_smem[dev];
+        return RFX_OK;
+    }
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return cuda_fail("cudaDeviceGetAttribute", e);
     e = cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (e != cudaSuccess) return cuda_fail("cudaDeviceGetAttribute", e);
+    if (dev < 64) {
+        cache_sms[dev] = sms;
+        cache_smem[dev] = smem_optin;
+    }
     return RFX_OK;
 }
 

@@ -55,8 +55,8 @@ struct SlotTable {
 };
 
 struct Shared {
-    uint64_t full[NCW][MOE_MAX_STAGES];
-    uint64_t empty[NCW][MOE_MAX_STAGES];
+    uint64_t full[MOE_MAX_STAGES];
+    uint64_t empty[MOE_MAX_STAGES];
     uint64_t tqf[QN], tqe[QN];
     uint64_t hfull[2], hfree[2];
     uint64_t xfree;
@@ -64,7 +64,7 @@ struct Shared {
     int rcnt[2];
     volatile int repoch[2];
     volatile int abort_flag;
-    int cc[NCW];
+    volatile int consumed;   // stages released by all consumer warps (for the abort drain)
     SlotTable st;
 };
 
@@ -158,13 +158,10 @@ __device__ __forceinline__ MatRef slot_mats(const MoeParams& p, int e, int kind)
     return {p.down + (long long)e * p.sd, nullptr, p.fB};
 }
 
-__device__ __forceinline__ void warp_chunk_range(int w, int nch, int& c0, int& c1) {
-    const int kq = w >> 1;
-    c0 = kq * nch / 4;
-    c1 = (kq + 1) * nch / 4;
-}
-
 // ------------------------------------------------------------- producer ---
+//
+// Per task (32 rows = 2 row-groups) and per row-group, one stage per span of
+// up to 8 chunks: a single bulk copy per matrix of the contiguous span.
 
 __device__ void producer(const MoeParams& p, Shared& sh, uint8_t* ring, uint8_t* xh, int hbytes_max) {
     const SlotTable& S = sh.st;
@@ -172,14 +169,13 @@ __device__ void producer(const MoeParams& p, Shared& sh, uint8_t* ring, uint8_t*
     const int ntasks = S.nslots * (nrbA + nrbB);
     const uint64_t pol_w = policy_evict_first();
     const uint64_t pol_h = policy_evict_last();
-    int sc[NCW];
-#pragma unroll
-    for (int w = 0; w < NCW; ++w) sc[w] = 0;
-    int bseq = 0;
+    int sc = 0, bseq = 0;
     bool ok = true;
+    int next = (int)atomicAdd(p.ctrl + MOE_CTRL_TASK, 1u);
     for (int n = 0; ok; ++n) {
-        int t = (int)atomicAdd(p.ctrl + MOE_CTRL_TASK, 1u);
+        int t = next;
         if (t >= ntasks) t = -1;
+        else next = (int)atomicAdd(p.ctrl + MOE_CTRL_TASK, 1u);   // overlaps with this task's copies
         const int qi = n % QN;
         if (!mbar_wait(&sh.tqe[qi], ((n / QN) + 1) & 1, WAIT_LIMIT)) { ok = false; break; }
         sh.tq[qi] = t;
@@ -196,12 +192,11 @@ __device__ void producer(const MoeParams& p, Shared& sh, uint8_t* ring, uint8_t*
             if (bseq == 0 && !mbar_wait(&sh.xfree, 0, WAIT_LIMIT)) { ok = false; break; }
             const int buf = bseq & 1;
             if (!mbar_wait(&sh.hfree[buf], ((bseq >> 1) + 1) & 1, WAIT_LIMIT)) { ok = false; break; }
-            // all A tasks of this slot done?
             const uint32_t need = (uint32_t)nrbA;
             const long long t0 = clock64();
             while (ld_acquire_gpu(p.ctrl + MOE_CTRL_SLOT + tk.slot) < need) {
                 if (clock64() - t0 > WAIT_LIMIT) { ok = false; break; }
-                __nanosleep(64);
+                __nanosleep(32);
             }
             if (!ok) break;
             fence_proxy_async_global();
@@ -211,33 +206,25 @@ __device__ void producer(const MoeParams& p, Shared& sh, uint8_t* ring, uint8_t*
                      pol_h);
             ++bseq;
         }
-        int cr0[NCW], cr1[NCW];
-        int maxj = 0;
-#pragma unroll
-        for (int w = 0; w < NCW; ++w) {
-            warp_chunk_range(w, nch, cr0[w], cr1[w]);
-            maxj = max(maxj, cr1[w] - cr0[w]);
-        }
-        for (int j = 0; j < maxj && ok; ++j) {
-#pragma unroll
-            for (int w = 0; w < NCW; ++w) {
-                const int c = cr0[w] + j;
-                if (c >= cr1[w]) continue;
-                const int s = sc[w] % p.ns;
-                if (!mbar_wait(&sh.empty[w][s], ((sc[w] / p.ns) + 1) & 1, WAIT_LIMIT)) { ok = false; break; }
-                uint8_t* dst = ring + (w * p.ns + s) * MOE_STAGE_BYTES;
-                const int rg = 2 * tk.rb + (w & 1);
-                const long long off = rg * rgb + (long long)c * fullb;
-                const uint32_t cb = (uint32_t)rfx_chunk_bytes(m.fmt, rfx_chunk_tiles(K, c));
+        for (int rgl = 0; rgl < 2 && ok; ++rgl) {
+            const long long rgoff = (long long)(2 * tk.rb + rgl) * rgb;
+            for (int c0 = 0; c0 < nch; c0 += MOE_CHUNKS_PER_STAGE) {
+                const int c1 = min(nch, c0 + MOE_CHUNKS_PER_STAGE);
+                // bytes of chunks [c0, c1): full chunks plus a possibly partial last one
+                const uint32_t bytes = (uint32_t)((c1 - 1 - c0) * fullb + rfx_chunk_bytes(m.fmt, rfx_chunk_tiles(K, c1 - 1)));
+                const int s = sc % p.ns;
+                if (!mbar_wait(&sh.empty[s], ((sc / p.ns) + 1) & 1, WAIT_LIMIT)) { ok = false; break; }
+                uint8_t* dst = ring + s * MOE_STAGE_BYTES;
+                const long long off = rgoff + (long long)c0 * fullb;
                 if (tk.kind == 0) {
-                    mbar_arrive_expect_tx(&sh.full[w][s], 2 * cb);
-                    bulk_g2s(dst, m.a + off, cb, &sh.full[w][s], pol_w);
-                    bulk_g2s(dst + fullb, m.b + off, cb, &sh.full[w][s], pol_w);
+                    mbar_arrive_expect_tx(&sh.full[s], 2 * bytes);
+                    bulk_g2s(dst, m.a + off, bytes, &sh.full[s], pol_w);
+                    bulk_g2s(dst + MOE_HALF_BYTES, m.b + off, bytes, &sh.full[s], pol_w);
                 } else {
-                    mbar_arrive_expect_tx(&sh.full[w][s], cb);
-                    bulk_g2s(dst, m.a + off, cb, &sh.full[w][s], pol_w);
+                    mbar_arrive_expect_tx(&sh.full[s], bytes);
+                    bulk_g2s(dst, m.a + off, bytes, &sh.full[s], pol_w);
                 }
-                ++sc[w];
+                ++sc;
             }
         }
     }
@@ -245,14 +232,9 @@ __device__ void producer(const MoeParams& p, Shared& sh, uint8_t* ring, uint8_t*
         set_error(p.ctrl, MOE_ERR_TIMEOUT);
         sh.abort_flag = 1;
         // drain: wait (bounded) until every issued copy has landed
-#pragma unroll
-        for (int w = 0; w < NCW; ++w) {
-            for (int i = sh.cc[w]; i < sc[w]; ++i)
-                (void)mbar_wait(&sh.full[w][i % p.ns], (i / p.ns) & 1, WAIT_LIMIT);
-        }
+        for (int i = sh.consumed; i < sc; ++i) (void)mbar_wait(&sh.full[i % p.ns], (i / p.ns) & 1, WAIT_LIMIT);
         for (int b = 0; b < 2 && b < bseq; ++b)
             (void)mbar_wait(&sh.hfull[(bseq - 1 - b) & 1], ((bseq - 1 - b) >> 1) & 1, WAIT_LIMIT);
-        // release consumers still waiting on the task queue
         for (int qi = 0; qi < QN; ++qi) {
             sh.tq[qi] = -1;
             mbar_arrive(&sh.tqf[qi]);
@@ -262,18 +244,128 @@ __device__ void producer(const MoeParams& p, Shared& sh, uint8_t* ring, uint8_t*
 
 // ------------------------------------------------------------- consumers ---
 
-template <int FA, int FB>
+// The last of the NCW warps to deposit its partial sums for row-group unit r
+// returns true (and must call red_release afterwards).
+__device__ __forceinline__ bool red_deposit(Shared& sh, float* red, int r, int w, int lane, const float v[8],
+                                            bool& ok) {
+    const int rbuf = r & 1;
+    {
+        const long long t0 = clock64();
+        while (sh.repoch[rbuf] != r - 2) {
+            if (clock64() - t0 > WAIT_LIMIT) { ok = false; return false; }
+        }
+    }
+    float* my = red + ((rbuf * NCW + w) * 32 + lane) * 8;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) my[i] = v[i];
+    __threadfence_block();
+    __syncwarp();
+    int old = 0;
+    if (lane == 0) old = atomicAdd(&sh.rcnt[rbuf], 1);
+    old = __shfl_sync(0xffffffffu, old, 0);
+    if (old != NCW - 1) return false;
+    __threadfence_block();
+    return true;
+}
+
+__device__ __forceinline__ void red_release(Shared& sh, int r, int lane) {
+    __syncwarp();
+    if (lane == 0) {
+        sh.rcnt[r & 1] = 0;
+        __threadfence_block();
+        sh.repoch[r & 1] = r;
+    }
+    __syncwarp();
+}
+
+// SwiGLU of one row-group -> h (fp16 hi/lo pair per value) in the fragment
+// order of the down projection's B operand: [step][v][t'][4].
+__device__ void epilogue_a(const MoeParams& p, const float* rb0, int slot, int ncols, int rg, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    uint16_t* hs = p.hbuf + (long long)slot * (2LL * p.T * p.I);
+    float G[4] = {0.f, 0.f, 0.f, 0.f}, U[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int w = 0; w < NCW; ++w) {
+        const float* r = rb0 + (w * 32 + lane) * 8;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) { G[i] += r[i]; U[i] += r[4 + i]; }
+    }
+    uint32_t bad = 0;
+    const int step = rg;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int col = 2 * t + (i & 1);
+        const int rowhi = i >> 1;  // 0: row g, 1: row g+8
+        if (col >= ncols) continue;
+        const float gv = G[i];
+        const float h = gv / (1.0f + expf(-gv)) * U[i];
+        const __half hi = __float2half_rn(h);
+        const __half lo = __float2half_rn(h - __half2float(hi));
+        if (!(fabsf(h) <= 65504.0f)) bad = 1;
+        const int tp = g >> 1, pos = 2 * rowhi + (g & 1);
+        const long long base = ((long long)(step * 2 * ncols) * 4 + tp) * 4 + pos;
+        hs[base + (long long)(2 * col) * 16] = __half_as_ushort(hi);
+        hs[base + (long long)(2 * col + 1) * 16] = __half_as_ushort(lo);
+    }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) set_error(p.ctrl, MOE_ERR_RANGE);
+}
+
+// Partial down output of one row-group -> dpart; the last slot to finish the
+// row-group sums all slots' partials in a fixed order into y.
+__device__ void epilogue_b(const MoeParams& p, const SlotTable& S, const float* rb0, int slot, int ncols, int rg,
+                           int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    float* dp = p.dpart + (long long)slot * p.T * p.H;
+    float D[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int w = 0; w < NCW; ++w) {
+        const float* r = rb0 + (w * 32 + lane) * 8;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) D[i] += r[i];
+    }
+    const int row0 = 16 * rg + g;
+#pragma unroll
+    for (int nb = 0; nb < 2; ++nb) {
+        const int col = 4 * nb + t;  // virtual columns 2col (hi), 2col+1 (lo)
+        if (col < ncols) {
+            dp[(long long)col * p.H + row0] = D[4 * nb + 0] + D[4 * nb + 1];
+            dp[(long long)col * p.H + row0 + 8] = D[4 * nb + 2] + D[4 * nb + 3];
+        }
+    }
+    __threadfence();
+    __syncwarp();
+    uint32_t prev = 0;
+    if (lane == 0) prev = atom_add_acq_rel_gpu(p.ctrl + MOE_CTRL_ROWBLK + rg, 1u);
+    prev = __shfl_sync(0xffffffffu, prev, 0);
+    if (prev != (uint32_t)S.nslots - 1) return;
+    __threadfence();
+    for (int it = lane; it < 16 * p.T; it += 32) {
+        const int row = 16 * rg + (it & 15), c = it >> 4;
+        float acc = 0.f;
+        for (int j = 0; j < p.k; ++j) {
+            const int s2 = S.tslot[c][j];
+            if (s2 < 0) continue;
+            const float v = __ldcg(p.dpart + ((long long)s2 * p.T + S.tpos[c][j]) * p.H + row);
+            acc = fmaf(S.w[c][j], v, acc);
+        }
+        if (p.has_shared) acc += __ldcg(p.dpart + (long long)c * p.H + row);
+        p.y[(long long)c * p.H + row] = acc;
+    }
+    __syncwarp();
+    if (lane == 0) p.ctrl[MOE_CTRL_ROWBLK + rg] = 0u;
+}
+
 __device__ void consumer(const MoeParams& p, Shared& sh, uint8_t* ring, uint8_t* xh, int hbytes_max, float* red) {
     const SlotTable& S = sh.st;
     const int w = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
     const int nrbA = p.I / 32, nrbB = p.H / 32;
-    int cc = 0, bseq = 0;
-    bool first_b = true;
-    for (int n = 0;; ++n) {
+    int cc = 0, bseq = 0, r = 0;
+    bool first_b = true, ok = true;
+    for (int n = 0; ok; ++n) {
         const int qi = n % QN;
-        if (!mbar_wait(&sh.tqf[qi], (n / QN) & 1, WAIT_LIMIT)) { set_error(p.ctrl, MOE_ERR_TIMEOUT); sh.abort_flag = 1; break; }
+        if (!mbar_wait(&sh.tqf[qi], (n / QN) & 1, WAIT_LIMIT)) { ok = false; break; }
         const int task = sh.tq[qi];
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh.tqe[qi]);
@@ -286,11 +378,6 @@ __device__ void consumer(const MoeParams& p, Shared& sh, uint8_t* ring, uint8_t*
         const int fmt = tk.kind == 0 ? (e < 0 ? p.fsA : p.fA) : (e < 0 ? p.fsB : p.fB);
         const int fullb = (int)rfx_chunk_bytes(fmt, 8);
         const int nch = rfx_num_chunks(K);
-        int c0, c1;
-        warp_chunk_range(w, nch, c0, c1);
-        Acc<1> a0, a1;
-        Acc<2> d2;
-        a0.zero(); a1.zero(); d2.zero();
         const int buf_h = bseq & 1;
         if (tk.kind == 1) {
             if (first_b) {
@@ -299,9 +386,8 @@ __device__ void consumer(const MoeParams& p, Shared& sh, uint8_t* ring, uint8_t*
                 if (lane == 0) mbar_arrive(&sh.xfree);
                 first_b = false;
             }
-            if (!mbar_wait(&sh.hfull[buf_h], (bseq >> 1) & 1, WAIT_LIMIT)) { set_error(p.ctrl, MOE_ERR_TIMEOUT); sh.abort_flag = 1; break; }
+            if (!mbar_wait(&sh.hfull[buf_h], (bseq >> 1) & 1, WAIT_LIMIT)) { ok = false; break; }
         }
-        // B-operand sources
         BSrc bs[2];
         if (tk.kind == 0) {
             const int col = g < ncols ? S.cols[slot][g] : 0;
@@ -317,178 +403,104 @@ __device__ void consumer(const MoeParams& p, Shared& sh, uint8_t* ring, uint8_t*
             }
         }
         const bool two_nb = tk.kind == 1 && ncols > 4;
-        bool ok = true;
-        for (int c = c0; c < c1; ++c) {
-            const int s = cc % p.ns;
-            if (!mbar_wait(&sh.full[w][s], (cc / p.ns) & 1, WAIT_LIMIT)) { ok = false; break; }
-            const uint8_t* st = ring + (w * p.ns + s) * MOE_STAGE_BYTES;
-            const int nt = rfx_chunk_tiles(K, c);
-            const int step0 = c * 16;
-            if (tk.kind == 0) {
-                switch (fmt) {
-                    case 2: chunk_any2<2, false, 1>(st, st + fullb, nt, lane, g, bs, step0, a0, a1); break;
-                    case 3: chunk_any2<3, false, 1>(st, st + fullb, nt, lane, g, bs, step0, a0, a1); break;
-                    default: chunk_any2<4, false, 1>(st, st + fullb, nt, lane, g, bs, step0, a0, a1); break;
+        for (int rgl = 0; rgl < 2 && ok; ++rgl) {
+            Acc<1> a0, a1;
+            Acc<2> d2;
+            a0.zero(); a1.zero(); d2.zero();
+            for (int c0 = 0; c0 < nch; c0 += MOE_CHUNKS_PER_STAGE) {
+                const int s = cc % p.ns;
+                if (!mbar_wait(&sh.full[s], (cc / p.ns) & 1, WAIT_LIMIT)) { ok = false; break; }
+                const int c = c0 + w;
+                if (c < nch) {
+                    const uint8_t* st = ring + s * MOE_STAGE_BYTES + w * fullb;
+                    const int nt = rfx_chunk_tiles(K, c);
+                    const int step0 = c * 16;
+                    if (tk.kind == 0) {
+                        switch (fmt) {
+                            case 2: chunk_any2<2, false, 1>(st, st + MOE_HALF_BYTES, nt, lane, g, bs, step0, a0, a1); break;
+                            case 3: chunk_any2<3, false, 1>(st, st + MOE_HALF_BYTES, nt, lane, g, bs, step0, a0, a1); break;
+                            default: chunk_any2<4, false, 1>(st, st + MOE_HALF_BYTES, nt, lane, g, bs, step0, a0, a1); break;
+                        }
+                    } else if (!two_nb) {
+                        switch (fmt) {
+                            case 2: chunk_any<2, true, 1>(st, nt, lane, g, bs, step0, a0); break;
+                            case 3: chunk_any<3, true, 1>(st, nt, lane, g, bs, step0, a0); break;
+                            default: chunk_any<4, true, 1>(st, nt, lane, g, bs, step0, a0); break;
+                        }
+                    } else {
+                        switch (fmt) {
+                            case 2: chunk_any<2, true, 2>(st, nt, lane, g, bs, step0, d2); break;
+                            case 3: chunk_any<3, true, 2>(st, nt, lane, g, bs, step0, d2); break;
+                            default: chunk_any<4, true, 2>(st, nt, lane, g, bs, step0, d2); break;
+                        }
+                    }
                 }
-            } else if (!two_nb) {
-                switch (fmt) {
-                    case 2: chunk_any<2, true, 1>(st, nt, lane, g, bs, step0, a0); break;
-                    case 3: chunk_any<3, true, 1>(st, nt, lane, g, bs, step0, a0); break;
-                    default: chunk_any<4, true, 1>(st, nt, lane, g, bs, step0, a0); break;
-                }
-            } else {
-                switch (fmt) {
-                    case 2: chunk_any<2, true, 2>(st, nt, lane, g, bs, step0, d2); break;
-                    case 3: chunk_any<3, true, 2>(st, nt, lane, g, bs, step0, d2); break;
-                    default: chunk_any<4, true, 2>(st, nt, lane, g, bs, step0, d2); break;
-                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sh.empty[s]);
+                ++cc;
+                if (w == 0 && lane == 0) sh.consumed = cc;
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sh.empty[w][s]);
-            ++cc;
-            if (lane == 0) sh.cc[w] = cc;
+            if (!ok) break;
+            float v[8];
+            if (tk.kind == 0) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) { v[i] = a0.v[0][i]; v[4 + i] = a1.v[0][i]; }
+            } else if (!two_nb) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) { v[i] = a0.v[0][i]; v[4 + i] = 0.f; }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) { v[i] = d2.v[0][i]; v[4 + i] = d2.v[1][i]; }
+            }
+            const bool last = red_deposit(sh, red, r, w, lane, v, ok);
+            if (!ok) break;
+            if (last) {
+                const float* rb0 = red + (r & 1) * NCW * 32 * 8;
+                const int rg = 2 * tk.rb + rgl;
+                if (tk.kind == 0) {
+                    epilogue_a(p, rb0, slot, ncols, rg, lane);
+                    if (rgl == 1) {
+                        // both row-groups of the task are in h: publish
+                        fence_proxy_async_global();
+                        __threadfence();
+                        __syncwarp();
+                        if (lane == 0) atom_add_release_gpu(p.ctrl + MOE_CTRL_SLOT + slot, 1u);
+                    }
+                } else {
+                    epilogue_b(p, S, rb0, slot, ncols, rg, lane);
+                }
+                red_release(sh, r, lane);
+            }
+            ++r;
         }
-        if (!ok) { set_error(p.ctrl, MOE_ERR_TIMEOUT); sh.abort_flag = 1; break; }
+        if (!ok) break;
         if (tk.kind == 1) {
             __syncwarp();
             if (lane == 0) mbar_arrive(&sh.hfree[buf_h]);
             ++bseq;
         }
-        // ---- K-quarter reduction: the last warp to arrive finishes the task
-        const int rbuf = n & 1;
-        float* myred = red + ((rbuf * NCW + w) * 32 + lane) * 8;
-        {
-            const long long t0 = clock64();
-            while (sh.repoch[rbuf] != n - 2) {
-                if (clock64() - t0 > WAIT_LIMIT) { ok = false; break; }
-            }
-        }
-        if (!ok) { set_error(p.ctrl, MOE_ERR_TIMEOUT); sh.abort_flag = 1; break; }
-        if (tk.kind == 0) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) { myred[i] = a0.v[0][i]; myred[4 + i] = a1.v[0][i]; }
-        } else if (!two_nb) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) { myred[i] = a0.v[0][i]; myred[4 + i] = 0.f; }
-        } else {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) { myred[i] = d2.v[0][i]; myred[4 + i] = d2.v[1][i]; }
-        }
-        __threadfence_block();
-        __syncwarp();
-        int old = 0;
-        if (lane == 0) old = atomicAdd(&sh.rcnt[rbuf], 1);
-        old = __shfl_sync(0xffffffffu, old, 0);
-        if (old != NCW - 1) continue;
-        __threadfence_block();
-        const float* rb0 = red + rbuf * NCW * 32 * 8;
-        if (tk.kind == 0) {
-            // SwiGLU -> h (fp16 hi/lo pair per value) in the fragment order of
-            // the down projection's B operand: [step][v][t'][4]
-            uint16_t* hs = p.hbuf + (long long)slot * (2LL * p.T * p.I);
-            uint32_t bad = 0;
-#pragma unroll
-            for (int rgl = 0; rgl < 2; ++rgl) {
-                float G[4] = {0.f, 0.f, 0.f, 0.f}, U[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int kq = 0; kq < 4; ++kq) {
-                    const float* r = rb0 + ((2 * kq + rgl) * 32 + lane) * 8;
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) { G[i] += r[i]; U[i] += r[4 + i]; }
-                }
-                const int step = 2 * tk.rb + rgl;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int col = 2 * t + (i & 1);
-                    const int rowhi = i >> 1;  // 0: row g, 1: row g+8
-                    if (col >= ncols) continue;
-                    const float gv = G[i];
-                    const float h = gv / (1.0f + expf(-gv)) * U[i];
-                    const __half hi = __float2half_rn(h);
-                    const __half lo = __float2half_rn(h - __half2float(hi));
-                    if (!(fabsf(h) <= 65504.0f)) bad = 1;
-                    const int tp = g >> 1, pos = 2 * rowhi + (g & 1);
-                    const long long base = ((long long)(step * 2 * ncols) * 4 + tp) * 4 + pos;
-                    hs[base + (long long)(2 * col) * 16] = __half_as_ushort(hi);
-                    hs[base + (long long)(2 * col + 1) * 16] = __half_as_ushort(lo);
-                }
-            }
-            if (__any_sync(0xffffffffu, bad) && lane == 0) set_error(p.ctrl, MOE_ERR_RANGE);
-            fence_proxy_async_global();
-            __threadfence();
-            __syncwarp();
-            if (lane == 0) atom_add_release_gpu(p.ctrl + MOE_CTRL_SLOT + slot, 1u);
-        } else {
-            float* dp = p.dpart + (long long)slot * p.T * p.H;
-#pragma unroll
-            for (int rgl = 0; rgl < 2; ++rgl) {
-                float D[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int kq = 0; kq < 4; ++kq) {
-                    const float* r = rb0 + ((2 * kq + rgl) * 32 + lane) * 8;
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) D[i] += r[i];
-                }
-                const int row0 = 32 * tk.rb + 16 * rgl + g;
-#pragma unroll
-                for (int nb = 0; nb < 2; ++nb) {
-                    const int col = 4 * nb + t;  // virtual columns 2col (hi), 2col+1 (lo)
-                    if (col < ncols) {
-                        dp[(long long)col * p.H + row0] = D[4 * nb + 0] + D[4 * nb + 1];
-                        dp[(long long)col * p.H + row0 + 8] = D[4 * nb + 2] + D[4 * nb + 3];
-                    }
-                }
-            }
-            __threadfence();
-            __syncwarp();
-            uint32_t prev = 0;
-            if (lane == 0) prev = atom_add_acq_rel_gpu(p.ctrl + MOE_CTRL_ROWBLK + tk.rb, 1u);
-            prev = __shfl_sync(0xffffffffu, prev, 0);
-            if (prev == (uint32_t)S.nslots - 1) {
-                __threadfence();
-                const int row = 32 * tk.rb + lane;
-                for (int c = 0; c < p.T; ++c) {
-                    float acc = 0.f;
-                    for (int j = 0; j < p.k; ++j) {
-                        const int s2 = S.tslot[c][j];
-                        if (s2 < 0) continue;
-                        const float v = __ldcg(p.dpart + ((long long)s2 * p.T + S.tpos[c][j]) * p.H + row);
-                        acc = fmaf(S.w[c][j], v, acc);
-                    }
-                    if (p.has_shared) acc += __ldcg(p.dpart + (long long)c * p.H + row);
-                    p.y[(long long)c * p.H + row] = acc;
-                }
-                __syncwarp();
-                if (lane == 0) p.ctrl[MOE_CTRL_ROWBLK + tk.rb] = 0u;
-            }
-        }
-        __syncwarp();
-        if (lane == 0) {
-            sh.rcnt[rbuf] = 0;
-            __threadfence_block();
-            sh.repoch[rbuf] = n;
-        }
-        __syncwarp();
+    }
+    if (!ok) {
+        set_error(p.ctrl, MOE_ERR_TIMEOUT);
+        sh.abort_flag = 1;
     }
 }
 
-template <int FA, int FB>
 __global__ void __launch_bounds__(NTHREADS, 1) moe_decode_kernel(MoeParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t* ring = base;
-    uint8_t* xh = ring + NCW * p.ns * MOE_STAGE_BYTES;
+    uint8_t* xh = ring + p.ns * MOE_STAGE_BYTES;
     float* red = (float*)(xh + p.xh_bytes);
     Shared& sh = *(Shared*)((uint8_t*)red + 2 * NCW * 32 * 8 * sizeof(float));
     const int hbytes_max = 4 * p.T * p.I;
     const int w = threadIdx.x >> 5;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < NCW; ++i)
-            for (int s = 0; s < p.ns; ++s) {
-                mbar_init(&sh.full[i][s], 1);
-                mbar_init(&sh.empty[i][s], 1);
-            }
+        for (int s = 0; s < p.ns; ++s) {
+            mbar_init(&sh.full[s], 1);
+            mbar_init(&sh.empty[s], NCW);
+        }
         for (int i = 0; i < QN; ++i) {
             mbar_init(&sh.tqf[i], 1);
             mbar_init(&sh.tqe[i], NCW);
@@ -501,7 +513,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_decode_kernel(MoeParams p) {
         }
         mbar_init(&sh.xfree, NCW);
         sh.abort_flag = 0;
-        for (int i = 0; i < NCW; ++i) sh.cc[i] = 0;
+        sh.consumed = 0;
         fence_barrier_init();
     }
     if (w == NCW) {
@@ -512,8 +524,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_decode_kernel(MoeParams p) {
         const uint32_t* x32 = (const uint32_t*)p.x;
         for (int i = threadIdx.x; i < npairs; i += NCW * 32) {
             const int c = (2 * i) / p.H, k = (2 * i) % p.H;
-            const int step = k >> 4, r = k & 15;
-            const int tt = (r & 7) >> 1, half = r >> 3;
+            const int step = k >> 4, rr = k & 15;
+            const int tt = (rr & 7) >> 1, half = rr >> 3;
             *(uint32_t*)(xh + c * p.x_stride + (step * 4 + tt) * 8 + half * 4) = x32[i];
         }
     }
@@ -521,7 +533,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_decode_kernel(MoeParams p) {
     if (w == NCW) {
         if ((threadIdx.x & 31) == 0) producer(p, sh, ring, xh, hbytes_max);
     } else {
-        consumer<FA, FB>(p, sh, ring, xh, hbytes_max, red);
+        consumer(p, sh, ring, xh, hbytes_max, red);
     }
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -539,14 +551,23 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_decode_kernel(MoeParams p) {
 
 // Shared-memory bytes of a launch (plus 1 KB alignment slack).
 size_t moe_decode_smem_bytes(int ns, int xh_bytes) {
-    return 1024 + (size_t)NCW * ns * MOE_STAGE_BYTES + xh_bytes + 2 * NCW * 32 * 8 * sizeof(float) + sizeof(Shared);
+    return 1024 + (size_t)ns * MOE_STAGE_BYTES + xh_bytes + 2 * NCW * 32 * 8 * sizeof(float) + sizeof(Shared);
 }
 
 cudaError_t moe_decode_launch(const MoeParams& p, int grid, cudaStream_t stream) {
     const size_t smem = moe_decode_smem_bytes(p.ns, p.xh_bytes);
-    auto kern = moe_decode_kernel<0, 0>;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = moe_decode_kernel;
+    // raise the dynamic shared-memory limit once (not a stream operation, so
+    // it stays out of any graph capture after the first call)
+    static int set_bytes[64] = {0};
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
+    if (dev < 64 && set_bytes[dev] < (int)smem) {
+        err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (err != cudaSuccess) return err;
+        set_bytes[dev] = (int)smem;
+    }
     kern<<<grid, NTHREADS, smem, stream>>>(p);
     return cudaGetLastError();
 }

@@ -9,7 +9,9 @@
 #define MOE_MAXK 8            // routed experts per token
 #define MOE_MAXS (MOE_MAXT * MOE_MAXK + 1)
 #define MOE_MAX_STAGES 6
-#define MOE_STAGE_BYTES 4352  // two full FP4 chunks (gate + up)
+#define MOE_CHUNKS_PER_STAGE 8
+#define MOE_HALF_BYTES 17408   // 8 full FP4 chunks of one matrix
+#define MOE_STAGE_BYTES 34816  // gate + up halves
 
 // workspace control words (uint32)
 #define MOE_CTRL_TASK 0
@@ -57,7 +59,7 @@ struct MoeWs {
 inline MoeWs moe_ws_layout(int T, int k, int H, int I) {
     MoeWs L;
     const size_t ns = (size_t)T * k + 1;
-    const size_t ctrl_words = MOE_CTRL_ROWBLK + (size_t)H / 32;
+    const size_t ctrl_words = MOE_CTRL_ROWBLK + (size_t)H / 16;
     L.ctrl_off = 0;
     L.h_off = (ctrl_words * 4 + 255) / 256 * 256;
     L.d_off = L.h_off + (ns * 4 * T * I + 255) / 256 * 256;

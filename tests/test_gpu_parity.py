@@ -56,7 +56,7 @@ def test_device_pack_equals_host_pack(fmt, rows, cols):
 @pytest.mark.parametrize("T,E,k", [(64, 256, 6), (5, 8, 2), (3, 16, 16), (7, 1000, 8), (1, 40, 3)])
 def test_router_bit_exact(T, E, k):
     L = synth.logits(11, 0, 0, T, E, 1.1 if E == 256 else 0.0)
-    L[0, 3] = L[0, 7] = L[0, 9] = 9.0           # ties go to the lower index
+    L[0, 1] = L[0, E // 2] = L[0, E - 1] = 9.0   # ties go to the lower index
     if T > 1:
         L[1, :] = 0.5                           # all equal
     idx_o, w_o = oracle.router_topk(L, k)
