@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--copies", type=int, default=COPIES, help="rotating layer copies (>= 8 keeps steps L2-cold)")
+    ap.add_argument("--only-q1", action="store_true", help="skip the q=4 verify measurement")
     return ap.parse_args()
 
 
@@ -180,7 +182,7 @@ def run_reference(args, rank, world):
 class Workload:
     """C rotating copies of one synthetic full-size layer plus seeded inputs."""
 
-    def __init__(self, q: int, ntok: int, dev):
+    def __init__(self, q: int, ntok: int, dev, copies: int = COPIES):
         import torch
         import numpy as np
         import synth
@@ -190,7 +192,8 @@ class Workload:
         self.base = base
         self.layers = [base.moe_layer(max_T=q)]
         self._keep = [base]
-        for c in range(1, COPIES):
+        self.copies = copies
+        for c in range(1, copies):
             bufs = [b.clone() for b in base.bufs]
             sh = [b.clone() for b in base.shared]
             import block_quantized_moe_rocmfpx_b200 as rfx
@@ -207,7 +210,7 @@ class Workload:
         self.x = torch.from_numpy(self.x_h).view(torch.bfloat16).to(dev).view(ntok, q, H)
         self.idx = torch.empty((ntok, q, K_TOP), dtype=torch.int32, device=dev)
         self.w = torch.empty((ntok, q, K_TOP), dtype=torch.float32, device=dev)
-        self.y = torch.empty((COPIES, q, H), dtype=torch.float32, device=dev)
+        self.y = torch.empty((copies, q, H), dtype=torch.float32, device=dev)
 
     def step(self, t: int, route: bool = True, ffn: bool = True):
         import block_quantized_moe_rocmfpx_b200 as rfx
@@ -215,7 +218,7 @@ class Workload:
         if route:
             rfx.moe_router_topk(self.logits[s], K_TOP, self.idx[s], self.w[s])
         if ffn:
-            self.layers[t % COPIES].forward(self.x[s], self.idx[s], self.w[s], self.y[t % COPIES])
+            self.layers[t % self.copies].forward(self.x[s], self.idx[s], self.w[s], self.y[t % self.copies])
 
     def algo_bytes(self, tokens) -> float:
         """Bytes one pass must move: packed blocks of the union of routed
@@ -252,10 +255,10 @@ def time_graph(g, stream):
     return e0.elapsed_time(e1)
 
 
-def measure(q: int, steps: int, warmup: int, dev, rank, world, want_clocks: bool, want_e2e: bool):
+def measure(q: int, steps: int, warmup: int, dev, rank, world, want_clocks: bool, want_e2e: bool, copies: int):
     import torch
     import torch.distributed as dist
-    wl = Workload(q, NTOK, dev)
+    wl = Workload(q, NTOK, dev, copies)
     stream = torch.cuda.Stream(device=dev)
     with torch.cuda.stream(stream):
         for t in range(3):            # eager warm-up (kernel attributes, lazy loading)
@@ -323,7 +326,7 @@ def e2e(wl, steps, stream):
         xd.copy_(xh[t], non_blocking=True)
         ld.copy_(lh[t], non_blocking=True)
         rfx.moe_router_topk(ld, K_TOP, idx, w)
-        wl.layers[t % COPIES].forward(xd, idx, w, yd)
+        wl.layers[t % wl.copies].forward(xd, idx, w, yd)
         yh[t].copy_(yd, non_blocking=True)
 
     with torch.cuda.stream(stream):
@@ -361,8 +364,9 @@ def main():
         __graft_entry__.build()
     if world > 1:
         dist.barrier()
-    r1 = measure(1, args.steps, max(3, args.warmup), dev, rank, world, True, not args.no_e2e)
-    r4 = measure(4, args.steps, max(3, args.warmup), dev, rank, world, False, False)
+    r1 = measure(1, args.steps, max(3, args.warmup), dev, rank, world, True, not args.no_e2e, args.copies)
+    r4 = r1 if args.only_q1 else measure(4, args.steps, max(3, args.warmup), dev, rank, world, False, False,
+                                         args.copies)
 
     def reduce_max(v):
         if world == 1:
@@ -394,7 +398,7 @@ def main():
                                    "FP2 gate/up, FP3 down, FP4 shared; 2.30 GB packed), 1000 seeded tokens, "
                                    "Zipf(1.1) routing", "global_batch": world, "seq_len": 1,
                        "parallelism": "replicas" if world > 1 else "single",
-                       "l2": f"inputs larger than L2: {COPIES} rotating copies of the layer",
+                       "l2": f"inputs larger than L2: {args.copies} rotating copies of the layer",
                        "graph": "CUDA graph of all timed steps"},
             "roofline": {"bound": "hbm", "achieved": gbs1, "peak": peak, "unit": "GB/s", "frac": gbs1 / peak,
                          "traffic": None, "kernel": "moe_decode_kernel", "peak_kind": peak_kind,

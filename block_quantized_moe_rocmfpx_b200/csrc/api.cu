@@ -185,13 +185,18 @@ int moe_prepare(const moe_layer* layer, const void* x, int T, const int32_t* idx
     p.hbuf = (uint16_t*)(wsb + L.h_off);
     p.dpart = (float*)(wsb + L.d_off);
     p.x_stride = d.H / 16 * 32 + 32;
-    const size_t xb = (size_t)T * p.x_stride, hb = 2 * (size_t)4 * T * d.I;
+    const int nxc = (d.has_shared && d.f_sh_gate != d.f_gate) ? 2 : 1;
+    const size_t xb = (size_t)nxc * T * p.x_stride + (size_t)nxc * T * moe_sxs(d.H) * 4;
+    const size_t hb = 2 * (size_t)4 * T * (d.I + moe_sstr(d.I));
     p.xh_bytes = (int)((std::max(xb, hb) + 127) / 128 * 128);
+    // deepest ring first (memory in flight), then as many reduction buffers as fit
     p.ns = 0;
-    for (int ns = MOE_MAX_STAGES; ns >= 2; --ns)
-        if (moe_decode_smem_bytes(ns, p.xh_bytes) <= (size_t)smem_optin) { p.ns = ns; break; }
+    p.nred = 0;
+    for (int ns = 4; ns >= 2 && !p.ns; --ns)
+        for (int nr = MOE_MAX_RED; nr >= 4; --nr)
+            if (moe_decode_smem_bytes(ns, nr, p.xh_bytes) <= (size_t)smem_optin) { p.ns = ns; p.nred = nr; break; }
     if (!p.ns) return rfx_fail(RFX_EUNSUPPORTED, "moe_ffn_forward: shapes need more shared memory than the device has");
-    smem = moe_decode_smem_bytes(p.ns, p.xh_bytes);
+    smem = moe_decode_smem_bytes(p.ns, p.nred, p.xh_bytes);
     grid = sms;
     return RFX_OK;
 }

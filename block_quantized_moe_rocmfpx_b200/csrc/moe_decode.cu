@@ -19,13 +19,17 @@
 //  - Tasks: A = (slot, 32 gate/up rows) -> SwiGLU -> h; B = (slot, 32 down
 //    rows) -> partial d.  Tasks are handed out by a global atomic counter, A
 //    before B, so a B task only ever waits on A tasks already running.
-//  - Per CTA: one producer warp streams packed chunks HBM -> shared memory with
-//    1-D bulk copies (TMA, evict-first L2 policy) into per-warp stage rings;
-//    8 consumer warps (2 row-groups x 4 K-quarters) decode in registers and
-//    run mma.sync m16n8k16 (bf16 x for gate/up, fp16 hi/lo split of h for
-//    down).  K-quarter partials are reduced in shared memory by the last warp
-//    to arrive, in a fixed order.
-//  - Combine: the last B task to finish a 32-row block sums the slots'
+//  - Per CTA: lane 0 of the producer warp streams packed spans of 8 chunks
+//    HBM -> shared memory with 1-D bulk copies (TMA, evict-first L2 policy)
+//    into a ring of stages; lane 1 bulk-copies the SwiGLU output h of a slot
+//    once all of its gate/up rows are published.  8 consumer warps take one
+//    chunk of every stage each, decode it in registers (one AND per A
+//    register, see rfx_tile.cuh) and run mma.sync m16n8k16 in fp16: x
+//    normalised per column by a power of two for gate/up, an exact hi/lo fp16
+//    split of h for down.  3 epilogue warps sum the 8 warps' partials of
+//    each row-group in a fixed order and run SwiGLU or the combine, so the
+//    consumers never wait on global-memory latency.
+//  - Combine: the last down task to finish a 16-row group sums the slots'
 //    partials in a fixed order (routing order j, then shared), so y does not
 //    depend on scheduling and column t is bitwise the same for any T.
 //  - Every wait is bounded; a timeout sets a workspace error flag and the CTA
@@ -37,9 +41,14 @@
 
 namespace rfx {
 
-constexpr int NCW = 8;
-constexpr int NTHREADS = (NCW + 1) * 32;
+constexpr int NCW = 8;                       // consumer warps 0..7
+constexpr int WARP_PRODUCER = NCW;           // bulk-copy issue (one lane)
+constexpr int NEPI = 3;                      // epilogue warps: reductions, SwiGLU, combine
+constexpr int WARP_EPILOGUE0 = NCW + 1;
+constexpr int NTHREADS = (NCW + 1 + NEPI) * 32;
 constexpr int QN = 4;
+constexpr int NRED_MAX = MOE_MAX_RED;        // reduction buffers: unit r -> buffer r % p.nred,
+                                             // epilogue warp r % NEPI
 constexpr long long WAIT_LIMIT = 4000000000LL;
 
 struct SlotTable {
@@ -52,6 +61,13 @@ struct SlotTable {
     float w[MOE_MAXT][MOE_MAXK];
     unsigned mask[32];
     int prefix[32];
+    int idx[MOE_MAXT * MOE_MAXK];
+    unsigned char ok[MOE_MAXT * MOE_MAXK];
+};
+
+struct RedInfo {
+    int kind;      // 0: gate/up row-group, 1: down row-group, -1: end of work
+    int slot, ncols, rg, last_of_task;
 };
 
 struct Shared {
@@ -60,11 +76,16 @@ struct Shared {
     uint64_t tqf[QN], tqe[QN];
     uint64_t hfull[2], hfree[2];
     uint64_t xfree;
+    uint64_t xload;          // x bulk copy into the (not yet used) stage ring
+    uint64_t rfull[NRED_MAX], rempty[NRED_MAX];
+    uint64_t hqf[QN], hqe[QN];
+    int hq[QN];
     int tq[QN];
-    int rcnt[2];
-    volatile int repoch[2];
+    RedInfo rinfo[NRED_MAX];
     volatile int abort_flag;
     volatile int consumed;   // stages released by all consumer warps (for the abort drain)
+    unsigned xmax[MOE_MAXT]; // max |x| per column (fp32 bits)
+    int xn[MOE_MAXT];        // x is staged as x * 2^xn[c] (then 2^-s_b per tile position)
     SlotTable st;
 };
 
@@ -84,16 +105,21 @@ __device__ __forceinline__ void set_error(uint32_t* ctrl, uint32_t bits) { atomi
 __device__ void build_slots(const MoeParams& p, SlotTable& S) {
     const int lane = threadIdx.x & 31;
     const int n = p.T * p.k;
-    if (lane < 32) S.mask[lane] = 0u;
+    // one coalesced read of the routing into shared memory, then work from there
+    for (int i = lane; i < n; i += 32) {
+        S.idx[i] = p.idx[i];
+        S.w[i / p.k][i % p.k] = p.wts[i];
+    }
+    S.mask[lane] = 0u;
     __syncwarp();
     for (int i = lane; i < n; i += 32) {
         const int c = i / p.k, j = i % p.k;
-        int e = p.idx[i];
+        const int e = S.idx[i];
         bool ok = e >= 0 && e < p.E;
         if (!ok) set_error(p.ctrl, MOE_ERR_EXPERT);
         for (int jj = 0; jj < j && ok; ++jj)
-            if (p.idx[c * p.k + jj] == e) { ok = false; set_error(p.ctrl, MOE_ERR_DUP); }
-        S.w[c][j] = p.wts[i];
+            if (S.idx[c * p.k + jj] == e) { ok = false; set_error(p.ctrl, MOE_ERR_DUP); }
+        S.ok[i] = ok ? 1 : 0;
         S.tslot[c][j] = -1;
         if (ok) atomicOr(&S.mask[e >> 5], 1u << (e & 31));
     }
@@ -110,23 +136,19 @@ __device__ void build_slots(const MoeParams& p, SlotTable& S) {
         S.prefix[lane] = incl - pc;
         if (lane == 31) S.nslots = base + incl;
     }
-    __syncwarp();
     for (int s = lane; s < MOE_MAXS; s += 32) S.ncols[s] = 0;
     __syncwarp();
     for (int i = lane; i < n; i += 32) {
+        if (!S.ok[i]) continue;
         const int c = i / p.k, j = i % p.k;
-        const int e = p.idx[i];
-        bool ok = e >= 0 && e < p.E;
-        for (int jj = 0; jj < j && ok; ++jj)
-            if (p.idx[c * p.k + jj] == e) ok = false;
-        if (!ok) continue;
+        const int e = S.idx[i];
         const int s = base + S.prefix[e >> 5] + __popc(S.mask[e >> 5] & ((1u << (e & 31)) - 1u));
         // position of column c among the columns routing to e (columns ascend);
         // each earlier column counts once even if it repeats e (flagged above)
         int pos = 0;
         for (int c2 = 0; c2 < c; ++c2) {
             for (int j2 = 0; j2 < p.k; ++j2)
-                if (p.idx[c2 * p.k + j2] == e) { ++pos; break; }
+                if (S.idx[c2 * p.k + j2] == e) { ++pos; break; }
         }
         S.expert[s] = e;
         S.cols[s][pos] = (signed char)c;
@@ -163,126 +185,140 @@ __device__ __forceinline__ MatRef slot_mats(const MoeParams& p, int e, int kind)
 // Per task (32 rows = 2 row-groups) and per row-group, one stage per span of
 // up to 8 chunks: a single bulk copy per matrix of the contiguous span.
 
-__device__ void producer(const MoeParams& p, Shared& sh, uint8_t* ring, uint8_t* xh, int hbytes_max) {
+__device__ void producer(const MoeParams& p, Shared& sh, uint8_t* ring) {
     const SlotTable& S = sh.st;
     const int nrbA = p.I / 32, nrbB = p.H / 32;
     const int ntasks = S.nslots * (nrbA + nrbB);
     const uint64_t pol_w = policy_evict_first();
-    const uint64_t pol_h = policy_evict_last();
-    int sc = 0, bseq = 0;
+    int stage = 0;
+    uint32_t ephase = 1;          // parity to wait for on empty[stage] (fresh barriers pass)
+    int sc = 0;
     bool ok = true;
     int next = (int)atomicAdd(p.ctrl + MOE_CTRL_TASK, 1u);
+    int qi = 0, hi = 0;
+    uint32_t qphase = 1, hphase = 1;
     for (int n = 0; ok; ++n) {
         int t = next;
         if (t >= ntasks) t = -1;
-        else next = (int)atomicAdd(p.ctrl + MOE_CTRL_TASK, 1u);   // overlaps with this task's copies
-        const int qi = n % QN;
-        if (!mbar_wait(&sh.tqe[qi], ((n / QN) + 1) & 1, WAIT_LIMIT)) { ok = false; break; }
+        else next = (int)atomicAdd(p.ctrl + MOE_CTRL_TASK, 1u);   // used next iteration: latency hidden
+        if (!mbar_wait(&sh.tqe[qi], qphase, WAIT_LIMIT)) { ok = false; break; }
         sh.tq[qi] = t;
         mbar_arrive(&sh.tqf[qi]);
+        if (++qi == QN) { qi = 0; qphase ^= 1u; }
         if (t < 0) break;
         const Task tk = decode_task(t, S.nslots, nrbA, nrbB);
+        if (tk.kind == 1) {
+            // hand the h copy of this down task to the h lane
+            if (!mbar_wait(&sh.hqe[hi], hphase, WAIT_LIMIT)) { ok = false; break; }
+            sh.hq[hi] = tk.slot;
+            mbar_arrive(&sh.hqf[hi]);
+            if (++hi == QN) { hi = 0; hphase ^= 1u; }
+        }
         const int e = S.expert[tk.slot];
         const MatRef m = slot_mats(p, e, tk.kind);
         const int K = tk.kind == 0 ? p.H : p.I;
         const int nch = rfx_num_chunks(K);
         const long long rgb = rfx_rowgroup_bytes(m.fmt, K);
         const int fullb = (int)rfx_chunk_bytes(m.fmt, 8);
-        if (tk.kind == 1) {
-            if (bseq == 0 && !mbar_wait(&sh.xfree, 0, WAIT_LIMIT)) { ok = false; break; }
-            const int buf = bseq & 1;
-            if (!mbar_wait(&sh.hfree[buf], ((bseq >> 1) + 1) & 1, WAIT_LIMIT)) { ok = false; break; }
-            const uint32_t need = (uint32_t)nrbA;
-            const long long t0 = clock64();
-            while (ld_acquire_gpu(p.ctrl + MOE_CTRL_SLOT + tk.slot) < need) {
-                if (clock64() - t0 > WAIT_LIMIT) { ok = false; break; }
-                __nanosleep(32);
-            }
-            if (!ok) break;
-            fence_proxy_async_global();
-            const uint32_t hb = 4u * (uint32_t)S.ncols[tk.slot] * (uint32_t)p.I;
-            mbar_arrive_expect_tx(&sh.hfull[buf], hb);
-            bulk_g2s(xh + buf * hbytes_max, p.hbuf + (long long)tk.slot * (2LL * p.T * p.I), hb, &sh.hfull[buf],
-                     pol_h);
-            ++bseq;
-        }
+        const uint32_t lastb = (uint32_t)rfx_chunk_bytes(m.fmt, rfx_chunk_tiles(K, nch - 1));
+        const uint8_t* srcA = m.a + (long long)(2 * tk.rb) * rgb;
+        const uint8_t* srcB = tk.kind == 0 ? m.b + (long long)(2 * tk.rb) * rgb : nullptr;
         for (int rgl = 0; rgl < 2 && ok; ++rgl) {
-            const long long rgoff = (long long)(2 * tk.rb + rgl) * rgb;
             for (int c0 = 0; c0 < nch; c0 += MOE_CHUNKS_PER_STAGE) {
                 const int c1 = min(nch, c0 + MOE_CHUNKS_PER_STAGE);
-                // bytes of chunks [c0, c1): full chunks plus a possibly partial last one
-                const uint32_t bytes = (uint32_t)((c1 - 1 - c0) * fullb + rfx_chunk_bytes(m.fmt, rfx_chunk_tiles(K, c1 - 1)));
-                const int s = sc % p.ns;
-                if (!mbar_wait(&sh.empty[s], ((sc / p.ns) + 1) & 1, WAIT_LIMIT)) { ok = false; break; }
-                uint8_t* dst = ring + s * MOE_STAGE_BYTES;
-                const long long off = rgoff + (long long)c0 * fullb;
+                const uint32_t bytes = (uint32_t)((c1 - 1 - c0) * fullb) + (c1 == nch ? lastb : (uint32_t)fullb);
+                if (!mbar_wait(&sh.empty[stage], ephase, WAIT_LIMIT)) { ok = false; break; }
+                uint8_t* dst = ring + stage * MOE_STAGE_BYTES;
+                const long long off = (long long)rgl * rgb + (long long)c0 * fullb;
                 if (tk.kind == 0) {
-                    mbar_arrive_expect_tx(&sh.full[s], 2 * bytes);
-                    bulk_g2s(dst, m.a + off, bytes, &sh.full[s], pol_w);
-                    bulk_g2s(dst + MOE_HALF_BYTES, m.b + off, bytes, &sh.full[s], pol_w);
+                    mbar_arrive_expect_tx(&sh.full[stage], 2 * bytes);
+                    bulk_g2s(dst, srcA + off, bytes, &sh.full[stage], pol_w);
+                    bulk_g2s(dst + MOE_HALF_BYTES, srcB + off, bytes, &sh.full[stage], pol_w);
                 } else {
-                    mbar_arrive_expect_tx(&sh.full[s], bytes);
-                    bulk_g2s(dst, m.a + off, bytes, &sh.full[s], pol_w);
+                    mbar_arrive_expect_tx(&sh.full[stage], bytes);
+                    bulk_g2s(dst, srcA + off, bytes, &sh.full[stage], pol_w);
                 }
                 ++sc;
+                if (++stage == p.ns) { stage = 0; ephase ^= 1u; }
             }
         }
+    }
+    // stop the h lane
+    if (mbar_wait(&sh.hqe[hi], hphase, WAIT_LIMIT)) {
+        sh.hq[hi] = -1;
+        mbar_arrive(&sh.hqf[hi]);
+    } else {
+        ok = false;
     }
     if (!ok) {
         set_error(p.ctrl, MOE_ERR_TIMEOUT);
         sh.abort_flag = 1;
         // drain: wait (bounded) until every issued copy has landed
         for (int i = sh.consumed; i < sc; ++i) (void)mbar_wait(&sh.full[i % p.ns], (i / p.ns) & 1, WAIT_LIMIT);
+        for (int q = 0; q < QN; ++q) {
+            sh.tq[q] = -1;
+            mbar_arrive(&sh.tqf[q]);
+        }
+    }
+}
+
+// The h lane: for each down task, in order, wait until every gate/up
+// row-group of its slot is published, then bulk-copy the slot's h and its
+// block sums (and nothing of the weight stream waits on this).
+__device__ void h_loader(const MoeParams& p, Shared& sh, uint8_t* xh, int hbytes_max, int sstr) {
+    const SlotTable& S = sh.st;
+    const uint64_t pol_h = policy_evict_last();
+    const uint32_t need = (uint32_t)(p.I / 16);
+    int hi = 0;
+    uint32_t hphase = 0;
+    int bseq = 0;
+    uint32_t known_ready[3] = {0u, 0u, 0u};   // slots already seen complete (bit per slot)
+    bool ok = true;
+    while (true) {
+        if (!mbar_wait(&sh.hqf[hi], hphase, WAIT_LIMIT)) { ok = false; break; }
+        const int slot = sh.hq[hi];
+        mbar_arrive(&sh.hqe[hi]);
+        if (++hi == QN) { hi = 0; hphase ^= 1u; }
+        if (slot < 0) break;
+        if (bseq == 0 && !mbar_wait(&sh.xfree, 0, WAIT_LIMIT)) { ok = false; break; }
+        const int buf = bseq & 1;
+        if (!mbar_wait(&sh.hfree[buf], ((bseq >> 1) + 1) & 1, WAIT_LIMIT)) { ok = false; break; }
+        if (!(known_ready[slot >> 5] >> (slot & 31) & 1u)) {
+            const long long t0 = clock64();
+            while (ld_relaxed_gpu(p.ctrl + MOE_CTRL_SLOT + slot) < need) {
+                if (clock64() - t0 > WAIT_LIMIT) { ok = false; break; }
+                __nanosleep(20);
+            }
+            if (!ok) break;
+            known_ready[slot >> 5] |= 1u << (slot & 31);
+        }
+        fence_acq_rel_gpu();          // acquire side of the publishers' release
+        fence_proxy_async_global();   // generic-proxy writes of h -> bulk-copy (async proxy) reads
+        const uint32_t hb = 4u * (uint32_t)S.ncols[slot] * (uint32_t)(p.I + sstr);
+        mbar_arrive_expect_tx(&sh.hfull[buf], hb);
+        bulk_g2s(xh + buf * hbytes_max, p.hbuf + (long long)slot * (2LL * p.T * (p.I + sstr)), hb, &sh.hfull[buf],
+                 pol_h);
+        ++bseq;
+    }
+    if (!ok) {
+        set_error(p.ctrl, MOE_ERR_TIMEOUT);
+        sh.abort_flag = 1;
         for (int b = 0; b < 2 && b < bseq; ++b)
             (void)mbar_wait(&sh.hfull[(bseq - 1 - b) & 1], ((bseq - 1 - b) >> 1) & 1, WAIT_LIMIT);
-        for (int qi = 0; qi < QN; ++qi) {
-            sh.tq[qi] = -1;
-            mbar_arrive(&sh.tqf[qi]);
-        }
     }
 }
 
-// ------------------------------------------------------------- consumers ---
+// ------------------------------------------------------------- epilogues ---
 
-// The last of the NCW warps to deposit its partial sums for row-group unit r
-// returns true (and must call red_release afterwards).
-__device__ __forceinline__ bool red_deposit(Shared& sh, float* red, int r, int w, int lane, const float v[8],
-                                            bool& ok) {
-    const int rbuf = r & 1;
-    {
-        const long long t0 = clock64();
-        while (sh.repoch[rbuf] != r - 2) {
-            if (clock64() - t0 > WAIT_LIMIT) { ok = false; return false; }
-        }
-    }
-    float* my = red + ((rbuf * NCW + w) * 32 + lane) * 8;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) my[i] = v[i];
-    __threadfence_block();
-    __syncwarp();
-    int old = 0;
-    if (lane == 0) old = atomicAdd(&sh.rcnt[rbuf], 1);
-    old = __shfl_sync(0xffffffffu, old, 0);
-    if (old != NCW - 1) return false;
-    __threadfence_block();
-    return true;
-}
-
-__device__ __forceinline__ void red_release(Shared& sh, int r, int lane) {
-    __syncwarp();
-    if (lane == 0) {
-        sh.rcnt[r & 1] = 0;
-        __threadfence_block();
-        sh.repoch[r & 1] = r;
-    }
-    __syncwarp();
-}
-
-// SwiGLU of one row-group -> h (fp16 hi/lo pair per value) in the fragment
-// order of the down projection's B operand: [step][v][t'][4].
-__device__ void epilogue_a(const MoeParams& p, const float* rb0, int slot, int ncols, int rg, int lane) {
+// SwiGLU of one row-group: undo the per-column x scaling, h = silu(g) * u,
+// store h as an fp16 hi/lo pair in the fragment order of the down projection's
+// B operand ([step][v][t'][4], v = 2*col + {0 hi, 1 lo}) and the row-group's
+// sum of (hi + lo) per column (half of a 32-wide down block).
+__device__ void epilogue_a(const MoeParams& p, const Shared& sh, const float* rb0, int slot, int ncols, int rg,
+                           int lane, int sstr) {
     const int g = lane >> 2, t = lane & 3;
-    uint16_t* hs = p.hbuf + (long long)slot * (2LL * p.T * p.I);
+    uint16_t* hs = p.hbuf + (long long)slot * (2LL * p.T * (p.I + sstr));
+    float* hsum = (float*)(hs + 2LL * ncols * p.I);
     float G[4] = {0.f, 0.f, 0.f, 0.f}, U[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int w = 0; w < NCW; ++w) {
@@ -292,20 +328,32 @@ __device__ void epilogue_a(const MoeParams& p, const float* rb0, int slot, int n
     }
     uint32_t bad = 0;
     const int step = rg;
+    float part[2] = {0.f, 0.f};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int col = 2 * t + (i & 1);
         const int rowhi = i >> 1;  // 0: row g, 1: row g+8
         if (col >= ncols) continue;
-        const float gv = G[i];
-        const float h = gv / (1.0f + expf(-gv)) * U[i];
+        const float sc = __int_as_float((127 - sh.xn[sh.st.cols[slot][col]]) << 23);
+        const float gv = G[i] * sc, uv = U[i] * sc;
+        const float h = gv / (1.0f + expf(-gv)) * uv;
         const __half hi = __float2half_rn(h);
         const __half lo = __float2half_rn(h - __half2float(hi));
         if (!(fabsf(h) <= 65504.0f)) bad = 1;
+        part[i & 1] += __half2float(hi) + __half2float(lo);
         const int tp = g >> 1, pos = 2 * rowhi + (g & 1);
         const long long base = ((long long)(step * 2 * ncols) * 4 + tp) * 4 + pos;
         hs[base + (long long)(2 * col) * 16] = __half_as_ushort(hi);
         hs[base + (long long)(2 * col + 1) * 16] = __half_as_ushort(lo);
+    }
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+        part[0] += __shfl_xor_sync(0xffffffffu, part[0], o);
+        part[1] += __shfl_xor_sync(0xffffffffu, part[1], o);
+    }
+    if (g == 0) {
+        if (2 * t < ncols) hsum[(2 * t) * sstr + rg] = part[0];
+        if (2 * t + 1 < ncols) hsum[(2 * t + 1) * sstr + rg] = part[1];
     }
     if (__any_sync(0xffffffffu, bad) && lane == 0) set_error(p.ctrl, MOE_ERR_RANGE);
 }
@@ -332,13 +380,13 @@ __device__ void epilogue_b(const MoeParams& p, const SlotTable& S, const float* 
             dp[(long long)col * p.H + row0 + 8] = D[4 * nb + 2] + D[4 * nb + 3];
         }
     }
-    __threadfence();
+    // warp barrier, then one release/acquire atomic for the whole warp's stores
     __syncwarp();
     uint32_t prev = 0;
     if (lane == 0) prev = atom_add_acq_rel_gpu(p.ctrl + MOE_CTRL_ROWBLK + rg, 1u);
     prev = __shfl_sync(0xffffffffu, prev, 0);
     if (prev != (uint32_t)S.nslots - 1) return;
-    __threadfence();
+    __syncwarp();   // lane 0's acquire orders the other lanes' reads of dpart below
     for (int it = lane; it < 16 * p.T; it += 32) {
         const int row = 16 * rg + (it & 15), c = it >> 4;
         float acc = 0.f;
@@ -355,29 +403,194 @@ __device__ void epilogue_b(const MoeParams& p, const SlotTable& S, const float* 
     if (lane == 0) p.ctrl[MOE_CTRL_ROWBLK + rg] = 0u;
 }
 
-__device__ void consumer(const MoeParams& p, Shared& sh, uint8_t* ring, uint8_t* xh, int hbytes_max, float* red) {
+// An epilogue warp: units r = e, e + NEPI, ... in the order the consumers
+// deposit them; the 8 warps' partials are summed in warp order.
+__device__ void epilogue_warp(const MoeParams& p, Shared& sh, float* red, int e, int sstr) {
+    const int lane = threadIdx.x & 31;
+    for (int r = e;; r += NEPI) {
+        const int b = r % p.nred;
+        const uint32_t ph = (uint32_t)(r / p.nred) & 1u;
+        if (!mbar_wait(&sh.rfull[b], ph, WAIT_LIMIT)) {
+            set_error(p.ctrl, MOE_ERR_TIMEOUT);
+            sh.abort_flag = 1;
+            break;
+        }
+        const RedInfo ri = sh.rinfo[b];
+        if (ri.kind < 0) break;
+        const float* rb0 = red + b * NCW * 32 * 8;
+        if (ri.kind == 0) {
+            epilogue_a(p, sh, rb0, ri.slot, ri.ncols, ri.rg, lane, sstr);
+            // this row-group of h is complete: publish it to the down tasks
+            // (the bulk-copy reader fences the async proxy after its acquire)
+            __syncwarp();
+            if (lane == 0) red_add_release_gpu(p.ctrl + MOE_CTRL_SLOT + ri.slot, 1u);
+        } else {
+            epilogue_b(p, sh.st, rb0, ri.slot, ri.ncols, ri.rg, lane);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.rempty[b]);
+    }
+}
+
+// ------------------------------------------------------------- consumers ---
+
+struct RedCursor {
+    int b = 0;
+    uint32_t ph = 0;   // parity of the rfull phase being filled; rempty waits for ph ^ 1
+};
+
+// Deposit this warp's partials for the next reduction unit.
+__device__ __forceinline__ bool red_deposit(const MoeParams& p, Shared& sh, float* red, RedCursor& rc, int w, int lane,
+                                            const float v[8], const RedInfo& info) {
+    if (!mbar_wait(&sh.rempty[rc.b], rc.ph ^ 1u, WAIT_LIMIT)) return false;
+    float* my = red + ((rc.b * NCW + w) * 32 + lane) * 8;
+    *reinterpret_cast<float4*>(my) = make_float4(v[0], v[1], v[2], v[3]);
+    *reinterpret_cast<float4*>(my + 4) = make_float4(v[4], v[5], v[6], v[7]);
+    if (w == 0 && lane == 0) sh.rinfo[rc.b] = info;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sh.rfull[rc.b]);
+    if (++rc.b == p.nred) { rc.b = 0; rc.ph ^= 1u; }
+    return true;
+}
+
+// Bit offset of tile (k/32) of a K-long row-group for format fmt (0 inside a
+// trailing partial chunk, which is decoded to exact levels).
+__device__ __forceinline__ int s_pos(int fmt, int k, int K) {
+    const int blk = k >> 5;
+    if ((blk >> 3) == (K >> 8) && (K & 255)) return 0;
+    const int b = blk & 7;
+    return fmt == 2 ? Plane<2>::s_of(b) : (fmt == 3 ? Plane<3>::s_of(b) : Plane<4>::s_of(b));
+}
+
+// Ring position of a consumer warp.
+struct Ring {
+    int stage = 0, cc = 0;
+    uint32_t fphase = 0;
+};
+
+// All stages of one gate/up row-group: warp w takes chunk w of every stage.
+template <int FMT, bool TWO>
+__device__ __forceinline__ bool rowgroup_a(const MoeParams& p, Shared& sh, uint8_t* ring, Ring& rg_, int nch, int w,
+                                        int lane, const BSrc& bs_in, const float* sA0, const float* sA1, float v[8]) {
+    const int g = lane >> 2;
+    const BSrc bs = bs_in;   // keep the operand source in registers
+    constexpr int FULLB = (int)(8 * 16 * (FMT * 4 + (FMT == 4 ? 1 : 2)));
+    AccA ag, au;
+    ag.zero();
+    au.zero();
+    for (int c0 = 0; c0 < nch; c0 += MOE_CHUNKS_PER_STAGE) {
+        if (!mbar_wait(&sh.full[rg_.stage], rg_.fphase, WAIT_LIMIT)) return false;
+        const int c = c0 + w;
+        if (c < nch) {
+            const uint8_t* st = ring + rg_.stage * MOE_STAGE_BYTES + w * FULLB;
+            const int nt = rfx_chunk_tiles(p.H, c);
+            if (nt == 8) {
+                float S0[8], S1[8];
+                const float4 a0 = ldsf4((const uint8_t*)(sA0 + 8 * c)), a1 = ldsf4((const uint8_t*)(sA0 + 8 * c + 4));
+                S0[0] = a0.x; S0[1] = a0.y; S0[2] = a0.z; S0[3] = a0.w;
+                S0[4] = a1.x; S0[5] = a1.y; S0[6] = a1.z; S0[7] = a1.w;
+                if (TWO) {
+                    const float4 b0 = ldsf4((const uint8_t*)(sA1 + 8 * c)), b1 = ldsf4((const uint8_t*)(sA1 + 8 * c + 4));
+                    S1[0] = b0.x; S1[1] = b0.y; S1[2] = b0.z; S1[3] = b0.w;
+                    S1[4] = b1.x; S1[5] = b1.y; S1[6] = b1.z; S1[7] = b1.w;
+                }
+                chunkA_full<FMT, TWO>(st, st + MOE_HALF_BYTES, lane, g, bs, c * 16, S0, S1, ag, au);
+            } else {
+                chunkA_partial<FMT, true>(st, st + MOE_HALF_BYTES, nt, lane, g, bs, c * 16, ag, au);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.empty[rg_.stage]);
+        ++rg_.cc;
+        if (w == 0 && lane == 0) sh.consumed = rg_.cc;
+        if (++rg_.stage == p.ns) { rg_.stage = 0; rg_.fphase ^= 1u; }
+    }
+    finishA<FMT>(ag, v);
+    finishA<FMT>(au, v + 4);
+    return true;
+}
+
+// All stages of one down row-group (usually a single stage of 8 chunks).
+template <int FMT, int NB>
+__device__ __forceinline__ bool rowgroup_b(const MoeParams& p, Shared& sh, uint8_t* ring, Ring& rg_, int nch, int w,
+                                        int lane, const BSrc* bs_in, const float* hsum, int ncols, int sstr,
+                                        float v[8]) {
+    const int g = lane >> 2, t = lane & 3;
+    BSrc bs[NB];   // keep the operand sources in registers
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) bs[nb] = bs_in[nb];
+    constexpr int FULLB = (int)(8 * 16 * (FMT * 4 + (FMT == 4 ? 1 : 2)));
+    AccB<NB> ab;
+    ab.zero();
+    for (int c0 = 0; c0 < nch; c0 += MOE_CHUNKS_PER_STAGE) {
+        if (!mbar_wait(&sh.full[rg_.stage], rg_.fphase, WAIT_LIMIT)) return false;
+        const int c = c0 + w;
+        if (c < nch) {
+            const uint8_t* st = ring + rg_.stage * MOE_STAGE_BYTES + w * FULLB;
+            const int nt = rfx_chunk_tiles(p.I, c);
+            if (nt == 8) {
+                // block sums of h for the lane's real column(s): two halves per block
+                float Sb[NB][8];
+#pragma unroll
+                for (int nb = 0; nb < NB; ++nb) {
+                    const int colr = 4 * nb + t;
+                    const float* hp = hsum + (colr < ncols ? colr : 0) * sstr + 16 * c;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float4 x4 = ldsf4((const uint8_t*)(hp + 4 * q));
+                        Sb[nb][2 * q] = x4.x + x4.y;
+                        Sb[nb][2 * q + 1] = x4.z + x4.w;
+                    }
+                }
+                chunkB_full<FMT, NB>(st, lane, g, bs, c * 16, Sb, ab);
+            } else {
+                chunkB_partial<FMT, NB>(st, nt, lane, g, bs, c * 16, ab);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.empty[rg_.stage]);
+        ++rg_.cc;
+        if (w == 0 && lane == 0) sh.consumed = rg_.cc;
+        if (++rg_.stage == p.ns) { rg_.stage = 0; rg_.fphase ^= 1u; }
+    }
+    float vb[NB][4];
+    finishB<FMT, NB>(ab, vb);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[i] = vb[0][i];
+        v[4 + i] = NB > 1 ? vb[NB - 1][i] : 0.f;
+    }
+    return true;
+}
+
+__device__ void consumer(const MoeParams& p, Shared& sh, uint8_t* ring, uint8_t* xh, int hbytes_max, float* red,
+                         int sstr) {
     const SlotTable& S = sh.st;
     const int w = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
     const int nrbA = p.I / 32, nrbB = p.H / 32;
-    int cc = 0, bseq = 0, r = 0;
+    const int nxc = (p.has_shared && p.fsA != p.fA) ? 2 : 1;
+    const float* sx = (const float*)(xh + nxc * p.T * p.x_stride);   // [copy][col][sxs]
+    const int sxs = moe_sxs(p.H);
+    Ring ring_pos;
+    int bseq = 0;
+    int qi = 0;
+    uint32_t qphase = 0;
+    RedCursor rc;
     bool first_b = true, ok = true;
-    for (int n = 0; ok; ++n) {
-        const int qi = n % QN;
-        if (!mbar_wait(&sh.tqf[qi], (n / QN) & 1, WAIT_LIMIT)) { ok = false; break; }
+    while (ok) {
+        if (!mbar_wait(&sh.tqf[qi], qphase, WAIT_LIMIT)) { ok = false; break; }
         const int task = sh.tq[qi];
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh.tqe[qi]);
+        if (++qi == QN) { qi = 0; qphase ^= 1u; }
         if (task < 0 || sh.abort_flag) break;
         const Task tk = decode_task(task, S.nslots, nrbA, nrbB);
         const int slot = tk.slot;
         const int e = S.expert[slot];
         const int ncols = S.ncols[slot];
-        const int K = tk.kind == 0 ? p.H : p.I;
         const int fmt = tk.kind == 0 ? (e < 0 ? p.fsA : p.fA) : (e < 0 ? p.fsB : p.fB);
-        const int fullb = (int)rfx_chunk_bytes(fmt, 8);
-        const int nch = rfx_num_chunks(K);
         const int buf_h = bseq & 1;
         if (tk.kind == 1) {
             if (first_b) {
@@ -388,90 +601,50 @@ __device__ void consumer(const MoeParams& p, Shared& sh, uint8_t* ring, uint8_t*
             }
             if (!mbar_wait(&sh.hfull[buf_h], (bseq >> 1) & 1, WAIT_LIMIT)) { ok = false; break; }
         }
-        BSrc bs[2];
-        if (tk.kind == 0) {
-            const int col = g < ncols ? S.cols[slot][g] : 0;
-            bs[0] = {xh + col * p.x_stride + t * 8, 32, g < ncols};
-            bs[1] = bs[0];
-        } else {
-            const uint8_t* hs = xh + buf_h * hbytes_max;
-            const int vst = 64 * ncols;  // bytes per k16 step
-#pragma unroll
-            for (int nb = 0; nb < 2; ++nb) {
-                const int v = 8 * nb + g;
-                bs[nb] = {hs + (v * 4 + t) * 8, vst, v < 2 * ncols};
-            }
-        }
-        const bool two_nb = tk.kind == 1 && ncols > 4;
         for (int rgl = 0; rgl < 2 && ok; ++rgl) {
-            Acc<1> a0, a1;
-            Acc<2> d2;
-            a0.zero(); a1.zero(); d2.zero();
-            for (int c0 = 0; c0 < nch; c0 += MOE_CHUNKS_PER_STAGE) {
-                const int s = cc % p.ns;
-                if (!mbar_wait(&sh.full[s], (cc / p.ns) & 1, WAIT_LIMIT)) { ok = false; break; }
-                const int c = c0 + w;
-                if (c < nch) {
-                    const uint8_t* st = ring + s * MOE_STAGE_BYTES + w * fullb;
-                    const int nt = rfx_chunk_tiles(K, c);
-                    const int step0 = c * 16;
-                    if (tk.kind == 0) {
-                        switch (fmt) {
-                            case 2: chunk_any2<2, false, 1>(st, st + MOE_HALF_BYTES, nt, lane, g, bs, step0, a0, a1); break;
-                            case 3: chunk_any2<3, false, 1>(st, st + MOE_HALF_BYTES, nt, lane, g, bs, step0, a0, a1); break;
-                            default: chunk_any2<4, false, 1>(st, st + MOE_HALF_BYTES, nt, lane, g, bs, step0, a0, a1); break;
-                        }
-                    } else if (!two_nb) {
-                        switch (fmt) {
-                            case 2: chunk_any<2, true, 1>(st, nt, lane, g, bs, step0, a0); break;
-                            case 3: chunk_any<3, true, 1>(st, nt, lane, g, bs, step0, a0); break;
-                            default: chunk_any<4, true, 1>(st, nt, lane, g, bs, step0, a0); break;
-                        }
-                    } else {
-                        switch (fmt) {
-                            case 2: chunk_any<2, true, 2>(st, nt, lane, g, bs, step0, d2); break;
-                            case 3: chunk_any<3, true, 2>(st, nt, lane, g, bs, step0, d2); break;
-                            default: chunk_any<4, true, 2>(st, nt, lane, g, bs, step0, d2); break;
-                        }
-                    }
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sh.empty[s]);
-                ++cc;
-                if (w == 0 && lane == 0) sh.consumed = cc;
-            }
-            if (!ok) break;
             float v[8];
             if (tk.kind == 0) {
-#pragma unroll
-                for (int i = 0; i < 4; ++i) { v[i] = a0.v[0][i]; v[4 + i] = a1.v[0][i]; }
-            } else if (!two_nb) {
-#pragma unroll
-                for (int i = 0; i < 4; ++i) { v[i] = a0.v[0][i]; v[4 + i] = 0.f; }
-            } else {
-#pragma unroll
-                for (int i = 0; i < 4; ++i) { v[i] = d2.v[0][i]; v[4 + i] = d2.v[1][i]; }
-            }
-            const bool last = red_deposit(sh, red, r, w, lane, v, ok);
-            if (!ok) break;
-            if (last) {
-                const float* rb0 = red + (r & 1) * NCW * 32 * 8;
-                const int rg = 2 * tk.rb + rgl;
-                if (tk.kind == 0) {
-                    epilogue_a(p, rb0, slot, ncols, rg, lane);
-                    if (rgl == 1) {
-                        // both row-groups of the task are in h: publish
-                        fence_proxy_async_global();
-                        __threadfence();
-                        __syncwarp();
-                        if (lane == 0) atom_add_release_gpu(p.ctrl + MOE_CTRL_SLOT + slot, 1u);
-                    }
-                } else {
-                    epilogue_b(p, S, rb0, slot, ncols, rg, lane);
+                const int ci = (e < 0 && nxc == 2) ? 1 : 0;
+                const int col0 = g < ncols ? S.cols[slot][g] : 0;
+                const BSrc bs{xh + (ci * p.T + col0) * p.x_stride + t * 8, 32, g < ncols};
+                const int c0 = 2 * t < ncols ? S.cols[slot][2 * t] : 0;
+                const int c1 = 2 * t + 1 < ncols ? S.cols[slot][2 * t + 1] : 0;
+                const float* sA0 = sx + (ci * p.T + c0) * sxs;
+                const float* sA1 = sx + (ci * p.T + c1) * sxs;
+                const int nch = rfx_num_chunks(p.H);
+                const bool two = ncols > 1;
+                switch (fmt * 2 + (two ? 1 : 0)) {
+                    case 4: ok = rowgroup_a<2, false>(p, sh, ring, ring_pos, nch, w, lane, bs, sA0, sA1, v); break;
+                    case 5: ok = rowgroup_a<2, true>(p, sh, ring, ring_pos, nch, w, lane, bs, sA0, sA1, v); break;
+                    case 6: ok = rowgroup_a<3, false>(p, sh, ring, ring_pos, nch, w, lane, bs, sA0, sA1, v); break;
+                    case 7: ok = rowgroup_a<3, true>(p, sh, ring, ring_pos, nch, w, lane, bs, sA0, sA1, v); break;
+                    case 8: ok = rowgroup_a<4, false>(p, sh, ring, ring_pos, nch, w, lane, bs, sA0, sA1, v); break;
+                    default: ok = rowgroup_a<4, true>(p, sh, ring, ring_pos, nch, w, lane, bs, sA0, sA1, v); break;
                 }
-                red_release(sh, r, lane);
+            } else {
+                const uint8_t* hs = xh + buf_h * hbytes_max;
+                const int vst = 64 * ncols;  // bytes per k16 step
+                BSrc bs[2];
+#pragma unroll
+                for (int nb = 0; nb < 2; ++nb) {
+                    const int vv = 8 * nb + g;
+                    bs[nb] = {hs + (vv * 4 + t) * 8, vst, vv < 2 * ncols};
+                }
+                const float* hsum = (const float*)(hs + 4 * ncols * p.I);
+                const int nch = rfx_num_chunks(p.I);
+                const bool two_nb = ncols > 4;
+                switch (fmt * 2 + (two_nb ? 1 : 0)) {
+                    case 4: ok = rowgroup_b<2, 1>(p, sh, ring, ring_pos, nch, w, lane, bs, hsum, ncols, sstr, v); break;
+                    case 5: ok = rowgroup_b<2, 2>(p, sh, ring, ring_pos, nch, w, lane, bs, hsum, ncols, sstr, v); break;
+                    case 6: ok = rowgroup_b<3, 1>(p, sh, ring, ring_pos, nch, w, lane, bs, hsum, ncols, sstr, v); break;
+                    case 7: ok = rowgroup_b<3, 2>(p, sh, ring, ring_pos, nch, w, lane, bs, hsum, ncols, sstr, v); break;
+                    case 8: ok = rowgroup_b<4, 1>(p, sh, ring, ring_pos, nch, w, lane, bs, hsum, ncols, sstr, v); break;
+                    default: ok = rowgroup_b<4, 2>(p, sh, ring, ring_pos, nch, w, lane, bs, hsum, ncols, sstr, v); break;
+                }
             }
-            ++r;
+            if (!ok) break;
+            const RedInfo info{tk.kind, slot, ncols, 2 * tk.rb + rgl, rgl == 1};
+            if (!red_deposit(p, sh, red, rc, w, lane, v, info)) { ok = false; break; }
         }
         if (!ok) break;
         if (tk.kind == 1) {
@@ -484,6 +657,55 @@ __device__ void consumer(const MoeParams& p, Shared& sh, uint8_t* ring, uint8_t*
         set_error(p.ctrl, MOE_ERR_TIMEOUT);
         sh.abort_flag = 1;
     }
+    // one end-of-work unit for each epilogue warp
+    const RedInfo fin{-1, 0, 0, 0, 0};
+    const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int i = 0; i < NEPI; ++i) (void)red_deposit(p, sh, red, rc, w, lane, z, fin);
+}
+
+// x (bf16 [T][H]) -> shared memory for the gate/up B operand: per column
+// c, x * 2^xn[c] with xn[c] putting max|x| in [2^13, 2^14), times 2^-s_b for
+// the tile's bit offset in the gate/up format (one copy per format in use),
+// rounded to fp16 in fragment order [c][step][t][k 2t,2t+1,2t+8,2t+9]; plus
+// the block sums of the staged values (times 2^s_b) for the offset correction.
+__device__ void stage_x(const MoeParams& p, Shared& sh, uint8_t* xh, const uint32_t* x32) {
+    const int tid = threadIdx.x;   // 0 .. NCW*32-1
+    const int npairs = p.T * p.H / 2;
+    for (int i = tid; i < npairs; i += NCW * 32) {
+        const uint32_t v = x32[i];
+        const uint32_t m = max((v << 16) & 0x7fffffffu, v & 0x7fff0000u);
+        atomicMax(&sh.xmax[(2 * i) / p.H], m);
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
+    if (tid < p.T) {
+        const uint32_t m = sh.xmax[tid];
+        int n = m ? 13 - ((int)((m >> 23) & 255u) - 127) : 0;
+        sh.xn[tid] = max(-100, min(100, n));
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
+    const int nxc = (p.has_shared && p.fsA != p.fA) ? 2 : 1;
+    float* sx = (float*)(xh + nxc * p.T * p.x_stride);
+    const int hw = tid >> 4, l16 = tid & 15;
+    const unsigned hmask = 0xffffu << (tid & 16);
+    const int nblk = p.T * p.H / 32;
+    for (int ci = 0; ci < nxc; ++ci) {
+        const int fmt = ci == 0 ? p.fA : p.fsA;
+        for (int blk = hw; blk < nblk; blk += NCW * 2) {
+            const int i = blk * 16 + l16;
+            const int c = (2 * i) / p.H, k = (2 * i) % p.H;
+            const int s = s_pos(fmt, k, p.H);
+            const uint32_t v = x32[i];
+            const float sc = __int_as_float((127 + sh.xn[c] - s) << 23);
+            const float f0 = __uint_as_float(v << 16) * sc, f1 = __uint_as_float(v & 0xffff0000u) * sc;
+            const __half2 h2 = __floats2half2_rn(f0, f1);
+            const int step = k >> 4, rr = k & 15;
+            *(__half2*)(xh + (ci * p.T + c) * p.x_stride + (step * 4 + ((rr & 7) >> 1)) * 8 + (rr >> 3) * 4) = h2;
+            float sum = (__low2float(h2) + __high2float(h2)) * __int_as_float((127 + s) << 23);
+#pragma unroll
+            for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(hmask, sum, o);
+            if (l16 == 0) sx[(ci * p.T + c) * moe_sxs(p.H) + (k >> 5)] = sum;
+        }
+    }
 }
 
 __global__ void __launch_bounds__(NTHREADS, 1) moe_decode_kernel(MoeParams p) {
@@ -492,8 +714,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_decode_kernel(MoeParams p) {
     uint8_t* ring = base;
     uint8_t* xh = ring + p.ns * MOE_STAGE_BYTES;
     float* red = (float*)(xh + p.xh_bytes);
-    Shared& sh = *(Shared*)((uint8_t*)red + 2 * NCW * 32 * 8 * sizeof(float));
-    const int hbytes_max = 4 * p.T * p.I;
+    Shared& sh = *(Shared*)((uint8_t*)red + p.nred * NCW * 32 * 8 * sizeof(float));
+    const int sstr = moe_sstr(p.I);
+    const int hbytes_max = 4 * p.T * (p.I + sstr);
     const int w = threadIdx.x >> 5;
 
     if (threadIdx.x == 0) {
@@ -508,32 +731,47 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_decode_kernel(MoeParams p) {
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sh.hfull[i], 1);
             mbar_init(&sh.hfree[i], NCW);
-            sh.rcnt[i] = 0;
-            sh.repoch[i] = i - 2;
+        }
+        for (int i = 0; i < p.nred; ++i) {
+            mbar_init(&sh.rfull[i], NCW);
+            mbar_init(&sh.rempty[i], 1);
         }
         mbar_init(&sh.xfree, NCW);
+        for (int i = 0; i < QN; ++i) {
+            mbar_init(&sh.hqf[i], 1);
+            mbar_init(&sh.hqe[i], 1);
+        }
         sh.abort_flag = 0;
         sh.consumed = 0;
+        for (int c = 0; c < MOE_MAXT; ++c) sh.xmax[c] = 0u;
+        mbar_init(&sh.xload, 1);
         fence_barrier_init();
     }
-    if (w == NCW) {
-        build_slots(p, sh.st);
-    } else {
-        // x (bf16 [T][H]) -> shared, fragment order [c][step][t][k 2t,2t+1,2t+8,2t+9]
-        const int npairs = p.T * p.H / 2;
-        const uint32_t* x32 = (const uint32_t*)p.x;
-        for (int i = threadIdx.x; i < npairs; i += NCW * 32) {
-            const int c = (2 * i) / p.H, k = (2 * i) % p.H;
-            const int step = k >> 4, rr = k & 15;
-            const int tt = (rr & 7) >> 1, half = rr >> 3;
-            *(uint32_t*)(xh + c * p.x_stride + (step * 4 + tt) * 8 + half * 4) = x32[i];
-        }
-    }
     __syncthreads();
-    if (w == NCW) {
-        if ((threadIdx.x & 31) == 0) producer(p, sh, ring, xh, hbytes_max);
+    // x: one bulk copy into the stage ring (free until the main loop) when it
+    // fits and is 16-byte aligned, else read straight from global memory
+    const uint32_t xbytes = (uint32_t)(p.T * p.H * 2);
+    const bool xbulk = xbytes <= (uint32_t)(p.ns * MOE_STAGE_BYTES) && (((uintptr_t)p.x & 15u) == 0);
+    if (xbulk && threadIdx.x == 0) {
+        mbar_arrive_expect_tx(&sh.xload, xbytes);
+        bulk_g2s(ring, p.x, xbytes, &sh.xload, policy_evict_last());
+    }
+    if (w == WARP_PRODUCER) {
+        build_slots(p, sh.st);
+    } else if (w < NCW) {
+        if (xbulk && !mbar_wait(&sh.xload, 0, WAIT_LIMIT)) set_error(p.ctrl, MOE_ERR_TIMEOUT);
+        stage_x(p, sh, xh, xbulk ? (const uint32_t*)ring : (const uint32_t*)p.x);
+    }
+    if (w == WARP_PRODUCER + 1 && xbulk) (void)mbar_wait(&sh.xload, 0, WAIT_LIMIT);   // copy landed before reuse
+    __syncthreads();
+    if (w == WARP_PRODUCER) {
+        const int lane = threadIdx.x & 31;
+        if (lane == 0) producer(p, sh, ring);
+        else if (lane == 1) h_loader(p, sh, xh, hbytes_max, sstr);
+    } else if (w >= WARP_EPILOGUE0) {
+        epilogue_warp(p, sh, red, w - WARP_EPILOGUE0, sstr);
     } else {
-        consumer(p, sh, ring, xh, hbytes_max, red);
+        consumer(p, sh, ring, xh, hbytes_max, red, sstr);
     }
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -550,12 +788,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_decode_kernel(MoeParams p) {
 }
 
 // Shared-memory bytes of a launch (plus 1 KB alignment slack).
-size_t moe_decode_smem_bytes(int ns, int xh_bytes) {
-    return 1024 + (size_t)ns * MOE_STAGE_BYTES + xh_bytes + 2 * NCW * 32 * 8 * sizeof(float) + sizeof(Shared);
+size_t moe_decode_smem_bytes(int ns, int nred, int xh_bytes) {
+    return 1024 + (size_t)ns * MOE_STAGE_BYTES + xh_bytes + (size_t)nred * NCW * 32 * 8 * sizeof(float) + sizeof(Shared);
 }
 
 cudaError_t moe_decode_launch(const MoeParams& p, int grid, cudaStream_t stream) {
-    const size_t smem = moe_decode_smem_bytes(p.ns, p.xh_bytes);
+    const size_t smem = moe_decode_smem_bytes(p.ns, p.nred, p.xh_bytes);
     auto kern = moe_decode_kernel;
     // raise the dynamic shared-memory limit once (not a stream operation, so
     // it stays out of any graph capture after the first call)

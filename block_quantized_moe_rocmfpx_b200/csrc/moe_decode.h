@@ -9,6 +9,7 @@
 #define MOE_MAXK 8            // routed experts per token
 #define MOE_MAXS (MOE_MAXT * MOE_MAXK + 1)
 #define MOE_MAX_STAGES 6
+#define MOE_MAX_RED 8          // reduction buffers
 #define MOE_CHUNKS_PER_STAGE 8
 #define MOE_HALF_BYTES 17408   // 8 full FP4 chunks of one matrix
 #define MOE_STAGE_BYTES 34816  // gate + up halves
@@ -44,12 +45,20 @@ struct MoeParams {
     const float* wts;      // [T][k]
     float* y;              // [T][H]
     uint32_t* ctrl;
-    uint16_t* hbuf;        // fp16 [MAXS_T][2*T*I]
+    uint16_t* hbuf;        // per slot: fp16 h fragments [2*T*I] then fp32 block sums [T][sstr]
     float* dpart;          // fp32 [MAXS_T][T][H]
-    int ns;                // stages per consumer warp
+    int ns;                // stages in the ring
+    int nred;              // reduction buffers
     int x_stride;          // bytes per x column in shared memory
     int xh_bytes;          // bytes of the x / h region
 };
+
+// Floats per column of the h block-sum table: one per 16-row group of I,
+// padded to a multiple of 4 (16 bytes).
+inline __host__ __device__ int moe_sstr(int I) { return ((I / 16) + 3) & ~3; }
+
+// Floats per column of the x block-sum table (H/32 padded to 16-byte rows).
+inline __host__ __device__ int moe_sxs(int H) { return ((H / 32) + 3) & ~3; }
 
 // Workspace layout for (T, k, H, I).
 struct MoeWs {
@@ -62,12 +71,12 @@ inline MoeWs moe_ws_layout(int T, int k, int H, int I) {
     const size_t ctrl_words = MOE_CTRL_ROWBLK + (size_t)H / 16;
     L.ctrl_off = 0;
     L.h_off = (ctrl_words * 4 + 255) / 256 * 256;
-    L.d_off = L.h_off + (ns * 4 * T * I + 255) / 256 * 256;
+    L.d_off = L.h_off + (ns * 4 * T * (size_t)(I + moe_sstr(I)) + 255) / 256 * 256;
     L.total = L.d_off + (ns * T * H * 4 + 255) / 256 * 256;
     return L;
 }
 
-size_t moe_decode_smem_bytes(int ns, int xh_bytes);
+size_t moe_decode_smem_bytes(int ns, int nred, int xh_bytes);
 cudaError_t moe_decode_launch(const MoeParams& p, int grid, cudaStream_t stream);
 
 }  // namespace rfx

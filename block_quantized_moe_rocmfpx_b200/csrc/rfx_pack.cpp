@@ -50,6 +50,50 @@ inline void reg_coords(int g, int t, int r, int& row, int& k) {
     k = 16 * m + 2 * t + 8 * (j >> 1);
 }
 
+// ---- full chunks (8 tiles): "plane" layout ----
+// Register r of tile b sits at the same bit offset for every r, in a
+// different word per r, so one AND yields an fp16 subnormal code * 2^(s-24).
+//   FP2: word r, field b (bits 2b | 16+2b).                         8 words
+//   FP4: word r (tiles 0..3) or 8+r (tiles 4..7), field b&3 (4f | 16+4f).  16 words
+//   FP3: tiles 0..4: word r, field b (bits 3b | 16+3b).
+//        tiles 5, 6: r<4 -> word 8+r, field b-5; r>=4 -> word 8+r-4, field b-2.
+//        tile 7:     r<4 -> word 8+r, field 2;   r>=4 -> bit i of the low code at
+//        bit 15, of the high code at bit 31, of word 3(r-4)+i.          12 words
+struct FieldRef { int word, shift, spare; };
+static FieldRef full_field(int fmt, int b, int r) {
+    if (fmt == 2) return {r, 2 * b, 0};
+    if (fmt == 4) return {(b < 4 ? r : 8 + r), 4 * (b & 3), 0};
+    if (b < 5) return {r, 3 * b, 0};
+    if (b < 7) return r < 4 ? FieldRef{8 + r, 3 * (b - 5), 0} : FieldRef{8 + r - 4, 3 * (b - 2), 0};
+    if (r < 4) return {8 + r, 6, 0};
+    return {3 * (r - 4), 0, 1};
+}
+
+void pack_lane_full(int fmt, const TileView* tv, int g, int t, uint8_t* out) {
+    uint32_t w[16] = {0};
+    const uint32_t m = (1u << fmt) - 1u;
+    for (int b = 0; b < 8; ++b)
+        for (int r = 0; r < 8; ++r) {
+            int row, k;
+            reg_coords(g, t, r, row, k);
+            const uint32_t lo = (uint32_t)tv[b].code(row, k) & m, hi = (uint32_t)tv[b].code(row, k + 1) & m;
+            const FieldRef f = full_field(fmt, b, r);
+            if (!f.spare) {
+                w[f.word] |= lo << f.shift;
+                w[f.word] |= hi << (16 + f.shift);
+            } else {
+                for (int i = 0; i < 3; ++i) {
+                    w[f.word + i] |= ((lo >> i) & 1u) << 15;
+                    w[f.word + i] |= ((hi >> i) & 1u) << 31;
+                }
+            }
+        }
+    std::memcpy(out, w, 4 * 4 * fmt);
+}
+
+void unpack_lane_full(int fmt, const struct TileOut* to, int g, int t, const uint8_t* in);
+
+// ---- partial chunks (< 8 tiles): per-tile layout ----
 // Write the lane's codes of one tile (FP2 / FP4) or tile pair / lone tile (FP3).
 void pack_lane_fp2(const TileView& tv, int g, int t, uint8_t* out) {
     uint32_t w = 0;
@@ -162,6 +206,30 @@ void unpack_lane_fp3_pair(const TileOut& a, const TileOut& b, int g, int t, cons
     }
 }
 
+void unpack_lane_full(int fmt, const TileOut* to, int g, int t, const uint8_t* in) {
+    uint32_t w[16];
+    std::memcpy(w, in, 4 * 4 * fmt);
+    const uint32_t m = (1u << fmt) - 1u;
+    for (int b = 0; b < 8; ++b)
+        for (int r = 0; r < 8; ++r) {
+            int row, k;
+            reg_coords(g, t, r, row, k);
+            const FieldRef f = full_field(fmt, b, r);
+            uint32_t lo = 0, hi = 0;
+            if (!f.spare) {
+                lo = (w[f.word] >> f.shift) & m;
+                hi = (w[f.word] >> (16 + f.shift)) & m;
+            } else {
+                for (int i = 0; i < 3; ++i) {
+                    lo |= ((w[f.word + i] >> 15) & 1u) << i;
+                    hi |= ((w[f.word + i] >> 31) & 1u) << i;
+                }
+            }
+            to[b].set(row, k, (int)lo);
+            to[b].set(row, k + 1, (int)hi);
+        }
+}
+
 void unpack_lane_fp3_lone(const TileOut& to, int g, int t, const uint8_t* in) {
     uint64_t s = 0;
     for (int i = 0; i < 6; ++i) s |= (uint64_t)in[i] << (8 * i);
@@ -211,7 +279,11 @@ extern "C" int rfx_pack(rfx_format f, const uint8_t* codes, const void* scales, 
             for (int L = 0; L < 32; ++L) {
                 const int g = L >> 2, t = L & 3;
                 uint8_t* lane = chunk + (int64_t)L * nt * ltb;
-                if (f == RFX_FP3) {
+                if (nt == 8) {
+                    TileView tv[8];
+                    for (int b = 0; b < 8; ++b) tv[b] = TileView{codes, rows, cols, rg * 16, (int64_t)(8 * j + b) * 32};
+                    pack_lane_full(f, tv, g, t, lane);
+                } else if (f == RFX_FP3) {
                     int b = 0;
                     for (; b + 1 < nt; b += 2) {
                         TileView A{codes, rows, cols, rg * 16, (int64_t)(8 * j + b) * 32};
@@ -265,7 +337,11 @@ extern "C" int rfx_unpack(rfx_format f, const void* src, int64_t rows, int64_t c
             for (int L = 0; L < 32; ++L) {
                 const int g = L >> 2, t = L & 3;
                 const uint8_t* lane = chunk + (int64_t)L * nt * ltb;
-                if (f == RFX_FP3) {
+                if (nt == 8) {
+                    TileOut to[8];
+                    for (int b = 0; b < 8; ++b) to[b] = TileOut{codes, rows, cols, rg * 16, (int64_t)(8 * j + b) * 32};
+                    unpack_lane_full(f, to, g, t, lane);
+                } else if (f == RFX_FP3) {
                     int b = 0;
                     for (; b + 1 < nt; b += 2) {
                         TileOut A{codes, rows, cols, rg * 16, (int64_t)(8 * j + b) * 32};

@@ -1,13 +1,21 @@
 // rfx_tile.cuh -- per-chunk tensor-core work on packed ROCmFPX-style codes.
 //
-// A "chunk" is up to 8 tiles (16 rows x 32-weight block each) of one
-// row-group, laid out as in include/rfx.h.  Every packed block is decoded once
-// in registers and multiplied against the B fragments of all the token columns
-// at once (decode once, apply to every verify column: ainomam.com,
-// "APU 实现 token 自由…", section "Lucebox 的优化三板斧").  Per tile:
-//   C = A_lo(16x16) B(step 2b) + A_hi(16x16) B(step 2b+1)      (mma.sync, fp32)
-//   acc[row][col] += scale[row] * C[row][col]                   (fp32 FFMA)
-// so each block is accumulated exactly and scaled once, in fp32.
+// A "chunk" is up to 8 tiles (16 rows x one 32-weight block each) of one
+// row-group (layout in include/rfx.h).  Every packed block is decoded once in
+// registers and multiplied against the B fragments of all the token columns at
+// once (decode once, apply to every verify column: ainomam.com, "APU 实现 token
+// 自由…", section "Lucebox 的优化三板斧").
+//
+// Full chunks (8 tiles) use the plane layout: the 8 A-registers of tile b sit
+// at one bit offset s_b in 8 different words, so a single AND turns each into
+// two fp16 subnormals of value code * 2^(s_b - 24).  The tensor core computes
+// sum_k code_k * B_k exactly; with level = code - off, the block dot product is
+//     sum_k level_k B_k = sum_k code_k B_k - off * sum_k B_k,
+// so each lane also accumulates scale * (block sum of B) and subtracts off times
+// it at the end.  The 2^(s_b - 24) factor is removed either by pre-scaling the
+// B operand by 2^-s_b (gate/up: x is staged that way) or by keeping one
+// accumulator per distinct s_b (down: h is used as it is).  Partial chunks use
+// the per-tile layout and an exact magic-exponent decode of the levels.
 #pragma once
 #include "rfx_device.cuh"
 #include "rfx_layout.h"
@@ -18,8 +26,9 @@ __device__ __forceinline__ uint2 lds64(const uint8_t* p) { return *reinterpret_c
 __device__ __forceinline__ uint4 lds128(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
 __device__ __forceinline__ uint32_t lds32(const uint8_t* p) { return *reinterpret_cast<const uint32_t*>(p); }
 __device__ __forceinline__ uint32_t lds16(const uint8_t* p) { return *reinterpret_cast<const uint16_t*>(p); }
+__device__ __forceinline__ float4 ldsf4(const uint8_t* p) { return *reinterpret_cast<const float4*>(p); }
 
-// B-operand source: 4 16-bit values (k = 2t, 2t+1, 2t+8, 2t+9 of a k16 step)
+// B-operand source: 4 fp16 values (k = 2t, 2t+1, 2t+8, 2t+9 of a k16 step)
 // per lane at base + step * stride; lanes whose column is empty read zero.
 struct BSrc {
     const uint8_t* base;
@@ -32,53 +41,94 @@ struct BSrc {
     }
 };
 
-template <int NB>
-struct Acc {
-    float v[NB][4];
-    __device__ __forceinline__ void zero() {
-#pragma unroll
-        for (int n = 0; n < NB; ++n)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) v[n][i] = 0.f;
+// --------------------------------------------------------- plane layout ---
+
+// Shift exponent s_b of tile b of a full chunk (bit offset of its fields after
+// the optional pre-shift), and the number of distinct values.
+template <int FMT> struct Plane {
+    static constexpr int NW = 4 * FMT;           // code words per lane
+    static constexpr int NSW = FMT == 4 ? 4 : 8;  // scale words per g
+    static constexpr int CODE_BYTES = 8 * 16 * FMT * 4;
+    static constexpr float OFF = ((1 << FMT) - 1) * 0.5f;
+    static constexpr int NCLS = FMT == 2 ? 5 : (FMT == 3 ? 3 : 2);
+    __host__ __device__ static constexpr int s_of(int b) {
+        return FMT == 2 ? (b < 5 ? 2 * b : 2 * b - 10)
+                        : (FMT == 3 ? (b == 0 || b == 3 || b == 5 ? 0 : (b == 2 || b == 7 ? 6 : 3)) : 4 * (b & 1));
     }
+    __host__ __device__ static constexpr int cls_of(int b) { return s_of(b) / (FMT == 2 ? 2 : (FMT == 3 ? 3 : 4)); }
+    __host__ __device__ static constexpr int s_of_cls(int c) { return c * (FMT == 2 ? 2 : (FMT == 3 ? 3 : 4)); }
 };
 
-// One tile: a[0..3] = k 0..15, a[4..7] = k 16..31; s0/s1 scales of rows g/g+8.
-template <bool F16, int NB>
-__device__ __forceinline__ void tile_mma(const uint32_t a[8], const uint2 blo[NB], const uint2 bhi[NB], float s0,
-                                         float s1, Acc<NB>& acc) {
-    const float z[4] = {0.f, 0.f, 0.f, 0.f};
+template <int BITS, int S>
+__device__ __forceinline__ uint32_t fld(uint32_t w) {
+    constexpr uint32_t m = ((1u << BITS) - 1u) << S;
+    return w & (m | (m << 16));
+}
+
+// The 8 A registers of tile B of a full chunk; W = lane words, Wsh = W >> (10,
+// 9, 8 for FP2, FP3, FP4).
+template <int FMT, int B>
+__device__ __forceinline__ void plane_regs(const uint32_t* W, const uint32_t* Wsh, uint32_t a[8]) {
+    constexpr int S = Plane<FMT>::s_of(B);
+    if constexpr (FMT == 2) {
 #pragma unroll
-    for (int n = 0; n < NB; ++n) {
-        float c[4];
-        mma16816<F16>(c, a, blo[n].x, blo[n].y, z);
-        mma16816<F16>(c, a + 4, bhi[n].x, bhi[n].y, c);
-        acc.v[n][0] = fmaf(s0, c[0], acc.v[n][0]);
-        acc.v[n][1] = fmaf(s0, c[1], acc.v[n][1]);
-        acc.v[n][2] = fmaf(s1, c[2], acc.v[n][2]);
-        acc.v[n][3] = fmaf(s1, c[3], acc.v[n][3]);
+        for (int r = 0; r < 8; ++r) a[r] = fld<2, S>(B < 5 ? W[r] : Wsh[r]);
+    } else if constexpr (FMT == 4) {
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const int wi = (B < 4 ? 0 : 8) + r;
+            a[r] = fld<4, S>((B & 2) ? Wsh[wi] : W[wi]);
+        }
+    } else {
+        if constexpr (B < 3) {
+#pragma unroll
+            for (int r = 0; r < 8; ++r) a[r] = fld<3, S>(W[r]);
+        } else if constexpr (B < 5) {
+#pragma unroll
+            for (int r = 0; r < 8; ++r) a[r] = fld<3, S>(Wsh[r]);
+        } else if constexpr (B < 7) {
+#pragma unroll
+            for (int r = 0; r < 4; ++r) a[r] = fld<3, S>(W[8 + r]);
+#pragma unroll
+            for (int r = 0; r < 4; ++r) a[4 + r] = fld<3, S>(Wsh[8 + r]);
+        } else {
+#pragma unroll
+            for (int r = 0; r < 4; ++r) a[r] = fld<3, 6>(W[8 + r]);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t w0 = W[3 * j], w1 = W[3 * j + 1], w2 = W[3 * j + 2];
+                a[4 + j] = ((w0 >> 9) & 0x00400040u) | ((w1 >> 8) & 0x00800080u) | ((w2 >> 7) & 0x01000100u);
+            }
+        }
     }
 }
 
-// Lane words of a full chunk (8 tiles) and its scale words.
+template <int FMT>
+__device__ __forceinline__ void plane_shift(const uint32_t* W, uint32_t* Wsh) {
+    constexpr int SH = FMT == 2 ? 10 : (FMT == 3 ? 9 : 8);
+#pragma unroll
+    for (int i = 0; i < Plane<FMT>::NW; ++i) Wsh[i] = W[i] >> SH;
+}
+
+// Lane words and scale words of a full chunk.
 template <int FMT>
 struct FullChunk {
-    static constexpr int NW = FMT * 4;           // 8, 12, 16 words of codes per lane
-    static constexpr int NS = FMT == 4 ? 4 : 8;  // scale words per g
-    static constexpr int CODE_BYTES = 8 * 16 * FMT * 4;
-    uint32_t wd[NW];
-    uint32_t sc[NS];
+    uint32_t wd[Plane<FMT>::NW];
+    uint32_t sh[Plane<FMT>::NW];
+    uint32_t sc[Plane<FMT>::NSW];
     __device__ __forceinline__ void load(const uint8_t* st, int lane, int g) {
+        constexpr int NW = Plane<FMT>::NW, NSW = Plane<FMT>::NSW;
 #pragma unroll
         for (int i = 0; i < NW / 4; ++i) {
             uint4 v = lds128(st + lane * (NW * 4) + 16 * i);
             wd[4 * i] = v.x; wd[4 * i + 1] = v.y; wd[4 * i + 2] = v.z; wd[4 * i + 3] = v.w;
         }
 #pragma unroll
-        for (int i = 0; i < NS / 4; ++i) {
-            uint4 v = lds128(st + CODE_BYTES + g * (NS * 4) + 16 * i);
+        for (int i = 0; i < NSW / 4; ++i) {
+            uint4 v = lds128(st + Plane<FMT>::CODE_BYTES + g * (NSW * 4) + 16 * i);
             sc[4 * i] = v.x; sc[4 * i + 1] = v.y; sc[4 * i + 2] = v.z; sc[4 * i + 3] = v.w;
         }
+        plane_shift<FMT>(wd, sh);
     }
     __device__ __forceinline__ void scales(int b, float& s0, float& s1) const {
         if constexpr (FMT == 4) {
@@ -92,92 +142,158 @@ struct FullChunk {
     }
 };
 
-// Decode the registers of tiles [b, b + TPG) (TPG = 2 for FP3 pairs, else 1).
-template <int FMT> struct Grp { static constexpr int TPG = FMT == 3 ? 2 : 1; };
-
-template <int FMT, bool F16>
-__device__ __forceinline__ void unpack_group(const uint32_t* wd, int grp, uint32_t a[16]) {
-    if constexpr (FMT == 2) {
-        unpack_fp2<F16>(wd[grp], a);
-    } else if constexpr (FMT == 4) {
-        unpack_fp4_word<F16>(wd[2 * grp], a);
-        unpack_fp4_word<F16>(wd[2 * grp + 1], a + 4);
-    } else {
-        unpack_fp3_pair<F16>(wd[3 * grp], wd[3 * grp + 1], wd[3 * grp + 2], a);
+// acc[i] (i = 0..3: rows g,g,g+8,g+8 x cols 2t,2t+1,2t,2t+1) and the matching
+// offset-correction sums.
+struct AccA {
+    float acc[4];
+    float corr[4];
+    __device__ __forceinline__ void zero() {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) { acc[i] = 0.f; corr[i] = 0.f; }
     }
+};
+
+__device__ __forceinline__ void mma_tile(float c[4], const uint32_t a[8], uint2 blo, uint2 bhi) {
+    const float z[4] = {0.f, 0.f, 0.f, 0.f};
+    mma16816<true>(c, a, blo.x, blo.y, z);
+    mma16816<true>(c, a + 4, bhi.x, bhi.y, c);
 }
 
-// Full chunk of one matrix: accumulate into acc.  step0 = k16 step of tile 0.
-template <int FMT, bool F16, int NB>
-__device__ __forceinline__ void chunk_full(const uint8_t* st, int lane, int g, const BSrc* bs, int step0,
-                                           Acc<NB>& acc) {
-    FullChunk<FMT> fc;
-    fc.load(st, lane, g);
-    constexpr int TPG = Grp<FMT>::TPG;
-#pragma unroll
-    for (int grp = 0; grp < 8 / TPG; ++grp) {
-        uint32_t a[16];
-        unpack_group<FMT, F16>(fc.wd, grp, a);
-#pragma unroll
-        for (int u = 0; u < TPG; ++u) {
-            const int b = grp * TPG + u;
-            uint2 blo[NB], bhi[NB];
-#pragma unroll
-            for (int n = 0; n < NB; ++n) {
-                blo[n] = bs[n].get(step0 + 2 * b);
-                bhi[n] = bs[n].get(step0 + 2 * b + 1);
-            }
-            float s0, s1;
-            fc.scales(b, s0, s1);
-            tile_mma<F16, NB>(a + 8 * u, blo, bhi, s0, s1, acc);
-        }
-    }
-}
-
-// Two matrices (gate, up) sharing the B fragments, full chunks.
-template <int FMT, bool F16, int NB>
-__device__ __forceinline__ void chunk_full2(const uint8_t* st0, const uint8_t* st1, int lane, int g, const BSrc* bs,
-                                            int step0, Acc<NB>& acc0, Acc<NB>& acc1) {
+// One full gate/up chunk pair sharing the x fragments (x pre-scaled by
+// 2^-s_b): all tiles accumulate in units of 2^-24.  S[b] / S1[b] are the
+// block sums of the lane's two columns; TWO = the second column can be live.
+template <int FMT, bool TWO>
+__device__ __forceinline__ void chunkA_full(const uint8_t* st0, const uint8_t* st1, int lane, int g, const BSrc& bs,
+                                            int step0, const float* S0, const float* S1, AccA& ag, AccA& au) {
     FullChunk<FMT> f0, f1;
     f0.load(st0, lane, g);
     f1.load(st1, lane, g);
-    constexpr int TPG = Grp<FMT>::TPG;
 #pragma unroll
-    for (int grp = 0; grp < 8 / TPG; ++grp) {
-        uint32_t a0[16], a1[16];
-        unpack_group<FMT, F16>(f0.wd, grp, a0);
-        unpack_group<FMT, F16>(f1.wd, grp, a1);
-#pragma unroll
-        for (int u = 0; u < TPG; ++u) {
-            const int b = grp * TPG + u;
-            uint2 blo[NB], bhi[NB];
-#pragma unroll
-            for (int n = 0; n < NB; ++n) {
-                blo[n] = bs[n].get(step0 + 2 * b);
-                bhi[n] = bs[n].get(step0 + 2 * b + 1);
-            }
-            float s0, s1;
-            f0.scales(b, s0, s1);
-            tile_mma<F16, NB>(a0 + 8 * u, blo, bhi, s0, s1, acc0);
-            f1.scales(b, s0, s1);
-            tile_mma<F16, NB>(a1 + 8 * u, blo, bhi, s0, s1, acc1);
+    for (int b = 0; b < 8; ++b) {
+        const uint2 blo = bs.get(step0 + 2 * b), bhi = bs.get(step0 + 2 * b + 1);
+        uint32_t a[8];
+        float c[4], s0, s1;
+        switch (b) {
+            case 0: plane_regs<FMT, 0>(f0.wd, f0.sh, a); break;
+            case 1: plane_regs<FMT, 1>(f0.wd, f0.sh, a); break;
+            case 2: plane_regs<FMT, 2>(f0.wd, f0.sh, a); break;
+            case 3: plane_regs<FMT, 3>(f0.wd, f0.sh, a); break;
+            case 4: plane_regs<FMT, 4>(f0.wd, f0.sh, a); break;
+            case 5: plane_regs<FMT, 5>(f0.wd, f0.sh, a); break;
+            case 6: plane_regs<FMT, 6>(f0.wd, f0.sh, a); break;
+            default: plane_regs<FMT, 7>(f0.wd, f0.sh, a); break;
+        }
+        mma_tile(c, a, blo, bhi);
+        f0.scales(b, s0, s1);
+        ag.acc[0] = fmaf(s0, c[0], ag.acc[0]);
+        ag.acc[2] = fmaf(s1, c[2], ag.acc[2]);
+        ag.corr[0] = fmaf(s0, S0[b], ag.corr[0]);
+        ag.corr[2] = fmaf(s1, S0[b], ag.corr[2]);
+        if (TWO) {
+            ag.acc[1] = fmaf(s0, c[1], ag.acc[1]);
+            ag.acc[3] = fmaf(s1, c[3], ag.acc[3]);
+            ag.corr[1] = fmaf(s0, S1[b], ag.corr[1]);
+            ag.corr[3] = fmaf(s1, S1[b], ag.corr[3]);
+        }
+        switch (b) {
+            case 0: plane_regs<FMT, 0>(f1.wd, f1.sh, a); break;
+            case 1: plane_regs<FMT, 1>(f1.wd, f1.sh, a); break;
+            case 2: plane_regs<FMT, 2>(f1.wd, f1.sh, a); break;
+            case 3: plane_regs<FMT, 3>(f1.wd, f1.sh, a); break;
+            case 4: plane_regs<FMT, 4>(f1.wd, f1.sh, a); break;
+            case 5: plane_regs<FMT, 5>(f1.wd, f1.sh, a); break;
+            case 6: plane_regs<FMT, 6>(f1.wd, f1.sh, a); break;
+            default: plane_regs<FMT, 7>(f1.wd, f1.sh, a); break;
+        }
+        mma_tile(c, a, blo, bhi);
+        f1.scales(b, s0, s1);
+        au.acc[0] = fmaf(s0, c[0], au.acc[0]);
+        au.acc[2] = fmaf(s1, c[2], au.acc[2]);
+        au.corr[0] = fmaf(s0, S0[b], au.corr[0]);
+        au.corr[2] = fmaf(s1, S0[b], au.corr[2]);
+        if (TWO) {
+            au.acc[1] = fmaf(s0, c[1], au.acc[1]);
+            au.acc[3] = fmaf(s1, c[3], au.acc[3]);
+            au.corr[1] = fmaf(s0, S1[b], au.corr[1]);
+            au.corr[3] = fmaf(s1, S1[b], au.corr[3]);
         }
     }
 }
 
-// Registers and scales of tile b of a partial chunk (nt < 8 tiles).
-template <int FMT, bool F16>
+// Down projection accumulators: one per distinct bit offset (class) and per
+// n-block of virtual columns (hi / lo halves of h), plus the per-row
+// correction sums of the lane's real column.
+template <int NB>
+struct AccB {
+    float acc[5][NB][4];
+    float corr[NB][2];
+    __device__ __forceinline__ void zero() {
+#pragma unroll
+        for (int c = 0; c < 5; ++c)
+#pragma unroll
+            for (int n = 0; n < NB; ++n)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[c][n][i] = 0.f;
+#pragma unroll
+        for (int n = 0; n < NB; ++n) { corr[n][0] = 0.f; corr[n][1] = 0.f; }
+    }
+};
+
+// One full down chunk (h used as it is; B operands hi/lo split fp16).
+// Sb[n][b] = block sum of h for the lane's real column of n-block n.
+template <int FMT, int NB>
+__device__ __forceinline__ void chunkB_full(const uint8_t* st, int lane, int g, const BSrc* bs, int step0,
+                                            const float (*Sb)[8], AccB<NB>& ab) {
+    FullChunk<FMT> f;
+    f.load(st, lane, g);
+#pragma unroll
+    for (int b = 0; b < 8; ++b) {
+        uint32_t a[8];
+        switch (b) {
+            case 0: plane_regs<FMT, 0>(f.wd, f.sh, a); break;
+            case 1: plane_regs<FMT, 1>(f.wd, f.sh, a); break;
+            case 2: plane_regs<FMT, 2>(f.wd, f.sh, a); break;
+            case 3: plane_regs<FMT, 3>(f.wd, f.sh, a); break;
+            case 4: plane_regs<FMT, 4>(f.wd, f.sh, a); break;
+            case 5: plane_regs<FMT, 5>(f.wd, f.sh, a); break;
+            case 6: plane_regs<FMT, 6>(f.wd, f.sh, a); break;
+            default: plane_regs<FMT, 7>(f.wd, f.sh, a); break;
+        }
+        float s0, s1;
+        f.scales(b, s0, s1);
+        constexpr int dummy = 0;
+        (void)dummy;
+        const int cls = Plane<FMT>::cls_of(b);
+#pragma unroll
+        for (int n = 0; n < NB; ++n) {
+            float c[4];
+            mma_tile(c, a, bs[n].get(step0 + 2 * b), bs[n].get(step0 + 2 * b + 1));
+            ab.acc[cls][n][0] = fmaf(s0, c[0], ab.acc[cls][n][0]);
+            ab.acc[cls][n][1] = fmaf(s0, c[1], ab.acc[cls][n][1]);
+            ab.acc[cls][n][2] = fmaf(s1, c[2], ab.acc[cls][n][2]);
+            ab.acc[cls][n][3] = fmaf(s1, c[3], ab.acc[cls][n][3]);
+            ab.corr[n][0] = fmaf(s0, Sb[n][b], ab.corr[n][0]);
+            ab.corr[n][1] = fmaf(s1, Sb[n][b], ab.corr[n][1]);
+        }
+    }
+}
+
+// ------------------------------------------------------- partial chunks ---
+
+// Registers (exact levels, fp16) and scales of tile b of a partial chunk
+// (nt < 8 tiles, per-tile layout).
+template <int FMT>
 __device__ __forceinline__ void partial_tile(const uint8_t* st, int nt, int lane, int g, int b, uint32_t a[8],
                                              float& s0, float& s1) {
     const int code_bytes = nt * 16 * FMT * 4;
     if constexpr (FMT == 2) {
-        unpack_fp2<F16>(lds32(st + lane * 4 * nt + 4 * b), a);
+        unpack_fp2<true>(lds32(st + lane * 4 * nt + 4 * b), a);
         float2 f = scale_f16x2(lds32(st + code_bytes + (g * nt + b) * 4));
         s0 = f.x; s1 = f.y;
     } else if constexpr (FMT == 4) {
         const uint8_t* p = st + lane * 8 * nt + 8 * b;
-        unpack_fp4_word<F16>(lds32(p), a);
-        unpack_fp4_word<F16>(lds32(p + 4), a + 4);
+        unpack_fp4_word<true>(lds32(p), a);
+        unpack_fp4_word<true>(lds32(p + 4), a + 4);
         uint32_t e = lds16(st + code_bytes + (g * nt + b) * 2);
         s0 = scale_e8m0(e & 0xFFu);
         s1 = scale_e8m0(e >> 8);
@@ -185,17 +301,16 @@ __device__ __forceinline__ void partial_tile(const uint8_t* st, int nt, int lane
         const uint8_t* lp = st + lane * 6 * nt;       // 2-byte aligned
         const int pair = b >> 1;
         const bool lone = (b == nt - 1) && (nt & 1);
+        const uint8_t* p = lp + 12 * pair;
         if (lone) {
-            const uint8_t* p = lp + 12 * pair;
             uint64_t s = (uint64_t)lds16(p) | ((uint64_t)lds16(p + 2) << 16) | ((uint64_t)lds16(p + 4) << 32);
-            unpack_fp3_lone<F16>(s, a);
+            unpack_fp3_lone<true>(s, a);
         } else {
-            const uint8_t* p = lp + 12 * pair;
             uint32_t w0 = lds16(p) | (lds16(p + 2) << 16);
             uint32_t w1 = lds16(p + 4) | (lds16(p + 6) << 16);
             uint32_t w2 = lds16(p + 8) | (lds16(p + 10) << 16);
             uint32_t r[16];
-            unpack_fp3_pair<F16>(w0, w1, w2, r);
+            unpack_fp3_pair<true>(w0, w1, w2, r);
 #pragma unroll
             for (int i = 0; i < 8; ++i) a[i] = (b & 1) ? r[8 + i] : r[i];
         }
@@ -204,39 +319,73 @@ __device__ __forceinline__ void partial_tile(const uint8_t* st, int nt, int lane
     }
 }
 
-template <int FMT, bool F16, int NB>
-__device__ __noinline__ void chunk_partial(const uint8_t* st, int nt, int lane, int g, const BSrc* bs, int step0,
-                                           Acc<NB>& acc) {
+// A partial chunk adds s * (exact level dot product) in units of 2^-24 so that
+// it shares the full chunks' accumulator (no offset correction: levels exact).
+template <int FMT, bool TWO>
+__device__ __forceinline__ void chunkA_partial(const uint8_t* st0, const uint8_t* st1, int nt, int lane, int g,
+                                               const BSrc& bs, int step0, AccA& ag, AccA& au) {
     for (int b = 0; b < nt; ++b) {
+        const uint2 blo = bs.get(step0 + 2 * b), bhi = bs.get(step0 + 2 * b + 1);
         uint32_t a[8];
-        float s0, s1;
-        partial_tile<FMT, F16>(st, nt, lane, g, b, a, s0, s1);
-        uint2 blo[NB], bhi[NB];
-#pragma unroll
-        for (int n = 0; n < NB; ++n) {
-            blo[n] = bs[n].get(step0 + 2 * b);
-            bhi[n] = bs[n].get(step0 + 2 * b + 1);
-        }
-        tile_mma<F16, NB>(a, blo, bhi, s0, s1, acc);
+        float c[4], s0, s1;
+        partial_tile<FMT>(st0, nt, lane, g, b, a, s0, s1);
+        mma_tile(c, a, blo, bhi);
+        s0 *= 0x1.0p-24f; s1 *= 0x1.0p-24f;
+        ag.acc[0] = fmaf(s0, c[0], ag.acc[0]); ag.acc[1] = fmaf(s0, c[1], ag.acc[1]);
+        ag.acc[2] = fmaf(s1, c[2], ag.acc[2]); ag.acc[3] = fmaf(s1, c[3], ag.acc[3]);
+        partial_tile<FMT>(st1, nt, lane, g, b, a, s0, s1);
+        mma_tile(c, a, blo, bhi);
+        s0 *= 0x1.0p-24f; s1 *= 0x1.0p-24f;
+        au.acc[0] = fmaf(s0, c[0], au.acc[0]); au.acc[1] = fmaf(s0, c[1], au.acc[1]);
+        au.acc[2] = fmaf(s1, c[2], au.acc[2]); au.acc[3] = fmaf(s1, c[3], au.acc[3]);
     }
 }
 
-// Dispatch one chunk of nt tiles of one matrix.
-template <int FMT, bool F16, int NB>
-__device__ __forceinline__ void chunk_any(const uint8_t* st, int nt, int lane, int g, const BSrc* bs, int step0,
-                                          Acc<NB>& acc) {
-    if (nt == 8) chunk_full<FMT, F16, NB>(st, lane, g, bs, step0, acc);
-    else chunk_partial<FMT, F16, NB>(st, nt, lane, g, bs, step0, acc);
+template <int FMT, int NB>
+__device__ __forceinline__ void chunkB_partial(const uint8_t* st, int nt, int lane, int g, const BSrc* bs, int step0,
+                                               AccB<NB>& ab) {
+    for (int b = 0; b < nt; ++b) {
+        uint32_t a[8];
+        float s0, s1;
+        partial_tile<FMT>(st, nt, lane, g, b, a, s0, s1);
+        s0 *= 0x1.0p-24f; s1 *= 0x1.0p-24f;   // class 0: scaled by 2^24 at the end
+#pragma unroll
+        for (int n = 0; n < NB; ++n) {
+            float c[4];
+            mma_tile(c, a, bs[n].get(step0 + 2 * b), bs[n].get(step0 + 2 * b + 1));
+            ab.acc[0][n][0] = fmaf(s0, c[0], ab.acc[0][n][0]);
+            ab.acc[0][n][1] = fmaf(s0, c[1], ab.acc[0][n][1]);
+            ab.acc[0][n][2] = fmaf(s1, c[2], ab.acc[0][n][2]);
+            ab.acc[0][n][3] = fmaf(s1, c[3], ab.acc[0][n][3]);
+        }
+    }
 }
 
-template <int FMT, bool F16, int NB>
-__device__ __forceinline__ void chunk_any2(const uint8_t* st0, const uint8_t* st1, int nt, int lane, int g,
-                                           const BSrc* bs, int step0, Acc<NB>& acc0, Acc<NB>& acc1) {
-    if (nt == 8) {
-        chunk_full2<FMT, F16, NB>(st0, st1, lane, g, bs, step0, acc0, acc1);
-    } else {
-        chunk_partial<FMT, F16, NB>(st0, nt, lane, g, bs, step0, acc0);
-        chunk_partial<FMT, F16, NB>(st1, nt, lane, g, bs, step0, acc1);
+// Final per-lane values.  A: 2^24 * acc - off * corr (x16 units).
+template <int FMT>
+__device__ __forceinline__ void finishA(const AccA& a, float v[4]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = fmaf(-Plane<FMT>::OFF, a.corr[i], a.acc[i] * 0x1.0p24f);
+}
+
+// B: sum_cls 2^(24 - s_cls) acc[cls] - off * corr, the correction folded into
+// the hi virtual column (v[n][0], v[n][2]).
+template <int FMT, int NB>
+__device__ __forceinline__ void finishB(const AccB<NB>& a, float v[NB][4]) {
+#pragma unroll
+    for (int n = 0; n < NB; ++n)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float s = 0.f;
+#pragma unroll
+            for (int c = Plane<FMT>::NCLS - 1; c >= 0; --c)
+                s = fmaf(a.acc[c][n][i], __int_as_float((127 + 24 - Plane<FMT>::s_of_cls(c)) << 23), s);
+            v[n][i] = s;
+        }
+#pragma unroll
+    for (int n = 0; n < NB; ++n) {
+        v[n][0] = fmaf(-Plane<FMT>::OFF, a.corr[n][0], v[n][0]);
+        v[n][2] = fmaf(-Plane<FMT>::OFF, a.corr[n][1], v[n][2]);
     }
 }
 

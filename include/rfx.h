@@ -49,15 +49,27 @@
  * the lane owns 8 "registers" r = 0..7, each two codes (low, high element):
  *   m = r>>2, j = r&3, row = g + 8*(j&1), k0 = 16m + 2t + 8*(j>>1) inside the
  *   block; low = code[row][k0], high = code[row][k0+1].
- *   FP2: one 32-bit word per tile; r at bits [2r,2r+2) (low) and [16+2r,..) (high).
- *   FP4: two 32-bit words per tile; word m holds r at bits [4j,4j+4) and [16+4j,..).
- *   FP3: tiles are paired (96 bits per lane per pair, 3 words); pair register
- *        R = 8*(tile&1) + r.  For R < 15: word R/5, field p = R%5 at bits
- *        [3p,3p+3) (low) and [16+3p,..) (high).  R = 15: bit i of the low code
- *        at bit 15 of word i, bit i of the high code at bit 31 of word i.  A
- *        lone last tile of a chunk (odd nt) is a 48-bit little-endian stream of
- *        its 16 codes, code 2r+e (e = 0 low, 1 high) at bits [3(2r+e), +3).
- *   Scales of a chunk: [g][tile][row g, row g+8], binary16 or E8M0 bytes.
+ * A field of a register is a pair of b-bit slots at bit offset f of the two
+ * 16-bit halves of a 32-bit word: low code at bits [f, f+b), high code at
+ * [16+f, 16+f+b).
+ * Full chunks (8 tiles, "plane" layout: the 8 registers of a tile share one
+ * offset, in 8 different words):
+ *   FP2: 8 words;  register r of tile b -> word r, f = 2b.
+ *   FP4: 16 words; register r of tile b -> word r (b < 4) or 8+r (b >= 4),
+ *        f = 4*(b&3).
+ *   FP3: 12 words; tiles 0..4: word r, f = 3b; tiles 5, 6: r < 4 -> word 8+r,
+ *        f = 3(b-5); r >= 4 -> word 4+r, f = 3(b-2); tile 7: r < 4 -> word 8+r,
+ *        f = 6; r >= 4 -> bit i (i = 0..2) of the low code at bit 15 and of the
+ *        high code at bit 31 of word 3(r-4)+i.
+ * Partial chunks (nt < 8, "tile" layout):
+ *   FP2: one word per tile; r at f = 2r.
+ *   FP4: two words per tile; word m holds r = 4m+j at f = 4j.
+ *   FP3: tiles paired (96 bits per lane per pair, 3 words); pair register
+ *        R = 8*(tile&1) + r.  R < 15: word R/5, f = 3(R%5).  R = 15: bit i of
+ *        the low code at bit 15 and of the high code at bit 31 of word i.  A
+ *        lone last tile (odd nt) is a 48-bit little-endian stream of its 16
+ *        codes, code 2r+e (e = 0 low, 1 high) at bits [3(2r+e), +3).
+ * Scales of a chunk: [g][tile][row g, row g+8], binary16 or E8M0 bytes.
  */
 #ifndef RFX_H
 #define RFX_H

@@ -69,38 +69,73 @@ def _reg_coords(g, t, r):
     return g + 8 * (j & 1), 16 * m + 2 * t + 8 * (j >> 1)
 
 
+def _full_field(fmt, b, r):
+    """(word, offset, spare) of register r of tile b in a full chunk, as rfx.h states."""
+    if fmt == 2:
+        return r, 2 * b, False
+    if fmt == 4:
+        return (r if b < 4 else 8 + r), 4 * (b & 3), False
+    if b < 5:
+        return r, 3 * b, False
+    if b < 7:
+        return (8 + r, 3 * (b - 5), False) if r < 4 else (4 + r, 3 * (b - 2), False)
+    return (8 + r, 6, False) if r < 4 else (3 * (r - 4), 0, True)
+
+
 def test_layout_matches_header_description():
-    """Rebuild the first chunk of a row-group from the bit positions rfx.h documents."""
+    """Rebuild packed chunks from the bit positions rfx.h documents."""
     rows, cols = 16, 256 + 96          # one full chunk and one partial chunk of 3 tiles
     for fmt in (2, 3, 4):
         spec = synth.MatrixSpec(4, 0, 1, 0, fmt, rows, cols)
         c, s = spec.codes(), spec.scales()
         packed = rfx.rfx_pack(fmt, c, s)
-        nt = 8
-        lane_bytes = nt * 2 * fmt
+        m = (1 << fmt) - 1
+        # full chunk 0: plane layout
+        lane_bytes = 8 * 2 * fmt
         for L in (0, 5, 31):
             g, t = L >> 2, L & 3
-            lane = packed[L * lane_bytes:(L + 1) * lane_bytes]
-            words = np.frombuffer(lane.tobytes(), dtype=np.uint32)
-            for b in range(nt):
+            words = [int(v) for v in np.frombuffer(packed[L * lane_bytes:(L + 1) * lane_bytes].tobytes(), np.uint32)]
+            for b in range(8):
                 for r in range(8):
                     row, k = _reg_coords(g, t, r)
                     lo, hi = int(c[row, 32 * b + k]), int(c[row, 32 * b + k + 1])
+                    wi, f, spare = _full_field(fmt, b, r)
+                    if not spare:
+                        assert (words[wi] >> f) & m == lo and (words[wi] >> (16 + f)) & m == hi
+                    else:
+                        assert sum(((words[wi + i] >> 15) & 1) << i for i in range(3)) == lo
+                        assert sum(((words[wi + i] >> 31) & 1) << i for i in range(3)) == hi
+        # partial chunk 1 (3 tiles): tile layout
+        chunk1 = packed[8 * 16 * (4 * fmt + (1 if fmt == 4 else 2)):]
+        nt = 3
+        for L in (0, 9, 31):
+            g, t = L >> 2, L & 3
+            lane = chunk1[L * nt * 2 * fmt:(L + 1) * nt * 2 * fmt].tobytes()
+            for b in range(nt):
+                for r in range(8):
+                    row, k = _reg_coords(g, t, r)
+                    kk = 256 + 32 * b + k
+                    lo, hi = int(c[row, kk]), int(c[row, kk + 1])
                     if fmt == 2:
-                        w = int(words[b])
+                        w = int(np.frombuffer(lane[4 * b:4 * b + 4], np.uint32)[0])
                         assert (w >> (2 * r)) & 3 == lo and (w >> (16 + 2 * r)) & 3 == hi
                     elif fmt == 4:
-                        w, j = int(words[2 * b + (r >> 2)]), r & 3
+                        w = int(np.frombuffer(lane[8 * b + 4 * (r >> 2):8 * b + 4 * (r >> 2) + 4], np.uint32)[0])
+                        j = r & 3
                         assert (w >> (4 * j)) & 15 == lo and (w >> (16 + 4 * j)) & 15 == hi
                     else:
-                        R = 8 * (b & 1) + r
-                        ws = [int(v) for v in words[3 * (b >> 1):3 * (b >> 1) + 3]]
-                        if R < 15:
-                            w, p = ws[R // 5], R % 5
-                            assert (w >> (3 * p)) & 7 == lo and (w >> (16 + 3 * p)) & 7 == hi
-                        else:
-                            assert sum(((ws[i] >> 15) & 1) << i for i in range(3)) == lo
-                            assert sum(((ws[i] >> 31) & 1) << i for i in range(3)) == hi
+                        if b < 2:   # pair (0, 1): 3 words
+                            ws = [int(v) for v in np.frombuffer(lane[0:12], np.uint32)]
+                            R = 8 * b + r
+                            if R < 15:
+                                w, p_ = ws[R // 5], R % 5
+                                assert (w >> (3 * p_)) & 7 == lo and (w >> (16 + 3 * p_)) & 7 == hi
+                            else:
+                                assert sum(((ws[i] >> 15) & 1) << i for i in range(3)) == lo
+                                assert sum(((ws[i] >> 31) & 1) << i for i in range(3)) == hi
+                        else:       # lone tile 2: 48-bit stream
+                            st = int.from_bytes(lane[12:18], "little")
+                            assert (st >> (3 * (2 * r))) & 7 == lo and (st >> (3 * (2 * r + 1))) & 7 == hi
         # scales of the first chunk: [g][tile][row g, row g+8]
         sb = 1 if fmt == 4 else 2
         sc = packed[8 * 16 * 4 * fmt: 8 * 16 * 4 * fmt + 8 * 8 * 2 * sb]
