@@ -58,10 +58,11 @@ _ws_bytes = _proto("moe_ffn_workspace_bytes", _sz, [_vp, _i32])
 _ws_init = _proto("rfx_ws_init", _i32, [_vp, _sz, _vp])
 _ws_status = _proto("rfx_ws_status", _i32, [_vp, _vp])
 _forward = _proto("moe_ffn_forward", _i32, [_vp, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp])
+_forward_static = _proto("moe_ffn_forward_static", _i32, [_vp, _vp, _i32, _vp, _vp, _vp, _vp])
 
 EXPORTED = ["rfx_last_error", "rfx_packed_bytes", "rfx_pack", "rfx_unpack", "rfx_pack_device", "moe_router_topk",
             "rfx_gemv_q", "moe_layer_create", "moe_layer_destroy", "moe_ffn_workspace_bytes", "rfx_ws_init",
-            "rfx_ws_status", "moe_ffn_forward"]
+            "rfx_ws_status", "moe_ffn_forward", "moe_ffn_forward_static"]
 
 
 class RfxError(RuntimeError):
@@ -169,6 +170,12 @@ def rfx_ws_status(ws, stream=None) -> int:
 def moe_ffn_forward(handle: int, x, T: int, idx, w, y, ws, stream=None):
     _check(_forward(handle, _ptr(x), T, _ptr(idx), _ptr(w), _ptr(y), _ptr(ws), ws.numel() * ws.element_size(),
                     _stream(stream)))
+
+
+def moe_ffn_forward_static(handle: int, x, T: int, idx, w, y, stream=None):
+    """moe_ffn_forward with the library's built-in 16 MiB workspace, for callers
+    that cannot allocate device memory (see include/rfx.h)."""
+    _check(_forward_static(handle, _ptr(x), T, _ptr(idx), _ptr(w), _ptr(y), _stream(stream)))
 
 
 # --------------------------------------------------------- convenience ---

@@ -130,6 +130,12 @@ extern "C" size_t moe_ffn_workspace_bytes(const moe_layer* layer, int T) {
     return rfx::moe_ws_layout(T, layer->d.k, layer->d.H, layer->d.I).total;
 }
 
+// Bytes at the start of a workspace that hold control words (they must be
+// zero before a call; the kernel returns them to zero when it finishes).
+size_t rfx_moe_ctrl_bytes(const moe_layer* layer) {
+    return layer ? rfx::moe_ws_layout(1, layer->d.k, layer->d.H, layer->d.I).h_off : 0;
+}
+
 extern "C" int rfx_ws_init(void* ws, size_t ws_bytes, void* stream) {
     if (!ws) return rfx_fail(RFX_EINVAL, "rfx_ws_init: null workspace");
     cudaError_t e = cudaMemsetAsync(ws, 0, ws_bytes, (cudaStream_t)stream);

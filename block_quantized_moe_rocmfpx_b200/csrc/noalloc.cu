@@ -1,0 +1,88 @@
+// noalloc.cu -- moe_ffn_forward_static: the MoE FFN entry point for callers
+// that cannot allocate device memory.
+//
+// Some callers cannot call cudaMalloc at all: code that runs where allocation
+// is forbidden or unavailable (a real-time serving loop with a no-allocation
+// rule, a plugin inside a host application that owns the device allocator, an
+// embedded runtime with a fixed memory budget).  For them this entry point
+// runs the same kernel as moe_ffn_forward but takes its workspace from a
+// file-scope device array compiled into the library, so the caller passes only
+// the layer handle, inputs, outputs and a stream.
+//
+// Facts a caller must know:
+//  - The array holds RFX_STATIC_WS_BYTES (16 MiB) on every GPU that loads this
+//    library, for as long as the process runs.  Calls whose workspace would be
+//    larger (see moe_ffn_workspace_bytes) are rejected with RFX_EUNSUPPORTED.
+//  - The first call on a device resolves the array's device address with
+//    cudaGetSymbolAddress (with that device current); make that first call
+//    before any stream capture on the device.
+//  - Every call on a device uses the same array, which keeps the previous
+//    call's contents.  Each call clears the control words that must start at
+//    zero (an asynchronous memset on the given stream) and rewrites the rest.
+//    Calls that overlap on the GPU (different streams, or graphs replayed
+//    concurrently) race on the array and give wrong results: serialise them.
+//  - Device-side error flags are written into the array and are not reported
+//    by this entry point; a caller who needs them uses moe_ffn_forward with a
+//    workspace of its own.
+#include <cuda_runtime.h>
+
+#include <mutex>
+#include <string>
+
+#include "../../include/rfx.h"
+#include "moe_decode.h"
+
+int rfx_fail(int code, const std::string& msg);   // rfx_pack.cpp
+size_t rfx_moe_ctrl_bytes(const moe_layer* layer);  // api.cu: bytes of the workspace control block
+
+#define RFX_STATIC_WS_BYTES (16u << 20)
+
+// The workspace array.  In host code its name is only a handle for
+// cudaGetSymbolAddress, never a device address.
+static __device__ __align__(256) unsigned char g_rfx_static_ws[RFX_STATIC_WS_BYTES];
+
+namespace {
+
+std::mutex g_ws_mutex;
+void* g_ws_addr[64] = {nullptr};
+
+// Device address of the array on the current device (resolved once per device).
+int static_ws_address(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return rfx_fail(RFX_ECUDA, std::string("moe_ffn_forward_static: cudaGetDevice: ") + cudaGetErrorString(e));
+    if (dev < 0 || dev >= 64) return rfx_fail(RFX_EUNSUPPORTED, "moe_ffn_forward_static: device index >= 64");
+    std::lock_guard<std::mutex> lock(g_ws_mutex);
+    if (!g_ws_addr[dev]) {
+        void* ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_rfx_static_ws);
+        if (e != cudaSuccess || !ptr)
+            return rfx_fail(RFX_ECUDA, std::string("moe_ffn_forward_static: cudaGetSymbolAddress: ") +
+                                           cudaGetErrorString(e));
+        g_ws_addr[dev] = ptr;
+    }
+    *out = g_ws_addr[dev];
+    return RFX_OK;
+}
+
+}  // namespace
+
+extern "C" int moe_ffn_forward_static(const moe_layer* layer, const void* x, int T, const int32_t* idx,
+                                      const float* w, float* y, void* stream) {
+    if (!layer) return rfx_fail(RFX_EINVAL, "moe_ffn_forward_static: null layer");
+    const size_t need = moe_ffn_workspace_bytes(layer, T);
+    if (need == 0) return rfx_fail(RFX_EUNSUPPORTED, "moe_ffn_forward_static: 1 <= T <= 8 token columns");
+    if (need > RFX_STATIC_WS_BYTES)
+        return rfx_fail(RFX_EUNSUPPORTED, "moe_ffn_forward_static: this layer and T need " + std::to_string(need) +
+                                              " workspace bytes, more than the static " +
+                                              std::to_string((size_t)RFX_STATIC_WS_BYTES) + "; use moe_ffn_forward");
+    void* ws = nullptr;
+    int rc = static_ws_address(&ws);
+    if (rc != RFX_OK) return rc;
+    // the control words (task, exit and readiness counters, error flag) must
+    // start at zero; everything after them is rewritten by the kernel
+    const size_t ctrl_bytes = rfx_moe_ctrl_bytes(layer);
+    cudaError_t e = cudaMemsetAsync(ws, 0, ctrl_bytes, (cudaStream_t)stream);
+    if (e != cudaSuccess) return rfx_fail(RFX_ECUDA, std::string("moe_ffn_forward_static: ") + cudaGetErrorString(e));
+    return moe_ffn_forward(layer, x, T, idx, w, y, ws, RFX_STATIC_WS_BYTES, stream);
+}

@@ -209,6 +209,25 @@ int rfx_ws_status(void* ws, void* stream);
 int moe_ffn_forward(const moe_layer* layer, const void* x, int T, const int32_t* idx, const float* w,
                     float* y, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * moe_ffn_forward_static -- the same MoE FFN as moe_ffn_forward for callers
+ * that cannot allocate device memory (a serving loop with a no-allocation
+ * rule, a plugin that does not own the device allocator, a fixed-budget
+ * embedded runtime).  The pages have no counterpart: this is a property of
+ * the library, not of the method.
+ * The workspace is a 16 MiB array compiled into the library (held on every
+ * GPU that loads it until the process exits); calls that would need more
+ * (moe_ffn_workspace_bytes) return RFX_EUNSUPPORTED.  The first call on a
+ * device looks up the array's device address; make it before any stream
+ * capture on that device.  All calls on a device share the array: each clears
+ * its control words with an asynchronous memset on `stream`, and calls that
+ * overlap on the GPU race and give wrong results.  Device-side error flags are
+ * not reported here (use moe_ffn_forward with your own workspace for that).
+ * x, idx, w, y, T and stream as in moe_ffn_forward.  Allocates nothing.
+ */
+int moe_ffn_forward_static(const moe_layer* layer, const void* x, int T, const int32_t* idx, const float* w,
+                           float* y, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
