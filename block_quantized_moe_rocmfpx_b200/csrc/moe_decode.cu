@@ -19,14 +19,14 @@
 //  - Tasks: A = (slot, 32 gate/up rows) -> SwiGLU -> h; B = (slot, 32 down
 //    rows) -> partial d.  Tasks are handed out by a global atomic counter, A
 //    before B, so a B task only ever waits on A tasks already running.
-//  - Per CTA: lane 0 of the producer warp streams packed spans of 8 chunks
+//  - Per CTA: one lane of the producer warp streams packed spans of 8 chunks
 //    HBM -> shared memory with 1-D bulk copies (TMA, evict-first L2 policy)
-//    into a ring of stages; lane 1 bulk-copies the SwiGLU output h of a slot
-//    once all of its gate/up rows are published.  8 consumer warps take one
+//    into a ring of stages; one lane of the h warp bulk-copies the SwiGLU
+//    output h of a slot once all of its gate/up rows are published.  8 consumer warps take one
 //    chunk of every stage each, decode it in registers (one AND per A
 //    register, see rfx_tile.cuh) and run mma.sync m16n8k16 in fp16: x
 //    normalised per column by a power of two for gate/up, an exact hi/lo fp16
-//    split of h for down.  3 epilogue warps sum the 8 warps' partials of
+//    split of h for down.  2 epilogue warps sum the 8 warps' partials of
 //    each row-group in a fixed order and run SwiGLU or the combine, so the
 //    consumers never wait on global-memory latency.
 //  - Combine: the last down task to finish a 16-row group sums the slots'
@@ -42,10 +42,11 @@
 namespace rfx {
 
 constexpr int NCW = 8;                       // consumer warps 0..7
-constexpr int WARP_PRODUCER = NCW;           // bulk-copy issue (one lane)
-constexpr int NEPI = 3;                      // epilogue warps: reductions, SwiGLU, combine
-constexpr int WARP_EPILOGUE0 = NCW + 1;
-constexpr int NTHREADS = (NCW + 1 + NEPI) * 32;
+constexpr int WARP_PRODUCER = NCW;           // weight bulk copies (one lane)
+constexpr int WARP_HLOAD = NCW + 1;          // h bulk copies of the down tasks (one lane)
+constexpr int NEPI = 2;                      // epilogue warps: reductions, SwiGLU, combine
+constexpr int WARP_EPILOGUE0 = NCW + 2;
+constexpr int NTHREADS = (NCW + 2 + NEPI) * 32;
 constexpr int QN = 4;
 constexpr int NRED_MAX = MOE_MAX_RED;        // reduction buffers: unit r -> buffer r % p.nred,
                                              // epilogue warp r % NEPI
@@ -70,17 +71,26 @@ struct RedInfo {
     int slot, ncols, rg, last_of_task;
 };
 
+// What a ring stage holds, written by the producer with the stage.
+enum : short { REC_FIRST = 1, REC_LAST = 2, REC_TFIRST = 4, REC_TLAST = 8 };
+struct __align__(16) StageRec {
+    short kind;    // 0: gate/up span, 1: down span, -1: end of work (no copy)
+    short slot;
+    short rg;      // row-group of the matrix (rows 16*rg ..)
+    short c0;      // first chunk of the span
+    short flags;   // REC_*: first / last span of the row-group, of the task
+    short pad[3];
+};
+
 struct Shared {
     uint64_t full[MOE_MAX_STAGES];
     uint64_t empty[MOE_MAX_STAGES];
-    uint64_t tqf[QN], tqe[QN];
     uint64_t hfull[2], hfree[2];
     uint64_t xfree;
-    uint64_t xload;          // x bulk copy into the (not yet used) stage ring
     uint64_t rfull[NRED_MAX], rempty[NRED_MAX];
     uint64_t hqf[QN], hqe[QN];
     int hq[QN];
-    int tq[QN];
+    StageRec rec[MOE_MAX_STAGES];
     RedInfo rinfo[NRED_MAX];
     volatile int abort_flag;
     volatile int consumed;   // stages released by all consumer warps (for the abort drain)
@@ -183,7 +193,9 @@ __device__ __forceinline__ MatRef slot_mats(const MoeParams& p, int e, int kind)
 // ------------------------------------------------------------- producer ---
 //
 // Per task (32 rows = 2 row-groups) and per row-group, one stage per span of
-// up to 8 chunks: a single bulk copy per matrix of the contiguous span.
+// up to 8 chunks: a single bulk copy per matrix of the contiguous span.  The
+// stage record (what the stage holds) is written before the arrive that
+// publishes the stage, so a consumer reads it after its acquire on `full`.
 
 __device__ void producer(const MoeParams& p, Shared& sh, uint8_t* ring) {
     const SlotTable& S = sh.st;
@@ -195,17 +207,12 @@ __device__ void producer(const MoeParams& p, Shared& sh, uint8_t* ring) {
     int sc = 0;
     bool ok = true;
     int next = (int)atomicAdd(p.ctrl + MOE_CTRL_TASK, 1u);
-    int qi = 0, hi = 0;
-    uint32_t qphase = 1, hphase = 1;
-    for (int n = 0; ok; ++n) {
-        int t = next;
-        if (t >= ntasks) t = -1;
-        else next = (int)atomicAdd(p.ctrl + MOE_CTRL_TASK, 1u);   // used next iteration: latency hidden
-        if (!mbar_wait(&sh.tqe[qi], qphase, WAIT_LIMIT)) { ok = false; break; }
-        sh.tq[qi] = t;
-        mbar_arrive(&sh.tqf[qi]);
-        if (++qi == QN) { qi = 0; qphase ^= 1u; }
-        if (t < 0) break;
+    int hi = 0;
+    uint32_t hphase = 1;
+    while (ok) {
+        const int t = next;
+        if (t >= ntasks) break;
+        next = (int)atomicAdd(p.ctrl + MOE_CTRL_TASK, 1u);   // used next iteration: latency hidden
         const Task tk = decode_task(t, S.nslots, nrbA, nrbB);
         if (tk.kind == 1) {
             // hand the h copy of this down task to the h lane
@@ -228,6 +235,14 @@ __device__ void producer(const MoeParams& p, Shared& sh, uint8_t* ring) {
                 const int c1 = min(nch, c0 + MOE_CHUNKS_PER_STAGE);
                 const uint32_t bytes = (uint32_t)((c1 - 1 - c0) * fullb) + (c1 == nch ? lastb : (uint32_t)fullb);
                 if (!mbar_wait(&sh.empty[stage], ephase, WAIT_LIMIT)) { ok = false; break; }
+                StageRec r{};
+                r.kind = (short)tk.kind;
+                r.slot = (short)tk.slot;
+                r.rg = (short)(2 * tk.rb + rgl);
+                r.c0 = (short)c0;
+                r.flags = (short)((c0 == 0 ? REC_FIRST : 0) | (c1 == nch ? REC_LAST : 0) |
+                                  (rgl == 0 && c0 == 0 ? REC_TFIRST : 0) | (rgl == 1 && c1 == nch ? REC_TLAST : 0));
+                sh.rec[stage] = r;
                 uint8_t* dst = ring + stage * MOE_STAGE_BYTES;
                 const long long off = (long long)rgl * rgb + (long long)c0 * fullb;
                 if (tk.kind == 0) {
@@ -243,6 +258,17 @@ __device__ void producer(const MoeParams& p, Shared& sh, uint8_t* ring) {
             }
         }
     }
+    // end-of-work record: a stage with no copy
+    if (ok) {
+        if (mbar_wait(&sh.empty[stage], ephase, WAIT_LIMIT)) {
+            StageRec r{};
+            r.kind = -1;
+            sh.rec[stage] = r;
+            mbar_arrive(&sh.full[stage]);
+        } else {
+            ok = false;
+        }
+    }
     // stop the h lane
     if (mbar_wait(&sh.hqe[hi], hphase, WAIT_LIMIT)) {
         sh.hq[hi] = -1;
@@ -255,10 +281,6 @@ __device__ void producer(const MoeParams& p, Shared& sh, uint8_t* ring) {
         sh.abort_flag = 1;
         // drain: wait (bounded) until every issued copy has landed
         for (int i = sh.consumed; i < sc; ++i) (void)mbar_wait(&sh.full[i % p.ns], (i / p.ns) & 1, WAIT_LIMIT);
-        for (int q = 0; q < QN; ++q) {
-            sh.tq[q] = -1;
-            mbar_arrive(&sh.tqf[q]);
-        }
     }
 }
 
@@ -285,9 +307,11 @@ __device__ void h_loader(const MoeParams& p, Shared& sh, uint8_t* xh, int hbytes
         if (!mbar_wait(&sh.hfree[buf], ((bseq >> 1) + 1) & 1, WAIT_LIMIT)) { ok = false; break; }
         if (!(known_ready[slot >> 5] >> (slot & 31) & 1u)) {
             const long long t0 = clock64();
+            unsigned nap = 32;
             while (ld_relaxed_gpu(p.ctrl + MOE_CTRL_SLOT + slot) < need) {
                 if (clock64() - t0 > WAIT_LIMIT) { ok = false; break; }
-                __nanosleep(20);
+                __nanosleep(nap);
+                nap = min(nap * 2u, 256u);
             }
             if (!ok) break;
             known_ready[slot >> 5] |= 1u << (slot & 31);
@@ -466,191 +490,193 @@ __device__ __forceinline__ int s_pos(int fmt, int k, int K) {
 struct Ring {
     int stage = 0, cc = 0;
     uint32_t fphase = 0;
+    __device__ __forceinline__ void release(const MoeParams& p, Shared& sh, int w, int lane) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.empty[stage]);
+        ++cc;
+        if (w == 0 && lane == 0) sh.consumed = cc;
+        if (++stage == p.ns) { stage = 0; fphase ^= 1u; }
+    }
 };
 
-// All stages of one gate/up row-group: warp w takes chunk w of every stage.
+__device__ __forceinline__ void ld8(const float* src, float d[8]) {
+    const float4 a = ldsf4((const uint8_t*)src), b = ldsf4((const uint8_t*)(src + 4));
+    d[0] = a.x; d[1] = a.y; d[2] = a.z; d[3] = a.w;
+    d[4] = b.x; d[5] = b.y; d[6] = b.z; d[7] = b.w;
+}
+
+// One gate/up chunk pair (chunk c of the stage's span, this warp's share).
 template <int FMT, bool TWO>
-__device__ __forceinline__ bool rowgroup_a(const MoeParams& p, Shared& sh, uint8_t* ring, Ring& rg_, int nch, int w,
-                                        int lane, const BSrc& bs_in, const float* sA0, const float* sA1, float v[8]) {
-    const int g = lane >> 2;
-    const BSrc bs = bs_in;   // keep the operand source in registers
-    constexpr int FULLB = (int)(8 * 16 * (FMT * 4 + (FMT == 4 ? 1 : 2)));
-    AccA ag, au;
-    ag.zero();
-    au.zero();
-    for (int c0 = 0; c0 < nch; c0 += MOE_CHUNKS_PER_STAGE) {
-        if (!mbar_wait(&sh.full[rg_.stage], rg_.fphase, WAIT_LIMIT)) return false;
-        const int c = c0 + w;
-        if (c < nch) {
-            const uint8_t* st = ring + rg_.stage * MOE_STAGE_BYTES + w * FULLB;
-            const int nt = rfx_chunk_tiles(p.H, c);
-            if (nt == 8) {
-                float S0[8], S1[8];
-                const float4 a0 = ldsf4((const uint8_t*)(sA0 + 8 * c)), a1 = ldsf4((const uint8_t*)(sA0 + 8 * c + 4));
-                S0[0] = a0.x; S0[1] = a0.y; S0[2] = a0.z; S0[3] = a0.w;
-                S0[4] = a1.x; S0[5] = a1.y; S0[6] = a1.z; S0[7] = a1.w;
-                if (TWO) {
-                    const float4 b0 = ldsf4((const uint8_t*)(sA1 + 8 * c)), b1 = ldsf4((const uint8_t*)(sA1 + 8 * c + 4));
-                    S1[0] = b0.x; S1[1] = b0.y; S1[2] = b0.z; S1[3] = b0.w;
-                    S1[4] = b1.x; S1[5] = b1.y; S1[6] = b1.z; S1[7] = b1.w;
-                }
-                chunkA_full<FMT, TWO>(st, st + MOE_HALF_BYTES, lane, g, bs, c * 16, S0, S1, ag, au);
-            } else {
-                chunkA_partial<FMT, true>(st, st + MOE_HALF_BYTES, nt, lane, g, bs, c * 16, ag, au);
-            }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sh.empty[rg_.stage]);
-        ++rg_.cc;
-        if (w == 0 && lane == 0) sh.consumed = rg_.cc;
-        if (++rg_.stage == p.ns) { rg_.stage = 0; rg_.fphase ^= 1u; }
+__device__ __forceinline__ void stepA(const uint8_t* st, int c, int H, int lane, int g, const BSrc& bs, const float* sA0,
+                                      const float* sA1, AccA& ag, AccA& au) {
+    const int nt = rfx_chunk_tiles(H, c);
+    if (nt == 8) {
+        float S0[8], S1[8];
+        ld8(sA0 + 8 * c, S0);
+        if (TWO) ld8(sA1 + 8 * c, S1);
+        chunkA_full<FMT, TWO>(st, st + MOE_HALF_BYTES, lane, g, bs, c * 16, S0, S1, ag, au);
+    } else {
+        chunkA_partial<FMT, true>(st, st + MOE_HALF_BYTES, nt, lane, g, bs, c * 16, ag, au);
     }
-    finishA<FMT>(ag, v);
-    finishA<FMT>(au, v + 4);
-    return true;
 }
 
-// All stages of one down row-group (usually a single stage of 8 chunks).
+// One down chunk.
 template <int FMT, int NB>
-__device__ __forceinline__ bool rowgroup_b(const MoeParams& p, Shared& sh, uint8_t* ring, Ring& rg_, int nch, int w,
-                                        int lane, const BSrc* bs_in, const float* hsum, int ncols, int sstr,
-                                        float v[8]) {
-    const int g = lane >> 2, t = lane & 3;
-    BSrc bs[NB];   // keep the operand sources in registers
+__device__ __forceinline__ void stepB(const uint8_t* st, int c, int I, int lane, int g, int t, const BSrc* bs,
+                                      const float* hsum, int ncols, int sstr, AccB<NB>& ab) {
+    const int nt = rfx_chunk_tiles(I, c);
+    if (nt == 8) {
+        // block sums of h for the lane's real column(s): two halves per block
+        float Sb[NB][8];
 #pragma unroll
-    for (int nb = 0; nb < NB; ++nb) bs[nb] = bs_in[nb];
-    constexpr int FULLB = (int)(8 * 16 * (FMT * 4 + (FMT == 4 ? 1 : 2)));
-    AccB<NB> ab;
-    ab.zero();
-    for (int c0 = 0; c0 < nch; c0 += MOE_CHUNKS_PER_STAGE) {
-        if (!mbar_wait(&sh.full[rg_.stage], rg_.fphase, WAIT_LIMIT)) return false;
-        const int c = c0 + w;
-        if (c < nch) {
-            const uint8_t* st = ring + rg_.stage * MOE_STAGE_BYTES + w * FULLB;
-            const int nt = rfx_chunk_tiles(p.I, c);
-            if (nt == 8) {
-                // block sums of h for the lane's real column(s): two halves per block
-                float Sb[NB][8];
+        for (int nb = 0; nb < NB; ++nb) {
+            const int colr = 4 * nb + t;
+            const float* hp = hsum + (colr < ncols ? colr : 0) * sstr + 16 * c;
 #pragma unroll
-                for (int nb = 0; nb < NB; ++nb) {
-                    const int colr = 4 * nb + t;
-                    const float* hp = hsum + (colr < ncols ? colr : 0) * sstr + 16 * c;
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const float4 x4 = ldsf4((const uint8_t*)(hp + 4 * q));
-                        Sb[nb][2 * q] = x4.x + x4.y;
-                        Sb[nb][2 * q + 1] = x4.z + x4.w;
-                    }
-                }
-                chunkB_full<FMT, NB>(st, lane, g, bs, c * 16, Sb, ab);
-            } else {
-                chunkB_partial<FMT, NB>(st, nt, lane, g, bs, c * 16, ab);
+            for (int q = 0; q < 4; ++q) {
+                const float4 x4 = ldsf4((const uint8_t*)(hp + 4 * q));
+                Sb[nb][2 * q] = x4.x + x4.y;
+                Sb[nb][2 * q + 1] = x4.z + x4.w;
             }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sh.empty[rg_.stage]);
-        ++rg_.cc;
-        if (w == 0 && lane == 0) sh.consumed = rg_.cc;
-        if (++rg_.stage == p.ns) { rg_.stage = 0; rg_.fphase ^= 1u; }
+        chunkB_full<FMT, NB>(st, lane, g, bs, c * 16, Sb, ab);
+    } else {
+        chunkB_partial<FMT, NB>(st, nt, lane, g, bs, c * 16, ab);
     }
-    float vb[NB][4];
-    finishB<FMT, NB>(ab, vb);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        v[i] = vb[0][i];
-        v[4 + i] = NB > 1 ? vb[NB - 1][i] : 0.f;
-    }
-    return true;
 }
 
+__device__ __forceinline__ int full_chunk_bytes(int fmt) { return 128 * rfx_block_bytes(fmt); }
+
+// Consumer warp: one flat loop over the ring.  Every CTA's stream holds all of
+// its gate/up spans before its down spans (tasks are handed out A first), so
+// the two phases are two loops with their own accumulators.
+template <int QC>
 __device__ void consumer(const MoeParams& p, Shared& sh, uint8_t* ring, uint8_t* xh, int hbytes_max, float* red,
                          int sstr) {
+    constexpr bool TWO = QC >= 2;           // a second live column per lane in the gate/up output
+    constexpr int NB = QC >= 3 ? 2 : 1;     // n-blocks of virtual (hi, lo) columns in the down projection
     const SlotTable& S = sh.st;
     const int w = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
-    const int nrbA = p.I / 32, nrbB = p.H / 32;
     const int nxc = (p.has_shared && p.fsA != p.fA) ? 2 : 1;
     const float* sx = (const float*)(xh + nxc * p.T * p.x_stride);   // [copy][col][sxs]
     const int sxs = moe_sxs(p.H);
+    const int nchA = rfx_num_chunks(p.H), nchB = rfx_num_chunks(p.I);
     Ring ring_pos;
-    int bseq = 0;
-    int qi = 0;
-    uint32_t qphase = 0;
     RedCursor rc;
-    bool first_b = true, ok = true;
-    while (ok) {
-        if (!mbar_wait(&sh.tqf[qi], qphase, WAIT_LIMIT)) { ok = false; break; }
-        const int task = sh.tq[qi];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sh.tqe[qi]);
-        if (++qi == QN) { qi = 0; qphase ^= 1u; }
-        if (task < 0 || sh.abort_flag) break;
-        const Task tk = decode_task(task, S.nslots, nrbA, nrbB);
-        const int slot = tk.slot;
-        const int e = S.expert[slot];
-        const int ncols = S.ncols[slot];
-        const int fmt = tk.kind == 0 ? (e < 0 ? p.fsA : p.fA) : (e < 0 ? p.fsB : p.fB);
-        const int buf_h = bseq & 1;
-        if (tk.kind == 1) {
-            if (first_b) {
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sh.xfree);
-                first_b = false;
-            }
-            if (!mbar_wait(&sh.hfull[buf_h], (bseq >> 1) & 1, WAIT_LIMIT)) { ok = false; break; }
-        }
-        for (int rgl = 0; rgl < 2 && ok; ++rgl) {
-            float v[8];
-            if (tk.kind == 0) {
+    bool ok = true;
+    StageRec r{};
+    // ---- gate/up spans -> SwiGLU partials
+    {
+        AccA ag, au;
+        ag.zero();
+        au.zero();
+        BSrc bs{xh, 0, false};
+        const float* sA0 = sx;
+        const float* sA1 = sx;
+        int slot = 0, ncols = 0, fmt = 2;
+        while (true) {
+            if (!mbar_wait(&sh.full[ring_pos.stage], ring_pos.fphase, WAIT_LIMIT)) { ok = false; break; }
+            r = sh.rec[ring_pos.stage];
+            if (r.kind != 0) break;
+            if (r.flags & REC_FIRST) {
+                slot = r.slot;
+                const int e = S.expert[slot];
+                ncols = S.ncols[slot];
+                fmt = e < 0 ? p.fsA : p.fA;
                 const int ci = (e < 0 && nxc == 2) ? 1 : 0;
                 const int col0 = g < ncols ? S.cols[slot][g] : 0;
-                const BSrc bs{xh + (ci * p.T + col0) * p.x_stride + t * 8, 32, g < ncols};
+                bs = BSrc{xh + (ci * p.T + col0) * p.x_stride + t * 8, 32, g < ncols};
                 const int c0 = 2 * t < ncols ? S.cols[slot][2 * t] : 0;
                 const int c1 = 2 * t + 1 < ncols ? S.cols[slot][2 * t + 1] : 0;
-                const float* sA0 = sx + (ci * p.T + c0) * sxs;
-                const float* sA1 = sx + (ci * p.T + c1) * sxs;
-                const int nch = rfx_num_chunks(p.H);
-                const bool two = ncols > 1;
-                switch (fmt * 2 + (two ? 1 : 0)) {
-                    case 4: ok = rowgroup_a<2, false>(p, sh, ring, ring_pos, nch, w, lane, bs, sA0, sA1, v); break;
-                    case 5: ok = rowgroup_a<2, true>(p, sh, ring, ring_pos, nch, w, lane, bs, sA0, sA1, v); break;
-                    case 6: ok = rowgroup_a<3, false>(p, sh, ring, ring_pos, nch, w, lane, bs, sA0, sA1, v); break;
-                    case 7: ok = rowgroup_a<3, true>(p, sh, ring, ring_pos, nch, w, lane, bs, sA0, sA1, v); break;
-                    case 8: ok = rowgroup_a<4, false>(p, sh, ring, ring_pos, nch, w, lane, bs, sA0, sA1, v); break;
-                    default: ok = rowgroup_a<4, true>(p, sh, ring, ring_pos, nch, w, lane, bs, sA0, sA1, v); break;
-                }
-            } else {
+                sA0 = sx + (ci * p.T + c0) * sxs;
+                sA1 = sx + (ci * p.T + c1) * sxs;
+                ag.zero();
+                au.zero();
+            }
+            const int c = r.c0 + w;
+            if (c < nchA) {
+                const uint8_t* st = ring + ring_pos.stage * MOE_STAGE_BYTES + w * full_chunk_bytes(fmt);
+                if (fmt == 2) stepA<2, TWO>(st, c, p.H, lane, g, bs, sA0, sA1, ag, au);
+                else if (fmt == 3) stepA<3, TWO>(st, c, p.H, lane, g, bs, sA0, sA1, ag, au);
+                else stepA<4, TWO>(st, c, p.H, lane, g, bs, sA0, sA1, ag, au);
+            }
+            ring_pos.release(p, sh, w, lane);
+            if (r.flags & REC_LAST) {
+                float v[8];
+                if (fmt == 2) { finishA<2>(ag, v); finishA<2>(au, v + 4); }
+                else if (fmt == 3) { finishA<3>(ag, v); finishA<3>(au, v + 4); }
+                else { finishA<4>(ag, v); finishA<4>(au, v + 4); }
+                const RedInfo info{0, slot, ncols, r.rg, (r.flags & REC_TLAST) ? 1 : 0};
+                if (!red_deposit(p, sh, red, rc, w, lane, v, info)) { ok = false; break; }
+            }
+        }
+    }
+    // ---- down spans -> partial outputs
+    if (ok && r.kind == 1) {
+        // the staged x is no longer read: the h lane may overwrite it
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.xfree);
+        AccB<NB> ab;
+        ab.zero();
+        BSrc bs[NB];
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) bs[nb] = BSrc{xh, 0, false};
+        const float* hsum = (const float*)xh;
+        int bseq = 0, slot = 0, ncols = 0, fmt = 3;
+        while (true) {
+            const int buf_h = bseq & 1;
+            if (r.flags & REC_TFIRST) {
+                if (!mbar_wait(&sh.hfull[buf_h], (bseq >> 1) & 1, WAIT_LIMIT)) { ok = false; break; }
+            }
+            if (r.flags & REC_FIRST) {
+                slot = r.slot;
+                const int e = S.expert[slot];
+                ncols = S.ncols[slot];
+                fmt = e < 0 ? p.fsB : p.fB;
                 const uint8_t* hs = xh + buf_h * hbytes_max;
                 const int vst = 64 * ncols;  // bytes per k16 step
-                BSrc bs[2];
 #pragma unroll
-                for (int nb = 0; nb < 2; ++nb) {
+                for (int nb = 0; nb < NB; ++nb) {
                     const int vv = 8 * nb + g;
-                    bs[nb] = {hs + (vv * 4 + t) * 8, vst, vv < 2 * ncols};
+                    bs[nb] = BSrc{hs + (vv * 4 + t) * 8, vst, vv < 2 * ncols};
                 }
-                const float* hsum = (const float*)(hs + 4 * ncols * p.I);
-                const int nch = rfx_num_chunks(p.I);
-                const bool two_nb = ncols > 4;
-                switch (fmt * 2 + (two_nb ? 1 : 0)) {
-                    case 4: ok = rowgroup_b<2, 1>(p, sh, ring, ring_pos, nch, w, lane, bs, hsum, ncols, sstr, v); break;
-                    case 5: ok = rowgroup_b<2, 2>(p, sh, ring, ring_pos, nch, w, lane, bs, hsum, ncols, sstr, v); break;
-                    case 6: ok = rowgroup_b<3, 1>(p, sh, ring, ring_pos, nch, w, lane, bs, hsum, ncols, sstr, v); break;
-                    case 7: ok = rowgroup_b<3, 2>(p, sh, ring, ring_pos, nch, w, lane, bs, hsum, ncols, sstr, v); break;
-                    case 8: ok = rowgroup_b<4, 1>(p, sh, ring, ring_pos, nch, w, lane, bs, hsum, ncols, sstr, v); break;
-                    default: ok = rowgroup_b<4, 2>(p, sh, ring, ring_pos, nch, w, lane, bs, hsum, ncols, sstr, v); break;
-                }
+                hsum = (const float*)(hs + 4 * ncols * p.I);
+                ab.zero();
             }
-            if (!ok) break;
-            const RedInfo info{tk.kind, slot, ncols, 2 * tk.rb + rgl, rgl == 1};
-            if (!red_deposit(p, sh, red, rc, w, lane, v, info)) { ok = false; break; }
-        }
-        if (!ok) break;
-        if (tk.kind == 1) {
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sh.hfree[buf_h]);
-            ++bseq;
+            const int c = r.c0 + w;
+            if (c < nchB) {
+                const uint8_t* st = ring + ring_pos.stage * MOE_STAGE_BYTES + w * full_chunk_bytes(fmt);
+                if (fmt == 3) stepB<3, NB>(st, c, p.I, lane, g, t, bs, hsum, ncols, sstr, ab);
+                else if (fmt == 2) stepB<2, NB>(st, c, p.I, lane, g, t, bs, hsum, ncols, sstr, ab);
+                else stepB<4, NB>(st, c, p.I, lane, g, t, bs, hsum, ncols, sstr, ab);
+            }
+            ring_pos.release(p, sh, w, lane);
+            if (r.flags & REC_LAST) {
+                float vb[NB][4];
+                if (fmt == 3) finishB<3, NB>(ab, vb);
+                else if (fmt == 2) finishB<2, NB>(ab, vb);
+                else finishB<4, NB>(ab, vb);
+                float v[8];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    v[i] = vb[0][i];
+                    v[4 + i] = NB > 1 ? vb[NB - 1][i] : 0.f;
+                }
+                const RedInfo info{1, slot, ncols, r.rg, (r.flags & REC_TLAST) ? 1 : 0};
+                if (!red_deposit(p, sh, red, rc, w, lane, v, info)) { ok = false; break; }
+            }
+            if (r.flags & REC_TLAST) {
+                // every span of this down task is consumed: release its h buffer
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sh.hfree[buf_h]);
+                ++bseq;
+            }
+            if (!mbar_wait(&sh.full[ring_pos.stage], ring_pos.fphase, WAIT_LIMIT)) { ok = false; break; }
+            r = sh.rec[ring_pos.stage];
+            if (r.kind != 1) break;
         }
     }
     if (!ok) {
@@ -663,51 +689,80 @@ __device__ void consumer(const MoeParams& p, Shared& sh, uint8_t* ring, uint8_t*
     for (int i = 0; i < NEPI; ++i) (void)red_deposit(p, sh, red, rc, w, lane, z, fin);
 }
 
-// x (bf16 [T][H]) -> shared memory for the gate/up B operand: per column
-// c, x * 2^xn[c] with xn[c] putting max|x| in [2^13, 2^14), times 2^-s_b for
-// the tile's bit offset in the gate/up format (one copy per format in use),
-// rounded to fp16 in fragment order [c][step][t][k 2t,2t+1,2t+8,2t+9]; plus
-// the block sums of the staged values (times 2^s_b) for the offset correction.
-__device__ void stage_x(const MoeParams& p, Shared& sh, uint8_t* xh, const uint32_t* x32) {
-    const int tid = threadIdx.x;   // 0 .. NCW*32-1
-    const int npairs = p.T * p.H / 2;
-    for (int i = tid; i < npairs; i += NCW * 32) {
-        const uint32_t v = x32[i];
-        const uint32_t m = max((v << 16) & 0x7fffffffu, v & 0x7fff0000u);
-        atomicMax(&sh.xmax[(2 * i) / p.H], m);
+// x (bf16 [T][H], global) -> shared memory for the gate/up B operand: per
+// column c, x * 2^xn[c] with xn[c] putting max|x| in [2^13, 2^14), times
+// 2^-s_b for the tile's bit offset in the gate/up format (one copy per format
+// in use), rounded to fp16 in fragment order [c][step][t][k 2t,2t+1,2t+8,2t+9];
+// plus the block sums of the staged values (times 2^s_b) for the offset
+// correction.  Run by `nthr` threads (sid = 0 .. nthr-1, whole warps); one item
+// is one (step, t) fragment of a column, 8 consecutive items one 32-block.
+__device__ void stage_x(const MoeParams& p, Shared& sh, uint8_t* xh, int sid, int nthr) {
+    const uint32_t* x32 = reinterpret_cast<const uint32_t*>(p.x);
+    const int lane = sid & 31;
+    const int per_col = p.H / 4;      // items per column
+    const int hp = p.H / 2;           // bf16 pairs per column
+    // pass 1: max |x| per column (a warp's items never straddle a column)
+    for (int c = 0; c < p.T; ++c) {
+        uint32_t m = 0u;
+        for (int j0 = sid - lane; j0 < per_col; j0 += nthr) {
+            const int j = j0 + lane;
+            if (j < per_col) {
+                const int step = j >> 2, tt = j & 3;
+                const uint32_t* src = x32 + (size_t)c * hp + step * 8 + tt;
+                const uint32_t v0 = __ldg(src), v1 = __ldg(src + 4);
+                m = max(m, max((v0 << 16) & 0x7fffffffu, v0 & 0x7fff0000u));
+                m = max(m, max((v1 << 16) & 0x7fffffffu, v1 & 0x7fff0000u));
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0 && m) atomicMax(&sh.xmax[c], m);
     }
-    asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
-    if (tid < p.T) {
-        const uint32_t m = sh.xmax[tid];
-        int n = m ? 13 - ((int)((m >> 23) & 255u) - 127) : 0;
-        sh.xn[tid] = max(-100, min(100, n));
+    asm volatile("bar.sync 1, %0;" ::"r"(nthr) : "memory");
+    if (sid < p.T) {
+        const uint32_t m = sh.xmax[sid];
+        const int n = m ? 13 - ((int)((m >> 23) & 255u) - 127) : 0;
+        sh.xn[sid] = max(-100, min(100, n));
     }
-    asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
+    asm volatile("bar.sync 1, %0;" ::"r"(nthr) : "memory");
+    // pass 2: scale, round to fp16, write fragments and block sums
     const int nxc = (p.has_shared && p.fsA != p.fA) ? 2 : 1;
     float* sx = (float*)(xh + nxc * p.T * p.x_stride);
-    const int hw = tid >> 4, l16 = tid & 15;
-    const unsigned hmask = 0xffffu << (tid & 16);
-    const int nblk = p.T * p.H / 32;
+    const int sxs = moe_sxs(p.H);
     for (int ci = 0; ci < nxc; ++ci) {
         const int fmt = ci == 0 ? p.fA : p.fsA;
-        for (int blk = hw; blk < nblk; blk += NCW * 2) {
-            const int i = blk * 16 + l16;
-            const int c = (2 * i) / p.H, k = (2 * i) % p.H;
-            const int s = s_pos(fmt, k, p.H);
-            const uint32_t v = x32[i];
-            const float sc = __int_as_float((127 + sh.xn[c] - s) << 23);
-            const float f0 = __uint_as_float(v << 16) * sc, f1 = __uint_as_float(v & 0xffff0000u) * sc;
-            const __half2 h2 = __floats2half2_rn(f0, f1);
-            const int step = k >> 4, rr = k & 15;
-            *(__half2*)(xh + (ci * p.T + c) * p.x_stride + (step * 4 + ((rr & 7) >> 1)) * 8 + (rr >> 3) * 4) = h2;
-            float sum = (__low2float(h2) + __high2float(h2)) * __int_as_float((127 + s) << 23);
-#pragma unroll
-            for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(hmask, sum, o);
-            if (l16 == 0) sx[(ci * p.T + c) * moe_sxs(p.H) + (k >> 5)] = sum;
+        for (int c = 0; c < p.T; ++c) {
+            const int xn = sh.xn[c];
+            uint8_t* dst = xh + (ci * p.T + c) * p.x_stride;
+            for (int j0 = sid - lane; j0 < per_col; j0 += nthr) {
+                const int j = j0 + lane;
+                float sum = 0.f;
+                if (j < per_col) {
+                    const int step = j >> 2, tt = j & 3;
+                    const uint32_t* src = x32 + (size_t)c * hp + step * 8 + tt;
+                    const uint32_t v0 = __ldg(src), v1 = __ldg(src + 4);
+                    const int sb = s_pos(fmt, step * 16, p.H);
+                    const float sc = __int_as_float((127 + xn - sb) << 23);
+                    const __half2 h0 = __floats2half2_rn(__uint_as_float(v0 << 16) * sc, __uint_as_float(v0 & 0xffff0000u) * sc);
+                    const __half2 h1 = __floats2half2_rn(__uint_as_float(v1 << 16) * sc, __uint_as_float(v1 & 0xffff0000u) * sc);
+                    uint2 o;
+                    o.x = *reinterpret_cast<const uint32_t*>(&h0);
+                    o.y = *reinterpret_cast<const uint32_t*>(&h1);
+                    *reinterpret_cast<uint2*>(dst + (step * 4 + tt) * 8) = o;
+                    sum = ((__low2float(h0) + __high2float(h0)) + (__low2float(h1) + __high2float(h1))) *
+                          __int_as_float((127 + sb) << 23);
+                }
+                // the 8 items of a block are 8 consecutive lanes
+                sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+                sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+                sum += __shfl_xor_sync(0xffffffffu, sum, 4);
+                if ((lane & 7) == 0 && j < per_col) sx[(ci * p.T + c) * sxs + (j >> 3)] = sum;
+            }
         }
     }
 }
 
+template <int QC>
 __global__ void __launch_bounds__(NTHREADS, 1) moe_decode_kernel(MoeParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -723,10 +778,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_decode_kernel(MoeParams p) {
         for (int s = 0; s < p.ns; ++s) {
             mbar_init(&sh.full[s], 1);
             mbar_init(&sh.empty[s], NCW);
-        }
-        for (int i = 0; i < QN; ++i) {
-            mbar_init(&sh.tqf[i], 1);
-            mbar_init(&sh.tqe[i], NCW);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sh.hfull[i], 1);
@@ -744,34 +795,26 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_decode_kernel(MoeParams p) {
         sh.abort_flag = 0;
         sh.consumed = 0;
         for (int c = 0; c < MOE_MAXT; ++c) sh.xmax[c] = 0u;
-        mbar_init(&sh.xload, 1);
         fence_barrier_init();
     }
     __syncthreads();
-    // x: one bulk copy into the stage ring (free until the main loop) when it
-    // fits and is 16-byte aligned, else read straight from global memory
-    const uint32_t xbytes = (uint32_t)(p.T * p.H * 2);
-    const bool xbulk = xbytes <= (uint32_t)(p.ns * MOE_STAGE_BYTES) && (((uintptr_t)p.x & 15u) == 0);
-    if (xbulk && threadIdx.x == 0) {
-        mbar_arrive_expect_tx(&sh.xload, xbytes);
-        bulk_g2s(ring, p.x, xbytes, &sh.xload, policy_evict_last());
-    }
+    // The producer warp derives the slot table and starts streaming weights at
+    // once; every other warp stages x meanwhile, then waits for the table.
     if (w == WARP_PRODUCER) {
         build_slots(p, sh.st);
-    } else if (w < NCW) {
-        if (xbulk && !mbar_wait(&sh.xload, 0, WAIT_LIMIT)) set_error(p.ctrl, MOE_ERR_TIMEOUT);
-        stage_x(p, sh, xh, xbulk ? (const uint32_t*)ring : (const uint32_t*)p.x);
-    }
-    if (w == WARP_PRODUCER + 1 && xbulk) (void)mbar_wait(&sh.xload, 0, WAIT_LIMIT);   // copy landed before reuse
-    __syncthreads();
-    if (w == WARP_PRODUCER) {
-        const int lane = threadIdx.x & 31;
-        if (lane == 0) producer(p, sh, ring);
-        else if (lane == 1) h_loader(p, sh, xh, hbytes_max, sstr);
-    } else if (w >= WARP_EPILOGUE0) {
-        epilogue_warp(p, sh, red, w - WARP_EPILOGUE0, sstr);
+        asm volatile("bar.arrive 2, %0;" ::"n"(NTHREADS) : "memory");
+        if ((threadIdx.x & 31) == 0) producer(p, sh, ring);
     } else {
-        consumer(p, sh, ring, xh, hbytes_max, red, sstr);
+        const int sid = w < WARP_PRODUCER ? threadIdx.x : threadIdx.x - 32;
+        stage_x(p, sh, xh, sid, NTHREADS - 32);
+        asm volatile("bar.sync 2, %0;" ::"n"(NTHREADS) : "memory");
+        if (w == WARP_HLOAD) {
+            if ((threadIdx.x & 31) == 0) h_loader(p, sh, xh, hbytes_max, sstr);
+        } else if (w >= WARP_EPILOGUE0) {
+            epilogue_warp(p, sh, red, w - WARP_EPILOGUE0, sstr);
+        } else {
+            consumer<QC>(p, sh, ring, xh, hbytes_max, red, sstr);
+        }
     }
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -794,17 +837,20 @@ size_t moe_decode_smem_bytes(int ns, int nred, int xh_bytes) {
 
 cudaError_t moe_decode_launch(const MoeParams& p, int grid, cudaStream_t stream) {
     const size_t smem = moe_decode_smem_bytes(p.ns, p.nred, p.xh_bytes);
-    auto kern = moe_decode_kernel;
+    // q-class: one live column per lane (T = 1), two (T <= 4), two n-blocks of
+    // the down projection's virtual columns (T <= 8)
+    auto kern = p.T == 1 ? moe_decode_kernel<1> : (p.T <= 4 ? moe_decode_kernel<2> : moe_decode_kernel<3>);
     // raise the dynamic shared-memory limit once (not a stream operation, so
     // it stays out of any graph capture after the first call)
-    static int set_bytes[64] = {0};
+    static int set_bytes[64][3] = {{0}};
+    const int qc = p.T == 1 ? 0 : (p.T <= 4 ? 1 : 2);
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
-    if (dev < 64 && set_bytes[dev] < (int)smem) {
+    if (dev >= 64 || set_bytes[dev][qc] < (int)smem) {
         err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (err != cudaSuccess) return err;
-        set_bytes[dev] = (int)smem;
+        if (dev < 64) set_bytes[dev][qc] = (int)smem;
     }
     kern<<<grid, NTHREADS, smem, stream>>>(p);
     return cudaGetLastError();
