@@ -191,6 +191,8 @@ int moe_prepare(const moe_layer* layer, const void* x, int T, const int32_t* idx
     p.hbuf = (uint16_t*)(wsb + L.h_off);
     p.dpart = (float*)(wsb + L.d_off);
     p.x_stride = d.H / 16 * 32 + 32;
+    // one region holds the staged x (gate/up phase: one copy per gate/up
+    // format in use, and its block sums), then two h buffers (down phase)
     const int nxc = (d.has_shared && d.f_sh_gate != d.f_gate) ? 2 : 1;
     const size_t xb = (size_t)nxc * T * p.x_stride + (size_t)nxc * T * moe_sxs(d.H) * 4;
     const size_t hb = 2 * (size_t)4 * T * (d.I + moe_sstr(d.I));
@@ -198,7 +200,7 @@ int moe_prepare(const moe_layer* layer, const void* x, int T, const int32_t* idx
     // deepest ring first (memory in flight), then as many reduction buffers as fit
     p.ns = 0;
     p.nred = 0;
-    for (int ns = 4; ns >= 2 && !p.ns; --ns)
+    for (int ns = MOE_MAX_STAGES; ns >= 2 && !p.ns; --ns)
         for (int nr = MOE_MAX_RED; nr >= 4; --nr)
             if (moe_decode_smem_bytes(ns, nr, p.xh_bytes) <= (size_t)smem_optin) { p.ns = ns; p.nred = nr; break; }
     if (!p.ns) return rfx_fail(RFX_EUNSUPPORTED, "moe_ffn_forward: shapes need more shared memory than the device has");

@@ -1,5 +1,5 @@
 // moe_decode.cu -- MoE FFN decode / speculative-verify step on packed
-// ROCmFPX-style experts, one persistent kernel per layer.
+// ROCmFPX-style experts: one persistent kernel per layer.
 //
 // What it computes (sources by page title and section):
 //  - ainomam.com, "APU 实现 token 自由…", section "Lucebox 的优化三板斧":
@@ -16,22 +16,25 @@
 //  - Grouping: every CTA derives the union of routed experts over the T
 //    columns (the "slots") from idx, so each expert is streamed once for all
 //    the columns routed to it; slot 0 is the shared expert (all columns).
-//  - Tasks: A = (slot, 32 gate/up rows) -> SwiGLU -> h; B = (slot, 32 down
-//    rows) -> partial d.  Tasks are handed out by a global atomic counter, A
-//    before B, so a B task only ever waits on A tasks already running.
-//  - Per CTA: one lane of the producer warp streams packed spans of 8 chunks
-//    HBM -> shared memory with 1-D bulk copies (TMA, evict-first L2 policy)
-//    into a ring of stages; one lane of the h warp bulk-copies the SwiGLU
-//    output h of a slot once all of its gate/up rows are published.  8 consumer warps take one
-//    chunk of every stage each, decode it in registers (one AND per A
-//    register, see rfx_tile.cuh) and run mma.sync m16n8k16 in fp16: x
-//    normalised per column by a power of two for gate/up, an exact hi/lo fp16
-//    split of h for down.  2 epilogue warps sum the 8 warps' partials of
-//    each row-group in a fixed order and run SwiGLU or the combine, so the
-//    consumers never wait on global-memory latency.
-//  - Combine: the last down task to finish a 16-row group sums the slots'
-//    partials in a fixed order (routing order j, then shared), so y does not
-//    depend on scheduling and column t is bitwise the same for any T.
+//  - One persistent kernel, one CTA per SM, three phases: (A) gate/up
+//    row-groups -> SwiGLU -> h of every slot, (B) down row-groups -> per-slot
+//    partial outputs, (C) fixed-order weighted combine -> y.  Each CTA owns a
+//    contiguous, cost-balanced range of 16-row groups in A and in B
+//    (slot-major, so a CTA's row-groups share an x column set or an h
+//    buffer).  The phases meet at two grid barriers (one release-add and one
+//    acquire poll per CTA each); the weight stream does not stop at the
+//    first one: the producer runs straight on into the down weights, only
+//    the copy of h waits for it.
+//  - Per CTA: one lane of the producer warp streams spans of 8 chunks HBM ->
+//    shared memory with 1-D bulk copies (TMA, evict-first L2 policy) into a
+//    ring of stages, each with a record of what it holds (8 gate + 8 up
+//    chunks, or two down row-groups of up to 8 chunks).  8 consumer warps
+//    take one chunk of each half of every stage, decode it in registers (one
+//    AND per A register, see rfx_tile.cuh) and run mma.sync m16n8k16 in fp16:
+//    x normalised per column by a power of two for gate/up, an exact hi/lo
+//    fp16 split of h for down.  2 epilogue warps sum the 8 warps' partials of
+//    each row-group in a fixed order and run SwiGLU (A) or store the partial
+//    (B), then run the combine (C).
 //  - Every wait is bounded; a timeout sets a workspace error flag and the CTA
 //    drains its in-flight copies and exits.
 #include <cuda_runtime.h>
@@ -43,146 +46,213 @@ namespace rfx {
 
 constexpr int NCW = 8;                       // consumer warps 0..7
 constexpr int WARP_PRODUCER = NCW;           // weight bulk copies (one lane)
-constexpr int WARP_HLOAD = NCW + 1;          // h bulk copies of the down tasks (one lane)
-constexpr int NEPI = 2;                      // epilogue warps: reductions, SwiGLU, combine
+constexpr int WARP_HLOAD = NCW + 1;          // first grid barrier, then h bulk copies (one lane)
+constexpr int NEPI = 2;                      // epilogue warps: reductions, SwiGLU / partial stores, combine
 constexpr int WARP_EPILOGUE0 = NCW + 2;
 constexpr int NTHREADS = (NCW + 2 + NEPI) * 32;
-constexpr int QN = 4;
-constexpr int NRED_MAX = MOE_MAX_RED;        // reduction buffers: unit r -> buffer r % p.nred,
+constexpr int NRED_MAX = MOE_MAX_RED;        // reduction buffers: unit r -> buffer r % nred,
                                              // epilogue warp r % NEPI
 constexpr long long WAIT_LIMIT = 4000000000LL;
 
-struct SlotTable {
+struct __align__(16) SlotTable {
+    float w[MOE_MAXT][MOE_MAXK];              // routing weights
+    signed char tslot[MOE_MAXT][MOE_MAXK];    // slot of (column, j), -1 if invalid
+    signed char tpos[MOE_MAXT][MOE_MAXK];     // position of the column among the slot's columns
     int nslots;
-    int expert[MOE_MAXS];
+    int expert[MOE_MAXS];                     // -1: shared expert
     int ncols[MOE_MAXS];
+    unsigned colmask[MOE_MAXS];               // columns routed to the slot (bit c)
     signed char cols[MOE_MAXS][MOE_MAXT];
-    signed char tslot[MOE_MAXT][MOE_MAXK];
-    signed char tpos[MOE_MAXT][MOE_MAXK];
-    float w[MOE_MAXT][MOE_MAXK];
-    unsigned mask[32];
+    unsigned mask[32];                        // experts in use (bit per expert)
     int prefix[32];
     int idx[MOE_MAXT * MOE_MAXK];
-    unsigned char ok[MOE_MAXT * MOE_MAXK];
 };
 
+// A reduction unit: a row-group's partials from the 8 consumer warps, or a
+// marker (end of the gate/up phase, end of work).
+enum : int { UNIT_A = 0, UNIT_B = 1, UNIT_A_END = 2, UNIT_END = 3 };
 struct RedInfo {
-    int kind;      // 0: gate/up row-group, 1: down row-group, -1: end of work
-    int slot, ncols, rg, last_of_task;
+    int kind, slot, ncols, rg;
 };
 
 // What a ring stage holds, written by the producer with the stage.
-enum : short { REC_FIRST = 1, REC_LAST = 2, REC_TFIRST = 4, REC_TLAST = 8 };
+enum : short { REC_FIRST = 1, REC_LAST = 2, REC_HNEW = 4, REC_HDONE = 8, REC_END = 16 };
 struct __align__(16) StageRec {
-    short kind;    // 0: gate/up span, 1: down span, -1: end of work (no copy)
+    short kind;    // 0: gate + up span, 1: down span(s)
     short slot;
-    short rg;      // row-group of the matrix (rows 16*rg ..)
+    short rg;      // row-group of the matrix (rows 16*rg ..); down: first of n
     short c0;      // first chunk of the span
-    short flags;   // REC_*: first / last span of the row-group, of the task
-    short pad[3];
+    short n;       // down: row-groups in the stage (one per half)
+    short flags;   // REC_*: first / last span of the row-group(s); first / last stage of a slot's h
+    short hseq;    // down: index of the slot in this CTA's range (h buffer hseq & 1)
+    short pad;
 };
 
 struct Shared {
     uint64_t full[MOE_MAX_STAGES];
     uint64_t empty[MOE_MAX_STAGES];
     uint64_t hfull[2], hfree[2];
-    uint64_t xfree;
     uint64_t rfull[NRED_MAX], rempty[NRED_MAX];
-    uint64_t hqf[QN], hqe[QN];
-    int hq[QN];
-    StageRec rec[MOE_MAX_STAGES];
+    uint64_t adone;          // both epilogue warps are past the gate/up phase
     RedInfo rinfo[NRED_MAX];
+    StageRec rec[MOE_MAX_STAGES];
     volatile int abort_flag;
     volatile int consumed;   // stages released by all consumer warps (for the abort drain)
+    int bar_ok;              // second grid barrier passed (epilogue warps)
+    int ua0, ua1, ub0, ub1;  // this CTA's row-groups in the two phases
     unsigned xmax[MOE_MAXT]; // max |x| per column (fp32 bits)
     int xn[MOE_MAXT];        // x is staged as x * 2^xn[c] (then 2^-s_b per tile position)
     SlotTable st;
 };
 
-struct Task {
-    int kind, slot, rb;
-};
-
-__device__ __forceinline__ Task decode_task(int t, int nslots, int nrbA, int nrbB) {
-    const int nA = nslots * nrbA;
-    if (t < nA) return {0, t / nrbA, t % nrbA};
-    t -= nA;
-    return {1, t / nrbB, t % nrbB};
-}
-
 __device__ __forceinline__ void set_error(uint32_t* ctrl, uint32_t bits) { atomicOr(ctrl + MOE_CTRL_ERR, bits); }
 
-__device__ void build_slots(const MoeParams& p, SlotTable& S) {
+// The routing of the T columns, loaded by the producer warp's lanes before
+// anything else (lane L holds entries L and L + 32 of idx / w).
+struct Routing {
+    int e0, e1;
+    float w0, w1;
+};
+
+__device__ __forceinline__ Routing load_routing(const MoeParams& p) {
     const int lane = threadIdx.x & 31;
     const int n = p.T * p.k;
-    // one coalesced read of the routing into shared memory, then work from there
-    for (int i = lane; i < n; i += 32) {
-        S.idx[i] = p.idx[i];
-        S.w[i / p.k][i % p.k] = p.wts[i];
-    }
-    S.mask[lane] = 0u;
-    __syncwarp();
-    for (int i = lane; i < n; i += 32) {
-        const int c = i / p.k, j = i % p.k;
-        const int e = S.idx[i];
-        bool ok = e >= 0 && e < p.E;
-        if (!ok) set_error(p.ctrl, MOE_ERR_EXPERT);
-        for (int jj = 0; jj < j && ok; ++jj)
-            if (S.idx[c * p.k + jj] == e) { ok = false; set_error(p.ctrl, MOE_ERR_DUP); }
-        S.ok[i] = ok ? 1 : 0;
-        S.tslot[c][j] = -1;
-        if (ok) atomicOr(&S.mask[e >> 5], 1u << (e & 31));
-    }
-    __syncwarp();
+    Routing r{-1, -1, 0.f, 0.f};
+    if (lane < n) { r.e0 = __ldg(p.idx + lane); r.w0 = __ldg(p.wts + lane); }
+    if (lane + 32 < n) { r.e1 = __ldg(p.idx + lane + 32); r.w1 = __ldg(p.wts + lane + 32); }
+    return r;
+}
+
+// Union of routed experts over the T columns for T * k <= 32 (one warp, one
+// entry per lane, no loops): slot 0 is the shared expert (if any), then the
+// distinct valid experts in order of first appearance (column-major).
+__device__ void build_slots_small(const MoeParams& p, SlotTable& S, const Routing& rt) {
+    const int lane = threadIdx.x & 31;
+    const unsigned lt = (1u << lane) - 1u;
+    const int n = p.T * p.k;
     const int base = p.has_shared ? 1 : 0;
+    const int c = lane / p.k, j = lane - c * p.k;
+    const int e = rt.e0;
+    const bool in = lane < n;
+    bool v = in && e >= 0 && e < p.E;
+    if (in && !v) set_error(p.ctrl, MOE_ERR_EXPERT);
+    // an expert repeated within a column counts once (the later entries are flagged)
+    const unsigned same = __match_any_sync(0xffffffffu, v ? e : -1 - lane);
+    const unsigned col_lanes = ((1u << p.k) - 1u) << (c * p.k);
+    if (v && (same & lt & col_lanes)) {
+        v = false;
+        set_error(p.ctrl, MOE_ERR_DUP);
+    }
+    const unsigned grp = __match_any_sync(0xffffffffu, v ? e : -1 - lane);   // valid entries of the same expert
+    const bool first = v && !(grp & lt);
+    const unsigned firsts = __ballot_sync(0xffffffffu, first);
+    int slot = base + __popc(firsts & lt);
+    slot = __shfl_sync(0xffffffffu, slot, __ffs(grp) - 1);
+    const int pos = __popc(grp & lt);            // earlier columns of this expert
+    if (in) {
+        S.w[c][j] = rt.w0;
+        S.tslot[c][j] = v ? (signed char)slot : (signed char)-1;
+        S.tpos[c][j] = (signed char)pos;
+    }
+    if (v) S.cols[slot][pos] = (signed char)c;
+    if (first) {
+        S.expert[slot] = e;
+        S.ncols[slot] = __popc(grp);
+    }
+    if (lane == 0) {
+        S.nslots = base + __popc(firsts);
+        if (p.has_shared) {
+            S.expert[0] = -1;
+            S.ncols[0] = p.T;
+            for (int cc = 0; cc < p.T; ++cc) S.cols[0][cc] = (signed char)cc;
+        }
+    }
+    __syncwarp();
+}
+
+// Union of routed experts over the T columns (one warp), any T * k <= 64:
+// slot 0 is the shared expert (if any), then the distinct valid experts in
+// ascending order.
+__device__ void build_slots(const MoeParams& p, SlotTable& S, const Routing& rt) {
+    const int lane = threadIdx.x & 31;
+    const int n = p.T * p.k;
+    const int base = p.has_shared ? 1 : 0;
+    S.mask[lane] = 0u;
+    for (int s = lane; s < MOE_MAXS; s += 32) S.colmask[s] = 0u;
+    if (lane < n) { S.idx[lane] = rt.e0; S.w[lane / p.k][lane % p.k] = rt.w0; }
+    if (lane + 32 < n) { S.idx[lane + 32] = rt.e1; S.w[(lane + 32) / p.k][(lane + 32) % p.k] = rt.w1; }
+    __syncwarp();
+    bool ok[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int i = lane + 32 * h;
+        ok[h] = false;
+        if (i >= n) continue;
+        const int c = i / p.k, j = i - (i / p.k) * p.k;
+        const int e = S.idx[i];
+        bool v = e >= 0 && e < p.E;
+        if (!v) set_error(p.ctrl, MOE_ERR_EXPERT);
+        for (int jj = 0; jj < j && v; ++jj)
+            if (S.idx[c * p.k + jj] == e) { v = false; set_error(p.ctrl, MOE_ERR_DUP); }
+        ok[h] = v;
+        S.tslot[c][j] = -1;
+        if (v) atomicOr(&S.mask[e >> 5], 1u << (e & 31));
+    }
+    __syncwarp();
     {
-        int pc = __popc(S.mask[lane]);
+        const int pc = __popc(S.mask[lane]);
         int incl = pc;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            int v = __shfl_up_sync(0xffffffffu, incl, o);
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
             if (lane >= o) incl += v;
         }
         S.prefix[lane] = incl - pc;
         if (lane == 31) S.nslots = base + incl;
     }
-    for (int s = lane; s < MOE_MAXS; s += 32) S.ncols[s] = 0;
     __syncwarp();
-    for (int i = lane; i < n; i += 32) {
-        if (!S.ok[i]) continue;
-        const int c = i / p.k, j = i % p.k;
+    int slot_of[2] = {-1, -1};
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        if (!ok[h]) continue;
+        const int i = lane + 32 * h;
         const int e = S.idx[i];
         const int s = base + S.prefix[e >> 5] + __popc(S.mask[e >> 5] & ((1u << (e & 31)) - 1u));
-        // position of column c among the columns routing to e (columns ascend);
-        // each earlier column counts once even if it repeats e (flagged above)
-        int pos = 0;
-        for (int c2 = 0; c2 < c; ++c2) {
-            for (int j2 = 0; j2 < p.k; ++j2)
-                if (S.idx[c2 * p.k + j2] == e) { ++pos; break; }
-        }
+        slot_of[h] = s;
         S.expert[s] = e;
+        atomicOr(&S.colmask[s], 1u << (i / p.k));
+    }
+    __syncwarp();
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        if (slot_of[h] < 0) continue;
+        const int i = lane + 32 * h;
+        const int c = i / p.k, j = i - c * p.k, s = slot_of[h];
+        const unsigned cm = S.colmask[s];
+        const int pos = __popc(cm & ((1u << c) - 1u));   // columns ascend within a slot
         S.cols[s][pos] = (signed char)c;
         S.tslot[c][j] = (signed char)s;
         S.tpos[c][j] = (signed char)pos;
-        atomicAdd(&S.ncols[s], 1);
+        if (pos == 0) S.ncols[s] = __popc(cm);
     }
     if (p.has_shared && lane == 0) {
         S.expert[0] = -1;
         S.ncols[0] = p.T;
+        S.colmask[0] = (1u << p.T) - 1u;
         for (int c = 0; c < p.T; ++c) S.cols[0][c] = (signed char)c;
     }
     __syncwarp();
 }
 
-// Packed stream of the A (gate, up) or B (down) matrix of a slot.
+// Packed stream of the gate/up (phase 0) or down (phase 1) matrices of a slot.
 struct MatRef {
     const uint8_t* a;
     const uint8_t* b;
     int fmt;
 };
 
-__device__ __forceinline__ MatRef slot_mats(const MoeParams& p, int e, int kind) {
-    if (kind == 0) {
+__device__ __forceinline__ MatRef slot_mats(const MoeParams& p, int e, int ph) {
+    if (ph == 0) {
         if (e < 0) return {p.shg, p.shu, p.fsA};
         return {p.gate + (long long)e * p.sg, p.up + (long long)e * p.su, p.fA};
     }
@@ -190,145 +260,219 @@ __device__ __forceinline__ MatRef slot_mats(const MoeParams& p, int e, int kind)
     return {p.down + (long long)e * p.sd, nullptr, p.fB};
 }
 
+// ------------------------------------------------------------ partition ---
+//
+// Row-groups ("units") are numbered slot-major: u = slot * nrg + rg.  All
+// units of a phase have the same number of tiles; their cost depends on the
+// format only, so a phase has two unit costs: the shared expert's (slot 0,
+// if any) and the routed experts'.  CTA b owns the units whose starting cost
+// in that order lies in [total * b / G, total * (b+1) / G).  The per-format
+// costs are the measured decode + mma cycles per tile of this implementation
+// (relative units).
+
+__device__ __forceinline__ int fmt_cost(int ph, int fmt) {
+    if (ph == 0) return fmt == 2 ? 59 : (fmt == 3 ? 70 : 79);
+    return fmt == 2 ? 70 : (fmt == 3 ? 81 : 94);
+}
+
+__device__ void cta_units(const MoeParams& p, int nslots, int ph, int nrg, int& u0, int& u1) {
+    const int ns = p.has_shared ? 1 : 0, nr = nslots - ns;
+    const int cs = fmt_cost(ph, ph == 0 ? p.fsA : p.fsB), cr = fmt_cost(ph, ph == 0 ? p.fA : p.fB);
+    const long long shared_total = (long long)ns * nrg * cs;
+    const long long total = shared_total + (long long)nr * nrg * cr;
+    auto unit_at = [&](long long target) -> int {   // first unit whose starting cost is >= target
+        if (target < shared_total) return (int)((target + cs - 1) / cs);
+        const long long k = (target - shared_total + cr - 1) / cr;
+        return ns * nrg + (int)min(k, (long long)nr * nrg);
+    };
+    u0 = unit_at(total * blockIdx.x / gridDim.x);
+    u1 = unit_at(total * (blockIdx.x + 1) / gridDim.x);
+}
+
 // ------------------------------------------------------------- producer ---
 //
-// Per task (32 rows = 2 row-groups) and per row-group, one stage per span of
-// up to 8 chunks: a single bulk copy per matrix of the contiguous span.  The
-// stage record (what the stage holds) is written before the arrive that
-// publishes the stage, so a consumer reads it after its acquire on `full`.
+// Gate/up: per row-group, one stage per span of up to 8 chunks (one bulk copy
+// of the span per matrix, gate in the first half of the stage, up in the
+// second).  Down: when a row-group fits one half (at most 8 chunks), a stage
+// holds two consecutive row-groups of a slot, else spans of 8 chunks.  The
+// stage record is written before the arrive that publishes the stage, so a
+// consumer reads it after its acquire on `full`.
+
+struct ProdRing {
+    int stage = 0, n = 0;
+    uint32_t phase = 1;   // producer: parity to wait for on empty[stage] (fresh barriers pass)
+};
+
+__device__ __forceinline__ bool claim(const MoeParams& p, Shared& sh, ProdRing& rg) {
+    return mbar_wait(&sh.empty[rg.stage], rg.phase, WAIT_LIMIT);
+}
+
+__device__ __forceinline__ void advance(const MoeParams& p, ProdRing& rg) {
+    ++rg.n;
+    if (++rg.stage == p.ns) { rg.stage = 0; rg.phase ^= 1u; }
+}
 
 __device__ void producer(const MoeParams& p, Shared& sh, uint8_t* ring) {
     const SlotTable& S = sh.st;
-    const int nrbA = p.I / 32, nrbB = p.H / 32;
-    const int ntasks = S.nslots * (nrbA + nrbB);
     const uint64_t pol_w = policy_evict_first();
-    int stage = 0;
-    uint32_t ephase = 1;          // parity to wait for on empty[stage] (fresh barriers pass)
-    int sc = 0;
+    ProdRing q;
     bool ok = true;
-    int next = (int)atomicAdd(p.ctrl + MOE_CTRL_TASK, 1u);
-    int hi = 0;
-    uint32_t hphase = 1;
-    while (ok) {
-        const int t = next;
-        if (t >= ntasks) break;
-        next = (int)atomicAdd(p.ctrl + MOE_CTRL_TASK, 1u);   // used next iteration: latency hidden
-        const Task tk = decode_task(t, S.nslots, nrbA, nrbB);
-        if (tk.kind == 1) {
-            // hand the h copy of this down task to the h lane
-            if (!mbar_wait(&sh.hqe[hi], hphase, WAIT_LIMIT)) { ok = false; break; }
-            sh.hq[hi] = tk.slot;
-            mbar_arrive(&sh.hqf[hi]);
-            if (++hi == QN) { hi = 0; hphase ^= 1u; }
-        }
-        const int e = S.expert[tk.slot];
-        const MatRef m = slot_mats(p, e, tk.kind);
-        const int K = tk.kind == 0 ? p.H : p.I;
-        const int nch = rfx_num_chunks(K);
-        const long long rgb = rfx_rowgroup_bytes(m.fmt, K);
-        const int fullb = (int)rfx_chunk_bytes(m.fmt, 8);
-        const uint32_t lastb = (uint32_t)rfx_chunk_bytes(m.fmt, rfx_chunk_tiles(K, nch - 1));
-        const uint8_t* srcA = m.a + (long long)(2 * tk.rb) * rgb;
-        const uint8_t* srcB = tk.kind == 0 ? m.b + (long long)(2 * tk.rb) * rgb : nullptr;
-        for (int rgl = 0; rgl < 2 && ok; ++rgl) {
+    // ---- gate/up
+    {
+        const int nrg = p.I / 16, nch = rfx_num_chunks(p.H);
+        for (int u = sh.ua0; u < sh.ua1 && ok; ++u) {
+            const int slot = u / nrg, rg = u - slot * nrg;
+            const MatRef m = slot_mats(p, S.expert[slot], 0);
+            const long long rgb = rfx_rowgroup_bytes(m.fmt, p.H);
+            const int fullb = (int)rfx_chunk_bytes(m.fmt, 8);
+            const uint32_t lastb = (uint32_t)rfx_chunk_bytes(m.fmt, rfx_chunk_tiles(p.H, nch - 1));
             for (int c0 = 0; c0 < nch; c0 += MOE_CHUNKS_PER_STAGE) {
                 const int c1 = min(nch, c0 + MOE_CHUNKS_PER_STAGE);
                 const uint32_t bytes = (uint32_t)((c1 - 1 - c0) * fullb) + (c1 == nch ? lastb : (uint32_t)fullb);
-                if (!mbar_wait(&sh.empty[stage], ephase, WAIT_LIMIT)) { ok = false; break; }
+                if (!claim(p, sh, q)) { ok = false; break; }
                 StageRec r{};
-                r.kind = (short)tk.kind;
-                r.slot = (short)tk.slot;
-                r.rg = (short)(2 * tk.rb + rgl);
+                r.kind = 0;
+                r.slot = (short)slot;
+                r.rg = (short)rg;
                 r.c0 = (short)c0;
-                r.flags = (short)((c0 == 0 ? REC_FIRST : 0) | (c1 == nch ? REC_LAST : 0) |
-                                  (rgl == 0 && c0 == 0 ? REC_TFIRST : 0) | (rgl == 1 && c1 == nch ? REC_TLAST : 0));
-                sh.rec[stage] = r;
-                uint8_t* dst = ring + stage * MOE_STAGE_BYTES;
-                const long long off = (long long)rgl * rgb + (long long)c0 * fullb;
-                if (tk.kind == 0) {
-                    mbar_arrive_expect_tx(&sh.full[stage], 2 * bytes);
-                    bulk_g2s(dst, srcA + off, bytes, &sh.full[stage], pol_w);
-                    bulk_g2s(dst + MOE_HALF_BYTES, srcB + off, bytes, &sh.full[stage], pol_w);
-                } else {
-                    mbar_arrive_expect_tx(&sh.full[stage], bytes);
-                    bulk_g2s(dst, srcA + off, bytes, &sh.full[stage], pol_w);
+                r.n = 1;
+                r.flags = (short)((c0 == 0 ? REC_FIRST : 0) | (c1 == nch ? REC_LAST : 0));
+                sh.rec[q.stage] = r;
+                uint8_t* dst = ring + q.stage * MOE_STAGE_BYTES;
+                const long long off = (long long)rg * rgb + (long long)c0 * fullb;
+                mbar_arrive_expect_tx(&sh.full[q.stage], 2 * bytes);
+                bulk_g2s(dst, m.a + off, bytes, &sh.full[q.stage], pol_w);
+                bulk_g2s(dst + MOE_HALF_BYTES, m.b + off, bytes, &sh.full[q.stage], pol_w);
+                advance(p, q);
+            }
+        }
+    }
+    // ---- down (needs nothing of the gate/up phase: no barrier here)
+    {
+        const int nrg = p.H / 16, nch = rfx_num_chunks(p.I);
+        int hseq = -1, prev_slot = -1;
+        for (int u = sh.ub0; u < sh.ub1 && ok;) {
+            const int slot = u / nrg, rg = u - slot * nrg;
+            if (slot != prev_slot) { ++hseq; prev_slot = slot; }
+            const MatRef m = slot_mats(p, S.expert[slot], 1);
+            const long long rgb = rfx_rowgroup_bytes(m.fmt, p.I);
+            const int fullb = (int)rfx_chunk_bytes(m.fmt, 8);
+            const uint32_t lastb = (uint32_t)rfx_chunk_bytes(m.fmt, rfx_chunk_tiles(p.I, nch - 1));
+            const bool hnew = (u == sh.ub0) || rg == 0;
+            if (nch <= MOE_CHUNKS_PER_STAGE) {
+                const int pair = (u + 1 < sh.ub1 && (u + 1) / nrg == slot) ? 2 : 1;
+                const int ul = u + pair - 1;
+                const bool hdone = (ul + 1 == sh.ub1) || ((ul + 1) / nrg != slot);
+                const uint32_t bytes = (uint32_t)rgb;
+                if (!claim(p, sh, q)) { ok = false; break; }
+                StageRec r{};
+                r.kind = 1;
+                r.slot = (short)slot;
+                r.rg = (short)rg;
+                r.c0 = 0;
+                r.n = (short)pair;
+                r.flags = (short)(REC_FIRST | REC_LAST | (hnew ? REC_HNEW : 0) | (hdone ? REC_HDONE : 0));
+                r.hseq = (short)hseq;
+                sh.rec[q.stage] = r;
+                uint8_t* dst = ring + q.stage * MOE_STAGE_BYTES;
+                mbar_arrive_expect_tx(&sh.full[q.stage], (uint32_t)pair * bytes);
+                for (int i = 0; i < pair; ++i)
+                    bulk_g2s(dst + i * MOE_HALF_BYTES, m.a + (long long)(rg + i) * rgb, bytes, &sh.full[q.stage], pol_w);
+                advance(p, q);
+                u += pair;
+            } else {
+                const bool hdone = (u + 1 == sh.ub1) || ((u + 1) / nrg != slot);
+                for (int c0 = 0; c0 < nch; c0 += MOE_CHUNKS_PER_STAGE) {
+                    const int c1 = min(nch, c0 + MOE_CHUNKS_PER_STAGE);
+                    const uint32_t bytes = (uint32_t)((c1 - 1 - c0) * fullb) + (c1 == nch ? lastb : (uint32_t)fullb);
+                    if (!claim(p, sh, q)) { ok = false; break; }
+                    StageRec r{};
+                    r.kind = 1;
+                    r.slot = (short)slot;
+                    r.rg = (short)rg;
+                    r.c0 = (short)c0;
+                    r.n = 1;
+                    r.flags = (short)((c0 == 0 ? REC_FIRST : 0) | (c1 == nch ? REC_LAST : 0) |
+                                      (c0 == 0 && hnew ? REC_HNEW : 0) | (c1 == nch && hdone ? REC_HDONE : 0));
+                    r.hseq = (short)hseq;
+                    sh.rec[q.stage] = r;
+                    uint8_t* dst = ring + q.stage * MOE_STAGE_BYTES;
+                    mbar_arrive_expect_tx(&sh.full[q.stage], bytes);
+                    bulk_g2s(dst, m.a + (long long)rg * rgb + (long long)c0 * fullb, bytes, &sh.full[q.stage], pol_w);
+                    advance(p, q);
                 }
-                ++sc;
-                if (++stage == p.ns) { stage = 0; ephase ^= 1u; }
+                ++u;
             }
         }
     }
     // end-of-work record: a stage with no copy
     if (ok) {
-        if (mbar_wait(&sh.empty[stage], ephase, WAIT_LIMIT)) {
+        if (claim(p, sh, q)) {
             StageRec r{};
             r.kind = -1;
-            sh.rec[stage] = r;
-            mbar_arrive(&sh.full[stage]);
+            r.flags = REC_END;
+            sh.rec[q.stage] = r;
+            mbar_arrive(&sh.full[q.stage]);
         } else {
             ok = false;
         }
-    }
-    // stop the h lane
-    if (mbar_wait(&sh.hqe[hi], hphase, WAIT_LIMIT)) {
-        sh.hq[hi] = -1;
-        mbar_arrive(&sh.hqf[hi]);
-    } else {
-        ok = false;
     }
     if (!ok) {
         set_error(p.ctrl, MOE_ERR_TIMEOUT);
         sh.abort_flag = 1;
         // drain: wait (bounded) until every issued copy has landed
-        for (int i = sh.consumed; i < sc; ++i) (void)mbar_wait(&sh.full[i % p.ns], (i / p.ns) & 1, WAIT_LIMIT);
+        for (int i = sh.consumed; i < q.n; ++i) (void)mbar_wait(&sh.full[i % p.ns], (i / p.ns) & 1, WAIT_LIMIT);
     }
 }
 
-// The h lane: for each down task, in order, wait until every gate/up
-// row-group of its slot is published, then bulk-copy the slot's h and its
-// block sums (and nothing of the weight stream waits on this).
+// ----------------------------------------------------------- grid barrier ---
+//
+// One thread per CTA: a release add on a 64-bit counter that only grows, then
+// an acquire poll until every CTA of this launch has added.  The target is the
+// next multiple of the grid size above the value this CTA saw, so the counter
+// needs no reset between calls (a timed-out call leaves it unaligned: the
+// workspace must then be re-initialised).  Returns false on timeout.
+__device__ bool grid_barrier(unsigned long long* ctr) {
+    const unsigned long long G = gridDim.x;
+    const unsigned long long old = atom_add_release_gpu_u64(ctr, 1ull);
+    const unsigned long long target = (old / G + 1) * G;
+    const long long t0 = clock64();
+    unsigned nap = 32;
+    while (ld_acquire_gpu_u64(ctr) < target) {
+        if (clock64() - t0 > WAIT_LIMIT) return false;
+        __nanosleep(nap);
+        nap = min(nap * 2u, 256u);
+    }
+    return true;
+}
+
+// The h lane: once every CTA has written its h (first grid barrier), for
+// each slot of the CTA's down range, in order, bulk-copy the slot's h and
+// block sums into buffer (slot index & 1) once the consumers released it.
 __device__ void h_loader(const MoeParams& p, Shared& sh, uint8_t* xh, int hbytes_max, int sstr) {
     const SlotTable& S = sh.st;
-    const uint64_t pol_h = policy_evict_last();
-    const uint32_t need = (uint32_t)(p.I / 16);
-    int hi = 0;
-    uint32_t hphase = 0;
-    int bseq = 0;
-    uint32_t known_ready[3] = {0u, 0u, 0u};   // slots already seen complete (bit per slot)
-    bool ok = true;
-    while (true) {
-        if (!mbar_wait(&sh.hqf[hi], hphase, WAIT_LIMIT)) { ok = false; break; }
-        const int slot = sh.hq[hi];
-        mbar_arrive(&sh.hqe[hi]);
-        if (++hi == QN) { hi = 0; hphase ^= 1u; }
-        if (slot < 0) break;
-        if (bseq == 0 && !mbar_wait(&sh.xfree, 0, WAIT_LIMIT)) { ok = false; break; }
-        const int buf = bseq & 1;
-        if (!mbar_wait(&sh.hfree[buf], ((bseq >> 1) + 1) & 1, WAIT_LIMIT)) { ok = false; break; }
-        if (!(known_ready[slot >> 5] >> (slot & 31) & 1u)) {
-            const long long t0 = clock64();
-            unsigned nap = 32;
-            while (ld_relaxed_gpu(p.ctrl + MOE_CTRL_SLOT + slot) < need) {
-                if (clock64() - t0 > WAIT_LIMIT) { ok = false; break; }
-                __nanosleep(nap);
-                nap = min(nap * 2u, 256u);
-            }
-            if (!ok) break;
-            known_ready[slot >> 5] |= 1u << (slot & 31);
+    bool ok = mbar_wait(&sh.adone, 0, WAIT_LIMIT) &&
+                    grid_barrier(reinterpret_cast<unsigned long long*>(p.ctrl + MOE_CTRL_BAR_H));
+    int n = 0;
+    if (ok && sh.ub0 < sh.ub1) {
+        fence_proxy_async_global();   // generic-proxy writes of h (other CTAs) -> bulk-copy reads
+        const uint64_t pol_h = policy_evict_last();
+        const int nrg = p.H / 16;
+        const int s0 = sh.ub0 / nrg, s1 = (sh.ub1 - 1) / nrg;
+        for (int slot = s0; slot <= s1; ++slot, ++n) {
+            const int buf = n & 1;
+            if (!mbar_wait(&sh.hfree[buf], ((n >> 1) + 1) & 1, WAIT_LIMIT)) { ok = false; break; }
+            const uint32_t hb = 4u * (uint32_t)S.ncols[slot] * (uint32_t)(p.I + sstr);
+            mbar_arrive_expect_tx(&sh.hfull[buf], hb);
+            bulk_g2s(xh + buf * hbytes_max, p.hbuf + (long long)slot * (2LL * p.T * (p.I + sstr)), hb,
+                     &sh.hfull[buf], pol_h);
         }
-        fence_acq_rel_gpu();          // acquire side of the publishers' release
-        fence_proxy_async_global();   // generic-proxy writes of h -> bulk-copy (async proxy) reads
-        const uint32_t hb = 4u * (uint32_t)S.ncols[slot] * (uint32_t)(p.I + sstr);
-        mbar_arrive_expect_tx(&sh.hfull[buf], hb);
-        bulk_g2s(xh + buf * hbytes_max, p.hbuf + (long long)slot * (2LL * p.T * (p.I + sstr)), hb, &sh.hfull[buf],
-                 pol_h);
-        ++bseq;
     }
     if (!ok) {
         set_error(p.ctrl, MOE_ERR_TIMEOUT);
         sh.abort_flag = 1;
-        for (int b = 0; b < 2 && b < bseq; ++b)
-            (void)mbar_wait(&sh.hfull[(bseq - 1 - b) & 1], ((bseq - 1 - b) >> 1) & 1, WAIT_LIMIT);
+        for (int b = 0; b < 2 && b < n; ++b)
+            (void)mbar_wait(&sh.hfull[(n - 1 - b) & 1], ((n - 1 - b) >> 1) & 1, WAIT_LIMIT);
     }
 }
 
@@ -382,10 +526,8 @@ __device__ void epilogue_a(const MoeParams& p, const Shared& sh, const float* rb
     if (__any_sync(0xffffffffu, bad) && lane == 0) set_error(p.ctrl, MOE_ERR_RANGE);
 }
 
-// Partial down output of one row-group -> dpart; the last slot to finish the
-// row-group sums all slots' partials in a fixed order into y.
-__device__ void epilogue_b(const MoeParams& p, const SlotTable& S, const float* rb0, int slot, int ncols, int rg,
-                           int lane) {
+// Partial down output of one row-group of one slot -> dpart[slot][col][rows].
+__device__ void epilogue_b(const MoeParams& p, const float* rb0, int slot, int ncols, int rg, int lane) {
     const int g = lane >> 2, t = lane & 3;
     float* dp = p.dpart + (long long)slot * p.T * p.H;
     float D[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -404,55 +546,63 @@ __device__ void epilogue_b(const MoeParams& p, const SlotTable& S, const float* 
             dp[(long long)col * p.H + row0 + 8] = D[4 * nb + 2] + D[4 * nb + 3];
         }
     }
-    // warp barrier, then one release/acquire atomic for the whole warp's stores
-    __syncwarp();
-    uint32_t prev = 0;
-    if (lane == 0) prev = atom_add_acq_rel_gpu(p.ctrl + MOE_CTRL_ROWBLK + rg, 1u);
-    prev = __shfl_sync(0xffffffffu, prev, 0);
-    if (prev != (uint32_t)S.nslots - 1) return;
-    __syncwarp();   // lane 0's acquire orders the other lanes' reads of dpart below
-    for (int it = lane; it < 16 * p.T; it += 32) {
-        const int row = 16 * rg + (it & 15), c = it >> 4;
-        float acc = 0.f;
-        for (int j = 0; j < p.k; ++j) {
-            const int s2 = S.tslot[c][j];
-            if (s2 < 0) continue;
-            const float v = __ldcg(p.dpart + ((long long)s2 * p.T + S.tpos[c][j]) * p.H + row);
-            acc = fmaf(S.w[c][j], v, acc);
-        }
-        if (p.has_shared) acc += __ldcg(p.dpart + (long long)c * p.H + row);
-        p.y[(long long)c * p.H + row] = acc;
-    }
-    __syncwarp();
-    if (lane == 0) p.ctrl[MOE_CTRL_ROWBLK + rg] = 0u;
 }
 
 // An epilogue warp: units r = e, e + NEPI, ... in the order the consumers
-// deposit them; the 8 warps' partials are summed in warp order.
+// deposit them; the 8 warps' partials are summed in warp order.  After the
+// last unit: the second grid barrier, then this CTA's slice of the combine.
 __device__ void epilogue_warp(const MoeParams& p, Shared& sh, float* red, int e, int sstr) {
     const int lane = threadIdx.x & 31;
+    bool ok = true;
     for (int r = e;; r += NEPI) {
         const int b = r % p.nred;
         const uint32_t ph = (uint32_t)(r / p.nred) & 1u;
-        if (!mbar_wait(&sh.rfull[b], ph, WAIT_LIMIT)) {
+        if (!mbar_wait(&sh.rfull[b], ph, WAIT_LIMIT)) { ok = false; break; }
+        const RedInfo ri = sh.rinfo[b];
+        if (ri.kind == UNIT_END) break;
+        const float* rb0 = red + b * NCW * 32 * 8;
+        if (ri.kind == UNIT_A) epilogue_a(p, sh, rb0, ri.slot, ri.ncols, ri.rg, lane, sstr);
+        else if (ri.kind == UNIT_B) epilogue_b(p, rb0, ri.slot, ri.ncols, ri.rg, lane);
+        __syncwarp();
+        if (lane == 0) {
+            mbar_arrive(&sh.rempty[b]);
+            if (ri.kind == UNIT_A_END) mbar_arrive(&sh.adone);   // this warp's h stores are all issued
+        }
+    }
+    // every partial of this CTA is stored; wait for all CTAs' (second barrier)
+    asm volatile("bar.sync 3, %0;" ::"n"(NEPI * 32) : "memory");
+    int& bar_ok = sh.bar_ok;
+    if (e == 0 && lane == 0)
+        bar_ok = ok && !sh.abort_flag && grid_barrier(reinterpret_cast<unsigned long long*>(p.ctrl + MOE_CTRL_BAR_D));
+    asm volatile("bar.sync 3, %0;" ::"n"(NEPI * 32) : "memory");
+    if (!bar_ok) {
+        if (e == 0 && lane == 0) {
             set_error(p.ctrl, MOE_ERR_TIMEOUT);
             sh.abort_flag = 1;
-            break;
         }
-        const RedInfo ri = sh.rinfo[b];
-        if (ri.kind < 0) break;
-        const float* rb0 = red + b * NCW * 32 * 8;
-        if (ri.kind == 0) {
-            epilogue_a(p, sh, rb0, ri.slot, ri.ncols, ri.rg, lane, sstr);
-            // this row-group of h is complete: publish it to the down tasks
-            // (the bulk-copy reader fences the async proxy after its acquire)
-            __syncwarp();
-            if (lane == 0) red_add_release_gpu(p.ctrl + MOE_CTRL_SLOT + ri.slot, 1u);
-        } else {
-            epilogue_b(p, sh.st, rb0, ri.slot, ri.ncols, ri.rg, lane);
+        return;
+    }
+    // combine: y[c] = sum_j w[c][j] * partial[slot(c, j)] + partial[shared], in
+    // the fixed order j = 0 .. k-1 then the shared expert (column c does not
+    // depend on T); this CTA owns elements [n b / G, n (b+1) / G)
+    const SlotTable& S = sh.st;
+    const long long n = (long long)p.T * p.H;
+    const int i0 = (int)(n * blockIdx.x / gridDim.x), i1 = (int)(n * (blockIdx.x + 1) / gridDim.x);
+    for (int i = i0 + e * 32 + lane; i < i1; i += NEPI * 32) {
+        const int c = i / p.H, r = i - c * p.H;
+        float v[MOE_MAXK];
+#pragma unroll
+        for (int j = 0; j < MOE_MAXK; ++j) {
+            const int s2 = j < p.k ? S.tslot[c][j] : -1;
+            v[j] = s2 >= 0 ? __ldcg(p.dpart + ((long long)s2 * p.T + S.tpos[c][j]) * p.H + r) : 0.f;
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sh.rempty[b]);
+        const float vs = p.has_shared ? __ldcg(p.dpart + (long long)c * p.H + r) : 0.f;
+        float acc = 0.f;
+#pragma unroll
+        for (int j = 0; j < MOE_MAXK; ++j)
+            if (j < p.k && S.tslot[c][j] >= 0) acc = fmaf(S.w[c][j], v[j], acc);
+        if (p.has_shared) acc += vs;
+        p.y[i] = acc;
     }
 }
 
@@ -464,7 +614,7 @@ struct RedCursor {
 };
 
 // Deposit this warp's partials for the next reduction unit.
-__device__ __forceinline__ bool red_deposit(const MoeParams& p, Shared& sh, float* red, RedCursor& rc, int w, int lane,
+__device__ __forceinline__ bool red_deposit(Shared& sh, int nred, float* red, RedCursor& rc, int w, int lane,
                                             const float v[8], const RedInfo& info) {
     if (!mbar_wait(&sh.rempty[rc.b], rc.ph ^ 1u, WAIT_LIMIT)) return false;
     float* my = red + ((rc.b * NCW + w) * 32 + lane) * 8;
@@ -473,7 +623,7 @@ __device__ __forceinline__ bool red_deposit(const MoeParams& p, Shared& sh, floa
     if (w == 0 && lane == 0) sh.rinfo[rc.b] = info;
     __syncwarp();
     if (lane == 0) mbar_arrive(&sh.rfull[rc.b]);
-    if (++rc.b == p.nred) { rc.b = 0; rc.ph ^= 1u; }
+    if (++rc.b == nred) { rc.b = 0; rc.ph ^= 1u; }
     return true;
 }
 
@@ -486,19 +636,6 @@ __device__ __forceinline__ int s_pos(int fmt, int k, int K) {
     return fmt == 2 ? Plane<2>::s_of(b) : (fmt == 3 ? Plane<3>::s_of(b) : Plane<4>::s_of(b));
 }
 
-// Ring position of a consumer warp.
-struct Ring {
-    int stage = 0, cc = 0;
-    uint32_t fphase = 0;
-    __device__ __forceinline__ void release(const MoeParams& p, Shared& sh, int w, int lane) {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sh.empty[stage]);
-        ++cc;
-        if (w == 0 && lane == 0) sh.consumed = cc;
-        if (++stage == p.ns) { stage = 0; fphase ^= 1u; }
-    }
-};
-
 __device__ __forceinline__ void ld8(const float* src, float d[8]) {
     const float4 a = ldsf4((const uint8_t*)src), b = ldsf4((const uint8_t*)(src + 4));
     d[0] = a.x; d[1] = a.y; d[2] = a.z; d[3] = a.w;
@@ -506,8 +643,8 @@ __device__ __forceinline__ void ld8(const float* src, float d[8]) {
 }
 
 // One gate/up chunk pair (chunk c of the stage's span, this warp's share).
-template <int FMT, bool TWO>
-__device__ __forceinline__ void stepA(const uint8_t* st, int c, int H, int lane, int g, const BSrc& bs, const float* sA0,
+template <int FMT, bool TWO, class SRC>
+__device__ __forceinline__ void stepA(const uint8_t* st, int c, int H, int lane, int g, const SRC& bs, const float* sA0,
                                       const float* sA1, AccA& ag, AccA& au) {
     const int nt = rfx_chunk_tiles(H, c);
     if (nt == 8) {
@@ -521,8 +658,8 @@ __device__ __forceinline__ void stepA(const uint8_t* st, int c, int H, int lane,
 }
 
 // One down chunk.
-template <int FMT, int NB>
-__device__ __forceinline__ void stepB(const uint8_t* st, int c, int I, int lane, int g, int t, const BSrc* bs,
+template <int FMT, int NB, class SRC>
+__device__ __forceinline__ void stepB(const uint8_t* st, int c, int I, int lane, int g, int t, const SRC* bs,
                                       const float* hsum, int ncols, int sstr, AccB<NB>& ab) {
     const int nt = rfx_chunk_tiles(I, c);
     if (nt == 8) {
@@ -547,14 +684,39 @@ __device__ __forceinline__ void stepB(const uint8_t* st, int c, int I, int lane,
 
 __device__ __forceinline__ int full_chunk_bytes(int fmt) { return 128 * rfx_block_bytes(fmt); }
 
-// Consumer warp: one flat loop over the ring.  Every CTA's stream holds all of
-// its gate/up spans before its down spans (tasks are handed out A first), so
-// the two phases are two loops with their own accumulators.
-template <int QC>
-__device__ void consumer(const MoeParams& p, Shared& sh, uint8_t* ring, uint8_t* xh, int hbytes_max, float* red,
-                         int sstr) {
-    constexpr bool TWO = QC >= 2;           // a second live column per lane in the gate/up output
-    constexpr int NB = QC >= 3 ? 2 : 1;     // n-blocks of virtual (hi, lo) columns in the down projection
+// A consumer warp's ring cursor.
+struct ConsRing {
+    int stage = 0, cc = 0;
+    uint32_t phase = 0;
+};
+
+__device__ __forceinline__ void cons_release(const MoeParams& p, Shared& sh, ConsRing& rp, int w, int lane) {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sh.empty[rp.stage]);
+    ++rp.cc;
+    if (w == 0 && lane == 0) sh.consumed = rp.cc;
+    if (++rp.stage == p.ns) { rp.stage = 0; rp.phase ^= 1u; }
+}
+
+__device__ __forceinline__ bool cons_next(Shared& sh, ConsRing& rp, StageRec& r) {
+    if (!mbar_wait(&sh.full[rp.stage], rp.phase, WAIT_LIMIT)) return false;
+    r = sh.rec[rp.stage];
+    return true;
+}
+
+__device__ __forceinline__ int fmt_a(const MoeParams& p, const SlotTable& S, int slot) {
+    return S.expert[slot] < 0 ? p.fsA : p.fA;
+}
+__device__ __forceinline__ int fmt_b(const MoeParams& p, const SlotTable& S, int slot) {
+    return S.expert[slot] < 0 ? p.fsB : p.fB;
+}
+
+// Gate/up stages of one format, from the current record r (first span of a
+// row-group) while the records stay gate/up spans of that format; returns with
+// the next record in r.
+template <int FMT, bool TWO>
+__device__ __forceinline__ bool loop_a(const MoeParams& p, Shared& sh, uint8_t* ring, uint8_t* xh, float* red, ConsRing& rp,
+                       RedCursor& rc, StageRec& r) {
     const SlotTable& S = sh.st;
     const int w = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -562,131 +724,150 @@ __device__ void consumer(const MoeParams& p, Shared& sh, uint8_t* ring, uint8_t*
     const int nxc = (p.has_shared && p.fsA != p.fA) ? 2 : 1;
     const float* sx = (const float*)(xh + nxc * p.T * p.x_stride);   // [copy][col][sxs]
     const int sxs = moe_sxs(p.H);
-    const int nchA = rfx_num_chunks(p.H), nchB = rfx_num_chunks(p.I);
-    Ring ring_pos;
-    RedCursor rc;
-    bool ok = true;
-    StageRec r{};
-    // ---- gate/up spans -> SwiGLU partials
-    {
-        AccA ag, au;
-        ag.zero();
-        au.zero();
-        BSrc bs{xh, 0, false};
-        const float* sA0 = sx;
-        const float* sA1 = sx;
-        int slot = 0, ncols = 0, fmt = 2;
-        while (true) {
-            if (!mbar_wait(&sh.full[ring_pos.stage], ring_pos.fphase, WAIT_LIMIT)) { ok = false; break; }
-            r = sh.rec[ring_pos.stage];
-            if (r.kind != 0) break;
-            if (r.flags & REC_FIRST) {
-                slot = r.slot;
-                const int e = S.expert[slot];
-                ncols = S.ncols[slot];
-                fmt = e < 0 ? p.fsA : p.fA;
-                const int ci = (e < 0 && nxc == 2) ? 1 : 0;
-                const int col0 = g < ncols ? S.cols[slot][g] : 0;
-                bs = BSrc{xh + (ci * p.T + col0) * p.x_stride + t * 8, 32, g < ncols};
-                const int c0 = 2 * t < ncols ? S.cols[slot][2 * t] : 0;
-                const int c1 = 2 * t + 1 < ncols ? S.cols[slot][2 * t + 1] : 0;
-                sA0 = sx + (ci * p.T + c0) * sxs;
-                sA1 = sx + (ci * p.T + c1) * sxs;
-                ag.zero();
-                au.zero();
-            }
-            const int c = r.c0 + w;
-            if (c < nchA) {
-                const uint8_t* st = ring + ring_pos.stage * MOE_STAGE_BYTES + w * full_chunk_bytes(fmt);
-                if (fmt == 2) stepA<2, TWO>(st, c, p.H, lane, g, bs, sA0, sA1, ag, au);
-                else if (fmt == 3) stepA<3, TWO>(st, c, p.H, lane, g, bs, sA0, sA1, ag, au);
-                else stepA<4, TWO>(st, c, p.H, lane, g, bs, sA0, sA1, ag, au);
-            }
-            ring_pos.release(p, sh, w, lane);
-            if (r.flags & REC_LAST) {
-                float v[8];
-                if (fmt == 2) { finishA<2>(ag, v); finishA<2>(au, v + 4); }
-                else if (fmt == 3) { finishA<3>(ag, v); finishA<3>(au, v + 4); }
-                else { finishA<4>(ag, v); finishA<4>(au, v + 4); }
-                const RedInfo info{0, slot, ncols, r.rg, (r.flags & REC_TLAST) ? 1 : 0};
-                if (!red_deposit(p, sh, red, rc, w, lane, v, info)) { ok = false; break; }
-            }
+    const int nch = rfx_num_chunks(p.H);
+    constexpr int FULLB = 128 * (FMT * 4 + (FMT == 4 ? 1 : 2));
+    AccA ag, au;
+    BSrcK<32> bs{xh, 0};
+    const float* sA0 = sx;
+    const float* sA1 = sx;
+    int slot = 0, ncols = 1;
+    while (true) {
+        if (r.flags & REC_FIRST) {
+            slot = r.slot;
+            ncols = S.ncols[slot];
+            const int ci = (S.expert[slot] < 0 && nxc == 2) ? 1 : 0;
+            const int colg = S.cols[slot][g < ncols ? g : 0];
+            bs.base = xh + (ci * p.T + colg) * p.x_stride + t * 8;
+            const int c0 = S.cols[slot][2 * t < ncols ? 2 * t : 0];
+            const int c1 = S.cols[slot][2 * t + 1 < ncols ? 2 * t + 1 : 0];
+            sA0 = sx + (ci * p.T + c0) * sxs;
+            sA1 = sx + (ci * p.T + c1) * sxs;
+            ag.zero();
+            au.zero();
         }
+        const int c = r.c0 + w;
+        if (c < nch) stepA<FMT, TWO>(ring + rp.stage * MOE_STAGE_BYTES + w * FULLB, c, p.H, lane, g, bs, sA0, sA1, ag, au);
+        cons_release(p, sh, rp, w, lane);
+        if (r.flags & REC_LAST) {
+            float v[8];
+            finishA<FMT>(ag, v);
+            finishA<FMT>(au, v + 4);
+            if (!red_deposit(sh, p.nred, red, rc, w, lane, v, RedInfo{UNIT_A, slot, ncols, r.rg})) return false;
+        }
+        if (!cons_next(sh, rp, r)) return false;
+        if (r.kind != 0 || ((r.flags & REC_FIRST) && fmt_a(p, S, r.slot) != FMT)) return true;
     }
-    // ---- down spans -> partial outputs
-    if (ok && r.kind == 1) {
-        // the staged x is no longer read: the h lane may overwrite it
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sh.xfree);
-        AccB<NB> ab;
-        ab.zero();
-        BSrc bs[NB];
+}
+
+// Down stages of one format (one or two row-groups per stage, see the
+// producer), from the current record r while the records stay down spans of
+// that format; returns with the next record in r.
+template <int FMT, int NB, int HSTRIDE>
+__device__ __forceinline__ bool loop_b(const MoeParams& p, Shared& sh, uint8_t* ring, uint8_t* xh, int hbytes_max, float* red, int sstr,
+                       ConsRing& rp, RedCursor& rc, StageRec& r) {
+    const SlotTable& S = sh.st;
+    const int w = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int nch = rfx_num_chunks(p.I);
+    constexpr int FULLB = 128 * (FMT * 4 + (FMT == 4 ? 1 : 2));
+    AccB<NB> ab;
+    BSrcK<HSTRIDE> bs[NB];
+    const float* hsum = (const float*)xh;
+    int slot = -1, hseq = -1, ncols = 1;
+    while (true) {
+        const int buf_h = r.hseq & 1;
+        if (r.flags & REC_HNEW) {
+            if (!mbar_wait(&sh.hfull[buf_h], (r.hseq >> 1) & 1, WAIT_LIMIT)) return false;
+        }
+        if (r.slot != slot || r.hseq != hseq) {
+            slot = r.slot;
+            hseq = r.hseq;
+            ncols = S.ncols[slot];
+            const uint8_t* hs = xh + buf_h * hbytes_max;
+            const int vst = 64 * ncols;  // bytes per k16 step
 #pragma unroll
-        for (int nb = 0; nb < NB; ++nb) bs[nb] = BSrc{xh, 0, false};
-        const float* hsum = (const float*)xh;
-        int bseq = 0, slot = 0, ncols = 0, fmt = 3;
-        while (true) {
-            const int buf_h = bseq & 1;
-            if (r.flags & REC_TFIRST) {
-                if (!mbar_wait(&sh.hfull[buf_h], (bseq >> 1) & 1, WAIT_LIMIT)) { ok = false; break; }
+            for (int nb = 0; nb < NB; ++nb) {
+                const int vv = min(8 * nb + g, 2 * ncols - 1);
+                bs[nb] = BSrcK<HSTRIDE>{hs + (vv * 4 + t) * 8, vst};
             }
-            if (r.flags & REC_FIRST) {
-                slot = r.slot;
-                const int e = S.expert[slot];
-                ncols = S.ncols[slot];
-                fmt = e < 0 ? p.fsB : p.fB;
-                const uint8_t* hs = xh + buf_h * hbytes_max;
-                const int vst = 64 * ncols;  // bytes per k16 step
+            hsum = (const float*)(hs + 4 * ncols * p.I);
+        }
+        const int c = r.c0 + w;
+        float v[2][8];
 #pragma unroll
-                for (int nb = 0; nb < NB; ++nb) {
-                    const int vv = 8 * nb + g;
-                    bs[nb] = BSrc{hs + (vv * 4 + t) * 8, vst, vv < 2 * ncols};
-                }
-                hsum = (const float*)(hs + 4 * ncols * p.I);
-                ab.zero();
-            }
-            const int c = r.c0 + w;
-            if (c < nchB) {
-                const uint8_t* st = ring + ring_pos.stage * MOE_STAGE_BYTES + w * full_chunk_bytes(fmt);
-                if (fmt == 3) stepB<3, NB>(st, c, p.I, lane, g, t, bs, hsum, ncols, sstr, ab);
-                else if (fmt == 2) stepB<2, NB>(st, c, p.I, lane, g, t, bs, hsum, ncols, sstr, ab);
-                else stepB<4, NB>(st, c, p.I, lane, g, t, bs, hsum, ncols, sstr, ab);
-            }
-            ring_pos.release(p, sh, w, lane);
+        for (int i = 0; i < 2; ++i) {
+            if (i >= r.n) break;
+            if (r.flags & REC_FIRST) ab.zero();
+            if (c < nch)
+                stepB<FMT, NB>(ring + rp.stage * MOE_STAGE_BYTES + i * MOE_HALF_BYTES + w * FULLB, c, p.I, lane, g, t, bs,
+                               hsum, ncols, sstr, ab);
             if (r.flags & REC_LAST) {
                 float vb[NB][4];
-                if (fmt == 3) finishB<3, NB>(ab, vb);
-                else if (fmt == 2) finishB<2, NB>(ab, vb);
-                else finishB<4, NB>(ab, vb);
-                float v[8];
+                finishB<FMT, NB>(ab, vb);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    v[i] = vb[0][i];
-                    v[4 + i] = NB > 1 ? vb[NB - 1][i] : 0.f;
+                for (int k = 0; k < 4; ++k) {
+                    v[i][k] = vb[0][k];
+                    v[i][4 + k] = NB > 1 ? vb[NB - 1][k] : 0.f;
                 }
-                const RedInfo info{1, slot, ncols, r.rg, (r.flags & REC_TLAST) ? 1 : 0};
-                if (!red_deposit(p, sh, red, rc, w, lane, v, info)) { ok = false; break; }
             }
-            if (r.flags & REC_TLAST) {
-                // every span of this down task is consumed: release its h buffer
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sh.hfree[buf_h]);
-                ++bseq;
-            }
-            if (!mbar_wait(&sh.full[ring_pos.stage], ring_pos.fphase, WAIT_LIMIT)) { ok = false; break; }
-            r = sh.rec[ring_pos.stage];
-            if (r.kind != 1) break;
         }
+        cons_release(p, sh, rp, w, lane);
+        if (r.flags & REC_LAST) {
+            if (!red_deposit(sh, p.nred, red, rc, w, lane, v[0], RedInfo{UNIT_B, slot, ncols, r.rg})) return false;
+            if (r.n > 1 && !red_deposit(sh, p.nred, red, rc, w, lane, v[1], RedInfo{UNIT_B, slot, ncols, r.rg + 1}))
+                return false;
+        }
+        if (r.flags & REC_HDONE) {
+            // every stage of this slot is consumed: release its h buffer
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.hfree[buf_h]);
+        }
+        if (!cons_next(sh, rp, r)) return false;
+        if (r.kind != 1 || fmt_b(p, S, r.slot) != FMT) return true;
+    }
+}
+
+// Consumer warp: the records of a CTA's stream are all its gate/up spans, then
+// all its down spans, then the end record.  Each phase runs one loop per
+// format (a CTA's range usually holds one or two formats).
+template <int QC>
+__device__ void consumer(const MoeParams& p, Shared& sh, uint8_t* ring, uint8_t* xh, int hbytes_max, float* red,
+                         int sstr) {
+    constexpr bool TWO = QC >= 2;           // a second live column per lane in the gate/up output
+    constexpr int NB = QC >= 3 ? 2 : 1;     // n-blocks of virtual (hi, lo) columns in the down projection
+    constexpr int HSTRIDE = QC == 1 ? 64 : 0;   // bytes per k16 step of h (one column: 2 virtual x 4 lanes x 8 B)
+    const SlotTable& S = sh.st;
+    const int w = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    ConsRing rp;
+    RedCursor rc;
+    StageRec r{};
+    bool ok = cons_next(sh, rp, r);
+    while (ok && r.kind == 0) {
+        const int f = fmt_a(p, S, r.slot);
+        if (f == 2) ok = loop_a<2, TWO>(p, sh, ring, xh, red, rp, rc, r);
+        else if (f == 3) ok = loop_a<3, TWO>(p, sh, ring, xh, red, rp, rc, r);
+        else ok = loop_a<4, TWO>(p, sh, ring, xh, red, rp, rc, r);
+    }
+    // the staged x is no longer read (the h copies will overwrite it); tell
+    // each epilogue warp that the gate/up phase is over
+    fence_proxy_async_smem();
+    const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int i = 0; i < NEPI && ok; ++i)
+        if (!red_deposit(sh, p.nred, red, rc, w, lane, z, RedInfo{UNIT_A_END, 0, 0, 0})) ok = false;
+    while (ok && r.kind == 1) {
+        const int f = fmt_b(p, S, r.slot);
+        if (f == 3) ok = loop_b<3, NB, HSTRIDE>(p, sh, ring, xh, hbytes_max, red, sstr, rp, rc, r);
+        else if (f == 2) ok = loop_b<2, NB, HSTRIDE>(p, sh, ring, xh, hbytes_max, red, sstr, rp, rc, r);
+        else ok = loop_b<4, NB, HSTRIDE>(p, sh, ring, xh, hbytes_max, red, sstr, rp, rc, r);
     }
     if (!ok) {
         set_error(p.ctrl, MOE_ERR_TIMEOUT);
         sh.abort_flag = 1;
     }
     // one end-of-work unit for each epilogue warp
-    const RedInfo fin{-1, 0, 0, 0, 0};
-    const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int i = 0; i < NEPI; ++i) (void)red_deposit(p, sh, red, rc, w, lane, z, fin);
+    for (int i = 0; i < NEPI; ++i) (void)red_deposit(sh, p.nred, red, rc, w, lane, z, RedInfo{UNIT_END, 0, 0, 0});
 }
 
 // x (bf16 [T][H], global) -> shared memory for the gate/up B operand: per
@@ -762,18 +943,20 @@ __device__ void stage_x(const MoeParams& p, Shared& sh, uint8_t* xh, int sid, in
     }
 }
 
+// ---------------------------------------------------------------- kernel ---
+
 template <int QC>
 __global__ void __launch_bounds__(NTHREADS, 1) moe_decode_kernel(MoeParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    uint8_t* ring = base;
+    uint8_t* ring = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t* xh = ring + p.ns * MOE_STAGE_BYTES;
     float* red = (float*)(xh + p.xh_bytes);
     Shared& sh = *(Shared*)((uint8_t*)red + p.nred * NCW * 32 * 8 * sizeof(float));
     const int sstr = moe_sstr(p.I);
     const int hbytes_max = 4 * p.T * (p.I + sstr);
     const int w = threadIdx.x >> 5;
-
+    Routing rt{};
+    if (w == WARP_PRODUCER) rt = load_routing(p);   // in flight during the barrier set-up
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.ns; ++s) {
             mbar_init(&sh.full[s], 1);
@@ -787,21 +970,22 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_decode_kernel(MoeParams p) {
             mbar_init(&sh.rfull[i], NCW);
             mbar_init(&sh.rempty[i], 1);
         }
-        mbar_init(&sh.xfree, NCW);
-        for (int i = 0; i < QN; ++i) {
-            mbar_init(&sh.hqf[i], 1);
-            mbar_init(&sh.hqe[i], 1);
-        }
+        mbar_init(&sh.adone, NEPI);
         sh.abort_flag = 0;
         sh.consumed = 0;
         for (int c = 0; c < MOE_MAXT; ++c) sh.xmax[c] = 0u;
         fence_barrier_init();
     }
     __syncthreads();
-    // The producer warp derives the slot table and starts streaming weights at
-    // once; every other warp stages x meanwhile, then waits for the table.
+    // The producer warp derives the slot table and its row-groups and starts
+    // streaming weights at once; every other warp stages x meanwhile.
     if (w == WARP_PRODUCER) {
-        build_slots(p, sh.st);
+        if (p.T * p.k <= 32) build_slots_small(p, sh.st, rt);
+        else build_slots(p, sh.st, rt);
+        if ((threadIdx.x & 31) == 0) {
+            cta_units(p, sh.st.nslots, 0, p.I / 16, sh.ua0, sh.ua1);
+            cta_units(p, sh.st.nslots, 1, p.H / 16, sh.ub0, sh.ub1);
+        }
         asm volatile("bar.arrive 2, %0;" ::"n"(NTHREADS) : "memory");
         if ((threadIdx.x & 31) == 0) producer(p, sh, ring);
     } else {
@@ -816,18 +1000,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_decode_kernel(MoeParams p) {
             consumer<QC>(p, sh, ring, xh, hbytes_max, red, sstr);
         }
     }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        const uint32_t prev = atom_add_acq_rel_gpu(p.ctrl + MOE_CTRL_EXIT, 1u);
-        if (prev == gridDim.x - 1) {
-            // last CTA out: reset the counters for the next call on this workspace
-            for (int s = 0; s < sh.st.nslots; ++s) p.ctrl[MOE_CTRL_SLOT + s] = 0u;
-            p.ctrl[MOE_CTRL_TASK] = 0u;
-            __threadfence();
-            p.ctrl[MOE_CTRL_EXIT] = 0u;
-        }
-    }
 }
 
 // Shared-memory bytes of a launch (plus 1 KB alignment slack).
@@ -839,11 +1011,11 @@ cudaError_t moe_decode_launch(const MoeParams& p, int grid, cudaStream_t stream)
     const size_t smem = moe_decode_smem_bytes(p.ns, p.nred, p.xh_bytes);
     // q-class: one live column per lane (T = 1), two (T <= 4), two n-blocks of
     // the down projection's virtual columns (T <= 8)
-    auto kern = p.T == 1 ? moe_decode_kernel<1> : (p.T <= 4 ? moe_decode_kernel<2> : moe_decode_kernel<3>);
-    // raise the dynamic shared-memory limit once (not a stream operation, so
-    // it stays out of any graph capture after the first call)
-    static int set_bytes[64][3] = {{0}};
     const int qc = p.T == 1 ? 0 : (p.T <= 4 ? 1 : 2);
+    auto kern = qc == 0 ? moe_decode_kernel<1> : (qc == 1 ? moe_decode_kernel<2> : moe_decode_kernel<3>);
+    // raise the dynamic shared-memory limit once per device and kernel (not a
+    // stream operation, so it stays out of any graph capture after the first call)
+    static int set_bytes[64][3] = {{0}};
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
@@ -852,8 +1024,19 @@ cudaError_t moe_decode_launch(const MoeParams& p, int grid, cudaStream_t stream)
         if (err != cudaSuccess) return err;
         if (dev < 64) set_bytes[dev][qc] = (int)smem;
     }
-    kern<<<grid, NTHREADS, smem, stream>>>(p);
-    return cudaGetLastError();
+    // cooperative: every CTA is resident at once (the two grid barriers need it)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(NTHREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeCooperative;
+    at[0].val.cooperative = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    err = cudaLaunchKernelEx(&cfg, kern, p);
+    return err;
 }
 
 }  // namespace rfx

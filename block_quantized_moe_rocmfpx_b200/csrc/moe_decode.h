@@ -8,18 +8,18 @@
 #define MOE_MAXT 8            // token columns per call (decode / verify)
 #define MOE_MAXK 8            // routed experts per token
 #define MOE_MAXS (MOE_MAXT * MOE_MAXK + 1)
-#define MOE_MAX_STAGES 6
+#define MOE_MAX_STAGES 8
 #define MOE_MAX_RED 8          // reduction buffers
 #define MOE_CHUNKS_PER_STAGE 8
 #define MOE_HALF_BYTES 17408   // 8 full FP4 chunks of one matrix
-#define MOE_STAGE_BYTES 34816  // gate + up halves
+#define MOE_STAGE_BYTES 34816  // two halves: gate + up, or two down row-groups
 
-// workspace control words (uint32)
-#define MOE_CTRL_TASK 0
-#define MOE_CTRL_EXIT 1
+// workspace control words (uint32 index); the grid-barrier counters are
+// 64-bit and only grow
 #define MOE_CTRL_ERR 2
-#define MOE_CTRL_SLOT 8
-#define MOE_CTRL_ROWBLK (MOE_CTRL_SLOT + MOE_MAXS + 7)
+#define MOE_CTRL_BAR_H 4       // u64: gate/up phase done (h complete)
+#define MOE_CTRL_BAR_D 6       // u64: down phase done (partials complete)
+#define MOE_CTRL_WORDS 64
 
 // device error bits
 #define MOE_ERR_EXPERT 1u
@@ -68,9 +68,8 @@ struct MoeWs {
 inline MoeWs moe_ws_layout(int T, int k, int H, int I) {
     MoeWs L;
     const size_t ns = (size_t)T * k + 1;
-    const size_t ctrl_words = MOE_CTRL_ROWBLK + (size_t)H / 16;
     L.ctrl_off = 0;
-    L.h_off = (ctrl_words * 4 + 255) / 256 * 256;
+    L.h_off = (MOE_CTRL_WORDS * 4 + 255) / 256 * 256;
     L.d_off = L.h_off + (ns * 4 * T * (size_t)(I + moe_sstr(I)) + 255) / 256 * 256;
     L.total = L.d_off + (ns * T * H * 4 + 255) / 256 * 256;
     return L;

@@ -41,6 +41,18 @@ struct BSrc {
     }
 };
 
+// B-operand source with a compile-time step stride (STRIDE > 0) or a run-time
+// one (STRIDE == 0), and no predicate: a lane whose column is empty points at
+// a real column, whose products only reach output columns that are dropped.
+template <int STRIDE>
+struct BSrcK {
+    const uint8_t* base;
+    int stride;
+    __device__ __forceinline__ uint2 get(int step) const {
+        return lds64(base + step * (STRIDE > 0 ? STRIDE : stride));
+    }
+};
+
 // --------------------------------------------------------- plane layout ---
 
 // Shift exponent s_b of tile b of a full chunk (bit offset of its fields after
@@ -162,8 +174,8 @@ __device__ __forceinline__ void mma_tile(float c[4], const uint32_t a[8], uint2 
 // One full gate/up chunk pair sharing the x fragments (x pre-scaled by
 // 2^-s_b): all tiles accumulate in units of 2^-24.  S[b] / S1[b] are the
 // block sums of the lane's two columns; TWO = the second column can be live.
-template <int FMT, bool TWO>
-__device__ __forceinline__ void chunkA_full(const uint8_t* st0, const uint8_t* st1, int lane, int g, const BSrc& bs,
+template <int FMT, bool TWO, class SRC>
+__device__ __forceinline__ void chunkA_full(const uint8_t* st0, const uint8_t* st1, int lane, int g, const SRC& bs,
                                             int step0, const float* S0, const float* S1, AccA& ag, AccA& au) {
     FullChunk<FMT> f0, f1;
     f0.load(st0, lane, g);
@@ -241,8 +253,8 @@ struct AccB {
 
 // One full down chunk (h used as it is; B operands hi/lo split fp16).
 // Sb[n][b] = block sum of h for the lane's real column of n-block n.
-template <int FMT, int NB>
-__device__ __forceinline__ void chunkB_full(const uint8_t* st, int lane, int g, const BSrc* bs, int step0,
+template <int FMT, int NB, class SRC>
+__device__ __forceinline__ void chunkB_full(const uint8_t* st, int lane, int g, const SRC* bs, int step0,
                                             const float (*Sb)[8], AccB<NB>& ab) {
     FullChunk<FMT> f;
     f.load(st, lane, g);
@@ -321,9 +333,9 @@ __device__ __forceinline__ void partial_tile(const uint8_t* st, int nt, int lane
 
 // A partial chunk adds s * (exact level dot product) in units of 2^-24 so that
 // it shares the full chunks' accumulator (no offset correction: levels exact).
-template <int FMT, bool TWO>
+template <int FMT, bool TWO, class SRC>
 __device__ __forceinline__ void chunkA_partial(const uint8_t* st0, const uint8_t* st1, int nt, int lane, int g,
-                                               const BSrc& bs, int step0, AccA& ag, AccA& au) {
+                                               const SRC& bs, int step0, AccA& ag, AccA& au) {
     for (int b = 0; b < nt; ++b) {
         const uint2 blo = bs.get(step0 + 2 * b), bhi = bs.get(step0 + 2 * b + 1);
         uint32_t a[8];
@@ -341,8 +353,8 @@ __device__ __forceinline__ void chunkA_partial(const uint8_t* st0, const uint8_t
     }
 }
 
-template <int FMT, int NB>
-__device__ __forceinline__ void chunkB_partial(const uint8_t* st, int nt, int lane, int g, const BSrc* bs, int step0,
+template <int FMT, int NB, class SRC>
+__device__ __forceinline__ void chunkB_partial(const uint8_t* st, int nt, int lane, int g, const SRC* bs, int step0,
                                                AccB<NB>& ab) {
     for (int b = 0; b < nt; ++b) {
         uint32_t a[8];
