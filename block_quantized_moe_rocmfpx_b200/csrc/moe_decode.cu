@@ -478,6 +478,22 @@ __device__ void h_loader(const MoeParams& p, Shared& sh, uint8_t* xh, int hbytes
 
 // ------------------------------------------------------------- epilogues ---
 
+// A reduction buffer holds the 8 consumer warps' partials of one unit as
+// [warp][half][lane][4 floats]: every 128-bit access of a warp covers 512
+// contiguous bytes (no bank conflicts).  Sums them in warp order.
+__device__ __forceinline__ void red_sum(const float* rb0, int lane, float lo[4], float hi[4]) {
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+#pragma unroll
+    for (int w = 0; w < NCW; ++w) {
+        const float4 x = ldsf4((const uint8_t*)(rb0 + ((w * 2 + 0) * 32 + lane) * 4));
+        const float4 y = ldsf4((const uint8_t*)(rb0 + ((w * 2 + 1) * 32 + lane) * 4));
+        a.x += x.x; a.y += x.y; a.z += x.z; a.w += x.w;
+        b.x += y.x; b.y += y.y; b.z += y.z; b.w += y.w;
+    }
+    lo[0] = a.x; lo[1] = a.y; lo[2] = a.z; lo[3] = a.w;
+    hi[0] = b.x; hi[1] = b.y; hi[2] = b.z; hi[3] = b.w;
+}
+
 // SwiGLU of one row-group: undo the per-column x scaling, h = silu(g) * u,
 // store h as an fp16 hi/lo pair in the fragment order of the down projection's
 // B operand ([step][v][t'][4], v = 2*col + {0 hi, 1 lo}) and the row-group's
@@ -487,13 +503,8 @@ __device__ void epilogue_a(const MoeParams& p, const Shared& sh, const float* rb
     const int g = lane >> 2, t = lane & 3;
     uint16_t* hs = p.hbuf + (long long)slot * (2LL * p.T * (p.I + sstr));
     float* hsum = (float*)(hs + 2LL * ncols * p.I);
-    float G[4] = {0.f, 0.f, 0.f, 0.f}, U[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int w = 0; w < NCW; ++w) {
-        const float* r = rb0 + (w * 32 + lane) * 8;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) { G[i] += r[i]; U[i] += r[4 + i]; }
-    }
+    float G[4], U[4];
+    red_sum(rb0, lane, G, U);
     uint32_t bad = 0;
     const int step = rg;
     float part[2] = {0.f, 0.f};
@@ -530,13 +541,8 @@ __device__ void epilogue_a(const MoeParams& p, const Shared& sh, const float* rb
 __device__ void epilogue_b(const MoeParams& p, const float* rb0, int slot, int ncols, int rg, int lane) {
     const int g = lane >> 2, t = lane & 3;
     float* dp = p.dpart + (long long)slot * p.T * p.H;
-    float D[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int w = 0; w < NCW; ++w) {
-        const float* r = rb0 + (w * 32 + lane) * 8;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) D[i] += r[i];
-    }
+    float D[8];
+    red_sum(rb0, lane, D, D + 4);
     const int row0 = 16 * rg + g;
 #pragma unroll
     for (int nb = 0; nb < 2; ++nb) {
@@ -617,9 +623,9 @@ struct RedCursor {
 __device__ __forceinline__ bool red_deposit(Shared& sh, int nred, float* red, RedCursor& rc, int w, int lane,
                                             const float v[8], const RedInfo& info) {
     if (!mbar_wait(&sh.rempty[rc.b], rc.ph ^ 1u, WAIT_LIMIT)) return false;
-    float* my = red + ((rc.b * NCW + w) * 32 + lane) * 8;
+    float* my = red + ((rc.b * NCW + w) * 2 * 32 + lane) * 4;   // [buffer][warp][half][lane][4]
     *reinterpret_cast<float4*>(my) = make_float4(v[0], v[1], v[2], v[3]);
-    *reinterpret_cast<float4*>(my + 4) = make_float4(v[4], v[5], v[6], v[7]);
+    *reinterpret_cast<float4*>(my + 32 * 4) = make_float4(v[4], v[5], v[6], v[7]);
     if (w == 0 && lane == 0) sh.rinfo[rc.b] = info;
     __syncwarp();
     if (lane == 0) mbar_arrive(&sh.rfull[rc.b]);

@@ -72,7 +72,8 @@ __global__ void pack_kernel(int fmt, const uint8_t* __restrict__ codes, const ui
                 }
             }
         }
-        put_bytes(lanep, w, 4 * fmt);
+        // slab-major full chunk: word i of this lane at rfx_full_word_off(lane, i)
+        for (int i = 0; i < 4 * fmt; ++i) put_bytes(chunk + rfx_full_word_off(lane, i), &w[i], 1);
     } else {
         for (int b = 0; b < nt; ++b) {
             const long long k0 = (long long)(8 * j + b) * 32;
@@ -137,7 +138,7 @@ __global__ void pack_kernel(int fmt, const uint8_t* __restrict__ codes, const ui
     for (int i = lane; i < 8 * nt * 2; i += 32) {
         const int gg = i / (2 * nt), b = (i / 2) % nt, h = i & 1;
         const long long row = rg * 16 + gg + 8 * h;
-        uint8_t* d = sc + (long long)i * sb;
+        uint8_t* d = nt == 8 ? sc + rfx_full_scale_off(fmt, gg, b, h) : sc + (long long)i * sb;
         for (int q = 0; q < sb; ++q) d[q] = row < rows ? scales[(row * nb + 8 * j + b) * sb + q] : (uint8_t)0;
     }
 }

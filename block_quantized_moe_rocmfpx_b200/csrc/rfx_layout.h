@@ -45,6 +45,17 @@ RFX_HD int64_t rfx_padded_rows(int64_t N) { return (N + 15) / 16 * 16; }
 RFX_HD int64_t rfx_matrix_bytes(int fmt, int64_t N, int64_t K) {
     return rfx_padded_rows(N) / 16 * rfx_rowgroup_bytes(fmt, K);
 }
+// Full chunks (8 tiles) are stored slab-major so that each 128-bit shared
+// memory load of a warp reads 512 contiguous bytes: code word w (0 .. 4*fmt-1)
+// of lane L sits at byte ((w/4)*32 + L)*16 + (w%4)*4 of the chunk's codes, and
+// the scale of (row g + 8h, tile b) at byte ((b/4)*8 + g)*16 + (b%4)*4 + 2h of
+// its scales (binary16; E8M0 scales are [g][b][h] bytes, already 16 bytes per
+// g).
+RFX_HD int rfx_full_word_off(int lane, int w) { return (((w >> 2) * 32 + lane) << 4) + ((w & 3) << 2); }
+RFX_HD int rfx_full_scale_off(int fmt, int g, int b, int h) {
+    return fmt == 4 ? (g * 8 + b) * 2 + h : (((b >> 2) * 8 + g) << 4) + ((b & 3) << 2) + 2 * h;
+}
+
 // number of chunks of a row-group and tiles in chunk j
 RFX_HD int rfx_num_chunks(int64_t K) { return (int)((K / 32 + 7) / 8); }
 RFX_HD int rfx_chunk_tiles(int64_t K, int j) {

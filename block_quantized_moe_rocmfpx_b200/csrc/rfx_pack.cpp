@@ -88,7 +88,9 @@ void pack_lane_full(int fmt, const TileView* tv, int g, int t, uint8_t* out) {
                 }
             }
         }
-    std::memcpy(out, w, 4 * 4 * fmt);
+    // slab-major: word i of lane L at rfx_full_word_off(L, i) from the chunk start
+    const int L = 4 * g + t;
+    for (int i = 0; i < 4 * fmt; ++i) std::memcpy(out + rfx_full_word_off(L, i), &w[i], 4);
 }
 
 void unpack_lane_full(int fmt, const struct TileOut* to, int g, int t, const uint8_t* in);
@@ -208,7 +210,8 @@ void unpack_lane_fp3_pair(const TileOut& a, const TileOut& b, int g, int t, cons
 
 void unpack_lane_full(int fmt, const TileOut* to, int g, int t, const uint8_t* in) {
     uint32_t w[16];
-    std::memcpy(w, in, 4 * 4 * fmt);
+    const int L = 4 * g + t;
+    for (int i = 0; i < 4 * fmt; ++i) std::memcpy(&w[i], in + rfx_full_word_off(L, i), 4);
     const uint32_t m = (1u << fmt) - 1u;
     for (int b = 0; b < 8; ++b)
         for (int r = 0; r < 8; ++r) {
@@ -282,7 +285,7 @@ extern "C" int rfx_pack(rfx_format f, const uint8_t* codes, const void* scales, 
                 if (nt == 8) {
                     TileView tv[8];
                     for (int b = 0; b < 8; ++b) tv[b] = TileView{codes, rows, cols, rg * 16, (int64_t)(8 * j + b) * 32};
-                    pack_lane_full(f, tv, g, t, lane);
+                    pack_lane_full(f, tv, g, t, chunk);
                 } else if (f == RFX_FP3) {
                     int b = 0;
                     for (; b + 1 < nt; b += 2) {
@@ -307,7 +310,7 @@ extern "C" int rfx_pack(rfx_format f, const uint8_t* codes, const void* scales, 
                     for (int h = 0; h < 2; ++h) {
                         int64_t r = rg * 16 + g + 8 * h;
                         int64_t bi = r * nb + 8 * j + b;
-                        uint8_t* d = sc + ((int64_t)(g * nt + b) * 2 + h) * sb;
+                        uint8_t* d = nt == 8 ? sc + rfx_full_scale_off(f, g, b, h) : sc + ((int64_t)(g * nt + b) * 2 + h) * sb;
                         if (r >= rows) { std::memset(d, 0, sb); continue; }
                         std::memcpy(d, (const uint8_t*)scales + bi * sb, sb);
                     }
@@ -340,7 +343,7 @@ extern "C" int rfx_unpack(rfx_format f, const void* src, int64_t rows, int64_t c
                 if (nt == 8) {
                     TileOut to[8];
                     for (int b = 0; b < 8; ++b) to[b] = TileOut{codes, rows, cols, rg * 16, (int64_t)(8 * j + b) * 32};
-                    unpack_lane_full(f, to, g, t, lane);
+                    unpack_lane_full(f, to, g, t, chunk);
                 } else if (f == RFX_FP3) {
                     int b = 0;
                     for (; b + 1 < nt; b += 2) {
@@ -366,7 +369,8 @@ extern "C" int rfx_unpack(rfx_format f, const void* src, int64_t rows, int64_t c
                         int64_t r = rg * 16 + g + 8 * h;
                         if (r >= rows) continue;
                         int64_t bi = r * nb + 8 * j + b;
-                        std::memcpy((uint8_t*)scales + bi * sb, sc + ((int64_t)(g * nt + b) * 2 + h) * sb, sb);
+                        const uint8_t* d = nt == 8 ? sc + rfx_full_scale_off(f, g, b, h) : sc + ((int64_t)(g * nt + b) * 2 + h) * sb;
+                        std::memcpy((uint8_t*)scales + bi * sb, d, sb);
                     }
         }
     }

@@ -128,16 +128,18 @@ struct FullChunk {
     uint32_t wd[Plane<FMT>::NW];
     uint32_t sh[Plane<FMT>::NW];
     uint32_t sc[Plane<FMT>::NSW];
+    // slab-major chunk (rfx_layout.h): every 128-bit load of the warp reads
+    // 512 contiguous code bytes or 128 contiguous scale bytes
     __device__ __forceinline__ void load(const uint8_t* st, int lane, int g) {
         constexpr int NW = Plane<FMT>::NW, NSW = Plane<FMT>::NSW;
 #pragma unroll
         for (int i = 0; i < NW / 4; ++i) {
-            uint4 v = lds128(st + lane * (NW * 4) + 16 * i);
+            uint4 v = lds128(st + (i * 32 + lane) * 16);
             wd[4 * i] = v.x; wd[4 * i + 1] = v.y; wd[4 * i + 2] = v.z; wd[4 * i + 3] = v.w;
         }
 #pragma unroll
         for (int i = 0; i < NSW / 4; ++i) {
-            uint4 v = lds128(st + Plane<FMT>::CODE_BYTES + g * (NSW * 4) + 16 * i);
+            uint4 v = lds128(st + Plane<FMT>::CODE_BYTES + (i * 8 + g) * 16);
             sc[4 * i] = v.x; sc[4 * i + 1] = v.y; sc[4 * i + 2] = v.z; sc[4 * i + 3] = v.w;
         }
         plane_shift<FMT>(wd, sh);

@@ -44,8 +44,11 @@
  * layout: row-groups of 16 rows (rows padded to a multiple of 16 with zero
  * codes and zero scales), each a contiguous stream of chunks of up to 8 tiles
  * (tile = 16 rows x 1 block).  A chunk of nt tiles holds nt*16*codebytes of
- * codes followed by nt*16*scalebytes of scales.  Codes are lane-major: lane
- * L = 4g+t (g = 0..7, t = 0..3) owns nt*2b bytes at offset L*nt*2b.  Per tile
+ * codes followed by nt*16*scalebytes of scales.  Lane L = 4g+t (g = 0..7,
+ * t = 0..3) owns nt*2b bytes of codes (b = bits per code): in a partial chunk
+ * (nt < 8) at offset L*nt*2b ("lane-major"); in a full chunk as 32-bit words
+ * w = 0 .. 4b-1 with word w at byte ((w/4)*32 + L)*16 + (w%4)*4 ("slab-major",
+ * so each 128-bit load of a warp reads 512 contiguous bytes).  Per tile
  * the lane owns 8 "registers" r = 0..7, each two codes (low, high element):
  *   m = r>>2, j = r&3, row = g + 8*(j&1), k0 = 16m + 2t + 8*(j>>1) inside the
  *   block; low = code[row][k0], high = code[row][k0+1].
@@ -69,7 +72,9 @@
  *        the low code at bit 15 and of the high code at bit 31 of word i.  A
  *        lone last tile (odd nt) is a 48-bit little-endian stream of its 16
  *        codes, code 2r+e (e = 0 low, 1 high) at bits [3(2r+e), +3).
- * Scales of a chunk: [g][tile][row g, row g+8], binary16 or E8M0 bytes.
+ * Scales of a partial chunk: [g][tile][row g, row g+8], binary16 or E8M0
+ * bytes.  Full chunk: E8M0 the same; binary16 the scale of (row g + 8h, tile
+ * b) at byte ((b/4)*8 + g)*16 + (b%4)*4 + 2h.
  */
 #ifndef RFX_H
 #define RFX_H

@@ -90,11 +90,11 @@ def test_layout_matches_header_description():
         c, s = spec.codes(), spec.scales()
         packed = rfx.rfx_pack(fmt, c, s)
         m = (1 << fmt) - 1
-        # full chunk 0: plane layout
-        lane_bytes = 8 * 2 * fmt
+        # full chunk 0: plane layout, slab-major words
         for L in (0, 5, 31):
             g, t = L >> 2, L & 3
-            words = [int(v) for v in np.frombuffer(packed[L * lane_bytes:(L + 1) * lane_bytes].tobytes(), np.uint32)]
+            words = [int(np.frombuffer(packed[((w // 4) * 32 + L) * 16 + (w % 4) * 4:][:4].tobytes(), np.uint32)[0])
+                     for w in range(4 * fmt)]
             for b in range(8):
                 for r in range(8):
                     row, k = _reg_coords(g, t, r)
@@ -136,13 +136,25 @@ def test_layout_matches_header_description():
                         else:       # lone tile 2: 48-bit stream
                             st = int.from_bytes(lane[12:18], "little")
                             assert (st >> (3 * (2 * r))) & 7 == lo and (st >> (3 * (2 * r + 1))) & 7 == hi
-        # scales of the first chunk: [g][tile][row g, row g+8]
+        # scales of the first (full) chunk: E8M0 [g][tile][row g, row g+8] bytes; binary16 at
+        # ((b/4)*8 + g)*16 + (b%4)*4 + 2h
         sb = 1 if fmt == 4 else 2
-        sc = packed[8 * 16 * 4 * fmt: 8 * 16 * 4 * fmt + 8 * 8 * 2 * sb]
-        sc = np.frombuffer(sc.tobytes(), dtype=np.uint8 if fmt == 4 else np.uint16).reshape(8, 8, 2)
+        sc = packed[8 * 16 * 4 * fmt: 8 * 16 * 4 * fmt + 8 * 8 * 2 * sb].tobytes()
         for g in range(8):
             for b in range(8):
-                assert sc[g, b, 0] == s[g, b] and sc[g, b, 1] == s[g + 8, b]
+                for h in range(2):
+                    if fmt == 4:
+                        got = sc[(g * 8 + b) * 2 + h]
+                    else:
+                        o = ((b // 4) * 8 + g) * 16 + (b % 4) * 4 + 2 * h
+                        got = int(np.frombuffer(sc[o:o + 2], np.uint16)[0])
+                    assert got == s[g + 8 * h, b]
+        # scales of the partial chunk 1: [g][tile][row g, row g+8]
+        sc1 = chunk1[nt * 16 * 4 * fmt: nt * 16 * 4 * fmt + 8 * nt * 2 * sb].tobytes()
+        sc1 = np.frombuffer(sc1, dtype=np.uint8 if fmt == 4 else np.uint16).reshape(8, nt, 2)
+        for g in range(8):
+            for b in range(nt):
+                assert sc1[g, b, 0] == s[g, 8 + b] and sc1[g, b, 1] == s[g + 8, 8 + b]
 
 
 def test_pack_rejects_bad_values():
