@@ -94,12 +94,13 @@ struct Shared {
     uint64_t hfull[2], hfree[2];
     uint64_t rfull[NRED_MAX], rempty[NRED_MAX];
     uint64_t adone;          // both epilogue warps are past the gate/up phase
+    uint64_t xload;          // bulk copy of x into the (not yet used) reduction buffers
     RedInfo rinfo[NRED_MAX];
     StageRec rec[MOE_MAX_STAGES];
     volatile int abort_flag;
     volatile int consumed;   // stages released by all consumer warps (for the abort drain)
     int bar_ok;              // second grid barrier passed (epilogue warps)
-    int ua0, ua1, ub0, ub1;  // this CTA's row-groups in the two phases
+    int ub0, ub1;            // this CTA's down row-groups
     unsigned xmax[MOE_MAXT]; // max |x| per column (fp32 bits)
     int xn[MOE_MAXT];        // x is staged as x * 2^xn[c] (then 2^-s_b per tile position)
     SlotTable st;
@@ -262,22 +263,19 @@ __device__ __forceinline__ MatRef slot_mats(const MoeParams& p, int e, int ph) {
 
 // ------------------------------------------------------------ partition ---
 //
-// Row-groups ("units") are numbered slot-major: u = slot * nrg + rg.  All
-// units of a phase have the same number of tiles; their cost depends on the
-// format only, so a phase has two unit costs: the shared expert's (slot 0,
-// if any) and the routed experts'.  CTA b owns the units whose starting cost
-// in that order lies in [total * b / G, total * (b+1) / G).  The per-format
-// costs are the measured decode + mma cycles per tile of this implementation
-// (relative units).
+// Down row-groups ("units") are numbered slot-major: u = slot * nrg + rg.
+// They are split statically (each CTA copies the h of only the one or two
+// slots of its range): CTA b owns the units whose starting cost lies in
+// [total * b / G, total * (b+1) / G).  All units have the same tiles; their
+// cost depends on the format only (measured decode + mma cycles per tile of
+// this implementation, relative units), so there are two unit costs: the
+// shared expert's (slot 0, if any) and the routed experts'.
+__device__ __forceinline__ int down_cost(int fmt) { return fmt == 2 ? 70 : (fmt == 3 ? 81 : 94); }
 
-__device__ __forceinline__ int fmt_cost(int ph, int fmt) {
-    if (ph == 0) return fmt == 2 ? 59 : (fmt == 3 ? 70 : 79);
-    return fmt == 2 ? 70 : (fmt == 3 ? 81 : 94);
-}
-
-__device__ void cta_units(const MoeParams& p, int nslots, int ph, int nrg, int& u0, int& u1) {
+__device__ void down_units(const MoeParams& p, int nslots, int& u0, int& u1) {
+    const int nrg = p.H / 16;
     const int ns = p.has_shared ? 1 : 0, nr = nslots - ns;
-    const int cs = fmt_cost(ph, ph == 0 ? p.fsA : p.fsB), cr = fmt_cost(ph, ph == 0 ? p.fA : p.fB);
+    const int cs = down_cost(p.fsB), cr = down_cost(p.fB);
     const long long shared_total = (long long)ns * nrg * cs;
     const long long total = shared_total + (long long)nr * nrg * cr;
     auto unit_at = [&](long long target) -> int {   // first unit whose starting cost is >= target
@@ -312,6 +310,11 @@ __device__ __forceinline__ void advance(const MoeParams& p, ProdRing& rg) {
     if (++rg.stage == p.ns) { rg.stage = 0; rg.phase ^= 1u; }
 }
 
+// Gate/up row-groups are handed out dynamically (a global counter), one at a
+// time, so CTAs that run faster take more; they are numbered slot-major, the
+// shared expert (the largest units) first, and the next grab is always in
+// flight while the current row-group streams.  Down row-groups come from the
+// CTA's static range.
 __device__ void producer(const MoeParams& p, Shared& sh, uint8_t* ring) {
     const SlotTable& S = sh.st;
     const uint64_t pol_w = policy_evict_first();
@@ -320,7 +323,12 @@ __device__ void producer(const MoeParams& p, Shared& sh, uint8_t* ring) {
     // ---- gate/up
     {
         const int nrg = p.I / 16, nch = rfx_num_chunks(p.H);
-        for (int u = sh.ua0; u < sh.ua1 && ok; ++u) {
+        const int nunits = S.nslots * nrg;
+        int next = (int)atomicAdd(p.ctrl + MOE_CTRL_TASK_A, 1u);
+        while (ok) {
+            const int u = next;
+            if (u >= nunits) break;
+            next = (int)atomicAdd(p.ctrl + MOE_CTRL_TASK_A, 1u);
             const int slot = u / nrg, rg = u - slot * nrg;
             const MatRef m = slot_mats(p, S.expert[slot], 0);
             const long long rgb = rfx_rowgroup_bytes(m.fmt, p.H);
@@ -360,10 +368,10 @@ __device__ void producer(const MoeParams& p, Shared& sh, uint8_t* ring) {
             const uint32_t lastb = (uint32_t)rfx_chunk_bytes(m.fmt, rfx_chunk_tiles(p.I, nch - 1));
             const bool hnew = (u == sh.ub0) || rg == 0;
             if (nch <= MOE_CHUNKS_PER_STAGE) {
+                // one stage holds two consecutive row-groups of the slot (one per half)
                 const int pair = (u + 1 < sh.ub1 && (u + 1) / nrg == slot) ? 2 : 1;
                 const int ul = u + pair - 1;
                 const bool hdone = (ul + 1 == sh.ub1) || ((ul + 1) / nrg != slot);
-                const uint32_t bytes = (uint32_t)rgb;
                 if (!claim(p, sh, q)) { ok = false; break; }
                 StageRec r{};
                 r.kind = 1;
@@ -375,9 +383,10 @@ __device__ void producer(const MoeParams& p, Shared& sh, uint8_t* ring) {
                 r.hseq = (short)hseq;
                 sh.rec[q.stage] = r;
                 uint8_t* dst = ring + q.stage * MOE_STAGE_BYTES;
-                mbar_arrive_expect_tx(&sh.full[q.stage], (uint32_t)pair * bytes);
+                mbar_arrive_expect_tx(&sh.full[q.stage], (uint32_t)(pair * rgb));
                 for (int i = 0; i < pair; ++i)
-                    bulk_g2s(dst + i * MOE_HALF_BYTES, m.a + (long long)(rg + i) * rgb, bytes, &sh.full[q.stage], pol_w);
+                    bulk_g2s(dst + i * MOE_HALF_BYTES, m.a + (long long)(rg + i) * rgb, (uint32_t)rgb, &sh.full[q.stage],
+                             pol_w);
                 advance(p, q);
                 u += pair;
             } else {
@@ -449,10 +458,13 @@ __device__ bool grid_barrier(unsigned long long* ctr) {
 // The h lane: once every CTA has written its h (first grid barrier), for
 // each slot of the CTA's down range, in order, bulk-copy the slot's h and
 // block sums into buffer (slot index & 1) once the consumers released it.
+// CTA 0 also resets the gate/up task counter (every CTA has taken its last
+// gate/up row-group before it arrives).
 __device__ void h_loader(const MoeParams& p, Shared& sh, uint8_t* xh, int hbytes_max, int sstr) {
     const SlotTable& S = sh.st;
     bool ok = mbar_wait(&sh.adone, 0, WAIT_LIMIT) &&
-                    grid_barrier(reinterpret_cast<unsigned long long*>(p.ctrl + MOE_CTRL_BAR_H));
+              grid_barrier(reinterpret_cast<unsigned long long*>(p.ctrl + MOE_CTRL_BAR_H));
+    if (ok && blockIdx.x == 0) p.ctrl[MOE_CTRL_TASK_A] = 0u;
     int n = 0;
     if (ok && sh.ub0 < sh.ub1) {
         fence_proxy_async_global();   // generic-proxy writes of h (other CTAs) -> bulk-copy reads
@@ -883,8 +895,7 @@ __device__ void consumer(const MoeParams& p, Shared& sh, uint8_t* ring, uint8_t*
 // plus the block sums of the staged values (times 2^s_b) for the offset
 // correction.  Run by `nthr` threads (sid = 0 .. nthr-1, whole warps); one item
 // is one (step, t) fragment of a column, 8 consecutive items one 32-block.
-__device__ void stage_x(const MoeParams& p, Shared& sh, uint8_t* xh, int sid, int nthr) {
-    const uint32_t* x32 = reinterpret_cast<const uint32_t*>(p.x);
+__device__ void stage_x(const MoeParams& p, Shared& sh, uint8_t* xh, const uint32_t* x32, int sid, int nthr) {
     const int lane = sid & 31;
     const int per_col = p.H / 4;      // items per column
     const int hp = p.H / 2;           // bf16 pairs per column
@@ -896,7 +907,7 @@ __device__ void stage_x(const MoeParams& p, Shared& sh, uint8_t* xh, int sid, in
             if (j < per_col) {
                 const int step = j >> 2, tt = j & 3;
                 const uint32_t* src = x32 + (size_t)c * hp + step * 8 + tt;
-                const uint32_t v0 = __ldg(src), v1 = __ldg(src + 4);
+                const uint32_t v0 = src[0], v1 = src[4];
                 m = max(m, max((v0 << 16) & 0x7fffffffu, v0 & 0x7fff0000u));
                 m = max(m, max((v1 << 16) & 0x7fffffffu, v1 & 0x7fff0000u));
             }
@@ -927,7 +938,7 @@ __device__ void stage_x(const MoeParams& p, Shared& sh, uint8_t* xh, int sid, in
                 if (j < per_col) {
                     const int step = j >> 2, tt = j & 3;
                     const uint32_t* src = x32 + (size_t)c * hp + step * 8 + tt;
-                    const uint32_t v0 = __ldg(src), v1 = __ldg(src + 4);
+                    const uint32_t v0 = src[0], v1 = src[4];
                     const int sb = s_pos(fmt, step * 16, p.H);
                     const float sc = __int_as_float((127 + xn - sb) << 23);
                     const __half2 h0 = __floats2half2_rn(__uint_as_float(v0 << 16) * sc, __uint_as_float(v0 & 0xffff0000u) * sc);
@@ -977,10 +988,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_decode_kernel(MoeParams p) {
             mbar_init(&sh.rempty[i], 1);
         }
         mbar_init(&sh.adone, NEPI);
+        mbar_init(&sh.xload, 1);
         sh.abort_flag = 0;
         sh.consumed = 0;
         for (int c = 0; c < MOE_MAXT; ++c) sh.xmax[c] = 0u;
         fence_barrier_init();
+    }
+    // x: one bulk copy into the reduction buffers (first written after the
+    // staging below) when it fits and is 16-byte aligned, else read from global
+    const uint32_t xbytes = (uint32_t)(p.T * p.H * 2);
+    const bool xbulk = xbytes <= (uint32_t)(p.nred * NCW * 32 * 8 * 4) && (((uintptr_t)p.x & 15u) == 0);
+    if (xbulk && threadIdx.x == 0) {
+        mbar_arrive_expect_tx(&sh.xload, xbytes);
+        bulk_g2s(red, p.x, xbytes, &sh.xload, policy_evict_first());
     }
     __syncthreads();
     // The producer warp derives the slot table and its row-groups and starts
@@ -988,15 +1008,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_decode_kernel(MoeParams p) {
     if (w == WARP_PRODUCER) {
         if (p.T * p.k <= 32) build_slots_small(p, sh.st, rt);
         else build_slots(p, sh.st, rt);
-        if ((threadIdx.x & 31) == 0) {
-            cta_units(p, sh.st.nslots, 0, p.I / 16, sh.ua0, sh.ua1);
-            cta_units(p, sh.st.nslots, 1, p.H / 16, sh.ub0, sh.ub1);
-        }
+        if ((threadIdx.x & 31) == 0) down_units(p, sh.st.nslots, sh.ub0, sh.ub1);
         asm volatile("bar.arrive 2, %0;" ::"n"(NTHREADS) : "memory");
         if ((threadIdx.x & 31) == 0) producer(p, sh, ring);
     } else {
         const int sid = w < WARP_PRODUCER ? threadIdx.x : threadIdx.x - 32;
-        stage_x(p, sh, xh, sid, NTHREADS - 32);
+        if (xbulk && !mbar_wait(&sh.xload, 0, WAIT_LIMIT)) set_error(p.ctrl, MOE_ERR_TIMEOUT);
+        stage_x(p, sh, xh, xbulk ? (const uint32_t*)red : reinterpret_cast<const uint32_t*>(p.x), sid, NTHREADS - 32);
         asm volatile("bar.sync 2, %0;" ::"n"(NTHREADS) : "memory");
         if (w == WARP_HLOAD) {
             if ((threadIdx.x & 31) == 0) h_loader(p, sh, xh, hbytes_max, sstr);

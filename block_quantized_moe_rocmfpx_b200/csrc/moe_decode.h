@@ -16,6 +16,7 @@
 
 // workspace control words (uint32 index); the grid-barrier counters are
 // 64-bit and only grow
+#define MOE_CTRL_TASK_A 0      // next gate/up row-group to hand out (reset after the first barrier)
 #define MOE_CTRL_ERR 2
 #define MOE_CTRL_BAR_H 4       // u64: gate/up phase done (h complete)
 #define MOE_CTRL_BAR_D 6       // u64: down phase done (partials complete)
