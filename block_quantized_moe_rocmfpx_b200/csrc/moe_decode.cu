@@ -812,30 +812,25 @@ __device__ __forceinline__ bool loop_b(const MoeParams& p, Shared& sh, uint8_t* 
             hsum = (const float*)(hs + 4 * ncols * p.I);
         }
         const int c = r.c0 + w;
-        float v[2][8];
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            if (i >= r.n) break;
+        // the stage's row-groups one after the other (one copy of the chunk code)
+#pragma unroll 1
+        for (int i = 0; i < r.n; ++i) {
             if (r.flags & REC_FIRST) ab.zero();
             if (c < nch)
                 stepB<FMT, NB>(ring + rp.stage * MOE_STAGE_BYTES + i * MOE_HALF_BYTES + w * FULLB, c, p.I, lane, g, t, bs,
                                hsum, ncols, sstr, ab);
             if (r.flags & REC_LAST) {
-                float vb[NB][4];
+                float vb[NB][4], v[8];
                 finishB<FMT, NB>(ab, vb);
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    v[i][k] = vb[0][k];
-                    v[i][4 + k] = NB > 1 ? vb[NB - 1][k] : 0.f;
+                    v[k] = vb[0][k];
+                    v[4 + k] = NB > 1 ? vb[NB - 1][k] : 0.f;
                 }
+                if (!red_deposit(sh, p.nred, red, rc, w, lane, v, RedInfo{UNIT_B, slot, ncols, r.rg + i})) return false;
             }
         }
         cons_release(p, sh, rp, w, lane);
-        if (r.flags & REC_LAST) {
-            if (!red_deposit(sh, p.nred, red, rc, w, lane, v[0], RedInfo{UNIT_B, slot, ncols, r.rg})) return false;
-            if (r.n > 1 && !red_deposit(sh, p.nred, red, rc, w, lane, v[1], RedInfo{UNIT_B, slot, ncols, r.rg + 1}))
-                return false;
-        }
         if (r.flags & REC_HDONE) {
             // every stage of this slot is consumed: release its h buffer
             __syncwarp();
