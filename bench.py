@@ -36,6 +36,10 @@ ZIPF_S = 1.1
 NTOK = 1000
 COPIES = 8
 SEED = 0
+# DRAM bytes (read + write) of one q=1 launch of moe_decode_kernel from the ncu
+# capture summarised in profiles/moe_decode_q1_full_layer.md; set to None
+# whenever the kernel changes until it is captured again.
+TRAFFIC_Q1 = 67_831_552 + 1_007_104
 
 
 def parse():
@@ -409,7 +413,7 @@ def main():
                        "l2": f"inputs larger than L2: {args.copies} rotating copies of the layer",
                        "graph": "CUDA graph of all timed steps"},
             "roofline": {"bound": "hbm", "achieved": gbs1, "peak": peak, "unit": "GB/s", "frac": gbs1 / peak,
-                         "traffic": None, "kernel": "moe_decode_kernel", "peak_kind": peak_kind,
+                         "traffic": TRAFFIC_Q1, "kernel": "moe_decode_kernel", "peak_kind": peak_kind,
                          "algo_bytes_per_launch": r1["bytes"] / args.steps,
                          "kernel_us": r1["ms_ffn"] * 1e3 / args.steps},
             "q4": {"value": world * 4 * args.steps / (ms4 / 1e3), "unit": "tokens/s", "ms_per_step": ms4 / args.steps,

@@ -79,7 +79,7 @@ extern "C" int moe_ffn_forward_static(const moe_layer* layer, const void* x, int
     void* ws = nullptr;
     int rc = static_ws_address(&ws);
     if (rc != RFX_OK) return rc;
-    // the control words (task, exit and readiness counters, error flag) must
+    // the control words (task counter, grid-barrier counters, error flag) must
     // start at zero; everything after them is rewritten by the kernel
     const size_t ctrl_bytes = rfx_moe_ctrl_bytes(layer);
     cudaError_t e = cudaMemsetAsync(ws, 0, ctrl_bytes, (cudaStream_t)stream);

@@ -210,6 +210,11 @@ int rfx_ws_status(void* ws, void* stream);
  * x: device bf16 bits [T][H].  idx: device int32 [T][k], distinct per row,
  * in [0, E).  w: device fp32 [T][k].  y: device fp32 [T][H].
  * Limits: 1 <= T <= 8 (decode / verify), H % 32 == 0, I % 32 == 0, k <= 8.
+ * One cooperative launch of one CTA per SM (all CTAs resident at once: the
+ * gate/up, down and combine phases meet at two grid barriers whose counters
+ * live in the workspace).  A workspace must not be used by two calls that
+ * overlap on the GPU.  After a call that reported a device error through
+ * rfx_ws_status, re-initialise the workspace with rfx_ws_init before reuse.
  */
 int moe_ffn_forward(const moe_layer* layer, const void* x, int T, const int32_t* idx, const float* w,
                     float* y, void* ws, size_t ws_bytes, void* stream);
