@@ -21,7 +21,7 @@ RFX_FP2, RFX_FP3, RFX_FP4 = 2, 3, 4
 MAX_T = 8
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m block_quantized_moe_rocmfpx_b200.build` "
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python block_quantized_moe_rocmfpx_b200/build.py` "
                       "(nvcc, sm_100a); there is no fallback implementation")
 
 _lib = ctypes.CDLL(LIB_PATH)
@@ -59,10 +59,14 @@ _ws_init = _proto("rfx_ws_init", _i32, [_vp, _sz, _vp])
 _ws_status = _proto("rfx_ws_status", _i32, [_vp, _vp])
 _forward = _proto("moe_ffn_forward", _i32, [_vp, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp])
 _forward_static = _proto("moe_ffn_forward_static", _i32, [_vp, _vp, _i32, _vp, _vp, _vp, _vp])
+_rms = _proto("moe_rms_norm_bf16", _i32, [_vp, _i32, _i32, _vp, _vp])
+_stack_ws = _proto("moe_stack_workspace_bytes", _sz, [_vp, _i32, _i32])
+_stack = _proto("moe_stack_forward", _i32, [_vp, _i32, _vp, _vp, _i32, _vp, _vp, _sz, _vp])
 
 EXPORTED = ["rfx_last_error", "rfx_packed_bytes", "rfx_pack", "rfx_unpack", "rfx_pack_device", "moe_router_topk",
             "rfx_gemv_q", "moe_layer_create", "moe_layer_destroy", "moe_ffn_workspace_bytes", "rfx_ws_init",
-            "rfx_ws_status", "moe_ffn_forward", "moe_ffn_forward_static"]
+            "rfx_ws_status", "moe_ffn_forward", "moe_ffn_forward_static", "moe_rms_norm_bf16",
+            "moe_stack_workspace_bytes", "moe_stack_forward"]
 
 
 class RfxError(RuntimeError):
@@ -176,6 +180,28 @@ def moe_ffn_forward_static(handle: int, x, T: int, idx, w, y, stream=None):
     """moe_ffn_forward with the library's built-in 16 MiB workspace, for callers
     that cannot allocate device memory (see include/rfx.h)."""
     _check(_forward_static(handle, _ptr(x), T, _ptr(idx), _ptr(w), _ptr(y), _stream(stream)))
+
+
+def moe_rms_norm_bf16(y, x_next, stream=None):
+    """y fp32 [T][H] -> x_next bf16 [T][H] = bf16(y / sqrt(mean(y^2))) per column (device tensors)."""
+    T, H = y.shape
+    _check(_rms(_ptr(y), T, H, _ptr(x_next), _stream(stream)))
+
+
+def _handles(layers):
+    arr = (_vp * len(layers))(*[(l.handle if hasattr(l, "handle") else l) for l in layers])
+    return arr
+
+
+def moe_stack_workspace_bytes(layers, T: int) -> int:
+    return int(_stack_ws(_handles(layers), len(layers), T))
+
+
+def moe_stack_forward(layers, logits, x, y, ws, stream=None):
+    """L layers (MoeLayer or handles); logits fp32 [L][T][E], x bf16 [T][H], y fp32 [T][H] (device)."""
+    T = x.shape[0]
+    _check(_stack(_handles(layers), len(layers), _ptr(logits), _ptr(x), T, _ptr(y), _ptr(ws),
+                  ws.numel() * ws.element_size(), _stream(stream)))
 
 
 # --------------------------------------------------------- convenience ---

@@ -11,6 +11,7 @@
 #include "gemv.h"
 #include "moe_decode.h"
 #include "rfx_layout.h"
+#include "stack.h"
 
 int rfx_fail(int code, const std::string& msg);  // rfx_pack.cpp
 
@@ -220,4 +221,85 @@ extern "C" int moe_ffn_forward(const moe_layer* layer, const void* x, int T, con
     if (rc != RFX_OK) return rc;
     cudaError_t e = rfx::moe_decode_launch(p, grid, (cudaStream_t)stream);
     return e == cudaSuccess ? RFX_OK : cuda_fail("moe_ffn_forward", e);
+}
+
+// ------------------------------------------------------------------ stack ---
+
+extern "C" int moe_rms_norm_bf16(const float* y, int T, int H, void* x_next, void* stream) {
+    if (T < 0 || H < 1) return rfx_fail(RFX_EINVAL, "moe_rms_norm_bf16: need T >= 0 and H >= 1");
+    if (T == 0) return RFX_OK;
+    if (!y || !x_next) return rfx_fail(RFX_EINVAL, "moe_rms_norm_bf16: null pointer");
+    cudaError_t e = rfx::rms_bf16_launch(y, T, H, (uint16_t*)x_next, (cudaStream_t)stream);
+    return e == cudaSuccess ? RFX_OK : cuda_fail("moe_rms_norm_bf16", e);
+}
+
+namespace {
+
+struct StackWs {
+    size_t ffn, idx, w, ybuf, xbuf, total;
+};
+
+StackWs stack_ws_layout(const moe_layer* const* layers, int L, int T) {
+    StackWs W{};
+    size_t ffn = 0;
+    for (int l = 0; l < L; ++l) ffn = std::max(ffn, moe_ffn_workspace_bytes(layers[l], T));
+    const moe_layer_desc& d = layers[0]->d;
+    auto up = [](size_t n) { return (n + 255) / 256 * 256; };
+    W.ffn = 0;
+    W.idx = up(ffn);
+    W.w = W.idx + up((size_t)T * d.k * 4);
+    W.ybuf = W.w + up((size_t)T * d.k * 4);
+    W.xbuf = W.ybuf + up((size_t)T * d.H * 4);
+    W.total = W.xbuf + 2 * up((size_t)T * d.H * 2);
+    return W;
+}
+
+int stack_check(const moe_layer* const* layers, int L, int T, const char* who) {
+    if (!layers || L < 1) return rfx_fail(RFX_EINVAL, std::string(who) + ": need L >= 1 layers");
+    if (T < 1 || T > MOE_MAXT) return rfx_fail(RFX_EUNSUPPORTED, std::string(who) + ": 1 <= T <= 8 token columns");
+    for (int l = 0; l < L; ++l) {
+        if (!layers[l]) return rfx_fail(RFX_EINVAL, std::string(who) + ": null layer");
+        const moe_layer_desc& a = layers[l]->d;
+        const moe_layer_desc& b = layers[0]->d;
+        if (a.H != b.H || a.E != b.E || a.k != b.k)
+            return rfx_fail(RFX_EINVAL, std::string(who) + ": all layers need the same H, E and k");
+    }
+    return RFX_OK;
+}
+
+}  // namespace
+
+extern "C" size_t moe_stack_workspace_bytes(const moe_layer* const* layers, int L, int T) {
+    if (stack_check(layers, L, T, "moe_stack_workspace_bytes") != RFX_OK) return 0;
+    return stack_ws_layout(layers, L, T).total;
+}
+
+extern "C" int moe_stack_forward(const moe_layer* const* layers, int L, const float* logits, const void* x, int T,
+                                 float* y, void* ws, size_t ws_bytes, void* stream) {
+    int rc = stack_check(layers, L, T, "moe_stack_forward");
+    if (rc != RFX_OK) return rc;
+    if (!logits || !x || !y || !ws) return rfx_fail(RFX_EINVAL, "moe_stack_forward: null pointer");
+    if ((uintptr_t)ws & 255u) return rfx_fail(RFX_EINVAL, "moe_stack_forward: ws must be 256-byte aligned");
+    const StackWs W = stack_ws_layout(layers, L, T);
+    if (ws_bytes < W.total) return rfx_fail(RFX_EINVAL, "moe_stack_forward: workspace smaller than moe_stack_workspace_bytes");
+    const moe_layer_desc& d = layers[0]->d;
+    uint8_t* b = (uint8_t*)ws;
+    int32_t* idx = (int32_t*)(b + W.idx);
+    float* wts = (float*)(b + W.w);
+    float* ybuf = (float*)(b + W.ybuf);
+    uint16_t* xb[2] = {(uint16_t*)(b + W.xbuf), (uint16_t*)(b + W.xbuf + (W.total - W.xbuf) / 2)};
+    const void* xin = x;
+    for (int l = 0; l < L; ++l) {
+        rc = moe_router_topk(logits + (size_t)l * T * d.E, T, d.E, d.k, idx, wts, stream);
+        if (rc != RFX_OK) return rc;
+        float* yl = l + 1 == L ? y : ybuf;
+        rc = moe_ffn_forward(layers[l], xin, T, idx, wts, yl, b + W.ffn, W.idx - W.ffn, stream);
+        if (rc != RFX_OK) return rc;
+        if (l + 1 < L) {
+            rc = moe_rms_norm_bf16(ybuf, T, d.H, xb[l & 1], stream);
+            if (rc != RFX_OK) return rc;
+            xin = xb[l & 1];
+        }
+    }
+    return RFX_OK;
 }

@@ -238,6 +238,30 @@ int moe_ffn_forward(const moe_layer* layer, const void* x, int T, const int32_t*
 int moe_ffn_forward_static(const moe_layer* layer, const void* x, int T, const int32_t* idx, const float* w,
                            float* y, void* stream);
 
+/*
+ * Layer chaining for a stack of MoE layers (m.mzlw.cn, "Lucebox专攻DeepSeek
+ * V4…", section "MoE 专家并行": 43 MoE layers; the chaining rule is this
+ * library's stack workload): x_next[t] = bf16(y[t] / sqrt(mean(y[t]^2))),
+ * the mean over the H values of column t, computed in fp64 and rounded once
+ * to bf16 (nearest even).  y: device fp32 [T][H]; x_next: device bf16 bits
+ * [T][H] (may not alias y).  T == 0 is a no-op.
+ */
+int moe_rms_norm_bf16(const float* y, int T, int H, void* x_next, void* stream);
+
+/*
+ * A stack of L layers for T <= 8 token columns, all on `stream`: for l = 0..L-1,
+ * (idx, w) = moe_router_topk(logits[l]), y_l = moe_ffn_forward(layer l, x_l),
+ * x_{l+1} = moe_rms_norm_bf16(y_l); y receives y_{L-1}.  logits: device fp32
+ * [L][T][E]; x: device bf16 bits [T][H] (x_0); y: device fp32 [T][H].  All
+ * layers must share H, E and k.  The workspace (moe_stack_workspace_bytes,
+ * 256-byte aligned, caller-owned) holds one moe_ffn_forward workspace (zero it
+ * once with rfx_ws_init), the routing and the chained activations.  Launches
+ * 3 kernels per layer and can be captured in a CUDA graph.
+ */
+size_t moe_stack_workspace_bytes(const moe_layer* const* layers, int L, int T);
+int moe_stack_forward(const moe_layer* const* layers, int L, const float* logits, const void* x, int T, float* y,
+                      void* ws, size_t ws_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

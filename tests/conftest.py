@@ -10,11 +10,21 @@ if ROOT not in sys.path:
 GOLDEN = os.path.join(ROOT, "tests", "golden")
 
 
+def _librfx_build():
+    """The package's build script, loaded by path: importing the package itself
+    needs the library it builds."""
+    import importlib.util
+    path = os.path.join(ROOT, "block_quantized_moe_rocmfpx_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("_librfx_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA B200 (sm_100a) device")
     # build the in-tree libraries if a source changed (nvcc cross-compiles sm_100a on any host)
-    from block_quantized_moe_rocmfpx_b200 import build as _b
-    _b.build()
+    _librfx_build().build()
     import synth
     synth.build()
     synth.build_dev()
