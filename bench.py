@@ -52,6 +52,9 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--copies", type=int, default=COPIES, help="rotating layer copies (>= 8 keeps steps L2-cold)")
     ap.add_argument("--only-q1", action="store_true", help="skip the q=4 verify measurement")
+    ap.add_argument("--stack", action="store_true",
+                    help="also time the 43-layer stack (98.7 GB of distinct layers resident, FFN only)")
+    ap.add_argument("--stack-only", action="store_true", help="time only the 43-layer stack")
     return ap.parse_args()
 
 
@@ -245,6 +248,68 @@ class Workload:
         return tot
 
 
+STACK_LAYERS = 43
+
+
+def measure_stack(qs, steps: int, warmup: int, dev):
+    """The 43-layer stack: distinct seeded full-size layers resident in HBM,
+    each token step one moe_stack_forward call (router, MoE FFN and the
+    unit-RMS bf16 chaining per layer), captured in one CUDA graph."""
+    import time
+    import numpy as np
+    import torch
+    import synth
+    import block_quantized_moe_rocmfpx_b200 as rfx
+    from synth.layers import SynthLayer
+    t0 = time.time()
+    layers = [SynthLayer(SEED, l, H, I, E, K_TOP, device=dev) for l in range(STACK_LAYERS)]
+    gen_s = time.time() - t0
+    out = {"layers": STACK_LAYERS, "resident_gb": sum(
+        E * sum(l.strides) + sum(b.numel() for b in l.shared) for l in layers) / 1e9, "generate_s": gen_s}
+    stream = torch.cuda.Stream(device=dev)
+    for q in qs:
+        mls = [l.moe_layer(max_T=q) for l in layers]
+        ntok = 64
+        logits_h = np.stack([np.stack([synth.logits(SEED, l, t * q, q, E, ZIPF_S) for l in range(STACK_LAYERS)])
+                             for t in range(ntok)])                                  # [tok][L][q][E]
+        x_h = np.stack([synth.x_bf16(SEED, t * q, q, H) for t in range(ntok)])       # [tok][q][H]
+        logits = torch.from_numpy(logits_h).to(dev)
+        x = torch.from_numpy(x_h).view(torch.bfloat16).to(dev)
+        y = torch.empty((q, H), dtype=torch.float32, device=dev)
+        ws = torch.empty(rfx.moe_stack_workspace_bytes(mls, q), dtype=torch.uint8, device=dev)
+        rfx.rfx_ws_init(ws)
+        # bytes one step must move: each layer's union of routed experts + shared + activations
+        nbytes = 0.0
+        for t in range(ntok):
+            for l in range(STACK_LAYERS):
+                idx_o = np.argsort(-logits_h[t, l], axis=-1, kind="stable")[:, :K_TOP]
+                nbytes += layers[l].union_bytes(idx_o.ravel()) + q * (2 * H + 8 * K_TOP + 4 * H + 4 * E)
+        per_step = nbytes / ntok
+        with torch.cuda.stream(stream):
+            def step(t):
+                rfx.moe_stack_forward(mls, logits[t % ntok], x[t % ntok], y, ws, stream)
+            for t in range(3):
+                step(t)
+            torch.cuda.synchronize()
+            g = graph_of(step, steps, stream)
+            gw = graph_of(step, max(3, warmup), stream)
+            gw.replay()
+            torch.cuda.synchronize()
+            ms = time_graph(g, stream)
+            del g, gw
+        st = rfx_status_of(ws)
+        out[f"q{q}"] = {"value": q * steps / (ms / 1e3), "unit": "tokens/s", "ms_per_token_step": ms / steps,
+                        "achieved_gbs": per_step * steps / (ms / 1e3) / 1e9, "bytes_per_step": per_step,
+                        "device_status": st}
+        del mls
+    return out
+
+
+def rfx_status_of(ws) -> int:
+    import block_quantized_moe_rocmfpx_b200 as rfx
+    return rfx.rfx_ws_status(ws)
+
+
 def graph_of(fn, n, stream):
     import torch
     g = torch.cuda.CUDAGraph()
@@ -376,6 +441,15 @@ def main():
         __graft_entry__.build()
     if world > 1:
         dist.barrier()
+    if args.stack_only:
+        st = measure_stack((1, 4), min(args.steps, 200), max(3, args.warmup), dev)
+        peak, peak_kind = peaks()
+        for q in (1, 4):
+            st[f"q{q}"]["frac"] = st[f"q{q}"]["achieved_gbs"] / peak
+        if rank == 0:
+            print(json.dumps({"metric": "43-layer MoE-FFN stack decode tokens/s (FFN only)", "stack": st,
+                              "peak_gbs": peak, "peak_kind": peak_kind}), flush=True)
+        return
     r1 = measure(1, args.steps, max(3, args.warmup), dev, rank, world, True, not args.no_e2e, args.copies)
     r4 = r1 if args.only_q1 else measure(4, args.steps, max(3, args.warmup), dev, rank, world, False, False,
                                          args.copies)
