@@ -62,11 +62,22 @@ _forward_static = _proto("moe_ffn_forward_static", _i32, [_vp, _vp, _i32, _vp, _
 _rms = _proto("moe_rms_norm_bf16", _i32, [_vp, _i32, _i32, _vp, _vp])
 _stack_ws = _proto("moe_stack_workspace_bytes", _sz, [_vp, _i32, _i32])
 _stack = _proto("moe_stack_forward", _i32, [_vp, _i32, _vp, _vp, _i32, _vp, _vp, _sz, _vp])
+_pf_ws_bytes = _proto("moe_prefill_workspace_bytes", _sz, [_vp, _i32])
+_prefill = _proto("moe_ffn_prefill", _i32, [_vp, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp])
+
+
+class moe_prefill_ws_view(ctypes.Structure):
+    _fields_ = [("counts", _vp), ("row_token", _vp), ("row_weight", _vp), ("h", _vp),
+                ("routed_rows", _i64), ("h_rows", _i64)]
+
+
+_pf_view = _proto("moe_prefill_view", _i32, [_vp, _i32, _vp, ctypes.POINTER(moe_prefill_ws_view)])
 
 EXPORTED = ["rfx_last_error", "rfx_packed_bytes", "rfx_pack", "rfx_unpack", "rfx_pack_device", "moe_router_topk",
             "rfx_gemv_q", "moe_layer_create", "moe_layer_destroy", "moe_ffn_workspace_bytes", "rfx_ws_init",
             "rfx_ws_status", "moe_ffn_forward", "moe_ffn_forward_static", "moe_rms_norm_bf16",
-            "moe_stack_workspace_bytes", "moe_stack_forward"]
+            "moe_stack_workspace_bytes", "moe_stack_forward", "moe_prefill_workspace_bytes", "moe_ffn_prefill",
+            "moe_prefill_view"]
 
 
 class RfxError(RuntimeError):
@@ -204,6 +215,35 @@ def moe_stack_forward(layers, logits, x, y, ws, stream=None):
                   ws.numel() * ws.element_size(), _stream(stream)))
 
 
+def moe_prefill_workspace_bytes(handle: int, T: int) -> int:
+    return int(_pf_ws_bytes(handle, T))
+
+
+def moe_ffn_prefill(handle: int, x, T: int, idx, w, y, ws, stream=None):
+    """Grouped-GEMM prefill (bf16 operands, tcgen05): x bf16 [T][H], idx int32 [T][k],
+    w fp32 [T][k], y fp32 [T][H], ws uint8 (moe_prefill_workspace_bytes), all device."""
+    _check(_prefill(handle, _ptr(x), T, _ptr(idx), _ptr(w), _ptr(y), _ptr(ws), ws.numel() * ws.element_size(),
+                    _stream(stream)))
+
+
+def moe_prefill_view(handle: int, T: int, ws, I: int, E: int):
+    """Tensors viewing a prefill workspace after a call: counts int32 [E], row_token
+    int32 [T*k], row_weight fp32 [T*k], h bf16 bits int16 [T*k + T][I]."""
+    import torch
+    v = moe_prefill_ws_view()
+    _check(_pf_view(handle, T, _ptr(ws), ctypes.byref(v)))
+    base = ws.data_ptr()
+
+    def sub(ptr, nbytes, dtype):
+        off = int(ptr) - base
+        return ws[off:off + nbytes].view(dtype)
+
+    rr, hr = int(v.routed_rows), int(v.h_rows)
+    return {"counts": sub(v.counts, 4 * E, torch.int32), "row_token": sub(v.row_token, 4 * rr, torch.int32),
+            "row_weight": sub(v.row_weight, 4 * rr, torch.float32),
+            "h": sub(v.h, 2 * hr * I, torch.int16).view(hr, I)}
+
+
 # --------------------------------------------------------- convenience ---
 
 class MoeLayer:
@@ -239,6 +279,24 @@ class MoeLayer:
         if T > self.max_T:
             raise ValueError(f"T={T} > max_T={self.max_T}")
         moe_ffn_forward(self.handle, x, T, idx, w, y, self.ws, stream)
+
+    def prefill(self, x, idx, w, y, stream=None):
+        """moe_ffn_prefill with a workspace kept on the layer (grown on demand)."""
+        import torch
+        T = x.shape[0]
+        nbytes = moe_prefill_workspace_bytes(self.handle, T)
+        if nbytes == 0:
+            raise RfxError(-2, f"prefill unsupported for T={T}, H={self.H}, I={self.I}")
+        if getattr(self, "pf_ws", None) is None or self.pf_ws.numel() < nbytes:
+            self.pf_ws = torch.empty(nbytes, dtype=torch.uint8, device=x.device)
+            rfx_ws_init(self.pf_ws)
+        moe_ffn_prefill(self.handle, x, T, idx, w, y, self.pf_ws, stream)
+
+    def prefill_view(self, T: int):
+        return moe_prefill_view(self.handle, T, self.pf_ws, self.I, self.E)
+
+    def prefill_status(self, stream=None) -> int:
+        return rfx_ws_status(self.pf_ws, stream)
 
     def status(self, stream=None) -> int:
         return rfx_ws_status(self.ws, stream)

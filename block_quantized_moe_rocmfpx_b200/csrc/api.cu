@@ -10,6 +10,7 @@
 #include "../../include/rfx.h"
 #include "gemv.h"
 #include "moe_decode.h"
+#include "prefill.h"
 #include "rfx_layout.h"
 #include "stack.h"
 
@@ -126,8 +127,11 @@ extern "C" int moe_layer_create(const moe_layer_desc* d, moe_layer** out) {
 
 extern "C" void moe_layer_destroy(moe_layer* layer) { delete layer; }
 
+extern "C" size_t moe_prefill_workspace_bytes(const moe_layer* layer, int T);
+
 extern "C" size_t moe_ffn_workspace_bytes(const moe_layer* layer, int T) {
-    if (!layer || T < 1 || T > MOE_MAXT) return 0;
+    if (!layer || T < 1) return 0;
+    if (T > MOE_MAXT) return moe_prefill_workspace_bytes(layer, T);
     return rfx::moe_ws_layout(T, layer->d.k, layer->d.H, layer->d.I).total;
 }
 
@@ -214,6 +218,7 @@ int moe_prepare(const moe_layer* layer, const void* x, int T, const int32_t* idx
 
 extern "C" int moe_ffn_forward(const moe_layer* layer, const void* x, int T, const int32_t* idx, const float* w,
                                float* y, void* ws, size_t ws_bytes, void* stream) {
+    if (T > MOE_MAXT) return moe_ffn_prefill(layer, x, T, idx, w, y, ws, ws_bytes, stream);
     rfx::MoeParams p;
     int grid = 0;
     size_t smem = 0;
@@ -221,6 +226,87 @@ extern "C" int moe_ffn_forward(const moe_layer* layer, const void* x, int T, con
     if (rc != RFX_OK) return rc;
     cudaError_t e = rfx::moe_decode_launch(p, grid, (cudaStream_t)stream);
     return e == cudaSuccess ? RFX_OK : cuda_fail("moe_ffn_forward", e);
+}
+
+// ---------------------------------------------------------------- prefill ---
+
+namespace {
+
+const int PF_MAX_T = 1 << 16;
+
+int prefill_check(const moe_layer* layer, int T, const char* who) {
+    if (!layer) return rfx_fail(RFX_EINVAL, std::string(who) + ": null layer");
+    const moe_layer_desc& d = layer->d;
+    if (T < 1 || T > PF_MAX_T) return rfx_fail(RFX_EUNSUPPORTED, std::string(who) + ": 1 <= T <= 65536 tokens");
+    if (d.H % 256 || d.I % 256)
+        return rfx_fail(RFX_EUNSUPPORTED, std::string(who) + ": the prefill path needs H and I multiples of 256");
+    return RFX_OK;
+}
+
+rfx::PfWs prefill_layout(const moe_layer* layer, int T) {
+    const moe_layer_desc& d = layer->d;
+    return rfx::pf_ws_layout(T, d.k, d.E, d.H, d.I);
+}
+
+}  // namespace
+
+extern "C" size_t moe_prefill_workspace_bytes(const moe_layer* layer, int T) {
+    if (!layer || T < 1 || T > PF_MAX_T || layer->d.H % 256 || layer->d.I % 256) return 0;
+    return prefill_layout(layer, T).total;
+}
+
+extern "C" int moe_ffn_prefill(const moe_layer* layer, const void* x, int T, const int32_t* idx, const float* w,
+                               float* y, void* ws, size_t ws_bytes, void* stream) {
+    int rc = prefill_check(layer, T, "moe_ffn_prefill");
+    if (rc != RFX_OK) return rc;
+    if (!x || !idx || !w || !y || !ws) return rfx_fail(RFX_EINVAL, "moe_ffn_prefill: null pointer");
+    if (!aligned16(x) || !aligned16(y) || ((uintptr_t)ws & 255u))
+        return rfx_fail(RFX_EINVAL, "moe_ffn_prefill: x and y must be 16-byte and ws 256-byte aligned");
+    const rfx::PfWs L = prefill_layout(layer, T);
+    if (ws_bytes < L.total) return rfx_fail(RFX_EINVAL, "moe_ffn_prefill: workspace smaller than moe_prefill_workspace_bytes");
+    int sms = 0, smem_optin = 0;
+    rc = device_props(sms, smem_optin);
+    if (rc != RFX_OK) return rc;
+    if (std::max(rfx::pf_gemm_smem_bytes(0), rfx::pf_gemm_smem_bytes(1)) > (size_t)smem_optin)
+        return rfx_fail(RFX_EUNSUPPORTED, "moe_ffn_prefill: the device has too little shared memory per block");
+    const moe_layer_desc& d = layer->d;
+    rfx::PfParams p{};
+    p.H = d.H; p.I = d.I; p.E = d.E; p.k = d.k; p.T = T;
+    p.fA = d.f_gate; p.fB = d.f_down;
+    p.fsA = d.has_shared ? d.f_sh_gate : 2;
+    p.fsB = d.has_shared ? d.f_sh_down : 2;
+    p.gate = (const uint8_t*)d.gate; p.up = (const uint8_t*)d.up; p.down = (const uint8_t*)d.down;
+    p.sg = (long long)d.stride_gate; p.su = (long long)d.stride_up; p.sd = (long long)d.stride_down;
+    p.has_shared = d.has_shared ? 1 : 0;
+    p.shg = (const uint8_t*)d.sh_gate; p.shu = (const uint8_t*)d.sh_up; p.shd = (const uint8_t*)d.sh_down;
+    p.x = (const uint16_t*)x; p.idx = idx; p.wts = w; p.y = y;
+    uint8_t* b = (uint8_t*)ws;
+    p.ctrl = (uint32_t*)(b + L.ctrl);
+    p.cnt = (int32_t*)(b + L.cnt);
+    p.perm_tok = (int32_t*)(b + L.perm_tok);
+    p.perm_w = (float*)(b + L.perm_w);
+    p.tiles = (int4*)(b + L.tiles);
+    p.xp = (uint16_t*)(b + L.xp);
+    p.hp = (uint16_t*)(b + L.hp);
+    p.max_tiles = L.max_tiles;
+    cudaError_t e = rfx::pf_launch(p, sms, (cudaStream_t)stream);
+    if (e == cudaErrorInvalidValue) return rfx_fail(RFX_ECUDA, "moe_ffn_prefill: tensor-map encoding failed");
+    return e == cudaSuccess ? RFX_OK : cuda_fail("moe_ffn_prefill", e);
+}
+
+extern "C" int moe_prefill_view(const moe_layer* layer, int T, const void* ws, moe_prefill_ws_view* v) {
+    int rc = prefill_check(layer, T, "moe_prefill_view");
+    if (rc != RFX_OK) return rc;
+    if (!ws || !v) return rfx_fail(RFX_EINVAL, "moe_prefill_view: null pointer");
+    const rfx::PfWs L = prefill_layout(layer, T);
+    const uint8_t* b = (const uint8_t*)ws;
+    v->counts = (const int32_t*)(b + L.cnt);
+    v->row_token = (const int32_t*)(b + L.perm_tok);
+    v->row_weight = (const float*)(b + L.perm_w);
+    v->h = b + L.hp;
+    v->routed_rows = (int64_t)T * layer->d.k;
+    v->h_rows = (int64_t)T * layer->d.k + T;
+    return RFX_OK;
 }
 
 // ------------------------------------------------------------------ stack ---

@@ -1,0 +1,684 @@
+// prefill.cu -- the MoE FFN for many tokens (prefill): the same mathematics
+// as the decode path (m.mzlw.cn, "Lucebox专攻DeepSeek V4…", section "MoE 专家
+// 并行": top-6 of 256 routed experts plus one shared expert, gate/up -> SwiGLU
+// -> down, weighted combine) run as a grouped GEMM on the tcgen05 tensor
+// cores.  The packed ROCmFPX-style blocks (taozi.news, "DeepSeek V4 Flash 在
+// 128GB 锐龙 AI MAX+ 上跑到 32 tok/s", section "ROCmFPX：把 284B 权重压进
+// 128 GB") are dequantised to bf16 in shared memory, once per (expert,
+// 128-row tile, token tile), and fed to the tensor cores as the M = 128
+// operand; the tokens routed to the expert are the N operand (16..256).
+//
+// Operand precision: every weight enters the MMA as bf16(level * scale)
+// (rounded to nearest even from the exact product) and the SwiGLU output
+// enters the down projection as bf16(h); accumulation is fp32 in tensor
+// memory.
+//
+// Steps (one stream, six launches):
+//   pf_count   tokens per routed expert, and the expert-id range check
+//   pf_place   rows grouped by expert, tokens in ascending order inside an
+//              expert (stable, so the grouping is unique): token and weight
+//   pf_tiles   token tiles of <= 256 rows: the shared expert's first, then the
+//              routed experts by descending token count (heaviest work first)
+//   pf_gather  the routed rows of x copied into grouped order; y zeroed
+//   pf_gemm<0> gate/up GEMM + SwiGLU -> h (bf16), per (tile, 128-row block of I)
+//   pf_gemm<1> down GEMM, per (tile, 128-row block of H); the epilogue adds
+//              w * d into y[token] (fp32 atomics: the order of the k + 1
+//              additions per output element is not fixed)
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "moe_decode.h"
+#include "prefill.h"
+#include "rfx_layout.h"
+#include "rfx_tile.cuh"
+#include "tc.cuh"
+
+namespace rfx {
+namespace {
+
+constexpr long long PF_WAIT = 1000000000LL;   // SM clocks before a wait gives up (about half a second)
+
+constexpr int PF_THREADS = 448;
+constexpr int W_PROD = 0;     // TMA loads of the token rows (B operand)
+constexpr int W_MMA = 1;      // tensor-memory allocation and MMA issue
+constexpr int W_DQ0 = 2;      // 8 dequantisation warps, one 16-row group each
+constexpr int N_DQ = 8;
+constexpr int W_EPI0 = 10;    // 4 epilogue warps, one tensor-memory lane quarter each
+constexpr int N_EPI = 4;
+constexpr uint32_t TMEM_COLS = 512;
+
+template <int MODE>
+struct PfCfg {
+    static constexpr int NMAT = MODE == 0 ? 2 : 1;                 // gate + up, or down
+    static constexpr int A_MAT = PF_BM * PF_BK * 2;                // 16 KB bf16 per matrix
+    static constexpr int A_BYTES = NMAT * A_MAT;
+    static constexpr int B_BYTES = PF_TILE_N * PF_BK * 2;          // 32 KB bf16
+    static constexpr int STAGE = A_BYTES + B_BYTES;
+    static constexpr int NS = MODE == 0 ? 3 : 4;                    // pipeline stages
+    static constexpr int NACC = MODE == 0 ? 1 : 2;                  // accumulator buffers of 256 (MODE 1) columns
+    static_assert(A_MAT % 1024 == 0 && STAGE % 1024 == 0, "swizzle atoms must stay 1024-byte aligned");
+};
+
+struct PfShared {
+    uint64_t fullA[4];    // dequantised A tiles written (8 warp arrivals)
+    uint64_t fullB[4];    // B rows landed (1 arrival + bytes)
+    uint64_t empty[4];    // stage read by the tensor cores (MMA commit)
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
+    uint64_t drain;
+    uint32_t tmem;
+    volatile int abort;
+};
+
+__device__ __forceinline__ void pf_set_error(uint32_t* ctrl, uint32_t bits) { atomicOr(ctrl + PF_CTRL_ERR, bits); }
+
+// Bounded wait; gives up when another role of the CTA has aborted or after
+// PF_WAIT clocks (then records a timeout and aborts the CTA).
+__device__ __noinline__ bool pf_wait(PfShared& sh, uint32_t* ctrl, uint64_t* bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+        if (sh.abort) return false;
+        if (clock64() - t0 > PF_WAIT) {
+            sh.abort = 1;
+            pf_set_error(ctrl, MOE_ERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+// Whole-warp wait: every lane acquires; the outcome is made uniform.
+__device__ __forceinline__ bool pf_wait_warp(PfShared& sh, uint32_t* ctrl, uint64_t* bar, uint32_t parity) {
+    const bool ok = pf_wait(sh, ctrl, bar, parity);
+    return __all_sync(0xffffffffu, ok);
+}
+
+// ----------------------------------------------------------- grouping ---
+
+constexpr int GRP_CHUNK = 2048;
+
+// cnt[e] for the 8 experts of this CTA (one warp each); CTA 0 warp 0 also
+// checks every id against [0, E).
+__global__ void __launch_bounds__(256) pf_count_kernel(const int32_t* __restrict__ idx, int n, int E,
+                                                       int32_t* __restrict__ cnt, uint32_t* __restrict__ ctrl) {
+    __shared__ int32_t s_idx[GRP_CHUNK];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int e = blockIdx.x * 8 + warp;
+    int c = 0;
+    bool bad = false;
+    for (int base = 0; base < n; base += GRP_CHUNK) {
+        const int m = min(GRP_CHUNK, n - base);
+        __syncthreads();
+        for (int i = threadIdx.x; i < m; i += 256) s_idx[i] = idx[base + i];
+        __syncthreads();
+        for (int i = lane; i < m; i += 32) {
+            const int v = s_idx[i];
+            c += v == e;
+            if (blockIdx.x == 0 && warp == 0) bad |= v < 0 || v >= E;
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+    if (lane == 0 && e < E) cnt[e] = c;
+    if (__any_sync(0xffffffffu, bad) && lane == 0) pf_set_error(ctrl, MOE_ERR_EXPERT);
+}
+
+// Rows of expert e start at off(e) = sum of the counts of the experts below
+// it; the entries (t, j) routed to e take them in ascending entry order
+// t * k + j (ballot prefix counts inside each group of 32 entries).
+__global__ void __launch_bounds__(256) pf_place_kernel(const int32_t* __restrict__ idx,
+                                                       const float* __restrict__ wts, int n, int k, int E,
+                                                       const int32_t* __restrict__ cnt,
+                                                       int32_t* __restrict__ perm_tok, float* __restrict__ perm_w) {
+    __shared__ int32_t s_idx[GRP_CHUNK];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int e = blockIdx.x * 8 + warp;
+    int off = 0;
+    for (int i = lane; i < min(e, E); i += 32) off += cnt[i];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) off += __shfl_xor_sync(0xffffffffu, off, o);
+    int run = 0;
+    for (int base = 0; base < n; base += GRP_CHUNK) {
+        const int m = min(GRP_CHUNK, n - base);
+        __syncthreads();
+        for (int i = threadIdx.x; i < m; i += 256) s_idx[i] = idx[base + i];
+        __syncthreads();
+        if (e >= E) continue;
+        for (int i0 = 0; i0 < m; i0 += 32) {
+            const int i = i0 + lane;
+            const bool hit = i < m && s_idx[i] == e;
+            const uint32_t b = __ballot_sync(0xffffffffu, hit);
+            if (hit) {
+                const int pos = off + run + __popc(b & ((1u << lane) - 1u));
+                perm_tok[pos] = (base + i) / k;
+                perm_w[pos] = wts[base + i];
+            }
+            run += __popc(b);
+        }
+    }
+}
+
+// Exclusive prefix sum over the 1024 threads of the block; *total gets the sum.
+__device__ int block_excl_scan(int v, int* ws, int* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += u;
+    }
+    __syncthreads();
+    if (lane == 31) ws[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+        const int s = ws[lane];
+        int si = s;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, si, o);
+            if (lane >= o) si += u;
+        }
+        ws[lane] = si - s;
+        if (lane == 31) ws[32] = si;
+    }
+    __syncthreads();
+    const int r = ws[warp] + inc - v;
+    *total = ws[32];
+    return r;
+}
+
+// One CTA of 1024 threads (E <= 1024): expert offsets, the descending-count
+// order (ties: lower expert id first), and the token tiles.  A count c is cut
+// into ceil(c / 256) tiles of nearly equal size.
+__global__ void __launch_bounds__(1024) pf_tiles_kernel(PfParams p) {
+    __shared__ int s_cnt[1024], s_off[1024], s_ord[1024];
+    __shared__ int s_ws[33];
+    const int tid = threadIdx.x;
+    const int c = tid < p.E ? p.cnt[tid] : 0;
+    s_cnt[tid] = c;
+    int rows = 0;
+    s_off[tid] = block_excl_scan(c, s_ws, &rows);
+    __syncthreads();
+    if (tid < p.E) {
+        int r = 0;
+        for (int e2 = 0; e2 < p.E; ++e2) {
+            const int c2 = s_cnt[e2];
+            r += c2 > c || (c2 == c && e2 < tid);
+        }
+        s_ord[r] = tid;
+    }
+    __syncthreads();
+    const int eo = tid < p.E ? s_ord[tid] : -1;
+    const int co = eo >= 0 ? s_cnt[eo] : 0;
+    const int nt = (co + PF_TILE_N - 1) / PF_TILE_N;
+    int nt_total = 0;
+    const int tb = block_excl_scan(nt, s_ws, &nt_total);
+    const int nts = p.has_shared ? (p.T + PF_TILE_N - 1) / PF_TILE_N : 0;
+    if (nt > 0) {
+        const int sz = (co + nt - 1) / nt;
+        for (int j = 0; j < nt; ++j)
+            p.tiles[nts + tb + j] = make_int4(s_off[eo] + j * sz, min(sz, co - j * sz), eo, 0);
+    }
+    if (tid < nts) {
+        const int sz = (p.T + nts - 1) / nts;
+        p.tiles[tid] = make_int4(p.T * p.k + tid * sz, min(sz, p.T - tid * sz), -1, 0);
+    }
+    if (tid == 0) {
+        p.ctrl[PF_CTRL_NTILES] = (uint32_t)(nts + nt_total);
+        p.ctrl[PF_CTRL_ROWS] = (uint32_t)rows;
+    }
+}
+
+// x rows in grouped order (16-byte copies), and y = 0.
+__global__ void __launch_bounds__(256) pf_gather_kernel(PfParams p) {
+    const int nch = p.H / 8;   // 16-byte chunks per row
+    const long long rows = (long long)p.ctrl[PF_CTRL_ROWS];
+    const long long items = rows * nch;
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    const uint4* xs = reinterpret_cast<const uint4*>(p.x);
+    uint4* xd = reinterpret_cast<uint4*>(p.xp);
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < items; i += stride) {
+        const long long r = i / nch;
+        const int ch = (int)(i - r * nch);
+        xd[i] = __ldg(xs + (long long)p.perm_tok[r] * nch + ch);
+    }
+    float4* y4 = reinterpret_cast<float4*>(p.y);
+    const long long ny = (long long)p.T * p.H / 4;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < ny; i += stride)
+        y4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// --------------------------------------------------------- grouped GEMM ---
+
+struct PfUnit {
+    int row0, n, e, rt, npad;
+};
+
+__device__ __forceinline__ PfUnit pf_unit(const PfParams& p, int u, int RT) {
+    const int4 t = p.tiles[u / RT];
+    PfUnit U;
+    U.row0 = t.x;
+    U.n = t.y;
+    U.e = t.z;
+    U.rt = u % RT;
+    U.npad = (t.y + 15) & ~15;
+    return U;
+}
+
+// One lane's share of a full chunk (8 tiles = 16 rows x 256 k) of one matrix,
+// read straight from global memory (slab-major layout, include/rfx.h).
+template <int F>
+struct PfChunk {
+    static constexpr int NW = 4 * F;
+    static constexpr int NSW = F == 4 ? 4 : 8;
+    uint32_t wd[NW];
+    uint32_t sc[NSW];
+    __device__ __forceinline__ void load(const uint8_t* ch, int lane, int g) {
+#pragma unroll
+        for (int i = 0; i < F; ++i) {
+            const uint4 v = ldg_stream(ch + (i * 32 + lane) * 16);
+            wd[4 * i] = v.x; wd[4 * i + 1] = v.y; wd[4 * i + 2] = v.z; wd[4 * i + 3] = v.w;
+        }
+        constexpr int CODE = Plane<F>::CODE_BYTES;
+#pragma unroll
+        for (int i = 0; i < NSW / 4; ++i) {
+            const uint4 v = ldg_stream(ch + CODE + (i * 8 + g) * 16);
+            sc[4 * i] = v.x; sc[4 * i + 1] = v.y; sc[4 * i + 2] = v.z; sc[4 * i + 3] = v.w;
+        }
+    }
+    static __device__ __forceinline__ uint4 ldg_stream(const uint8_t* p) {
+        uint4 v;
+        asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                     : "l"(p));
+        return v;
+    }
+};
+
+// Tile B of a chunk -> bf16 into the swizzled A tile.  Register r of the lane
+// holds row g + 8 (r & 1), k = 32 (B & 1) + 16 (r >> 2) + 8 ((r >> 1) & 1) + 2t
+// (+1 in the high half) of the 64-wide stage; its 4 bytes go to 16-byte chunk
+// k / 8 of that row, stored at chunk position (k / 8) ^ g.  `base` is the
+// stage's matrix tile address plus the lane's row-group, g and t offsets; xo[c]
+// = ((c ^ g) << 4).
+template <int F, int B>
+__device__ __forceinline__ void pf_decode_tile(const PfChunk<F>& c, const uint32_t* sh, uint32_t base,
+                                               const uint32_t* xo) {
+    uint32_t a[8];
+    plane_regs<F, B>(c.wd, sh, a);
+    constexpr int S = Plane<F>::s_of(B);
+    constexpr uint32_t MAGIC = ((uint32_t)(25 - S) << 10) * 0x10001u;   // fp16 2^(10-S) in both halves
+    constexpr float K = -((float)(1 << (10 - S)) + Plane<F>::OFF);
+    constexpr int BP = B & 1;
+    if constexpr (F == 4) {
+        const uint32_t w = c.sc[B >> 1] >> (16 * (B & 1));
+        const float s0 = scale_e8m0(w & 0xFFu), s1 = scale_e8m0((w >> 8) & 0xFFu);
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const uint32_t out = deq_pair_pow2scale(a[r] | MAGIC, K, (r & 1) ? s1 : s0);
+            const int cidx = 4 * BP + 2 * (r >> 2) + ((r >> 1) & 1);
+            sts32(base + (r & 1) * 1024 + xo[cidx], out);
+        }
+    } else {
+        const uint32_t w = c.sc[B];
+        const float2 s = scale_f16x2(w);
+        const float C0 = K * s.x, C1 = K * s.y;
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const uint32_t v = a[r] | MAGIC;
+            const uint32_t out = (r & 1) ? deq_pair_f16scale<1>(v, w, C1) : deq_pair_f16scale<0>(v, w, C0);
+            const int cidx = 4 * BP + 2 * (r >> 2) + ((r >> 1) & 1);
+            sts32(base + (r & 1) * 1024 + xo[cidx], out);
+        }
+    }
+}
+
+template <int F, int KK>
+__device__ __forceinline__ void pf_decode_kstep(const PfChunk<F>& c, const uint32_t* sh, uint32_t base,
+                                                const uint32_t* xo) {
+    pf_decode_tile<F, 2 * KK>(c, sh, base, xo);
+    pf_decode_tile<F, 2 * KK + 1>(c, sh, base, xo);
+}
+
+template <int F>
+__device__ __forceinline__ void pf_shift(const PfChunk<F>& c, uint32_t* sh) {
+    constexpr int SH = F == 2 ? 10 : (F == 3 ? 9 : 8);
+#pragma unroll
+    for (int i = 0; i < 4 * F; ++i) sh[i] = c.wd[i] >> SH;
+}
+
+// Dequantisation of one unit by one warp (row-group d of the 128-row tile):
+// chunk by chunk (4 stages each), the next chunk's words loaded while the
+// current one is decoded.  Returns false on abort.
+template <int MODE, int F>
+__device__ bool pf_dq_unit(const PfParams& p, PfShared& sh, uint8_t* stages, const PfUnit& U, int d, int lane,
+                           int g, const uint32_t* xo, uint32_t lane_off, int& gstep) {
+    using Cfg = PfCfg<MODE>;
+    const int K = MODE == 0 ? p.H : p.I;
+    const long long rgb = (long long)(K / 32) * 16 * rfx_block_bytes(F);   // row-group stream bytes
+    const int cb = 128 * rfx_block_bytes(F);                              // full chunk bytes
+    const long long rg = (long long)U.rt * (PF_BM / 16) + d;
+    const uint8_t* m0;
+    const uint8_t* m1 = nullptr;
+    if (MODE == 0) {
+        m0 = (U.e >= 0 ? p.gate + (long long)U.e * p.sg : p.shg) + rg * rgb;
+        m1 = (U.e >= 0 ? p.up + (long long)U.e * p.su : p.shu) + rg * rgb;
+    } else {
+        m0 = (U.e >= 0 ? p.down + (long long)U.e * p.sd : p.shd) + rg * rgb;
+    }
+    const int nch = K / 256;
+    PfChunk<F> c0, c1;
+    c0.load(m0, lane, g);
+    if (MODE == 0) c1.load(m1, lane, g);
+    for (int ch = 0; ch < nch; ++ch) {
+        PfChunk<F> n0, n1;
+        if (ch + 1 < nch) {
+            n0.load(m0 + (long long)(ch + 1) * cb, lane, g);
+            if (MODE == 0) n1.load(m1 + (long long)(ch + 1) * cb, lane, g);
+        }
+        uint32_t s0[4 * F], s1[4 * F];
+        pf_shift<F>(c0, s0);
+        if (MODE == 0) pf_shift<F>(c1, s1);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            const int s = gstep % Cfg::NS;
+            const uint32_t ph = (uint32_t)(gstep / Cfg::NS) & 1u;
+            if (!pf_wait_warp(sh, p.ctrl, &sh.empty[s], ph ^ 1u)) return false;
+            const uint32_t base = smem_u32(stages + (size_t)s * Cfg::STAGE) + lane_off;
+            switch (kk) {
+                case 0: pf_decode_kstep<F, 0>(c0, s0, base, xo); break;
+                case 1: pf_decode_kstep<F, 1>(c0, s0, base, xo); break;
+                case 2: pf_decode_kstep<F, 2>(c0, s0, base, xo); break;
+                default: pf_decode_kstep<F, 3>(c0, s0, base, xo); break;
+            }
+            if (MODE == 0) {
+                switch (kk) {
+                    case 0: pf_decode_kstep<F, 0>(c1, s1, base + Cfg::A_MAT, xo); break;
+                    case 1: pf_decode_kstep<F, 1>(c1, s1, base + Cfg::A_MAT, xo); break;
+                    case 2: pf_decode_kstep<F, 2>(c1, s1, base + Cfg::A_MAT, xo); break;
+                    default: pf_decode_kstep<F, 3>(c1, s1, base + Cfg::A_MAT, xo); break;
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.fullA[s]);
+            ++gstep;
+        }
+        if (ch + 1 < nch) {
+            c0 = n0;
+            if (MODE == 0) c1 = n1;
+        }
+    }
+    return true;
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
+
+__device__ __forceinline__ uint16_t f32_to_bf16_rne(float v) {
+    uint16_t r;
+    asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(r) : "f"(v));
+    return r;
+}
+
+// Persistent grouped GEMM, one CTA per SM, units handed out round-robin in
+// the tiles' order (heaviest first).  MODE 0: gate/up + SwiGLU -> hp.  MODE 1:
+// down, y[token] += w * d.
+template <int MODE>
+__global__ void __launch_bounds__(PF_THREADS, 1)
+    pf_gemm_kernel(const PfParams p, const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmX) {
+    using Cfg = PfCfg<MODE>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+    uint8_t* stages = smem_raw + pad;
+    PfShared& sh = *reinterpret_cast<PfShared*>(stages + (size_t)Cfg::NS * Cfg::STAGE);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < Cfg::NS; ++s) {
+            mbar_init(&sh.fullA[s], N_DQ);
+            mbar_init(&sh.fullB[s], 1);
+            mbar_init(&sh.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sh.acc_full[b], 1);
+            mbar_init(&sh.acc_empty[b], N_EPI);
+        }
+        mbar_init(&sh.drain, 1);
+        sh.abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == W_MMA) {
+        __syncwarp();
+        tmem_alloc(&sh.tmem, TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == W_PROD && lane == 0) {
+        tma_prefetch_desc(&tmB);
+        if (MODE == 0) tma_prefetch_desc(&tmX);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sh.tmem;
+
+    const int RT = (MODE == 0 ? p.I : p.H) / PF_BM;
+    const int nk = (MODE == 0 ? p.H : p.I) / PF_BK;
+    const int nunits = (int)p.ctrl[PF_CTRL_NTILES] * RT;
+    const int rk = p.T * p.k;
+
+    if (warp == W_PROD) {
+        if (lane == 0) {
+            const uint64_t pol = policy_evict_last();
+            int gstep = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
+                const PfUnit U = pf_unit(p, u, RT);
+                const bool shx = MODE == 0 && U.e < 0;
+                const void* tm = shx ? (const void*)&tmX : (const void*)&tmB;
+                const int rbase = shx ? U.row0 - rk : U.row0;
+                const int n16 = U.npad / 16;
+                for (int ks = 0; ks < nk; ++ks, ++gstep) {
+                    const int s = gstep % Cfg::NS;
+                    const uint32_t ph = (uint32_t)(gstep / Cfg::NS) & 1u;
+                    if (!pf_wait(sh, p.ctrl, &sh.empty[s], ph ^ 1u)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&sh.fullB[s], (uint32_t)n16 * (16 * PF_BK * 2));
+                    uint8_t* dst = stages + (size_t)s * Cfg::STAGE + Cfg::A_BYTES;
+                    for (int j = 0; j < n16; ++j)
+                        tma_load_2d(dst + j * (16 * PF_BK * 2), tm, ks * PF_BK, rbase + 16 * j, &sh.fullB[s], pol);
+                }
+            }
+            // no copy may still be landing when the CTA exits
+            for (int i = 1; i <= Cfg::NS && gstep - i >= 0; ++i) {
+                const int gi = gstep - i;
+                (void)pf_wait(sh, p.ctrl, &sh.fullB[gi % Cfg::NS], (uint32_t)(gi / Cfg::NS) & 1u);
+            }
+        }
+    } else if (warp == W_MMA) {
+        if (lane == 0) {
+            int gstep = 0, i = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x, ++i) {
+                const PfUnit U = pf_unit(p, u, RT);
+                const uint32_t idesc = idesc_bf16_m128((uint32_t)U.npad);
+                const int b = i % Cfg::NACC, use = i / Cfg::NACC;
+                if (!pf_wait(sh, p.ctrl, &sh.acc_empty[b], (uint32_t)(use & 1) ^ 1u)) break;
+                tc_fence_after();
+                const uint32_t dacc = tmem + (uint32_t)(b * 256);
+                for (int ks = 0; ks < nk; ++ks, ++gstep) {
+                    const int s = gstep % Cfg::NS;
+                    const uint32_t ph = (uint32_t)(gstep / Cfg::NS) & 1u;
+                    if (!pf_wait(sh, p.ctrl, &sh.fullA[s], ph) || !pf_wait(sh, p.ctrl, &sh.fullB[s], ph)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t aaddr = smem_u32(stages + (size_t)s * Cfg::STAGE);
+                    const uint32_t baddr = aaddr + Cfg::A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < PF_BK / 16; ++kk) {
+                        const uint32_t acc = (ks | kk) != 0;
+                        const uint64_t bdesc = sw128_desc(baddr + kk * 32);
+                        tc_mma_bf16(dacc, sw128_desc(aaddr + kk * 32), bdesc, idesc, acc);
+                        if (MODE == 0) tc_mma_bf16(tmem + 256, sw128_desc(aaddr + Cfg::A_MAT + kk * 32), bdesc, idesc, acc);
+                    }
+                    tc_commit(&sh.empty[s]);
+                }
+                if (ok) tc_commit(&sh.acc_full[b]);
+            }
+            tc_commit(&sh.drain);
+            (void)pf_wait(sh, p.ctrl, &sh.drain, 0);
+        }
+    } else if (warp < W_EPI0) {
+        const int d = warp - W_DQ0;
+        const int g = lane >> 2, t = lane & 3;
+        uint32_t xo[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) xo[c] = (uint32_t)((c ^ g) << 4);
+        const uint32_t lane_off = (uint32_t)(2 * d * 1024 + g * 128 + 4 * t);
+        int gstep = 0;
+        for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+            const PfUnit U = pf_unit(p, u, RT);
+            const int f = MODE == 0 ? (U.e >= 0 ? p.fA : p.fsA) : (U.e >= 0 ? p.fB : p.fsB);
+            bool ok;
+            if (f == 2) ok = pf_dq_unit<MODE, 2>(p, sh, stages, U, d, lane, g, xo, lane_off, gstep);
+            else if (f == 3) ok = pf_dq_unit<MODE, 3>(p, sh, stages, U, d, lane, g, xo, lane_off, gstep);
+            else ok = pf_dq_unit<MODE, 4>(p, sh, stages, U, d, lane, g, xo, lane_off, gstep);
+            if (!ok) break;
+        }
+    } else {
+        const int q = warp & 3;   // tensor-memory lane quarter this warp may read
+        const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
+        int i = 0;
+        for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++i) {
+            const PfUnit U = pf_unit(p, u, RT);
+            const int b = i % Cfg::NACC, use = i / Cfg::NACC;
+            if (!pf_wait_warp(sh, p.ctrl, &sh.acc_full[b], (uint32_t)use & 1u)) break;
+            tc_fence_after();
+            const int row = U.rt * PF_BM + 32 * q + lane;
+            if (MODE == 0) {
+                uint16_t* hrow = p.hp + row;
+                for (int c0 = 0; c0 < U.n; c0 += 16) {
+                    uint32_t gv[16], uv[16];
+                    tmem_ld16(tq + (uint32_t)c0, gv);
+                    tmem_ld16(tq + 256u + (uint32_t)c0, uv);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        if (c0 + j < U.n)
+                            hrow[(long long)(U.row0 + c0 + j) * p.I] =
+                                f32_to_bf16_rne(silu_mul(__uint_as_float(gv[j]), __uint_as_float(uv[j])));
+                }
+            } else {
+                float* ycol = p.y + row;
+                const uint32_t tb = tq + (uint32_t)(b * 256);
+                for (int c0 = 0; c0 < U.n; c0 += 32) {
+                    int tok = 0;
+                    float wv = 0.f;
+                    if (c0 + lane < U.n) {
+                        const int pr = U.row0 + c0 + lane;
+                        tok = U.e >= 0 ? p.perm_tok[pr] : pr - rk;
+                        wv = U.e >= 0 ? p.perm_w[pr] : 1.0f;
+                    }
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf) {
+                        if (c0 + 16 * hf >= U.n) break;
+                        uint32_t dv[16];
+                        tmem_ld16(tb + (uint32_t)(c0 + 16 * hf), dv);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int c = c0 + 16 * hf + j;
+                            const int tk = __shfl_sync(0xffffffffu, tok, 16 * hf + j);
+                            const float ww = __shfl_sync(0xffffffffu, wv, 16 * hf + j);
+                            if (c < U.n) atomicAdd(ycol + (long long)tk * p.H, ww * __uint_as_float(dv[j]));
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.acc_empty[b]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == W_MMA) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------- host side ---
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    }
+    return fn;
+}
+
+// bf16 matrix [rows][cols] (row stride cols * 2 bytes), boxes of 64 columns x
+// 16 rows in the 128-byte swizzled layout; rows beyond `rows` read as zero.
+bool make_tmap(CUtensorMap* m, const void* base, long long rows, long long cols) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    const cuuint32_t box[2] = {PF_BK, 16};
+    const cuuint32_t es[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+size_t pf_gemm_smem_bytes(int mode) {
+    const size_t st = mode == 0 ? (size_t)PfCfg<0>::NS * PfCfg<0>::STAGE : (size_t)PfCfg<1>::NS * PfCfg<1>::STAGE;
+    return 1024 + st + sizeof(PfShared);
+}
+
+cudaError_t pf_launch(const PfParams& p, int sms, cudaStream_t stream) {
+    static bool attr_done[64] = {false};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 64 && !attr_done[dev]) {
+        e = cudaFuncSetAttribute(pf_gemm_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)pf_gemm_smem_bytes(0));
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(pf_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)pf_gemm_smem_bytes(1));
+        if (e != cudaSuccess) return e;
+        attr_done[dev] = true;
+    }
+    CUtensorMap tm_xp, tm_x, tm_h;
+    const long long rk = (long long)p.T * p.k;
+    if (!make_tmap(&tm_xp, p.xp, rk, p.H) || !make_tmap(&tm_x, p.x, p.T, p.H) ||
+        !make_tmap(&tm_h, p.hp, rk + p.T, p.I))
+        return cudaErrorInvalidValue;
+    const int n = p.T * p.k;
+    const int gb = (p.E + 7) / 8;
+    pf_count_kernel<<<gb, 256, 0, stream>>>(p.idx, n, p.E, p.cnt, p.ctrl);
+    pf_place_kernel<<<gb, 256, 0, stream>>>(p.idx, p.wts, n, p.k, p.E, p.cnt, p.perm_tok, p.perm_w);
+    pf_tiles_kernel<<<1, 1024, 0, stream>>>(p);
+    pf_gather_kernel<<<sms * 4, 256, 0, stream>>>(p);
+    pf_gemm_kernel<0><<<sms, PF_THREADS, pf_gemm_smem_bytes(0), stream>>>(p, tm_xp, tm_x);
+    pf_gemm_kernel<1><<<sms, PF_THREADS, pf_gemm_smem_bytes(1), stream>>>(p, tm_h, tm_h);
+    return cudaGetLastError();
+}
+
+}  // namespace rfx

@@ -184,7 +184,8 @@ int moe_layer_create(const moe_layer_desc* d, moe_layer** out);
 void moe_layer_destroy(moe_layer* layer);
 
 /*
- * Device workspace bytes moe_ffn_forward needs for T token columns.  The
+ * Device workspace bytes moe_ffn_forward needs for T token columns (T > 8:
+ * the prefill workspace, moe_prefill_workspace_bytes).  The
  * workspace holds counters, the SwiGLU intermediate and per-expert partial
  * outputs; it must be zeroed once (rfx_ws_init) before its first use and may
  * then be reused by successive calls on the same stream.  Calls that overlap
@@ -210,6 +211,8 @@ int rfx_ws_status(void* ws, void* stream);
  * x: device bf16 bits [T][H].  idx: device int32 [T][k], distinct per row,
  * in [0, E).  w: device fp32 [T][k].  y: device fp32 [T][H].
  * Limits: 1 <= T <= 8 (decode / verify), H % 32 == 0, I % 32 == 0, k <= 8.
+ * T > 8 runs moe_ffn_prefill instead (bf16 operands; its own limits and
+ * workspace size).
  * One cooperative launch of one CTA per SM (all CTAs resident at once: the
  * gate/up, down and combine phases meet at two grid barriers whose counters
  * live in the workspace).  A workspace must not be used by two calls that
@@ -218,6 +221,54 @@ int rfx_ws_status(void* ws, void* stream);
  */
 int moe_ffn_forward(const moe_layer* layer, const void* x, int T, const int32_t* idx, const float* w,
                     float* y, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Prefill: the same MoE FFN for many tokens as a grouped GEMM on the tcgen05
+ * tensor cores ([AI] "Lucebox 的优化三板斧" and [MZ] "MoE 专家并行" for the
+ * layer; the page pair's prefill runs the experts as dense contractions).
+ *   y[t] = sum_j w[t][j] * down~_{e_tj}( bf16( silu(gate~ x[t]) * (up~ x[t]) ) )
+ *          + the same for the shared expert (weight 1)
+ * where M~ is the matrix with every weight rounded once to bf16 (nearest
+ * even) from its exact value level * scale, the inner products are
+ * accumulated in fp32, and bf16() rounds the SwiGLU output to nearest even.
+ * The rows routed to each expert are grouped (expert ascending, inside an
+ * expert the entries (t, j) in ascending t*k + j order); every packed block of
+ * an expert is read and dequantised into shared memory once per 128-row tile
+ * and group of up to 256 of its tokens.  The k + 1 contributions to y[t] are
+ * added with fp32 atomics, so their order (and the last bit of y) may vary
+ * from run to run.
+ * x: device bf16 bits [T][H], 16-byte aligned.  idx: device int32 [T][k] in
+ * [0, E) (an id repeated within a row counts twice; an id out of range sets
+ * the device error flag and the entry is skipped).  w: device fp32 [T][k].
+ * y: device fp32 [T][H], 16-byte aligned (overwritten).  ws: 256-byte
+ * aligned, moe_prefill_workspace_bytes(layer, T) bytes; only the error flag
+ * word needs zeroing (rfx_ws_init) and calls on one workspace must not
+ * overlap on the GPU.  Limits: 1 <= T <= 65536, H % 256 == 0, I % 256 == 0.
+ * Six launches on `stream` (grouping, gather, gate/up GEMM, down GEMM); can
+ * be captured in a CUDA graph.  Returns RFX_EUNSUPPORTED outside the limits.
+ */
+size_t moe_prefill_workspace_bytes(const moe_layer* layer, int T);
+int moe_ffn_prefill(const moe_layer* layer, const void* x, int T, const int32_t* idx, const float* w, float* y,
+                    void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Device pointers into a prefill workspace after a moe_ffn_prefill call (for
+ * inspection and tests): counts[E] tokens per routed expert; row_token and
+ * row_weight [routed_rows] the token and combine weight of each grouped row
+ * (rows of expert e start at the sum of the counts of the experts below e;
+ * only the first sum(counts) rows are defined); h bf16 bits [h_rows][I], the
+ * SwiGLU output of every grouped row, then of the shared expert for tokens
+ * 0..T-1 (rows routed_rows + t).
+ */
+typedef struct {
+    const int32_t* counts;
+    const int32_t* row_token;
+    const float* row_weight;
+    const void* h;
+    int64_t routed_rows;
+    int64_t h_rows;
+} moe_prefill_ws_view;
+int moe_prefill_view(const moe_layer* layer, int T, const void* ws, moe_prefill_ws_view* view);
 
 /*
  * moe_ffn_forward_static -- the same MoE FFN as moe_ffn_forward for callers

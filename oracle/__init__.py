@@ -62,6 +62,8 @@ def lib():
             L.oracle_dequant.argtypes = [i32, vp, vp, i64, i64, vp]
             L.oracle_gemv.restype = i32
             L.oracle_gemv.argtypes = [i32, vp, vp, i64, i64, vp, i32, vp, vp]
+            L.oracle_gemv_bf16w.restype = i32
+            L.oracle_gemv_bf16w.argtypes = [i32, vp, vp, i64, i64, vp, i32, vp, vp]
             L.oracle_router_topk.restype = i32
             L.oracle_router_topk.argtypes = [vp, i64, i32, i32, vp, vp]
             L.oracle_expert_ffn.restype = i32
@@ -131,16 +133,33 @@ def dequant(m: Mat) -> np.ndarray:
     return W
 
 
-def gemv(m: Mat, x: np.ndarray):
-    """y[q][N] = W x for x[q][K] (fp64); returns (y, mag) with mag = |W||x|."""
+def gemv(m: Mat, x: np.ndarray, bf16_weights: bool = False):
+    """y[q][N] = W x for x[q][K] (fp64); returns (y, mag) with mag = |W||x|.
+    bf16_weights: every weight rounded once to bf16 first (prefill operands)."""
     x = _c(np.atleast_2d(x), np.float64)
     N, K = m.shape
     q = x.shape[0]
     assert x.shape[1] == K
     y = np.empty((q, N), dtype=np.float64)
     mag = np.empty((q, N), dtype=np.float64)
-    _check(lib().oracle_gemv(m.bits, _p(m.codes), _p(m.scales), N, K, _p(x), q, _p(y), _p(mag)), "gemv")
+    fn = lib().oracle_gemv_bf16w if bf16_weights else lib().oracle_gemv
+    _check(fn(m.bits, _p(m.codes), _p(m.scales), N, K, _p(x), q, _p(y), _p(mag)), "gemv")
     return y, mag
+
+
+def group_rows(idx: np.ndarray, w: np.ndarray, E: int):
+    """Prefill grouping of the routed entries: counts[E] tokens per expert and,
+    for the rows grouped by ascending expert with the entries (t, j) of one
+    expert in ascending t*k + j order (a stable sort of the flattened ids),
+    the token, the combine weight and the entry t*k + j of every row.  Ids
+    outside [0, E) get no row."""
+    idx = np.asarray(idx, dtype=np.int64)
+    T, k = idx.shape
+    flat = idx.reshape(-1)
+    ok = (flat >= 0) & (flat < E)
+    order = np.argsort(np.where(ok, flat, E), kind="stable")[: int(ok.sum())]
+    counts = np.bincount(flat[ok], minlength=E).astype(np.int32)
+    return counts, (order // k).astype(np.int32), np.asarray(w, dtype=np.float64).reshape(-1)[order], order
 
 
 def router_topk(logits: np.ndarray, k: int):

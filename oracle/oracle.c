@@ -149,6 +149,18 @@ int oracle_gemv(int bits, const uint8_t* codes, const void* scales, int64_t N, i
 }
 
 /*
+ * The same with every weight rounded to bf16 (nearest even) from its exact
+ * value: the prefill operand precision (the prefill of the pages' model runs
+ * the experts as dense contractions on bf16 tensor-core operands, here
+ * dequantised once per weight and rounded once).
+ */
+int oracle_gemv_bf16w(int bits, const uint8_t* codes, const void* scales, int64_t N, int64_t K,
+                      const double* x, int q, double* y, double* mag) {
+    oracle_mat M = {bits, codes, scales};
+    return gemv_mat(&M, N, K, x, q, y, mag, 1);
+}
+
+/*
  * Router: for each token the k largest logits, ordered by descending value,
  * equal values by ascending expert index; w = softmax over the k selected.
  */

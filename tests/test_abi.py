@@ -192,7 +192,10 @@ def test_layer_create_validation():
     d.stride_down = rfx.rfx_packed_bytes(3, 4096, 2048)
     h = rfx.moe_layer_create(d)
     assert h
-    assert rfx.moe_ffn_workspace_bytes(h, 4) > 0 and rfx.moe_ffn_workspace_bytes(h, 9) == 0
+    assert rfx.moe_ffn_workspace_bytes(h, 4) > 0
+    # T > 8 takes the prefill path and its workspace
+    assert rfx.moe_ffn_workspace_bytes(h, 9) == rfx.moe_prefill_workspace_bytes(h, 9) > 0
+    assert rfx.moe_prefill_workspace_bytes(h, 0) == 0 and rfx.moe_ffn_workspace_bytes(h, 0) == 0
     rfx.moe_layer_destroy(h)
     for field, val in (("H", 100), ("k", 9), ("f_up", 3), ("stride_down", 16), ("gate", 8), ("E", 2000)):
         bad = rfx.moe_layer_desc.from_buffer_copy(d)

@@ -264,6 +264,41 @@ def test_prefill_operand_rounding_matches_torch_bf16():
     np.testing.assert_allclose(d, Wd @ href, rtol=1e-12, atol=1e-14)
 
 
+def test_gemv_bf16_weights_matches_torch_rounding():
+    for bits in (2, 3, 4):
+        m = rand_mat(bits, 24, 96, 40 + bits)
+        x = synth.bf16_to_f64(synth.x_bf16(11, 0, 3, 96))
+        bf = torch.tensor(dense_by_table(bits, m.codes, m.scales), dtype=torch.float32).to(torch.bfloat16)
+        W = bf.to(torch.float64).numpy()
+        y, mag = oracle.gemv(m, x, bf16_weights=True)
+        np.testing.assert_allclose(y, x @ W.T, rtol=1e-13, atol=1e-13 * np.abs(mag).max())
+        np.testing.assert_allclose(mag, np.abs(x) @ np.abs(W).T, rtol=1e-13)
+        # the rounding is not a no-op for the fp16-scaled formats
+        if bits != 4:
+            assert not np.array_equal(W, dense_by_table(bits, m.codes, m.scales))
+
+
+def test_group_rows_brute_force():
+    rng = np.random.default_rng(9)
+    T, k, E = 37, 3, 11
+    idx = rng.integers(0, E, size=(T, k))
+    idx[4, 1] = idx[4, 0]            # a repeated id counts twice
+    idx[6, 2] = E + 3                # out of range: no row
+    w = rng.random((T, k))
+    counts, tok, wt, ent = oracle.group_rows(idx, w, E)
+    rows = []
+    for e in range(E):               # expert by expert, entries in row-major order
+        for t in range(T):
+            for j in range(k):
+                if idx[t, j] == e:
+                    rows.append((t, w[t, j], t * k + j))
+    assert counts.tolist() == [sum(1 for t in range(T) for j in range(k) if idx[t, j] == e) for e in range(E)]
+    assert tok.tolist() == [r[0] for r in rows]
+    assert np.array_equal(wt, np.array([r[1] for r in rows]))
+    assert ent.tolist() == [r[2] for r in rows]
+    assert counts.sum() == T * k - 1
+
+
 def test_rms_bf16_closed_form_and_torch():
     assert np.array_equal(oracle.rms_bf16(np.full(16, -3.0)), -np.ones(16))
     y = np.random.default_rng(2).standard_normal(4096) * 7.0
