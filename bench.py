@@ -55,6 +55,9 @@ def parse():
     ap.add_argument("--stack", action="store_true",
                     help="also time the 43-layer stack (98.7 GB of distinct layers resident, FFN only)")
     ap.add_argument("--stack-only", action="store_true", help="time only the 43-layer stack")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill grouped-GEMM measurement")
+    ap.add_argument("--prefill-only", action="store_true", help="time only the prefill (T = 2048 and 8192)")
+    ap.add_argument("--prefill-steps", type=int, default=20)
     return ap.parse_args()
 
 
@@ -305,6 +308,77 @@ def measure_stack(qs, steps: int, warmup: int, dev):
     return out
 
 
+PREFILL_TS = (2048, 8192)
+PREFILL_BATCHES = 2
+
+
+def measure_prefill(T: int, steps: int, warmup: int, dev, layer=None):
+    """Prefill of one full-size layer: T tokens, Zipf(1.1)-skewed top-6 routing,
+    each step = router top-k + moe_ffn_prefill (grouping, gather, gate/up
+    tcgen05 GEMM + SwiGLU, down tcgen05 GEMM + combine), captured in a graph.
+    Two seeded token batches alternate (x is T x 8 KB; the touched experts'
+    packed weights, about 1 GB, are larger than L2)."""
+    import numpy as np
+    import torch
+    import synth
+    import block_quantized_moe_rocmfpx_b200 as rfx
+    from synth.layers import SynthLayer
+    lay = layer if layer is not None else SynthLayer(SEED, 0, H, I, E, K_TOP, device=dev)
+    ml = lay.moe_layer()
+    nb = PREFILL_BATCHES
+    logits_h = [synth.logits(SEED, 0, 100000 + b * T, T, E, ZIPF_S) for b in range(nb)]
+    x_h = [synth.x_bf16(SEED, 100000 + b * T, T, H) for b in range(nb)]
+    logits = [torch.from_numpy(a).to(dev) for a in logits_h]
+    x = [torch.from_numpy(a).view(torch.bfloat16).to(dev) for a in x_h]
+    idx = [torch.empty((T, K_TOP), dtype=torch.int32, device=dev) for _ in range(nb)]
+    w = [torch.empty((T, K_TOP), dtype=torch.float32, device=dev) for _ in range(nb)]
+    y = [torch.empty((T, H), dtype=torch.float32, device=dev) for _ in range(nb)]
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(t):
+        b = t % nb
+        rfx.moe_router_topk(logits[b], K_TOP, idx[b], w[b], stream)
+        ml.prefill(x[b], idx[b], w[b], y[b], stream)
+
+    with torch.cuda.stream(stream):
+        for t in range(3):
+            step(t)
+        torch.cuda.synchronize()
+        gw = graph_of(step, max(3, warmup), stream)
+        g = graph_of(step, steps, stream)
+        gw.replay()
+        torch.cuda.synchronize()
+        ms = time_graph(g, stream)
+        del g, gw
+    st = ml.prefill_status()
+    # algorithmic work: 2 flops per multiply-add of the real (unpadded) rows;
+    # bytes: packed blocks of the touched experts + the shared expert, x and y
+    flops = 2.0 * T * (K_TOP + 1) * 3 * H * I
+    nbytes = []
+    for b in range(nb):
+        top = np.argsort(-logits_h[b], axis=-1, kind="stable")[:, :K_TOP]
+        nbytes.append(lay.union_bytes(top.ravel()) + T * (2 * H + 4 * H))
+    per_step_bytes = sum(nbytes) / nb
+    t_step = ms / steps / 1e3
+    peak_tf, peak_gbs = peaks_tensor(), peaks()[0]
+    t_min = max(flops / (peak_tf * 1e12), per_step_bytes / (peak_gbs * 1e9))
+    return {"T": T, "ms_per_step": ms / steps, "value": T / t_step, "unit": "tokens/s",
+            "tflops": flops / t_step / 1e12, "flops_per_step": flops, "bytes_per_step": per_step_bytes,
+            "roofline": {"bound": "tensor" if flops / (peak_tf * 1e12) >= per_step_bytes / (peak_gbs * 1e9)
+                         else "hbm", "peak_tflops": peak_tf, "peak_gbs": peak_gbs, "t_min_ms": t_min * 1e3,
+                         "frac": t_min / t_step, "peak_kind": "bf16_tflops_sustained of measured"},
+            "device_status": st, "steps": steps}
+
+
+def peaks_tensor() -> float:
+    """Measured sustained dense bf16 TFLOP/s (a kernel timed inside a long step)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops_sustained"])
+    except Exception:
+        return 1400.0
+
+
 def rfx_status_of(ws) -> int:
     import block_quantized_moe_rocmfpx_b200 as rfx
     return rfx.rfx_ws_status(ws)
@@ -450,6 +524,12 @@ def main():
             print(json.dumps({"metric": "43-layer MoE-FFN stack decode tokens/s (FFN only)", "stack": st,
                               "peak_gbs": peak, "peak_kind": peak_kind}), flush=True)
         return
+    if args.prefill_only:
+        pf = [measure_prefill(T, args.prefill_steps, max(3, args.warmup), dev) for T in PREFILL_TS]
+        if rank == 0:
+            print(json.dumps({"metric": "MoE-FFN prefill grouped GEMM tokens/s and TFLOP/s", "prefill": pf}),
+                  flush=True)
+        return
     r1 = measure(1, args.steps, max(3, args.warmup), dev, rank, world, True, not args.no_e2e, args.copies)
     r4 = r1 if args.only_q1 else measure(4, args.steps, max(3, args.warmup), dev, rank, world, False, False,
                                          args.copies)
@@ -468,6 +548,9 @@ def main():
         e2e_ms = reduce_max(r1["e2e"]["steps"] / r1["e2e"]["value"] * 1e3)
         e2e_v = dict(r1["e2e"])
         e2e_v["value"] = world * r1["e2e"]["steps"] / (e2e_ms / 1e3)
+    pf = None
+    if not args.no_prefill:
+        pf = [measure_prefill(T, args.prefill_steps, max(3, args.warmup), dev) for T in PREFILL_TS]
     if world > 1:
         dist.barrier()
     if rank == 0:
@@ -498,6 +581,7 @@ def main():
             "gpu_launches": 2 * args.steps,
             "clocks": r1["clocks"],
             "device_status": {"q1": r1["status"], "q4": r4["status"]},
+            "prefill": pf,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -38,14 +38,17 @@ namespace {
 
 constexpr long long PF_WAIT = 1000000000LL;   // SM clocks before a wait gives up (about half a second)
 
-constexpr int PF_THREADS = 448;
+constexpr int PF_THREADS = 480;
 constexpr int W_PROD = 0;     // TMA loads of the token rows (B operand)
 constexpr int W_MMA = 1;      // tensor-memory allocation and MMA issue
 constexpr int W_DQ0 = 2;      // 8 dequantisation warps, one 16-row group each
 constexpr int N_DQ = 8;
 constexpr int W_EPI0 = 10;    // 4 epilogue warps, one tensor-memory lane quarter each
 constexpr int N_EPI = 4;
+constexpr int W_PLOAD = 14;   // bulk copies of the packed weight chunks
 constexpr uint32_t TMEM_COLS = 512;
+constexpr int CB_MAX = 128 * 17;   // bytes of the largest full chunk (FP4)
+constexpr int PF_BOX_ROWS = 64;    // token rows per TMA box (the B stage holds 256)
 
 template <int MODE>
 struct PfCfg {
@@ -53,22 +56,33 @@ struct PfCfg {
     static constexpr int A_MAT = PF_BM * PF_BK * 2;                // 16 KB bf16 per matrix
     static constexpr int A_BYTES = NMAT * A_MAT;
     static constexpr int B_BYTES = PF_TILE_N * PF_BK * 2;          // 32 KB bf16
-    static constexpr int STAGE = A_BYTES + B_BYTES;
-    static constexpr int NS = MODE == 0 ? 3 : 4;                    // pipeline stages
+    static constexpr int NSA = MODE == 0 ? 2 : 3;                   // dequantised A stages
+    static constexpr int NSB = 4;                                   // token-row B stages
+    static constexpr int P_STAGE = NMAT * (PF_BM / 16) * CB_MAX;   // packed chunks of one 256-wide k block
+    static constexpr int NP = MODE == 0 ? 1 : 2;                    // packed stages (released once in registers)
     static constexpr int NACC = MODE == 0 ? 1 : 2;                  // accumulator buffers of 256 (MODE 1) columns
-    static_assert(A_MAT % 1024 == 0 && STAGE % 1024 == 0, "swizzle atoms must stay 1024-byte aligned");
+    // header (barriers) in the first 1 KB, then the rings from a 1024-byte boundary
+    static constexpr size_t RINGS = (size_t)NSA * A_BYTES + (size_t)NSB * B_BYTES + (size_t)NP * P_STAGE;
+    static constexpr size_t SMEM = 1024 + RINGS;
+    static_assert(A_MAT % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms must stay 1024-byte aligned");
+    static_assert(P_STAGE % 128 == 0, "bulk-copy destinations must stay 16-byte aligned");
+    static_assert(SMEM <= 232448, "more shared memory than a B200 block may have");
 };
 
 struct PfShared {
     uint64_t fullA[4];    // dequantised A tiles written (8 warp arrivals)
+    uint64_t emptyA[4];   // A stage read by the tensor cores (MMA commit)
     uint64_t fullB[4];    // B rows landed (1 arrival + bytes)
-    uint64_t empty[4];    // stage read by the tensor cores (MMA commit)
+    uint64_t emptyB[4];   // B stage read by the tensor cores (MMA commit)
+    uint64_t pfull[2];    // packed chunks landed (1 arrival + bytes)
+    uint64_t pempty[2];   // packed chunks taken into registers (8 warp arrivals)
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t drain;
     uint32_t tmem;
     volatile int abort;
 };
+static_assert(sizeof(PfShared) <= 1024, "barrier header must fit the first 1 KB");
 
 __device__ __forceinline__ void pf_set_error(uint32_t* ctrl, uint32_t bits) { atomicOr(ctrl + PF_CTRL_ERR, bits); }
 
@@ -132,6 +146,7 @@ __global__ void __launch_bounds__(256) pf_place_kernel(const int32_t* __restrict
                                                        const int32_t* __restrict__ cnt,
                                                        int32_t* __restrict__ perm_tok, float* __restrict__ perm_w) {
     __shared__ int32_t s_idx[GRP_CHUNK];
+    __shared__ float s_w[GRP_CHUNK];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int e = blockIdx.x * 8 + warp;
     int off = 0;
@@ -142,7 +157,10 @@ __global__ void __launch_bounds__(256) pf_place_kernel(const int32_t* __restrict
     for (int base = 0; base < n; base += GRP_CHUNK) {
         const int m = min(GRP_CHUNK, n - base);
         __syncthreads();
-        for (int i = threadIdx.x; i < m; i += 256) s_idx[i] = idx[base + i];
+        for (int i = threadIdx.x; i < m; i += 256) {
+            s_idx[i] = idx[base + i];
+            s_w[i] = wts[base + i];
+        }
         __syncthreads();
         if (e >= E) continue;
         for (int i0 = 0; i0 < m; i0 += 32) {
@@ -152,7 +170,7 @@ __global__ void __launch_bounds__(256) pf_place_kernel(const int32_t* __restrict
             if (hit) {
                 const int pos = off + run + __popc(b & ((1u << lane) - 1u));
                 perm_tok[pos] = (base + i) / k;
-                perm_w[pos] = wts[base + i];
+                perm_w[pos] = s_w[i];
             }
             run += __popc(b);
         }
@@ -267,7 +285,8 @@ __device__ __forceinline__ PfUnit pf_unit(const PfParams& p, int u, int RT) {
 }
 
 // One lane's share of a full chunk (8 tiles = 16 rows x 256 k) of one matrix,
-// read straight from global memory (slab-major layout, include/rfx.h).
+// read from the packed stage in shared memory (slab-major layout,
+// include/rfx.h: every 128-bit load of the warp reads 512 contiguous bytes).
 template <int F>
 struct PfChunk {
     static constexpr int NW = 4 * F;
@@ -277,22 +296,15 @@ struct PfChunk {
     __device__ __forceinline__ void load(const uint8_t* ch, int lane, int g) {
 #pragma unroll
         for (int i = 0; i < F; ++i) {
-            const uint4 v = ldg_stream(ch + (i * 32 + lane) * 16);
+            const uint4 v = lds128(ch + (i * 32 + lane) * 16);
             wd[4 * i] = v.x; wd[4 * i + 1] = v.y; wd[4 * i + 2] = v.z; wd[4 * i + 3] = v.w;
         }
         constexpr int CODE = Plane<F>::CODE_BYTES;
 #pragma unroll
         for (int i = 0; i < NSW / 4; ++i) {
-            const uint4 v = ldg_stream(ch + CODE + (i * 8 + g) * 16);
+            const uint4 v = lds128(ch + CODE + (i * 8 + g) * 16);
             sc[4 * i] = v.x; sc[4 * i + 1] = v.y; sc[4 * i + 2] = v.z; sc[4 * i + 3] = v.w;
         }
-    }
-    static __device__ __forceinline__ uint4 ldg_stream(const uint8_t* p) {
-        uint4 v;
-        asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                     : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                     : "l"(p));
-        return v;
     }
 };
 
@@ -348,44 +360,39 @@ __device__ __forceinline__ void pf_shift(const PfChunk<F>& c, uint32_t* sh) {
     for (int i = 0; i < 4 * F; ++i) sh[i] = c.wd[i] >> SH;
 }
 
+struct PfRings {
+    uint8_t* a;         // NSA x dequantised A tiles (gate, up / down)
+    uint8_t* b;         // NSB x token-row B tiles
+    uint8_t* pk;        // NP x packed chunks [matrix][row-group][CB_MAX]
+};
+
 // Dequantisation of one unit by one warp (row-group d of the 128-row tile):
-// chunk by chunk (4 stages each), the next chunk's words loaded while the
-// current one is decoded.  Returns false on abort.
+// per 256-wide k block, the packed chunk(s) come from the packed ring into
+// registers (the ring slot is released at once), then 4 stages of A are
+// written.  Returns false on abort.
 template <int MODE, int F>
-__device__ bool pf_dq_unit(const PfParams& p, PfShared& sh, uint8_t* stages, const PfUnit& U, int d, int lane,
-                           int g, const uint32_t* xo, uint32_t lane_off, int& gstep) {
+__device__ bool pf_dq_unit(const PfParams& p, PfShared& sh, const PfRings& R, int nk, int d, int lane, int g,
+                           const uint32_t* xo, uint32_t lane_off, int& gstep, int& pstep) {
     using Cfg = PfCfg<MODE>;
-    const int K = MODE == 0 ? p.H : p.I;
-    const long long rgb = (long long)(K / 32) * 16 * rfx_block_bytes(F);   // row-group stream bytes
-    const int cb = 128 * rfx_block_bytes(F);                              // full chunk bytes
-    const long long rg = (long long)U.rt * (PF_BM / 16) + d;
-    const uint8_t* m0;
-    const uint8_t* m1 = nullptr;
-    if (MODE == 0) {
-        m0 = (U.e >= 0 ? p.gate + (long long)U.e * p.sg : p.shg) + rg * rgb;
-        m1 = (U.e >= 0 ? p.up + (long long)U.e * p.su : p.shu) + rg * rgb;
-    } else {
-        m0 = (U.e >= 0 ? p.down + (long long)U.e * p.sd : p.shd) + rg * rgb;
-    }
-    const int nch = K / 256;
-    PfChunk<F> c0, c1;
-    c0.load(m0, lane, g);
-    if (MODE == 0) c1.load(m1, lane, g);
-    for (int ch = 0; ch < nch; ++ch) {
-        PfChunk<F> n0, n1;
-        if (ch + 1 < nch) {
-            n0.load(m0 + (long long)(ch + 1) * cb, lane, g);
-            if (MODE == 0) n1.load(m1 + (long long)(ch + 1) * cb, lane, g);
-        }
+    const int nch = nk / 4;
+    for (int ch = 0; ch < nch; ++ch, ++pstep) {
+        const int pc = pstep % Cfg::NP;
+        if (!pf_wait_warp(sh, p.ctrl, &sh.pfull[pc], (uint32_t)(pstep / Cfg::NP) & 1u)) return false;
+        const uint8_t* pst = R.pk + (size_t)pc * Cfg::P_STAGE + (size_t)d * CB_MAX;
+        PfChunk<F> c0, c1;
+        c0.load(pst, lane, g);
+        if (MODE == 0) c1.load(pst + (PF_BM / 16) * CB_MAX, lane, g);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.pempty[pc]);
         uint32_t s0[4 * F], s1[4 * F];
         pf_shift<F>(c0, s0);
         if (MODE == 0) pf_shift<F>(c1, s1);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-            const int s = gstep % Cfg::NS;
-            const uint32_t ph = (uint32_t)(gstep / Cfg::NS) & 1u;
-            if (!pf_wait_warp(sh, p.ctrl, &sh.empty[s], ph ^ 1u)) return false;
-            const uint32_t base = smem_u32(stages + (size_t)s * Cfg::STAGE) + lane_off;
+            const int s = gstep % Cfg::NSA;
+            const uint32_t ph = (uint32_t)(gstep / Cfg::NSA) & 1u;
+            if (!pf_wait_warp(sh, p.ctrl, &sh.emptyA[s], ph ^ 1u)) return false;
+            const uint32_t base = smem_u32(R.a + (size_t)s * Cfg::A_BYTES) + lane_off;
             switch (kk) {
                 case 0: pf_decode_kstep<F, 0>(c0, s0, base, xo); break;
                 case 1: pf_decode_kstep<F, 1>(c0, s0, base, xo); break;
@@ -405,20 +412,22 @@ __device__ bool pf_dq_unit(const PfParams& p, PfShared& sh, uint8_t* stages, con
             if (lane == 0) mbar_arrive(&sh.fullA[s]);
             ++gstep;
         }
-        if (ch + 1 < nch) {
-            c0 = n0;
-            if (MODE == 0) c1 = n1;
-        }
     }
     return true;
 }
 
-__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
+// silu(g) * u with the hardware exponential and a fast reciprocal (relative
+// error a few fp32 ulps, far below the bf16 rounding that follows).
+__device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
 
 __device__ __forceinline__ uint16_t f32_to_bf16_rne(float v) {
     uint16_t r;
     asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(r) : "f"(v));
     return r;
+}
+
+__device__ __forceinline__ int pf_fmt(const PfParams& p, int mode, int e) {
+    return mode == 0 ? (e >= 0 ? p.fA : p.fsA) : (e >= 0 ? p.fB : p.fsB);
 }
 
 // Persistent grouped GEMM, one CTA per SM, units handed out round-robin in
@@ -428,17 +437,34 @@ template <int MODE>
 __global__ void __launch_bounds__(PF_THREADS, 1)
     pf_gemm_kernel(const PfParams p, const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmX) {
     using Cfg = PfCfg<MODE>;
-    extern __shared__ uint8_t smem_raw[];
-    const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
-    uint8_t* stages = smem_raw + pad;
-    PfShared& sh = *reinterpret_cast<PfShared*>(stages + (size_t)Cfg::NS * Cfg::STAGE);
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    PfShared& sh = *reinterpret_cast<PfShared*>(smem_raw);
+    // rings from the first 1024-byte boundary after the header; the launch
+    // reserves 1 KB for the header, so the block's dynamic shared memory must
+    // start 1024-byte aligned (checked below)
+    const uint32_t off = ((smem_u32(smem_raw) + (uint32_t)sizeof(PfShared) + 1023u) & ~1023u) - smem_u32(smem_raw);
+    PfRings R;
+    R.a = smem_raw + off;
+    R.b = R.a + (size_t)Cfg::NSA * Cfg::A_BYTES;
+    R.pk = R.b + (size_t)Cfg::NSB * Cfg::B_BYTES;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (off > 1024u) {   // the rings would overrun the allocation: report and do nothing
+        if (threadIdx.x == 0) pf_set_error(p.ctrl, MOE_ERR_TIMEOUT);
+        return;
+    }
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < Cfg::NS; ++s) {
+        for (int s = 0; s < Cfg::NSA; ++s) {
             mbar_init(&sh.fullA[s], N_DQ);
+            mbar_init(&sh.emptyA[s], 1);
+        }
+        for (int s = 0; s < Cfg::NSB; ++s) {
             mbar_init(&sh.fullB[s], 1);
-            mbar_init(&sh.empty[s], 1);
+            mbar_init(&sh.emptyB[s], 1);
+        }
+        for (int s = 0; s < Cfg::NP; ++s) {
+            mbar_init(&sh.pfull[s], 1);
+            mbar_init(&sh.pempty[s], N_DQ);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sh.acc_full[b], 1);
@@ -463,7 +489,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     const uint32_t tmem = sh.tmem;
 
     const int RT = (MODE == 0 ? p.I : p.H) / PF_BM;
-    const int nk = (MODE == 0 ? p.H : p.I) / PF_BK;
+    const int K = MODE == 0 ? p.H : p.I;
+    const int nk = K / PF_BK;
     const int nunits = (int)p.ctrl[PF_CTRL_NTILES] * RT;
     const int rk = p.T * p.k;
 
@@ -477,21 +504,61 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 const bool shx = MODE == 0 && U.e < 0;
                 const void* tm = shx ? (const void*)&tmX : (const void*)&tmB;
                 const int rbase = shx ? U.row0 - rk : U.row0;
-                const int n16 = U.npad / 16;
+                const int nbox = (U.npad + PF_BOX_ROWS - 1) / PF_BOX_ROWS;
                 for (int ks = 0; ks < nk; ++ks, ++gstep) {
-                    const int s = gstep % Cfg::NS;
-                    const uint32_t ph = (uint32_t)(gstep / Cfg::NS) & 1u;
-                    if (!pf_wait(sh, p.ctrl, &sh.empty[s], ph ^ 1u)) { ok = false; break; }
-                    mbar_arrive_expect_tx(&sh.fullB[s], (uint32_t)n16 * (16 * PF_BK * 2));
-                    uint8_t* dst = stages + (size_t)s * Cfg::STAGE + Cfg::A_BYTES;
-                    for (int j = 0; j < n16; ++j)
-                        tma_load_2d(dst + j * (16 * PF_BK * 2), tm, ks * PF_BK, rbase + 16 * j, &sh.fullB[s], pol);
+                    const int s = gstep % Cfg::NSB;
+                    const uint32_t ph = (uint32_t)(gstep / Cfg::NSB) & 1u;
+                    if (!pf_wait(sh, p.ctrl, &sh.emptyB[s], ph ^ 1u)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&sh.fullB[s], (uint32_t)nbox * (PF_BOX_ROWS * PF_BK * 2));
+                    uint8_t* dst = R.b + (size_t)s * Cfg::B_BYTES;
+                    for (int j = 0; j < nbox; ++j)
+                        tma_load_2d(dst + j * (PF_BOX_ROWS * PF_BK * 2), tm, ks * PF_BK, rbase + PF_BOX_ROWS * j,
+                                    &sh.fullB[s], pol);
                 }
             }
             // no copy may still be landing when the CTA exits
-            for (int i = 1; i <= Cfg::NS && gstep - i >= 0; ++i) {
+            for (int i = 1; i <= Cfg::NSB && gstep - i >= 0; ++i) {
                 const int gi = gstep - i;
-                (void)pf_wait(sh, p.ctrl, &sh.fullB[gi % Cfg::NS], (uint32_t)(gi / Cfg::NS) & 1u);
+                (void)pf_wait(sh, p.ctrl, &sh.fullB[gi % Cfg::NSB], (uint32_t)(gi / Cfg::NSB) & 1u);
+            }
+        }
+    } else if (warp == W_PLOAD) {
+        if (lane == 0) {
+            const uint64_t pol = policy_evict_first();
+            int pstep = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
+                const PfUnit U = pf_unit(p, u, RT);
+                const int f = pf_fmt(p, MODE, U.e);
+                const long long rgb = (long long)(K / 32) * 16 * rfx_block_bytes(f);
+                const uint32_t cb = 128u * (uint32_t)rfx_block_bytes(f);
+                const uint8_t* m0;
+                const uint8_t* m1 = nullptr;
+                if (MODE == 0) {
+                    m0 = U.e >= 0 ? p.gate + (long long)U.e * p.sg : p.shg;
+                    m1 = U.e >= 0 ? p.up + (long long)U.e * p.su : p.shu;
+                } else {
+                    m0 = U.e >= 0 ? p.down + (long long)U.e * p.sd : p.shd;
+                }
+                const long long rg0 = (long long)U.rt * (PF_BM / 16);
+                for (int ch = 0; ch < nk / 4; ++ch, ++pstep) {
+                    const int pc = pstep % Cfg::NP;
+                    if (!pf_wait(sh, p.ctrl, &sh.pempty[pc], ((uint32_t)(pstep / Cfg::NP) & 1u) ^ 1u)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&sh.pfull[pc], (uint32_t)Cfg::NMAT * (PF_BM / 16) * cb);
+                    uint8_t* dst = R.pk + (size_t)pc * Cfg::P_STAGE;
+                    for (int m = 0; m < Cfg::NMAT; ++m) {
+                        const uint8_t* src = (m == 0 ? m0 : m1) + rg0 * rgb + (long long)ch * cb;
+                        for (int rg = 0; rg < PF_BM / 16; ++rg)
+                            bulk_g2s(dst + (m * (PF_BM / 16) + rg) * CB_MAX, src + rg * rgb, cb, &sh.pfull[pc], pol);
+                    }
+                }
+            }
+            for (int i = 1; i <= Cfg::NP && pstep - i >= 0; ++i) {
+                const int pi = pstep - i;
+                (void)pf_wait(sh, p.ctrl, &sh.pfull[pi % Cfg::NP], (uint32_t)(pi / Cfg::NP) & 1u);
             }
         }
     } else if (warp == W_MMA) {
@@ -506,15 +573,15 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 tc_fence_after();
                 const uint32_t dacc = tmem + (uint32_t)(b * 256);
                 for (int ks = 0; ks < nk; ++ks, ++gstep) {
-                    const int s = gstep % Cfg::NS;
-                    const uint32_t ph = (uint32_t)(gstep / Cfg::NS) & 1u;
-                    if (!pf_wait(sh, p.ctrl, &sh.fullA[s], ph) || !pf_wait(sh, p.ctrl, &sh.fullB[s], ph)) {
+                    const int sa = gstep % Cfg::NSA, sb = gstep % Cfg::NSB;
+                    if (!pf_wait(sh, p.ctrl, &sh.fullA[sa], (uint32_t)(gstep / Cfg::NSA) & 1u) ||
+                        !pf_wait(sh, p.ctrl, &sh.fullB[sb], (uint32_t)(gstep / Cfg::NSB) & 1u)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t aaddr = smem_u32(stages + (size_t)s * Cfg::STAGE);
-                    const uint32_t baddr = aaddr + Cfg::A_BYTES;
+                    const uint32_t aaddr = smem_u32(R.a + (size_t)sa * Cfg::A_BYTES);
+                    const uint32_t baddr = smem_u32(R.b + (size_t)sb * Cfg::B_BYTES);
 #pragma unroll
                     for (int kk = 0; kk < PF_BK / 16; ++kk) {
                         const uint32_t acc = (ks | kk) != 0;
@@ -522,7 +589,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                         tc_mma_bf16(dacc, sw128_desc(aaddr + kk * 32), bdesc, idesc, acc);
                         if (MODE == 0) tc_mma_bf16(tmem + 256, sw128_desc(aaddr + Cfg::A_MAT + kk * 32), bdesc, idesc, acc);
                     }
-                    tc_commit(&sh.empty[s]);
+                    tc_commit(&sh.emptyA[sa]);
+                    tc_commit(&sh.emptyB[sb]);
                 }
                 if (ok) tc_commit(&sh.acc_full[b]);
             }
@@ -536,14 +604,14 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
 #pragma unroll
         for (int c = 0; c < 8; ++c) xo[c] = (uint32_t)((c ^ g) << 4);
         const uint32_t lane_off = (uint32_t)(2 * d * 1024 + g * 128 + 4 * t);
-        int gstep = 0;
+        int gstep = 0, pstep = 0;
         for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
             const PfUnit U = pf_unit(p, u, RT);
-            const int f = MODE == 0 ? (U.e >= 0 ? p.fA : p.fsA) : (U.e >= 0 ? p.fB : p.fsB);
+            const int f = pf_fmt(p, MODE, U.e);
             bool ok;
-            if (f == 2) ok = pf_dq_unit<MODE, 2>(p, sh, stages, U, d, lane, g, xo, lane_off, gstep);
-            else if (f == 3) ok = pf_dq_unit<MODE, 3>(p, sh, stages, U, d, lane, g, xo, lane_off, gstep);
-            else ok = pf_dq_unit<MODE, 4>(p, sh, stages, U, d, lane, g, xo, lane_off, gstep);
+            if (f == 2) ok = pf_dq_unit<MODE, 2>(p, sh, R, nk, d, lane, g, xo, lane_off, gstep, pstep);
+            else if (f == 3) ok = pf_dq_unit<MODE, 3>(p, sh, R, nk, d, lane, g, xo, lane_off, gstep, pstep);
+            else ok = pf_dq_unit<MODE, 4>(p, sh, R, nk, d, lane, g, xo, lane_off, gstep, pstep);
             if (!ok) break;
         }
     } else {
@@ -631,13 +699,13 @@ EncodeTiledFn encode_fn() {
 }
 
 // bf16 matrix [rows][cols] (row stride cols * 2 bytes), boxes of 64 columns x
-// 16 rows in the 128-byte swizzled layout; rows beyond `rows` read as zero.
+// 64 rows in the 128-byte swizzled layout; rows beyond `rows` read as zero.
 bool make_tmap(CUtensorMap* m, const void* base, long long rows, long long cols) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-    const cuuint32_t box[2] = {PF_BK, 16};
+    const cuuint32_t box[2] = {PF_BK, PF_BOX_ROWS};
     const cuuint32_t es[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -646,10 +714,7 @@ bool make_tmap(CUtensorMap* m, const void* base, long long rows, long long cols)
 
 }  // namespace
 
-size_t pf_gemm_smem_bytes(int mode) {
-    const size_t st = mode == 0 ? (size_t)PfCfg<0>::NS * PfCfg<0>::STAGE : (size_t)PfCfg<1>::NS * PfCfg<1>::STAGE;
-    return 1024 + st + sizeof(PfShared);
-}
+size_t pf_gemm_smem_bytes(int mode) { return mode == 0 ? PfCfg<0>::SMEM : PfCfg<1>::SMEM; }
 
 cudaError_t pf_launch(const PfParams& p, int sms, cudaStream_t stream) {
     static bool attr_done[64] = {false};
