@@ -39,13 +39,13 @@ namespace {
 constexpr long long PF_WAIT = 1000000000LL;   // SM clocks before a wait gives up (about half a second)
 
 constexpr int PF_THREADS = 480;
-constexpr int W_PROD = 0;     // TMA loads of the token rows (B operand)
-constexpr int W_MMA = 1;      // tensor-memory allocation and MMA issue
-constexpr int W_DQ0 = 2;      // 8 dequantisation warps, one 16-row group each
+constexpr int W_PROD = 0;     // TMA loads of the token rows (B operand); hands out the units
+constexpr int W_MMA = 1;      // tensor-memory allocation; first MMA issuer
+constexpr int W_MMA2 = 2;     // second MMA issuer
+constexpr int W_DQ0 = 3;      // 8 dequantisation warps, one 16-row group each
 constexpr int N_DQ = 8;
-constexpr int W_EPI0 = 10;    // 4 epilogue warps, one tensor-memory lane quarter each
+constexpr int W_EPI0 = 11;    // 4 epilogue warps, one tensor-memory lane quarter each (warp % 4)
 constexpr int N_EPI = 4;
-constexpr int W_PLOAD = 14;   // bulk copies of the packed weight chunks
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int CB_MAX = 128 * 17;   // bytes of the largest full chunk (FP4)
 constexpr int PF_BOX_ROWS = 64;    // token rows per TMA box (the B stage holds 256)
@@ -56,29 +56,34 @@ struct PfCfg {
     static constexpr int A_MAT = PF_BM * PF_BK * 2;                // 16 KB bf16 per matrix
     static constexpr int A_BYTES = NMAT * A_MAT;
     static constexpr int B_BYTES = PF_TILE_N * PF_BK * 2;          // 32 KB bf16
-    static constexpr int NSA = MODE == 0 ? 2 : 3;                   // dequantised A stages
-    static constexpr int NSB = 4;                                   // token-row B stages
-    static constexpr int P_STAGE = NMAT * (PF_BM / 16) * CB_MAX;   // packed chunks of one 256-wide k block
-    static constexpr int NP = MODE == 0 ? 1 : 2;                    // packed stages (released once in registers)
+    static constexpr int NS = MODE == 0 ? 3 : 4;                    // stages of (dequantised A, token-row B)
+    static constexpr int P_WARP = NMAT * CB_MAX;                    // one dequantisation warp's packed chunk(s)
+    static constexpr int P_STAGE = (PF_BM / 16) * P_WARP;
     static constexpr int NACC = MODE == 0 ? 1 : 2;                  // accumulator buffers of 256 (MODE 1) columns
+    // MODE 0: issuer 0 runs the gate MMAs and issuer 1 the up MMAs of every
+    // stage; MODE 1: issuer 0 the even and issuer 1 the odd stages
+    static constexpr int EMPTY_ARRIVALS = MODE == 0 ? 2 : 1;
     // header (barriers) in the first 1 KB, then the rings from a 1024-byte boundary
-    static constexpr size_t RINGS = (size_t)NSA * A_BYTES + (size_t)NSB * B_BYTES + (size_t)NP * P_STAGE;
+    static constexpr size_t RINGS = (size_t)NS * (A_BYTES + B_BYTES) + (size_t)P_STAGE;
     static constexpr size_t SMEM = 1024 + RINGS;
     static_assert(A_MAT % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms must stay 1024-byte aligned");
     static_assert(P_STAGE % 128 == 0, "bulk-copy destinations must stay 16-byte aligned");
     static_assert(SMEM <= 232448, "more shared memory than a B200 block may have");
 };
 
+constexpr int UQ = 4;                       // unit queue slots
+constexpr int UQ_READERS = 2 + N_DQ + N_EPI;  // MMA issuers, dequantisation and epilogue warps
+
 struct PfShared {
-    uint64_t fullA[4];    // dequantised A tiles written (8 warp arrivals)
-    uint64_t emptyA[4];   // A stage read by the tensor cores (MMA commit)
-    uint64_t fullB[4];    // B rows landed (1 arrival + bytes)
-    uint64_t emptyB[4];   // B stage read by the tensor cores (MMA commit)
-    uint64_t pfull[2];    // packed chunks landed (1 arrival + bytes)
-    uint64_t pempty[2];   // packed chunks taken into registers (8 warp arrivals)
+    uint64_t full[4];     // stage ready: A written (8 warp arrivals) and B landed (1 arrival + bytes)
+    uint64_t empty[4];    // stage read by the tensor cores (MMA commits)
+    uint64_t first[2];    // MODE 1: the unit's first (zeroing) MMA has been issued
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
+    uint64_t uq_full[UQ];    // unit id published (producer)
+    uint64_t uq_empty[UQ];   // unit id read by every other role
     uint64_t drain;
+    volatile int uq[UQ];
     uint32_t tmem;
     volatile int abort;
 };
@@ -100,6 +105,18 @@ __device__ __noinline__ bool pf_wait(PfShared& sh, uint32_t* ctrl, uint64_t* bar
             return false;
         }
     }
+}
+
+// Bounded wait that does not give up on an abort: used before the CTA exits,
+// so that no copy or MMA of this CTA is still writing its memory.
+__device__ __noinline__ bool pf_wait_drain(uint32_t* ctrl, uint64_t* bar, uint32_t parity) {
+    const long long t0 = clock64();
+    while (!mbar_try_wait_sleep(bar, parity, 20000u))
+        if (clock64() - t0 > PF_WAIT) {
+            pf_set_error(ctrl, MOE_ERR_TIMEOUT);
+            return false;
+        }
+    return true;
 }
 
 // Whole-warp wait: every lane acquires; the outcome is made uniform.
@@ -245,6 +262,8 @@ __global__ void __launch_bounds__(1024) pf_tiles_kernel(PfParams p) {
     if (tid == 0) {
         p.ctrl[PF_CTRL_NTILES] = (uint32_t)(nts + nt_total);
         p.ctrl[PF_CTRL_ROWS] = (uint32_t)rows;
+        p.ctrl[PF_CTRL_NEXT0] = 0;
+        p.ctrl[PF_CTRL_NEXT1] = 0;
     }
 }
 
@@ -361,57 +380,93 @@ __device__ __forceinline__ void pf_shift(const PfChunk<F>& c, uint32_t* sh) {
 }
 
 struct PfRings {
-    uint8_t* a;         // NSA x dequantised A tiles (gate, up / down)
-    uint8_t* b;         // NSB x token-row B tiles
-    uint8_t* pk;        // NP x packed chunks [matrix][row-group][CB_MAX]
+    uint8_t* a;         // NS x dequantised A tiles (gate, up / down)
+    uint8_t* b;         // NS x token-row B tiles
+    uint8_t* pk;        // per dequantisation warp: its packed chunk(s) [matrix][CB_MAX]
 };
 
-// Dequantisation of one unit by one warp (row-group d of the 128-row tile):
-// per 256-wide k block, the packed chunk(s) come from the packed ring into
-// registers (the ring slot is released at once), then 4 stages of A are
-// written.  Returns false on abort.
+// Where the packed chunk(s) of (unit, 256-wide k block) of one row-group come from.
+struct PfSrc {
+    const uint8_t* m0;
+    const uint8_t* m1;
+    long long rgb;      // row-group stream bytes
+    int cb;             // chunk bytes
+    int f;
+};
+
+__device__ __forceinline__ PfSrc pf_src(const PfParams& p, int mode, const PfUnit& U, int d) {
+    PfSrc S;
+    S.f = mode == 0 ? (U.e >= 0 ? p.fA : p.fsA) : (U.e >= 0 ? p.fB : p.fsB);
+    const int K = mode == 0 ? p.H : p.I;
+    S.rgb = (long long)(K / 32) * 16 * rfx_block_bytes(S.f);
+    S.cb = 128 * rfx_block_bytes(S.f);
+    const long long off = ((long long)U.rt * (PF_BM / 16) + d) * S.rgb;
+    if (mode == 0) {
+        S.m0 = (U.e >= 0 ? p.gate + (long long)U.e * p.sg : p.shg) + off;
+        S.m1 = (U.e >= 0 ? p.up + (long long)U.e * p.su : p.shu) + off;
+    } else {
+        S.m0 = (U.e >= 0 ? p.down + (long long)U.e * p.sd : p.shd) + off;
+        S.m1 = nullptr;
+    }
+    return S;
+}
+
+// The warp copies chunk `ch` of its row-group (both matrices in MODE 0) into
+// its slot with 16-byte asynchronous copies, one commit group per lane.
+template <int MODE>
+__device__ __forceinline__ void pf_prefetch(const PfSrc& S, int ch, uint32_t slot, int lane, uint64_t pol) {
+    const int pieces = S.cb / 16;
+    const uint8_t* s0 = S.m0 + (long long)ch * S.cb;
+    for (int i = lane; i < pieces; i += 32) cp_async16(slot + 16 * i, s0 + 16 * i, pol);
+    if (MODE == 0) {
+        const uint8_t* s1 = S.m1 + (long long)ch * S.cb;
+        for (int i = lane; i < pieces; i += 32) cp_async16(slot + CB_MAX + 16 * i, s1 + 16 * i, pol);
+    }
+    cp_async_commit();
+}
+
+// One 256-wide k block of one unit by one warp: the packed chunk(s) from the
+// warp's slot into registers, the next copy started into the freed slot, then
+// 4 stages of A written.  Returns false on abort.
 template <int MODE, int F>
-__device__ bool pf_dq_unit(const PfParams& p, PfShared& sh, const PfRings& R, int nk, int d, int lane, int g,
-                           const uint32_t* xo, uint32_t lane_off, int& gstep, int& pstep) {
+__device__ bool pf_dq_chunk(const PfParams& p, PfShared& sh, const PfRings& R, const uint8_t* slot, int lane, int g,
+                            const uint32_t* xo, uint32_t lane_off, int& gstep, const PfSrc* nsrc, int nch,
+                            uint32_t slot_s, uint64_t pol) {
     using Cfg = PfCfg<MODE>;
-    const int nch = nk / 4;
-    for (int ch = 0; ch < nch; ++ch, ++pstep) {
-        const int pc = pstep % Cfg::NP;
-        if (!pf_wait_warp(sh, p.ctrl, &sh.pfull[pc], (uint32_t)(pstep / Cfg::NP) & 1u)) return false;
-        const uint8_t* pst = R.pk + (size_t)pc * Cfg::P_STAGE + (size_t)d * CB_MAX;
-        PfChunk<F> c0, c1;
-        c0.load(pst, lane, g);
-        if (MODE == 0) c1.load(pst + (PF_BM / 16) * CB_MAX, lane, g);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sh.pempty[pc]);
-        uint32_t s0[4 * F], s1[4 * F];
-        pf_shift<F>(c0, s0);
-        if (MODE == 0) pf_shift<F>(c1, s1);
+    cp_async_wait_all();
+    __syncwarp();
+    PfChunk<F> c0, c1;
+    c0.load(slot, lane, g);
+    if (MODE == 0) c1.load(slot + CB_MAX, lane, g);
+    __syncwarp();
+    if (nsrc) pf_prefetch<MODE>(*nsrc, nch, slot_s, lane, pol);
+    uint32_t s0[4 * F], s1[4 * F];
+    pf_shift<F>(c0, s0);
+    if (MODE == 0) pf_shift<F>(c1, s1);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-            const int s = gstep % Cfg::NSA;
-            const uint32_t ph = (uint32_t)(gstep / Cfg::NSA) & 1u;
-            if (!pf_wait_warp(sh, p.ctrl, &sh.emptyA[s], ph ^ 1u)) return false;
-            const uint32_t base = smem_u32(R.a + (size_t)s * Cfg::A_BYTES) + lane_off;
-            switch (kk) {
-                case 0: pf_decode_kstep<F, 0>(c0, s0, base, xo); break;
-                case 1: pf_decode_kstep<F, 1>(c0, s0, base, xo); break;
-                case 2: pf_decode_kstep<F, 2>(c0, s0, base, xo); break;
-                default: pf_decode_kstep<F, 3>(c0, s0, base, xo); break;
-            }
-            if (MODE == 0) {
-                switch (kk) {
-                    case 0: pf_decode_kstep<F, 0>(c1, s1, base + Cfg::A_MAT, xo); break;
-                    case 1: pf_decode_kstep<F, 1>(c1, s1, base + Cfg::A_MAT, xo); break;
-                    case 2: pf_decode_kstep<F, 2>(c1, s1, base + Cfg::A_MAT, xo); break;
-                    default: pf_decode_kstep<F, 3>(c1, s1, base + Cfg::A_MAT, xo); break;
-                }
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sh.fullA[s]);
-            ++gstep;
+    for (int kk = 0; kk < 4; ++kk) {
+        const int s = gstep % Cfg::NS;
+        const uint32_t ph = (uint32_t)(gstep / Cfg::NS) & 1u;
+        if (!pf_wait_warp(sh, p.ctrl, &sh.empty[s], ph ^ 1u)) return false;
+        const uint32_t base = smem_u32(R.a + (size_t)s * Cfg::A_BYTES) + lane_off;
+        switch (kk) {
+            case 0: pf_decode_kstep<F, 0>(c0, s0, base, xo); break;
+            case 1: pf_decode_kstep<F, 1>(c0, s0, base, xo); break;
+            case 2: pf_decode_kstep<F, 2>(c0, s0, base, xo); break;
+            default: pf_decode_kstep<F, 3>(c0, s0, base, xo); break;
         }
+        if (MODE == 0) {
+            switch (kk) {
+                case 0: pf_decode_kstep<F, 0>(c1, s1, base + Cfg::A_MAT, xo); break;
+                case 1: pf_decode_kstep<F, 1>(c1, s1, base + Cfg::A_MAT, xo); break;
+                case 2: pf_decode_kstep<F, 2>(c1, s1, base + Cfg::A_MAT, xo); break;
+                default: pf_decode_kstep<F, 3>(c1, s1, base + Cfg::A_MAT, xo); break;
+            }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.full[s]);
+        ++gstep;
     }
     return true;
 }
@@ -426,13 +481,22 @@ __device__ __forceinline__ uint16_t f32_to_bf16_rne(float v) {
     return r;
 }
 
-__device__ __forceinline__ int pf_fmt(const PfParams& p, int mode, int e) {
-    return mode == 0 ? (e >= 0 ? p.fA : p.fsA) : (e >= 0 ? p.fB : p.fsB);
+// Unit i of this CTA from the queue (whole warp or a single thread); -1 ends.
+__device__ __forceinline__ int pf_take_unit(PfShared& sh, uint32_t* ctrl, int i, bool warp_wide, bool& ok) {
+    const int slot = i % UQ;
+    const uint32_t ph = (uint32_t)(i / UQ) & 1u;
+    ok = warp_wide ? pf_wait_warp(sh, ctrl, &sh.uq_full[slot], ph) : pf_wait(sh, ctrl, &sh.uq_full[slot], ph);
+    if (!ok) return -1;
+    const int u = sh.uq[slot];
+    if (warp_wide) __syncwarp();
+    if (!warp_wide || (threadIdx.x & 31) == 0) mbar_arrive(&sh.uq_empty[slot]);
+    return u;
 }
 
-// Persistent grouped GEMM, one CTA per SM, units handed out round-robin in
-// the tiles' order (heaviest first).  MODE 0: gate/up + SwiGLU -> hp.  MODE 1:
-// down, y[token] += w * d.
+// Persistent grouped GEMM, one CTA per SM.  Units (token tile, 128-row block)
+// are taken from a global counter in the tiles' order (heaviest first) by the
+// producer thread and passed to the other roles through a small queue.
+// MODE 0: gate/up + SwiGLU -> hp.  MODE 1: down, y[token] += w * d.
 template <int MODE>
 __global__ void __launch_bounds__(PF_THREADS, 1)
     pf_gemm_kernel(const PfParams p, const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmX) {
@@ -445,8 +509,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     const uint32_t off = ((smem_u32(smem_raw) + (uint32_t)sizeof(PfShared) + 1023u) & ~1023u) - smem_u32(smem_raw);
     PfRings R;
     R.a = smem_raw + off;
-    R.b = R.a + (size_t)Cfg::NSA * Cfg::A_BYTES;
-    R.pk = R.b + (size_t)Cfg::NSB * Cfg::B_BYTES;
+    R.b = R.a + (size_t)Cfg::NS * Cfg::A_BYTES;
+    R.pk = R.b + (size_t)Cfg::NS * Cfg::B_BYTES;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (off > 1024u) {   // the rings would overrun the allocation: report and do nothing
         if (threadIdx.x == 0) pf_set_error(p.ctrl, MOE_ERR_TIMEOUT);
@@ -454,23 +518,20 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     }
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < Cfg::NSA; ++s) {
-            mbar_init(&sh.fullA[s], N_DQ);
-            mbar_init(&sh.emptyA[s], 1);
-        }
-        for (int s = 0; s < Cfg::NSB; ++s) {
-            mbar_init(&sh.fullB[s], 1);
-            mbar_init(&sh.emptyB[s], 1);
-        }
-        for (int s = 0; s < Cfg::NP; ++s) {
-            mbar_init(&sh.pfull[s], 1);
-            mbar_init(&sh.pempty[s], N_DQ);
+        for (int s = 0; s < Cfg::NS; ++s) {
+            mbar_init(&sh.full[s], N_DQ + 1);
+            mbar_init(&sh.empty[s], Cfg::EMPTY_ARRIVALS);
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&sh.acc_full[b], 1);
+            mbar_init(&sh.acc_full[b], 2);
             mbar_init(&sh.acc_empty[b], N_EPI);
+            mbar_init(&sh.first[b], 1);
         }
-        mbar_init(&sh.drain, 1);
+        for (int q = 0; q < UQ; ++q) {
+            mbar_init(&sh.uq_full[q], 1);
+            mbar_init(&sh.uq_empty[q], UQ_READERS);
+        }
+        mbar_init(&sh.drain, 2);
         sh.abort = 0;
         fence_barrier_init();
     }
@@ -497,105 +558,100 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     if (warp == W_PROD) {
         if (lane == 0) {
             const uint64_t pol = policy_evict_last();
+            uint32_t* next = p.ctrl + (MODE == 0 ? PF_CTRL_NEXT0 : PF_CTRL_NEXT1);
+            // units are published one ahead of the one being loaded, so that the
+            // dequantisation warps can start fetching the next unit's weights
+            // while the current one is still in flight
+            auto publish = [&](int i, int u) -> bool {
+                const int slot = i % UQ;
+                if (!pf_wait(sh, p.ctrl, &sh.uq_empty[slot], ((uint32_t)(i / UQ) & 1u) ^ 1u)) return false;
+                sh.uq[slot] = u;
+                mbar_arrive(&sh.uq_full[slot]);
+                return true;
+            };
+            auto grab = [&]() -> int {
+                const int u = (int)atomicAdd(next, 1u);
+                return u < nunits ? u : -1;
+            };
             int gstep = 0;
-            bool ok = true;
-            for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
+            int u = grab();
+            bool ok = publish(0, u);
+            for (int i = 0; ok && u >= 0; ++i) {
+                const int un = grab();
+                if (!publish(i + 1, un)) break;
                 const PfUnit U = pf_unit(p, u, RT);
                 const bool shx = MODE == 0 && U.e < 0;
                 const void* tm = shx ? (const void*)&tmX : (const void*)&tmB;
                 const int rbase = shx ? U.row0 - rk : U.row0;
                 const int nbox = (U.npad + PF_BOX_ROWS - 1) / PF_BOX_ROWS;
                 for (int ks = 0; ks < nk; ++ks, ++gstep) {
-                    const int s = gstep % Cfg::NSB;
-                    const uint32_t ph = (uint32_t)(gstep / Cfg::NSB) & 1u;
-                    if (!pf_wait(sh, p.ctrl, &sh.emptyB[s], ph ^ 1u)) { ok = false; break; }
-                    mbar_arrive_expect_tx(&sh.fullB[s], (uint32_t)nbox * (PF_BOX_ROWS * PF_BK * 2));
+                    const int s = gstep % Cfg::NS;
+                    const uint32_t ph = (uint32_t)(gstep / Cfg::NS) & 1u;
+                    if (!pf_wait(sh, p.ctrl, &sh.empty[s], ph ^ 1u)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&sh.full[s], (uint32_t)nbox * (PF_BOX_ROWS * PF_BK * 2));
                     uint8_t* dst = R.b + (size_t)s * Cfg::B_BYTES;
                     for (int j = 0; j < nbox; ++j)
                         tma_load_2d(dst + j * (PF_BOX_ROWS * PF_BK * 2), tm, ks * PF_BK, rbase + PF_BOX_ROWS * j,
-                                    &sh.fullB[s], pol);
+                                    &sh.full[s], pol);
                 }
+                u = un;
             }
-            // no copy may still be landing when the CTA exits
-            for (int i = 1; i <= Cfg::NSB && gstep - i >= 0; ++i) {
+            // no copy may still be landing when the CTA exits: the last stages
+            // this thread filled must have completed (or the CTA aborted, and
+            // then the bounded wait gives up)
+            for (int i = 1; i <= Cfg::NS && gstep - i >= 0; ++i) {
                 const int gi = gstep - i;
-                (void)pf_wait(sh, p.ctrl, &sh.fullB[gi % Cfg::NSB], (uint32_t)(gi / Cfg::NSB) & 1u);
+                (void)pf_wait_drain(p.ctrl, &sh.full[gi % Cfg::NS], (uint32_t)(gi / Cfg::NS) & 1u);
             }
         }
-    } else if (warp == W_PLOAD) {
+    } else if (warp == W_MMA || warp == W_MMA2) {
         if (lane == 0) {
-            const uint64_t pol = policy_evict_first();
-            int pstep = 0;
-            bool ok = true;
-            for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
-                const PfUnit U = pf_unit(p, u, RT);
-                const int f = pf_fmt(p, MODE, U.e);
-                const long long rgb = (long long)(K / 32) * 16 * rfx_block_bytes(f);
-                const uint32_t cb = 128u * (uint32_t)rfx_block_bytes(f);
-                const uint8_t* m0;
-                const uint8_t* m1 = nullptr;
-                if (MODE == 0) {
-                    m0 = U.e >= 0 ? p.gate + (long long)U.e * p.sg : p.shg;
-                    m1 = U.e >= 0 ? p.up + (long long)U.e * p.su : p.shu;
-                } else {
-                    m0 = U.e >= 0 ? p.down + (long long)U.e * p.sd : p.shd;
-                }
-                const long long rg0 = (long long)U.rt * (PF_BM / 16);
-                for (int ch = 0; ch < nk / 4; ++ch, ++pstep) {
-                    const int pc = pstep % Cfg::NP;
-                    if (!pf_wait(sh, p.ctrl, &sh.pempty[pc], ((uint32_t)(pstep / Cfg::NP) & 1u) ^ 1u)) {
-                        ok = false;
-                        break;
-                    }
-                    mbar_arrive_expect_tx(&sh.pfull[pc], (uint32_t)Cfg::NMAT * (PF_BM / 16) * cb);
-                    uint8_t* dst = R.pk + (size_t)pc * Cfg::P_STAGE;
-                    for (int m = 0; m < Cfg::NMAT; ++m) {
-                        const uint8_t* src = (m == 0 ? m0 : m1) + rg0 * rgb + (long long)ch * cb;
-                        for (int rg = 0; rg < PF_BM / 16; ++rg)
-                            bulk_g2s(dst + (m * (PF_BM / 16) + rg) * CB_MAX, src + rg * rgb, cb, &sh.pfull[pc], pol);
-                    }
-                }
-            }
-            for (int i = 1; i <= Cfg::NP && pstep - i >= 0; ++i) {
-                const int pi = pstep - i;
-                (void)pf_wait(sh, p.ctrl, &sh.pfull[pi % Cfg::NP], (uint32_t)(pi / Cfg::NP) & 1u);
-            }
-        }
-    } else if (warp == W_MMA) {
-        if (lane == 0) {
-            int gstep = 0, i = 0;
-            bool ok = true;
-            for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x, ++i) {
+            const int who = warp - W_MMA;
+            int gstep = 0;
+            for (int i = 0;; ++i) {
+                bool ok;
+                const int u = pf_take_unit(sh, p.ctrl, i, false, ok);
+                if (u < 0) break;
                 const PfUnit U = pf_unit(p, u, RT);
                 const uint32_t idesc = idesc_bf16_m128((uint32_t)U.npad);
                 const int b = i % Cfg::NACC, use = i / Cfg::NACC;
                 if (!pf_wait(sh, p.ctrl, &sh.acc_empty[b], (uint32_t)(use & 1) ^ 1u)) break;
                 tc_fence_after();
-                const uint32_t dacc = tmem + (uint32_t)(b * 256);
+                // MODE 0: this issuer's own accumulator (gate or up); MODE 1: the
+                // unit's buffer, shared by both issuers
+                const uint32_t dacc = tmem + (uint32_t)((MODE == 0 ? who : b) * 256);
+                const uint32_t aoff = MODE == 0 ? (uint32_t)(who * Cfg::A_MAT) : 0u;
                 for (int ks = 0; ks < nk; ++ks, ++gstep) {
-                    const int sa = gstep % Cfg::NSA, sb = gstep % Cfg::NSB;
-                    if (!pf_wait(sh, p.ctrl, &sh.fullA[sa], (uint32_t)(gstep / Cfg::NSA) & 1u) ||
-                        !pf_wait(sh, p.ctrl, &sh.fullB[sb], (uint32_t)(gstep / Cfg::NSB) & 1u)) {
+                    if (MODE == 1 && (ks & 1) != who) continue;
+                    const int s = gstep % Cfg::NS;
+                    if (!pf_wait(sh, p.ctrl, &sh.full[s], (uint32_t)(gstep / Cfg::NS) & 1u)) {
+                        ok = false;
+                        break;
+                    }
+                    if (MODE == 1 && who == 1 && ks == 1 &&
+                        !pf_wait(sh, p.ctrl, &sh.first[b], (uint32_t)(use & 1))) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t aaddr = smem_u32(R.a + (size_t)sa * Cfg::A_BYTES);
-                    const uint32_t baddr = smem_u32(R.b + (size_t)sb * Cfg::B_BYTES);
+                    const uint32_t aaddr = smem_u32(R.a + (size_t)s * Cfg::A_BYTES) + aoff;
+                    const uint32_t baddr = smem_u32(R.b + (size_t)s * Cfg::B_BYTES);
 #pragma unroll
-                    for (int kk = 0; kk < PF_BK / 16; ++kk) {
-                        const uint32_t acc = (ks | kk) != 0;
-                        const uint64_t bdesc = sw128_desc(baddr + kk * 32);
-                        tc_mma_bf16(dacc, sw128_desc(aaddr + kk * 32), bdesc, idesc, acc);
-                        if (MODE == 0) tc_mma_bf16(tmem + 256, sw128_desc(aaddr + Cfg::A_MAT + kk * 32), bdesc, idesc, acc);
+                    for (int kk = 0; kk < PF_BK / 16; ++kk)
+                        tc_mma_bf16(dacc, sw128_desc(aaddr + kk * 32), sw128_desc(baddr + kk * 32), idesc,
+                                    (ks | kk) != 0);
+                    tc_commit(&sh.empty[s]);
+                    // the zeroing MMA is issued: the other issuer may add to the buffer
+                    if (MODE == 1 && ks == 0) {
+                        tc_fence_before();
+                        mbar_arrive(&sh.first[b]);
                     }
-                    tc_commit(&sh.emptyA[sa]);
-                    tc_commit(&sh.emptyB[sb]);
                 }
-                if (ok) tc_commit(&sh.acc_full[b]);
+                if (!ok) break;
+                tc_commit(&sh.acc_full[b]);
             }
             tc_commit(&sh.drain);
-            (void)pf_wait(sh, p.ctrl, &sh.drain, 0);
+            (void)pf_wait_drain(p.ctrl, &sh.drain, 0);
         }
     } else if (warp < W_EPI0) {
         const int d = warp - W_DQ0;
@@ -604,21 +660,51 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
 #pragma unroll
         for (int c = 0; c < 8; ++c) xo[c] = (uint32_t)((c ^ g) << 4);
         const uint32_t lane_off = (uint32_t)(2 * d * 1024 + g * 128 + 4 * t);
-        int gstep = 0, pstep = 0;
-        for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
-            const PfUnit U = pf_unit(p, u, RT);
-            const int f = pf_fmt(p, MODE, U.e);
-            bool ok;
-            if (f == 2) ok = pf_dq_unit<MODE, 2>(p, sh, R, nk, d, lane, g, xo, lane_off, gstep, pstep);
-            else if (f == 3) ok = pf_dq_unit<MODE, 3>(p, sh, R, nk, d, lane, g, xo, lane_off, gstep, pstep);
-            else ok = pf_dq_unit<MODE, 4>(p, sh, R, nk, d, lane, g, xo, lane_off, gstep, pstep);
-            if (!ok) break;
+        const uint8_t* slot = R.pk + (size_t)d * Cfg::P_WARP;
+        const uint32_t slot_s = smem_u32(slot);
+        const uint64_t pol = policy_evict_first();
+        const int nch = nk / 4;
+        int gstep = 0;
+        bool ok;
+        int u = pf_take_unit(sh, p.ctrl, 0, true, ok);
+        PfSrc cur{};
+        if (u >= 0) {
+            cur = pf_src(p, MODE, pf_unit(p, u, RT), d);
+            pf_prefetch<MODE>(cur, 0, slot_s, lane, pol);
         }
+        for (int i = 0; u >= 0; ++i) {
+            int un = -1;
+            PfSrc nxt{};
+            for (int ch = 0; ch < nch && ok; ++ch) {
+                const PfSrc* ns = nullptr;
+                int nc = 0;
+                if (ch + 1 < nch) {
+                    ns = &cur;
+                    nc = ch + 1;
+                } else {
+                    un = pf_take_unit(sh, p.ctrl, i + 1, true, ok);
+                    if (!ok) break;
+                    if (un >= 0) {
+                        nxt = pf_src(p, MODE, pf_unit(p, un, RT), d);
+                        ns = &nxt;
+                    }
+                }
+                if (cur.f == 2) ok = pf_dq_chunk<MODE, 2>(p, sh, R, slot, lane, g, xo, lane_off, gstep, ns, nc, slot_s, pol);
+                else if (cur.f == 3) ok = pf_dq_chunk<MODE, 3>(p, sh, R, slot, lane, g, xo, lane_off, gstep, ns, nc, slot_s, pol);
+                else ok = pf_dq_chunk<MODE, 4>(p, sh, R, slot, lane, g, xo, lane_off, gstep, ns, nc, slot_s, pol);
+            }
+            if (!ok) break;
+            u = un;
+            cur = nxt;
+        }
+        cp_async_wait_all();   // nothing may still be landing in the slot when the CTA exits
     } else {
         const int q = warp & 3;   // tensor-memory lane quarter this warp may read
         const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
-        int i = 0;
-        for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++i) {
+        for (int i = 0;; ++i) {
+            bool ok;
+            const int u = pf_take_unit(sh, p.ctrl, i, true, ok);
+            if (u < 0) break;
             const PfUnit U = pf_unit(p, u, RT);
             const int b = i % Cfg::NACC, use = i / Cfg::NACC;
             if (!pf_wait_warp(sh, p.ctrl, &sh.acc_full[b], (uint32_t)use & 1u)) break;

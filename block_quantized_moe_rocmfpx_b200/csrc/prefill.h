@@ -13,6 +13,8 @@
 #define PF_CTRL_ERR 2
 #define PF_CTRL_NTILES 8     // token tiles (written by the grouping)
 #define PF_CTRL_ROWS 9       // routed rows (sum of the per-expert counts)
+#define PF_CTRL_NEXT0 10     // next unit to hand out, gate/up GEMM (reset by the grouping)
+#define PF_CTRL_NEXT1 11     // next unit to hand out, down GEMM
 #define PF_CTRL_WORDS 64
 
 #define PF_TILE_N 256        // most tokens per token tile (the MMA's largest N)

@@ -143,6 +143,15 @@ __device__ __forceinline__ uint32_t deq_pair_pow2scale(uint32_t v, float K, floa
     return out;
 }
 
+// 16-byte asynchronous copy global -> shared through the load/store unit
+// (completion tracked per thread: commit a group, then wait for it).
+__device__ __forceinline__ void cp_async16(uint32_t saddr, const void* src, uint64_t policy) {
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(saddr), "l"(src), "l"(policy)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
 __device__ __forceinline__ void sts32(uint32_t saddr, uint32_t v) {
     asm volatile("st.shared.b32 [%0], %1;" ::"r"(saddr), "r"(v) : "memory");
 }
