@@ -283,6 +283,8 @@ extern "C" int moe_ffn_prefill(const moe_layer* layer, const void* x, int T, con
     uint8_t* b = (uint8_t*)ws;
     p.ctrl = (uint32_t*)(b + L.ctrl);
     p.cnt = (int32_t*)(b + L.cnt);
+    p.cnt_part = (int32_t*)(b + L.cnt_part);
+    p.off = (int32_t*)(b + L.off);
     p.perm_tok = (int32_t*)(b + L.perm_tok);
     p.perm_w = (float*)(b + L.perm_w);
     p.tiles = (int4*)(b + L.tiles);

@@ -14,11 +14,13 @@
 // memory.
 //
 // Steps (one stream, six launches):
-//   pf_count   tokens per routed expert, and the expert-id range check
+//   pf_count   tokens per routed expert in each slice of 1024 routed entries,
+//              and the expert-id range check
+//   pf_tiles   per-expert totals and first rows; token tiles of <= 256 rows:
+//              the shared expert's first, then the routed experts by
+//              descending token count (heaviest work first)
 //   pf_place   rows grouped by expert, tokens in ascending order inside an
 //              expert (stable, so the grouping is unique): token and weight
-//   pf_tiles   token tiles of <= 256 rows: the shared expert's first, then the
-//              routed experts by descending token count (heaviest work first)
 //   pf_gather  the routed rows of x copied into grouped order; y zeroed
 //   pf_gemm<0> gate/up GEMM + SwiGLU -> h (bf16), per (tile, 128-row block of I)
 //   pf_gemm<1> down GEMM, per (tile, 128-row block of H); the epilogue adds
@@ -127,70 +129,83 @@ __device__ __forceinline__ bool pf_wait_warp(PfShared& sh, uint32_t* ctrl, uint6
 
 // ----------------------------------------------------------- grouping ---
 
-constexpr int GRP_CHUNK = 2048;
+// Routed entries t*k + j are cut into slices of PF_SLICE; a grouping CTA
+// handles 8 experts (one warp each) of one slice.
+__device__ __forceinline__ void grp_stage(const int32_t* __restrict__ src, int32_t* dst, int m) {
+    for (int i = threadIdx.x; i < m; i += 256) dst[i] = src[i];
+}
 
-// cnt[e] for the 8 experts of this CTA (one warp each); CTA 0 warp 0 also
-// checks every id against [0, E).
+// cnt_part[slice][e]; the CTAs of expert block 0 also check every id against [0, E).
 __global__ void __launch_bounds__(256) pf_count_kernel(const int32_t* __restrict__ idx, int n, int E,
-                                                       int32_t* __restrict__ cnt, uint32_t* __restrict__ ctrl) {
-    __shared__ int32_t s_idx[GRP_CHUNK];
+                                                       int32_t* __restrict__ cnt_part, uint32_t* __restrict__ ctrl) {
+    __shared__ __align__(16) int32_t s_idx[PF_SLICE];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int e = blockIdx.x * 8 + warp;
+    const int base = blockIdx.y * PF_SLICE;
+    const int m = min(PF_SLICE, n - base);
+    grp_stage(idx + base, s_idx, m);
+    __syncthreads();
     int c = 0;
     bool bad = false;
-    for (int base = 0; base < n; base += GRP_CHUNK) {
-        const int m = min(GRP_CHUNK, n - base);
-        __syncthreads();
-        for (int i = threadIdx.x; i < m; i += 256) s_idx[i] = idx[base + i];
-        __syncthreads();
-        for (int i = lane; i < m; i += 32) {
-            const int v = s_idx[i];
-            c += v == e;
-            if (blockIdx.x == 0 && warp == 0) bad |= v < 0 || v >= E;
-        }
+    for (int i0 = 0; i0 < m; i0 += 128) {
+        const int i = i0 + 4 * lane;
+        const int4 v = *reinterpret_cast<const int4*>(s_idx + i);
+        const int vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (i + j < m) {
+                c += vv[j] == e;
+                if (blockIdx.x == 0 && warp == 0) bad |= vv[j] < 0 || vv[j] >= E;
+            }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
-    if (lane == 0 && e < E) cnt[e] = c;
+    if (lane == 0 && e < E) cnt_part[(long long)blockIdx.y * E + e] = c;
     if (__any_sync(0xffffffffu, bad) && lane == 0) pf_set_error(ctrl, MOE_ERR_EXPERT);
 }
 
-// Rows of expert e start at off(e) = sum of the counts of the experts below
-// it; the entries (t, j) routed to e take them in ascending entry order
-// t * k + j (ballot prefix counts inside each group of 32 entries).
+// The entries (t, j) routed to e take rows off[e] + (hits of e in the slices
+// before this one) + ..., in ascending entry order t * k + j.  Per step a warp
+// looks at 128 entries, lane L at entries 4L .. 4L+3: the hits of the lower
+// lanes (4 ballots) plus the lane's own earlier hits give each hit its row.
 __global__ void __launch_bounds__(256) pf_place_kernel(const int32_t* __restrict__ idx,
                                                        const float* __restrict__ wts, int n, int k, int E,
-                                                       const int32_t* __restrict__ cnt,
+                                                       const int32_t* __restrict__ cnt_part,
+                                                       const int32_t* __restrict__ off_e,
                                                        int32_t* __restrict__ perm_tok, float* __restrict__ perm_w) {
-    __shared__ int32_t s_idx[GRP_CHUNK];
-    __shared__ float s_w[GRP_CHUNK];
+    __shared__ __align__(16) int32_t s_idx[PF_SLICE];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int e = blockIdx.x * 8 + warp;
+    const int base = blockIdx.y * PF_SLICE;
+    const int m = min(PF_SLICE, n - base);
+    grp_stage(idx + base, s_idx, m);
+    __syncthreads();
+    if (e >= E) return;
     int off = 0;
-    for (int i = lane; i < min(e, E); i += 32) off += cnt[i];
+    for (int s = lane; s < (int)blockIdx.y; s += 32) off += cnt_part[(long long)s * E + e];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) off += __shfl_xor_sync(0xffffffffu, off, o);
-    int run = 0;
-    for (int base = 0; base < n; base += GRP_CHUNK) {
-        const int m = min(GRP_CHUNK, n - base);
-        __syncthreads();
-        for (int i = threadIdx.x; i < m; i += 256) {
-            s_idx[i] = idx[base + i];
-            s_w[i] = wts[base + i];
+    off += off_e[e];
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int i0 = 0; i0 < m; i0 += 128) {
+        const int i = i0 + 4 * lane;
+        const int4 v = *reinterpret_cast<const int4*>(s_idx + i);
+        const bool h0 = i < m && v.x == e, h1 = i + 1 < m && v.y == e;
+        const bool h2 = i + 2 < m && v.z == e, h3 = i + 3 < m && v.w == e;
+        const uint32_t b0 = __ballot_sync(0xffffffffu, h0), b1 = __ballot_sync(0xffffffffu, h1);
+        const uint32_t b2 = __ballot_sync(0xffffffffu, h2), b3 = __ballot_sync(0xffffffffu, h3);
+        if (h0 | h1 | h2 | h3) {
+            int pos = off + __popc(b0 & lt) + __popc(b1 & lt) + __popc(b2 & lt) + __popc(b3 & lt);
+            const bool hv[4] = {h0, h1, h2, h3};
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (hv[j]) {
+                    perm_tok[pos] = (base + i + j) / k;
+                    perm_w[pos] = wts[base + i + j];
+                    ++pos;
+                }
         }
-        __syncthreads();
-        if (e >= E) continue;
-        for (int i0 = 0; i0 < m; i0 += 32) {
-            const int i = i0 + lane;
-            const bool hit = i < m && s_idx[i] == e;
-            const uint32_t b = __ballot_sync(0xffffffffu, hit);
-            if (hit) {
-                const int pos = off + run + __popc(b & ((1u << lane) - 1u));
-                perm_tok[pos] = (base + i) / k;
-                perm_w[pos] = s_w[i];
-            }
-            run += __popc(b);
-        }
+        off += __popc(b0) + __popc(b1) + __popc(b2) + __popc(b3);
     }
 }
 
@@ -230,10 +245,16 @@ __global__ void __launch_bounds__(1024) pf_tiles_kernel(PfParams p) {
     __shared__ int s_cnt[1024], s_off[1024], s_ord[1024];
     __shared__ int s_ws[33];
     const int tid = threadIdx.x;
-    const int c = tid < p.E ? p.cnt[tid] : 0;
+    const int slices = (p.T * p.k + PF_SLICE - 1) / PF_SLICE;
+    int c = 0;
+    if (tid < p.E) {
+        for (int s = 0; s < slices; ++s) c += p.cnt_part[(long long)s * p.E + tid];
+        p.cnt[tid] = c;
+    }
     s_cnt[tid] = c;
     int rows = 0;
     s_off[tid] = block_excl_scan(c, s_ws, &rows);
+    if (tid < p.E) p.off[tid] = s_off[tid];
     __syncthreads();
     if (tid < p.E) {
         int r = 0;
@@ -822,10 +843,10 @@ cudaError_t pf_launch(const PfParams& p, int sms, cudaStream_t stream) {
         !make_tmap(&tm_h, p.hp, rk + p.T, p.I))
         return cudaErrorInvalidValue;
     const int n = p.T * p.k;
-    const int gb = (p.E + 7) / 8;
-    pf_count_kernel<<<gb, 256, 0, stream>>>(p.idx, n, p.E, p.cnt, p.ctrl);
-    pf_place_kernel<<<gb, 256, 0, stream>>>(p.idx, p.wts, n, p.k, p.E, p.cnt, p.perm_tok, p.perm_w);
+    const dim3 gg((p.E + 7) / 8, (n + PF_SLICE - 1) / PF_SLICE);
+    pf_count_kernel<<<gg, 256, 0, stream>>>(p.idx, n, p.E, p.cnt_part, p.ctrl);
     pf_tiles_kernel<<<1, 1024, 0, stream>>>(p);
+    pf_place_kernel<<<gg, 256, 0, stream>>>(p.idx, p.wts, n, p.k, p.E, p.cnt_part, p.off, p.perm_tok, p.perm_w);
     pf_gather_kernel<<<sms * 4, 256, 0, stream>>>(p);
     pf_gemm_kernel<0><<<sms, PF_THREADS, pf_gemm_smem_bytes(0), stream>>>(p, tm_xp, tm_x);
     pf_gemm_kernel<1><<<sms, PF_THREADS, pf_gemm_smem_bytes(1), stream>>>(p, tm_h, tm_h);

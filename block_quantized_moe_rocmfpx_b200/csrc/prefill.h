@@ -20,6 +20,7 @@
 #define PF_TILE_N 256        // most tokens per token tile (the MMA's largest N)
 #define PF_BM 128            // weight rows per tile (the MMA's M)
 #define PF_BK 64             // reduction step per pipeline stage (one 128-byte swizzle atom of bf16)
+#define PF_SLICE 1024        // routed entries per grouping CTA
 
 namespace rfx {
 
@@ -41,6 +42,8 @@ struct PfParams {
     // workspace
     uint32_t* ctrl;
     int32_t* cnt;           // [E] tokens per routed expert
+    int32_t* cnt_part;      // [slices][E] tokens per routed expert in each slice of PF_SLICE entries
+    int32_t* off;           // [E] first grouped row of each routed expert
     int32_t* perm_tok;      // [T*k] token of each routed row (rows grouped by expert, stable)
     float* perm_w;          // [T*k] combine weight of each routed row
     int4* tiles;            // token tiles {row0, n, expert (-1 = shared), 0}
@@ -50,7 +53,7 @@ struct PfParams {
 };
 
 struct PfWs {
-    size_t ctrl, cnt, perm_tok, perm_w, tiles, xp, hp, total;
+    size_t ctrl, cnt, cnt_part, off, perm_tok, perm_w, tiles, xp, hp, total;
     int max_tiles;
 };
 
@@ -62,7 +65,10 @@ inline PfWs pf_ws_layout(int T, int k, int E, int H, int I) {
                         ((size_t)T + PF_TILE_N - 1) / PF_TILE_N + 1);
     L.ctrl = 0;
     L.cnt = up(PF_CTRL_WORDS * 4);
-    L.perm_tok = L.cnt + up((size_t)E * 4);
+    const size_t slices = (R + PF_SLICE - 1) / PF_SLICE;
+    L.cnt_part = L.cnt + up((size_t)E * 4);
+    L.off = L.cnt_part + up(slices * E * 4);
+    L.perm_tok = L.off + up((size_t)E * 4);
     L.perm_w = L.perm_tok + up(R * 4);
     L.tiles = L.perm_w + up(R * 4);
     L.xp = L.tiles + up((size_t)L.max_tiles * 16);
