@@ -40,14 +40,11 @@ namespace {
 
 constexpr long long PF_WAIT = 1000000000LL;   // SM clocks before a wait gives up (about half a second)
 
-constexpr int PF_THREADS = 480;
 constexpr int W_PROD = 0;     // TMA loads of the token rows (B operand); hands out the units
 constexpr int W_MMA = 1;      // tensor-memory allocation; first MMA issuer
 constexpr int W_MMA2 = 2;     // second MMA issuer
-constexpr int W_DQ0 = 3;      // 8 dequantisation warps, one 16-row group each
-constexpr int N_DQ = 8;
-constexpr int W_EPI0 = 11;    // 4 epilogue warps, one tensor-memory lane quarter each (warp % 4)
-constexpr int N_EPI = 4;
+constexpr int W_DQ0 = 3;      // dequantisation warps (count per mode below), then
+constexpr int N_EPI = 4;      // 4 epilogue warps, one tensor-memory lane quarter each (warp % 4)
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int CB_MAX = 128 * 17;   // bytes of the largest full chunk (FP4)
 constexpr int PF_BOX_ROWS = 64;    // token rows per TMA box (the B stage holds 256)
@@ -55,12 +52,16 @@ constexpr int PF_BOX_ROWS = 64;    // token rows per TMA box (the B stage holds 
 template <int MODE>
 struct PfCfg {
     static constexpr int NMAT = MODE == 0 ? 2 : 1;                 // gate + up, or down
+    // MODE 0: two dequantisation warps per 16-row group (gate, up); MODE 1: one
+    static constexpr int N_DQ = MODE == 0 ? 16 : 8;
+    static constexpr int W_EPI0 = W_DQ0 + N_DQ;
+    static constexpr int THREADS = 32 * (W_EPI0 + N_EPI);
+    static constexpr int UQ_READERS = 2 + N_DQ + N_EPI;           // MMA issuers, dequantisation and epilogue warps
     static constexpr int A_MAT = PF_BM * PF_BK * 2;                // 16 KB bf16 per matrix
     static constexpr int A_BYTES = NMAT * A_MAT;
     static constexpr int B_BYTES = PF_TILE_N * PF_BK * 2;          // 32 KB bf16
     static constexpr int NS = MODE == 0 ? 3 : 4;                    // stages of (dequantised A, token-row B)
-    static constexpr int P_WARP = NMAT * CB_MAX;                    // one dequantisation warp's packed chunk(s)
-    static constexpr int P_STAGE = (PF_BM / 16) * P_WARP;
+    static constexpr int P_STAGE = N_DQ * CB_MAX;                   // one packed chunk per dequantisation warp
     static constexpr int NACC = MODE == 0 ? 1 : 2;                  // accumulator buffers of 256 (MODE 1) columns
     // MODE 0: issuer 0 runs the gate MMAs and issuer 1 the up MMAs of every
     // stage; MODE 1: issuer 0 the even and issuer 1 the odd stages
@@ -74,10 +75,10 @@ struct PfCfg {
 };
 
 constexpr int UQ = 4;                       // unit queue slots
-constexpr int UQ_READERS = 2 + N_DQ + N_EPI;  // MMA issuers, dequantisation and epilogue warps
 
 struct PfShared {
-    uint64_t full[4];     // stage ready: A written (8 warp arrivals) and B landed (1 arrival + bytes)
+    uint64_t full[4];     // stage ready: A written (one arrival per dequantisation warp) and B
+                          // landed (1 arrival + bytes)
     uint64_t empty[4];    // stage read by the tensor cores (MMA commits)
     uint64_t first[2];    // MODE 1: the unit's first (zeroing) MMA has been issued
     uint64_t acc_full[2];
@@ -403,85 +404,87 @@ __device__ __forceinline__ void pf_shift(const PfChunk<F>& c, uint32_t* sh) {
 struct PfRings {
     uint8_t* a;         // NS x dequantised A tiles (gate, up / down)
     uint8_t* b;         // NS x token-row B tiles
-    uint8_t* pk;        // per dequantisation warp: its packed chunk(s) [matrix][CB_MAX]
+    uint8_t* pk;        // per dequantisation warp: its packed chunk [CB_MAX]
 };
 
-// Where the packed chunk(s) of (unit, 256-wide k block) of one row-group come from.
+// Where the packed chunks of (unit, 256-wide k block) of one warp's row-group
+// and matrix come from.
 struct PfSrc {
-    const uint8_t* m0;
-    const uint8_t* m1;
-    long long rgb;      // row-group stream bytes
+    const uint8_t* m;   // the row-group's stream
     int cb;             // chunk bytes
     int f;
 };
 
-__device__ __forceinline__ PfSrc pf_src(const PfParams& p, int mode, const PfUnit& U, int d) {
+// rg = 16-row group of the unit's 128-row block, sub = the warp's half (MODE 0:
+// gate or up matrix; MODE 1: even or odd tiles of the down matrix)
+__device__ __forceinline__ PfSrc pf_src(const PfParams& p, int mode, const PfUnit& U, int rg, int sub) {
     PfSrc S;
     S.f = mode == 0 ? (U.e >= 0 ? p.fA : p.fsA) : (U.e >= 0 ? p.fB : p.fsB);
     const int K = mode == 0 ? p.H : p.I;
-    S.rgb = (long long)(K / 32) * 16 * rfx_block_bytes(S.f);
+    const long long rgb = (long long)(K / 32) * 16 * rfx_block_bytes(S.f);
     S.cb = 128 * rfx_block_bytes(S.f);
-    const long long off = ((long long)U.rt * (PF_BM / 16) + d) * S.rgb;
-    if (mode == 0) {
-        S.m0 = (U.e >= 0 ? p.gate + (long long)U.e * p.sg : p.shg) + off;
-        S.m1 = (U.e >= 0 ? p.up + (long long)U.e * p.su : p.shu) + off;
-    } else {
-        S.m0 = (U.e >= 0 ? p.down + (long long)U.e * p.sd : p.shd) + off;
-        S.m1 = nullptr;
-    }
+    const long long off = ((long long)U.rt * (PF_BM / 16) + rg) * rgb;
+    if (mode == 0)
+        S.m = (sub == 0 ? (U.e >= 0 ? p.gate + (long long)U.e * p.sg : p.shg)
+                        : (U.e >= 0 ? p.up + (long long)U.e * p.su : p.shu)) + off;
+    else
+        S.m = (U.e >= 0 ? p.down + (long long)U.e * p.sd : p.shd) + off;
     return S;
 }
 
-// The warp copies chunk `ch` of its row-group (both matrices in MODE 0) into
-// its slot with 16-byte asynchronous copies, one commit group per lane.
-template <int MODE>
+// The warp copies chunk `ch` into its slot with 16-byte asynchronous copies,
+// one commit group per lane.
 __device__ __forceinline__ void pf_prefetch(const PfSrc& S, int ch, uint32_t slot, int lane, uint64_t pol) {
     const int pieces = S.cb / 16;
-    const uint8_t* s0 = S.m0 + (long long)ch * S.cb;
-    for (int i = lane; i < pieces; i += 32) cp_async16(slot + 16 * i, s0 + 16 * i, pol);
-    if (MODE == 0) {
-        const uint8_t* s1 = S.m1 + (long long)ch * S.cb;
-        for (int i = lane; i < pieces; i += 32) cp_async16(slot + CB_MAX + 16 * i, s1 + 16 * i, pol);
-    }
+    const uint8_t* src = S.m + (long long)ch * S.cb;
+    for (int i = lane; i < pieces; i += 32) cp_async16(slot + 16 * i, src + 16 * i, pol);
     cp_async_commit();
 }
 
-// One 256-wide k block of one unit by one warp: the packed chunk(s) from the
+// One 256-wide k block of one unit by one warp: the packed chunk from the
 // warp's slot into registers, the next copy started into the freed slot, then
-// 4 stages of A written.  Returns false on abort.
+// its part of 4 stages of A written (MODE 0: both tiles of its matrix per
+// stage; MODE 1: the tile of its parity).  `base` already points at the
+// warp's matrix and row-group.  Returns false on abort.
 template <int MODE, int F>
 __device__ bool pf_dq_chunk(const PfParams& p, PfShared& sh, const PfRings& R, const uint8_t* slot, int lane, int g,
-                            const uint32_t* xo, uint32_t lane_off, int& gstep, const PfSrc* nsrc, int nch,
+                            int sub, const uint32_t* xo, uint32_t lane_off, int& gstep, const PfSrc* nsrc, int nch,
                             uint32_t slot_s, uint64_t pol) {
     using Cfg = PfCfg<MODE>;
     cp_async_wait_all();
     __syncwarp();
-    PfChunk<F> c0, c1;
+    PfChunk<F> c0;
     c0.load(slot, lane, g);
-    if (MODE == 0) c1.load(slot + CB_MAX, lane, g);
     __syncwarp();
-    if (nsrc) pf_prefetch<MODE>(*nsrc, nch, slot_s, lane, pol);
-    uint32_t s0[4 * F], s1[4 * F];
+    if (nsrc) pf_prefetch(*nsrc, nch, slot_s, lane, pol);
+    uint32_t s0[4 * F];
     pf_shift<F>(c0, s0);
-    if (MODE == 0) pf_shift<F>(c1, s1);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
         const int s = gstep % Cfg::NS;
         const uint32_t ph = (uint32_t)(gstep / Cfg::NS) & 1u;
         if (!pf_wait_warp(sh, p.ctrl, &sh.empty[s], ph ^ 1u)) return false;
         const uint32_t base = smem_u32(R.a + (size_t)s * Cfg::A_BYTES) + lane_off;
-        switch (kk) {
-            case 0: pf_decode_kstep<F, 0>(c0, s0, base, xo); break;
-            case 1: pf_decode_kstep<F, 1>(c0, s0, base, xo); break;
-            case 2: pf_decode_kstep<F, 2>(c0, s0, base, xo); break;
-            default: pf_decode_kstep<F, 3>(c0, s0, base, xo); break;
-        }
-        if (MODE == 0) {
+        if (MODE == 0 || Cfg::N_DQ == 8) {   // both tiles of the stage
             switch (kk) {
-                case 0: pf_decode_kstep<F, 0>(c1, s1, base + Cfg::A_MAT, xo); break;
-                case 1: pf_decode_kstep<F, 1>(c1, s1, base + Cfg::A_MAT, xo); break;
-                case 2: pf_decode_kstep<F, 2>(c1, s1, base + Cfg::A_MAT, xo); break;
-                default: pf_decode_kstep<F, 3>(c1, s1, base + Cfg::A_MAT, xo); break;
+                case 0: pf_decode_kstep<F, 0>(c0, s0, base, xo); break;
+                case 1: pf_decode_kstep<F, 1>(c0, s0, base, xo); break;
+                case 2: pf_decode_kstep<F, 2>(c0, s0, base, xo); break;
+                default: pf_decode_kstep<F, 3>(c0, s0, base, xo); break;
+            }
+        } else if (sub == 0) {
+            switch (kk) {
+                case 0: pf_decode_tile<F, 0>(c0, s0, base, xo); break;
+                case 1: pf_decode_tile<F, 2>(c0, s0, base, xo); break;
+                case 2: pf_decode_tile<F, 4>(c0, s0, base, xo); break;
+                default: pf_decode_tile<F, 6>(c0, s0, base, xo); break;
+            }
+        } else {
+            switch (kk) {
+                case 0: pf_decode_tile<F, 1>(c0, s0, base, xo); break;
+                case 1: pf_decode_tile<F, 3>(c0, s0, base, xo); break;
+                case 2: pf_decode_tile<F, 5>(c0, s0, base, xo); break;
+                default: pf_decode_tile<F, 7>(c0, s0, base, xo); break;
             }
         }
         fence_proxy_async_smem();
@@ -519,7 +522,7 @@ __device__ __forceinline__ int pf_take_unit(PfShared& sh, uint32_t* ctrl, int i,
 // producer thread and passed to the other roles through a small queue.
 // MODE 0: gate/up + SwiGLU -> hp.  MODE 1: down, y[token] += w * d.
 template <int MODE>
-__global__ void __launch_bounds__(PF_THREADS, 1)
+__global__ void __launch_bounds__(PfCfg<MODE>::THREADS, 1)
     pf_gemm_kernel(const PfParams p, const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmX) {
     using Cfg = PfCfg<MODE>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -540,7 +543,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < Cfg::NS; ++s) {
-            mbar_init(&sh.full[s], N_DQ + 1);
+            mbar_init(&sh.full[s], Cfg::N_DQ + 1);
             mbar_init(&sh.empty[s], Cfg::EMPTY_ARRIVALS);
         }
         for (int b = 0; b < 2; ++b) {
@@ -550,7 +553,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         }
         for (int q = 0; q < UQ; ++q) {
             mbar_init(&sh.uq_full[q], 1);
-            mbar_init(&sh.uq_empty[q], UQ_READERS);
+            mbar_init(&sh.uq_empty[q], Cfg::UQ_READERS);
         }
         mbar_init(&sh.drain, 2);
         sh.abort = 0;
@@ -674,14 +677,16 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             tc_commit(&sh.drain);
             (void)pf_wait_drain(p.ctrl, &sh.drain, 0);
         }
-    } else if (warp < W_EPI0) {
+    } else if (warp < Cfg::W_EPI0) {
         const int d = warp - W_DQ0;
+        const int rg = Cfg::N_DQ == 16 ? d >> 1 : d, sub = Cfg::N_DQ == 16 ? d & 1 : 0;
         const int g = lane >> 2, t = lane & 3;
         uint32_t xo[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) xo[c] = (uint32_t)((c ^ g) << 4);
-        const uint32_t lane_off = (uint32_t)(2 * d * 1024 + g * 128 + 4 * t);
-        const uint8_t* slot = R.pk + (size_t)d * Cfg::P_WARP;
+        // the warp's matrix (MODE 0) and row-group inside the stage's A tiles
+        const uint32_t lane_off = (uint32_t)((MODE == 0 ? sub * Cfg::A_MAT : 0) + 2 * rg * 1024 + g * 128 + 4 * t);
+        const uint8_t* slot = R.pk + (size_t)d * CB_MAX;
         const uint32_t slot_s = smem_u32(slot);
         const uint64_t pol = policy_evict_first();
         const int nch = nk / 4;
@@ -690,8 +695,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         int u = pf_take_unit(sh, p.ctrl, 0, true, ok);
         PfSrc cur{};
         if (u >= 0) {
-            cur = pf_src(p, MODE, pf_unit(p, u, RT), d);
-            pf_prefetch<MODE>(cur, 0, slot_s, lane, pol);
+            cur = pf_src(p, MODE, pf_unit(p, u, RT), rg, sub);
+            pf_prefetch(cur, 0, slot_s, lane, pol);
         }
         for (int i = 0; u >= 0; ++i) {
             int un = -1;
@@ -706,13 +711,13 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                     un = pf_take_unit(sh, p.ctrl, i + 1, true, ok);
                     if (!ok) break;
                     if (un >= 0) {
-                        nxt = pf_src(p, MODE, pf_unit(p, un, RT), d);
+                        nxt = pf_src(p, MODE, pf_unit(p, un, RT), rg, sub);
                         ns = &nxt;
                     }
                 }
-                if (cur.f == 2) ok = pf_dq_chunk<MODE, 2>(p, sh, R, slot, lane, g, xo, lane_off, gstep, ns, nc, slot_s, pol);
-                else if (cur.f == 3) ok = pf_dq_chunk<MODE, 3>(p, sh, R, slot, lane, g, xo, lane_off, gstep, ns, nc, slot_s, pol);
-                else ok = pf_dq_chunk<MODE, 4>(p, sh, R, slot, lane, g, xo, lane_off, gstep, ns, nc, slot_s, pol);
+                if (cur.f == 2) ok = pf_dq_chunk<MODE, 2>(p, sh, R, slot, lane, g, sub, xo, lane_off, gstep, ns, nc, slot_s, pol);
+                else if (cur.f == 3) ok = pf_dq_chunk<MODE, 3>(p, sh, R, slot, lane, g, sub, xo, lane_off, gstep, ns, nc, slot_s, pol);
+                else ok = pf_dq_chunk<MODE, 4>(p, sh, R, slot, lane, g, sub, xo, lane_off, gstep, ns, nc, slot_s, pol);
             }
             if (!ok) break;
             u = un;
@@ -848,8 +853,8 @@ cudaError_t pf_launch(const PfParams& p, int sms, cudaStream_t stream) {
     pf_tiles_kernel<<<1, 1024, 0, stream>>>(p);
     pf_place_kernel<<<gg, 256, 0, stream>>>(p.idx, p.wts, n, p.k, p.E, p.cnt_part, p.off, p.perm_tok, p.perm_w);
     pf_gather_kernel<<<sms * 4, 256, 0, stream>>>(p);
-    pf_gemm_kernel<0><<<sms, PF_THREADS, pf_gemm_smem_bytes(0), stream>>>(p, tm_xp, tm_x);
-    pf_gemm_kernel<1><<<sms, PF_THREADS, pf_gemm_smem_bytes(1), stream>>>(p, tm_h, tm_h);
+    pf_gemm_kernel<0><<<sms, PfCfg<0>::THREADS, pf_gemm_smem_bytes(0), stream>>>(p, tm_xp, tm_x);
+    pf_gemm_kernel<1><<<sms, PfCfg<1>::THREADS, pf_gemm_smem_bytes(1), stream>>>(p, tm_h, tm_h);
     return cudaGetLastError();
 }
 
