@@ -61,6 +61,24 @@ def parse():
     return ap.parse_args()
 
 
+def max_over_ranks(v: float, world: int, device) -> float:
+    """The largest of every rank's value (device time of the timed region):
+    the job is as slow as its slowest replica.  Every rank must call it."""
+    if world == 1:
+        return float(v)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(world: int, units_per_rank: int, ms_max: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest
+    rank's time (each rank runs an independent replica of the same work)."""
+    return world * units_per_rank / (ms_max / 1e3)
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -535,11 +553,7 @@ def main():
                                          args.copies)
 
     def reduce_max(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return max_over_ranks(v, world, dev)
 
     ms1, ms4 = reduce_max(r1["ms"]), reduce_max(r4["ms"])
     ms1f, ms4f = reduce_max(r1["ms_ffn"]), reduce_max(r4["ms_ffn"])
@@ -557,7 +571,7 @@ def main():
         peak, peak_kind = peaks()
         gbs1 = r1["bytes"] / (r1["ms_ffn"] / 1e3) / 1e9
         gbs4 = r4["bytes"] / (r4["ms_ffn"] / 1e3) / 1e9
-        value = world * args.steps / (ms1 / 1e3)
+        value = whole_job_value(world, args.steps, ms1)
         base = None if args.no_cpu_baseline else cpu_baseline(200, 1, budget_s=15.0)
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
