@@ -243,3 +243,64 @@ def test_prefill_rejects_unsupported_shapes():
         ml.prefill(torch.zeros((16, 352), dtype=torch.bfloat16, device=DEV),
                    torch.zeros((16, 3), dtype=torch.int32, device=DEV),
                    torch.zeros((16, 3), device=DEV), torch.zeros((16, 352), device=DEV))
+
+
+def _prefill_with_idx(lay, T, idx_np, w_np, xb):
+    ml = lay.moe_layer()
+    idx = to_dev(idx_np.astype(np.int32))
+    w = to_dev(w_np.astype(np.float32))
+    y = torch.full((T, lay.H), float("nan"), dtype=torch.float32, device=DEV)
+    ml.prefill(to_dev(xb, torch.bfloat16), idx, w, y)
+    assert ml.prefill_status() == rfx.RFX_OK, rfx.rfx_last_error()
+    return y.cpu().numpy(), ml.prefill_view(T)
+
+
+def _check_against_oracle(lay, idx_np, w_np, xb, y, v, tokens):
+    """Grouping bit-exact; y teacher-forced on the GPU's h; y end to end."""
+    T, k = idx_np.shape
+    counts, ent = check_grouping(idx_np, w_np.astype(np.float32), v, lay.E)
+    h_gpu = bf16_bits_to_f64(v["h"])
+    ol = OracleLayer(lay)
+    xf = synth.bf16_to_f64(xb)
+    w64 = w_np.astype(np.float32).astype(np.float64)
+    ytf, mtf = teacher_forced_y(ol, lay, idx_np, w64, ent, counts, h_gpu, list(tokens))
+    for t in tokens:
+        check_close(y[t], ytf[t], mtf[t], what=f"teacher-forced token {t}")
+        ref, _ = ol.token(xf[t], idx_np[t], w64[t], bf16_ops=True)
+        assert np.linalg.norm(y[t] - ref) / np.linalg.norm(ref) <= 3e-3
+
+
+def test_prefill_single_token():
+    # T = 1 through the prefill path: every expert tile has one row (N padded to 16)
+    lay = SynthLayer(67, 0, 512, 256, 8, 2)
+    logits = synth.logits(67, 0, 0, 1, 8, 0.0)
+    xb = synth.x_bf16(67, 0, 1, 512)
+    full_check(lay, 1, logits, xb)
+
+
+def test_prefill_every_token_on_the_same_experts():
+    # degenerate routing: all T tokens pick experts 5 and 2; the others get no
+    # rows; expert 5 and 2 each need ceil(T / 256) token tiles
+    lay = SynthLayer(71, 0, 512, 256, 8, 2)
+    T = 600
+    idx = np.tile(np.array([[5, 2]]), (T, 1))
+    w = np.tile(np.array([[0.75, 0.25]]), (T, 1))
+    xb = synth.x_bf16(71, 0, T, 512)
+    y, v = _prefill_with_idx(lay, T, idx, w, xb)
+    assert v["counts"].cpu().numpy().tolist() == [0, 0, T, 0, 0, T, 0, 0]
+    _check_against_oracle(lay, idx, w, xb, y, v, tokens=[0, 255, 256, 511, 599])
+
+
+def test_prefill_repeated_expert_in_a_row_counts_twice():
+    # an id repeated within a row makes two rows (two contributions), as the
+    # oracle's sum over the k entries does
+    lay = SynthLayer(73, 0, 512, 256, 8, 2)
+    T = 20
+    rng = np.random.default_rng(73)
+    idx = rng.integers(0, 8, size=(T, 2))
+    idx[3] = [6, 6]
+    idx[11] = [0, 0]
+    w = rng.random((T, 2)) * 0.5
+    xb = synth.x_bf16(73, 0, T, 512)
+    y, v = _prefill_with_idx(lay, T, idx, w, xb)
+    _check_against_oracle(lay, idx, w, xb, y, v, tokens=[3, 11, 0, 19])
