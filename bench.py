@@ -327,6 +327,10 @@ def measure_stack(qs, steps: int, warmup: int, dev):
 
 
 PREFILL_TS = (2048, 8192)
+# DRAM bytes (read + write) of the two prefill GEMM kernels for one T=2048 step,
+# from the ncu capture summarised in profiles/prefill_grouped_gemm_t2048.md; set
+# to None whenever those kernels change until they are captured again.
+PREFILL_TRAFFIC = {2048: 755_878_656 + 41_874_944 + 526_722_560 + 6_292_992}
 PREFILL_BATCHES = 2
 
 
@@ -384,7 +388,8 @@ def measure_prefill(T: int, steps: int, warmup: int, dev, layer=None):
             "tflops": flops / t_step / 1e12, "flops_per_step": flops, "bytes_per_step": per_step_bytes,
             "roofline": {"bound": "tensor" if flops / (peak_tf * 1e12) >= per_step_bytes / (peak_gbs * 1e9)
                          else "hbm", "peak_tflops": peak_tf, "peak_gbs": peak_gbs, "t_min_ms": t_min * 1e3,
-                         "frac": t_min / t_step, "peak_kind": "bf16_tflops_sustained of measured"},
+                         "frac": t_min / t_step, "peak_kind": "bf16_tflops_sustained of measured",
+                         "traffic": PREFILL_TRAFFIC.get(T)},
             "device_status": st, "steps": steps}
 
 
