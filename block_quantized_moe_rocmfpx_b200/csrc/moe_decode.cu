@@ -890,31 +890,42 @@ __device__ void consumer(const MoeParams& p, Shared& sh, uint8_t* ring, uint8_t*
 // plus the block sums of the staged values (times 2^s_b) for the offset
 // correction.  Run by `nthr` threads (sid = 0 .. nthr-1, whole warps); one item
 // is one (step, t) fragment of a column, 8 consecutive items one 32-block.
+// The columns (T <= MAXC) are handled side by side in each item step, so the
+// per-column chains (loads, shuffles) overlap.
+template <int MAXC>
 __device__ void stage_x(const MoeParams& p, Shared& sh, uint8_t* xh, const uint32_t* x32, int sid, int nthr) {
     const int lane = sid & 31;
     const int per_col = p.H / 4;      // items per column
     const int hp = p.H / 2;           // bf16 pairs per column
     // pass 1: max |x| per column (a warp's items never straddle a column)
-    for (int c = 0; c < p.T; ++c) {
-        uint32_t m = 0u;
-        for (int j0 = sid - lane; j0 < per_col; j0 += nthr) {
-            const int j = j0 + lane;
-            if (j < per_col) {
-                const int step = j >> 2, tt = j & 3;
-                const uint32_t* src = x32 + (size_t)c * hp + step * 8 + tt;
-                const uint32_t v0 = src[0], v1 = src[4];
-                m = max(m, max((v0 << 16) & 0x7fffffffu, v0 & 0x7fff0000u));
-                m = max(m, max((v1 << 16) & 0x7fffffffu, v1 & 0x7fff0000u));
-            }
-        }
+    uint32_t m[MAXC];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if (lane == 0 && m) atomicMax(&sh.xmax[c], m);
+    for (int c = 0; c < MAXC; ++c) m[c] = 0u;
+    for (int j0 = sid - lane; j0 < per_col; j0 += nthr) {
+        const int j = j0 + lane;
+        if (j < per_col) {
+            const int step = j >> 2, tt = j & 3;
+#pragma unroll
+            for (int c = 0; c < MAXC; ++c)
+                if (c < p.T) {
+                    const uint32_t* src = x32 + (size_t)c * hp + step * 8 + tt;
+                    const uint32_t v0 = src[0], v1 = src[4];
+                    m[c] = max(m[c], max((v0 << 16) & 0x7fffffffu, v0 & 0x7fff0000u));
+                    m[c] = max(m[c], max((v1 << 16) & 0x7fffffffu, v1 & 0x7fff0000u));
+                }
+        }
     }
+#pragma unroll
+    for (int c = 0; c < MAXC; ++c)
+        if (c < p.T) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m[c] = max(m[c], __shfl_xor_sync(0xffffffffu, m[c], o));
+            if (lane == 0 && m[c]) atomicMax(&sh.xmax[c], m[c]);
+        }
     asm volatile("bar.sync 1, %0;" ::"r"(nthr) : "memory");
     if (sid < p.T) {
-        const uint32_t m = sh.xmax[sid];
-        const int n = m ? 13 - ((int)((m >> 23) & 255u) - 127) : 0;
+        const uint32_t mm = sh.xmax[sid];
+        const int n = mm ? 13 - ((int)((mm >> 23) & 255u) - 127) : 0;
         sh.xn[sid] = max(-100, min(100, n));
     }
     asm volatile("bar.sync 1, %0;" ::"r"(nthr) : "memory");
@@ -922,35 +933,44 @@ __device__ void stage_x(const MoeParams& p, Shared& sh, uint8_t* xh, const uint3
     const int nxc = (p.has_shared && p.fsA != p.fA) ? 2 : 1;
     float* sx = (float*)(xh + nxc * p.T * p.x_stride);
     const int sxs = moe_sxs(p.H);
+    int xn[MAXC];
+#pragma unroll
+    for (int c = 0; c < MAXC; ++c) xn[c] = c < p.T ? sh.xn[c] : 0;
     for (int ci = 0; ci < nxc; ++ci) {
         const int fmt = ci == 0 ? p.fA : p.fsA;
-        for (int c = 0; c < p.T; ++c) {
-            const int xn = sh.xn[c];
-            uint8_t* dst = xh + (ci * p.T + c) * p.x_stride;
-            for (int j0 = sid - lane; j0 < per_col; j0 += nthr) {
-                const int j = j0 + lane;
-                float sum = 0.f;
-                if (j < per_col) {
-                    const int step = j >> 2, tt = j & 3;
+        for (int j0 = sid - lane; j0 < per_col; j0 += nthr) {
+            const int j = j0 + lane;
+            const int step = j >> 2, tt = j & 3;
+            const int sb = s_pos(fmt, step * 16, p.H);
+            float sum[MAXC];
+#pragma unroll
+            for (int c = 0; c < MAXC; ++c) {
+                sum[c] = 0.f;
+                if (c < p.T && j < per_col) {
+                    uint8_t* dst = xh + (ci * p.T + c) * p.x_stride;
                     const uint32_t* src = x32 + (size_t)c * hp + step * 8 + tt;
                     const uint32_t v0 = src[0], v1 = src[4];
-                    const int sb = s_pos(fmt, step * 16, p.H);
-                    const float sc = __int_as_float((127 + xn - sb) << 23);
+                    const float sc = __int_as_float((127 + xn[c] - sb) << 23);
                     const __half2 h0 = __floats2half2_rn(__uint_as_float(v0 << 16) * sc, __uint_as_float(v0 & 0xffff0000u) * sc);
                     const __half2 h1 = __floats2half2_rn(__uint_as_float(v1 << 16) * sc, __uint_as_float(v1 & 0xffff0000u) * sc);
                     uint2 o;
                     o.x = *reinterpret_cast<const uint32_t*>(&h0);
                     o.y = *reinterpret_cast<const uint32_t*>(&h1);
                     *reinterpret_cast<uint2*>(dst + (step * 4 + tt) * 8) = o;
-                    sum = ((__low2float(h0) + __high2float(h0)) + (__low2float(h1) + __high2float(h1))) *
-                          __int_as_float((127 + sb) << 23);
+                    sum[c] = ((__low2float(h0) + __high2float(h0)) + (__low2float(h1) + __high2float(h1))) *
+                             __int_as_float((127 + sb) << 23);
                 }
-                // the 8 items of a block are 8 consecutive lanes
-                sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-                sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-                sum += __shfl_xor_sync(0xffffffffu, sum, 4);
-                if ((lane & 7) == 0 && j < per_col) sx[(ci * p.T + c) * sxs + (j >> 3)] = sum;
             }
+            // the 8 items of a block are 8 consecutive lanes
+#pragma unroll
+            for (int c = 0; c < MAXC; ++c)
+                if (c < p.T) {
+                    float v = sum[c];
+                    v += __shfl_xor_sync(0xffffffffu, v, 1);
+                    v += __shfl_xor_sync(0xffffffffu, v, 2);
+                    v += __shfl_xor_sync(0xffffffffu, v, 4);
+                    if ((lane & 7) == 0 && j < per_col) sx[(ci * p.T + c) * sxs + (j >> 3)] = v;
+                }
         }
     }
 }
@@ -1009,7 +1029,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_decode_kernel(MoeParams p) {
     } else {
         const int sid = w < WARP_PRODUCER ? threadIdx.x : threadIdx.x - 32;
         if (xbulk && !mbar_wait(&sh.xload, 0, WAIT_LIMIT)) set_error(p.ctrl, MOE_ERR_TIMEOUT);
-        stage_x(p, sh, xh, xbulk ? (const uint32_t*)red : reinterpret_cast<const uint32_t*>(p.x), sid, NTHREADS - 32);
+        stage_x<QC == 1 ? 1 : (QC == 2 ? 4 : MOE_MAXT)>(
+            p, sh, xh, xbulk ? (const uint32_t*)red : reinterpret_cast<const uint32_t*>(p.x), sid, NTHREADS - 32);
         asm volatile("bar.sync 2, %0;" ::"n"(NTHREADS) : "memory");
         if (w == WARP_HLOAD) {
             if ((threadIdx.x & 31) == 0) h_loader(p, sh, xh, hbytes_max, sstr);
