@@ -275,8 +275,6 @@ __device__ __forceinline__ void chunkB_full(const uint8_t* st, int lane, int g, 
         }
         float s0, s1;
         f.scales(b, s0, s1);
-        constexpr int dummy = 0;
-        (void)dummy;
         const int cls = Plane<FMT>::cls_of(b);
 #pragma unroll
         for (int n = 0; n < NB; ++n) {
