@@ -987,8 +987,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_decode_kernel(MoeParams p) {
     const int sstr = moe_sstr(p.I);
     const int hbytes_max = 4 * p.T * (p.I + sstr);
     const int w = threadIdx.x >> 5;
-    Routing rt{};
-    if (w == WARP_PRODUCER) rt = load_routing(p);   // in flight during the barrier set-up
+    grid_dep_launch();   // the next kernel may launch (it waits for this one before its stores)
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.ns; ++s) {
             mbar_init(&sh.full[s], 1);
@@ -1009,6 +1008,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_decode_kernel(MoeParams p) {
         for (int c = 0; c < MOE_MAXT; ++c) sh.xmax[c] = 0u;
         fence_barrier_init();
     }
+    // everything below may read what the previous kernel wrote (routing, x,
+    // the workspace counters)
+    grid_dep_wait();
+    Routing rt{};
+    if (w == WARP_PRODUCER) rt = load_routing(p);
     // x: one bulk copy into the reduction buffers (first written after the
     // staging below) when it fits and is 16-byte aligned, else read from global
     const uint32_t xbytes = (uint32_t)(p.T * p.H * 2);
@@ -1070,11 +1074,15 @@ cudaError_t moe_decode_launch(const MoeParams& p, int grid, cudaStream_t stream)
     cfg.blockDim = dim3(NTHREADS);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute at[1];
+    cudaLaunchAttribute at[2];
     at[0].id = cudaLaunchAttributeCooperative;
     at[0].val.cooperative = 1;
+    // programmatic dependent of the kernel before it (the router): the CTAs
+    // start and set up while it finishes, and wait for it before any load
+    at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     err = cudaLaunchKernelEx(&cfg, kern, p);
     return err;
 }

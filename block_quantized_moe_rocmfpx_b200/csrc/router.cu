@@ -1,34 +1,56 @@
 // router.cu -- router top-k + softmax over the selected logits, one warp per
-// token (the warp's work is router_warp in router_dev.cuh).
+// token (the warp's work is router_warp in router_dev.cuh).  Launched as a
+// programmatic dependent of the kernel before it: it reads the logits at once
+// and waits for that kernel only before it stores idx / w (which the previous
+// MoE kernel may still be reading); it lets the next kernel launch at once.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "rfx_device.cuh"
 #include "router_dev.cuh"
 
 namespace rfx {
 
 constexpr int ROUTER_WARPS = 8;
 
+struct WaitForPrevious {
+    __device__ void operator()() const { grid_dep_wait(); }
+};
+
 template <int PER_LANE>
 __global__ void __launch_bounds__(ROUTER_WARPS * 32) router_topk_kernel(const float* __restrict__ logits, int T, int E,
                                                                        int k, int32_t* __restrict__ idx,
                                                                        float* __restrict__ w) {
+    grid_dep_launch();
     const int tok = blockIdx.x * ROUTER_WARPS + (threadIdx.x >> 5);
     if (tok >= T) return;
-    router_warp<PER_LANE>(logits + (long long)tok * E, E, k, idx + (long long)tok * k, w + (long long)tok * k);
+    router_warp<PER_LANE>(logits + (long long)tok * E, E, k, idx + (long long)tok * k, w + (long long)tok * k,
+                          WaitForPrevious());
+}
+
+template <int PER_LANE>
+cudaError_t launch(const float* logits, int T, int E, int k, int32_t* idx, float* w, cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((T + ROUTER_WARPS - 1) / ROUTER_WARPS);
+    cfg.blockDim = dim3(ROUTER_WARPS * 32);
+    cfg.stream = stream;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, router_topk_kernel<PER_LANE>, logits, T, E, k, idx, w);
 }
 
 cudaError_t router_topk_launch(const float* logits, int T, int E, int k, int32_t* idx, float* w,
                                cudaStream_t stream) {
-    const int grid = (T + ROUTER_WARPS - 1) / ROUTER_WARPS;
     const int per = (E + 31) / 32;
-    if (per <= 1) router_topk_kernel<1><<<grid, ROUTER_WARPS * 32, 0, stream>>>(logits, T, E, k, idx, w);
-    else if (per <= 2) router_topk_kernel<2><<<grid, ROUTER_WARPS * 32, 0, stream>>>(logits, T, E, k, idx, w);
-    else if (per <= 4) router_topk_kernel<4><<<grid, ROUTER_WARPS * 32, 0, stream>>>(logits, T, E, k, idx, w);
-    else if (per <= 8) router_topk_kernel<8><<<grid, ROUTER_WARPS * 32, 0, stream>>>(logits, T, E, k, idx, w);
-    else if (per <= 16) router_topk_kernel<16><<<grid, ROUTER_WARPS * 32, 0, stream>>>(logits, T, E, k, idx, w);
-    else router_topk_kernel<32><<<grid, ROUTER_WARPS * 32, 0, stream>>>(logits, T, E, k, idx, w);
-    return cudaGetLastError();
+    if (per <= 1) return launch<1>(logits, T, E, k, idx, w, stream);
+    if (per <= 2) return launch<2>(logits, T, E, k, idx, w, stream);
+    if (per <= 4) return launch<4>(logits, T, E, k, idx, w, stream);
+    if (per <= 8) return launch<8>(logits, T, E, k, idx, w, stream);
+    if (per <= 16) return launch<16>(logits, T, E, k, idx, w, stream);
+    return launch<32>(logits, T, E, k, idx, w, stream);
 }
 
 }  // namespace rfx

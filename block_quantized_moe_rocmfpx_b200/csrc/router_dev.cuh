@@ -1,6 +1,4 @@
-// router_dev.cuh -- one warp's router top-k + softmax for one token (shared by
-// the router kernel and the fused routing of the MoE decode kernel, so both
-// give the same bits).
+// router_dev.cuh -- one warp's router top-k + softmax for one token.
 //
 // ainomam.com, "APU 实现 token 自由…", section "Lucebox 的优化三板斧" (tuned
 // TOP-K / ARGSORT routing kernels; 6 of 256 experts active) and m.mzlw.cn,
@@ -15,10 +13,14 @@
 
 namespace rfx {
 
-// Lane j < k writes idx_out[j] and w_out[j].  E <= 32 * PER_LANE.
-template <int PER_LANE>
+// Lane j < k writes idx_out[j] and w_out[j].  E <= 32 * PER_LANE.  BEFORE_STORE
+// runs after the arithmetic and before the stores.
+struct NoHook {
+    __device__ void operator()() const {}
+};
+template <int PER_LANE, class Hook = NoHook>
 __device__ __forceinline__ void router_warp(const float* __restrict__ l, int E, int k, int32_t* idx_out,
-                                            float* w_out) {
+                                            float* w_out, Hook before_store = Hook()) {
     const int lane = threadIdx.x & 31;
     float v[PER_LANE];
     uint32_t live = 0;
@@ -55,21 +57,11 @@ __device__ __forceinline__ void router_warp(const float* __restrict__ l, int E, 
         const float vj = __shfl_sync(0xffffffffu, sel_v, j);
         z += expf(vj - v0);
     }
+    before_store();
     if (lane < k) {
         idx_out[lane] = sel_e;
         w_out[lane] = expf(sel_v - v0) / z;
     }
-}
-
-// The same with PER_LANE chosen from E at run time (E <= 1024).
-__device__ __forceinline__ void router_warp_any(const float* l, int E, int k, int32_t* idx_out, float* w_out) {
-    const int per = (E + 31) / 32;
-    if (per <= 1) router_warp<1>(l, E, k, idx_out, w_out);
-    else if (per <= 2) router_warp<2>(l, E, k, idx_out, w_out);
-    else if (per <= 4) router_warp<4>(l, E, k, idx_out, w_out);
-    else if (per <= 8) router_warp<8>(l, E, k, idx_out, w_out);
-    else if (per <= 16) router_warp<16>(l, E, k, idx_out, w_out);
-    else router_warp<32>(l, E, k, idx_out, w_out);
 }
 
 }  // namespace rfx
