@@ -162,6 +162,35 @@ def group_rows(idx: np.ndarray, w: np.ndarray, E: int):
     return counts, (order // k).astype(np.int32), np.asarray(w, dtype=np.float64).reshape(-1)[order], order
 
 
+def router_logits(w_router: np.ndarray, bias, x: np.ndarray):
+    """Router projection ahead of the top-k: (logits fp64 [T][E], mag fp64 [T][E])
+    with logits[t][e] = sum_h W[e][h] x[t][h] + b[e] and mag = sum_h |W[e][h]|
+    |x[t][h]| + |b[e]| (for the per-element bound).  W: uint16 bf16 bits [E][H];
+    x: uint16 bf16 bits [T][H]; bias: fp32 [E] or None.  Both operands widen
+    exactly to fp64; the sum is a plain fp64 matrix product.
+
+    The projection is the MoE gate that decides the routing, kept at high
+    precision: FP8 in the bit allocation of ai-manual.ru, "DeepSeek V4 Flash на
+    AMD Ryzen AI MAX+ 395…", section "Технические детали ROCmFPX"; sensitive
+    projections at FP4 or above in taozi.news, "DeepSeek V4 Flash 在 128GB 锐龙 AI
+    MAX+ 上跑到 32 tok/s", section "ROCmFPX：把 284B 权重压进 128 GB".  This
+    library reads "high precision" as bf16 weights.
+    """
+    W = _bf16_bits_to_f64(np.asarray(w_router, dtype=np.uint16))
+    X = _bf16_bits_to_f64(np.atleast_2d(np.asarray(x, dtype=np.uint16)))
+    logits = X @ W.T
+    mag = np.abs(X) @ np.abs(W).T
+    if bias is not None:
+        b = np.asarray(bias, dtype=np.float32).astype(np.float64)
+        logits = logits + b[None, :]
+        mag = mag + np.abs(b)[None, :]
+    return logits, mag
+
+
+def _bf16_bits_to_f64(u16: np.ndarray) -> np.ndarray:
+    return (u16.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
 def router_topk(logits: np.ndarray, k: int):
     """(idx int32 [T][k], w fp64 [T][k]) for fp32 logits [T][E]."""
     logits = _c(np.atleast_2d(logits), np.float32)

@@ -14,6 +14,7 @@ tag   stream
 10..15 block scales of the same six matrices
 100   expert permutation of the Zipf routing bias
 101   router logits (normal draws)
+102   router projection weights (normal draws)
 200   activations x
 ====  =====================================
 """
@@ -36,6 +37,7 @@ KIND_GATE, KIND_UP, KIND_DOWN, KIND_SH_GATE, KIND_SH_UP, KIND_SH_DOWN = range(6)
 TAG_SCALE_OFFSET = 10
 TAG_PERM = 100
 TAG_LOGITS = 101
+TAG_WROUTER = 102
 TAG_X = 200
 
 
@@ -129,6 +131,21 @@ def logits(seed: int, layer: int, tok0: int, T: int, E: int, zipf_s: float) -> n
     out = np.empty((T, E), dtype=np.float32)
     lib().synth_logits(key(seed, layer, TAG_LOGITS, 0), _p(bias), tok0, T, E, _p(out))
     return out
+
+
+def router_weight_bf16(seed: int, layer: int, E: int, H: int) -> np.ndarray:
+    """uint16 [E][H] bf16 router projection weights: N(0,1) draws in bf16 times
+    2^-floor(log2(H)/2) (an exact power of two near 1/sqrt(H), so that W x has
+    about unit variance for x ~ N(0,1))."""
+    raw = normal_bf16(key(seed, layer, TAG_WROUTER, 0), E * H).reshape(E, H)
+    sh = int(np.floor(np.log2(H) / 2))
+    f = (raw.astype(np.uint32) << 16).view(np.float32) * np.float32(2.0 ** -sh)   # exact: a power of two
+    return (f.view(np.uint32) >> 16).astype(np.uint16)
+
+
+def router_bias_f32(seed: int, layer: int, E: int, s: float) -> np.ndarray:
+    """fp32 [E] per-expert routing bias: the Zipf log-popularity of the logits workload."""
+    return zipf_bias(seed, layer, E, s).astype(np.float32)
 
 
 def x_bf16(seed: int, tok0: int, T: int, H: int, stream: int = 0) -> np.ndarray:

@@ -10,6 +10,7 @@ transposed operand or swapped gate/up fails at least one of them.
 import json
 import math
 import os
+import struct
 
 import numpy as np
 import pytest
@@ -308,3 +309,63 @@ def test_rms_bf16_closed_form_and_torch():
     # fp64 sums differ in the last bit, and check the scale closes to unit RMS
     assert np.mean(got == ref) > 0.999
     assert math.sqrt(np.mean(got * got)) == pytest.approx(1.0, abs=4e-3)
+
+
+def _bf16_bits(vals):
+    """bf16 bit patterns (uint16) of values exactly representable in bf16."""
+    f = np.asarray(vals, dtype=np.float32)
+    u = f.view(np.uint32)
+    assert not (u & 0xFFFF).any(), "value not exact in bf16"
+    return (u >> 16).astype(np.uint16)
+
+
+def _bf16_value(u):
+    return struct.unpack("<f", struct.pack("<I", int(u) << 16))[0]
+
+
+def test_router_logits_unit_vector_probe():
+    """Row e of W one-hot at column p(e): logits[t][e] = x[t][p(e)] + b[e]
+    exactly (a transposed operand or a wrong index fails)."""
+    E, H, T = 12, 64, 3
+    perm = np.random.default_rng(3).permutation(H)[:E]
+    W = np.zeros((E, H), dtype=np.float32)
+    W[np.arange(E), perm] = 1.0
+    x = synth.x_bf16(5, 0, T, H)
+    b = np.linspace(-2.0, 3.0, E).astype(np.float32)
+    lg, mag = oracle.router_logits(_bf16_bits(W), b, x)
+    xf = synth.bf16_to_f64(x)
+    assert np.array_equal(lg, xf[:, perm] + b.astype(np.float64)[None, :])
+    assert np.array_equal(mag, np.abs(xf[:, perm]) + np.abs(b.astype(np.float64))[None, :])
+
+
+def test_router_logits_closed_form_and_bias_only():
+    E, H, T = 5, 96, 2
+    W = np.full((E, H), 0.375, dtype=np.float32)            # exact in bf16
+    x = _bf16_bits(np.full((T, H), -1.25, dtype=np.float32))
+    lg, _ = oracle.router_logits(_bf16_bits(W), None, x)
+    assert np.all(lg == H * 0.375 * -1.25)
+    b = np.array([0.5, -7.0, 1e-3, 0.0, 42.0], dtype=np.float32)
+    lg0, mag0 = oracle.router_logits(np.zeros((E, H), dtype=np.uint16), b, x)
+    assert np.array_equal(lg0, np.broadcast_to(b.astype(np.float64), (T, E)))
+    assert np.array_equal(mag0, np.broadcast_to(np.abs(b.astype(np.float64)), (T, E)))
+
+
+def test_router_logits_brute_force():
+    """Plain loops over the bf16 values (a second routine) on a tiny case."""
+    E, H, T = 4, 32, 2
+    W = synth.router_weight_bf16(9, 1, E, H)
+    x = synth.x_bf16(9, 3, T, H)
+    b = synth.router_bias_f32(9, 1, E, 1.1)
+    lg, mag = oracle.router_logits(W, b, x)
+    for t in range(T):
+        for e in range(E):
+            s = 0.0
+            m = 0.0
+            for h in range(H):
+                p = _bf16_value(W[e, h]) * _bf16_value(x[t, h])
+                s += p
+                m += abs(p)
+            s += float(b[e])
+            m += abs(float(b[e]))
+            assert abs(lg[t, e] - s) <= 1e-14 * m
+            assert abs(mag[t, e] - m) <= 1e-14 * m
