@@ -51,6 +51,9 @@ _pack = _proto("rfx_pack", _i32, [_i32, _vp, _vp, _i64, _i64, _vp, _sz])
 _unpack = _proto("rfx_unpack", _i32, [_i32, _vp, _i64, _i64, _vp, _vp])
 _pack_device = _proto("rfx_pack_device", _i32, [_i32, _vp, _vp, _i64, _i64, _vp, _vp])
 _router = _proto("moe_router_topk", _i32, [_vp, _i32, _i32, _i32, _vp, _vp, _vp])
+_router_logits = _proto("moe_router_logits", _i32, [_vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp])
+_router_proj_topk = _proto("moe_router_project_topk", _i32,
+                           [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp])
 _gemv = _proto("rfx_gemv_q", _i32, [_i32, _vp, _i64, _i64, _vp, _i32, _i32, _vp, _vp])
 _layer_create = _proto("moe_layer_create", _i32, [ctypes.POINTER(moe_layer_desc), ctypes.POINTER(_vp)])
 _layer_destroy = _proto("moe_layer_destroy", None, [_vp])
@@ -77,7 +80,7 @@ EXPORTED = ["rfx_last_error", "rfx_packed_bytes", "rfx_pack", "rfx_unpack", "rfx
             "rfx_gemv_q", "moe_layer_create", "moe_layer_destroy", "moe_ffn_workspace_bytes", "rfx_ws_init",
             "rfx_ws_status", "moe_ffn_forward", "moe_ffn_forward_static", "moe_rms_norm_bf16",
             "moe_stack_workspace_bytes", "moe_stack_forward", "moe_prefill_workspace_bytes", "moe_ffn_prefill",
-            "moe_prefill_view"]
+            "moe_prefill_view", "moe_router_logits", "moe_router_project_topk"]
 
 
 class RfxError(RuntimeError):
@@ -149,6 +152,22 @@ def moe_router_topk(logits, k: int, idx, w, stream=None):
     """logits fp32 [T][E] (device) -> idx int32 [T][k], w fp32 [T][k] (device, preallocated)."""
     T, E = logits.shape
     _check(_router(_ptr(logits), T, E, k, _ptr(idx), _ptr(w), _stream(stream)))
+
+
+def moe_router_logits(w_router, bias, x, logits, stream=None):
+    """logits fp32 [T][E] = W x + bias for w_router bf16 [E][H], bias fp32 [E] or
+    None, x bf16 [T][H] (device tensors)."""
+    E, H = w_router.shape
+    T = x.shape[0]
+    _check(_router_logits(_ptr(w_router), _ptr(bias), _ptr(x), T, H, E, _ptr(logits), _stream(stream)))
+
+
+def moe_router_project_topk(w_router, bias, x, k: int, logits, idx, w, stream=None):
+    """moe_router_logits, then moe_router_topk: fills logits [T][E], idx [T][k], w [T][k]."""
+    E, H = w_router.shape
+    T = x.shape[0]
+    _check(_router_proj_topk(_ptr(w_router), _ptr(bias), _ptr(x), T, H, E, k, _ptr(logits), _ptr(idx), _ptr(w),
+                             _stream(stream)))
 
 
 def rfx_gemv_q(fmt: int, W, N: int, K: int, x, y, stream=None):

@@ -73,6 +73,29 @@ extern "C" int moe_router_topk(const float* logits, int T, int E, int k, int32_t
     return e == cudaSuccess ? RFX_OK : cuda_fail("moe_router_topk", e);
 }
 
+extern "C" int moe_router_logits(const void* w_router, const float* bias, const void* x, int T, int H, int E,
+                                 float* logits, void* stream) {
+    if (T < 0 || E < 1 || H < 32 || H % 32 != 0)
+        return rfx_fail(RFX_EINVAL, "moe_router_logits: need T >= 0, E >= 1 and H a positive multiple of 32");
+    if ((long long)T > 8LL * 65535) return rfx_fail(RFX_EUNSUPPORTED, "moe_router_logits: T <= 524280");
+    if (T == 0) return RFX_OK;
+    if (!w_router || !x || !logits) return rfx_fail(RFX_EINVAL, "moe_router_logits: null pointer");
+    if (((uintptr_t)w_router & 15u) || ((uintptr_t)x & 15u))
+        return rfx_fail(RFX_EINVAL, "moe_router_logits: w_router and x must be 16-byte aligned");
+    cudaError_t e = rfx::router_logits_launch((const uint16_t*)w_router, bias, (const uint16_t*)x, T, H, E, logits,
+                                              (cudaStream_t)stream);
+    return e == cudaSuccess ? RFX_OK : cuda_fail("moe_router_logits", e);
+}
+
+extern "C" int moe_router_project_topk(const void* w_router, const float* bias, const void* x, int T, int H, int E,
+                                       int k, float* logits, int32_t* idx, float* w, void* stream) {
+    if (T < 0 || E < 1 || E > 1024 || k < 1 || k > E || k > 16)
+        return rfx_fail(RFX_EINVAL, "moe_router_project_topk: need T >= 0, 1 <= E <= 1024, 1 <= k <= min(E, 16)");
+    int rc = moe_router_logits(w_router, bias, x, T, H, E, logits, stream);
+    if (rc != RFX_OK) return rc;
+    return moe_router_topk(logits, T, E, k, idx, w, stream);
+}
+
 extern "C" int rfx_gemv_q(rfx_format f, const void* W, int64_t N, int64_t K, const void* x, int x_is_fp32, int q,
                           float* y, void* stream) {
     if (!fmt_ok(f)) return rfx_fail(RFX_EINVAL, "rfx_gemv_q: bad format");

@@ -1,8 +1,9 @@
 // router.cu -- router top-k + softmax over the selected logits, one warp per
 // token (the warp's work is router_warp in router_dev.cuh).  Launched as a
-// programmatic dependent of the kernel before it: it reads the logits at once
-// and waits for that kernel only before it stores idx / w (which the previous
-// MoE kernel may still be reading); it lets the next kernel launch at once.
+// programmatic dependent of the kernel before it: the launch overlaps that
+// kernel's tail, and every load waits until it has finished (the logits may be
+// its output, and idx / w may still be its input); the next kernel may launch
+// at once.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -13,19 +14,15 @@ namespace rfx {
 
 constexpr int ROUTER_WARPS = 8;
 
-struct WaitForPrevious {
-    __device__ void operator()() const { grid_dep_wait(); }
-};
-
 template <int PER_LANE>
 __global__ void __launch_bounds__(ROUTER_WARPS * 32) router_topk_kernel(const float* __restrict__ logits, int T, int E,
                                                                        int k, int32_t* __restrict__ idx,
                                                                        float* __restrict__ w) {
     grid_dep_launch();
+    grid_dep_wait();
     const int tok = blockIdx.x * ROUTER_WARPS + (threadIdx.x >> 5);
     if (tok >= T) return;
-    router_warp<PER_LANE>(logits + (long long)tok * E, E, k, idx + (long long)tok * k, w + (long long)tok * k,
-                          WaitForPrevious());
+    router_warp<PER_LANE>(logits + (long long)tok * E, E, k, idx + (long long)tok * k, w + (long long)tok * k);
 }
 
 template <int PER_LANE>

@@ -13,14 +13,10 @@
 
 namespace rfx {
 
-// Lane j < k writes idx_out[j] and w_out[j].  E <= 32 * PER_LANE.  BEFORE_STORE
-// runs after the arithmetic and before the stores.
-struct NoHook {
-    __device__ void operator()() const {}
-};
-template <int PER_LANE, class Hook = NoHook>
+// Lane j < k writes idx_out[j] and w_out[j].  E <= 32 * PER_LANE.
+template <int PER_LANE>
 __device__ __forceinline__ void router_warp(const float* __restrict__ l, int E, int k, int32_t* idx_out,
-                                            float* w_out, Hook before_store = Hook()) {
+                                            float* w_out) {
     const int lane = threadIdx.x & 31;
     float v[PER_LANE];
     uint32_t live = 0;
@@ -57,7 +53,6 @@ __device__ __forceinline__ void router_warp(const float* __restrict__ l, int E, 
         const float vj = __shfl_sync(0xffffffffu, sel_v, j);
         z += expf(vj - v0);
     }
-    before_store();
     if (lane < k) {
         idx_out[lane] = sel_e;
         w_out[lane] = expf(sel_v - v0) / z;

@@ -20,6 +20,9 @@
  *       ROCmFPX量化达成42 tok/s", section "MoE 专家并行" -- 43 MoE layers, 256
  *       routed experts, top-6 plus 1 shared expert; section "DSpark 草稿模型"
  *       -- verify width q2..q5.
+ *  [AM] ai-manual.ru, "DeepSeek V4 Flash на AMD Ryzen AI MAX+ 395: как
+ *       достичь 32 tok/s локального инференса", section "Технические детали
+ *       ROCmFPX" -- the MoE gate (router projection) kept at 8 bits.
  *
  * Conventions
  *  - Every function returns an rfx_status (0 = OK).  No exception crosses the
@@ -144,6 +147,29 @@ int rfx_pack_device(rfx_format f, const uint8_t* codes, const void* scales, int6
  * Limits: 1 <= E <= 1024, 1 <= k <= min(E, 16), T >= 0 (T = 0 is a no-op).
  */
 int moe_router_topk(const float* logits, int T, int E, int k, int32_t* idx, float* w, void* stream);
+
+/*
+ * Router projection ahead of the top-k: logits[t][e] = sum_h W[e][h] x[t][h]
+ * + bias[e], fp32 accumulation (per element a fixed order: independent of T).
+ * The gate that decides the routing is kept at high precision ([AM]
+ * "Технические детали ROCmFPX": FP8; [TZ] "ROCmFPX：把 284B 权重压进 128 GB":
+ * sensitive projections FP4 or above); this library reads it as bf16.
+ * w_router: device bf16 bits [E][H]; bias: device fp32 [E] or NULL; x: device
+ * bf16 bits [T][H]; both 16-byte aligned.  logits: device fp32 [T][E].
+ * Limits: H % 32 == 0, E >= 1, 0 <= T <= 524280 (T = 0 is a no-op).  One launch
+ * (programmatic dependent of the kernel before it: it reads W at once and x
+ * only after that kernel has finished).
+ */
+int moe_router_logits(const void* w_router, const float* bias, const void* x, int T, int H, int E, float* logits,
+                      void* stream);
+
+/*
+ * moe_router_logits followed by moe_router_topk (two launches, the second a
+ * programmatic dependent of the first): logits [T][E], idx [T][k], w [T][k]
+ * on the device.  Limits: both calls' (E <= 1024, k <= min(E, 16)).
+ */
+int moe_router_project_topk(const void* w_router, const float* bias, const void* x, int T, int H, int E, int k,
+                            float* logits, int32_t* idx, float* w, void* stream);
 
 /* --------------------------------------------------------------- GEMV --- */
 

@@ -181,6 +181,16 @@ def test_device_calls_reject_bad_arguments_before_cuda():
     assert lib.rfx_gemv_q(2, None, 16, 64, None, 0, 9, None, None) == rfx.RFX_EUNSUPPORTED
     assert lib.rfx_gemv_q(2, None, 16, 48, None, 0, 1, None, None) == rfx.RFX_EINVAL
     assert lib.rfx_gemv_q(6, None, 16, 64, None, 0, 1, None, None) == rfx.RFX_EINVAL
+    # router projection: H a positive multiple of 32, E >= 1, T >= 0, aligned operands
+    assert lib.moe_router_logits(None, None, None, 4, 48, 256, None, None) == rfx.RFX_EINVAL
+    assert lib.moe_router_logits(None, None, None, 4, 64, 0, None, None) == rfx.RFX_EINVAL
+    assert lib.moe_router_logits(None, None, None, -1, 64, 8, None, None) == rfx.RFX_EINVAL
+    assert lib.moe_router_logits(None, None, None, 0, 64, 8, None, None) == rfx.RFX_OK      # T = 0: no-op
+    assert lib.moe_router_logits(None, None, None, 2, 64, 8, None, None) == rfx.RFX_EINVAL  # null pointers
+    assert lib.moe_router_logits(ctypes.c_void_p(0x1008), None, ctypes.c_void_p(0x2000), 2, 64, 8,
+                                 ctypes.c_void_p(0x3000), None) == rfx.RFX_EINVAL             # W not 16-byte aligned
+    assert lib.moe_router_project_topk(None, None, None, 1, 64, 8, 9, None, None, None, None) == rfx.RFX_EINVAL
+    assert lib.moe_router_project_topk(None, None, None, 1, 64, 2000, 6, None, None, None, None) == rfx.RFX_EINVAL
 
 
 def test_layer_create_validation():
