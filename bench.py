@@ -58,6 +58,8 @@ def parse():
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill grouped-GEMM measurement")
     ap.add_argument("--prefill-only", action="store_true", help="time only the prefill (T = 2048 and 8192)")
     ap.add_argument("--prefill-steps", type=int, default=20)
+    ap.add_argument("--no-router-proj", action="store_true", help="skip the router projection measurement")
+    ap.add_argument("--router-proj-only", action="store_true", help="time only the router projection + top-k")
     return ap.parse_args()
 
 
@@ -393,6 +395,51 @@ def measure_prefill(T: int, steps: int, warmup: int, dev, layer=None):
             "device_status": st, "steps": steps}
 
 
+ROUTER_PROJ_COPIES = 80   # 80 x 2 MB of router weights rotate: every call reads them from DRAM
+ROUTER_PROJ_TS = (1, 4, 2048)
+
+
+def measure_router_proj(T: int, steps: int, warmup: int, dev):
+    """Router projection + top-k (moe_router_project_topk: logits = W_router x +
+    bias, bf16 W [256][4096], then top-6) for T token columns, captured in a
+    graph; ROUTER_PROJ_COPIES weight copies rotate so that W is read from DRAM.
+    Roofline (HBM): W + x + bias read, logits written, by the projection kernel."""
+    import torch
+    import synth
+    import block_quantized_moe_rocmfpx_b200 as rfx
+    nc = ROUTER_PROJ_COPIES
+    W0 = torch.from_numpy(synth.router_weight_bf16(SEED, 0, E, H).view("int16")).to(dev)
+    Ws = [W0] + [W0.clone() for _ in range(nc - 1)]
+    b = torch.from_numpy(synth.router_bias_f32(SEED, 0, E, ZIPF_S)).to(dev)
+    x = torch.from_numpy(synth.x_bf16(SEED, 300000, T, H).view("int16")).to(dev)
+    lg = torch.empty((T, E), dtype=torch.float32, device=dev)
+    idx = torch.empty((T, K_TOP), dtype=torch.int32, device=dev)
+    w = torch.empty((T, K_TOP), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(t):
+        rfx.moe_router_project_topk(Ws[t % nc], b, x, K_TOP, lg, idx, w, stream)
+
+    with torch.cuda.stream(stream):
+        for t in range(3):
+            step(t)
+        torch.cuda.synchronize()
+        gw = graph_of(step, max(3, warmup), stream)
+        g = graph_of(step, steps, stream)
+        gw.replay()
+        torch.cuda.synchronize()
+        ms = time_graph(g, stream)
+        del g, gw
+    us = ms * 1e3 / steps
+    nbytes = E * H * 2 + T * H * 2 + E * 4 + T * E * 4
+    peak, peak_kind = peaks()
+    gbs = nbytes / (us * 1e-6) / 1e9
+    return {"T": T, "us_per_call": us, "bytes_per_call": nbytes, "achieved_gbs": gbs,
+            "roofline": {"bound": "hbm", "peak_gbs": peak, "frac": gbs / peak, "peak_kind": peak_kind,
+                         "t_min_us": nbytes / (peak * 1e9) * 1e6},
+            "launches_per_call": 2, "steps": steps}
+
+
 def peaks_tensor() -> float:
     """Measured sustained dense bf16 TFLOP/s (a kernel timed inside a long step)."""
     try:
@@ -547,6 +594,12 @@ def main():
             print(json.dumps({"metric": "43-layer MoE-FFN stack decode tokens/s (FFN only)", "stack": st,
                               "peak_gbs": peak, "peak_kind": peak_kind}), flush=True)
         return
+    if args.router_proj_only:
+        rp = [measure_router_proj(T, min(args.steps, 400), max(3, args.warmup), dev) for T in ROUTER_PROJ_TS]
+        if rank == 0:
+            print(json.dumps({"metric": "router projection + top-k (W_router x + bias, top-6) us per call",
+                              "router_projection": rp}), flush=True)
+        return
     if args.prefill_only:
         pf = [measure_prefill(T, args.prefill_steps, max(3, args.warmup), dev) for T in PREFILL_TS]
         if rank == 0:
@@ -567,6 +620,9 @@ def main():
         e2e_ms = reduce_max(r1["e2e"]["steps"] / r1["e2e"]["value"] * 1e3)
         e2e_v = dict(r1["e2e"])
         e2e_v["value"] = world * r1["e2e"]["steps"] / (e2e_ms / 1e3)
+    rp = None
+    if not args.no_router_proj:
+        rp = [measure_router_proj(T, min(args.steps, 400), max(3, args.warmup), dev) for T in ROUTER_PROJ_TS]
     pf = None
     if not args.no_prefill:
         pf = [measure_prefill(T, args.prefill_steps, max(3, args.warmup), dev) for T in PREFILL_TS]
@@ -601,6 +657,7 @@ def main():
             "clocks": r1["clocks"],
             "device_status": {"q1": r1["status"], "q4": r4["status"]},
             "prefill": pf,
+            "router_projection": rp,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
