@@ -8,14 +8,21 @@
 // 128GB 锐龙 AI MAX+ 上跑到 32 tok/s", section "ROCmFPX：把 284B 权重压进 128
 // GB"); this library reads that as bf16 weights.
 //
-// B200 design: a GEMV over E rows (2 MB for 256 x 4096), HBM-bound, spread over
-// all SMs.  A CTA owns two rows and up to 8 columns; each of its 8 warps takes a
+// B200 design, T <= 8 (decode / verify): a GEMV over E rows (2 MB for 256 x
+// 4096), HBM-bound, spread over all SMs.  A CTA owns two rows and up to 8 columns; each of its 8 warps takes a
 // quarter of H for one row (16-byte loads of 8 bf16 of W and of x, fp32 FMAs in
 // index order per lane, then a butterfly over the lanes); the four quarters
 // are added in a fixed tree, so a logit's bits depend neither on T nor on the
 // launch.  W is a constant input: each warp asks L2 for its slice before the
 // kernel waits for the previous one (programmatic dependent launch); x may come
 // from that kernel and is read after the wait.
+//
+// T > 8 (prefill): a tensor-core GEMM, logits^T = W x^T, bf16 operands with
+// fp32 accumulation (mma.sync m16n8k16: every product is exact, the sums are
+// fp32 in a fixed order per element).  A CTA computes 64 experts x 32 tokens
+// (256 CTAs at E = 256, T = 2048); K runs in chunks of 64 staged by cp.async
+// through a 4-deep shared-memory ring (padded rows: conflict-free ldmatrix);
+// 4 warps of 32 x 16.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -94,9 +101,134 @@ __global__ void __launch_bounds__(RP_THREADS) router_logits_kernel(const uint16_
     }
 }
 
+// ------------------------------------------------------------- T > 8 ---
+
+constexpr int RM_BM = 64, RM_BN = 32, RM_BK = 64, RM_STAGES = 4;
+constexpr int RM_LD = RM_BK + 8;   // padded row (144 bytes): ldmatrix rows hit distinct banks
+constexpr int RM_THREADS = 128;
+constexpr int RM_STAGE_ELEMS = (RM_BM + RM_BN) * RM_LD;
+constexpr size_t RM_SMEM = (size_t)RM_STAGES * RM_STAGE_ELEMS * 2;
+
+__device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, bool valid) {
+    const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(valid ? 16 : 0) : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4(const void* p, uint32_t r[4]) {
+    const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(p));
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(a));
+}
+
+__global__ void __launch_bounds__(RM_THREADS) router_logits_mma_kernel(const uint16_t* __restrict__ W,
+                                                                      const float* __restrict__ bias,
+                                                                      const uint16_t* __restrict__ x, int T, int H,
+                                                                      int E, float* __restrict__ logits) {
+    extern __shared__ __align__(16) uint16_t rm_smem[];   // [stage][A rows 64 | B rows 32][RM_LD]
+    grid_dep_launch();
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int e0 = blockIdx.x * RM_BM, t0 = blockIdx.y * RM_BN;
+    const int wm = (warp >> 1) * 32, wn = (warp & 1) * 16;
+    const int nk = (H + RM_BK - 1) / RM_BK;
+    // stage tiles: A 64 rows x 8 pieces of 16 bytes (4 per thread), B 32 x 8 (2 per thread);
+    // a K tail shorter than 64 (H % 64 == 32) is zero-filled
+    auto load = [&](int kc) {
+        uint16_t* sa = rm_smem + (kc % RM_STAGES) * RM_STAGE_ELEMS;
+        uint16_t* sb = sa + RM_BM * RM_LD;
+        const int pc = tid & 7, k = kc * RM_BK + pc * 8;
+        const bool kv = k < H;
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            const int r = (tid >> 3) + 16 * h;
+            const bool v = kv && e0 + r < E;
+            cp_async16_zfill(sa + r * RM_LD + pc * 8, W + (size_t)(v ? e0 + r : 0) * H + (kv ? k : 0), v);
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int r = (tid >> 3) + 16 * h;
+            const bool v = kv && t0 + r < T;
+            cp_async16_zfill(sb + r * RM_LD + pc * 8, x + (size_t)(v ? t0 + r : 0) * H + (kv ? k : 0), v);
+        }
+    };
+    grid_dep_wait();   // x may be the previous kernel's output
+    float acc[2][2][4];
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[i][j][c] = 0.f;
+#pragma unroll
+    for (int s = 0; s < RM_STAGES - 1; ++s) {
+        if (s < nk) load(s);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    }
+    for (int kc = 0; kc < nk; ++kc) {
+        asm volatile("cp.async.wait_group %0;" ::"n"(RM_STAGES - 2) : "memory");
+        __syncthreads();   // stage kc landed for all threads; stage kc - 1 is free again
+        if (kc + RM_STAGES - 1 < nk) load(kc + RM_STAGES - 1);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        const uint16_t* sa = rm_smem + (kc % RM_STAGES) * RM_STAGE_ELEMS;
+        const uint16_t* sb = sa + RM_BM * RM_LD;
+#pragma unroll
+        for (int ks = 0; ks < RM_BK; ks += 16) {
+            uint32_t a[2][4], b[4];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) ldsm_x4(sa + (wm + 16 * i + (lane & 15)) * RM_LD + ks + (lane >> 4) * 8, a[i]);
+            // B is stored [token][k]: matrices (n 0-7, k 0-7), (n 0-7, k 8-15), (n 8-15, k 0-7), (n 8-15, k 8-15)
+            ldsm_x4(sb + (wn + (lane & 7) + ((lane >> 4) << 3)) * RM_LD + ks + ((lane >> 3) & 1) * 8, b);
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) mma16816<false>(acc[i][j], a[i], b[2 * j], b[2 * j + 1], acc[i][j]);
+        }
+    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    // acc[i][j]: rows (experts) wm + 16 i + g (+8), columns (tokens) wn + 8 j + 2 t (+1)
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+            const int e = e0 + wm + 16 * i + g + 8 * hr;
+            if (e >= E) continue;
+            const float bv = bias ? __ldg(bias + e) : 0.f;
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    const int tok = t0 + wn + 8 * j + 2 * t + cc;
+                    if (tok < T) logits[(size_t)tok * E + e] = acc[i][j][2 * hr + cc] + bv;
+                }
+        }
+}
+
 cudaError_t router_logits_launch(const uint16_t* W, const float* bias, const uint16_t* x, int T, int H, int E,
                                  float* logits, cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
+    if (T > RP_COLS) {
+        // once per device (not a stream operation: stays out of graph captures after the first call)
+        static bool attr_set[64] = {false};
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        if (dev >= 64 || !attr_set[dev]) {
+            e = cudaFuncSetAttribute(router_logits_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)RM_SMEM);
+            if (e != cudaSuccess) return e;
+            if (dev < 64) attr_set[dev] = true;
+        }
+        cfg.gridDim = dim3((unsigned)((E + RM_BM - 1) / RM_BM), (unsigned)((T + RM_BN - 1) / RM_BN));
+        cfg.blockDim = dim3(RM_THREADS);
+        cfg.dynamicSmemBytes = RM_SMEM;
+        cfg.stream = stream;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        at[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = at;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, router_logits_mma_kernel, W, bias, x, T, H, E, logits);
+    }
     cfg.gridDim = dim3((unsigned)((E + RP_ROWS - 1) / RP_ROWS), (unsigned)((T + RP_COLS - 1) / RP_COLS));
     cfg.blockDim = dim3(RP_THREADS);
     cfg.stream = stream;

@@ -11,12 +11,14 @@ import synth
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
-# fp32 accumulation depth of one logit: 8-term FMA chains per 16-byte chunk,
-# H / (4 * 8 * 32) chunks per lane, a 5-level butterfly, a 2-level tree of the
-# quarters and the bias add; each rounding is at most 2^-24 of the running
-# magnitude, bounded by mag = sum |W||x| + |b|.
-def bound(H):
-    depth = 8 * max(1, H // 1024) + 5 + 2 + 1
+# fp32 accumulation depth of one logit, each rounding at most 2^-24 of the
+# running magnitude (bounded by mag = sum |W||x| + |b|).  T <= 8 (GEMV): 8-term
+# FMA chains per 16-byte chunk, H / (4 * 8 * 32) chunks per lane, a 5-level
+# butterfly, a 2-level tree of the quarters and the bias add.  T > 8 (tensor
+# core): H / 16 accumulation steps, each counted twice (the tensor core may
+# truncate rather than round), and the bias add.
+def bound(H, T):
+    depth = 8 * max(1, H // 1024) + 5 + 2 + 1 if T <= 8 else 2 * (H // 16) + 1
     return depth * 2.0 ** -24
 
 
@@ -39,40 +41,43 @@ def run(E, H, T, seed=0, with_bias=True, k=None):
     return W, b, x, lg.cpu().numpy(), idx.cpu().numpy(), w.cpu().numpy()
 
 
-def check_logits(W, b, x, lg, H):
+def check_logits(W, b, x, lg, H, T):
     ref, mag = oracle.router_logits(W, b, x)
     err = np.abs(lg.astype(np.float64) - ref)
     assert np.all(np.isfinite(lg))
-    assert np.all(err <= bound(H) * mag), float((err / mag).max())
+    assert np.all(err <= bound(H, T) * mag), float((err / mag).max())
     rel = np.linalg.norm(lg - ref) / np.linalg.norm(ref)
-    assert rel <= 1e-6, rel
+    assert rel <= (1e-6 if T <= 8 else 1e-5), rel
 
 
-@pytest.mark.parametrize("T", [1, 4, 5, 8, 9, 37])
+@pytest.mark.parametrize("T", [1, 4, 5, 8, 9, 37, 64, 65, 200])
 def test_router_logits_full_size(T):
     E, H = 256, 4096
     W, b, x, lg, _, _ = run(E, H, T, seed=T)
-    check_logits(W, b, x, lg, H)
+    check_logits(W, b, x, lg, H, T)
 
 
 @pytest.mark.parametrize("E,H,T,bias", [(8, 512, 1, False), (8, 512, 3, True), (3, 96, 5, True), (1000, 64, 2, True),
-                                        (257, 4096, 8, False)])
+                                        (257, 4096, 8, False), (8, 512, 30, True), (3, 96, 70, True),
+                                        (1000, 64, 129, False), (257, 4096, 100, True)])
 def test_router_logits_shapes(E, H, T, bias):
     W, b, x, lg, _, _ = run(E, H, T, seed=E + H, with_bias=bias)
-    check_logits(W, b, x, lg, H)
+    check_logits(W, b, x, lg, H, T)
 
 
-def test_router_logits_columns_independent():
-    """A column's logits have the same bits whatever the other columns."""
-    E, H, T = 256, 4096, 11
+@pytest.mark.parametrize("T,sub", [(8, 1), (300, 9)])
+def test_router_logits_columns_independent(T, sub):
+    """A column's logits have the same bits whatever the other columns (within
+    one path: T <= 8 and T > 8 use different arithmetic)."""
+    E, H = 256, 4096
     W, b, x, lg, _, _ = run(E, H, T, seed=2)
     Wd = torch.from_numpy(W.view(np.int16)).to(DEV)
     bd = torch.from_numpy(b).to(DEV)
-    for t in (0, 7, 10):
-        xd = torch.from_numpy(x[t:t + 1].view(np.int16)).to(DEV)
-        one = torch.empty((1, E), dtype=torch.float32, device=DEV)
-        rfx.moe_router_logits(Wd, bd, xd, one)
-        assert np.array_equal(one.cpu().numpy()[0], lg[t])
+    for t in (0, 5, T - sub):
+        xd = torch.from_numpy(np.ascontiguousarray(x[t:t + sub]).view(np.int16)).to(DEV)
+        part = torch.empty((sub, E), dtype=torch.float32, device=DEV)
+        rfx.moe_router_logits(Wd, bd, xd, part)
+        assert np.array_equal(part.cpu().numpy(), lg[t:t + sub])
 
 
 @pytest.mark.parametrize("E,H,T,k", [(256, 4096, 1, 6), (256, 4096, 4, 6), (256, 4096, 2048, 6), (8, 512, 3, 2)])
@@ -81,10 +86,10 @@ def test_router_project_topk_teacher_forced(E, H, T, k):
     decision is taken in the kernel's precision: fp32 logits)."""
     W, b, x, lg, idx, w = run(E, H, T, seed=7 + T, k=k)
     if T <= 64:
-        check_logits(W, b, x, lg, H)
+        check_logits(W, b, x, lg, H, T)
     else:   # large T: a seeded sample of columns against the oracle
         rows = np.random.default_rng(T).choice(T, 48, replace=False)
-        check_logits(W, b, x[rows], lg[rows], H)
+        check_logits(W, b, x[rows], lg[rows], H, T)
     ridx, rw = oracle.router_topk(lg, k)
     assert np.array_equal(idx, ridx)
     assert np.allclose(w, rw, rtol=1e-6, atol=0)
