@@ -39,7 +39,7 @@ SEED = 0
 # DRAM bytes (read + write) of one q=1 launch of moe_decode_kernel from the ncu
 # capture summarised in profiles/moe_decode_q1_full_layer.md; set to None
 # whenever the kernel changes until it is captured again.
-TRAFFIC_Q1 = 67_540_480 + 1_108_224
+TRAFFIC_Q1 = 67_844_608 + 2_448_384
 
 
 def parse():
