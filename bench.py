@@ -527,9 +527,10 @@ class _Null:
 
 
 def e2e(wl, steps, stream):
-    """Same workload through the public API with host buffers: per step, the
-    token's x and router logits go host->device from pinned memory, the router
-    and the MoE FFN run, and y comes back device->host."""
+    """Same workload through the C-ABI call with host buffers
+    (moe_ffn_forward_host): per step, the token's x and router logits go
+    host->device from pinned memory, the router and the MoE FFN run, and y comes
+    back device->host, all enqueued by one call."""
     import torch
     import block_quantized_moe_rocmfpx_b200 as rfx
     q = wl.q
@@ -537,18 +538,9 @@ def e2e(wl, steps, stream):
     xh = torch.from_numpy(wl.x_h).view(torch.bfloat16).view(wl.ntok, q, H).pin_memory()
     lh = torch.from_numpy(wl.logits_h).view(wl.ntok, q, E).pin_memory()
     yh = torch.empty((n, q, H), dtype=torch.float32).pin_memory()
-    xd = torch.empty((q, H), dtype=torch.bfloat16, device=wl.dev)
-    ld = torch.empty((q, E), dtype=torch.float32, device=wl.dev)
-    idx = torch.empty((q, K_TOP), dtype=torch.int32, device=wl.dev)
-    w = torch.empty((q, K_TOP), dtype=torch.float32, device=wl.dev)
-    yd = torch.empty((q, H), dtype=torch.float32, device=wl.dev)
 
     def one(t):
-        xd.copy_(xh[t], non_blocking=True)
-        ld.copy_(lh[t], non_blocking=True)
-        rfx.moe_router_topk(ld, K_TOP, idx, w)
-        wl.layers[t % wl.copies].forward(xd, idx, w, yd)
-        yh[t].copy_(yd, non_blocking=True)
+        wl.layers[t % wl.copies].forward_host(xh[t], lh[t], yh[t], stream)
 
     with torch.cuda.stream(stream):
         for t in range(5):

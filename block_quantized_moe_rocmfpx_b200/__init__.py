@@ -61,6 +61,8 @@ _ws_bytes = _proto("moe_ffn_workspace_bytes", _sz, [_vp, _i32])
 _ws_init = _proto("rfx_ws_init", _i32, [_vp, _sz, _vp])
 _ws_status = _proto("rfx_ws_status", _i32, [_vp, _vp])
 _forward = _proto("moe_ffn_forward", _i32, [_vp, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp])
+_host_scratch = _proto("moe_ffn_host_scratch_bytes", _sz, [_vp, _i32])
+_forward_host = _proto("moe_ffn_forward_host", _i32, [_vp, _vp, _vp, _i32, _vp, _vp, _sz, _vp])
 _forward_static = _proto("moe_ffn_forward_static", _i32, [_vp, _vp, _i32, _vp, _vp, _vp, _vp])
 _rms = _proto("moe_rms_norm_bf16", _i32, [_vp, _i32, _i32, _vp, _vp])
 _stack_ws = _proto("moe_stack_workspace_bytes", _sz, [_vp, _i32, _i32])
@@ -80,7 +82,8 @@ EXPORTED = ["rfx_last_error", "rfx_packed_bytes", "rfx_pack", "rfx_unpack", "rfx
             "rfx_gemv_q", "moe_layer_create", "moe_layer_destroy", "moe_ffn_workspace_bytes", "rfx_ws_init",
             "rfx_ws_status", "moe_ffn_forward", "moe_ffn_forward_static", "moe_rms_norm_bf16",
             "moe_stack_workspace_bytes", "moe_stack_forward", "moe_prefill_workspace_bytes", "moe_ffn_prefill",
-            "moe_prefill_view", "moe_router_logits", "moe_router_project_topk"]
+            "moe_prefill_view", "moe_router_logits", "moe_router_project_topk",
+            "moe_ffn_host_scratch_bytes", "moe_ffn_forward_host"]
 
 
 class RfxError(RuntimeError):
@@ -206,6 +209,17 @@ def moe_ffn_forward(handle: int, x, T: int, idx, w, y, ws, stream=None):
                     _stream(stream)))
 
 
+def moe_ffn_host_scratch_bytes(handle: int, T: int) -> int:
+    return int(_host_scratch(handle, T))
+
+
+def moe_ffn_forward_host(handle: int, x, logits, T: int, y, scratch, stream=None):
+    """Router + MoE FFN from host buffers (x bf16 [T][H], logits fp32 [T][E], y fp32
+    [T][H], pinned CPU tensors or arrays); scratch: device, zeroed once."""
+    _check(_forward_host(handle, _ptr(x), _ptr(logits), T, _ptr(y), _ptr(scratch),
+                         scratch.numel() * scratch.element_size(), _stream(stream)))
+
+
 def moe_ffn_forward_static(handle: int, x, T: int, idx, w, y, stream=None):
     """moe_ffn_forward with the library's built-in 16 MiB workspace, for callers
     that cannot allocate device memory (see include/rfx.h)."""
@@ -298,6 +312,23 @@ class MoeLayer:
         if T > self.max_T:
             raise ValueError(f"T={T} > max_T={self.max_T}")
         moe_ffn_forward(self.handle, x, T, idx, w, y, self.ws, stream)
+
+    def forward_host(self, x, logits, y, stream=None):
+        """Router + FFN from host buffers (see moe_ffn_forward_host); the device
+        scratch is kept on the layer (grown on demand, zeroed when made)."""
+        import torch
+        T = x.shape[0]
+        nbytes = moe_ffn_host_scratch_bytes(self.handle, T)
+        if nbytes == 0:
+            raise RfxError(-2, f"unsupported T={T}")
+        if getattr(self, "host_scratch", None) is None or self.host_scratch.numel() < nbytes:
+            self.host_scratch = torch.empty(nbytes, dtype=torch.uint8, device=self.ws.device)
+            rfx_ws_init(self.host_scratch)
+        moe_ffn_forward_host(self.handle, x, logits, T, y, self.host_scratch, stream)
+
+    def host_status(self, stream=None) -> int:
+        """Device flag of the host-call scratch (its workspace comes first)."""
+        return rfx_ws_status(self.host_scratch, stream)
 
     def prefill(self, x, idx, w, y, stream=None):
         """moe_ffn_prefill with a workspace kept on the layer (grown on demand)."""

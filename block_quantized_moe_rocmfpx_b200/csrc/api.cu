@@ -251,6 +251,69 @@ extern "C" int moe_ffn_forward(const moe_layer* layer, const void* x, int T, con
     return e == cudaSuccess ? RFX_OK : cuda_fail("moe_ffn_forward", e);
 }
 
+// ------------------------------------------------------------ host buffers ---
+
+namespace {
+
+// Host-call scratch: the moe_ffn_forward workspace first (so rfx_ws_status
+// reads its error flag at offset 0), then the device copies and the routing.
+struct HostScratch {
+    size_t ffn, x, logits, idx, w, y, total;
+};
+
+HostScratch host_scratch_layout(const moe_layer_desc& d, int T, size_t ffn_bytes) {
+    auto up = [](size_t n) { return (n + 255) / 256 * 256; };
+    HostScratch S;
+    S.ffn = 0;
+    S.x = up(ffn_bytes);
+    S.logits = S.x + up((size_t)T * d.H * 2);
+    S.idx = S.logits + up((size_t)T * d.E * 4);
+    S.w = S.idx + up((size_t)T * d.k * 4);
+    S.y = S.w + up((size_t)T * d.k * 4);
+    S.total = S.y + up((size_t)T * d.H * 4);
+    return S;
+}
+
+}  // namespace
+
+extern "C" size_t moe_ffn_host_scratch_bytes(const moe_layer* layer, int T) {
+    if (!layer || T < 1) return 0;
+    const size_t ffn = moe_ffn_workspace_bytes(layer, T);
+    if (!ffn) return 0;
+    return host_scratch_layout(layer->d, T, ffn).total;
+}
+
+extern "C" int moe_ffn_forward_host(const moe_layer* layer, const void* x, const float* logits, int T, float* y,
+                                    void* scratch, size_t scratch_bytes, void* stream) {
+    if (!layer) return rfx_fail(RFX_EINVAL, "moe_ffn_forward_host: null layer");
+    if (T < 1) return rfx_fail(RFX_EINVAL, "moe_ffn_forward_host: T >= 1");
+    if (!x || !logits || !y || !scratch) return rfx_fail(RFX_EINVAL, "moe_ffn_forward_host: null pointer");
+    if ((uintptr_t)scratch & 255u) return rfx_fail(RFX_EINVAL, "moe_ffn_forward_host: scratch must be 256-byte aligned");
+    const size_t ffn = moe_ffn_workspace_bytes(layer, T);
+    if (!ffn) return rfx_fail(RFX_EUNSUPPORTED, "moe_ffn_forward_host: no workspace size for this layer and T");
+    const moe_layer_desc& d = layer->d;
+    const HostScratch S = host_scratch_layout(d, T, ffn);
+    if (scratch_bytes < S.total)
+        return rfx_fail(RFX_EINVAL, "moe_ffn_forward_host: scratch smaller than moe_ffn_host_scratch_bytes");
+    uint8_t* b = (uint8_t*)scratch;
+    void* xd = b + S.x;
+    float* ld = (float*)(b + S.logits);
+    int32_t* idx = (int32_t*)(b + S.idx);
+    float* w = (float*)(b + S.w);
+    float* yd = (float*)(b + S.y);
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = cudaMemcpyAsync(xd, x, (size_t)T * d.H * 2, cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return cuda_fail("moe_ffn_forward_host", e);
+    e = cudaMemcpyAsync(ld, logits, (size_t)T * d.E * 4, cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return cuda_fail("moe_ffn_forward_host", e);
+    int rc = moe_router_topk(ld, T, d.E, d.k, idx, w, stream);
+    if (rc != RFX_OK) return rc;
+    rc = moe_ffn_forward(layer, xd, T, idx, w, yd, b + S.ffn, S.x, stream);
+    if (rc != RFX_OK) return rc;
+    e = cudaMemcpyAsync(y, yd, (size_t)T * d.H * 4, cudaMemcpyDeviceToHost, st);
+    return e == cudaSuccess ? RFX_OK : cuda_fail("moe_ffn_forward_host", e);
+}
+
 // ---------------------------------------------------------------- prefill ---
 
 namespace {

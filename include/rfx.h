@@ -249,6 +249,22 @@ int moe_ffn_forward(const moe_layer* layer, const void* x, int T, const int32_t*
                     float* y, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * The same step from host buffers: x (bf16 bits [T][H]) and the router
+ * logits (fp32 [T][E]) are copied host -> device, moe_router_topk and
+ * moe_ffn_forward run, and y (fp32 [T][H]) is copied device -> host, all
+ * enqueued on `stream` (one cudaMemcpyAsync per buffer; the host buffers should
+ * be pinned for the copies to be asynchronous; y is valid after the stream
+ * synchronises).  scratch: device, 256-byte aligned,
+ * moe_ffn_host_scratch_bytes(layer, T) bytes, caller-owned, zeroed once with
+ * rfx_ws_init before its first use; it holds the moe_ffn_forward workspace
+ * first (so rfx_ws_status(scratch) reads its device flag), then the device
+ * copies and the routing.  T > 8 runs the prefill path.
+ */
+size_t moe_ffn_host_scratch_bytes(const moe_layer* layer, int T);
+int moe_ffn_forward_host(const moe_layer* layer, const void* x, const float* logits, int T, float* y, void* scratch,
+                         size_t scratch_bytes, void* stream);
+
+/*
  * Prefill: the same MoE FFN for many tokens as a grouped GEMM on the tcgen05
  * tensor cores ([AI] "Lucebox 的优化三板斧" and [MZ] "MoE 专家并行" for the
  * layer; the page pair's prefill runs the experts as dense contractions).

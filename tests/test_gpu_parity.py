@@ -226,3 +226,45 @@ def test_moe_bad_expert_ids_set_the_device_flag(full_layer):
     ml.forward(x, idx, w, y)
     assert ml.status() == rfx.RFX_EDEVICE
     assert ml.status() == rfx.RFX_OK          # the flag is cleared once read
+
+
+@pytest.mark.parametrize("T", [1, 4])
+def test_forward_host_equals_device_path(full_layer, T):
+    """moe_ffn_forward_host (host x / logits in, host y out, one call) gives the
+    bits of the router call and moe_ffn_forward on device buffers."""
+    ml = full_layer.moe_layer()
+    L = synth.logits(8, 0, 60 * T, T, 256, 1.1)
+    xb = synth.x_bf16(8, 60 * T, T, 4096)
+    idx = torch.empty((T, 6), dtype=torch.int32, device=DEV)
+    w = torch.empty((T, 6), dtype=torch.float32, device=DEV)
+    y = torch.empty((T, 4096), dtype=torch.float32, device=DEV)
+    rfx.moe_router_topk(to_dev(L), 6, idx, w)
+    ml.forward(to_dev(xb, torch.bfloat16), idx, w, y)
+    xh = torch.from_numpy(xb).view(torch.bfloat16).pin_memory()
+    lh = torch.from_numpy(L).pin_memory()
+    yh = torch.full((T, 4096), float("nan"), dtype=torch.float32).pin_memory()
+    for _ in range(2):                          # the scratch is reused
+        ml.forward_host(xh, lh, yh)
+        torch.cuda.synchronize()
+        assert torch.equal(yh, y.cpu())
+    assert ml.host_status() == rfx.RFX_OK
+    assert ml.status() == rfx.RFX_OK
+
+
+def test_forward_host_prefill_path():
+    H, I, E, k, T = 512, 256, 16, 4, 40
+    lay = SynthLayer(29, 0, H, I, E, k)
+    ml = lay.moe_layer(max_T=T)
+    L = synth.logits(29, 0, 0, T, E, 1.1)
+    xb = synth.x_bf16(29, 0, T, H)
+    idx = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    w = torch.empty((T, k), dtype=torch.float32, device=DEV)
+    y = torch.empty((T, H), dtype=torch.float32, device=DEV)
+    rfx.moe_router_topk(to_dev(L), k, idx, w)
+    ml.prefill(to_dev(xb, torch.bfloat16), idx, w, y)
+    yh = torch.empty((T, H), dtype=torch.float32).pin_memory()
+    ml.forward_host(torch.from_numpy(xb).view(torch.bfloat16).pin_memory(), torch.from_numpy(L).pin_memory(), yh)
+    torch.cuda.synchronize()
+    # the prefill combine adds with fp32 atomics: equal up to the order of the adds
+    assert torch.allclose(yh, y.cpu(), rtol=1e-5, atol=1e-5)
+    assert ml.host_status() == rfx.RFX_OK
