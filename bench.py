@@ -59,6 +59,7 @@ def parse():
     ap.add_argument("--prefill-only", action="store_true", help="time only the prefill (T = 2048 and 8192)")
     ap.add_argument("--prefill-steps", type=int, default=20)
     ap.add_argument("--no-router-proj", action="store_true", help="skip the router projection measurement")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the q = 2, 3, 5 and uniform-routing decode sweep")
     ap.add_argument("--router-proj-only", action="store_true", help="time only the router projection + top-k")
     return ap.parse_args()
 
@@ -220,7 +221,7 @@ def run_reference(args, rank, world):
 class Workload:
     """C rotating copies of one synthetic full-size layer plus seeded inputs."""
 
-    def __init__(self, q: int, ntok: int, dev, copies: int = COPIES):
+    def __init__(self, q: int, ntok: int, dev, copies: int = COPIES, zipf_s: float = ZIPF_S):
         import torch
         import numpy as np
         import synth
@@ -242,7 +243,7 @@ class Workload:
         torch.cuda.synchronize()
         self.ntok = ntok
         nb = ntok * q
-        self.logits_h = synth.logits(SEED, 0, 0, nb, E, ZIPF_S)
+        self.logits_h = synth.logits(SEED, 0, 0, nb, E, zipf_s)
         self.x_h = synth.x_bf16(SEED, 0, nb, H)
         self.logits = torch.from_numpy(self.logits_h).to(dev).view(ntok, q, E)
         self.x = torch.from_numpy(self.x_h).view(torch.bfloat16).to(dev).view(ntok, q, H)
@@ -476,10 +477,11 @@ def time_graph(g, stream):
     return e0.elapsed_time(e1)
 
 
-def measure(q: int, steps: int, warmup: int, dev, rank, world, want_clocks: bool, want_e2e: bool, copies: int):
+def measure(q: int, steps: int, warmup: int, dev, rank, world, want_clocks: bool, want_e2e: bool, copies: int,
+            zipf_s: float = ZIPF_S):
     import torch
     import torch.distributed as dist
-    wl = Workload(q, NTOK, dev, copies)
+    wl = Workload(q, NTOK, dev, copies, zipf_s)
     stream = torch.cuda.Stream(device=dev)
     with torch.cuda.stream(stream):
         for t in range(3):            # eager warm-up (kernel attributes, lazy loading)
@@ -508,7 +510,9 @@ def measure(q: int, steps: int, warmup: int, dev, rank, world, want_clocks: bool
     ms_ffn = time_graph(g_ffn, stream)
     status = max(ml.status() for ml in wl.layers[:1])
     abytes = wl.algo_bytes(range(off, off + steps))
-    res = {"ms": ms, "ms_ffn": ms_ffn, "bytes": abytes, "clocks": clk, "status": status}
+    idx_all = wl.idx.cpu().numpy()
+    union = sum(len(set(idx_all[(off + t) % wl.ntok].ravel().tolist())) for t in range(steps)) / steps
+    res = {"ms": ms, "ms_ffn": ms_ffn, "bytes": abytes, "clocks": clk, "status": status, "union": union}
     if want_e2e:
         res["e2e"] = e2e(wl, steps, stream)
     del g_warm, g_main, g_ffn
@@ -612,6 +616,21 @@ def main():
         e2e_ms = reduce_max(r1["e2e"]["steps"] / r1["e2e"]["value"] * 1e3)
         e2e_v = dict(r1["e2e"])
         e2e_v["value"] = world * r1["e2e"]["steps"] / (e2e_ms / 1e3)
+    sweep = None
+    if not args.no_sweep:
+        # verify widths and routing modes beside the headline (Zipf q=1 / q=4): the
+        # same layer, fewer steps; the kernel-only time and the measured union size
+        peak_s, _ = peaks()
+        sweep = []
+        for q, zs in ((2, ZIPF_S), (3, ZIPF_S), (5, ZIPF_S), (1, 0.0), (4, 0.0)):
+            n = min(args.steps, 200)
+            r = measure(q, n, max(3, args.warmup), dev, rank, world, False, False, args.copies, zs)
+            ms_f = reduce_max(r["ms_ffn"])
+            gbs = r["bytes"] / (ms_f / 1e3) / 1e9
+            sweep.append({"q": q, "routing": "zipf(1.1)" if zs > 0 else "uniform", "steps": n,
+                          "kernel_us": ms_f * 1e3 / n, "tokens_per_s_step": world * q * n / (reduce_max(r["ms"]) / 1e3),
+                          "achieved_gbs": gbs, "frac": gbs / peak_s, "union_experts": r["union"],
+                          "algo_bytes_per_launch": r["bytes"] / n, "device_status": r["status"]})
     rp = None
     if not args.no_router_proj:
         rp = [measure_router_proj(T, min(args.steps, 400), max(3, args.warmup), dev) for T in ROUTER_PROJ_TS]
@@ -641,6 +660,7 @@ def main():
                          "algo_bytes_per_launch": r1["bytes"] / args.steps,
                          "kernel_us": r1["ms_ffn"] * 1e3 / args.steps},
             "q4": {"value": world * 4 * args.steps / (ms4 / 1e3), "unit": "tokens/s", "ms_per_step": ms4 / args.steps,
+                   "union_experts": r4["union"],
                    "achieved_gbs": gbs4, "frac": gbs4 / peak, "kernel_us": r4["ms_ffn"] * 1e3 / args.steps,
                    "algo_bytes_per_launch": r4["bytes"] / args.steps},
             "cpu_baseline": base,
@@ -650,6 +670,7 @@ def main():
             "device_status": {"q1": r1["status"], "q4": r4["status"]},
             "prefill": pf,
             "router_projection": rp,
+            "q_sweep": sweep,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
