@@ -241,6 +241,8 @@ int moe_prepare(const moe_layer* layer, const void* x, int T, const int32_t* idx
 
 extern "C" int moe_ffn_forward(const moe_layer* layer, const void* x, int T, const int32_t* idx, const float* w,
                                float* y, void* ws, size_t ws_bytes, void* stream) {
+    if (!layer) return rfx_fail(RFX_EINVAL, "moe_ffn_forward: null layer");
+    if (T == 0) return RFX_OK;   // no token columns: nothing to do
     if (T > MOE_MAXT) return moe_ffn_prefill(layer, x, T, idx, w, y, ws, ws_bytes, stream);
     rfx::MoeParams p;
     int grid = 0;
@@ -286,7 +288,8 @@ extern "C" size_t moe_ffn_host_scratch_bytes(const moe_layer* layer, int T) {
 extern "C" int moe_ffn_forward_host(const moe_layer* layer, const void* x, const float* logits, int T, float* y,
                                     void* scratch, size_t scratch_bytes, void* stream) {
     if (!layer) return rfx_fail(RFX_EINVAL, "moe_ffn_forward_host: null layer");
-    if (T < 1) return rfx_fail(RFX_EINVAL, "moe_ffn_forward_host: T >= 1");
+    if (T == 0) return RFX_OK;   // no token columns: nothing to do
+    if (T < 1) return rfx_fail(RFX_EINVAL, "moe_ffn_forward_host: T >= 0");
     if (!x || !logits || !y || !scratch) return rfx_fail(RFX_EINVAL, "moe_ffn_forward_host: null pointer");
     if ((uintptr_t)scratch & 255u) return rfx_fail(RFX_EINVAL, "moe_ffn_forward_host: scratch must be 256-byte aligned");
     const size_t ffn = moe_ffn_workspace_bytes(layer, T);
@@ -343,6 +346,7 @@ extern "C" size_t moe_prefill_workspace_bytes(const moe_layer* layer, int T) {
 
 extern "C" int moe_ffn_prefill(const moe_layer* layer, const void* x, int T, const int32_t* idx, const float* w,
                                float* y, void* ws, size_t ws_bytes, void* stream) {
+    if (layer && T == 0) return RFX_OK;   // no tokens: nothing to do
     int rc = prefill_check(layer, T, "moe_ffn_prefill");
     if (rc != RFX_OK) return rc;
     if (!x || !idx || !w || !y || !ws) return rfx_fail(RFX_EINVAL, "moe_ffn_prefill: null pointer");
@@ -450,6 +454,7 @@ extern "C" size_t moe_stack_workspace_bytes(const moe_layer* const* layers, int 
 
 extern "C" int moe_stack_forward(const moe_layer* const* layers, int L, const float* logits, const void* x, int T,
                                  float* y, void* ws, size_t ws_bytes, void* stream) {
+    if (layers && L >= 1 && T == 0) return RFX_OK;   // no token columns: nothing to do
     int rc = stack_check(layers, L, T, "moe_stack_forward");
     if (rc != RFX_OK) return rc;
     if (!logits || !x || !y || !ws) return rfx_fail(RFX_EINVAL, "moe_stack_forward: null pointer");

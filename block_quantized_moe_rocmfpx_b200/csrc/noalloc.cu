@@ -70,6 +70,7 @@ int static_ws_address(void** out) {
 extern "C" int moe_ffn_forward_static(const moe_layer* layer, const void* x, int T, const int32_t* idx,
                                       const float* w, float* y, void* stream) {
     if (!layer) return rfx_fail(RFX_EINVAL, "moe_ffn_forward_static: null layer");
+    if (T == 0) return RFX_OK;   // no token columns: nothing to do
     const size_t need = moe_ffn_workspace_bytes(layer, T);
     if (need == 0) return rfx_fail(RFX_EUNSUPPORTED, "moe_ffn_forward_static: 1 <= T <= 8 token columns");
     if (need > RFX_STATIC_WS_BYTES)

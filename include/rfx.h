@@ -236,7 +236,8 @@ int rfx_ws_status(void* ws, void* stream);
  * and decoded once and applied to every column routed to that expert.
  * x: device bf16 bits [T][H].  idx: device int32 [T][k], distinct per row,
  * in [0, E).  w: device fp32 [T][k].  y: device fp32 [T][H].
- * Limits: 1 <= T <= 8 (decode / verify), H % 32 == 0, I % 32 == 0, k <= 8.
+ * Limits: 1 <= T <= 8 (decode / verify), H % 32 == 0, I % 32 == 0, k <= 8;
+ * T == 0 is a no-op (so for every call below that takes T).
  * T > 8 runs moe_ffn_prefill instead (bf16 operands; its own limits and
  * workspace size).
  * One cooperative launch of one CTA per SM (all CTAs resident at once: the

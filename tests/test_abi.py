@@ -218,3 +218,27 @@ def test_layer_create_validation():
         rfx.moe_layer_create(bad)
     lib = ctypes.CDLL(rfx.LIB_PATH)
     assert lib.moe_ffn_forward(None, None, 1, None, None, None, None, 0, None) == rfx.RFX_EINVAL
+
+
+def test_zero_token_calls_are_noops():
+    """T = 0 returns OK without touching any buffer (reading: an empty batch is
+    a no-op), for every entry point that takes T."""
+    lib = ctypes.CDLL(rfx.LIB_PATH)
+    d = rfx.moe_layer_desc()
+    d.H, d.I, d.E, d.k = 512, 256, 8, 2
+    d.f_gate, d.f_up, d.f_down = 2, 2, 3
+    d.gate = d.up = d.down = 256
+    d.stride_gate = d.stride_up = rfx.rfx_packed_bytes(2, 256, 512)
+    d.stride_down = rfx.rfx_packed_bytes(3, 512, 256)
+    h = rfx.moe_layer_create(d)
+    try:
+        assert lib.moe_ffn_forward(ctypes.c_void_p(h), None, 0, None, None, None, None, 0, None) == rfx.RFX_OK
+        assert lib.moe_ffn_prefill(ctypes.c_void_p(h), None, 0, None, None, None, None, 0, None) == rfx.RFX_OK
+        assert lib.moe_ffn_forward_static(ctypes.c_void_p(h), None, 0, None, None, None, None) == rfx.RFX_OK
+        assert lib.moe_ffn_forward_host(ctypes.c_void_p(h), None, None, 0, None, None, 0, None) == rfx.RFX_OK
+        arr = (ctypes.c_void_p * 1)(h)
+        assert lib.moe_stack_forward(arr, 1, None, None, 0, None, None, 0, None) == rfx.RFX_OK
+        # a null layer is still an error
+        assert lib.moe_ffn_forward(None, None, 0, None, None, None, None, 0, None) == rfx.RFX_EINVAL
+    finally:
+        rfx.moe_layer_destroy(h)
