@@ -268,3 +268,22 @@ def test_forward_host_prefill_path():
     # the prefill combine adds with fp32 atomics: equal up to the order of the adds
     assert torch.allclose(yh, y.cpu(), rtol=1e-5, atol=1e-5)
     assert ml.host_status() == rfx.RFX_OK
+
+
+@pytest.mark.parametrize("T", [1, 3])
+def test_moe_wide_hidden_top8(T):
+    """H = 7168 (a DeepSeek-V3-like hidden size), top-8 of 256 + shared: the
+    widest decode shape tested; at T = 3 the x staging leaves room for a
+    2-stage ring only."""
+    H, I, E, k = 7168, 2048, 256, 8
+    lay = SynthLayer(91, 0, H, I, E, k)
+    L = synth.logits(91, 0, 0, T, E, 1.1)
+    xb = synth.x_bf16(91, 0, T, H)
+    ml, idx, w, y = run_layer(lay, L, xb, T, k)
+    idx_o, w_o = oracle.router_topk(L, k)
+    assert np.array_equal(idx, idx_o)
+    ol = OracleLayer(lay)
+    xf = synth.bf16_to_f64(xb)
+    for t in range(T):
+        ref, mag = ol.token(xf[t], idx_o[t], w_o[t])
+        check_close(y[t], ref, mag, what=f"H={H} top-{k} T={T} t={t}")

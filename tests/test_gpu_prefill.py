@@ -304,3 +304,50 @@ def test_prefill_repeated_expert_in_a_row_counts_twice():
     xb = synth.x_bf16(73, 0, T, 512)
     y, v = _prefill_with_idx(lay, T, idx, w, xb)
     _check_against_oracle(lay, idx, w, xb, y, v, tokens=[3, 11, 0, 19])
+
+
+def test_prefill_max_tokens(full_layer):
+    """T = 65536, the call's maximum: the whole grouping against the oracle,
+    h and y (teacher-forced) on sampled tokens (only their h rows are copied)."""
+    lay, T, k = full_layer, 65536, 6
+    logits = synth.logits(0, 0, 200000, T, 256, 1.1)
+    xb = synth.x_bf16(0, 200000, T, 4096)
+    ml = lay.moe_layer()
+    idx_d = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    w_d = torch.empty((T, k), dtype=torch.float32, device=DEV)
+    rfx.moe_router_topk(to_dev(logits), k, idx_d, w_d)
+    y_d = torch.full((T, lay.H), float("nan"), dtype=torch.float32, device=DEV)
+    ml.prefill(to_dev(xb, torch.bfloat16), idx_d, w_d, y_d)
+    assert ml.prefill_status() == rfx.RFX_OK, rfx.rfx_last_error()
+    idx, w = idx_d.cpu().numpy(), w_d.cpu().numpy()
+    idx_o, w_o = oracle.router_topk(logits, k)
+    assert np.array_equal(idx, idx_o)
+    v = ml.prefill_view(T)
+    counts, ent = check_grouping(idx, w, v, lay.E)
+    assert int(counts.sum()) == T * k
+    tokens = [0, 1, 4097, 32768, 65534, 65535]
+    row_of = np.empty(T * k, dtype=np.int64)
+    row_of[ent] = np.arange(ent.size)
+    rows = [int(row_of[t * k + j]) for t in tokens for j in range(k)] + [T * k + t for t in tokens]
+    h_rows = bf16_bits_to_f64(v["h"][torch.tensor(rows, device=DEV)])
+    hmap = dict(zip(rows, h_rows))
+    ol = OracleLayer(lay)
+    xf = synth.bf16_to_f64(xb[tokens])
+    y = y_d[torch.tensor(tokens, device=DEV)].cpu().numpy()
+    hc = HCheck()
+    for i, t in enumerate(tokens):
+        yt, mt = np.zeros(lay.H), np.zeros(lay.H)
+        for j in range(k):
+            mats = ol.expert(int(idx[t, j]))
+            hr = hmap[int(row_of[t * k + j])]
+            hc.add(hr, mats, xf[i], f"h token {t} slot {j}")
+            d, m = oracle.gemv(mats[2], hr[None, :], bf16_weights=True)
+            yt += w_o[t, j] * d[0]
+            mt += abs(w_o[t, j]) * m[0]
+        hs = hmap[T * k + t]
+        hc.add(hs, ol.shared(), xf[i], f"h token {t} shared")
+        d, m = oracle.gemv(ol.shared()[2], hs[None, :], bf16_weights=True)
+        yt += d[0]
+        mt += m[0]
+        check_close(y[i], yt, mt, what=f"teacher-forced token {t}")
+    hc.done()
