@@ -46,34 +46,41 @@ def lib():
     with _lock:
         if _lib is None:
             build()
-            L = ctypes.CDLL(_SO)
-            i32, i64, vp, dbl = ctypes.c_int, ctypes.c_int64, ctypes.c_void_p, ctypes.c_double
-            L.oracle_block_bytes.restype = i32
-            L.oracle_block_bytes.argtypes = [i32]
-            L.oracle_bits_per_weight.restype = dbl
-            L.oracle_bits_per_weight.argtypes = [i32]
-            L.oracle_level.restype = dbl
-            L.oracle_level.argtypes = [i32, i32]
-            L.oracle_bf16_round.restype = dbl
-            L.oracle_bf16_round.argtypes = [dbl]
-            L.oracle_silu.restype = dbl
-            L.oracle_silu.argtypes = [dbl]
-            L.oracle_dequant.restype = i32
-            L.oracle_dequant.argtypes = [i32, vp, vp, i64, i64, vp]
-            L.oracle_gemv.restype = i32
-            L.oracle_gemv.argtypes = [i32, vp, vp, i64, i64, vp, i32, vp, vp]
-            L.oracle_gemv_bf16w.restype = i32
-            L.oracle_gemv_bf16w.argtypes = [i32, vp, vp, i64, i64, vp, i32, vp, vp]
-            L.oracle_router_topk.restype = i32
-            L.oracle_router_topk.argtypes = [vp, i64, i32, i32, vp, vp]
-            L.oracle_expert_ffn.restype = i32
-            L.oracle_expert_ffn.argtypes = [i32, i32, vp, vp, vp, vp, i32, vp, vp, vp]
-            L.oracle_moe_token.restype = i32
-            L.oracle_moe_token.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp, vp, i32, vp, vp]
-            L.oracle_rms_bf16.restype = None
-            L.oracle_rms_bf16.argtypes = [vp, i64, vp]
-            _lib = L
+            _lib = load(_SO)
     return _lib
+
+
+def load(path: str):
+    """A compiled oracle library at `path` with the argument types set (lib()
+    uses it for the library built here; the mutation test for a planted-bug
+    copy)."""
+    L = ctypes.CDLL(path)
+    i32, i64, vp, dbl = ctypes.c_int, ctypes.c_int64, ctypes.c_void_p, ctypes.c_double
+    L.oracle_block_bytes.restype = i32
+    L.oracle_block_bytes.argtypes = [i32]
+    L.oracle_bits_per_weight.restype = dbl
+    L.oracle_bits_per_weight.argtypes = [i32]
+    L.oracle_level.restype = dbl
+    L.oracle_level.argtypes = [i32, i32]
+    L.oracle_bf16_round.restype = dbl
+    L.oracle_bf16_round.argtypes = [dbl]
+    L.oracle_silu.restype = dbl
+    L.oracle_silu.argtypes = [dbl]
+    L.oracle_dequant.restype = i32
+    L.oracle_dequant.argtypes = [i32, vp, vp, i64, i64, vp]
+    L.oracle_gemv.restype = i32
+    L.oracle_gemv.argtypes = [i32, vp, vp, i64, i64, vp, i32, vp, vp]
+    L.oracle_gemv_bf16w.restype = i32
+    L.oracle_gemv_bf16w.argtypes = [i32, vp, vp, i64, i64, vp, i32, vp, vp]
+    L.oracle_router_topk.restype = i32
+    L.oracle_router_topk.argtypes = [vp, i64, i32, i32, vp, vp]
+    L.oracle_expert_ffn.restype = i32
+    L.oracle_expert_ffn.argtypes = [i32, i32, vp, vp, vp, vp, i32, vp, vp, vp]
+    L.oracle_moe_token.restype = i32
+    L.oracle_moe_token.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp, vp, i32, vp, vp]
+    L.oracle_rms_bf16.restype = None
+    L.oracle_rms_bf16.argtypes = [vp, i64, vp]
+    return L
 
 
 def _p(a):
