@@ -369,3 +369,20 @@ def test_router_logits_brute_force():
             m += abs(float(b[e]))
             assert abs(lg[t, e] - s) <= 1e-14 * m
             assert abs(mag[t, e] - m) <= 1e-14 * m
+
+
+def test_moe_token_with_a_format_per_expert():
+    """ROCmFPX MIX (a format chosen per expert and matrix): each expert's
+    matrices decode with their own format; the token equals the dense sum."""
+    H, I = 64, 32
+    fmts = [(2, 2, 3), (3, 3, 2), (4, 4, 4), (2, 3, 4)]   # (gate, up, down) per expert
+    ex = [tuple(oracle.Mat(b, *(lambda s: (s.codes(), s.scales()))(synth.MatrixSpec(33, 0, kind, e, b, r, c)))
+                for kind, b, r, c in zip((0, 1, 2), f, (I, I, H), (H, H, I))) for e, f in enumerate(fmts)]
+    _, sh = _tiny_layer(33)
+    x = synth.bf16_to_f64(synth.x_bf16(3, 0, 1, H))[0]
+    sel, w = [3, 1, 2], np.array([0.5, 0.3, 0.2])
+    y, mag = oracle.moe_token([ex[e] for e in sel], w, sh, x)
+    ref = sum(wj * _dense_ffn(ex[e], x)[0] for wj, e in zip(w, sel)) + _dense_ffn(sh, x)[0]
+    refm = sum(wj * _dense_ffn(ex[e], x)[1] for wj, e in zip(w, sel)) + _dense_ffn(sh, x)[1]
+    np.testing.assert_allclose(y, ref, rtol=0, atol=1e-13 * refm.max())
+    np.testing.assert_allclose(mag, refm, rtol=1e-12)
