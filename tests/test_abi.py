@@ -242,3 +242,24 @@ def test_zero_token_calls_are_noops():
         assert lib.moe_ffn_forward(None, None, 0, None, None, None, None, 0, None) == rfx.RFX_EINVAL
     finally:
         rfx.moe_layer_destroy(h)
+
+
+def test_host_call_scratch_bytes():
+    """moe_ffn_host_scratch_bytes = the moe_ffn_forward workspace (decode or
+    prefill) + the padded device copies of x, logits, idx, w and y."""
+    d = rfx.moe_layer_desc()
+    d.H, d.I, d.E, d.k = 4096, 2048, 256, 6
+    d.f_gate, d.f_up, d.f_down = 2, 2, 3
+    d.gate = d.up = d.down = 256
+    d.stride_gate = d.stride_up = rfx.rfx_packed_bytes(2, 2048, 4096)
+    d.stride_down = rfx.rfx_packed_bytes(3, 4096, 2048)
+    h = rfx.moe_layer_create(d)
+    try:
+        up = lambda n: (n + 255) // 256 * 256
+        for T in (1, 4, 8, 9, 2048):
+            ws = rfx.moe_ffn_workspace_bytes(h, T)
+            want = up(ws) + up(T * 4096 * 2) + up(T * 256 * 4) + 2 * up(T * 6 * 4) + up(T * 4096 * 4)
+            assert rfx.moe_ffn_host_scratch_bytes(h, T) == want, T
+        assert rfx.moe_ffn_host_scratch_bytes(h, 0) == 0
+    finally:
+        rfx.moe_layer_destroy(h)
