@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstring>
 #include <new>
 #include <string>
@@ -29,24 +30,30 @@ int cuda_fail(const char* where, cudaError_t e) {
     return rfx_fail(RFX_ECUDA, std::string(where) + ": " + cudaGetErrorString(e));
 }
 
-// SM count and opt-in shared memory of the current device, queried once per device.
+// SM count and opt-in shared memory of the current device, queried once per
+// device (thread-safe: the shared-memory size is published before the SM
+// count, and a reader that sees the count sees the size).
 int device_props(int& sms, int& smem_optin) {
-    static int cache_sms[64] = {0}, cache_smem[64] = {0};
+    static std::atomic<int> cache_sms[64] = {}, cache_smem[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
-    if (dev < 64 && cache_sms[dev]) {
-        sms = cache_sms[dev];
-        smem_optin = cache_smem[dev];
-        return RFX_OK;
+    const bool cached = dev >= 0 && dev < 64;
+    if (cached) {
+        const int s = cache_sms[dev].load(std::memory_order_acquire);
+        if (s) {
+            sms = s;
+            smem_optin = cache_smem[dev].load(std::memory_order_relaxed);
+            return RFX_OK;
+        }
     }
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return cuda_fail("cudaDeviceGetAttribute", e);
     e = cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (e != cudaSuccess) return cuda_fail("cudaDeviceGetAttribute", e);
-    if (dev < 64) {
-        cache_sms[dev] = sms;
-        cache_smem[dev] = smem_optin;
+    if (cached) {
+        cache_smem[dev].store(smem_optin, std::memory_order_relaxed);
+        cache_sms[dev].store(sms, std::memory_order_release);
     }
     return RFX_OK;
 }

@@ -14,6 +14,7 @@
 #include <cuda_runtime.h>
 
 #include "gemv.h"
+#include "launch_util.h"
 #include "rfx_tile.cuh"
 
 namespace rfx {
@@ -229,15 +230,9 @@ size_t gemv_smem_bytes(int q, long long K, bool x_fp32) {
 template <int FMT, bool F32X, int NB>
 static cudaError_t launch_t(const GemvParams& p, size_t smem, cudaStream_t stream) {
     auto kern = gemv_kernel<FMT, F32X, NB>;
-    static int set_bytes[64] = {0};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    static SmemLimit limit;   // one per instantiation
+    cudaError_t e = limit.ensure((const void*)kern, (int)smem);
     if (e != cudaSuccess) return e;
-    if (dev < 64 && set_bytes[dev] < (int)smem) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        set_bytes[dev] = (int)smem;
-    }
     const long long ngroups = (p.N + 15) / 16;
     const int grid = (int)((ngroups + 1) / 2);
     kern<<<grid, GEMV_WARPS * 32, smem, stream>>>(p);

@@ -39,6 +39,7 @@
 //    drains its in-flight copies and exits.
 #include <cuda_runtime.h>
 
+#include "launch_util.h"
 #include "moe_decode.h"
 #include "rfx_tile.cuh"
 
@@ -1057,17 +1058,10 @@ cudaError_t moe_decode_launch(const MoeParams& p, int grid, cudaStream_t stream)
     // the down projection's virtual columns (T <= 8)
     const int qc = p.T == 1 ? 0 : (p.T <= 4 ? 1 : 2);
     auto kern = qc == 0 ? moe_decode_kernel<1> : (qc == 1 ? moe_decode_kernel<2> : moe_decode_kernel<3>);
-    // raise the dynamic shared-memory limit once per device and kernel (not a
-    // stream operation, so it stays out of any graph capture after the first call)
-    static int set_bytes[64][3] = {{0}};
-    int dev = 0;
-    cudaError_t err = cudaGetDevice(&dev);
+    // the dynamic shared-memory limit, once per device and kernel
+    static SmemLimit limit[3];
+    cudaError_t err = limit[qc].ensure((const void*)kern, (int)smem);
     if (err != cudaSuccess) return err;
-    if (dev >= 64 || set_bytes[dev][qc] < (int)smem) {
-        err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (err != cudaSuccess) return err;
-        if (dev < 64) set_bytes[dev][qc] = (int)smem;
-    }
     // cooperative: every CTA is resident at once (the two grid barriers need it)
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);

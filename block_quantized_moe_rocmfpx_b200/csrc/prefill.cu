@@ -29,6 +29,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "launch_util.h"
 #include "moe_decode.h"
 #include "prefill.h"
 #include "rfx_layout.h"
@@ -829,19 +830,11 @@ bool make_tmap(CUtensorMap* m, const void* base, long long rows, long long cols)
 size_t pf_gemm_smem_bytes(int mode) { return mode == 0 ? PfCfg<0>::SMEM : PfCfg<1>::SMEM; }
 
 cudaError_t pf_launch(const PfParams& p, int sms, cudaStream_t stream) {
-    static bool attr_done[64] = {false};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    static SmemLimit limit[2];
+    cudaError_t e = limit[0].ensure((const void*)pf_gemm_kernel<0>, (int)pf_gemm_smem_bytes(0));
     if (e != cudaSuccess) return e;
-    if (dev < 64 && !attr_done[dev]) {
-        e = cudaFuncSetAttribute(pf_gemm_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)pf_gemm_smem_bytes(0));
-        if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(pf_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)pf_gemm_smem_bytes(1));
-        if (e != cudaSuccess) return e;
-        attr_done[dev] = true;
-    }
+    e = limit[1].ensure((const void*)pf_gemm_kernel<1>, (int)pf_gemm_smem_bytes(1));
+    if (e != cudaSuccess) return e;
     CUtensorMap tm_xp, tm_x, tm_h;
     const long long rk = (long long)p.T * p.k;
     if (!make_tmap(&tm_xp, p.xp, rk, p.H) || !make_tmap(&tm_x, p.x, p.T, p.H) ||

@@ -27,6 +27,7 @@
 #include <stdint.h>
 
 #include "gemv.h"
+#include "launch_util.h"
 #include "rfx_device.cuh"
 
 namespace rfx {
@@ -208,16 +209,9 @@ cudaError_t router_logits_launch(const uint16_t* W, const float* bias, const uin
                                  float* logits, cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
     if (T > RP_COLS) {
-        // once per device (not a stream operation: stays out of graph captures after the first call)
-        static bool attr_set[64] = {false};
-        int dev = 0;
-        cudaError_t e = cudaGetDevice(&dev);
+        static SmemLimit limit;
+        cudaError_t e = limit.ensure((const void*)router_logits_mma_kernel, (int)RM_SMEM);
         if (e != cudaSuccess) return e;
-        if (dev >= 64 || !attr_set[dev]) {
-            e = cudaFuncSetAttribute(router_logits_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)RM_SMEM);
-            if (e != cudaSuccess) return e;
-            if (dev < 64) attr_set[dev] = true;
-        }
         cfg.gridDim = dim3((unsigned)((E + RM_BM - 1) / RM_BM), (unsigned)((T + RM_BN - 1) / RM_BN));
         cfg.blockDim = dim3(RM_THREADS);
         cfg.dynamicSmemBytes = RM_SMEM;
