@@ -29,8 +29,9 @@
  *    ABI.  rfx_last_error() gives a thread-local message for the last failure.
  *  - "device" pointers are CUDA global-memory pointers of the current device;
  *    "host" pointers are CPU memory.  All buffers are owned by the caller; the
- *    library never allocates device memory (except rfx_layer_create, which
- *    allocates only a small host struct).
+ *    library never allocates device memory (moe_layer_create allocates only a
+ *    small host struct; moe_ffn_forward_static uses a workspace array compiled
+ *    into the library).
  *  - Device calls are asynchronous on `stream` (a cudaStream_t, NULL = legacy
  *    default stream).  The return code covers argument validation and launch
  *    errors.  Errors found on the device (expert id out of range, an
