@@ -68,6 +68,7 @@ _rms = _proto("moe_rms_norm_bf16", _i32, [_vp, _i32, _i32, _vp, _vp])
 _stack_ws = _proto("moe_stack_workspace_bytes", _sz, [_vp, _i32, _i32])
 _stack = _proto("moe_stack_forward", _i32, [_vp, _i32, _vp, _vp, _i32, _vp, _vp, _sz, _vp])
 _pf_ws_bytes = _proto("moe_prefill_workspace_bytes", _sz, [_vp, _i32])
+_debug_fault = _proto("rfx_debug_set_fault", _i32, [_i32, ctypes.c_longlong])
 _prefill = _proto("moe_ffn_prefill", _i32, [_vp, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp])
 
 
@@ -83,7 +84,7 @@ EXPORTED = ["rfx_last_error", "rfx_packed_bytes", "rfx_pack", "rfx_unpack", "rfx
             "rfx_ws_status", "moe_ffn_forward", "moe_ffn_forward_static", "moe_rms_norm_bf16",
             "moe_stack_workspace_bytes", "moe_stack_forward", "moe_prefill_workspace_bytes", "moe_ffn_prefill",
             "moe_prefill_view", "moe_router_logits", "moe_router_project_topk",
-            "moe_ffn_host_scratch_bytes", "moe_ffn_forward_host"]
+            "moe_ffn_host_scratch_bytes", "moe_ffn_forward_host", "rfx_debug_set_fault"]
 
 
 class RfxError(RuntimeError):
@@ -224,6 +225,12 @@ def moe_ffn_forward_static(handle: int, x, T: int, idx, w, y, stream=None):
     """moe_ffn_forward with the library's built-in 16 MiB workspace, for callers
     that cannot allocate device memory (see include/rfx.h)."""
     _check(_forward_static(handle, _ptr(x), T, _ptr(idx), _ptr(w), _ptr(y), _stream(stream)))
+
+
+def rfx_debug_set_fault(fault: int, wait_cycles: int = 0):
+    """Test hook of the device error path (rfx.h): plant a wait that cannot end
+    and shorten every bounded wait; fault=0, wait_cycles=0 restores normal use."""
+    _check(_debug_fault(fault, wait_cycles))
 
 
 def moe_rms_norm_bf16(y, x_next, stream=None):

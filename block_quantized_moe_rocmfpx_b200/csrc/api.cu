@@ -166,10 +166,36 @@ extern "C" size_t moe_ffn_workspace_bytes(const moe_layer* layer, int T) {
 }
 
 // Bytes at the start of a workspace that hold control words (they must be
-// zero before a call; the kernel returns them to zero when it finishes).
-size_t rfx_moe_ctrl_bytes(const moe_layer* layer) {
-    return layer ? rfx::moe_ws_layout(1, layer->d.k, layer->d.H, layer->d.I).h_off : 0;
+// zero before a call; the kernels return them to zero when they finish): the
+// decode control block for T <= 8, the prefill one above.
+size_t rfx_moe_ctrl_bytes(const moe_layer* layer, int T) {
+    if (!layer) return 0;
+    if (T > MOE_MAXT) return rfx::pf_ws_layout(T, layer->d.k, layer->d.E, layer->d.H, layer->d.I).cnt;
+    return (size_t)MOE_CTRL_WORDS * 4;
 }
+
+// Test hook for the device error path (rfx.h): a fault to inject and a wait
+// limit for later moe_ffn_forward / moe_ffn_prefill launches.
+namespace {
+std::atomic<int> g_fault{0};
+std::atomic<long long> g_wait{0};
+}  // namespace
+
+extern "C" int rfx_debug_set_fault(int fault, long long wait_cycles) {
+    if (fault < 0 || fault > 3 || wait_cycles < 0) return rfx_fail(RFX_EINVAL, "rfx_debug_set_fault: bad argument");
+    g_fault.store(fault);
+    g_wait.store(wait_cycles);
+    return RFX_OK;
+}
+
+namespace rfx {
+long long moe_default_wait_limit();
+int debug_fault() { return g_fault.load(); }
+long long debug_wait(long long dflt) {
+    const long long w = g_wait.load();
+    return w > 0 ? w : dflt;
+}
+}  // namespace rfx
 
 extern "C" int rfx_ws_init(void* ws, size_t ws_bytes, void* stream) {
     if (!ws) return rfx_fail(RFX_EINVAL, "rfx_ws_init: null workspace");
@@ -190,9 +216,8 @@ extern "C" int rfx_ws_status(void* ws, void* stream) {
         if (e != cudaSuccess) return cuda_fail("rfx_ws_status", e);
     }
     if (err & MOE_ERR_TIMEOUT) return rfx_fail(RFX_EDEVICE, "device: a bounded wait timed out");
-    if (err & (MOE_ERR_EXPERT | MOE_ERR_DUP))
-        return rfx_fail(RFX_EDEVICE, "device: expert id out of range or repeated within a token column");
-    if (err & MOE_ERR_RANGE) return rfx_fail(RFX_ERANGE, "device: SwiGLU output beyond the binary16 range");
+    if (err & MOE_ERR_EXPERT) return rfx_fail(RFX_EDEVICE, "device: expert id out of range");
+    if (err & MOE_ERR_RANGE) return rfx_fail(RFX_ERANGE, "device: a SwiGLU intermediate is not a finite fp32 value");
     return RFX_OK;
 }
 
@@ -205,8 +230,8 @@ int moe_prepare(const moe_layer* layer, const void* x, int T, const int32_t* idx
     const moe_layer_desc& d = layer->d;
     if (T < 1 || T > MOE_MAXT) return rfx_fail(RFX_EUNSUPPORTED, "moe_ffn_forward: 1 <= T <= 8 token columns");
     if (!x || !idx || !w || !y || !ws) return rfx_fail(RFX_EINVAL, "moe_ffn_forward: null pointer");
-    if (((uintptr_t)x & 3u) || ((uintptr_t)ws & 255u))
-        return rfx_fail(RFX_EINVAL, "moe_ffn_forward: x must be 4-byte and ws 256-byte aligned");
+    if (((uintptr_t)x & 15u) || ((uintptr_t)ws & 255u))
+        return rfx_fail(RFX_EINVAL, "moe_ffn_forward: x must be 16-byte and ws 256-byte aligned");
     const MoeWs L = moe_ws_layout(T, d.k, d.H, d.I);
     if (ws_bytes < L.total) return rfx_fail(RFX_EINVAL, "moe_ffn_forward: workspace smaller than moe_ffn_workspace_bytes");
     int sms = 0, smem_optin = 0;
@@ -223,23 +248,48 @@ int moe_prepare(const moe_layer* layer, const void* x, int T, const int32_t* idx
     p.x = (const uint16_t*)x; p.idx = idx; p.wts = w; p.y = y;
     uint8_t* wsb = (uint8_t*)ws;
     p.ctrl = (uint32_t*)(wsb + L.ctrl_off);
-    p.hbuf = (uint16_t*)(wsb + L.h_off);
+    p.hfrag = wsb + L.hf_off;
     p.dpart = (float*)(wsb + L.d_off);
+    p.hslot_bytes = (long long)L.hslot;
+    p.wait_limit = debug_wait(moe_default_wait_limit());
+    p.fault = debug_fault();
+    if (p.fault > 2) p.fault = 0;
     p.x_stride = d.H / 16 * 32 + 32;
-    // one region holds the staged x (gate/up phase: one copy per gate/up
-    // format in use, and its block sums), then two h buffers (down phase)
+    // Shared memory: the ring, the staged x (gate/up phase: one copy per
+    // gate/up format in use, and its block sums) and two h buffers (down
+    // phase), the reduction buffers.  An h buffer placed over the staged x is
+    // filled only once this CTA's gate/up stages are consumed, so the plans
+    // that keep the first (or both) buffers clear of x come first.
+    const int qc = moe_qclass(T);
+    auto r128 = [](size_t n) { return (n + 127) / 128 * 128; };
     const int nxc = (d.has_shared && d.f_sh_gate != d.f_gate) ? 2 : 1;
-    const size_t xb = (size_t)nxc * T * p.x_stride + (size_t)nxc * T * moe_sxs(d.H) * 4;
-    const size_t hb = 2 * (size_t)4 * T * (d.I + moe_sstr(d.I));
-    p.xh_bytes = (int)((std::max(xb, hb) + 127) / 128 * 128);
-    // deepest ring first (memory in flight), then as many reduction buffers as fit
+    const size_t xb = r128((size_t)nxc * T * p.x_stride + (size_t)nxc * T * moe_sxs(d.H) * 4);
+    const size_t hb = r128((size_t)moe_h_image_bytes(T, d.I));
+    p.x_bytes = (int)xb;
+    struct HPlan { size_t region, h0, h1; };
+    const HPlan plans[3] = {{xb + 2 * hb, xb, xb + hb},                                   // both clear of x
+                            {std::max(xb, hb) + hb, std::max(xb, hb), 0},                 // buffer 0 clear of x
+                            {std::max(xb, 2 * hb), 0, hb}};                               // both over x
+    const int order[4][2] = {{0, 4}, {1, 3}, {2, 3}, {-1, 2}};   // (plan, fewest stages); -1: any plan
     p.ns = 0;
-    p.nred = 0;
-    for (int ns = MOE_MAX_STAGES; ns >= 2 && !p.ns; --ns)
-        for (int nr = MOE_MAX_RED; nr >= 4; --nr)
-            if (moe_decode_smem_bytes(ns, nr, p.xh_bytes) <= (size_t)smem_optin) { p.ns = ns; p.nred = nr; break; }
+    for (int o = 0; o < 4 && !p.ns; ++o)
+        for (int pi = 0; pi < 3 && !p.ns; ++pi) {
+            if (order[o][0] >= 0 && order[o][0] != pi) continue;
+            for (int ns = MOE_MAX_STAGES; ns >= order[o][1] && !p.ns; --ns)
+                // a multiple of the 3 epilogue warps: they take units in turn, so
+                // every buffer stays with one warp and its phases are waited on in order
+                for (int nr = MOE_MAX_RED; nr >= 3; nr -= 3)
+                    if (moe_decode_smem_bytes(ns, nr, (int)plans[pi].region, qc) <= (size_t)smem_optin) {
+                        p.ns = ns;
+                        p.nred = nr;
+                        p.xh_bytes = (int)plans[pi].region;
+                        p.hoff0 = (int)plans[pi].h0;
+                        p.hoff1 = (int)plans[pi].h1;
+                        break;
+                    }
+        }
     if (!p.ns) return rfx_fail(RFX_EUNSUPPORTED, "moe_ffn_forward: shapes need more shared memory than the device has");
-    smem = moe_decode_smem_bytes(p.ns, p.nred, p.xh_bytes);
+    smem = moe_decode_smem_bytes(p.ns, p.nred, p.xh_bytes, qc);
     grid = sms;
     return RFX_OK;
 }
@@ -388,6 +438,8 @@ extern "C" int moe_ffn_prefill(const moe_layer* layer, const void* x, int T, con
     p.xp = (uint16_t*)(b + L.xp);
     p.hp = (uint16_t*)(b + L.hp);
     p.max_tiles = L.max_tiles;
+    p.wait_limit = rfx::debug_wait(rfx::pf_default_wait_limit());
+    p.fault = rfx::debug_fault() == 3 ? 3 : 0;
     cudaError_t e = rfx::pf_launch(p, sms, (cudaStream_t)stream);
     if (e == cudaErrorInvalidValue) return rfx_fail(RFX_ECUDA, "moe_ffn_prefill: tensor-map encoding failed");
     return e == cudaSuccess ? RFX_OK : cuda_fail("moe_ffn_prefill", e);

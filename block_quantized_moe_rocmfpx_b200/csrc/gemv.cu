@@ -169,15 +169,15 @@ __global__ void __launch_bounds__(GEMV_WARPS * 32) gemv_kernel(GemvParams p) {
                     uint32_t a[8];
                     float s0, s1;
                     partial_tile<FMT>(st, nt, lane, g, b, a, s0, s1);
-                    s0 *= 0x1.0p-24f; s1 *= 0x1.0p-24f;
 #pragma unroll
                     for (int nb = 0; nb < NB; ++nb) {
                         float cc[4];
                         mma_tile(cc, a, bs[nb].get(step0 + 2 * b), bs[nb].get(step0 + 2 * b + 1));
-                        acc[nb][0] = fmaf(s0, cc[0], acc[nb][0]);
-                        acc[nb][1] = fmaf(s0, cc[1], acc[nb][1]);
-                        acc[nb][2] = fmaf(s1, cc[2], acc[nb][2]);
-                        acc[nb][3] = fmaf(s1, cc[3], acc[nb][3]);
+                        // the exact level dot product in units of 2^-24 (scale untouched: it may be 2^-127)
+                        acc[nb][0] = fmaf(s0, cc[0] * 0x1.0p-24f, acc[nb][0]);
+                        acc[nb][1] = fmaf(s0, cc[1] * 0x1.0p-24f, acc[nb][1]);
+                        acc[nb][2] = fmaf(s1, cc[2] * 0x1.0p-24f, acc[nb][2]);
+                        acc[nb][3] = fmaf(s1, cc[3] * 0x1.0p-24f, acc[nb][3]);
                     }
                 }
             }

@@ -39,7 +39,7 @@
 namespace rfx {
 namespace {
 
-constexpr long long PF_WAIT = 1000000000LL;   // SM clocks before a wait gives up (about half a second)
+constexpr long long PF_WAIT = 1000000000LL;   // default SM clocks before a wait gives up (about half a second)
 
 constexpr int W_PROD = 0;     // TMA loads of the token rows (B operand); hands out the units
 constexpr int W_MMA = 1;      // tensor-memory allocation; first MMA issuer
@@ -90,20 +90,21 @@ struct PfShared {
     volatile int uq[UQ];
     uint32_t tmem;
     volatile int abort;
+    long long limit;   // SM clocks before a bounded wait gives up
 };
 static_assert(sizeof(PfShared) <= 1024, "barrier header must fit the first 1 KB");
 
 __device__ __forceinline__ void pf_set_error(uint32_t* ctrl, uint32_t bits) { atomicOr(ctrl + PF_CTRL_ERR, bits); }
 
 // Bounded wait; gives up when another role of the CTA has aborted or after
-// PF_WAIT clocks (then records a timeout and aborts the CTA).
+// sh.limit clocks (then records a timeout and aborts the CTA).
 __device__ __noinline__ bool pf_wait(PfShared& sh, uint32_t* ctrl, uint64_t* bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
         if (sh.abort) return false;
-        if (clock64() - t0 > PF_WAIT) {
+        if (clock64() - t0 > sh.limit) {
             sh.abort = 1;
             pf_set_error(ctrl, MOE_ERR_TIMEOUT);
             return false;
@@ -113,10 +114,10 @@ __device__ __noinline__ bool pf_wait(PfShared& sh, uint32_t* ctrl, uint64_t* bar
 
 // Bounded wait that does not give up on an abort: used before the CTA exits,
 // so that no copy or MMA of this CTA is still writing its memory.
-__device__ __noinline__ bool pf_wait_drain(uint32_t* ctrl, uint64_t* bar, uint32_t parity) {
+__device__ __noinline__ bool pf_wait_drain(uint32_t* ctrl, uint64_t* bar, uint32_t parity, long long limit) {
     const long long t0 = clock64();
     while (!mbar_try_wait_sleep(bar, parity, 20000u))
-        if (clock64() - t0 > PF_WAIT) {
+        if (clock64() - t0 > limit) {
             pf_set_error(ctrl, MOE_ERR_TIMEOUT);
             return false;
         }
@@ -497,8 +498,11 @@ __device__ bool pf_dq_chunk(const PfParams& p, PfShared& sh, const PfRings& R, c
 }
 
 // silu(g) * u with the hardware exponential and a fast reciprocal (relative
-// error a few fp32 ulps, far below the bf16 rounding that follows).
-__device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
+// error a few fp32 ulps, far below the bf16 rounding that follows); the far
+// negative tail separately, so that tiny h keep their value.
+__device__ __forceinline__ float silu_mul(float g, float u) {
+    return g >= -64.f ? __fdividef(g, 1.0f + __expf(-g)) * u : silu_mul_tail(g, u);
+}
 
 __device__ __forceinline__ uint16_t f32_to_bf16_rne(float v) {
     uint16_t r;
@@ -558,6 +562,7 @@ __global__ void __launch_bounds__(PfCfg<MODE>::THREADS, 1)
         }
         mbar_init(&sh.drain, 2);
         sh.abort = 0;
+        sh.limit = p.wait_limit;
         fence_barrier_init();
     }
     if (warp == W_MMA) {
@@ -599,8 +604,12 @@ __global__ void __launch_bounds__(PfCfg<MODE>::THREADS, 1)
                 return u < nunits ? u : -1;
             };
             int gstep = 0;
-            int u = grab();
-            bool ok = publish(0, u);
+            bool ok = true;
+            // tests of the error path only: wait for the release of a stage that
+            // nothing has loaded (it never comes; the wait times out)
+            if (MODE == 1 && p.fault == 3) ok = pf_wait(sh, p.ctrl, &sh.empty[0], 0u);
+            int u = ok ? grab() : -1;
+            ok = ok && publish(0, u);
             for (int i = 0; ok && u >= 0; ++i) {
                 const int un = grab();
                 if (!publish(i + 1, un)) break;
@@ -626,7 +635,7 @@ __global__ void __launch_bounds__(PfCfg<MODE>::THREADS, 1)
             // then the bounded wait gives up)
             for (int i = 1; i <= Cfg::NS && gstep - i >= 0; ++i) {
                 const int gi = gstep - i;
-                (void)pf_wait_drain(p.ctrl, &sh.full[gi % Cfg::NS], (uint32_t)(gi / Cfg::NS) & 1u);
+                (void)pf_wait_drain(p.ctrl, &sh.full[gi % Cfg::NS], (uint32_t)(gi / Cfg::NS) & 1u, sh.limit);
             }
         }
     } else if (warp == W_MMA || warp == W_MMA2) {
@@ -676,7 +685,7 @@ __global__ void __launch_bounds__(PfCfg<MODE>::THREADS, 1)
                 tc_commit(&sh.acc_full[b]);
             }
             tc_commit(&sh.drain);
-            (void)pf_wait_drain(p.ctrl, &sh.drain, 0);
+            (void)pf_wait_drain(p.ctrl, &sh.drain, 0, sh.limit);
         }
     } else if (warp < Cfg::W_EPI0) {
         const int d = warp - W_DQ0;
@@ -828,6 +837,8 @@ bool make_tmap(CUtensorMap* m, const void* base, long long rows, long long cols)
 }  // namespace
 
 size_t pf_gemm_smem_bytes(int mode) { return mode == 0 ? PfCfg<0>::SMEM : PfCfg<1>::SMEM; }
+
+long long pf_default_wait_limit() { return PF_WAIT; }
 
 cudaError_t pf_launch(const PfParams& p, int sms, cudaStream_t stream) {
     static SmemLimit limit[2];

@@ -50,6 +50,8 @@ struct PfParams {
     uint16_t* xp;           // bf16 [T*k][H] routed rows of x, grouped
     uint16_t* hp;           // bf16 [T*k + T][I] SwiGLU output rows (routed rows, then the shared expert's)
     int max_tiles;
+    long long wait_limit;   // SM clocks before a bounded wait gives up
+    int fault;              // tests of the error path only: 3 = the down GEMM waits for a stage nothing loads
 };
 
 struct PfWs {
@@ -80,6 +82,7 @@ inline PfWs pf_ws_layout(int T, int k, int E, int H, int I) {
 size_t pf_gemm_smem_bytes(int mode);
 // Launch the whole prefill step on `stream`: grouping, gather, gate/up GEMM
 // with SwiGLU, down GEMM with the weighted combine into y.  `sms` = SM count.
+long long pf_default_wait_limit();
 cudaError_t pf_launch(const PfParams& p, int sms, cudaStream_t stream);
 
 }  // namespace rfx

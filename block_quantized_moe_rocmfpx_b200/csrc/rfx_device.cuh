@@ -28,6 +28,14 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 
+// silu(g) * u for g < -64, where sigmoid(g) equals exp(g) to fp32 precision.
+// exp(g) is taken as exp(g + 64 ln 2) * 2^-64 so that the products stay in
+// fp32's normal range while h itself is still representable (a plain
+// g / (1 + exp(-g)) gives 0 below g = -88.7, where the true value is ~1e-37).
+__device__ __forceinline__ float silu_mul_tail(float g, float u) {
+    return (g * __expf(g + 44.3614195558365f) * u) * 0x1.0p-64f;
+}
+
 // Programmatic dependent launch: let the next kernel in the stream start its
 // prologue now, and wait until the previous kernel has finished and its
 // writes are visible (a no-op when the launch had no such dependency).
@@ -54,6 +62,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Non-blocking test of the phase with the given parity (try_wait may suspend
+// the thread for a while; test_wait never does).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
         : "r"(smem_u32(bar)), "r"(parity)

@@ -253,11 +253,13 @@ struct AccB {
     }
 };
 
-// One full down chunk (h used as it is; B operands hi/lo split fp16).
-// Sb[n][b] = block sum of h for the lane's real column of n-block n.
+// One full down chunk (B operands: hi/lo fp16 pairs of h * 2^n, n a
+// power-of-two exponent per column and 32-block).  Sb[n][b] = block sum of
+// the staged h for the lane's real column of n-block n; Hs[n][b] = 2^-n of
+// that column and block, folded into the weight scale of the tile (exact).
 template <int FMT, int NB, class SRC>
 __device__ __forceinline__ void chunkB_full(const uint8_t* st, int lane, int g, const SRC* bs, int step0,
-                                            const float (*Sb)[8], AccB<NB>& ab) {
+                                            const float (*Sb)[8], const float (*Hs)[8], AccB<NB>& ab) {
     FullChunk<FMT> f;
     f.load(st, lane, g);
 #pragma unroll
@@ -280,12 +282,13 @@ __device__ __forceinline__ void chunkB_full(const uint8_t* st, int lane, int g, 
         for (int n = 0; n < NB; ++n) {
             float c[4];
             mma_tile(c, a, bs[n].get(step0 + 2 * b), bs[n].get(step0 + 2 * b + 1));
-            ab.acc[cls][n][0] = fmaf(s0, c[0], ab.acc[cls][n][0]);
-            ab.acc[cls][n][1] = fmaf(s0, c[1], ab.acc[cls][n][1]);
-            ab.acc[cls][n][2] = fmaf(s1, c[2], ab.acc[cls][n][2]);
-            ab.acc[cls][n][3] = fmaf(s1, c[3], ab.acc[cls][n][3]);
-            ab.corr[n][0] = fmaf(s0, Sb[n][b], ab.corr[n][0]);
-            ab.corr[n][1] = fmaf(s1, Sb[n][b], ab.corr[n][1]);
+            const float s0n = s0 * Hs[n][b], s1n = s1 * Hs[n][b];
+            ab.acc[cls][n][0] = fmaf(s0n, c[0], ab.acc[cls][n][0]);
+            ab.acc[cls][n][1] = fmaf(s0n, c[1], ab.acc[cls][n][1]);
+            ab.acc[cls][n][2] = fmaf(s1n, c[2], ab.acc[cls][n][2]);
+            ab.acc[cls][n][3] = fmaf(s1n, c[3], ab.acc[cls][n][3]);
+            ab.corr[n][0] = fmaf(s0n, Sb[n][b], ab.corr[n][0]);
+            ab.corr[n][1] = fmaf(s1n, Sb[n][b], ab.corr[n][1]);
         }
     }
 }
@@ -333,6 +336,8 @@ __device__ __forceinline__ void partial_tile(const uint8_t* st, int nt, int lane
 
 // A partial chunk adds s * (exact level dot product) in units of 2^-24 so that
 // it shares the full chunks' accumulator (no offset correction: levels exact).
+// The 2^-24 goes on the dot product, not on the scale: an E8M0 scale of 2^-127
+// times 2^-24 would fall below fp32's smallest subnormal.
 template <int FMT, bool TWO, class SRC>
 __device__ __forceinline__ void chunkA_partial(const uint8_t* st0, const uint8_t* st1, int nt, int lane, int g,
                                                const SRC& bs, int step0, AccA& ag, AccA& au) {
@@ -342,33 +347,32 @@ __device__ __forceinline__ void chunkA_partial(const uint8_t* st0, const uint8_t
         float c[4], s0, s1;
         partial_tile<FMT>(st0, nt, lane, g, b, a, s0, s1);
         mma_tile(c, a, blo, bhi);
-        s0 *= 0x1.0p-24f; s1 *= 0x1.0p-24f;
-        ag.acc[0] = fmaf(s0, c[0], ag.acc[0]); ag.acc[1] = fmaf(s0, c[1], ag.acc[1]);
-        ag.acc[2] = fmaf(s1, c[2], ag.acc[2]); ag.acc[3] = fmaf(s1, c[3], ag.acc[3]);
+        ag.acc[0] = fmaf(s0, c[0] * 0x1.0p-24f, ag.acc[0]); ag.acc[1] = fmaf(s0, c[1] * 0x1.0p-24f, ag.acc[1]);
+        ag.acc[2] = fmaf(s1, c[2] * 0x1.0p-24f, ag.acc[2]); ag.acc[3] = fmaf(s1, c[3] * 0x1.0p-24f, ag.acc[3]);
         partial_tile<FMT>(st1, nt, lane, g, b, a, s0, s1);
         mma_tile(c, a, blo, bhi);
-        s0 *= 0x1.0p-24f; s1 *= 0x1.0p-24f;
-        au.acc[0] = fmaf(s0, c[0], au.acc[0]); au.acc[1] = fmaf(s0, c[1], au.acc[1]);
-        au.acc[2] = fmaf(s1, c[2], au.acc[2]); au.acc[3] = fmaf(s1, c[3], au.acc[3]);
+        au.acc[0] = fmaf(s0, c[0] * 0x1.0p-24f, au.acc[0]); au.acc[1] = fmaf(s0, c[1] * 0x1.0p-24f, au.acc[1]);
+        au.acc[2] = fmaf(s1, c[2] * 0x1.0p-24f, au.acc[2]); au.acc[3] = fmaf(s1, c[3] * 0x1.0p-24f, au.acc[3]);
     }
 }
 
 template <int FMT, int NB, class SRC>
 __device__ __forceinline__ void chunkB_partial(const uint8_t* st, int nt, int lane, int g, const SRC* bs, int step0,
-                                               AccB<NB>& ab) {
+                                               const float (*Hs)[8], AccB<NB>& ab) {
     for (int b = 0; b < nt; ++b) {
         uint32_t a[8];
         float s0, s1;
         partial_tile<FMT>(st, nt, lane, g, b, a, s0, s1);
-        s0 *= 0x1.0p-24f; s1 *= 0x1.0p-24f;   // class 0: scaled by 2^24 at the end
 #pragma unroll
         for (int n = 0; n < NB; ++n) {
             float c[4];
             mma_tile(c, a, bs[n].get(step0 + 2 * b), bs[n].get(step0 + 2 * b + 1));
-            ab.acc[0][n][0] = fmaf(s0, c[0], ab.acc[0][n][0]);
-            ab.acc[0][n][1] = fmaf(s0, c[1], ab.acc[0][n][1]);
-            ab.acc[0][n][2] = fmaf(s1, c[2], ab.acc[0][n][2]);
-            ab.acc[0][n][3] = fmaf(s1, c[3], ab.acc[0][n][3]);
+            const float s0n = s0 * Hs[n][b], s1n = s1 * Hs[n][b];
+            // class 0 is scaled by 2^24 at the end
+            ab.acc[0][n][0] = fmaf(s0n, c[0] * 0x1.0p-24f, ab.acc[0][n][0]);
+            ab.acc[0][n][1] = fmaf(s0n, c[1] * 0x1.0p-24f, ab.acc[0][n][1]);
+            ab.acc[0][n][2] = fmaf(s1n, c[2] * 0x1.0p-24f, ab.acc[0][n][2]);
+            ab.acc[0][n][3] = fmaf(s1n, c[3] * 0x1.0p-24f, ab.acc[0][n][3]);
         }
     }
 }

@@ -34,9 +34,9 @@
  *    into the library).
  *  - Device calls are asynchronous on `stream` (a cudaStream_t, NULL = legacy
  *    default stream).  The return code covers argument validation and launch
- *    errors.  Errors found on the device (expert id out of range, an
- *    intermediate that overflows binary16, a bounded wait that timed out) set
- *    a flag in the workspace that rfx_ws_status() reads after a sync.
+ *    errors.  Errors found on the device (expert id out of range, a SwiGLU
+ *    intermediate that is not a finite fp32 value, a bounded wait that timed
+ *    out) set a flag in the workspace that rfx_ws_status() reads after a sync.
  *
  * Packed weight format (this library's reading: the pages give only the block
  * size and the bytes per block).  W[n][k] = scale[n][k/32] * level(code[n][k]):
@@ -96,7 +96,7 @@ typedef enum {
     RFX_EUNSUPPORTED = -2,  /* valid but outside what this build supports (e.g. q > 8) */
     RFX_ECUDA = -3,         /* a CUDA runtime call or launch failed */
     RFX_EDEVICE = -4,       /* device-side check failed (bad expert id, wait timeout) */
-    RFX_ERANGE = -5         /* an intermediate exceeded the binary16 range (|h| > 65504) */
+    RFX_ERANGE = -5         /* a SwiGLU intermediate overflowed fp32 (inputs outside the fp32 range) */
 } rfx_status;
 
 typedef enum { RFX_FP2 = 2, RFX_FP3 = 3, RFX_FP4 = 4 } rfx_format;
@@ -223,8 +223,8 @@ int rfx_ws_init(void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Read and clear the device error flag of a workspace.  Synchronises stream.
- * Returns RFX_OK, RFX_EDEVICE (bad expert id / duplicate id in a column /
- * wait timeout) or RFX_ERANGE (|h| > 65504 met).
+ * Returns RFX_OK, RFX_EDEVICE (expert id out of range / a bounded wait timed
+ * out) or RFX_ERANGE (a SwiGLU value was not a finite fp32 number).
  */
 int rfx_ws_status(void* ws, void* stream);
 
@@ -235,17 +235,26 @@ int rfx_ws_status(void* ws, void* stream);
  * with e_tj = idx[t][j], silu(z) = z / (1 + e^-z).  The experts routed by any
  * column are grouped: each packed block of each union expert is read from HBM
  * and decoded once and applied to every column routed to that expert.
- * x: device bf16 bits [T][H].  idx: device int32 [T][k], distinct per row,
- * in [0, E).  w: device fp32 [T][k].  y: device fp32 [T][H].
+ * x: device bf16 bits [T][H], 16-byte aligned.  idx: device int32 [T][k] in [0, E); an id
+ * repeated within a row contributes once per entry (its expert output is
+ * computed once and weighted by each of its w), an id out of range sets the
+ * device error flag and its entry is skipped.  w: device fp32 [T][k].
+ * y: device fp32 [T][H].
+ * Numerics: every product level * scale * x is exact and accumulated in fp32;
+ * h = silu(g) * u is carried into the down projection as a binary16 hi/lo
+ * pair of h * 2^n, n a power-of-two scale per expert and column chosen from
+ * max |h|, so any h within the fp32 range is representable to about 2^-22
+ * relative.  Column t of a T-column call equals a 1-column call bit for bit.
  * Limits: 1 <= T <= 8 (decode / verify), H % 32 == 0, I % 32 == 0, k <= 8;
  * T == 0 is a no-op (so for every call below that takes T).
  * T > 8 runs moe_ffn_prefill instead (bf16 operands; its own limits and
  * workspace size).
  * One cooperative launch of one CTA per SM (all CTAs resident at once: the
- * gate/up, down and combine phases meet at two grid barriers whose counters
- * live in the workspace).  A workspace must not be used by two calls that
- * overlap on the GPU.  After a call that reported a device error through
- * rfx_ws_status, re-initialise the workspace with rfx_ws_init before reuse.
+ * down rows of an expert wait, through counters in the workspace, for its
+ * gate/up rows, and the combine waits at one grid barrier).  A workspace must
+ * not be used by two calls that overlap on the GPU.  After a call that
+ * reported a device error through rfx_ws_status, re-initialise the workspace
+ * with rfx_ws_init before reuse.
  */
 int moe_ffn_forward(const moe_layer* layer, const void* x, int T, const int32_t* idx, const float* w,
                     float* y, void* ws, size_t ws_bytes, void* stream);
@@ -322,12 +331,15 @@ int moe_prefill_view(const moe_layer* layer, int T, const void* ws, moe_prefill_
  * the library, not of the method.
  * The workspace is a 16 MiB array compiled into the library (held on every
  * GPU that loads it until the process exits); calls that would need more
- * (moe_ffn_workspace_bytes) return RFX_EUNSUPPORTED.  The first call on a
- * device looks up the array's device address; make it before any stream
- * capture on that device.  All calls on a device share the array: each clears
- * its control words with an asynchronous memset on `stream`, and calls that
- * overlap on the GPU race and give wrong results.  Device-side error flags are
- * not reported here (use moe_ffn_forward with your own workspace for that).
+ * (moe_ffn_workspace_bytes) return RFX_EUNSUPPORTED.  T > 8 takes the prefill
+ * path in the same array, within the same 16 MiB limit.  Each call looks up
+ * the array's device address on the current device; the first lookup on a
+ * device loads the library's device code there, so make the first call
+ * before any stream capture on that device.  All calls on a device share the
+ * array: each clears its control words with an asynchronous memset on
+ * `stream`, and calls that overlap on the GPU race and give wrong results.
+ * Device-side error flags are not reported here (use moe_ffn_forward with
+ * your own workspace for that).
  * x, idx, w, y, T and stream as in moe_ffn_forward.  Allocates nothing.
  */
 int moe_ffn_forward_static(const moe_layer* layer, const void* x, int T, const int32_t* idx, const float* w,
@@ -356,6 +368,21 @@ int moe_rms_norm_bf16(const float* y, int T, int H, void* x_next, void* stream);
 size_t moe_stack_workspace_bytes(const moe_layer* const* layers, int L, int T);
 int moe_stack_forward(const moe_layer* const* layers, int L, const float* logits, const void* x, int T, float* y,
                       void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Test hook for the device error path (no counterpart on the pages).  From the
+ * next call on, on every thread: moe_ffn_forward (T <= 8) and moe_ffn_prefill
+ * launches give up each bounded wait after wait_cycles SM clocks (0: the
+ * default, about 2 s for decode and 0.5 s for prefill), and `fault` plants a
+ * wait that cannot end: 1 = the decode kernel's final grid barrier waits for
+ * one CTA more than the grid has; 2 = no expert of a decode call ever becomes
+ * ready for its down projection; 3 = the prefill down GEMM waits for a unit
+ * that is never handed out.  The kernel then sets its timeout flag, drains its
+ * copies and returns: rfx_ws_status gives RFX_EDEVICE, and the workspace needs
+ * rfx_ws_init before its next use.  fault = 0 restores normal operation.  Not
+ * for production use.
+ */
+int rfx_debug_set_fault(int fault, long long wait_cycles);
 
 #ifdef __cplusplus
 }

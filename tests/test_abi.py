@@ -263,3 +263,11 @@ def test_host_call_scratch_bytes():
         assert rfx.moe_ffn_host_scratch_bytes(h, 0) == 0
     finally:
         rfx.moe_layer_destroy(h)
+
+
+def test_fault_hook_rejects_bad_arguments():
+    with pytest.raises(rfx.RfxError):
+        rfx.rfx_debug_set_fault(7, 0)
+    with pytest.raises(rfx.RfxError):
+        rfx.rfx_debug_set_fault(0, -1)
+    rfx.rfx_debug_set_fault(0, 0)

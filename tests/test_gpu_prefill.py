@@ -65,8 +65,10 @@ def check_grouping(idx, w, v, E):
 
 
 def bf16_half_step(v):
+    """Half the bf16 spacing at |v|: 2^(e-9) for v = m 2^e (8 significant
+    bits), and no less than 2^-134 (bf16 subnormals are spaced 2^-133)."""
     _, e = np.frexp(np.abs(v))
-    return np.ldexp(1.0, e - 9)
+    return np.ldexp(1.0, np.maximum(e - 9, -134))
 
 
 def exact_h(mats, x):

@@ -68,3 +68,26 @@ def test_static_workspace_rejects_layers_that_do_not_fit():
         assert "static" in rfx.rfx_last_error()
     finally:
         rfx.moe_layer_destroy(h)
+
+
+def test_static_workspace_prefill_path_matches_moe_ffn_prefill_twice():
+    """T > 8 takes the prefill path inside the same built-in array."""
+    lay = SynthLayer(79, 0, 512, 256, 8, 2)
+    T, k = 12, 2
+    ml = lay.moe_layer(max_T=T)
+    for call, tok0 in enumerate((0, 40)):
+        L = synth.logits(79, 0, tok0, T, lay.E, 0.0)
+        xb = synth.x_bf16(79, tok0, T, lay.H)
+        x = torch.from_numpy(xb).view(torch.bfloat16).to(DEV)
+        idx = torch.empty((T, k), dtype=torch.int32, device=DEV)
+        w = torch.empty((T, k), dtype=torch.float32, device=DEV)
+        rfx.moe_router_topk(torch.from_numpy(L).to(DEV), k, idx, w)
+        y_ref = torch.full((T, lay.H), float("nan"), dtype=torch.float32, device=DEV)
+        ml.prefill(x, idx, w, y_ref)
+        y_st = torch.full((T, lay.H), float("nan"), dtype=torch.float32, device=DEV)
+        rfx.moe_ffn_forward_static(ml.handle, x, T, idx, w, y_st)
+        torch.cuda.synchronize()
+        assert ml.prefill_status() == rfx.RFX_OK
+        # the same kernels; only the order of the prefill's fp32 atomic adds may differ
+        torch.testing.assert_close(y_st, y_ref, rtol=1e-6, atol=1e-6 * float(y_ref.abs().max()),
+                                   msg=f"static prefill path, call {call}")
