@@ -10,6 +10,14 @@ beside it.  Weights are synthetic (seeded) and stay resident in HBM; 8 copies
 of the layer are rotated so that every step reads its weights from DRAM
 (inputs larger than L2).
 
+Beside the headline the same JSON line carries (each skippable by a flag):
+the q = 2, 3, 5 and uniform-routing sweep; the layer as a ROCmFPX MIX (a
+format per expert chosen by routing heat) at q = 1 and 4; the standalone
+quantised GEMV in each format at q = 1 and 4; the router projection + top-k;
+the prefill grouped GEMM at T = 2048 and 8192; the 43-layer stack at q = 1
+and 4 (98.7 GB of distinct layers resident); and the oracle timed on the
+host cores on a bounded sample.
+
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 With N > 1 (torchrun) every rank runs an independent replica of the workload
@@ -36,10 +44,37 @@ ZIPF_S = 1.1
 NTOK = 1000
 COPIES = 8
 SEED = 0
-# DRAM bytes (read + write) of one q=1 launch of moe_decode_kernel from the ncu
-# capture summarised in profiles/moe_decode_q1_full_layer.md; set to None
-# whenever the kernel changes until it is captured again.
-TRAFFIC_Q1 = 67_844_608 + 2_448_384
+CSRC = os.path.join(ROOT, "block_quantized_moe_rocmfpx_b200", "csrc")
+KERNEL_SOURCES = {
+    "moe_decode": ("moe_decode.cu", "moe_decode.h", "rfx_tile.cuh", "rfx_device.cuh", "rfx_layout.h"),
+    "prefill": ("prefill.cu", "prefill.h", "tc.cuh", "rfx_tile.cuh", "rfx_device.cuh", "rfx_layout.h"),
+}
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch from
+# one ncu capture: (kernel, workload) -> (digest of the kernel's sources when
+# it was captured, bytes, algorithmic bytes of that launch).  Reported scaled
+# to the run's mean algorithmic bytes per launch (the traffic grows with the
+# union of experts), and only while the sources still have that digest; after
+# any change the key reads null until the kernel is captured again.
+TRAFFIC = {
+    ("moe_decode", "q1"): ("4c5460ebb606468b", 67_087_616 + 1_176_064, 66_872_368),
+    ("moe_decode", "q4"): ("4c5460ebb606468b", 112_305_408 + 3_629_568, 111_513_792),
+}
+
+
+def source_digest(kernel: str) -> str:
+    import hashlib
+    h = hashlib.sha1()
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(CSRC, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic(kernel: str, workload: str, algo_bytes: float):
+    ent = TRAFFIC.get((kernel, workload))
+    if not ent or ent[0] != source_digest(kernel):
+        return None
+    return ent[1] * algo_bytes / ent[2]
 
 
 def parse():
@@ -52,8 +87,6 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--copies", type=int, default=COPIES, help="rotating layer copies (>= 8 keeps steps L2-cold)")
     ap.add_argument("--only-q1", action="store_true", help="skip the q=4 verify measurement")
-    ap.add_argument("--stack", action="store_true",
-                    help="also time the 43-layer stack (98.7 GB of distinct layers resident, FFN only)")
     ap.add_argument("--stack-only", action="store_true", help="time only the 43-layer stack")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill grouped-GEMM measurement")
     ap.add_argument("--prefill-only", action="store_true", help="time only the prefill (T = 2048 and 8192)")
@@ -61,6 +94,9 @@ def parse():
     ap.add_argument("--no-router-proj", action="store_true", help="skip the router projection measurement")
     ap.add_argument("--no-sweep", action="store_true", help="skip the q = 2, 3, 5 and uniform-routing decode sweep")
     ap.add_argument("--router-proj-only", action="store_true", help="time only the router projection + top-k")
+    ap.add_argument("--no-stack", action="store_true", help="skip the 43-layer stack measurement")
+    ap.add_argument("--no-mix", action="store_true", help="skip the ROCmFPX MIX (format per expert) measurement")
+    ap.add_argument("--no-gemv", action="store_true", help="skip the standalone quantised GEMV measurement")
     return ap.parse_args()
 
 
@@ -221,13 +257,13 @@ def run_reference(args, rank, world):
 class Workload:
     """C rotating copies of one synthetic full-size layer plus seeded inputs."""
 
-    def __init__(self, q: int, ntok: int, dev, copies: int = COPIES, zipf_s: float = ZIPF_S):
+    def __init__(self, q: int, ntok: int, dev, copies: int = COPIES, zipf_s: float = ZIPF_S, mix=None):
         import torch
         import numpy as np
         import synth
         from synth.layers import SynthLayer
         self.q, self.dev = q, dev
-        base = SynthLayer(SEED, 0, H, I, E, K_TOP, device=dev)
+        base = SynthLayer(SEED, 0, H, I, E, K_TOP, device=dev, mix=mix)
         self.base = base
         self.layers = [base.moe_layer(max_T=q)]
         self._keep = [base]
@@ -235,11 +271,8 @@ class Workload:
         for c in range(1, copies):
             bufs = [b.clone() for b in base.bufs]
             sh = [b.clone() for b in base.shared]
-            import block_quantized_moe_rocmfpx_b200 as rfx
-            ml = rfx.MoeLayer(H, I, E, K_TOP, base.fmts, *bufs, base.strides, shared=sh,
-                              shared_fmts=base.shared_fmts, max_T=q)
             self._keep.append((bufs, sh))
-            self.layers.append(ml)
+            self.layers.append(base.moe_layer(max_T=q, bufs=bufs, shared=sh))
         torch.cuda.synchronize()
         self.ntok = ntok
         nb = ntok * q
@@ -277,8 +310,10 @@ STACK_LAYERS = 43
 
 def measure_stack(qs, steps: int, warmup: int, dev):
     """The 43-layer stack: distinct seeded full-size layers resident in HBM,
-    each token step one moe_stack_forward call (router, MoE FFN and the
-    unit-RMS bf16 chaining per layer), captured in one CUDA graph."""
+    each token step one moe_stack_forward call (one router launch for all
+    layers, then one MoE FFN kernel per layer, each next layer applying the
+    unit-RMS bf16 chaining while it stages its input), captured in one CUDA
+    graph."""
     import time
     import numpy as np
     import torch
@@ -322,18 +357,17 @@ def measure_stack(qs, steps: int, warmup: int, dev):
             ms = time_graph(g, stream)
             del g, gw
         st = rfx_status_of(ws)
+        peak, _ = peaks()
+        gbs = per_step * steps / (ms / 1e3) / 1e9
         out[f"q{q}"] = {"value": q * steps / (ms / 1e3), "unit": "tokens/s", "ms_per_token_step": ms / steps,
-                        "achieved_gbs": per_step * steps / (ms / 1e3) / 1e9, "bytes_per_step": per_step,
+                        "us_per_layer": ms / steps / STACK_LAYERS * 1e3, "achieved_gbs": gbs, "frac": gbs / peak,
+                        "bytes_per_step": per_step, "launches_per_step": 1 + STACK_LAYERS, "steps": steps,
                         "device_status": st}
         del mls
     return out
 
 
 PREFILL_TS = (2048, 8192)
-# DRAM bytes (read + write) of the two prefill GEMM kernels for one T=2048 step,
-# from the ncu capture summarised in profiles/prefill_grouped_gemm_t2048.md; set
-# to None whenever those kernels change until they are captured again.
-PREFILL_TRAFFIC = {2048: 755_878_656 + 41_874_944 + 526_722_560 + 6_292_992}
 PREFILL_BATCHES = 2
 
 
@@ -392,7 +426,7 @@ def measure_prefill(T: int, steps: int, warmup: int, dev, layer=None):
             "roofline": {"bound": "tensor" if flops / (peak_tf * 1e12) >= per_step_bytes / (peak_gbs * 1e9)
                          else "hbm", "peak_tflops": peak_tf, "peak_gbs": peak_gbs, "t_min_ms": t_min * 1e3,
                          "frac": t_min / t_step, "peak_kind": "bf16_tflops_sustained of measured",
-                         "traffic": PREFILL_TRAFFIC.get(T)},
+                         "traffic": traffic("prefill", f"T{T}", per_step_bytes)},
             "device_status": st, "steps": steps}
 
 
@@ -441,6 +475,49 @@ def measure_router_proj(T: int, steps: int, warmup: int, dev):
             "launches_per_call": 2, "steps": steps}
 
 
+GEMV_N, GEMV_K = 131072, 4096   # one matrix larger than L2 in every format (168 to 285 MB packed)
+
+
+def measure_gemv(fmt: int, q: int, steps: int, warmup: int, dev):
+    """Standalone quantised GEMV (rfx_gemv_q): y[q][N] = W x for a packed
+    N x K matrix in one format, q bf16 columns, captured in a graph.  W is an
+    8192-row seeded slice packed once and repeated (the packed layout is
+    row-group after row-group), larger than L2 as a whole.  Roofline (HBM):
+    packed W + x read, y written."""
+    import torch
+    import synth
+    import block_quantized_moe_rocmfpx_b200 as rfx
+    N, K, R = GEMV_N, GEMV_K, 8192
+    spec = synth.MatrixSpec(SEED, 0, 0, 0, fmt, R, K)
+    sl = torch.from_numpy(rfx.rfx_pack(fmt, spec.codes(), spec.scales())).to(dev)
+    W = torch.empty(sl.numel() * (N // R), dtype=torch.uint8, device=dev)
+    for i in range(N // R):
+        W[i * sl.numel():(i + 1) * sl.numel()].copy_(sl)
+    x = torch.from_numpy(synth.x_bf16(SEED, 400000, q, K)).view(torch.bfloat16).to(dev)
+    y = torch.empty((q, N), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(t):
+        rfx.rfx_gemv_q(fmt, W, N, K, x, y, stream)
+
+    with torch.cuda.stream(stream):
+        for t in range(3):
+            step(t)
+        torch.cuda.synchronize()
+        gw = graph_of(step, max(3, warmup), stream)
+        g = graph_of(step, steps, stream)
+        gw.replay()
+        torch.cuda.synchronize()
+        ms = time_graph(g, stream)
+        del g, gw
+    us = ms * 1e3 / steps
+    nbytes = rfx.rfx_packed_bytes(fmt, N, K) + q * K * 2 + q * N * 4
+    peak, peak_kind = peaks()
+    gbs = nbytes / (us * 1e-6) / 1e9
+    return {"fmt": fmt, "q": q, "N": N, "K": K, "us_per_call": us, "bytes_per_call": nbytes, "achieved_gbs": gbs,
+            "frac": gbs / peak, "peak_kind": peak_kind, "steps": steps}
+
+
 def peaks_tensor() -> float:
     """Measured sustained dense bf16 TFLOP/s (a kernel timed inside a long step)."""
     try:
@@ -478,10 +555,10 @@ def time_graph(g, stream):
 
 
 def measure(q: int, steps: int, warmup: int, dev, rank, world, want_clocks: bool, want_e2e: bool, copies: int,
-            zipf_s: float = ZIPF_S):
+            zipf_s: float = ZIPF_S, mix=None):
     import torch
     import torch.distributed as dist
-    wl = Workload(q, NTOK, dev, copies, zipf_s)
+    wl = Workload(q, NTOK, dev, copies, zipf_s, mix)
     stream = torch.cuda.Stream(device=dev)
     with torch.cuda.stream(stream):
         for t in range(3):            # eager warm-up (kernel attributes, lazy loading)
@@ -584,8 +661,6 @@ def main():
     if args.stack_only:
         st = measure_stack((1, 4), min(args.steps, 200), max(3, args.warmup), dev)
         peak, peak_kind = peaks()
-        for q in (1, 4):
-            st[f"q{q}"]["frac"] = st[f"q{q}"]["achieved_gbs"] / peak
         if rank == 0:
             print(json.dumps({"metric": "43-layer MoE-FFN stack decode tokens/s (FFN only)", "stack": st,
                               "peak_gbs": peak, "peak_kind": peak_kind}), flush=True)
@@ -631,12 +706,40 @@ def main():
                           "kernel_us": ms_f * 1e3 / n, "tokens_per_s_step": world * q * n / (reduce_max(r["ms"]) / 1e3),
                           "achieved_gbs": gbs, "frac": gbs / peak_s, "union_experts": r["union"],
                           "algo_bytes_per_launch": r["bytes"] / n, "device_status": r["status"]})
+    mix = None
+    if not args.no_mix:
+        # ROCmFPX MIX: the same layer with a format per expert chosen by routing heat
+        from synth.layers import heat_mix
+        peak_s, _ = peaks()
+        hm = heat_mix(SEED, 0, E, ZIPF_S)
+        mix = {"assignment": "hottest 1/8 of experts FP4/FP4, next 3/8 FP3/FP3, rest FP2/FP3 (gate-up/down); "
+                             "shared FP4", "experts_per_format": {f"fp{f}": sum(1 for m in hm if m[0] == f)
+                                                                 for f in (2, 3, 4)}}
+        for q in (1, 4):
+            n = min(args.steps, 200)
+            r = measure(q, n, max(3, args.warmup), dev, rank, world, False, False, args.copies, ZIPF_S, hm)
+            ms_f = reduce_max(r["ms_ffn"])
+            gbs = r["bytes"] / (ms_f / 1e3) / 1e9
+            mix[f"q{q}"] = {"tokens_per_s_step": world * q * n / (reduce_max(r["ms"]) / 1e3),
+                            "kernel_us": ms_f * 1e3 / n, "achieved_gbs": gbs, "frac": gbs / peak_s,
+                            "algo_bytes_per_launch": r["bytes"] / n, "bytes_per_token": r["bytes"] / n / q,
+                            "union_experts": r["union"], "steps": n, "device_status": r["status"]}
+    gemv = None
+    if not args.no_gemv:
+        gemv = [measure_gemv(f, q, min(args.steps, 200), max(3, args.warmup), dev) for f in (2, 3, 4) for q in (1, 4)]
     rp = None
     if not args.no_router_proj:
         rp = [measure_router_proj(T, min(args.steps, 400), max(3, args.warmup), dev) for T in ROUTER_PROJ_TS]
     pf = None
     if not args.no_prefill:
         pf = [measure_prefill(T, args.prefill_steps, max(3, args.warmup), dev) for T in PREFILL_TS]
+    stack = None
+    if not args.no_stack:
+        import gc
+        import torch
+        gc.collect()
+        torch.cuda.empty_cache()
+        stack = measure_stack((1, 4), min(args.steps, 100), max(3, args.warmup), dev)
     if world > 1:
         dist.barrier()
     if rank == 0:
@@ -656,9 +759,13 @@ def main():
                        "l2": f"inputs larger than L2: {args.copies} rotating copies of the layer",
                        "graph": "CUDA graph of all timed steps"},
             "roofline": {"bound": "hbm", "achieved": gbs1, "peak": peak, "unit": "GB/s", "frac": gbs1 / peak,
-                         "traffic": TRAFFIC_Q1, "kernel": "moe_decode_kernel", "peak_kind": peak_kind,
-                         "algo_bytes_per_launch": r1["bytes"] / args.steps,
-                         "kernel_us": r1["ms_ffn"] * 1e3 / args.steps},
+                         "traffic": traffic("moe_decode", "q1", r1["bytes"] / args.steps),
+                         "kernel": "moe_decode_kernel",
+                         "peak_kind": peak_kind, "algo_bytes_per_launch": r1["bytes"] / args.steps,
+                         "kernel_us": r1["ms_ffn"] * 1e3 / args.steps,
+                         "q4": {"achieved": gbs4, "frac": gbs4 / peak, "kernel_us": r4["ms_ffn"] * 1e3 / args.steps,
+                                "algo_bytes_per_launch": r4["bytes"] / args.steps,
+                                "traffic": traffic("moe_decode", "q4", r4["bytes"] / args.steps)}},
             "q4": {"value": world * 4 * args.steps / (ms4 / 1e3), "unit": "tokens/s", "ms_per_step": ms4 / args.steps,
                    "union_experts": r4["union"],
                    "achieved_gbs": gbs4, "frac": gbs4 / peak, "kernel_us": r4["ms_ffn"] * 1e3 / args.steps,
@@ -671,6 +778,9 @@ def main():
             "prefill": pf,
             "router_projection": rp,
             "q_sweep": sweep,
+            "mix": mix,
+            "gemv": gemv,
+            "stack": stack,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

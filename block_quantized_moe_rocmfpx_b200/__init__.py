@@ -38,6 +38,11 @@ class moe_layer_desc(ctypes.Structure):
                 ("sh_gate", _vp), ("sh_up", _vp), ("sh_down", _vp)]
 
 
+class moe_expert_mix(ctypes.Structure):
+    _fields_ = [("f_gate_up", _i32), ("f_down", _i32),
+                ("off_gate", ctypes.c_uint64), ("off_up", ctypes.c_uint64), ("off_down", ctypes.c_uint64)]
+
+
 def _proto(name, res, args):
     f = getattr(_lib, name)
     f.restype = res
@@ -56,6 +61,8 @@ _router_proj_topk = _proto("moe_router_project_topk", _i32,
                            [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp])
 _gemv = _proto("rfx_gemv_q", _i32, [_i32, _vp, _i64, _i64, _vp, _i32, _i32, _vp, _vp])
 _layer_create = _proto("moe_layer_create", _i32, [ctypes.POINTER(moe_layer_desc), ctypes.POINTER(_vp)])
+_layer_create_mix = _proto("moe_layer_create_mix", _i32,
+                           [ctypes.POINTER(moe_layer_desc), ctypes.POINTER(moe_expert_mix), ctypes.POINTER(_vp)])
 _layer_destroy = _proto("moe_layer_destroy", None, [_vp])
 _ws_bytes = _proto("moe_ffn_workspace_bytes", _sz, [_vp, _i32])
 _ws_init = _proto("rfx_ws_init", _i32, [_vp, _sz, _vp])
@@ -80,7 +87,7 @@ class moe_prefill_ws_view(ctypes.Structure):
 _pf_view = _proto("moe_prefill_view", _i32, [_vp, _i32, _vp, ctypes.POINTER(moe_prefill_ws_view)])
 
 EXPORTED = ["rfx_last_error", "rfx_packed_bytes", "rfx_pack", "rfx_unpack", "rfx_pack_device", "moe_router_topk",
-            "rfx_gemv_q", "moe_layer_create", "moe_layer_destroy", "moe_ffn_workspace_bytes", "rfx_ws_init",
+            "rfx_gemv_q", "moe_layer_create", "moe_layer_create_mix", "moe_layer_destroy", "moe_ffn_workspace_bytes", "rfx_ws_init",
             "rfx_ws_status", "moe_ffn_forward", "moe_ffn_forward_static", "moe_rms_norm_bf16",
             "moe_stack_workspace_bytes", "moe_stack_forward", "moe_prefill_workspace_bytes", "moe_ffn_prefill",
             "moe_prefill_view", "moe_router_logits", "moe_router_project_topk",
@@ -188,6 +195,14 @@ def moe_layer_create(desc: moe_layer_desc) -> int:
     return h.value
 
 
+def moe_layer_create_mix(desc: moe_layer_desc, mix) -> int:
+    """mix: E tuples (f_gate_up, f_down, off_gate, off_up, off_down)."""
+    arr = (moe_expert_mix * len(mix))(*[moe_expert_mix(*m) for m in mix])
+    h = _vp()
+    _check(_layer_create_mix(ctypes.byref(desc), arr, ctypes.byref(h)))
+    return h.value
+
+
 def moe_layer_destroy(handle: int):
     _layer_destroy(handle)
 
@@ -290,11 +305,13 @@ class MoeLayer:
     """One MoE layer over caller-owned packed device buffers.
 
     ``gate``/``up``/``down`` are uint8 device tensors holding E packed experts
-    at a fixed stride; ``shared`` is (gate, up, down) or None.  Creates the
+    at a fixed stride (or, with ``mix``, at the table's offsets in the table's
+    formats); ``shared`` is (gate, up, down) or None.  Creates the
     host handle and a zeroed workspace for up to ``max_T`` token columns.
     """
 
-    def __init__(self, H, I, E, k, fmts, gate, up, down, strides, shared=None, shared_fmts=(4, 4, 4), max_T=MAX_T):
+    def __init__(self, H, I, E, k, fmts, gate, up, down, strides, shared=None, shared_fmts=(4, 4, 4), max_T=MAX_T,
+                 mix=None):
         import torch
         self.H, self.I, self.E, self.k = H, I, E, k
         self._keep = [gate, up, down] + (list(shared) if shared else [])
@@ -308,7 +325,8 @@ class MoeLayer:
             d.f_sh_gate, d.f_sh_up, d.f_sh_down = shared_fmts
             d.sh_gate, d.sh_up, d.sh_down = (_ptr(s) for s in shared)
         self.desc = d
-        self.handle = moe_layer_create(d)
+        # mix: ROCmFPX MIX table, E tuples (f_gate_up, f_down, off_gate, off_up, off_down)
+        self.handle = moe_layer_create(d) if mix is None else moe_layer_create_mix(d, mix)
         self.max_T = max_T
         nbytes = moe_ffn_workspace_bytes(self.handle, max_T)
         self.ws = torch.empty(nbytes, dtype=torch.uint8, device=gate.device)

@@ -1,5 +1,6 @@
 // api.cu -- C ABI entry points (include/rfx.h): argument checks, workspace
-// layout and kernel launches.  No entry point allocates device memory.
+// layout and kernel launches.  No entry point allocates device memory except
+// moe_layer_create_mix (its per-expert table, made once per layer).
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -7,6 +8,7 @@
 #include <cstring>
 #include <new>
 #include <string>
+#include <vector>
 
 #include "../../include/rfx.h"
 #include "gemv.h"
@@ -19,6 +21,8 @@ int rfx_fail(int code, const std::string& msg);  // rfx_pack.cpp
 
 struct moe_layer {
     moe_layer_desc d;
+    rfx::MoeMixEntry* mix_dev = nullptr;   // ROCmFPX MIX: device table [E], else null
+    int mix_count[5] = {0, 0, 0, 0, 0};    // routed experts per gate/up format (MIX)
 };
 
 namespace {
@@ -155,7 +159,58 @@ extern "C" int moe_layer_create(const moe_layer_desc* d, moe_layer** out) {
     return RFX_OK;
 }
 
-extern "C" void moe_layer_destroy(moe_layer* layer) { delete layer; }
+extern "C" int moe_layer_create_mix(const moe_layer_desc* d, const moe_expert_mix* mix, moe_layer** out) {
+    if (!d || !mix || !out) return rfx_fail(RFX_EINVAL, "moe_layer_create_mix: null pointer");
+    *out = nullptr;
+    // the descriptor's own checks, with routed formats and strides that always pass
+    moe_layer_desc u = *d;
+    u.f_gate = u.f_up = u.f_down = RFX_FP4;
+    u.stride_gate = u.stride_up = (rfx_packed_bytes(RFX_FP4, d->I, d->H) + 15) / 16 * 16;   // FP4 packs largest
+    u.stride_down = (rfx_packed_bytes(RFX_FP4, d->H, d->I) + 15) / 16 * 16;
+    moe_layer* L = nullptr;
+    int rc = moe_layer_create(&u, &L);
+    if (rc != RFX_OK) return rc;
+    std::vector<rfx::MoeMixEntry> tab((size_t)d->E);
+    for (int e = 0; e < d->E; ++e) {
+        const moe_expert_mix& m = mix[e];
+        if (!fmt_ok(m.f_gate_up) || !fmt_ok(m.f_down)) {
+            moe_layer_destroy(L);
+            return rfx_fail(RFX_EINVAL, "moe_layer_create_mix: bad format in entry " + std::to_string(e));
+        }
+        if (m.off_gate % 16 || m.off_up % 16 || m.off_down % 16) {
+            moe_layer_destroy(L);
+            return rfx_fail(RFX_EINVAL, "moe_layer_create_mix: offsets must be multiples of 16 (entry " +
+                                            std::to_string(e) + ")");
+        }
+        tab[e] = rfx::MoeMixEntry{(long long)m.off_gate, (long long)m.off_up, (long long)m.off_down, (int)m.f_gate_up,
+                                  (int)m.f_down};
+        ++L->mix_count[m.f_gate_up];
+    }
+    // the routed formats the descriptor reports: the most common ones
+    int fa = 2, fb = 2, cb[5] = {0, 0, 0, 0, 0};
+    for (int f = 2; f <= 4; ++f)
+        if (L->mix_count[f] > L->mix_count[fa]) fa = f;
+    for (int e = 0; e < d->E; ++e) ++cb[mix[e].f_down];
+    for (int f = 2; f <= 4; ++f)
+        if (cb[f] > cb[fb]) fb = f;
+    L->d = *d;
+    L->d.f_gate = L->d.f_up = (rfx_format)fa;
+    L->d.f_down = (rfx_format)fb;
+    L->d.stride_gate = L->d.stride_up = L->d.stride_down = 0;
+    cudaError_t e = cudaMalloc(&L->mix_dev, tab.size() * sizeof(rfx::MoeMixEntry));
+    if (e == cudaSuccess) e = cudaMemcpy(L->mix_dev, tab.data(), tab.size() * sizeof(rfx::MoeMixEntry), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) {
+        moe_layer_destroy(L);
+        return cuda_fail("moe_layer_create_mix", e);
+    }
+    *out = L;
+    return RFX_OK;
+}
+
+extern "C" void moe_layer_destroy(moe_layer* layer) {
+    if (layer && layer->mix_dev) cudaFree(layer->mix_dev);
+    delete layer;
+}
 
 extern "C" size_t moe_prefill_workspace_bytes(const moe_layer* layer, int T);
 
@@ -224,6 +279,40 @@ extern "C" int rfx_ws_status(void* ws, void* stream) {
 namespace rfx {
 
 // Fill launch parameters for T columns; returns RFX_OK or an error.
+// The staged x copies of the decode kernel (one per gate/up format that gets
+// its own, at most two): the most common routed format first, then the shared
+// expert's, else the next most common routed one.  A slot of any other format
+// reads copy 0 and corrects its scales.
+void x_copies(const moe_layer* layer, int& nxc, int xf[2], int& other) {
+    const moe_layer_desc& d = layer->d;
+    int cnt[5] = {0, 0, 0, 0, 0};
+    if (layer->mix_dev)
+        for (int f = 2; f <= 4; ++f) cnt[f] = layer->mix_count[f];
+    else
+        cnt[d.f_gate] = d.E;
+    int f0 = d.f_gate;
+    for (int f = 2; f <= 4; ++f)
+        if (cnt[f] > cnt[f0]) f0 = f;
+    xf[0] = f0;
+    xf[1] = f0;
+    nxc = 1;
+    if (d.has_shared && d.f_sh_gate != f0) {
+        xf[1] = d.f_sh_gate;
+        nxc = 2;
+    } else {
+        int f1 = 0;
+        for (int f = 2; f <= 4; ++f)
+            if (f != f0 && cnt[f] > 0 && (f1 == 0 || cnt[f] > cnt[f1])) f1 = f;
+        if (f1) {
+            xf[1] = f1;
+            nxc = 2;
+        }
+    }
+    other = 0;
+    for (int f = 2; f <= 4; ++f)
+        if (cnt[f] > 0 && f != xf[0] && f != xf[1]) other = 1;
+}
+
 int moe_prepare(const moe_layer* layer, const void* x, int T, const int32_t* idx, const float* w, float* y, void* ws,
                 size_t ws_bytes, MoeParams& p, int& grid, size_t& smem) {
     if (!layer) return rfx_fail(RFX_EINVAL, "moe_ffn_forward: null layer");
@@ -243,9 +332,11 @@ int moe_prepare(const moe_layer* layer, const void* x, int T, const int32_t* idx
     p.fsB = d.has_shared ? d.f_sh_down : 2;
     p.gate = (const uint8_t*)d.gate; p.up = (const uint8_t*)d.up; p.down = (const uint8_t*)d.down;
     p.sg = (long long)d.stride_gate; p.su = (long long)d.stride_up; p.sd = (long long)d.stride_down;
+    p.mix = layer->mix_dev;
+    x_copies(layer, p.nxc, p.xf, p.other);
     p.has_shared = d.has_shared ? 1 : 0;
     p.shg = (const uint8_t*)d.sh_gate; p.shu = (const uint8_t*)d.sh_up; p.shd = (const uint8_t*)d.sh_down;
-    p.x = (const uint16_t*)x; p.idx = idx; p.wts = w; p.y = y;
+    p.x = (const uint16_t*)x; p.xc = nullptr; p.idx = idx; p.wts = w; p.y = y;
     uint8_t* wsb = (uint8_t*)ws;
     p.ctrl = (uint32_t*)(wsb + L.ctrl_off);
     p.hfrag = wsb + L.hf_off;
@@ -262,7 +353,7 @@ int moe_prepare(const moe_layer* layer, const void* x, int T, const int32_t* idx
     // that keep the first (or both) buffers clear of x come first.
     const int qc = moe_qclass(T);
     auto r128 = [](size_t n) { return (n + 127) / 128 * 128; };
-    const int nxc = (d.has_shared && d.f_sh_gate != d.f_gate) ? 2 : 1;
+    const int nxc = p.nxc;
     const size_t xb = r128((size_t)nxc * T * p.x_stride + (size_t)nxc * T * moe_sxs(d.H) * 4);
     const size_t hb = r128((size_t)moe_h_image_bytes(T, d.I));
     p.x_bytes = (int)xb;
@@ -419,6 +510,7 @@ extern "C" int moe_ffn_prefill(const moe_layer* layer, const void* x, int T, con
     const moe_layer_desc& d = layer->d;
     rfx::PfParams p{};
     p.H = d.H; p.I = d.I; p.E = d.E; p.k = d.k; p.T = T;
+    p.mix = layer->mix_dev;
     p.fA = d.f_gate; p.fB = d.f_down;
     p.fsA = d.has_shared ? d.f_sh_gate : 2;
     p.fsB = d.has_shared ? d.f_sh_down : 2;
@@ -472,8 +564,10 @@ extern "C" int moe_rms_norm_bf16(const float* y, int T, int H, void* x_next, voi
 
 namespace {
 
+// Stack workspace: one decode workspace, the routing of every layer, two
+// fp32 activation buffers (layer l writes one while it reads the other).
 struct StackWs {
-    size_t ffn, idx, w, ybuf, xbuf, total;
+    size_t ffn, idx, w, ybuf[2], total;
 };
 
 StackWs stack_ws_layout(const moe_layer* const* layers, int L, int T) {
@@ -484,10 +578,10 @@ StackWs stack_ws_layout(const moe_layer* const* layers, int L, int T) {
     auto up = [](size_t n) { return (n + 255) / 256 * 256; };
     W.ffn = 0;
     W.idx = up(ffn);
-    W.w = W.idx + up((size_t)T * d.k * 4);
-    W.ybuf = W.w + up((size_t)T * d.k * 4);
-    W.xbuf = W.ybuf + up((size_t)T * d.H * 4);
-    W.total = W.xbuf + 2 * up((size_t)T * d.H * 2);
+    W.w = W.idx + up((size_t)L * T * d.k * 4);
+    W.ybuf[0] = W.w + up((size_t)L * T * d.k * 4);
+    W.ybuf[1] = W.ybuf[0] + up((size_t)T * d.H * 4);
+    W.total = W.ybuf[1] + up((size_t)T * d.H * 4);
     return W;
 }
 
@@ -524,20 +618,27 @@ extern "C" int moe_stack_forward(const moe_layer* const* layers, int L, const fl
     uint8_t* b = (uint8_t*)ws;
     int32_t* idx = (int32_t*)(b + W.idx);
     float* wts = (float*)(b + W.w);
-    float* ybuf = (float*)(b + W.ybuf);
-    uint16_t* xb[2] = {(uint16_t*)(b + W.xbuf), (uint16_t*)(b + W.xbuf + (W.total - W.xbuf) / 2)};
-    const void* xin = x;
+    // the routing of all layers in one launch (it depends on the logits alone)
+    rc = moe_router_topk(logits, L * T, d.E, d.k, idx, wts, stream);
+    if (rc != RFX_OK) return rc;
+    const float* prev = nullptr;
     for (int l = 0; l < L; ++l) {
-        rc = moe_router_topk(logits + (size_t)l * T * d.E, T, d.E, d.k, idx, wts, stream);
+        float* yl = l + 1 == L ? y : (float*)(b + W.ybuf[l & 1]);
+        rfx::MoeParams p;
+        int grid = 0;
+        size_t smem = 0;
+        const int32_t* il = idx + (size_t)l * T * d.k;
+        const float* wl = wts + (size_t)l * T * d.k;
+        rc = rfx::moe_prepare(layers[l], prev ? (const void*)prev : x, T, il, wl, yl, b + W.ffn, W.idx - W.ffn, p, grid,
+                              smem);
         if (rc != RFX_OK) return rc;
-        float* yl = l + 1 == L ? y : ybuf;
-        rc = moe_ffn_forward(layers[l], xin, T, idx, wts, yl, b + W.ffn, W.idx - W.ffn, stream);
-        if (rc != RFX_OK) return rc;
-        if (l + 1 < L) {
-            rc = moe_rms_norm_bf16(ybuf, T, d.H, xb[l & 1], stream);
-            if (rc != RFX_OK) return rc;
-            xin = xb[l & 1];
+        if (prev) {   // layer l > 0 takes the unit-RMS bf16 of the previous layer's y
+            p.x = nullptr;
+            p.xc = prev;
         }
+        cudaError_t e = rfx::moe_decode_launch(p, grid, (cudaStream_t)stream);
+        if (e != cudaSuccess) return cuda_fail("moe_stack_forward", e);
+        prev = yl;
     }
     return RFX_OK;
 }

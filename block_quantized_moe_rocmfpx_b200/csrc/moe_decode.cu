@@ -79,6 +79,9 @@ struct __align__(16) SlotTable {
     int ncols[MOE_MAXS];
     unsigned colmask[MOE_MAXS];               // columns routed to the slot (bit c)
     signed char cols[MOE_MAXS][MOE_MAXT];
+    signed char fa[MOE_MAXS];                 // gate/up format of the slot
+    signed char fb[MOE_MAXS];                 // down format
+    signed char ci[MOE_MAXS];                 // staged x copy its gate/up tiles read
     unsigned mask[32];                        // experts in use (bit per expert)
     int prefix[32];
     int idx[MOE_MAXT * MOE_MAXK];
@@ -118,6 +121,8 @@ struct Shared {
     int bar_ok;
     unsigned xmax[MOE_MAXT]; // max |x| per column (fp32 bits)
     int xn[MOE_MAXT];        // x is staged as x * 2^xn[c] (then 2^-s_b per tile position)
+    double rms_part[MOE_MAXT][8];   // chained input: per-warp sums of squares
+    double rms_r[MOE_MAXT], rms_ri[MOE_MAXT];   // its RMS per column and 1 / RMS
     SlotTable st;
 };
 
@@ -213,6 +218,17 @@ __device__ void build_slots(const MoeParams& p, SlotTable& S, const Routing& rt)
         for (int c = 0; c < p.T; ++c) S.cols[0][c] = (signed char)c;
     }
     __syncwarp();
+    // formats of every slot and the x copy of its gate/up tiles
+    for (int s = lane; s < S.nslots; s += 32) {
+        const int e = S.expert[s];
+        int fa = p.fA, fb = p.fB;
+        if (e < 0) { fa = p.fsA; fb = p.fsB; }
+        else if (p.mix) { fa = __ldg(&p.mix[e].fa); fb = __ldg(&p.mix[e].fb); }
+        S.fa[s] = (signed char)fa;
+        S.fb[s] = (signed char)fb;
+        S.ci[s] = (signed char)((p.nxc == 2 && p.xf[1] == fa) ? 1 : 0);
+    }
+    __syncwarp();
 }
 
 // Packed stream of the gate/up (phase 0) or down (phase 1) matrices of an
@@ -226,9 +242,14 @@ struct MatRef {
 __device__ __forceinline__ MatRef slot_mats(const MoeParams& p, int e, int ph) {
     if (ph == 0) {
         if (e < 0) return {p.shg, p.shu, p.fsA};
+        if (p.mix) {
+            const MoeMixEntry* m = p.mix + e;
+            return {p.gate + __ldg(&m->og), p.up + __ldg(&m->ou), __ldg(&m->fa)};
+        }
         return {p.gate + (long long)e * p.sg, p.up + (long long)e * p.su, p.fA};
     }
     if (e < 0) return {p.shd, nullptr, p.fsB};
+    if (p.mix) return {p.down + __ldg(&p.mix[e].od), nullptr, __ldg(&p.mix[e].fb)};
     return {p.down + (long long)e * p.sd, nullptr, p.fB};
 }
 
@@ -803,7 +824,7 @@ __device__ __forceinline__ void ld8(const float* src, float d[8]) {
 }
 
 // One gate/up chunk pair (chunk c of the stage's span, this warp's share).
-template <int FMT, bool TWO, class SRC>
+template <int FMT, int FC, bool TWO, class SRC>
 __device__ __forceinline__ void stepA(const uint8_t* st, int c, int H, int lane, int g, const SRC& bs, const float* sA0,
                                       const float* sA1, AccA& ag, AccA& au) {
     const int nt = rfx_chunk_tiles(H, c);
@@ -811,7 +832,7 @@ __device__ __forceinline__ void stepA(const uint8_t* st, int c, int H, int lane,
         float S0[8], S1[8];
         ld8(sA0 + 8 * c, S0);
         if (TWO) ld8(sA1 + 8 * c, S1);
-        chunkA_full<FMT, TWO>(st, st + MOE_HALF_BYTES, lane, g, bs, c * 16, S0, S1, ag, au);
+        chunkA_full<FMT, FC, TWO>(st, st + MOE_HALF_BYTES, lane, g, bs, c * 16, S0, S1, ag, au);
     } else {
         chunkA_partial<FMT, true>(st, st + MOE_HALF_BYTES, nt, lane, g, bs, c * 16, ag, au);
     }
@@ -871,24 +892,24 @@ __device__ __forceinline__ bool cons_next(const MoeParams& p, Shared& sh, ConsRi
     return true;
 }
 
-__device__ __forceinline__ int fmt_a(const MoeParams& p, const SlotTable& S, int slot) {
-    return S.expert[slot] < 0 ? p.fsA : p.fA;
+// Gate/up loop variant of a slot: 8 * its format + the format of its x copy
+// (when they differ, the scales carry the difference of the bit offsets).
+__device__ __forceinline__ int variant_a(const MoeParams& p, const SlotTable& S, int slot) {
+    return 8 * S.fa[slot] + p.xf[S.ci[slot]];
 }
-__device__ __forceinline__ int fmt_b(const MoeParams& p, const SlotTable& S, int slot) {
-    return S.expert[slot] < 0 ? p.fsB : p.fB;
-}
+__device__ __forceinline__ int fmt_b(const SlotTable& S, int slot) { return S.fb[slot]; }
 
-// Gate/up stages of one format, from the current record r (first span of a
-// row-group) while the records stay gate/up spans of that format; returns with
-// the next record in r.
-template <int FMT, bool TWO, int QC>
+// Gate/up stages of one variant (format FMT, x copy of format FC), from the
+// current record r (first span of a row-group) while the records stay gate/up
+// spans of that variant; returns with the next record in r.
+template <int FMT, int FC, bool TWO, int QC>
 __device__ __forceinline__ bool loop_a(const MoeParams& p, Shared& sh, uint8_t* ring, uint8_t* xh, uint8_t* red,
                                        ConsRing& rp, RedCursor& rc, StageRec& r) {
     const SlotTable& S = sh.st;
     const int w = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
-    const int nxc = (p.has_shared && p.fsA != p.fA) ? 2 : 1;
+    const int nxc = p.nxc;
     const float* sx = (const float*)(xh + nxc * p.T * p.x_stride);   // [copy][col][sxs]
     const int sxs = moe_sxs(p.H);
     const int nch = rfx_num_chunks(p.H);
@@ -902,7 +923,7 @@ __device__ __forceinline__ bool loop_a(const MoeParams& p, Shared& sh, uint8_t* 
         if (r.flags & REC_FIRST) {
             slot = r.slot;
             ncols = S.ncols[slot];
-            const int ci = (S.expert[slot] < 0 && nxc == 2) ? 1 : 0;
+            const int ci = S.ci[slot];
             const int colg = S.cols[slot][g < ncols ? g : 0];
             bs.base = xh + (ci * p.T + colg) * p.x_stride + t * 8;
             const int c0 = S.cols[slot][2 * t < ncols ? 2 * t : 0];
@@ -913,7 +934,8 @@ __device__ __forceinline__ bool loop_a(const MoeParams& p, Shared& sh, uint8_t* 
             au.zero();
         }
         const int c = r.c0 + w;
-        if (c < nch) stepA<FMT, TWO>(ring + rp.stage * MOE_STAGE_BYTES + w * FULLB, c, p.H, lane, g, bs, sA0, sA1, ag, au);
+        if (c < nch)
+            stepA<FMT, FC, TWO>(ring + rp.stage * MOE_STAGE_BYTES + w * FULLB, c, p.H, lane, g, bs, sA0, sA1, ag, au);
         cons_release(p, sh, rp, w, lane);
         if (r.flags & REC_LAST) {
             float v[8];
@@ -924,7 +946,24 @@ __device__ __forceinline__ bool loop_a(const MoeParams& p, Shared& sh, uint8_t* 
                 return false;
         }
         if (!cons_next(p, sh, rp, r)) return false;
-        if (r.kind != 0 || ((r.flags & REC_FIRST) && fmt_a(p, S, r.slot) != FMT)) return true;
+        if (r.kind != 0 || ((r.flags & REC_FIRST) && variant_a(p, S, r.slot) != 8 * FMT + FC)) return true;
+    }
+}
+
+// The variants whose x copy is of another format: ROCmFPX MIX layers with a
+// gate/up format that has no copy of its own (a kernel of their own, so that
+// the common variants keep their register allocation).
+template <bool TWO, int QC>
+__device__ __forceinline__ bool loop_a_other(const MoeParams& p, Shared& sh, uint8_t* ring, uint8_t* xh, uint8_t* red,
+                                             ConsRing& rp, RedCursor& rc, StageRec& r, int v) {
+    switch (v) {
+        case 8 * 2 + 3: return loop_a<2, 3, TWO, QC>(p, sh, ring, xh, red, rp, rc, r);
+        case 8 * 2 + 4: return loop_a<2, 4, TWO, QC>(p, sh, ring, xh, red, rp, rc, r);
+        case 8 * 3 + 2: return loop_a<3, 2, TWO, QC>(p, sh, ring, xh, red, rp, rc, r);
+        case 8 * 3 + 4: return loop_a<3, 4, TWO, QC>(p, sh, ring, xh, red, rp, rc, r);
+        case 8 * 4 + 2: return loop_a<4, 2, TWO, QC>(p, sh, ring, xh, red, rp, rc, r);
+        case 8 * 4 + 3: return loop_a<4, 3, TWO, QC>(p, sh, ring, xh, red, rp, rc, r);
+        default: return false;
     }
 }
 
@@ -998,13 +1037,13 @@ __device__ __forceinline__ bool loop_b(const MoeParams& p, Shared& sh, uint8_t* 
         }
         cons_release(p, sh, rp, w, lane);
         if (!cons_next(p, sh, rp, r)) return false;
-        if (r.kind != 1 || fmt_b(p, S, r.slot) != FMT) return true;
+        if (r.kind != 1 || fmt_b(S, r.slot) != FMT) return true;
     }
 }
 
 // Consumer warp: the records of a CTA's stream are its gate/up spans, then its
 // down spans, then the end record.  Each phase runs one loop per format.
-template <int QC>
+template <int QC, bool OTHER>
 __device__ void consumer(const MoeParams& p, Shared& sh, uint8_t* ring, uint8_t* xh, uint8_t* red) {
     constexpr bool TWO = QC >= 2;           // a second live column per lane in the gate/up output
     constexpr int NB = QC >= 3 ? 2 : 1;     // n-blocks of virtual (hi, lo) columns in the down projection
@@ -1018,13 +1057,15 @@ __device__ void consumer(const MoeParams& p, Shared& sh, uint8_t* ring, uint8_t*
     HView<NB, HSTRIDE> hv;
     bool ok = cons_next(p, sh, rp, r);
     while (ok && r.kind == 0) {
-        const int f = fmt_a(p, S, r.slot);
-        if (f == 2) ok = loop_a<2, TWO, QC>(p, sh, ring, xh, red, rp, rc, r);
-        else if (f == 3) ok = loop_a<3, TWO, QC>(p, sh, ring, xh, red, rp, rc, r);
-        else ok = loop_a<4, TWO, QC>(p, sh, ring, xh, red, rp, rc, r);
+        const int v = variant_a(p, S, r.slot);
+        if (v == 8 * 2 + 2) ok = loop_a<2, 2, TWO, QC>(p, sh, ring, xh, red, rp, rc, r);
+        else if (v == 8 * 3 + 3) ok = loop_a<3, 3, TWO, QC>(p, sh, ring, xh, red, rp, rc, r);
+        else if (v == 8 * 4 + 4) ok = loop_a<4, 4, TWO, QC>(p, sh, ring, xh, red, rp, rc, r);
+        else if constexpr (OTHER) ok = loop_a_other<TWO, QC>(p, sh, ring, xh, red, rp, rc, r, v);
+        else ok = false;
     }
     while (ok && r.kind == 1) {
-        const int f = fmt_b(p, S, r.slot);
+        const int f = fmt_b(S, r.slot);
         if (f == 3) ok = loop_b<3, NB, HSTRIDE, QC>(p, sh, ring, xh, red, rp, rc, r, hv);
         else if (f == 2) ok = loop_b<2, NB, HSTRIDE, QC>(p, sh, ring, xh, red, rp, rc, r, hv);
         else ok = loop_b<4, NB, HSTRIDE, QC>(p, sh, ring, xh, red, rp, rc, r, hv);
@@ -1077,7 +1118,7 @@ __device__ __forceinline__ void x_put(const MoeParams& p, Shared& sh, uint8_t* x
     const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
     const int step = j >> 1, half = j & 1;
     for (int ci = 0; ci < nxc; ++ci) {
-        const int fmt = ci == 0 ? p.fA : p.fsA;
+        const int fmt = p.xf[ci];
         const int sb = s_pos(fmt, j * 8, p.H);
         const float sc = __int_as_float((127 + sh.xn[c] - sb) << 23);
         float sum = 0.f;
@@ -1096,12 +1137,75 @@ __device__ __forceinline__ void x_put(const MoeParams& p, Shared& sh, uint8_t* x
     }
 }
 
+// Chained input (the next layer of a stack): x = bf16(y / r), r = sqrt of the
+// mean of y^2 per column, bit for bit what moe_rms_norm_bf16 gives: the sum
+// of squares in its order (threads 0..255, element i on thread i mod 256,
+// fp64 fma, then the two warp trees) and the nearest-even bf16 of the fp64
+// quotient y / r.
+__device__ void chain_rms(const MoeParams& p, Shared& sh, int sid, int nthr) {
+    const int lane = sid & 31;
+    if (sid < 256) {
+        for (int c = 0; c < p.T; ++c) {
+            const float* yc = p.xc + (long long)c * p.H;
+            double ss = 0.0;
+            for (int i = sid; i < p.H; i += 256) {
+                const double v = (double)__ldg(yc + i);
+                ss = fma(v, v, ss);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            if (lane == 0) sh.rms_part[c][sid >> 5] = ss;
+        }
+    }
+    asm volatile("bar.sync 1, %0;" ::"r"(nthr) : "memory");
+    if (sid < 32) {
+        for (int c = 0; c < p.T; ++c) {
+            double t = lane < 8 ? sh.rms_part[c][lane] : 0.0;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+            if (lane == 0) {
+                const double r = sqrt(t / (double)p.H);
+                sh.rms_r[c] = r;
+                sh.rms_ri[c] = 1.0 / r;
+            }
+        }
+    }
+    asm volatile("bar.sync 1, %0;" ::"r"(nthr) : "memory");
+}
+
+// bf16 bits of y / r.  The product y * (1/r) is within 3 fp64 ulps of the
+// rounded quotient; unless it lies within half an fp32 ulp (plus that margin)
+// of a bf16 rounding tie, or outside the normal bf16 range, its bf16 through
+// fp32 (two nearest-even steps) equals the quotient's.  Otherwise divide.
+__device__ __forceinline__ uint32_t chain_bf16(float y, double r, double ri) {
+    const double q = (double)y * ri;
+    const unsigned long long b = (unsigned long long)__double_as_longlong(q);
+    const int e = (int)((b >> 52) & 0x7FF);
+    const long long d = (long long)(b & ((1ull << 45) - 1ull)) - (1ll << 44);
+    constexpr long long WIN = (1ll << 28) + 8;
+    if (e < 1023 - 126 || e == 0x7FF || (d < WIN && d > -WIN)) return f64_to_bf16_rne((double)y / r);
+    return __bfloat16_as_ushort(__float2bfloat16_rn(__double2float_rn(q)));
+}
+
+// Item i (8 consecutive values of a column) of x as bf16 bits.
+__device__ __forceinline__ uint4 load_item(const MoeParams& p, const Shared& sh, int i, int per_col) {
+    if (!p.xc) return __ldg(reinterpret_cast<const uint4*>(p.x) + i);
+    const int c = i / per_col;
+    const float4 a = __ldg(reinterpret_cast<const float4*>(p.xc) + 2 * i);
+    const float4 b = __ldg(reinterpret_cast<const float4*>(p.xc) + 2 * i + 1);
+    const double r = sh.rms_r[c], ri = sh.rms_ri[c];
+    return make_uint4(chain_bf16(a.x, r, ri) | (chain_bf16(a.y, r, ri) << 16),
+                      chain_bf16(a.z, r, ri) | (chain_bf16(a.w, r, ri) << 16),
+                      chain_bf16(b.x, r, ri) | (chain_bf16(b.y, r, ri) << 16),
+                      chain_bf16(b.z, r, ri) | (chain_bf16(b.w, r, ri) << 16));
+}
+
 __device__ void stage_x(const MoeParams& p, Shared& sh, uint8_t* xh, int sid, int nthr) {
     const int lane = sid & 31;
     const int per_col = p.H / 8;
     const int nitems = p.T * per_col;
-    const uint4* x4 = reinterpret_cast<const uint4*>(p.x);
-    const int nxc = (p.has_shared && p.fsA != p.fA) ? 2 : 1;
+    if (p.xc) chain_rms(p, sh, sid, nthr);
+    const int nxc = p.nxc;
     float* sx = (float*)(xh + nxc * p.T * p.x_stride);
     const int sxs = moe_sxs(p.H);
     const bool one_round = nitems <= XR * nthr;   // then pass 2 reuses the loaded items
@@ -1111,7 +1215,7 @@ __device__ void stage_x(const MoeParams& p, Shared& sh, uint8_t* xh, int sid, in
 #pragma unroll
         for (int k = 0; k < XR; ++k) {
             const int i = r0 + sid + k * nthr;
-            v[k] = i < nitems ? __ldg(x4 + i) : make_uint4(0u, 0u, 0u, 0u);
+            v[k] = i < nitems ? load_item(p, sh, i, per_col) : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
         for (int k = 0; k < XR; ++k) {
@@ -1133,7 +1237,7 @@ __device__ void stage_x(const MoeParams& p, Shared& sh, uint8_t* xh, int sid, in
 #pragma unroll
             for (int k = 0; k < XR; ++k) {
                 const int i = r0 + sid + k * nthr;
-                v[k] = i < nitems ? __ldg(x4 + i) : make_uint4(0u, 0u, 0u, 0u);
+                v[k] = i < nitems ? load_item(p, sh, i, per_col) : make_uint4(0u, 0u, 0u, 0u);
             }
         }
 #pragma unroll
@@ -1147,7 +1251,7 @@ __device__ void stage_x(const MoeParams& p, Shared& sh, uint8_t* xh, int sid, in
 
 // ---------------------------------------------------------------- kernel ---
 
-template <int QC>
+template <int QC, bool OTHER>
 __global__ void __launch_bounds__(NTHREADS, 1) moe_decode_kernel(MoeParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* ring = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -1203,7 +1307,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) moe_decode_kernel(MoeParams p) {
         const int sid = w < WARP_PRODUCER ? threadIdx.x : threadIdx.x - 32;
         stage_x(p, sh, xh, sid, NSTAGE_THREADS);
         asm volatile("bar.sync 2, %0;" ::"n"(NTHREADS) : "memory");
-        if (w < NCW) consumer<QC>(p, sh, ring, xh, red);
+        if (w < NCW) consumer<QC, OTHER>(p, sh, ring, xh, red);
         else epilogue_warp<QC>(p, sh, red, w - WARP_EPI0);
     }
     __syncthreads();
@@ -1257,10 +1361,13 @@ size_t moe_decode_smem_bytes(int ns, int nred, int xh_bytes, int qc) {
 cudaError_t moe_decode_launch(const MoeParams& p, int grid, cudaStream_t stream) {
     const int qc = moe_qclass(p.T);
     const size_t smem = moe_decode_smem_bytes(p.ns, p.nred, p.xh_bytes, qc);
-    auto kern = qc == 1 ? moe_decode_kernel<1> : (qc == 2 ? moe_decode_kernel<2> : moe_decode_kernel<3>);
+    void (*kerns[2][3])(MoeParams) = {{moe_decode_kernel<1, false>, moe_decode_kernel<2, false>, moe_decode_kernel<3, false>},
+                                       {moe_decode_kernel<1, true>, moe_decode_kernel<2, true>, moe_decode_kernel<3, true>}};
+    const int ot = p.other ? 1 : 0;
+    auto kern = kerns[ot][qc - 1];
     // the dynamic shared-memory limit, once per device and kernel
-    static SmemLimit limit[3];
-    cudaError_t err = limit[qc - 1].ensure((const void*)kern, (int)smem);
+    static SmemLimit limit[2][3];
+    cudaError_t err = limit[ot][qc - 1].ensure((const void*)kern, (int)smem);
     if (err != cudaSuccess) return err;
     // cooperative: every CTA is resident at once (the final grid barrier needs it)
     cudaLaunchConfig_t cfg = {};

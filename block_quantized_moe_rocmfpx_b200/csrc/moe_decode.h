@@ -30,6 +30,14 @@
 
 namespace rfx {
 
+// ROCmFPX MIX: the packed matrices of routed expert e are at gate + og,
+// up + ou, down + od, gate and up in format fa, down in format fb.
+struct MoeMixEntry {
+    long long og, ou, od;
+    int fa, fb;
+};
+static_assert(sizeof(MoeMixEntry) == 32, "one 32-byte entry per expert");
+
 struct MoeParams {
     int H, I, E, k, T;
     int fA, fB, fsA, fsB;  // routed gate/up, routed down, shared gate/up, shared down formats
@@ -37,11 +45,16 @@ struct MoeParams {
     const uint8_t* up;
     const uint8_t* down;
     long long sg, su, sd;  // routed expert strides (bytes)
+    const MoeMixEntry* mix;  // device [E], or null: every routed expert at e * stride in fA / fB
+    int nxc;               // copies of the staged x (gate/up formats with their own copy)
+    int xf[2];             // format of each copy; a slot of another format reads copy 0 with compensated scales
+    int other;             // some routed expert's gate/up format has no copy (the kernel with those variants)
     int has_shared;
     const uint8_t* shg;
     const uint8_t* shu;
     const uint8_t* shd;
     const uint16_t* x;     // bf16 [T][H]
+    const float* xc;       // or, chained from a previous layer: fp32 [T][H], x = bf16(xc / rms(xc)) per column
     const int32_t* idx;    // [T][k]
     const float* wts;      // [T][k]
     float* y;              // [T][H]

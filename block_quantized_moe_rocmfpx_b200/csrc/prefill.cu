@@ -422,15 +422,20 @@ struct PfSrc {
 __device__ __forceinline__ PfSrc pf_src(const PfParams& p, int mode, const PfUnit& U, int rg, int sub) {
     PfSrc S;
     S.f = mode == 0 ? (U.e >= 0 ? p.fA : p.fsA) : (U.e >= 0 ? p.fB : p.fsB);
+    long long og = (long long)U.e * p.sg, ou = (long long)U.e * p.su, od = (long long)U.e * p.sd;
+    if (p.mix && U.e >= 0) {   // ROCmFPX MIX: the expert's own format and place
+        const MoeMixEntry* m = p.mix + U.e;
+        S.f = mode == 0 ? __ldg(&m->fa) : __ldg(&m->fb);
+        og = __ldg(&m->og); ou = __ldg(&m->ou); od = __ldg(&m->od);
+    }
     const int K = mode == 0 ? p.H : p.I;
     const long long rgb = (long long)(K / 32) * 16 * rfx_block_bytes(S.f);
     S.cb = 128 * rfx_block_bytes(S.f);
     const long long off = ((long long)U.rt * (PF_BM / 16) + rg) * rgb;
     if (mode == 0)
-        S.m = (sub == 0 ? (U.e >= 0 ? p.gate + (long long)U.e * p.sg : p.shg)
-                        : (U.e >= 0 ? p.up + (long long)U.e * p.su : p.shu)) + off;
+        S.m = (sub == 0 ? (U.e >= 0 ? p.gate + og : p.shg) : (U.e >= 0 ? p.up + ou : p.shu)) + off;
     else
-        S.m = (U.e >= 0 ? p.down + (long long)U.e * p.sd : p.shd) + off;
+        S.m = (U.e >= 0 ? p.down + od : p.shd) + off;
     return S;
 }
 

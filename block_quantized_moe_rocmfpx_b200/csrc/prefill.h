@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "moe_decode.h"
+
 // workspace control words (uint32 index).  Word 2 is the device error flag,
 // at the same place as in the decode workspace so that one status call reads
 // both.
@@ -31,6 +33,7 @@ struct PfParams {
     const uint8_t* up;
     const uint8_t* down;
     long long sg, su, sd;   // routed expert strides (bytes)
+    const MoeMixEntry* mix; // device [E], or null: every routed expert at e * stride in fA / fB
     int has_shared;
     const uint8_t* shg;
     const uint8_t* shu;

@@ -28,6 +28,44 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 
+// Round a double to bf16 bits, nearest-even, in one step (no intermediate
+// float rounding): sign, 8-bit exponent with bias 127, 7 explicit mantissa
+// bits; values below 2^-126 become bf16 subnormals, values beyond the largest
+// finite bf16 become infinity.
+__device__ __forceinline__ uint16_t f64_to_bf16_rne(double v) {
+    const unsigned long long d = (unsigned long long)__double_as_longlong(v);
+    const uint32_t sign = (uint32_t)(d >> 48) & 0x8000u;
+    const int e = (int)((d >> 52) & 0x7FF);
+    const unsigned long long m = d & ((1ull << 52) - 1ull);
+    if (e == 0x7FF) return (uint16_t)(sign | 0x7F80u | (m ? 0x40u : 0u));   // inf / nan
+    if (e == 0) return (uint16_t)sign;                                       // zero (and fp64 subnormals)
+    const int E = e - 1023;                                                  // unbiased exponent
+    const unsigned long long sig = (1ull << 52) | m;                         // 53-bit significand
+    int shift;                                                               // significand bits dropped
+    int be;                                                                  // bf16 biased exponent before rounding
+    if (E >= -126) {
+        shift = 45;
+        be = E + 127;
+    } else {
+        shift = 45 + (-126 - E);                                             // subnormal: fixed exponent 2^-126
+        be = 0;
+        if (shift > 54) return (uint16_t)sign;                               // rounds to zero
+    }
+    unsigned long long q = sig >> shift;
+    const unsigned long long rem = sig & ((1ull << shift) - 1ull), half = 1ull << (shift - 1);
+    if (rem > half || (rem == half && (q & 1ull))) ++q;
+    // q holds the implicit bit (normal) at bit 7; a carry out of it bumps the exponent
+    uint32_t bits;
+    if (be > 0) {
+        if (q >> 8) { q >>= 1; ++be; }
+        if (be >= 255) return (uint16_t)(sign | 0x7F80u);
+        bits = ((uint32_t)be << 7) | (uint32_t)(q & 0x7Fu);
+    } else {
+        bits = (uint32_t)q;   // subnormal; q == 0x80 is the smallest normal, which has the same bits
+    }
+    return (uint16_t)(sign | bits);
+}
+
 // silu(g) * u for g < -64, where sigmoid(g) equals exp(g) to fp32 precision.
 // exp(g) is taken as exp(g + 64 ln 2) * 2^-64 so that the products stay in
 // fp32's normal range while h itself is still representable (a plain

@@ -176,9 +176,14 @@ __device__ __forceinline__ void mma_tile(float c[4], const uint32_t a[8], uint2 
 // One full gate/up chunk pair sharing the x fragments (x pre-scaled by
 // 2^-s_b): all tiles accumulate in units of 2^-24.  S[b] / S1[b] are the
 // block sums of the lane's two columns; TWO = the second column can be live.
-template <int FMT, bool TWO, class SRC>
+// FC: the format whose bit offsets s'_b the x fragments were pre-scaled for.
+// When FC != FMT, 2^(s'_b - s_b) goes on the products' scales (a power of
+// two: exact); the block sums, which do not depend on the offsets, keep the
+// raw scale.
+template <int FMT, int FC, bool TWO, class SRC>
 __device__ __forceinline__ void chunkA_full(const uint8_t* st0, const uint8_t* st1, int lane, int g, const SRC& bs,
                                             int step0, const float* S0, const float* S1, AccA& ag, AccA& au) {
+    constexpr bool COMP = FC != FMT;
     FullChunk<FMT> f0, f1;
     f0.load(st0, lane, g);
     f1.load(st1, lane, g);
@@ -199,13 +204,16 @@ __device__ __forceinline__ void chunkA_full(const uint8_t* st0, const uint8_t* s
         }
         mma_tile(c, a, blo, bhi);
         f0.scales(b, s0, s1);
-        ag.acc[0] = fmaf(s0, c[0], ag.acc[0]);
-        ag.acc[2] = fmaf(s1, c[2], ag.acc[2]);
+        const float cmb = __int_as_float((127 + Plane<FC>::s_of(b) - Plane<FMT>::s_of(b)) << 23);
+        float p0 = s0, p1 = s1;
+        if (COMP) { p0 *= cmb; p1 *= cmb; }
+        ag.acc[0] = fmaf(p0, c[0], ag.acc[0]);
+        ag.acc[2] = fmaf(p1, c[2], ag.acc[2]);
         ag.corr[0] = fmaf(s0, S0[b], ag.corr[0]);
         ag.corr[2] = fmaf(s1, S0[b], ag.corr[2]);
         if (TWO) {
-            ag.acc[1] = fmaf(s0, c[1], ag.acc[1]);
-            ag.acc[3] = fmaf(s1, c[3], ag.acc[3]);
+            ag.acc[1] = fmaf(p0, c[1], ag.acc[1]);
+            ag.acc[3] = fmaf(p1, c[3], ag.acc[3]);
             ag.corr[1] = fmaf(s0, S1[b], ag.corr[1]);
             ag.corr[3] = fmaf(s1, S1[b], ag.corr[3]);
         }
@@ -221,13 +229,15 @@ __device__ __forceinline__ void chunkA_full(const uint8_t* st0, const uint8_t* s
         }
         mma_tile(c, a, blo, bhi);
         f1.scales(b, s0, s1);
-        au.acc[0] = fmaf(s0, c[0], au.acc[0]);
-        au.acc[2] = fmaf(s1, c[2], au.acc[2]);
+        p0 = s0; p1 = s1;
+        if (COMP) { p0 *= cmb; p1 *= cmb; }
+        au.acc[0] = fmaf(p0, c[0], au.acc[0]);
+        au.acc[2] = fmaf(p1, c[2], au.acc[2]);
         au.corr[0] = fmaf(s0, S0[b], au.corr[0]);
         au.corr[2] = fmaf(s1, S0[b], au.corr[2]);
         if (TWO) {
-            au.acc[1] = fmaf(s0, c[1], au.acc[1]);
-            au.acc[3] = fmaf(s1, c[3], au.acc[3]);
+            au.acc[1] = fmaf(p0, c[1], au.acc[1]);
+            au.acc[3] = fmaf(p1, c[3], au.acc[3]);
             au.corr[1] = fmaf(s0, S1[b], au.corr[1]);
             au.corr[3] = fmaf(s1, S1[b], au.corr[3]);
         }

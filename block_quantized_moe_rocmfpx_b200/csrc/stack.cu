@@ -5,47 +5,10 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "rfx_device.cuh"
 #include "stack.h"
 
 namespace rfx {
-
-// Round a double to bf16 bits, nearest-even, in one step (no intermediate
-// float rounding): sign, 8-bit exponent with bias 127, 7 explicit mantissa
-// bits; values below 2^-126 become bf16 subnormals, values beyond the largest
-// finite bf16 become infinity.
-__device__ __forceinline__ uint16_t f64_to_bf16_rne(double v) {
-    const unsigned long long d = (unsigned long long)__double_as_longlong(v);
-    const uint32_t sign = (uint32_t)(d >> 48) & 0x8000u;
-    const int e = (int)((d >> 52) & 0x7FF);
-    const unsigned long long m = d & ((1ull << 52) - 1ull);
-    if (e == 0x7FF) return (uint16_t)(sign | 0x7F80u | (m ? 0x40u : 0u));   // inf / nan
-    if (e == 0) return (uint16_t)sign;                                       // zero (and fp64 subnormals)
-    const int E = e - 1023;                                                  // unbiased exponent
-    const unsigned long long sig = (1ull << 52) | m;                         // 53-bit significand
-    int shift;                                                               // significand bits dropped
-    int be;                                                                  // bf16 biased exponent before rounding
-    if (E >= -126) {
-        shift = 45;
-        be = E + 127;
-    } else {
-        shift = 45 + (-126 - E);                                             // subnormal: fixed exponent 2^-126
-        be = 0;
-        if (shift > 54) return (uint16_t)sign;                               // rounds to zero
-    }
-    unsigned long long q = sig >> shift;
-    const unsigned long long rem = sig & ((1ull << shift) - 1ull), half = 1ull << (shift - 1);
-    if (rem > half || (rem == half && (q & 1ull))) ++q;
-    // q holds the implicit bit (normal) at bit 7; a carry out of it bumps the exponent
-    uint32_t bits;
-    if (be > 0) {
-        if (q >> 8) { q >>= 1; ++be; }
-        if (be >= 255) return (uint16_t)(sign | 0x7F80u);
-        bits = ((uint32_t)be << 7) | (uint32_t)(q & 0x7Fu);
-    } else {
-        bits = (uint32_t)q;   // subnormal; q == 0x80 is the smallest normal, which has the same bits
-    }
-    return (uint16_t)(sign | bits);
-}
 
 // One CTA per column: fp64 sum of squares, then x = bf16(y / sqrt(mean)).
 __global__ void __launch_bounds__(256) rms_bf16_kernel(const float* __restrict__ y, int H, uint16_t* __restrict__ x) {

@@ -211,6 +211,30 @@ int moe_layer_create(const moe_layer_desc* d, moe_layer** out);
 void moe_layer_destroy(moe_layer* layer);
 
 /*
+ * ROCmFPX MIX ([MZ] "ROCmFPX 量化"): the codebook width is chosen per routed
+ * expert from its routing heat (hot experts wider), so experts differ in
+ * format and in packed size.  Entry e describes routed expert e: the format
+ * of its gate and up matrices (one format for both), the format of its down
+ * matrix, and the byte offsets of the three packed matrices from the
+ * descriptor's gate, up and down bases (multiples of 16).
+ */
+typedef struct {
+    rfx_format f_gate_up, f_down;
+    uint64_t off_gate, off_up, off_down;
+} moe_expert_mix;
+
+/*
+ * As moe_layer_create, with a format per routed expert: mix is a host array
+ * of d->E entries; d's routed formats and strides are ignored (its bases,
+ * shapes and shared expert are used as given).  Copies the table to the
+ * current CUDA device (E * 32 bytes of device memory, allocated here and
+ * freed by moe_layer_destroy; the layer is then used on that device).  Every
+ * entry point that takes a layer accepts a MIX layer.  Errors: RFX_EINVAL for
+ * a bad format or an unaligned offset, RFX_ECUDA if the copy fails.
+ */
+int moe_layer_create_mix(const moe_layer_desc* d, const moe_expert_mix* mix, moe_layer** out);
+
+/*
  * Device workspace bytes moe_ffn_forward needs for T token columns (T > 8:
  * the prefill workspace, moe_prefill_workspace_bytes).  The
  * workspace holds counters, the SwiGLU intermediate and per-expert partial
@@ -362,8 +386,12 @@ int moe_rms_norm_bf16(const float* y, int T, int H, void* x_next, void* stream);
  * [L][T][E]; x: device bf16 bits [T][H] (x_0); y: device fp32 [T][H].  All
  * layers must share H, E and k.  The workspace (moe_stack_workspace_bytes,
  * 256-byte aligned, caller-owned) holds one moe_ffn_forward workspace (zero it
- * once with rfx_ws_init), the routing and the chained activations.  Launches
- * 3 kernels per layer and can be captured in a CUDA graph.
+ * once with rfx_ws_init), the routing of every layer and two fp32 activation
+ * buffers.  Launches 1 + L kernels: the router for all L * T rows at once,
+ * then one MoE FFN kernel per layer; for l > 0 that kernel reads y_{l-1} and
+ * applies the unit-RMS bf16 step itself while it stages x (the same bits as
+ * moe_rms_norm_bf16).  The result equals the step-by-step calls bit for bit.
+ * Can be captured in a CUDA graph.
  */
 size_t moe_stack_workspace_bytes(const moe_layer* const* layers, int L, int T);
 int moe_stack_forward(const moe_layer* const* layers, int L, const float* logits, const void* x, int T, float* y,

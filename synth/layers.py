@@ -24,20 +24,42 @@ class SynthLayer:
     """Packed device buffers of one synthetic layer (seed, layer)."""
 
     def __init__(self, seed: int, layer: int, H: int, I: int, E: int, k: int, fmts=(2, 2, 3), shared_fmts=(4, 4, 4),
-                 has_shared: bool = True, device="cuda", experts=None):
+                 has_shared: bool = True, device="cuda", experts=None, mix=None):
+        """mix: ROCmFPX MIX, E pairs (gate/up format, down format), one per
+        routed expert; the experts are then packed back to back (256-byte
+        aligned) and `fmts` is ignored."""
         import block_quantized_moe_rocmfpx_b200 as rfx
         self.seed, self.layer, self.H, self.I, self.E, self.k = seed, layer, H, I, E, k
         self.fmts, self.shared_fmts, self.has_shared = tuple(fmts), tuple(shared_fmts), has_shared
+        self.mix = None if mix is None else [(int(a), int(a), int(b)) for a, b in mix]
         shapes = ((I, H), (I, H), (H, I))
-        self.strides = tuple(_align(rfx.rfx_packed_bytes(f, r, c)) for f, (r, c) in zip(fmts, shapes))
-        self.bufs = [torch.empty(E * s, dtype=torch.uint8, device=device) for s in self.strides]
+        if self.mix is None:
+            self.expert_fmts = [self.fmts] * E
+            self.strides = tuple(_align(rfx.rfx_packed_bytes(f, r, c)) for f, (r, c) in zip(fmts, shapes))
+            self.offsets = [[e * s for e in range(E)] for s in self.strides]
+            sizes = [E * s for s in self.strides]
+        else:
+            assert len(self.mix) == E
+            self.expert_fmts = self.mix
+            self.strides = (0, 0, 0)
+            self.offsets, sizes = [], []
+            for i, (r, c) in enumerate(shapes):
+                off, o = [], 0
+                for e in range(E):
+                    off.append(o)
+                    o += _align(rfx.rfx_packed_bytes(self.mix[e][i], r, c))
+                self.offsets.append(off)
+                sizes.append(o)
+        self.bufs = [torch.empty(n, dtype=torch.uint8, device=device) for n in sizes]
         cmax = max(H, I) * max(H, I)
         codes = torch.empty(cmax, dtype=torch.uint8, device=device)
         scales = torch.empty(cmax // 32 * 2, dtype=torch.uint8, device=device)
         todo = range(E) if experts is None else experts
         for e in todo:
-            for kind, f, (r, c), buf, s in zip(ROUTED_KINDS, fmts, shapes, self.bufs, self.strides):
-                self._gen(kind, e, f, r, c, codes, scales, buf[e * s:(e + 1) * s])
+            for i, (kind, (r, c), buf) in enumerate(zip(ROUTED_KINDS, shapes, self.bufs)):
+                f = self.expert_fmts[e][i]
+                o = self.offsets[i][e]
+                self._gen(kind, e, f, r, c, codes, scales, buf[o:o + _align(rfx.rfx_packed_bytes(f, r, c))])
         self.shared = None
         if has_shared:
             self.shared = []
@@ -46,7 +68,9 @@ class SynthLayer:
                 self._gen(kind, 0, f, r, c, codes, scales, buf)
                 self.shared.append(buf)
         torch.cuda.synchronize()
-        self.packed_bytes_per_expert = sum(rfx.rfx_packed_bytes(f, r, c) for f, (r, c) in zip(fmts, shapes))
+        self.expert_bytes = [sum(rfx.rfx_packed_bytes(f, r, c) for f, (r, c) in zip(self.expert_fmts[e], shapes))
+                             for e in range(E)]
+        self.packed_bytes_per_expert = self.expert_bytes[0]
         self.shared_bytes = sum(rfx.rfx_packed_bytes(f, r, c) for f, (r, c) in zip(shared_fmts, shapes)) \
             if has_shared else 0
 
@@ -61,15 +85,38 @@ class SynthLayer:
         H, I = self.H, self.I
         routed = kind in ROUTED_KINDS
         idx = (ROUTED_KINDS if routed else SHARED_KINDS).index(kind)
-        f = (self.fmts if routed else self.shared_fmts)[idx]
+        f = (self.expert_fmts[expert] if routed else self.shared_fmts)[idx]
         r, c = ((I, H), (I, H), (H, I))[idx]
         return synth.MatrixSpec(self.seed, self.layer, kind, expert if routed else 0, f, r, c)
 
-    def moe_layer(self, max_T: int = 8):
+    def moe_layer(self, max_T: int = 8, bufs=None, shared=None):
+        """The library's layer handle over these buffers (or over copies of
+        them with the same layout: bufs, shared)."""
         import block_quantized_moe_rocmfpx_b200 as rfx
-        return rfx.MoeLayer(self.H, self.I, self.E, self.k, self.fmts, *self.bufs, self.strides,
-                            shared=self.shared, shared_fmts=self.shared_fmts, max_T=max_T)
+        bufs = self.bufs if bufs is None else bufs
+        shared = self.shared if shared is None else shared
+        mix = None
+        if self.mix is not None:
+            mix = [(self.mix[e][0], self.mix[e][2], self.offsets[0][e], self.offsets[1][e], self.offsets[2][e])
+                   for e in range(self.E)]
+        return rfx.MoeLayer(self.H, self.I, self.E, self.k, self.fmts, *bufs, self.strides,
+                            shared=shared, shared_fmts=self.shared_fmts, max_T=max_T, mix=mix)
 
     def union_bytes(self, experts) -> int:
         """Packed weight bytes one pass reads for the given union of routed experts."""
-        return len(set(int(e) for e in experts)) * self.packed_bytes_per_expert + self.shared_bytes
+        return sum(self.expert_bytes[e] for e in set(int(e) for e in experts)) + self.shared_bytes
+
+
+def heat_mix(seed: int, layer: int, E: int, zipf_s: float):
+    """ROCmFPX MIX chosen by routing heat: experts ranked by their Zipf
+    popularity; the hottest eighth FP4 gate/up and FP4 down, the next three
+    eighths FP3 / FP3, the rest FP2 / FP3 (the uniform layer's assignment)."""
+    import numpy as np
+    order = np.argsort(-synth.zipf_bias(seed, layer, E, zipf_s), kind="stable")
+    mix = [(2, 3)] * E
+    for r, e in enumerate(order):
+        if r < E // 8:
+            mix[e] = (4, 4)
+        elif r < E // 2:
+            mix[e] = (3, 3)
+    return mix

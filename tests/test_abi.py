@@ -220,6 +220,36 @@ def test_layer_create_validation():
     assert lib.moe_ffn_forward(None, None, 1, None, None, None, None, 0, None) == rfx.RFX_EINVAL
 
 
+def test_mix_layer_create_validation():
+    """moe_layer_create_mix checks every entry before it touches the device:
+    formats 2..4 and 16-byte offsets; the descriptor's own checks still apply."""
+    d = rfx.moe_layer_desc()
+    d.H, d.I, d.E, d.k = 512, 256, 3, 2
+    d.f_gate = d.f_up = d.f_down = 9          # ignored by the MIX entry point
+    d.gate = d.up = d.down = 256
+    good = [(2, 3, 0, 0, 0), (3, 3, 4096, 4096, 4096), (4, 2, 8192, 8192, 8192)]
+    for e, bad_entry in ((1, (5, 3, 4096, 4096, 4096)), (2, (4, 1, 8192, 8192, 8192)),
+                         (1, (3, 3, 4100, 4096, 4096)), (2, (4, 2, 8192, 8192, 8200))):
+        mix = list(good)
+        mix[e] = bad_entry
+        with pytest.raises(rfx.RfxError) as ei:
+            rfx.moe_layer_create_mix(d, mix)
+        assert ei.value.code == rfx.RFX_EINVAL
+    bad = rfx.moe_layer_desc.from_buffer_copy(d)
+    bad.k = 4                                   # k > E
+    with pytest.raises(rfx.RfxError):
+        rfx.moe_layer_create_mix(bad, good)
+
+
+def test_heat_mix_gives_hot_experts_the_widest_codebooks():
+    from synth.layers import heat_mix
+    mix = heat_mix(0, 0, 256, 1.1)
+    order = np.argsort(-synth.zipf_bias(0, 0, 256, 1.1), kind="stable")
+    assert [mix[e] for e in order[:32]] == [(4, 4)] * 32
+    assert {mix[e] for e in order[32:128]} == {(3, 3)}
+    assert {mix[e] for e in order[128:]} == {(2, 3)}
+
+
 def test_zero_token_calls_are_noops():
     """T = 0 returns OK without touching any buffer (reading: an empty batch is
     a no-op), for every entry point that takes T."""

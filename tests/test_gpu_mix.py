@@ -1,0 +1,131 @@
+"""ROCmFPX MIX on the GPU: a format per routed expert (moe_layer_create_mix).
+
+The pages (m.mzlw.cn, "Lucebox专攻DeepSeek V4…", section "ROCmFPX 量化") pick
+the codebook width of each expert from its routing heat and mix FP2, FP3 and
+FP4 in one layer.  Each case below runs the decode kernel (T <= 8) and the
+prefill grouped GEMM (T > 8) on such a layer and compares every column with
+the oracle, which decodes each expert in its own format.  The layers cover
+the x-staging cases of the decode kernel: a gate/up format with its own x
+copy, and a third format that reads another format's copy with corrected
+scales (with and without a shared expert).
+"""
+import numpy as np
+import pytest
+import torch
+
+import block_quantized_moe_rocmfpx_b200 as rfx
+import oracle
+import synth
+from helpers import OracleLayer, check_close
+from synth.layers import SynthLayer, heat_mix
+from test_gpu_prefill import full_check
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+# (gate/up, down) per routed expert: all nine pairs
+MIX9 = [(2, 2), (2, 3), (2, 4), (3, 2), (3, 3), (3, 4), (4, 2), (4, 3), (4, 4)]
+
+
+def to_dev(a, dtype=None):
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    if dtype is not None:
+        t = t.view(dtype)
+    return t.to(DEV)
+
+
+def run_decode(lay, L, xb, T, k):
+    ml = lay.moe_layer()
+    idx = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    w = torch.empty((T, k), dtype=torch.float32, device=DEV)
+    y = torch.full((T, lay.H), float("nan"), dtype=torch.float32, device=DEV)
+    rfx.moe_router_topk(to_dev(L), k, idx, w)
+    ml.forward(to_dev(xb, torch.bfloat16), idx, w, y)
+    assert ml.status() == rfx.RFX_OK, rfx.rfx_last_error()
+    return idx.cpu().numpy(), y.cpu().numpy()
+
+
+def check_decode(lay, seed, T, what):
+    L = synth.logits(seed, 0, 0, T, lay.E, 0.0)
+    xb = synth.x_bf16(seed, 0, T, lay.H)
+    idx, y = run_decode(lay, L, xb, T, lay.k)
+    idx_o, w_o = oracle.router_topk(L, lay.k)
+    assert np.array_equal(idx, idx_o)
+    ol = OracleLayer(lay)
+    xf = synth.bf16_to_f64(xb)
+    for t in range(T):
+        ref, mag = ol.token(xf[t], idx_o[t], w_o[t])
+        check_close(y[t], ref, mag, what=f"{what} T={T} t={t}")
+    return idx, y
+
+
+@pytest.mark.parametrize("T", [1, 2, 4, 5, 8])
+@pytest.mark.parametrize("shared", [(4, 4, 4), (2, 2, 3), None])
+def test_mix_decode_tiny(T, shared):
+    # 9 experts, k = 4: most columns touch all three gate/up formats
+    lay = SynthLayer(61, 0, 512, 256, 9, 4, mix=MIX9, has_shared=shared is not None,
+                     shared_fmts=shared or (4, 4, 4))
+    check_decode(lay, 61 + T, T, f"mix shared={shared}")
+
+
+def test_mix_decode_two_formats_without_a_third():
+    # routed FP2 and FP3, shared FP3: no slot needs another format's x copy
+    mix = [(2, 3), (3, 3), (2, 2), (3, 2), (2, 3), (3, 3), (2, 3), (3, 2)]
+    lay = SynthLayer(63, 0, 512, 256, 8, 3, mix=mix, shared_fmts=(3, 3, 3))
+    check_decode(lay, 63, 4, "two formats")
+
+
+def test_mix_decode_ragged_shapes():
+    # partial 256-wide chunks in both projections
+    lay = SynthLayer(65, 0, 352, 160, 9, 5, mix=MIX9)
+    check_decode(lay, 65, 3, "ragged mix")
+
+
+def test_mix_columns_are_independent():
+    # decode once, apply to every column: bit for bit the 1-column result
+    lay = SynthLayer(67, 0, 512, 256, 9, 4, mix=MIX9)
+    T = 5
+    L = synth.logits(67, 0, 0, T, lay.E, 0.0)
+    xb = synth.x_bf16(67, 0, T, lay.H)
+    _, y = run_decode(lay, L, xb, T, lay.k)
+    for t in range(T):
+        _, y1 = run_decode(lay, L[t:t + 1], xb[t:t + 1], 1, lay.k)
+        assert np.array_equal(y1[0], y[t]), f"column {t}"
+
+
+@pytest.mark.parametrize("T", [9, 100])
+def test_mix_prefill_tiny(T):
+    lay = SynthLayer(69, 0, 512, 256, 9, 4, mix=MIX9)
+    logits = synth.logits(69, 0, 0, T, 9, 0.0)
+    xb = synth.x_bf16(69, 0, T, 512)
+    full_check(lay, T, logits, xb)
+
+
+@pytest.fixture(scope="module")
+def full_mix_layer():
+    # the full-size layer with a heat-chosen mix (hot experts wider)
+    return SynthLayer(0, 0, 4096, 2048, 256, 6, mix=heat_mix(0, 0, 256, 1.1))
+
+
+@pytest.mark.parametrize("T", [1, 4, 5])
+def test_mix_decode_full_size(full_mix_layer, T):
+    lay = full_mix_layer
+    L = synth.logits(0, 0, 300, T, 256, 1.1)
+    xb = synth.x_bf16(0, 300, T, 4096)
+    idx, y = run_decode(lay, L, xb, T, 6)
+    idx_o, w_o = oracle.router_topk(L, 6)
+    assert np.array_equal(idx, idx_o)
+    fm = {lay.expert_fmts[int(e)][0] for e in idx.ravel()}
+    ol = OracleLayer(lay)
+    xf = synth.bf16_to_f64(xb)
+    for t in range(T):
+        ref, mag = ol.token(xf[t], idx_o[t], w_o[t])
+        check_close(y[t], ref, mag, what=f"full mix T={T} t={t} (gate/up formats {sorted(fm)})")
+
+
+def test_mix_prefill_full_size(full_mix_layer):
+    T = 256
+    logits = synth.logits(0, 0, 500, T, 256, 1.1)
+    xb = synth.x_bf16(0, 500, T, 4096)
+    full_check(full_mix_layer, T, logits, xb, tokens=range(0, T, 37))
+
