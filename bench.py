@@ -371,7 +371,7 @@ PREFILL_TS = (2048, 8192)
 PREFILL_BATCHES = 2
 
 
-def measure_prefill(T: int, steps: int, warmup: int, dev, layer=None):
+def measure_prefill(T: int, steps: int, warmup: int, dev, layer=None, exact=False):
     """Prefill of one full-size layer: T tokens, Zipf(1.1)-skewed top-6 routing,
     each step = router top-k + moe_ffn_prefill (grouping, gather, gate/up
     tcgen05 GEMM + SwiGLU, down tcgen05 GEMM + combine), captured in a graph.
@@ -397,7 +397,7 @@ def measure_prefill(T: int, steps: int, warmup: int, dev, layer=None):
     def step(t):
         b = t % nb
         rfx.moe_router_topk(logits[b], K_TOP, idx[b], w[b], stream)
-        ml.prefill(x[b], idx[b], w[b], y[b], stream)
+        ml.prefill(x[b], idx[b], w[b], y[b], stream, exact=exact)
 
     with torch.cuda.stream(stream):
         for t in range(3):
@@ -413,6 +413,8 @@ def measure_prefill(T: int, steps: int, warmup: int, dev, layer=None):
     # algorithmic work: 2 flops per multiply-add of the real (unpadded) rows;
     # bytes: packed blocks of the touched experts + the shared expert, x and y
     flops = 2.0 * T * (K_TOP + 1) * 3 * H * I
+    # the exact variant's tensor work: gate/up 2 MMAs per product, down 4
+    tflops_work = flops * ((2 * 2 + 4) / 3.0 if exact else 1.0)
     nbytes = []
     for b in range(nb):
         top = np.argsort(-logits_h[b], axis=-1, kind="stable")[:, :K_TOP]
@@ -420,13 +422,15 @@ def measure_prefill(T: int, steps: int, warmup: int, dev, layer=None):
     per_step_bytes = sum(nbytes) / nb
     t_step = ms / steps / 1e3
     peak_tf, peak_gbs = peaks_tensor(), peaks()[0]
-    t_min = max(flops / (peak_tf * 1e12), per_step_bytes / (peak_gbs * 1e9))
-    return {"T": T, "ms_per_step": ms / steps, "value": T / t_step, "unit": "tokens/s",
-            "tflops": flops / t_step / 1e12, "flops_per_step": flops, "bytes_per_step": per_step_bytes,
-            "roofline": {"bound": "tensor" if flops / (peak_tf * 1e12) >= per_step_bytes / (peak_gbs * 1e9)
+    t_min = max(tflops_work / (peak_tf * 1e12), per_step_bytes / (peak_gbs * 1e9))
+    return {"T": T, "precision": "exact (bf16 hi/lo weights, h1 + h2)" if exact else "bf16 operands",
+            "ms_per_step": ms / steps, "value": T / t_step, "unit": "tokens/s",
+            "tflops": flops / t_step / 1e12, "flops_per_step": flops, "tensor_flops_per_step": tflops_work,
+            "bytes_per_step": per_step_bytes,
+            "roofline": {"bound": "tensor" if tflops_work / (peak_tf * 1e12) >= per_step_bytes / (peak_gbs * 1e9)
                          else "hbm", "peak_tflops": peak_tf, "peak_gbs": peak_gbs, "t_min_ms": t_min * 1e3,
                          "frac": t_min / t_step, "peak_kind": "bf16_tflops_sustained of measured",
-                         "traffic": traffic("prefill", f"T{T}", per_step_bytes)},
+                         "traffic": None if exact else traffic("prefill", f"T{T}", per_step_bytes)},
             "device_status": st, "steps": steps}
 
 
@@ -733,6 +737,7 @@ def main():
     pf = None
     if not args.no_prefill:
         pf = [measure_prefill(T, args.prefill_steps, max(3, args.warmup), dev) for T in PREFILL_TS]
+        pf.append(measure_prefill(2048, args.prefill_steps, max(3, args.warmup), dev, exact=True))
     stack = None
     if not args.no_stack:
         import gc

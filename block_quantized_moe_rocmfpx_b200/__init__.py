@@ -77,11 +77,14 @@ _stack = _proto("moe_stack_forward", _i32, [_vp, _i32, _vp, _vp, _i32, _vp, _vp,
 _pf_ws_bytes = _proto("moe_prefill_workspace_bytes", _sz, [_vp, _i32])
 _debug_fault = _proto("rfx_debug_set_fault", _i32, [_i32, ctypes.c_longlong])
 _prefill = _proto("moe_ffn_prefill", _i32, [_vp, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp])
+_pf_ws_bytes_ex = _proto("moe_prefill_workspace_bytes_ex", _sz, [_vp, _i32, _i32])
+_prefill_ex = _proto("moe_ffn_prefill_ex", _i32, [_vp, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _i32, _vp])
+RFX_PREFILL_BF16, RFX_PREFILL_EXACT = 0, 1
 
 
 class moe_prefill_ws_view(ctypes.Structure):
     _fields_ = [("counts", _vp), ("row_token", _vp), ("row_weight", _vp), ("h", _vp),
-                ("routed_rows", _i64), ("h_rows", _i64)]
+                ("routed_rows", _i64), ("h_rows", _i64), ("h_lo", _vp)]
 
 
 _pf_view = _proto("moe_prefill_view", _i32, [_vp, _i32, _vp, ctypes.POINTER(moe_prefill_ws_view)])
@@ -90,6 +93,7 @@ EXPORTED = ["rfx_last_error", "rfx_packed_bytes", "rfx_pack", "rfx_unpack", "rfx
             "rfx_gemv_q", "moe_layer_create", "moe_layer_create_mix", "moe_layer_destroy", "moe_ffn_workspace_bytes", "rfx_ws_init",
             "rfx_ws_status", "moe_ffn_forward", "moe_ffn_forward_static", "moe_rms_norm_bf16",
             "moe_stack_workspace_bytes", "moe_stack_forward", "moe_prefill_workspace_bytes", "moe_ffn_prefill",
+            "moe_prefill_workspace_bytes_ex", "moe_ffn_prefill_ex",
             "moe_prefill_view", "moe_router_logits", "moe_router_project_topk",
             "moe_ffn_host_scratch_bytes", "moe_ffn_forward_host", "rfx_debug_set_fault"]
 
@@ -281,6 +285,16 @@ def moe_ffn_prefill(handle: int, x, T: int, idx, w, y, ws, stream=None):
                     _stream(stream)))
 
 
+def moe_prefill_workspace_bytes_ex(handle: int, T: int, precision: int) -> int:
+    return int(_pf_ws_bytes_ex(handle, T, precision))
+
+
+def moe_ffn_prefill_ex(handle: int, x, T: int, idx, w, y, ws, precision: int, stream=None):
+    """moe_ffn_prefill at a chosen precision (RFX_PREFILL_BF16 or RFX_PREFILL_EXACT)."""
+    _check(_prefill_ex(handle, _ptr(x), T, _ptr(idx), _ptr(w), _ptr(y), _ptr(ws), ws.numel() * ws.element_size(),
+                       precision, _stream(stream)))
+
+
 def moe_prefill_view(handle: int, T: int, ws, I: int, E: int):
     """Tensors viewing a prefill workspace after a call: counts int32 [E], row_token
     int32 [T*k], row_weight fp32 [T*k], h bf16 bits int16 [T*k + T][I]."""
@@ -296,7 +310,9 @@ def moe_prefill_view(handle: int, T: int, ws, I: int, E: int):
     rr, hr = int(v.routed_rows), int(v.h_rows)
     return {"counts": sub(v.counts, 4 * E, torch.int32), "row_token": sub(v.row_token, 4 * rr, torch.int32),
             "row_weight": sub(v.row_weight, 4 * rr, torch.float32),
-            "h": sub(v.h, 2 * hr * I, torch.int16).view(hr, I)}
+            "h": sub(v.h, 2 * hr * I, torch.int16).view(hr, I),
+            "h_lo": sub(v.h_lo, 2 * hr * I, torch.int16).view(hr, I) if int(v.h_lo) + 2 * hr * I <= base + ws.numel()
+            else None}
 
 
 # --------------------------------------------------------- convenience ---
@@ -355,17 +371,22 @@ class MoeLayer:
         """Device flag of the host-call scratch (its workspace comes first)."""
         return rfx_ws_status(self.host_scratch, stream)
 
-    def prefill(self, x, idx, w, y, stream=None):
-        """moe_ffn_prefill with a workspace kept on the layer (grown on demand)."""
+    def prefill(self, x, idx, w, y, stream=None, exact=False):
+        """moe_ffn_prefill (exact: moe_ffn_prefill_ex at RFX_PREFILL_EXACT) with a
+        workspace kept on the layer (grown on demand)."""
         import torch
         T = x.shape[0]
-        nbytes = moe_prefill_workspace_bytes(self.handle, T)
+        prec = RFX_PREFILL_EXACT if exact else RFX_PREFILL_BF16
+        nbytes = moe_prefill_workspace_bytes_ex(self.handle, T, prec)
         if nbytes == 0:
             raise RfxError(-2, f"prefill unsupported for T={T}, H={self.H}, I={self.I}")
         if getattr(self, "pf_ws", None) is None or self.pf_ws.numel() < nbytes:
             self.pf_ws = torch.empty(nbytes, dtype=torch.uint8, device=x.device)
             rfx_ws_init(self.pf_ws)
-        moe_ffn_prefill(self.handle, x, T, idx, w, y, self.pf_ws, stream)
+        if exact:
+            moe_ffn_prefill_ex(self.handle, x, T, idx, w, y, self.pf_ws, prec, stream)
+        else:
+            moe_ffn_prefill(self.handle, x, T, idx, w, y, self.pf_ws, stream)
 
     def prefill_view(self, T: int):
         return moe_prefill_view(self.handle, T, self.pf_ws, self.I, self.E)

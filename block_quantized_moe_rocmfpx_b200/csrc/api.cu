@@ -6,6 +6,7 @@
 #include <algorithm>
 #include <atomic>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <string>
 #include <vector>
@@ -23,6 +24,13 @@ struct moe_layer {
     moe_layer_desc d;
     rfx::MoeMixEntry* mix_dev = nullptr;   // ROCmFPX MIX: device table [E], else null
     int mix_count[5] = {0, 0, 0, 0, 0};    // routed experts per gate/up format (MIX)
+    // moe_ffn_forward_host: the uploads run on a stream of their own into two
+    // buffer sets used in turn, so that a call's uploads overlap the previous
+    // call's kernels (made on first use; calls on one layer are serialised)
+    std::mutex host_mu;
+    cudaStream_t up_stream = nullptr;
+    cudaEvent_t ev_free[2] = {nullptr, nullptr}, ev_ready[2] = {nullptr, nullptr};
+    unsigned host_calls = 0;
 };
 
 namespace {
@@ -208,7 +216,13 @@ extern "C" int moe_layer_create_mix(const moe_layer_desc* d, const moe_expert_mi
 }
 
 extern "C" void moe_layer_destroy(moe_layer* layer) {
-    if (layer && layer->mix_dev) cudaFree(layer->mix_dev);
+    if (!layer) return;
+    if (layer->mix_dev) cudaFree(layer->mix_dev);
+    for (int i = 0; i < 2; ++i) {
+        if (layer->ev_free[i]) cudaEventDestroy(layer->ev_free[i]);
+        if (layer->ev_ready[i]) cudaEventDestroy(layer->ev_ready[i]);
+    }
+    if (layer->up_stream) cudaStreamDestroy(layer->up_stream);
     delete layer;
 }
 
@@ -406,22 +420,36 @@ extern "C" int moe_ffn_forward(const moe_layer* layer, const void* x, int T, con
 namespace {
 
 // Host-call scratch: the moe_ffn_forward workspace first (so rfx_ws_status
-// reads its error flag at offset 0), then the device copies and the routing.
+// reads its error flag at offset 0), then two sets of device copies of x and
+// the logits (used in turn), the routing and y.
 struct HostScratch {
-    size_t ffn, x, logits, idx, w, y, total;
+    size_t ffn, x[2], logits[2], idx, w, y, total;
 };
 
 HostScratch host_scratch_layout(const moe_layer_desc& d, int T, size_t ffn_bytes) {
     auto up = [](size_t n) { return (n + 255) / 256 * 256; };
     HostScratch S;
     S.ffn = 0;
-    S.x = up(ffn_bytes);
-    S.logits = S.x + up((size_t)T * d.H * 2);
-    S.idx = S.logits + up((size_t)T * d.E * 4);
+    S.x[0] = up(ffn_bytes);
+    S.x[1] = S.x[0] + up((size_t)T * d.H * 2);
+    S.logits[0] = S.x[1] + up((size_t)T * d.H * 2);
+    S.logits[1] = S.logits[0] + up((size_t)T * d.E * 4);
+    S.idx = S.logits[1] + up((size_t)T * d.E * 4);
     S.w = S.idx + up((size_t)T * d.k * 4);
     S.y = S.w + up((size_t)T * d.k * 4);
     S.total = S.y + up((size_t)T * d.H * 4);
     return S;
+}
+
+// The upload stream and events of a layer, made on first use.
+cudaError_t host_streams(moe_layer* L) {
+    if (L->up_stream) return cudaSuccess;
+    cudaError_t e = cudaStreamCreateWithFlags(&L->up_stream, cudaStreamNonBlocking);
+    for (int i = 0; i < 2 && e == cudaSuccess; ++i) {
+        e = cudaEventCreateWithFlags(&L->ev_free[i], cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&L->ev_ready[i], cudaEventDisableTiming);
+    }
+    return e;
 }
 
 }  // namespace
@@ -447,20 +475,40 @@ extern "C" int moe_ffn_forward_host(const moe_layer* layer, const void* x, const
     if (scratch_bytes < S.total)
         return rfx_fail(RFX_EINVAL, "moe_ffn_forward_host: scratch smaller than moe_ffn_host_scratch_bytes");
     uint8_t* b = (uint8_t*)scratch;
-    void* xd = b + S.x;
-    float* ld = (float*)(b + S.logits);
     int32_t* idx = (int32_t*)(b + S.idx);
     float* w = (float*)(b + S.w);
     float* yd = (float*)(b + S.y);
     cudaStream_t st = (cudaStream_t)stream;
-    cudaError_t e = cudaMemcpyAsync(xd, x, (size_t)T * d.H * 2, cudaMemcpyHostToDevice, st);
+    moe_layer* L = const_cast<moe_layer*>(layer);
+    std::lock_guard<std::mutex> lock(L->host_mu);
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(st, &cap);
     if (e != cudaSuccess) return cuda_fail("moe_ffn_forward_host", e);
-    e = cudaMemcpyAsync(ld, logits, (size_t)T * d.E * 4, cudaMemcpyHostToDevice, st);
+    const bool side = cap == cudaStreamCaptureStatusNone;   // a graph capture keeps everything on `stream`
+    if (side) {
+        e = host_streams(L);
+        if (e != cudaSuccess) return cuda_fail("moe_ffn_forward_host", e);
+    }
+    const int s = side ? (int)(L->host_calls++ & 1u) : 0;
+    void* xd = b + S.x[s];
+    float* ld = (float*)(b + S.logits[s]);
+    // uploads: on the side stream once the kernels of the call that used this
+    // buffer set two calls ago have read it; `stream` waits for them
+    cudaStream_t us = side ? L->up_stream : st;
+    if (side) e = cudaStreamWaitEvent(us, L->ev_free[s], 0);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(xd, x, (size_t)T * d.H * 2, cudaMemcpyHostToDevice, us);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(ld, logits, (size_t)T * d.E * 4, cudaMemcpyHostToDevice, us);
+    if (side && e == cudaSuccess) e = cudaEventRecord(L->ev_ready[s], us);
+    if (side && e == cudaSuccess) e = cudaStreamWaitEvent(st, L->ev_ready[s], 0);
     if (e != cudaSuccess) return cuda_fail("moe_ffn_forward_host", e);
     int rc = moe_router_topk(ld, T, d.E, d.k, idx, w, stream);
     if (rc != RFX_OK) return rc;
-    rc = moe_ffn_forward(layer, xd, T, idx, w, yd, b + S.ffn, S.x, stream);
+    rc = moe_ffn_forward(layer, xd, T, idx, w, yd, b + S.ffn, S.x[0], stream);
     if (rc != RFX_OK) return rc;
+    if (side) {
+        e = cudaEventRecord(L->ev_free[s], st);
+        if (e != cudaSuccess) return cuda_fail("moe_ffn_forward_host", e);
+    }
     e = cudaMemcpyAsync(y, yd, (size_t)T * d.H * 4, cudaMemcpyDeviceToHost, st);
     return e == cudaSuccess ? RFX_OK : cuda_fail("moe_ffn_forward_host", e);
 }
@@ -480,33 +528,32 @@ int prefill_check(const moe_layer* layer, int T, const char* who) {
     return RFX_OK;
 }
 
-rfx::PfWs prefill_layout(const moe_layer* layer, int T) {
+rfx::PfWs prefill_layout(const moe_layer* layer, int T, bool exact = false) {
     const moe_layer_desc& d = layer->d;
-    return rfx::pf_ws_layout(T, d.k, d.E, d.H, d.I);
+    return rfx::pf_ws_layout(T, d.k, d.E, d.H, d.I, exact ? 2 : 1);
 }
 
-}  // namespace
-
-extern "C" size_t moe_prefill_workspace_bytes(const moe_layer* layer, int T) {
+size_t prefill_ws_bytes(const moe_layer* layer, int T, bool exact) {
     if (!layer || T < 1 || T > PF_MAX_T || layer->d.H % 256 || layer->d.I % 256) return 0;
-    return prefill_layout(layer, T).total;
+    return prefill_layout(layer, T, exact).total;
 }
 
-extern "C" int moe_ffn_prefill(const moe_layer* layer, const void* x, int T, const int32_t* idx, const float* w,
-                               float* y, void* ws, size_t ws_bytes, void* stream) {
+int prefill_impl(const moe_layer* layer, const void* x, int T, const int32_t* idx, const float* w, float* y, void* ws,
+                 size_t ws_bytes, bool exact, void* stream, const char* who) {
     if (layer && T == 0) return RFX_OK;   // no tokens: nothing to do
-    int rc = prefill_check(layer, T, "moe_ffn_prefill");
+    int rc = prefill_check(layer, T, who);
     if (rc != RFX_OK) return rc;
-    if (!x || !idx || !w || !y || !ws) return rfx_fail(RFX_EINVAL, "moe_ffn_prefill: null pointer");
+    const std::string W(who);
+    if (!x || !idx || !w || !y || !ws) return rfx_fail(RFX_EINVAL, W + ": null pointer");
     if (!aligned16(x) || !aligned16(y) || ((uintptr_t)ws & 255u))
-        return rfx_fail(RFX_EINVAL, "moe_ffn_prefill: x and y must be 16-byte and ws 256-byte aligned");
-    const rfx::PfWs L = prefill_layout(layer, T);
-    if (ws_bytes < L.total) return rfx_fail(RFX_EINVAL, "moe_ffn_prefill: workspace smaller than moe_prefill_workspace_bytes");
+        return rfx_fail(RFX_EINVAL, W + ": x and y must be 16-byte and ws 256-byte aligned");
+    const rfx::PfWs L = prefill_layout(layer, T, exact);
+    if (ws_bytes < L.total) return rfx_fail(RFX_EINVAL, W + ": workspace smaller than its size function gives");
     int sms = 0, smem_optin = 0;
     rc = device_props(sms, smem_optin);
     if (rc != RFX_OK) return rc;
-    if (std::max(rfx::pf_gemm_smem_bytes(0), rfx::pf_gemm_smem_bytes(1)) > (size_t)smem_optin)
-        return rfx_fail(RFX_EUNSUPPORTED, "moe_ffn_prefill: the device has too little shared memory per block");
+    if (std::max(rfx::pf_gemm_smem_bytes(0, exact), rfx::pf_gemm_smem_bytes(1, exact)) > (size_t)smem_optin)
+        return rfx_fail(RFX_EUNSUPPORTED, W + ": the device has too little shared memory per block");
     const moe_layer_desc& d = layer->d;
     rfx::PfParams p{};
     p.H = d.H; p.I = d.I; p.E = d.E; p.k = d.k; p.T = T;
@@ -530,11 +577,36 @@ extern "C" int moe_ffn_prefill(const moe_layer* layer, const void* x, int T, con
     p.xp = (uint16_t*)(b + L.xp);
     p.hp = (uint16_t*)(b + L.hp);
     p.max_tiles = L.max_tiles;
+    p.exact = exact ? 1 : 0;
     p.wait_limit = rfx::debug_wait(rfx::pf_default_wait_limit());
     p.fault = rfx::debug_fault() == 3 ? 3 : 0;
     cudaError_t e = rfx::pf_launch(p, sms, (cudaStream_t)stream);
-    if (e == cudaErrorInvalidValue) return rfx_fail(RFX_ECUDA, "moe_ffn_prefill: tensor-map encoding failed");
-    return e == cudaSuccess ? RFX_OK : cuda_fail("moe_ffn_prefill", e);
+    if (e == cudaErrorInvalidValue) return rfx_fail(RFX_ECUDA, W + ": tensor-map encoding failed");
+    return e == cudaSuccess ? RFX_OK : cuda_fail(who, e);
+}
+
+}  // namespace
+
+extern "C" size_t moe_prefill_workspace_bytes(const moe_layer* layer, int T) {
+    return prefill_ws_bytes(layer, T, false);
+}
+
+extern "C" int moe_ffn_prefill(const moe_layer* layer, const void* x, int T, const int32_t* idx, const float* w,
+                               float* y, void* ws, size_t ws_bytes, void* stream) {
+    return prefill_impl(layer, x, T, idx, w, y, ws, ws_bytes, false, stream, "moe_ffn_prefill");
+}
+
+extern "C" size_t moe_prefill_workspace_bytes_ex(const moe_layer* layer, int T, int precision) {
+    if (precision != RFX_PREFILL_BF16 && precision != RFX_PREFILL_EXACT) return 0;
+    return prefill_ws_bytes(layer, T, precision == RFX_PREFILL_EXACT);
+}
+
+extern "C" int moe_ffn_prefill_ex(const moe_layer* layer, const void* x, int T, const int32_t* idx, const float* w,
+                                  float* y, void* ws, size_t ws_bytes, int precision, void* stream) {
+    if (precision != RFX_PREFILL_BF16 && precision != RFX_PREFILL_EXACT)
+        return rfx_fail(RFX_EINVAL, "moe_ffn_prefill_ex: unknown precision");
+    return prefill_impl(layer, x, T, idx, w, y, ws, ws_bytes, precision == RFX_PREFILL_EXACT, stream,
+                        "moe_ffn_prefill_ex");
 }
 
 extern "C" int moe_prefill_view(const moe_layer* layer, int T, const void* ws, moe_prefill_ws_view* v) {
@@ -549,6 +621,7 @@ extern "C" int moe_prefill_view(const moe_layer* layer, int T, const void* ws, m
     v->h = b + L.hp;
     v->routed_rows = (int64_t)T * layer->d.k;
     v->h_rows = (int64_t)T * layer->d.k + T;
+    v->h_lo = b + L.hp + (size_t)v->h_rows * layer->d.I * 2;
     return RFX_OK;
 }
 

@@ -3,15 +3,18 @@
 // The mat-vec with in-kernel block dequantisation (taozi.news, "DeepSeek V4
 // Flash 在 128GB 锐龙 AI MAX+ 上跑到 32 tok/s", section "ROCmFPX：把 284B 权重压进
 // 128 GB"), each block decoded once for all q columns (ainomam.com, "APU 实现
-// token 自由…", section "Lucebox 的优化三板斧").  A CTA owns 32 output rows
-// (2 row-groups) and its 8 warps split K in quarters; packed chunks are read
-// straight from global memory with 128-bit loads.  x is staged once per CTA
+// token 自由…", section "Lucebox 的优化三板斧").  A persistent CTA takes 32
+// output rows (2 row-groups) at a time and its 8 warps split K in quarters;
+// packed chunks are read straight from global memory with 128-bit loads.  x
+// is staged once per CTA
 // in shared memory as fp16 in B-fragment order: each column scaled by a power
 // of two that puts max|x| in [2^13, 2^14) and each tile by 2^-s_b for the
 // format's bit offsets (see rfx_tile.cuh); fp32 x becomes an exact-to-2^-22
 // hi/lo pair of virtual columns.  K-quarter partials are summed in a fixed
 // order.
 #include <cuda_runtime.h>
+
+#include <algorithm>
 
 #include "gemv.h"
 #include "launch_util.h"
@@ -45,12 +48,16 @@ __global__ void __launch_bounds__(GEMV_WARPS * 32) gemv_kernel(GemvParams p) {
     if (threadIdx.x < 8) xmax[threadIdx.x] = 0u;
     __syncthreads();
     const long long n = (long long)p.q * K;
-    for (long long i = threadIdx.x; i < n; i += blockDim.x) {
-        const int c = (int)(i / K);
+    // max |x| per column: K is a multiple of 32, so a warp's 32 consecutive
+    // elements lie in one column (one shared atomic per warp and step)
+    for (long long i0 = threadIdx.x - lane; i0 < n; i0 += blockDim.x) {
+        const long long i = i0 + lane;
+        const int c = (int)(i0 / K);
         float v;
         if constexpr (F32X) v = ((const float*)p.x)[i];
         else v = __uint_as_float((uint32_t)((const uint16_t*)p.x)[i] << 16);
-        atomicMax(&xmax[c], __float_as_uint(fabsf(v)));
+        const uint32_t m = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(v)));
+        if (lane == 0 && m) atomicMax(&xmax[c], m);
     }
     __syncthreads();
     if (threadIdx.x < p.q) {
@@ -101,121 +108,129 @@ __global__ void __launch_bounds__(GEMV_WARPS * 32) gemv_kernel(GemvParams p) {
         const int v = 8 * nb + g;
         bs[nb] = {xs + (v * 4 + t) * 8, vstride, v < nv};
     }
-    const int rg = 2 * blockIdx.x + (w & 1);
     const int nch = rfx_num_chunks(p.K);
     const int kq = w >> 1;
     const int c0 = kq * nch / 4, c1 = (kq + 1) * nch / 4;
-    const uint8_t* Wrg = p.W + (long long)rg * rfx_rowgroup_bytes(FMT, p.K);
     const int fullb = (int)rfx_chunk_bytes(FMT, 8);
-    float acc[NB][4], corr[NB][4];
+    const long long rgb = rfx_rowgroup_bytes(FMT, p.K);
+    const long long npairs = ((p.N + 15) / 16 + 1) / 2;
+    // persistent: x is staged once per CTA, then the CTA takes row-group pairs
+    // blockIdx.x, blockIdx.x + gridDim.x, ...
+    for (long long pr = blockIdx.x; pr < npairs; pr += gridDim.x) {
+        const long long rg = 2 * pr + (w & 1);
+        const uint8_t* Wrg = p.W + rg * rgb;
+        float acc[NB][4], corr[NB][4];
 #pragma unroll
-    for (int nb = 0; nb < NB; ++nb)
+        for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) { acc[nb][i] = 0.f; corr[nb][i] = 0.f; }
-    const bool live = (long long)rg * 16 < p.N;
-    // block-sum rows of the lane's two virtual columns per n-block (for fp32 x
-    // the hi and lo halves each carry their own sum; the corrections add up)
-    const float* srow[NB][2];
+            for (int i = 0; i < 4; ++i) { acc[nb][i] = 0.f; corr[nb][i] = 0.f; }
+        const bool live = rg * 16 < p.N;
+        // block-sum rows of the lane's two virtual columns per n-block (for fp32 x
+        // the hi and lo halves each carry their own sum; the corrections add up)
+        const float* srow[NB][2];
 #pragma unroll
-    for (int nb = 0; nb < NB; ++nb)
+        for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            const int v = 8 * nb + 2 * t + j;
-            srow[nb][j] = v < nv ? sx + v * kbs : nullptr;
-        }
-    if (live) {
-        for (int c = c0; c < c1; ++c) {
-            const uint8_t* st = Wrg + (long long)c * fullb;
-            const int nt = rfx_chunk_tiles(p.K, c);
-            const int step0 = 16 * c;
-            if (nt == 8) {
-                FullChunk<FMT> f;
-                f.load(st, lane, g);
+            for (int j = 0; j < 2; ++j) {
+                const int v = 8 * nb + 2 * t + j;
+                srow[nb][j] = v < nv ? sx + v * kbs : nullptr;
+            }
+        if (live) {
+            for (int c = c0; c < c1; ++c) {
+                const uint8_t* st = Wrg + (long long)c * fullb;
+                const int nt = rfx_chunk_tiles(p.K, c);
+                const int step0 = 16 * c;
+                if (nt == 8) {
+                    FullChunk<FMT> f;
+                    f.load(st, lane, g);
 #pragma unroll
-                for (int b = 0; b < 8; ++b) {
-                    uint32_t a[8];
-                    switch (b) {
-                        case 0: plane_regs<FMT, 0>(f.wd, f.sh, a); break;
-                        case 1: plane_regs<FMT, 1>(f.wd, f.sh, a); break;
-                        case 2: plane_regs<FMT, 2>(f.wd, f.sh, a); break;
-                        case 3: plane_regs<FMT, 3>(f.wd, f.sh, a); break;
-                        case 4: plane_regs<FMT, 4>(f.wd, f.sh, a); break;
-                        case 5: plane_regs<FMT, 5>(f.wd, f.sh, a); break;
-                        case 6: plane_regs<FMT, 6>(f.wd, f.sh, a); break;
-                        default: plane_regs<FMT, 7>(f.wd, f.sh, a); break;
-                    }
-                    float s0, s1;
-                    f.scales(b, s0, s1);
+                    for (int b = 0; b < 8; ++b) {
+                        uint32_t a[8];
+                        switch (b) {
+                            case 0: plane_regs<FMT, 0>(f.wd, f.sh, a); break;
+                            case 1: plane_regs<FMT, 1>(f.wd, f.sh, a); break;
+                            case 2: plane_regs<FMT, 2>(f.wd, f.sh, a); break;
+                            case 3: plane_regs<FMT, 3>(f.wd, f.sh, a); break;
+                            case 4: plane_regs<FMT, 4>(f.wd, f.sh, a); break;
+                            case 5: plane_regs<FMT, 5>(f.wd, f.sh, a); break;
+                            case 6: plane_regs<FMT, 6>(f.wd, f.sh, a); break;
+                            default: plane_regs<FMT, 7>(f.wd, f.sh, a); break;
+                        }
+                        float s0, s1;
+                        f.scales(b, s0, s1);
 #pragma unroll
-                    for (int nb = 0; nb < NB; ++nb) {
-                        float cc[4];
-                        mma_tile(cc, a, bs[nb].get(step0 + 2 * b), bs[nb].get(step0 + 2 * b + 1));
-                        acc[nb][0] = fmaf(s0, cc[0], acc[nb][0]);
-                        acc[nb][1] = fmaf(s0, cc[1], acc[nb][1]);
-                        acc[nb][2] = fmaf(s1, cc[2], acc[nb][2]);
-                        acc[nb][3] = fmaf(s1, cc[3], acc[nb][3]);
+                        for (int nb = 0; nb < NB; ++nb) {
+                            float cc[4];
+                            mma_tile(cc, a, bs[nb].get(step0 + 2 * b), bs[nb].get(step0 + 2 * b + 1));
+                            acc[nb][0] = fmaf(s0, cc[0], acc[nb][0]);
+                            acc[nb][1] = fmaf(s0, cc[1], acc[nb][1]);
+                            acc[nb][2] = fmaf(s1, cc[2], acc[nb][2]);
+                            acc[nb][3] = fmaf(s1, cc[3], acc[nb][3]);
 #pragma unroll
-                        for (int j = 0; j < 2; ++j) {
-                            if (srow[nb][j]) {
-                                const float sb = srow[nb][j][8 * c + b];
-                                corr[nb][j] = fmaf(s0, sb, corr[nb][j]);
-                                corr[nb][2 + j] = fmaf(s1, sb, corr[nb][2 + j]);
+                            for (int j = 0; j < 2; ++j) {
+                                if (srow[nb][j]) {
+                                    const float sb = srow[nb][j][8 * c + b];
+                                    corr[nb][j] = fmaf(s0, sb, corr[nb][j]);
+                                    corr[nb][2 + j] = fmaf(s1, sb, corr[nb][2 + j]);
+                                }
                             }
                         }
                     }
-                }
-            } else {
-                for (int b = 0; b < nt; ++b) {
-                    uint32_t a[8];
-                    float s0, s1;
-                    partial_tile<FMT>(st, nt, lane, g, b, a, s0, s1);
+                } else {
+                    for (int b = 0; b < nt; ++b) {
+                        uint32_t a[8];
+                        float s0, s1;
+                        partial_tile<FMT>(st, nt, lane, g, b, a, s0, s1);
 #pragma unroll
-                    for (int nb = 0; nb < NB; ++nb) {
-                        float cc[4];
-                        mma_tile(cc, a, bs[nb].get(step0 + 2 * b), bs[nb].get(step0 + 2 * b + 1));
-                        // the exact level dot product in units of 2^-24 (scale untouched: it may be 2^-127)
-                        acc[nb][0] = fmaf(s0, cc[0] * 0x1.0p-24f, acc[nb][0]);
-                        acc[nb][1] = fmaf(s0, cc[1] * 0x1.0p-24f, acc[nb][1]);
-                        acc[nb][2] = fmaf(s1, cc[2] * 0x1.0p-24f, acc[nb][2]);
-                        acc[nb][3] = fmaf(s1, cc[3] * 0x1.0p-24f, acc[nb][3]);
+                        for (int nb = 0; nb < NB; ++nb) {
+                            float cc[4];
+                            mma_tile(cc, a, bs[nb].get(step0 + 2 * b), bs[nb].get(step0 + 2 * b + 1));
+                            // the exact level dot product in units of 2^-24 (scale untouched: it may be 2^-127)
+                            acc[nb][0] = fmaf(s0, cc[0] * 0x1.0p-24f, acc[nb][0]);
+                            acc[nb][1] = fmaf(s0, cc[1] * 0x1.0p-24f, acc[nb][1]);
+                            acc[nb][2] = fmaf(s1, cc[2] * 0x1.0p-24f, acc[nb][2]);
+                            acc[nb][3] = fmaf(s1, cc[3] * 0x1.0p-24f, acc[nb][3]);
+                        }
                     }
                 }
             }
         }
-    }
-    float* my = red + (w * 32 + lane) * 8;
+        float* my = red + (w * 32 + lane) * 8;
 #pragma unroll
-    for (int nb = 0; nb < NB; ++nb)
+        for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) my[4 * nb + i] = fmaf(-Plane<FMT>::OFF, corr[nb][i], acc[nb][i] * 0x1.0p24f);
-    __syncthreads();
-    if (w >= 2 || !live) return;
-    float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            for (int i = 0; i < 4; ++i) my[4 * nb + i] = fmaf(-Plane<FMT>::OFF, corr[nb][i], acc[nb][i] * 0x1.0p24f);
+        __syncthreads();
+        if (w < 2 && live) {
+            float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4) {
-        const float* r = red + ((2 * q4 + w) * 32 + lane) * 8;
+            for (int q4 = 0; q4 < 4; ++q4) {
+                const float* r = red + ((2 * q4 + w) * 32 + lane) * 8;
 #pragma unroll
-        for (int i = 0; i < 4 * NB; ++i) s[i] += r[i];
-    }
-    const long long row0 = (long long)rg * 16 + g, row1 = row0 + 8;
-#pragma unroll
-    for (int nb = 0; nb < NB; ++nb) {
-        if constexpr (!F32X) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int col = 8 * nb + 2 * t + (i & 1);
-                const long long row = (i >> 1) ? row1 : row0;
-                if (col < p.q && row < p.N)
-                    p.y[(long long)col * p.N + row] = s[4 * nb + i] * __int_as_float((127 - xn[col]) << 23);
+                for (int i = 0; i < 4 * NB; ++i) s[i] += r[i];
             }
-        } else {
-            const int col = 4 * nb + t;
-            if (col < p.q) {
-                const float sc = __int_as_float((127 - xn[col]) << 23);
-                if (row0 < p.N) p.y[(long long)col * p.N + row0] = (s[4 * nb + 0] + s[4 * nb + 1]) * sc;
-                if (row1 < p.N) p.y[(long long)col * p.N + row1] = (s[4 * nb + 2] + s[4 * nb + 3]) * sc;
+            const long long row0 = rg * 16 + g, row1 = row0 + 8;
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb) {
+                if constexpr (!F32X) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int col = 8 * nb + 2 * t + (i & 1);
+                        const long long row = (i >> 1) ? row1 : row0;
+                        if (col < p.q && row < p.N)
+                            p.y[(long long)col * p.N + row] = s[4 * nb + i] * __int_as_float((127 - xn[col]) << 23);
+                    }
+                } else {
+                    const int col = 4 * nb + t;
+                    if (col < p.q) {
+                        const float sc = __int_as_float((127 - xn[col]) << 23);
+                        if (row0 < p.N) p.y[(long long)col * p.N + row0] = (s[4 * nb + 0] + s[4 * nb + 1]) * sc;
+                        if (row1 < p.N) p.y[(long long)col * p.N + row1] = (s[4 * nb + 2] + s[4 * nb + 3]) * sc;
+                    }
+                }
             }
         }
+        __syncthreads();   // the reduction buffer is reused by the next pair
     }
 }
 
@@ -233,8 +248,16 @@ static cudaError_t launch_t(const GemvParams& p, size_t smem, cudaStream_t strea
     static SmemLimit limit;   // one per instantiation
     cudaError_t e = limit.ensure((const void*)kern, (int)smem);
     if (e != cudaSuccess) return e;
-    const long long ngroups = (p.N + 15) / 16;
-    const int grid = (int)((ngroups + 1) / 2);
+    // persistent grid: as many CTAs as are resident at once (x is staged once
+    // per CTA), never more than there are row-group pairs
+    int dev = 0, sms = 0, per_sm = 0;
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, GEMV_WARPS * 32, smem);
+    if (e != cudaSuccess) return e;
+    const long long npairs = ((p.N + 15) / 16 + 1) / 2;
+    const int grid = (int)std::min<long long>(npairs, (long long)sms * std::max(per_sm, 1));
     kern<<<grid, GEMV_WARPS * 32, smem, stream>>>(p);
     return cudaGetLastError();
 }

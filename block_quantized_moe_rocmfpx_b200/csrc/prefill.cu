@@ -50,18 +50,28 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr int CB_MAX = 128 * 17;   // bytes of the largest full chunk (FP4)
 constexpr int PF_BOX_ROWS = 64;    // token rows per TMA box (the B stage holds 256)
 
-template <int MODE>
+// EX (exact precision): every dequantised weight is the bf16 pair hi + lo
+// (hi = bf16(w), lo = bf16(w - hi): w = level * scale has at most 15
+// significant bits, so the pair is exact), and the SwiGLU output is the bf16
+// pair h1 + h2 (16 bits).  Gate/up: 2 MMAs per k-step and matrix; down: 4
+// (hi h1, hi h2, lo h1, lo h2).  A stage holds the hi tiles of every matrix,
+// then the lo tiles; MODE 1 stages hold the h1 rows, then the h2 rows.
+template <int MODE, bool EX = false>
 struct PfCfg {
     static constexpr int NMAT = MODE == 0 ? 2 : 1;                 // gate + up, or down
+    static constexpr int NPART = EX ? 2 : 1;                        // weight tiles per matrix (hi, lo)
+    static constexpr int BPART = (EX && MODE == 1) ? 2 : 1;         // token-row tiles per stage (h1, h2)
     // MODE 0: two dequantisation warps per 16-row group (gate, up); MODE 1: one
     static constexpr int N_DQ = MODE == 0 ? 16 : 8;
     static constexpr int W_EPI0 = W_DQ0 + N_DQ;
     static constexpr int THREADS = 32 * (W_EPI0 + N_EPI);
     static constexpr int UQ_READERS = 2 + N_DQ + N_EPI;           // MMA issuers, dequantisation and epilogue warps
     static constexpr int A_MAT = PF_BM * PF_BK * 2;                // 16 KB bf16 per matrix
-    static constexpr int A_BYTES = NMAT * A_MAT;
-    static constexpr int B_BYTES = PF_TILE_N * PF_BK * 2;          // 32 KB bf16
-    static constexpr int NS = MODE == 0 ? 3 : 4;                    // stages of (dequantised A, token-row B)
+    static constexpr int LO_OFF = NMAT * A_MAT;                     // the lo tiles after the hi tiles
+    static constexpr int A_BYTES = NPART * NMAT * A_MAT;
+    static constexpr int B_TILE = PF_TILE_N * PF_BK * 2;            // 32 KB bf16
+    static constexpr int B_BYTES = BPART * B_TILE;
+    static constexpr int NS = EX ? 2 : (MODE == 0 ? 3 : 4);         // stages of (dequantised A, token-row B)
     static constexpr int P_STAGE = N_DQ * CB_MAX;                   // one packed chunk per dequantisation warp
     static constexpr int NACC = MODE == 0 ? 1 : 2;                  // accumulator buffers of 256 (MODE 1) columns
     // MODE 0: issuer 0 runs the gate MMAs and issuer 1 the up MMAs of every
@@ -70,7 +80,7 @@ struct PfCfg {
     // header (barriers) in the first 1 KB, then the rings from a 1024-byte boundary
     static constexpr size_t RINGS = (size_t)NS * (A_BYTES + B_BYTES) + (size_t)P_STAGE;
     static constexpr size_t SMEM = 1024 + RINGS;
-    static_assert(A_MAT % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms must stay 1024-byte aligned");
+    static_assert(A_MAT % 1024 == 0 && B_TILE % 1024 == 0, "swizzle atoms must stay 1024-byte aligned");
     static_assert(P_STAGE % 128 == 0, "bulk-copy destinations must stay 16-byte aligned");
     static_assert(SMEM <= 232448, "more shared memory than a B200 block may have");
 };
@@ -357,7 +367,7 @@ struct PfChunk {
 // k / 8 of that row, stored at chunk position (k / 8) ^ g.  `base` is the
 // stage's matrix tile address plus the lane's row-group, g and t offsets; xo[c]
 // = ((c ^ g) << 4).
-template <int F, int B>
+template <int F, int B, int LO>
 __device__ __forceinline__ void pf_decode_tile(const PfChunk<F>& c, const uint32_t* sh, uint32_t base,
                                                const uint32_t* xo) {
     uint32_t a[8];
@@ -371,9 +381,15 @@ __device__ __forceinline__ void pf_decode_tile(const PfChunk<F>& c, const uint32
         const float s0 = scale_e8m0(w & 0xFFu), s1 = scale_e8m0((w >> 8) & 0xFFu);
 #pragma unroll
         for (int r = 0; r < 8; ++r) {
-            const uint32_t out = deq_pair_pow2scale(a[r] | MAGIC, K, (r & 1) ? s1 : s0);
             const int cidx = 4 * BP + 2 * (r >> 2) + ((r >> 1) & 1);
-            sts32(base + (r & 1) * 1024 + xo[cidx], out);
+            if constexpr (LO > 0) {
+                uint32_t hi, lo;
+                deq_pair_pow2scale_hilo(a[r] | MAGIC, K, (r & 1) ? s1 : s0, hi, lo);
+                sts32(base + (r & 1) * 1024 + xo[cidx], hi);
+                sts32(base + LO + (r & 1) * 1024 + xo[cidx], lo);
+            } else {
+                sts32(base + (r & 1) * 1024 + xo[cidx], deq_pair_pow2scale(a[r] | MAGIC, K, (r & 1) ? s1 : s0));
+            }
         }
     } else {
         const uint32_t w = c.sc[B];
@@ -382,18 +398,26 @@ __device__ __forceinline__ void pf_decode_tile(const PfChunk<F>& c, const uint32
 #pragma unroll
         for (int r = 0; r < 8; ++r) {
             const uint32_t v = a[r] | MAGIC;
-            const uint32_t out = (r & 1) ? deq_pair_f16scale<1>(v, w, C1) : deq_pair_f16scale<0>(v, w, C0);
             const int cidx = 4 * BP + 2 * (r >> 2) + ((r >> 1) & 1);
-            sts32(base + (r & 1) * 1024 + xo[cidx], out);
+            if constexpr (LO > 0) {
+                uint32_t hi, lo;
+                if (r & 1) deq_pair_f16scale_hilo<1>(v, w, C1, hi, lo);
+                else deq_pair_f16scale_hilo<0>(v, w, C0, hi, lo);
+                sts32(base + (r & 1) * 1024 + xo[cidx], hi);
+                sts32(base + LO + (r & 1) * 1024 + xo[cidx], lo);
+            } else {
+                const uint32_t out = (r & 1) ? deq_pair_f16scale<1>(v, w, C1) : deq_pair_f16scale<0>(v, w, C0);
+                sts32(base + (r & 1) * 1024 + xo[cidx], out);
+            }
         }
     }
 }
 
-template <int F, int KK>
+template <int F, int KK, int LO>
 __device__ __forceinline__ void pf_decode_kstep(const PfChunk<F>& c, const uint32_t* sh, uint32_t base,
                                                 const uint32_t* xo) {
-    pf_decode_tile<F, 2 * KK>(c, sh, base, xo);
-    pf_decode_tile<F, 2 * KK + 1>(c, sh, base, xo);
+    pf_decode_tile<F, 2 * KK, LO>(c, sh, base, xo);
+    pf_decode_tile<F, 2 * KK + 1, LO>(c, sh, base, xo);
 }
 
 template <int F>
@@ -453,11 +477,12 @@ __device__ __forceinline__ void pf_prefetch(const PfSrc& S, int ch, uint32_t slo
 // its part of 4 stages of A written (MODE 0: both tiles of its matrix per
 // stage; MODE 1: the tile of its parity).  `base` already points at the
 // warp's matrix and row-group.  Returns false on abort.
-template <int MODE, int F>
+template <int MODE, bool EX, int F>
 __device__ bool pf_dq_chunk(const PfParams& p, PfShared& sh, const PfRings& R, const uint8_t* slot, int lane, int g,
                             int sub, const uint32_t* xo, uint32_t lane_off, int& gstep, const PfSrc* nsrc, int nch,
                             uint32_t slot_s, uint64_t pol) {
-    using Cfg = PfCfg<MODE>;
+    using Cfg = PfCfg<MODE, EX>;
+    constexpr int LO = EX ? Cfg::LO_OFF : 0;
     cp_async_wait_all();
     __syncwarp();
     PfChunk<F> c0;
@@ -474,24 +499,24 @@ __device__ bool pf_dq_chunk(const PfParams& p, PfShared& sh, const PfRings& R, c
         const uint32_t base = smem_u32(R.a + (size_t)s * Cfg::A_BYTES) + lane_off;
         if (MODE == 0 || Cfg::N_DQ == 8) {   // both tiles of the stage
             switch (kk) {
-                case 0: pf_decode_kstep<F, 0>(c0, s0, base, xo); break;
-                case 1: pf_decode_kstep<F, 1>(c0, s0, base, xo); break;
-                case 2: pf_decode_kstep<F, 2>(c0, s0, base, xo); break;
-                default: pf_decode_kstep<F, 3>(c0, s0, base, xo); break;
+                case 0: pf_decode_kstep<F, 0, LO>(c0, s0, base, xo); break;
+                case 1: pf_decode_kstep<F, 1, LO>(c0, s0, base, xo); break;
+                case 2: pf_decode_kstep<F, 2, LO>(c0, s0, base, xo); break;
+                default: pf_decode_kstep<F, 3, LO>(c0, s0, base, xo); break;
             }
         } else if (sub == 0) {
             switch (kk) {
-                case 0: pf_decode_tile<F, 0>(c0, s0, base, xo); break;
-                case 1: pf_decode_tile<F, 2>(c0, s0, base, xo); break;
-                case 2: pf_decode_tile<F, 4>(c0, s0, base, xo); break;
-                default: pf_decode_tile<F, 6>(c0, s0, base, xo); break;
+                case 0: pf_decode_tile<F, 0, LO>(c0, s0, base, xo); break;
+                case 1: pf_decode_tile<F, 2, LO>(c0, s0, base, xo); break;
+                case 2: pf_decode_tile<F, 4, LO>(c0, s0, base, xo); break;
+                default: pf_decode_tile<F, 6, LO>(c0, s0, base, xo); break;
             }
         } else {
             switch (kk) {
-                case 0: pf_decode_tile<F, 1>(c0, s0, base, xo); break;
-                case 1: pf_decode_tile<F, 3>(c0, s0, base, xo); break;
-                case 2: pf_decode_tile<F, 5>(c0, s0, base, xo); break;
-                default: pf_decode_tile<F, 7>(c0, s0, base, xo); break;
+                case 0: pf_decode_tile<F, 1, LO>(c0, s0, base, xo); break;
+                case 1: pf_decode_tile<F, 3, LO>(c0, s0, base, xo); break;
+                case 2: pf_decode_tile<F, 5, LO>(c0, s0, base, xo); break;
+                default: pf_decode_tile<F, 7, LO>(c0, s0, base, xo); break;
             }
         }
         fence_proxy_async_smem();
@@ -531,10 +556,10 @@ __device__ __forceinline__ int pf_take_unit(PfShared& sh, uint32_t* ctrl, int i,
 // are taken from a global counter in the tiles' order (heaviest first) by the
 // producer thread and passed to the other roles through a small queue.
 // MODE 0: gate/up + SwiGLU -> hp.  MODE 1: down, y[token] += w * d.
-template <int MODE>
-__global__ void __launch_bounds__(PfCfg<MODE>::THREADS, 1)
+template <int MODE, bool EX>
+__global__ void __launch_bounds__(PfCfg<MODE, EX>::THREADS, 1)
     pf_gemm_kernel(const PfParams p, const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmX) {
-    using Cfg = PfCfg<MODE>;
+    using Cfg = PfCfg<MODE, EX>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     PfShared& sh = *reinterpret_cast<PfShared*>(smem_raw);
     // rings from the first 1024-byte boundary after the header; the launch
@@ -627,11 +652,13 @@ __global__ void __launch_bounds__(PfCfg<MODE>::THREADS, 1)
                     const int s = gstep % Cfg::NS;
                     const uint32_t ph = (uint32_t)(gstep / Cfg::NS) & 1u;
                     if (!pf_wait(sh, p.ctrl, &sh.empty[s], ph ^ 1u)) { ok = false; break; }
-                    mbar_arrive_expect_tx(&sh.full[s], (uint32_t)nbox * (PF_BOX_ROWS * PF_BK * 2));
+                    mbar_arrive_expect_tx(&sh.full[s], (uint32_t)(Cfg::BPART * nbox) * (PF_BOX_ROWS * PF_BK * 2));
                     uint8_t* dst = R.b + (size_t)s * Cfg::B_BYTES;
-                    for (int j = 0; j < nbox; ++j)
-                        tma_load_2d(dst + j * (PF_BOX_ROWS * PF_BK * 2), tm, ks * PF_BK, rbase + PF_BOX_ROWS * j,
-                                    &sh.full[s], pol);
+                    // exact down: the h1 rows, then the h2 rows (hrows further in the same map)
+                    for (int part = 0; part < Cfg::BPART; ++part)
+                        for (int j = 0; j < nbox; ++j)
+                            tma_load_2d(dst + part * Cfg::B_TILE + j * (PF_BOX_ROWS * PF_BK * 2), tm, ks * PF_BK,
+                                        rbase + part * (rk + p.T) + PF_BOX_ROWS * j, &sh.full[s], pol);
                 }
                 u = un;
             }
@@ -676,9 +703,21 @@ __global__ void __launch_bounds__(PfCfg<MODE>::THREADS, 1)
                     const uint32_t aaddr = smem_u32(R.a + (size_t)s * Cfg::A_BYTES) + aoff;
                     const uint32_t baddr = smem_u32(R.b + (size_t)s * Cfg::B_BYTES);
 #pragma unroll
-                    for (int kk = 0; kk < PF_BK / 16; ++kk)
+                    for (int kk = 0; kk < PF_BK / 16; ++kk) {
                         tc_mma_bf16(dacc, sw128_desc(aaddr + kk * 32), sw128_desc(baddr + kk * 32), idesc,
                                     (ks | kk) != 0);
+                        if constexpr (EX) {   // the remaining products of the hi/lo pairs, in a fixed order
+                            const uint32_t alo = aaddr + Cfg::LO_OFF + kk * 32;
+                            if constexpr (MODE == 1) {
+                                const uint32_t b2 = baddr + Cfg::B_TILE + kk * 32;
+                                tc_mma_bf16(dacc, sw128_desc(aaddr + kk * 32), sw128_desc(b2), idesc, true);
+                                tc_mma_bf16(dacc, sw128_desc(alo), sw128_desc(baddr + kk * 32), idesc, true);
+                                tc_mma_bf16(dacc, sw128_desc(alo), sw128_desc(b2), idesc, true);
+                            } else {
+                                tc_mma_bf16(dacc, sw128_desc(alo), sw128_desc(baddr + kk * 32), idesc, true);
+                            }
+                        }
+                    }
                     tc_commit(&sh.empty[s]);
                     // the zeroing MMA is issued: the other issuer may add to the buffer
                     if (MODE == 1 && ks == 0) {
@@ -730,9 +769,9 @@ __global__ void __launch_bounds__(PfCfg<MODE>::THREADS, 1)
                         ns = &nxt;
                     }
                 }
-                if (cur.f == 2) ok = pf_dq_chunk<MODE, 2>(p, sh, R, slot, lane, g, sub, xo, lane_off, gstep, ns, nc, slot_s, pol);
-                else if (cur.f == 3) ok = pf_dq_chunk<MODE, 3>(p, sh, R, slot, lane, g, sub, xo, lane_off, gstep, ns, nc, slot_s, pol);
-                else ok = pf_dq_chunk<MODE, 4>(p, sh, R, slot, lane, g, sub, xo, lane_off, gstep, ns, nc, slot_s, pol);
+                if (cur.f == 2) ok = pf_dq_chunk<MODE, EX, 2>(p, sh, R, slot, lane, g, sub, xo, lane_off, gstep, ns, nc, slot_s, pol);
+                else if (cur.f == 3) ok = pf_dq_chunk<MODE, EX, 3>(p, sh, R, slot, lane, g, sub, xo, lane_off, gstep, ns, nc, slot_s, pol);
+                else ok = pf_dq_chunk<MODE, EX, 4>(p, sh, R, slot, lane, g, sub, xo, lane_off, gstep, ns, nc, slot_s, pol);
             }
             if (!ok) break;
             u = un;
@@ -760,9 +799,14 @@ __global__ void __launch_bounds__(PfCfg<MODE>::THREADS, 1)
                     tmem_ld_wait();
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
-                        if (c0 + j < U.n)
-                            hrow[(long long)(U.row0 + c0 + j) * p.I] =
-                                f32_to_bf16_rne(silu_mul(__uint_as_float(gv[j]), __uint_as_float(uv[j])));
+                        if (c0 + j < U.n) {
+                            const float hv = silu_mul(__uint_as_float(gv[j]), __uint_as_float(uv[j]));
+                            const uint16_t h1 = f32_to_bf16_rne(hv);
+                            hrow[(long long)(U.row0 + c0 + j) * p.I] = h1;
+                            if constexpr (EX)   // h2 = bf16(h - h1): h1 + h2 carries 16 bits of h
+                                hrow[((long long)(rk + p.T) + U.row0 + c0 + j) * p.I] =
+                                    f32_to_bf16_rne(hv - __uint_as_float((uint32_t)h1 << 16));
+                        }
                 }
             } else {
                 float* ycol = p.y + row;
@@ -841,20 +885,29 @@ bool make_tmap(CUtensorMap* m, const void* base, long long rows, long long cols)
 
 }  // namespace
 
-size_t pf_gemm_smem_bytes(int mode) { return mode == 0 ? PfCfg<0>::SMEM : PfCfg<1>::SMEM; }
+size_t pf_gemm_smem_bytes(int mode, bool exact) {
+    if (exact) return mode == 0 ? PfCfg<0, true>::SMEM : PfCfg<1, true>::SMEM;
+    return mode == 0 ? PfCfg<0>::SMEM : PfCfg<1>::SMEM;
+}
 
 long long pf_default_wait_limit() { return PF_WAIT; }
 
-cudaError_t pf_launch(const PfParams& p, int sms, cudaStream_t stream) {
+template <bool EX>
+static cudaError_t pf_gemm_limits() {
     static SmemLimit limit[2];
-    cudaError_t e = limit[0].ensure((const void*)pf_gemm_kernel<0>, (int)pf_gemm_smem_bytes(0));
+    cudaError_t e = limit[0].ensure((const void*)pf_gemm_kernel<0, EX>, (int)pf_gemm_smem_bytes(0, EX));
     if (e != cudaSuccess) return e;
-    e = limit[1].ensure((const void*)pf_gemm_kernel<1>, (int)pf_gemm_smem_bytes(1));
+    return limit[1].ensure((const void*)pf_gemm_kernel<1, EX>, (int)pf_gemm_smem_bytes(1, EX));
+}
+
+cudaError_t pf_launch(const PfParams& p, int sms, cudaStream_t stream) {
+    cudaError_t e = p.exact ? pf_gemm_limits<true>() : pf_gemm_limits<false>();
     if (e != cudaSuccess) return e;
     CUtensorMap tm_xp, tm_x, tm_h;
     const long long rk = (long long)p.T * p.k;
+    // the h rows (exact: h1 rows, then as many h2 rows)
     if (!make_tmap(&tm_xp, p.xp, rk, p.H) || !make_tmap(&tm_x, p.x, p.T, p.H) ||
-        !make_tmap(&tm_h, p.hp, rk + p.T, p.I))
+        !make_tmap(&tm_h, p.hp, (p.exact ? 2 : 1) * (rk + p.T), p.I))
         return cudaErrorInvalidValue;
     const int n = p.T * p.k;
     const dim3 gg((p.E + 7) / 8, (n + PF_SLICE - 1) / PF_SLICE);
@@ -862,8 +915,13 @@ cudaError_t pf_launch(const PfParams& p, int sms, cudaStream_t stream) {
     pf_tiles_kernel<<<1, 1024, 0, stream>>>(p);
     pf_place_kernel<<<gg, 256, 0, stream>>>(p.idx, p.wts, n, p.k, p.E, p.cnt_part, p.off, p.perm_tok, p.perm_w);
     pf_gather_kernel<<<sms * 4, 256, 0, stream>>>(p);
-    pf_gemm_kernel<0><<<sms, PfCfg<0>::THREADS, pf_gemm_smem_bytes(0), stream>>>(p, tm_xp, tm_x);
-    pf_gemm_kernel<1><<<sms, PfCfg<1>::THREADS, pf_gemm_smem_bytes(1), stream>>>(p, tm_h, tm_h);
+    if (p.exact) {
+        pf_gemm_kernel<0, true><<<sms, PfCfg<0, true>::THREADS, pf_gemm_smem_bytes(0, true), stream>>>(p, tm_xp, tm_x);
+        pf_gemm_kernel<1, true><<<sms, PfCfg<1, true>::THREADS, pf_gemm_smem_bytes(1, true), stream>>>(p, tm_h, tm_h);
+    } else {
+        pf_gemm_kernel<0, false><<<sms, PfCfg<0>::THREADS, pf_gemm_smem_bytes(0, false), stream>>>(p, tm_xp, tm_x);
+        pf_gemm_kernel<1, false><<<sms, PfCfg<1>::THREADS, pf_gemm_smem_bytes(1, false), stream>>>(p, tm_h, tm_h);
+    }
     return cudaGetLastError();
 }
 

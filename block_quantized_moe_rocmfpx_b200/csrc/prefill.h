@@ -51,7 +51,9 @@ struct PfParams {
     float* perm_w;          // [T*k] combine weight of each routed row
     int4* tiles;            // token tiles {row0, n, expert (-1 = shared), 0}
     uint16_t* xp;           // bf16 [T*k][H] routed rows of x, grouped
-    uint16_t* hp;           // bf16 [T*k + T][I] SwiGLU output rows (routed rows, then the shared expert's)
+    uint16_t* hp;           // bf16 [T*k + T][I] SwiGLU output rows (routed rows, then the shared expert's);
+                            // exact precision: then as many rows of h - bf16(h)
+    int exact;              // 1: weights as bf16 hi + lo pairs and h as h1 + h2 (exact-precision prefill)
     int max_tiles;
     long long wait_limit;   // SM clocks before a bounded wait gives up
     int fault;              // tests of the error path only: 3 = the down GEMM waits for a stage nothing loads
@@ -62,7 +64,7 @@ struct PfWs {
     int max_tiles;
 };
 
-inline PfWs pf_ws_layout(int T, int k, int E, int H, int I) {
+inline PfWs pf_ws_layout(int T, int k, int E, int H, int I, int hparts = 1) {
     auto up = [](size_t n) { return (n + 255) / 256 * 256; };
     PfWs L;
     const size_t R = (size_t)T * k;
@@ -78,11 +80,11 @@ inline PfWs pf_ws_layout(int T, int k, int E, int H, int I) {
     L.tiles = L.perm_w + up(R * 4);
     L.xp = L.tiles + up((size_t)L.max_tiles * 16);
     L.hp = L.xp + up(R * H * 2);
-    L.total = L.hp + up((R + T) * I * 2);
+    L.total = L.hp + up((size_t)hparts * (R + T) * I * 2);
     return L;
 }
 
-size_t pf_gemm_smem_bytes(int mode);
+size_t pf_gemm_smem_bytes(int mode, bool exact);
 // Launch the whole prefill step on `stream`: grouping, gather, gate/up GEMM
 // with SwiGLU, down GEMM with the weighted combine into y.  `sms` = SM count.
 long long pf_default_wait_limit();

@@ -150,6 +150,39 @@ __device__ __forceinline__ uint32_t deq_pair_pow2scale(uint32_t v, float K, floa
     return out;
 }
 
+// The exact values of deq_pair_f16scale / deq_pair_pow2scale as bf16 pairs
+// hi + lo: hi = bf16(w), lo = bf16(w - hi).  w - hi is exact in fp32, and
+// since w = level * scale has at most 15 significant bits (11 of a binary16
+// scale, 4 of a level), lo holds it exactly.
+__device__ __forceinline__ void bf16_hilo(float f0, float f1, uint32_t& hi, uint32_t& lo) {
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(hi) : "f"(f1), "f"(f0));
+    const float r0 = f0 - __uint_as_float(hi << 16), r1 = f1 - __uint_as_float(hi & 0xffff0000u);
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(lo) : "f"(r1), "f"(r0));
+}
+template <int HS>
+__device__ __forceinline__ void deq_pair_f16scale_hilo(uint32_t v, uint32_t sc, float C, uint32_t& hi, uint32_t& lo) {
+    float f0, f1;
+    asm("{\n\t.reg .f16 a0, a1, s0, s1;\n\t"
+        "mov.b32 {a0, a1}, %2;\n\t"
+        "mov.b32 {s0, s1}, %3;\n\t"
+        "fma.rn.f32.f16 %0, a0, s%5, %4;\n\t"
+        "fma.rn.f32.f16 %1, a1, s%5, %4;\n\t}"
+        : "=f"(f0), "=f"(f1)
+        : "r"(v), "r"(sc), "f"(C), "n"(HS));
+    bf16_hilo(f0, f1, hi, lo);
+}
+__device__ __forceinline__ void deq_pair_pow2scale_hilo(uint32_t v, float K, float s, uint32_t& hi, uint32_t& lo) {
+    float f0, f1;
+    asm("{\n\t.reg .f16 a0, a1, one;\n\t"
+        "mov.b32 {a0, a1}, %2;\n\t"
+        "mov.b16 one, 0x3C00;\n\t"
+        "fma.rn.f32.f16 %0, a0, one, %3;\n\t"
+        "fma.rn.f32.f16 %1, a1, one, %3;\n\t}"
+        : "=f"(f0), "=f"(f1)
+        : "r"(v), "f"(K));
+    bf16_hilo(f0 * s, f1 * s, hi, lo);
+}
+
 // 16-byte asynchronous copy global -> shared through the load/store unit
 // (completion tracked per thread: commit a group, then wait for it).
 __device__ __forceinline__ void cp_async16(uint32_t saddr, const void* src, uint64_t policy) {

@@ -286,10 +286,15 @@ int moe_ffn_forward(const moe_layer* layer, const void* x, int T, const int32_t*
 /*
  * The same step from host buffers: x (bf16 bits [T][H]) and the router
  * logits (fp32 [T][E]) are copied host -> device, moe_router_topk and
- * moe_ffn_forward run, and y (fp32 [T][H]) is copied device -> host, all
- * enqueued on `stream` (one cudaMemcpyAsync per buffer; the host buffers should
- * be pinned for the copies to be asynchronous; y is valid after the stream
- * synchronises).  scratch: device, 256-byte aligned,
+ * moe_ffn_forward run, and y (fp32 [T][H]) is copied device -> host (one
+ * cudaMemcpyAsync per buffer; the host buffers should be pinned for the
+ * copies to be asynchronous).  The two uploads run on a stream the layer
+ * makes on first use, into one of two buffer sets used in turn, and `stream`
+ * waits for them: a call's uploads overlap the kernels of the call before
+ * it.  The kernels and the download run on `stream`; x, the logits and y may
+ * be reused once `stream` has synchronised.  Inside a CUDA graph capture
+ * everything stays on `stream`.  Calls on one layer are serialised by a lock
+ * in the layer.  scratch: device, 256-byte aligned,
  * moe_ffn_host_scratch_bytes(layer, T) bytes, caller-owned, zeroed once with
  * rfx_ws_init before its first use; it holds the moe_ffn_forward workspace
  * first (so rfx_ws_status(scratch) reads its device flag), then the device
@@ -329,6 +334,32 @@ int moe_ffn_prefill(const moe_layer* layer, const void* x, int T, const int32_t*
                     void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Prefill at a chosen operand precision (the prefill workload dequantises "to
+ * bf16 or fp8" for the tensor cores; the exact variant keeps the decode
+ * path's numbers, for a prefill whose result must agree with decode):
+ *   RFX_PREFILL_BF16  = moe_ffn_prefill (each weight rounded once to bf16,
+ *                       h rounded to bf16);
+ *   RFX_PREFILL_EXACT = each weight enters the tensor cores as the bf16 pair
+ *                       hi + lo, hi = bf16(w), lo = bf16(w - hi), which is
+ *                       w exactly (w = level * scale has at most 15
+ *                       significant bits); h enters the down projection as
+ *                       h1 + h2, h1 = bf16(h), h2 = bf16(h - h1) (16 bits,
+ *                       relative error <= 2^-18).  Gate/up take 2 MMAs per
+ *                       k-step and matrix, down 4 (hi h1, hi h2, lo h1,
+ *                       lo h2): about 2.7 times the tensor work of bf16.
+ *                       Accumulation in fp32.
+ * Same arguments, limits and behaviour as moe_ffn_prefill otherwise; the
+ * exact variant's workspace also holds the h2 rows
+ * (moe_prefill_workspace_bytes_ex).  Unknown precision: 0 bytes /
+ * RFX_EINVAL.
+ */
+#define RFX_PREFILL_BF16 0
+#define RFX_PREFILL_EXACT 1
+size_t moe_prefill_workspace_bytes_ex(const moe_layer* layer, int T, int precision);
+int moe_ffn_prefill_ex(const moe_layer* layer, const void* x, int T, const int32_t* idx, const float* w, float* y,
+                       void* ws, size_t ws_bytes, int precision, void* stream);
+
+/*
  * Device pointers into a prefill workspace after a moe_ffn_prefill call (for
  * inspection and tests): counts[E] tokens per routed expert; row_token and
  * row_weight [routed_rows] the token and combine weight of each grouped row
@@ -344,6 +375,7 @@ typedef struct {
     const void* h;
     int64_t routed_rows;
     int64_t h_rows;
+    const void* h_lo;   /* after an exact-precision call: h2 = bf16(h - h1) of every row, same layout as h */
 } moe_prefill_ws_view;
 int moe_prefill_view(const moe_layer* layer, int T, const void* ws, moe_prefill_ws_view* view);
 

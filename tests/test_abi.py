@@ -276,7 +276,8 @@ def test_zero_token_calls_are_noops():
 
 def test_host_call_scratch_bytes():
     """moe_ffn_host_scratch_bytes = the moe_ffn_forward workspace (decode or
-    prefill) + the padded device copies of x, logits, idx, w and y."""
+    prefill) + two padded device copies of x and of the logits (used in turn)
+    + idx, w and y."""
     d = rfx.moe_layer_desc()
     d.H, d.I, d.E, d.k = 4096, 2048, 256, 6
     d.f_gate, d.f_up, d.f_down = 2, 2, 3
@@ -288,7 +289,7 @@ def test_host_call_scratch_bytes():
         up = lambda n: (n + 255) // 256 * 256
         for T in (1, 4, 8, 9, 2048):
             ws = rfx.moe_ffn_workspace_bytes(h, T)
-            want = up(ws) + up(T * 4096 * 2) + up(T * 256 * 4) + 2 * up(T * 6 * 4) + up(T * 4096 * 4)
+            want = up(ws) + 2 * up(T * 4096 * 2) + 2 * up(T * 256 * 4) + 2 * up(T * 6 * 4) + up(T * 4096 * 4)
             assert rfx.moe_ffn_host_scratch_bytes(h, T) == want, T
         assert rfx.moe_ffn_host_scratch_bytes(h, 0) == 0
     finally:

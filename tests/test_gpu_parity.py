@@ -251,6 +251,30 @@ def test_forward_host_equals_device_path(full_layer, T):
     assert ml.status() == rfx.RFX_OK
 
 
+def test_forward_host_pipelined_calls(full_layer):
+    """Back-to-back host-buffer calls with no synchronisation between them:
+    each call's uploads overlap the previous call's kernels (two device buffer
+    sets in turn); every y equals the device path's bits for its own inputs."""
+    ml = full_layer.moe_layer()
+    T, n = 2, 6
+    Ls = [synth.logits(9, 0, 100 + 7 * i, T, 256, 1.1) for i in range(n)]
+    xbs = [synth.x_bf16(9, 100 + 7 * i, T, 4096) for i in range(n)]
+    xh = [torch.from_numpy(a).view(torch.bfloat16).pin_memory() for a in xbs]
+    lh = [torch.from_numpy(a).pin_memory() for a in Ls]
+    yh = [torch.full((T, 4096), float("nan"), dtype=torch.float32).pin_memory() for _ in range(n)]
+    for i in range(n):
+        ml.forward_host(xh[i], lh[i], yh[i])
+    torch.cuda.synchronize()
+    assert ml.host_status() == rfx.RFX_OK
+    for i in range(n):
+        idx = torch.empty((T, 6), dtype=torch.int32, device=DEV)
+        w = torch.empty((T, 6), dtype=torch.float32, device=DEV)
+        y = torch.empty((T, 4096), dtype=torch.float32, device=DEV)
+        rfx.moe_router_topk(to_dev(Ls[i]), 6, idx, w)
+        ml.forward(to_dev(xbs[i], torch.bfloat16), idx, w, y)
+        assert torch.equal(yh[i], y.cpu()), f"call {i}"
+
+
 def test_forward_host_prefill_path():
     H, I, E, k, T = 512, 256, 16, 4, 40
     lay = SynthLayer(29, 0, H, I, E, k)
