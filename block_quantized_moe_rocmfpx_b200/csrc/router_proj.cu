@@ -44,6 +44,10 @@ __device__ __forceinline__ void bf16x8(uint4 v, float f[8]) {
     f[6] = __uint_as_float(v.w << 16); f[7] = __uint_as_float(v.w & 0xffff0000u);
 }
 
+__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 __global__ void __launch_bounds__(RP_THREADS) router_logits_kernel(const uint16_t* __restrict__ W,
                                                                   const float* __restrict__ bias,
                                                                   const uint16_t* __restrict__ x, int T, int H, int E,
