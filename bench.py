@@ -476,7 +476,7 @@ def measure_router_proj(T: int, steps: int, warmup: int, dev):
     return {"T": T, "us_per_call": us, "bytes_per_call": nbytes, "achieved_gbs": gbs,
             "roofline": {"bound": "hbm", "peak_gbs": peak, "frac": gbs / peak, "peak_kind": peak_kind,
                          "t_min_us": nbytes / (peak * 1e9) * 1e6},
-            "launches_per_call": 2, "steps": steps}
+            "launches_per_call": 1 if T <= 8 else 2, "steps": steps}
 
 
 GEMV_N, GEMV_K = 131072, 4096   # one matrix larger than L2 in every format (168 to 285 MB packed)

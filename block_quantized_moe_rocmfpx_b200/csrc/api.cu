@@ -110,6 +110,16 @@ extern "C" int moe_router_project_topk(const void* w_router, const float* bias, 
                                        int k, float* logits, int32_t* idx, float* w, void* stream) {
     if (T < 0 || E < 1 || E > 1024 || k < 1 || k > E || k > 16)
         return rfx_fail(RFX_EINVAL, "moe_router_project_topk: need T >= 0, 1 <= E <= 1024, 1 <= k <= min(E, 16)");
+    if (T >= 1 && T <= 8) {   // decode / verify: projection and top-k in one cooperative launch
+        if (H < 32 || H % 32 != 0) return rfx_fail(RFX_EINVAL, "moe_router_project_topk: H a positive multiple of 32");
+        if (!w_router || !x || !logits || !idx || !w) return rfx_fail(RFX_EINVAL, "moe_router_project_topk: null pointer");
+        if (((uintptr_t)w_router & 15u) || ((uintptr_t)x & 15u))
+            return rfx_fail(RFX_EINVAL, "moe_router_project_topk: w_router and x must be 16-byte aligned");
+        cudaError_t e = rfx::router_project_topk_launch((const uint16_t*)w_router, bias, (const uint16_t*)x, T, H, E, k,
+                                                        logits, idx, w, (cudaStream_t)stream);
+        if (e != cudaErrorNotSupported) return e == cudaSuccess ? RFX_OK : cuda_fail("moe_router_project_topk", e);
+        // the grid does not fit the device at once: the two launches below
+    }
     int rc = moe_router_logits(w_router, bias, x, T, H, E, logits, stream);
     if (rc != RFX_OK) return rc;
     return moe_router_topk(logits, T, E, k, idx, w, stream);

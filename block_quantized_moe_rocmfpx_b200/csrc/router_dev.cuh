@@ -13,8 +13,10 @@
 
 namespace rfx {
 
-// Lane j < k writes idx_out[j] and w_out[j].  E <= 32 * PER_LANE.
-template <int PER_LANE>
+// Lane j < k writes idx_out[j] and w_out[j].  E <= 32 * PER_LANE.  COHERENT:
+// the logits were written earlier in the same kernel by other CTAs (read
+// through L2, not the read-only path).
+template <int PER_LANE, bool COHERENT = false>
 __device__ __forceinline__ void router_warp(const float* __restrict__ l, int E, int k, int32_t* idx_out,
                                             float* w_out) {
     const int lane = threadIdx.x & 31;
@@ -23,7 +25,7 @@ __device__ __forceinline__ void router_warp(const float* __restrict__ l, int E, 
 #pragma unroll
     for (int i = 0; i < PER_LANE; ++i) {
         const int e = lane + 32 * i;
-        v[i] = e < E ? __ldg(l + e) : 0.f;
+        v[i] = e < E ? (COHERENT ? __ldcg(l + e) : __ldg(l + e)) : 0.f;
         if (e < E) live |= 1u << i;
     }
     float sel_v = 0.f, v0 = 0.f;

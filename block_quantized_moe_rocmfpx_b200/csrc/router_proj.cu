@@ -26,11 +26,16 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <cooperative_groups.h>
+
 #include "gemv.h"
 #include "launch_util.h"
 #include "rfx_device.cuh"
+#include "router_dev.cuh"
 
 namespace rfx {
+
+namespace cg = cooperative_groups;
 
 constexpr int RP_ROWS = 2;     // router rows per CTA
 constexpr int RP_SPLIT = 4;    // warps per row (quarters of H)
@@ -48,11 +53,10 @@ __device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) 
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
-__global__ void __launch_bounds__(RP_THREADS) router_logits_kernel(const uint16_t* __restrict__ W,
-                                                                  const float* __restrict__ bias,
-                                                                  const uint16_t* __restrict__ x, int T, int H, int E,
-                                                                  float* __restrict__ logits) {
-    grid_dep_launch();
+// The projection of the CTA's RP_ROWS rows for up to RP_COLS columns.
+__device__ __forceinline__ void project_rows(const uint16_t* __restrict__ W, const float* __restrict__ bias,
+                                             const uint16_t* __restrict__ x, int T, int H, int E,
+                                             float* __restrict__ logits) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r = warp / RP_SPLIT, part = warp - r * RP_SPLIT;
     const int row = blockIdx.x * RP_ROWS + r;
@@ -67,17 +71,30 @@ __global__ void __launch_bounds__(RP_THREADS) router_logits_kernel(const uint16_
     for (int c = 0; c < RP_COLS; ++c) acc[c] = 0.f;
     if (row < E) {
         const uint4* w4 = reinterpret_cast<const uint4*>(wp);
-        for (int ch = lane; ch < kp / 8; ch += 32) {
-            float wf[8];
-            bf16x8(__ldg(w4 + ch), wf);
+        const int nch = kp / 8;   // 16-byte chunks of the warp's quarter
+        // four chunks per lane in flight at once (H = 4096: all of them)
+        for (int ch0 = lane; ch0 < nch; ch0 += 4 * 32) {
+            uint4 wv[4];
 #pragma unroll
-            for (int c = 0; c < RP_COLS; ++c) {
-                if (c >= nc) break;
-                const uint4* x4 = reinterpret_cast<const uint4*>(x + (size_t)(c0 + c) * H + (size_t)part * kp);
-                float xf[8];
-                bf16x8(__ldg(x4 + ch), xf);
+            for (int u = 0; u < 4; ++u) {
+                const int ch = ch0 + 32 * u;
+                wv[u] = ch < nch ? __ldg(w4 + ch) : make_uint4(0u, 0u, 0u, 0u);
+            }
 #pragma unroll
-                for (int i = 0; i < 8; ++i) acc[c] = fmaf(wf[i], xf[i], acc[c]);
+            for (int u = 0; u < 4; ++u) {
+                const int ch = ch0 + 32 * u;
+                if (ch >= nch) break;
+                float wf[8];
+                bf16x8(wv[u], wf);
+#pragma unroll
+                for (int c = 0; c < RP_COLS; ++c) {
+                    if (c >= nc) break;
+                    const uint4* x4 = reinterpret_cast<const uint4*>(x + (size_t)(c0 + c) * H + (size_t)part * kp);
+                    float xf[8];
+                    bf16x8(__ldg(x4 + ch), xf);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) acc[c] = fmaf(wf[i], xf[i], acc[c]);
+                }
             }
         }
     }
@@ -100,6 +117,32 @@ __global__ void __launch_bounds__(RP_THREADS) router_logits_kernel(const uint16_
             logits[(size_t)(c0 + c) * E + e] = v;
         }
     }
+}
+
+__global__ void __launch_bounds__(RP_THREADS) router_logits_kernel(const uint16_t* __restrict__ W,
+                                                                  const float* __restrict__ bias,
+                                                                  const uint16_t* __restrict__ x, int T, int H, int E,
+                                                                  float* __restrict__ logits) {
+    grid_dep_launch();
+    project_rows(W, bias, x, T, H, E, logits);
+}
+
+// T <= 8 with the top-k in the same launch (cooperative: every CTA is
+// resident): after a grid-wide barrier that orders the logit stores, warp t of
+// CTA 0 runs the router's warp top-k on column t.
+template <int PER_LANE>
+__global__ void __launch_bounds__(RP_THREADS) router_project_topk_kernel(const uint16_t* __restrict__ W,
+                                                                        const float* __restrict__ bias,
+                                                                        const uint16_t* __restrict__ x, int T, int H,
+                                                                        int E, int k, float* __restrict__ logits,
+                                                                        int32_t* __restrict__ idx,
+                                                                        float* __restrict__ w) {
+    grid_dep_launch();
+    project_rows(W, bias, x, T, H, E, logits);
+    cg::this_grid().sync();
+    const int warp = threadIdx.x >> 5;
+    if (blockIdx.x == 0 && warp < T)
+        router_warp<PER_LANE, true>(logits + (size_t)warp * E, E, k, idx + (size_t)warp * k, w + (size_t)warp * k);
 }
 
 // ------------------------------------------------------------- T > 8 ---
@@ -232,6 +275,50 @@ cudaError_t router_logits_launch(const uint16_t* W, const float* bias, const uin
     cfg.attrs = at;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, router_logits_kernel, W, bias, x, T, H, E, logits);
+}
+
+template <int PER_LANE>
+static cudaError_t launch_fused(const uint16_t* W, const float* bias, const uint16_t* x, int T, int H, int E, int k,
+                                float* logits, int32_t* idx, float* w, cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((E + RP_ROWS - 1) / RP_ROWS));
+    cfg.blockDim = dim3(RP_THREADS);
+    cfg.stream = stream;
+    cudaLaunchAttribute at[2];
+    at[0].id = cudaLaunchAttributeCooperative;
+    at[0].val.cooperative = 1;
+    at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, router_project_topk_kernel<PER_LANE>, W, bias, x, T, H, E, k, logits, idx, w);
+}
+
+// The fused launch when every CTA fits on the device at once, else the two
+// launches (cudaErrorNotSupported tells the caller to use them).
+template <int PER_LANE>
+static bool fused_fits(int E) {
+    int dev = 0, sms = 0, per_sm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, router_project_topk_kernel<PER_LANE>, RP_THREADS, 0) !=
+        cudaSuccess)
+        return false;
+    return (long long)per_sm * sms >= (E + RP_ROWS - 1) / RP_ROWS;
+}
+
+cudaError_t router_project_topk_launch(const uint16_t* W, const float* bias, const uint16_t* x, int T, int H, int E,
+                                       int k, float* logits, int32_t* idx, float* w, cudaStream_t stream) {
+    const int per = (E + 31) / 32;
+    const bool fits = per <= 1 ? fused_fits<1>(E) : per <= 2 ? fused_fits<2>(E) : per <= 4 ? fused_fits<4>(E)
+                      : per <= 8 ? fused_fits<8>(E) : per <= 16 ? fused_fits<16>(E) : fused_fits<32>(E);
+    if (!fits) return cudaErrorNotSupported;
+    if (per <= 1) return launch_fused<1>(W, bias, x, T, H, E, k, logits, idx, w, stream);
+    if (per <= 2) return launch_fused<2>(W, bias, x, T, H, E, k, logits, idx, w, stream);
+    if (per <= 4) return launch_fused<4>(W, bias, x, T, H, E, k, logits, idx, w, stream);
+    if (per <= 8) return launch_fused<8>(W, bias, x, T, H, E, k, logits, idx, w, stream);
+    if (per <= 16) return launch_fused<16>(W, bias, x, T, H, E, k, logits, idx, w, stream);
+    return launch_fused<32>(W, bias, x, T, H, E, k, logits, idx, w, stream);
 }
 
 }  // namespace rfx

@@ -165,9 +165,12 @@ int moe_router_logits(const void* w_router, const float* bias, const void* x, in
                       void* stream);
 
 /*
- * moe_router_logits followed by moe_router_topk (two launches, the second a
- * programmatic dependent of the first): logits [T][E], idx [T][k], w [T][k]
- * on the device.  Limits: both calls' (E <= 1024, k <= min(E, 16)).
+ * moe_router_logits followed by moe_router_topk: logits [T][E], idx [T][k],
+ * w [T][k] on the device, the same numbers as the two calls.  T <= 8 (decode /
+ * verify): one cooperative launch (every CTA resident; a grid-wide barrier
+ * orders the logit stores before one warp per column ranks them), a
+ * programmatic dependent of the kernel before it.  T > 8: the two launches.
+ * Limits: both calls' (E <= 1024, k <= min(E, 16)).
  */
 int moe_router_project_topk(const void* w_router, const float* bias, const void* x, int T, int H, int E, int k,
                             float* logits, int32_t* idx, float* w, void* stream);

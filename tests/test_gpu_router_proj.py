@@ -95,6 +95,21 @@ def test_router_project_topk_teacher_forced(E, H, T, k):
     assert np.allclose(w, rw, rtol=1e-6, atol=0)
 
 
+@pytest.mark.parametrize("E,H,T,k", [(256, 4096, 1, 6), (256, 4096, 8, 6), (1000, 512, 5, 16), (24, 256, 3, 4)])
+def test_router_project_topk_one_launch_equals_two(E, H, T, k):
+    """T <= 8 runs the projection and the top-k in one cooperative launch; its
+    logits, idx and w are bitwise those of moe_router_logits followed by
+    moe_router_topk."""
+    W, b, x, lg, idx, w = run(E, H, T, seed=31 + T, k=k)
+    _, _, _, lg2, _, _ = run(E, H, T, seed=31 + T)
+    assert np.array_equal(lg, lg2)
+    idx2 = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    w2 = torch.empty((T, k), dtype=torch.float32, device=DEV)
+    rfx.moe_router_topk(torch.from_numpy(lg2).to(DEV), k, idx2, w2)
+    assert np.array_equal(idx, idx2.cpu().numpy())
+    assert np.array_equal(w, w2.cpu().numpy())
+
+
 def test_router_logits_empty_is_a_noop():
     Wd = torch.zeros((8, 64), dtype=torch.int16, device=DEV)
     xd = torch.zeros((0, 64), dtype=torch.int16, device=DEV)
