@@ -1220,8 +1220,7 @@ __device__ void stage_x(const MoeParams& p, Shared& sh, uint8_t* xh, int sid, in
 #pragma unroll
         for (int k = 0; k < XR; ++k) {
             const int i0 = r0 + k * nthr + sid - lane;
-            if (i0 >= nitems) break;
-            x_max(sh, v[k], i0, lane, nitems, per_col);
+            if (i0 < nitems) x_max(sh, v[k], i0, lane, nitems, per_col);
         }
     }
     asm volatile("bar.sync 1, %0;" ::"r"(nthr) : "memory");
@@ -1243,8 +1242,7 @@ __device__ void stage_x(const MoeParams& p, Shared& sh, uint8_t* xh, int sid, in
 #pragma unroll
         for (int k = 0; k < XR; ++k) {
             const int i0 = r0 + k * nthr + sid - lane;
-            if (i0 >= nitems) break;
-            x_put(p, sh, xh, sx, sxs, nxc, v[k], i0, lane, nitems, per_col);
+            if (i0 < nitems) x_put(p, sh, xh, sx, sxs, nxc, v[k], i0, lane, nitems, per_col);
         }
     }
 }

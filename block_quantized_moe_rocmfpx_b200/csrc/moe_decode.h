@@ -73,16 +73,21 @@ struct MoeParams {
                            // the grid has; 2 = no slot ever counts as ready for the down projection
 };
 
-// Floats per column of the h block-sum table: one per 16-row group of I,
-// padded to a multiple of 4 (16 bytes).
-inline __host__ __device__ int moe_sstr(int I) { return ((I / 16) + 3) & ~3; }
+// Per-column tables read with 16-byte loads by lanes of different columns:
+// rows of 8k + 4 floats, so that column c starts c * 16 bytes further into
+// the 128-byte bank window (up to 8 columns, one 16-byte load each, without
+// bank conflicts) and every row stays 16-byte aligned.
+inline __host__ __device__ int moe_col_stride(int n) { return ((n + 7) & ~7) + 4; }
 
-// Floats per column of the x block-sum table (H/32 padded to 16-byte rows).
-inline __host__ __device__ int moe_sxs(int H) { return ((H / 32) + 3) & ~3; }
+// Floats per column of the h block-sum table: one per 16-row group of I.
+inline __host__ __device__ int moe_sstr(int I) { return moe_col_stride(I / 16); }
 
-// Floats per column of the h block-scale table: one per 32-block of I,
-// padded to a multiple of 8 (a chunk's 8 blocks are read as two 16-byte loads).
-inline __host__ __device__ int moe_sbs(int I) { return ((I / 32) + 7) & ~7; }
+// Floats per column of the x block-sum table: one per 32-block of H.
+inline __host__ __device__ int moe_sxs(int H) { return moe_col_stride(H / 32); }
+
+// Floats per column of the h block-scale table: one per 32-block of I (a
+// chunk's 8 blocks are read as two 16-byte loads).
+inline __host__ __device__ int moe_sbs(int I) { return moe_col_stride(I / 32); }
 
 // Bytes of a slot's h image for ncols columns: the fp16 hi/lo fragments of
 // h * 2^n (4 bytes per value), the 16-row block sums, the 2^-n factors.
