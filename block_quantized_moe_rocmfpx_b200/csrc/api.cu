@@ -513,12 +513,24 @@ extern "C" int moe_ffn_forward_host(const moe_layer* layer, const void* x, const
     if (e != cudaSuccess) return cuda_fail("moe_ffn_forward_host", e);
     int rc = moe_router_topk(ld, T, d.E, d.k, idx, w, stream);
     if (rc != RFX_OK) return rc;
-    rc = moe_ffn_forward(layer, xd, T, idx, w, yd, b + S.ffn, S.x[0], stream);
+    // decode: pinned host y that the device can address (page-locked and
+    // mapped, as cudaHostAlloc / cudaHostRegister memory is under unified
+    // addressing) takes the kernel's combine stores directly, with no copy
+    float* ydev = nullptr;
+    if (T <= MOE_MAXT) {
+        cudaPointerAttributes pa{};
+        if (cudaPointerGetAttributes(&pa, y) == cudaSuccess && pa.type == cudaMemoryTypeHost && pa.devicePointer)
+            ydev = (float*)pa.devicePointer;
+        else
+            (void)cudaGetLastError();   // not an error: pageable memory takes the copy below
+    }
+    rc = moe_ffn_forward(layer, xd, T, idx, w, ydev ? ydev : yd, b + S.ffn, S.x[0], stream);
     if (rc != RFX_OK) return rc;
     if (side) {
         e = cudaEventRecord(L->ev_free[s], st);
         if (e != cudaSuccess) return cuda_fail("moe_ffn_forward_host", e);
     }
+    if (ydev) return RFX_OK;
     e = cudaMemcpyAsync(y, yd, (size_t)T * d.H * 4, cudaMemcpyDeviceToHost, st);
     return e == cudaSuccess ? RFX_OK : cuda_fail("moe_ffn_forward_host", e);
 }

@@ -295,7 +295,9 @@ int moe_ffn_forward(const moe_layer* layer, const void* x, int T, const int32_t*
  * makes on first use, into one of two buffer sets used in turn, and `stream`
  * waits for them: a call's uploads overlap the kernels of the call before
  * it.  The kernels and the download run on `stream`; x, the logits and y may
- * be reused once `stream` has synchronised.  Inside a CUDA graph capture
+ * be reused once `stream` has synchronised.  For T <= 8 a y in page-locked
+ * host memory that the device can address (cudaHostAlloc, cudaHostRegister)
+ * receives the decode kernel's stores directly instead of a copy.  Inside a CUDA graph capture
  * everything stays on `stream`.  Calls on one layer are serialised by a lock
  * in the layer.  scratch: device, 256-byte aligned,
  * moe_ffn_host_scratch_bytes(layer, T) bytes, caller-owned, zeroed once with

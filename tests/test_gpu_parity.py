@@ -275,6 +275,23 @@ def test_forward_host_pipelined_calls(full_layer):
         assert torch.equal(yh[i], y.cpu()), f"call {i}"
 
 
+def test_forward_host_pageable_buffers(full_layer):
+    """Pageable (not page-locked) host buffers: the copies path, same bits."""
+    ml = full_layer.moe_layer()
+    T = 3
+    L = synth.logits(10, 0, 5, T, 256, 1.1)
+    xb = synth.x_bf16(10, 5, T, 4096)
+    idx = torch.empty((T, 6), dtype=torch.int32, device=DEV)
+    w = torch.empty((T, 6), dtype=torch.float32, device=DEV)
+    y = torch.empty((T, 4096), dtype=torch.float32, device=DEV)
+    rfx.moe_router_topk(to_dev(L), 6, idx, w)
+    ml.forward(to_dev(xb, torch.bfloat16), idx, w, y)
+    yh = torch.full((T, 4096), float("nan"), dtype=torch.float32)    # pageable
+    ml.forward_host(torch.from_numpy(xb).view(torch.bfloat16), torch.from_numpy(L), yh)
+    torch.cuda.synchronize()
+    assert torch.equal(yh, y.cpu())
+
+
 def test_forward_host_prefill_path():
     H, I, E, k, T = 512, 256, 16, 4, 40
     lay = SynthLayer(29, 0, H, I, E, k)
