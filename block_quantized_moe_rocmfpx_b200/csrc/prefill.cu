@@ -35,6 +35,7 @@
 #include "rfx_layout.h"
 #include "rfx_tile.cuh"
 #include "tc.cuh"
+#include "tmap.h"
 
 namespace rfx {
 namespace {
@@ -852,35 +853,10 @@ __global__ void __launch_bounds__(PfCfg<MODE, EX>::THREADS, 1)
 
 // ------------------------------------------------------------- host side ---
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* f = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(f);
-    }
-    return fn;
-}
-
-// bf16 matrix [rows][cols] (row stride cols * 2 bytes), boxes of 64 columns x
-// 64 rows in the 128-byte swizzled layout; rows beyond `rows` read as zero.
+// bf16 matrix [rows][cols], boxes of PF_BK columns x PF_BOX_ROWS rows.
 bool make_tmap(CUtensorMap* m, const void* base, long long rows, long long cols) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-    const cuuint32_t box[2] = {PF_BK, PF_BOX_ROWS};
-    const cuuint32_t es[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    static_assert(PF_BK == 64, "the tensor maps' boxes are 64 columns wide");
+    return make_tmap_bf16(m, base, rows, cols, PF_BOX_ROWS);
 }
 
 }  // namespace

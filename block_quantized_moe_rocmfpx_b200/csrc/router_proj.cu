@@ -9,20 +9,19 @@
 // GB"); this library reads that as bf16 weights.
 //
 // B200 design, T <= 8 (decode / verify): a GEMV over E rows (2 MB for 256 x
-// 4096), HBM-bound, spread over all SMs.  A CTA owns two rows and up to 8 columns; each of its 8 warps takes a
-// quarter of H for one row (16-byte loads of 8 bf16 of W and of x, fp32 FMAs in
+// 4096), HBM-bound, spread over all SMs.  A CTA owns two rows and up to 8
+// columns; each of its 8 warps takes a quarter of H for one row (16-byte loads of 8 bf16 of W and of x, fp32 FMAs in
 // index order per lane, then a butterfly over the lanes); the four quarters
 // are added in a fixed tree, so a logit's bits depend neither on T nor on the
 // launch.  W is a constant input: each warp asks L2 for its slice before the
 // kernel waits for the previous one (programmatic dependent launch); x may come
 // from that kernel and is read after the wait.
 //
-// T > 8 (prefill): a tensor-core GEMM, logits^T = W x^T, bf16 operands with
-// fp32 accumulation (mma.sync m16n8k16: every product is exact, the sums are
-// fp32 in a fixed order per element).  A CTA computes 64 experts x 32 tokens
-// (256 CTAs at E = 256, T = 2048); K runs in chunks of 64 staged by cp.async
-// through a 4-deep shared-memory ring (padded rows: conflict-free ldmatrix);
-// 4 warps of 32 x 16.
+// T > 8 (prefill): a tcgen05 GEMM, logits^T = W x^T, bf16 operands with fp32
+// accumulation in tensor memory (every product is exact; the sums are fp32
+// in the tensor core's fixed order per element, so a column's logits do not
+// depend on the other columns).  Operands by TMA, one MMA thread, 4 epilogue
+// warps (below).
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -32,6 +31,8 @@
 #include "launch_util.h"
 #include "rfx_device.cuh"
 #include "router_dev.cuh"
+#include "tc.cuh"
+#include "tmap.h"
 
 namespace rfx {
 
@@ -146,106 +147,123 @@ __global__ void __launch_bounds__(RP_THREADS) router_project_topk_kernel(const u
 }
 
 // ------------------------------------------------------------- T > 8 ---
+//
+// A CTA computes 128 experts x 128 tokens: K in steps of 64 through a 6-stage
+// ring of TMA boxes (128 rows of W, 128 rows of x, 128-byte swizzle; rows and
+// columns beyond the tensors read as zero); one thread issues the
+// 128 x 128 x 16 MMAs into a 128-column fp32 accumulator in tensor memory; 4
+// warps (one tensor-memory lane quarter each) add the bias and store the
+// logits.  Every wait is bounded; a CTA that gives up stores nothing (the
+// test of the call is its parity check).
+constexpr int RT_BM = 128, RT_BN = 128, RT_BK = 64, RT_NS = 6;
+constexpr int RT_TILE_A = RT_BM * RT_BK * 2, RT_TILE_B = RT_BN * RT_BK * 2, RT_STAGE = RT_TILE_A + RT_TILE_B;
+static_assert(RT_TILE_A % 1024 == 0 && RT_TILE_B % 1024 == 0, "swizzle atoms must stay 1024-byte aligned");
+constexpr int RT_THREADS = 256;   // warp 0: TMA; warp 1: tensor memory + MMA; warps 4..7: epilogue
+constexpr size_t RT_SMEM = 1024 + (size_t)RT_NS * RT_STAGE;
+constexpr long long RT_WAIT = 1000000000LL;   // SM clocks before a wait gives up
 
-constexpr int RM_BM = 64, RM_BN = 32, RM_BK = 64, RM_STAGES = 4;
-constexpr int RM_LD = RM_BK + 8;   // padded row (144 bytes): ldmatrix rows hit distinct banks
-constexpr int RM_THREADS = 128;
-constexpr int RM_STAGE_ELEMS = (RM_BM + RM_BN) * RM_LD;
-constexpr size_t RM_SMEM = (size_t)RM_STAGES * RM_STAGE_ELEMS * 2;
+struct RtShared {
+    uint64_t full[RT_NS], empty[RT_NS], acc;
+    uint32_t tmem;
+    volatile int abort;
+};
 
-__device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, bool valid) {
-    const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(valid ? 16 : 0) : "memory");
-}
-
-__device__ __forceinline__ void ldsm_x4(const void* p, uint32_t r[4]) {
-    const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(p));
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(a));
-}
-
-__global__ void __launch_bounds__(RM_THREADS) router_logits_mma_kernel(const uint16_t* __restrict__ W,
-                                                                      const float* __restrict__ bias,
-                                                                      const uint16_t* __restrict__ x, int T, int H,
-                                                                      int E, float* __restrict__ logits) {
-    extern __shared__ __align__(16) uint16_t rm_smem[];   // [stage][A rows 64 | B rows 32][RM_LD]
+__global__ void __launch_bounds__(RT_THREADS, 1)
+    router_logits_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                            const float* __restrict__ bias, int T, int H, int E, float* __restrict__ logits) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    RtShared& sh = *reinterpret_cast<RtShared*>(smem_raw);
+    const uint32_t off = ((smem_u32(smem_raw) + (uint32_t)sizeof(RtShared) + 1023u) & ~1023u) - smem_u32(smem_raw);
+    if (off > 1024u) return;   // the ring would overrun the allocation
+    uint8_t* ring = smem_raw + off;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int e0 = blockIdx.x * RT_BM, t0 = blockIdx.y * RT_BN;
+    const int nk = (H + RT_BK - 1) / RT_BK;
     grid_dep_launch();
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int e0 = blockIdx.x * RM_BM, t0 = blockIdx.y * RM_BN;
-    const int wm = (warp >> 1) * 32, wn = (warp & 1) * 16;
-    const int nk = (H + RM_BK - 1) / RM_BK;
-    // stage tiles: A 64 rows x 8 pieces of 16 bytes (4 per thread), B 32 x 8 (2 per thread);
-    // a K tail shorter than 64 (H % 64 == 32) is zero-filled
-    auto load = [&](int kc) {
-        uint16_t* sa = rm_smem + (kc % RM_STAGES) * RM_STAGE_ELEMS;
-        uint16_t* sb = sa + RM_BM * RM_LD;
-        const int pc = tid & 7, k = kc * RM_BK + pc * 8;
-        const bool kv = k < H;
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-            const int r = (tid >> 3) + 16 * h;
-            const bool v = kv && e0 + r < E;
-            cp_async16_zfill(sa + r * RM_LD + pc * 8, W + (size_t)(v ? e0 + r : 0) * H + (kv ? k : 0), v);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < RT_NS; ++s) {
+            mbar_init(&sh.full[s], 1);
+            mbar_init(&sh.empty[s], 1);
         }
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int r = (tid >> 3) + 16 * h;
-            const bool v = kv && t0 + r < T;
-            cp_async16_zfill(sb + r * RM_LD + pc * 8, x + (size_t)(v ? t0 + r : 0) * H + (kv ? k : 0), v);
-        }
-    };
-    grid_dep_wait();   // x may be the previous kernel's output
-    float acc[2][2][4];
-#pragma unroll
-    for (int i = 0; i < 2; ++i)
-#pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-            for (int c = 0; c < 4; ++c) acc[i][j][c] = 0.f;
-#pragma unroll
-    for (int s = 0; s < RM_STAGES - 1; ++s) {
-        if (s < nk) load(s);
-        asm volatile("cp.async.commit_group;" ::: "memory");
+        mbar_init(&sh.acc, 1);
+        sh.abort = 0;
+        fence_barrier_init();
     }
-    for (int kc = 0; kc < nk; ++kc) {
-        asm volatile("cp.async.wait_group %0;" ::"n"(RM_STAGES - 2) : "memory");
-        __syncthreads();   // stage kc landed for all threads; stage kc - 1 is free again
-        if (kc + RM_STAGES - 1 < nk) load(kc + RM_STAGES - 1);
-        asm volatile("cp.async.commit_group;" ::: "memory");
-        const uint16_t* sa = rm_smem + (kc % RM_STAGES) * RM_STAGE_ELEMS;
-        const uint16_t* sb = sa + RM_BM * RM_LD;
-#pragma unroll
-        for (int ks = 0; ks < RM_BK; ks += 16) {
-            uint32_t a[2][4], b[4];
-#pragma unroll
-            for (int i = 0; i < 2; ++i) ldsm_x4(sa + (wm + 16 * i + (lane & 15)) * RM_LD + ks + (lane >> 4) * 8, a[i]);
-            // B is stored [token][k]: matrices (n 0-7, k 0-7), (n 0-7, k 8-15), (n 8-15, k 0-7), (n 8-15, k 8-15)
-            ldsm_x4(sb + (wn + (lane & 7) + ((lane >> 4) << 3)) * RM_LD + ks + ((lane >> 3) & 1) * 8, b);
-#pragma unroll
-            for (int i = 0; i < 2; ++i)
-#pragma unroll
-                for (int j = 0; j < 2; ++j) mma16816<false>(acc[i][j], a[i], b[2 * j], b[2 * j + 1], acc[i][j]);
-        }
+    if (warp == 1) {
+        __syncwarp();
+        tmem_alloc(&sh.tmem, RT_BN);
+        tmem_relinquish();
     }
-    asm volatile("cp.async.wait_group 0;" ::: "memory");
-    // acc[i][j]: rows (experts) wm + 16 i + g (+8), columns (tokens) wn + 8 j + 2 t (+1)
-    const int g = lane >> 2, t = lane & 3;
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sh.tmem;
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmW);
+        tma_prefetch_desc(&tmX);
+        const uint64_t pol = policy_evict_last();
+        grid_dep_wait();   // x may be the previous kernel's output
+        int ks = 0;
+        for (; ks < nk; ++ks) {
+            const int s = ks % RT_NS;
+            if (!mbar_wait(&sh.empty[s], ((uint32_t)(ks / RT_NS) & 1u) ^ 1u, RT_WAIT)) {
+                sh.abort = 1;
+                break;
+            }
+            uint8_t* a = ring + (size_t)s * RT_STAGE;
+            mbar_arrive_expect_tx(&sh.full[s], RT_STAGE);
+            tma_load_2d(a, &tmW, ks * RT_BK, e0, &sh.full[s], pol);
+            tma_load_2d(a + RT_TILE_A, &tmX, ks * RT_BK, t0, &sh.full[s], pol);
+        }
+        // no copy may land after the CTA exits
+        for (int i = 1; i <= RT_NS && ks - i >= 0; ++i) {
+            const int g = ks - i;
+            (void)mbar_wait(&sh.full[g % RT_NS], (uint32_t)(g / RT_NS) & 1u, RT_WAIT);
+        }
+    } else if (warp == 1 && lane == 0) {
+        const uint32_t idesc = idesc_bf16_m128(RT_BN);
+        for (int ks = 0; ks < nk; ++ks) {
+            const int s = ks % RT_NS;
+            if (!mbar_wait(&sh.full[s], (uint32_t)(ks / RT_NS) & 1u, RT_WAIT) || sh.abort) {
+                sh.abort = 1;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t a = smem_u32(ring + (size_t)s * RT_STAGE), b = a + RT_TILE_A;
 #pragma unroll
-    for (int i = 0; i < 2; ++i)
+            for (int kk = 0; kk < RT_BK / 16; ++kk)
+                tc_mma_bf16(tmem, sw128_desc(a + kk * 32), sw128_desc(b + kk * 32), idesc, (ks | kk) != 0);
+            tc_commit(&sh.empty[s]);
+        }
+        tc_commit(&sh.acc);
+        // every MMA is done before tensor memory is released
+        if (!mbar_wait(&sh.acc, 0u, RT_WAIT)) sh.abort = 1;
+    } else if (warp >= 4) {
+        const int q = warp & 3;   // the tensor-memory lane quarter this warp may read
+        const bool ok = mbar_wait(&sh.acc, 0u, RT_WAIT);
+        tc_fence_after();
+        if (__all_sync(0xffffffffu, ok) && !sh.abort) {
+            const int e = e0 + 32 * q + lane;
+            const float bv = (bias && e < E) ? __ldg(bias + e) : 0.f;
+            for (int c0 = 0; c0 < RT_BN && t0 + c0 < T; c0 += 16) {
+                uint32_t v[16];
+                tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)c0, v);
+                tmem_ld_wait();
 #pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-            const int e = e0 + wm + 16 * i + g + 8 * hr;
-            if (e >= E) continue;
-            const float bv = bias ? __ldg(bias + e) : 0.f;
-#pragma unroll
-            for (int j = 0; j < 2; ++j)
-#pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    const int tok = t0 + wn + 8 * j + 2 * t + cc;
-                    if (tok < T) logits[(size_t)tok * E + e] = acc[i][j][2 * hr + cc] + bv;
+                for (int j = 0; j < 16; ++j) {
+                    const int t = t0 + c0 + j;
+                    if (e < E && t < T) logits[(size_t)t * E + e] = __uint_as_float(v[j]) + bv;
                 }
+            }
         }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, RT_BN);
+    }
 }
 
 cudaError_t router_logits_launch(const uint16_t* W, const float* bias, const uint16_t* x, int T, int H, int E,
@@ -253,18 +271,21 @@ cudaError_t router_logits_launch(const uint16_t* W, const float* bias, const uin
     cudaLaunchConfig_t cfg = {};
     if (T > RP_COLS) {
         static SmemLimit limit;
-        cudaError_t e = limit.ensure((const void*)router_logits_mma_kernel, (int)RM_SMEM);
+        cudaError_t e = limit.ensure((const void*)router_logits_tc_kernel, (int)RT_SMEM);
         if (e != cudaSuccess) return e;
-        cfg.gridDim = dim3((unsigned)((E + RM_BM - 1) / RM_BM), (unsigned)((T + RM_BN - 1) / RM_BN));
-        cfg.blockDim = dim3(RM_THREADS);
-        cfg.dynamicSmemBytes = RM_SMEM;
+        CUtensorMap tmW, tmX;
+        if (!make_tmap_bf16(&tmW, W, E, H, RT_BM) || !make_tmap_bf16(&tmX, x, T, H, RT_BN))
+            return cudaErrorInvalidValue;
+        cfg.gridDim = dim3((unsigned)((E + RT_BM - 1) / RT_BM), (unsigned)((T + RT_BN - 1) / RT_BN));
+        cfg.blockDim = dim3(RT_THREADS);
+        cfg.dynamicSmemBytes = RT_SMEM;
         cfg.stream = stream;
         cudaLaunchAttribute at[1];
         at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         at[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = at;
         cfg.numAttrs = 1;
-        return cudaLaunchKernelEx(&cfg, router_logits_mma_kernel, W, bias, x, T, H, E, logits);
+        return cudaLaunchKernelEx(&cfg, router_logits_tc_kernel, tmW, tmX, bias, T, H, E, logits);
     }
     cfg.gridDim = dim3((unsigned)((E + RP_ROWS - 1) / RP_ROWS), (unsigned)((T + RP_COLS - 1) / RP_COLS));
     cfg.blockDim = dim3(RP_THREADS);
