@@ -258,6 +258,7 @@ static cudaError_t launch_t(const GemvParams& p, size_t smem, cudaStream_t strea
     if (e != cudaSuccess) return e;
     const long long npairs = ((p.N + 15) / 16 + 1) / 2;
     const int grid = (int)std::min<long long>(npairs, (long long)sms * std::max(per_sm, 1));
+    (void)cudaGetLastError();   // an earlier call's launch error is not this launch's
     kern<<<grid, GEMV_WARPS * 32, smem, stream>>>(p);
     return cudaGetLastError();
 }

@@ -148,6 +148,7 @@ cudaError_t pack_device_launch(int fmt, const uint8_t* codes, const void* scales
     const long long ngroups = (rows + 15) / 16;
     if (ngroups == 0) return cudaSuccess;
     dim3 grid(rfx_num_chunks(cols), (unsigned)ngroups);
+    (void)cudaGetLastError();   // an earlier call's launch error is not this launch's
     pack_kernel<<<grid, 32, 0, stream>>>(fmt, codes, (const uint8_t*)scales, rows, cols, dst);
     return cudaGetLastError();
 }

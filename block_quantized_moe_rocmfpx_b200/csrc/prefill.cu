@@ -887,6 +887,7 @@ cudaError_t pf_launch(const PfParams& p, int sms, cudaStream_t stream) {
         return cudaErrorInvalidValue;
     const int n = p.T * p.k;
     const dim3 gg((p.E + 7) / 8, (n + PF_SLICE - 1) / PF_SLICE);
+    (void)cudaGetLastError();   // an earlier call's launch error is not this call's
     pf_count_kernel<<<gg, 256, 0, stream>>>(p.idx, n, p.E, p.cnt_part, p.ctrl);
     pf_tiles_kernel<<<1, 1024, 0, stream>>>(p);
     pf_place_kernel<<<gg, 256, 0, stream>>>(p.idx, p.wts, n, p.k, p.E, p.cnt_part, p.off, p.perm_tok, p.perm_w);

@@ -36,6 +36,7 @@ __global__ void __launch_bounds__(256) rms_bf16_kernel(const float* __restrict__
 }
 
 cudaError_t rms_bf16_launch(const float* y, int T, int H, uint16_t* x, cudaStream_t stream) {
+    (void)cudaGetLastError();   // an earlier call's launch error is not this launch's
     rms_bf16_kernel<<<T, 256, 0, stream>>>(y, H, x);
     return cudaGetLastError();
 }
