@@ -56,8 +56,10 @@ KERNEL_SOURCES = {
 # union of experts), and only while the sources still have that digest; after
 # any change the key reads null until the kernel is captured again.
 TRAFFIC = {
-    ("moe_decode", "q1"): ("4c5460ebb606468b", 67_087_616 + 1_176_064, 66_872_368),
-    ("moe_decode", "q4"): ("4c5460ebb606468b", 112_305_408 + 3_629_568, 111_513_792),
+    ("moe_decode", "q1"): ("984674259c5d15be", 67_111_424 + 929_024, 66_872_368),
+    ("moe_decode", "q4"): ("984674259c5d15be", 111_752_192 + 3_782_144, 111_513_792),
+    # both pf_gemm launches of one T = 2048 step (gate/up + down), token batch 0
+    ("prefill", "T2048"): ("ab522f207f7dd16d", 751_524_096 + 42_337_024 + 522_533_120 + 3_903_232, 1_070_858_240),
 }
 
 
