@@ -629,6 +629,7 @@ __device__ void epilogue_a(const MoeParams& p, Shared& sh, const uint8_t* rb, in
                            int lane) {
     const int g = lane >> 2, t = lane & 3;
     const int RB = moe_red_bytes(QC);
+    constexpr bool C1 = QC >= 2;   // the lane's second column (2t + 1) can be live
     float h[2][4];
     float m[2] = {0.f, 0.f};
     bool bad = false;
@@ -640,7 +641,7 @@ __device__ void epilogue_a(const MoeParams& p, Shared& sh, const uint8_t* rb, in
         for (int i = 0; i < 4; ++i) {
             const int col = 2 * t + (i & 1);
             float hv = 0.f;
-            if (col < ncols) {
+            if ((C1 || !(i & 1)) && col < ncols) {
                 const float sc = __int_as_float((127 - sh.xn[sh.st.cols[slot][col]]) << 23);
                 const float gv = G[i] * sc, uv = U[i] * sc;
                 hv = gv >= -64.f ? gv / (1.0f + expf(-gv)) * uv : silu_mul_tail(gv, uv);
@@ -1093,16 +1094,22 @@ __device__ void consumer(const MoeParams& p, Shared& sh, uint8_t* ring, uint8_t*
 // thread's loads (up to XR items) before using any.
 constexpr int XR = 8;
 
+// Column of item i: i / per_col as a multiply and shift, with
+// cdiv = floor(2^32 / per_col) + 1 (exact while i * per_col < 2^32; here
+// i < MOE_MAXT * per_col and per_col = H / 8).
+__device__ __forceinline__ int x_col(int i, uint32_t cdiv) { return (int)__umulhi((uint32_t)i, cdiv); }
+
 // Max |x| of one item per column into sh.xmax (one shared atomic per column
 // the warp's items touch; i0 = the warp's first item, warp-uniform).
-__device__ __forceinline__ void x_max(Shared& sh, const uint4& v, int i0, int lane, int nitems, int per_col) {
+__device__ __forceinline__ void x_max(Shared& sh, const uint4& v, int i0, int lane, int nitems, uint32_t cdiv) {
     const int i = i0 + lane;
     const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
     uint32_t m = 0u;
 #pragma unroll
     for (int e = 0; e < 4; ++e) m = max(m, max((wv[e] << 16) & 0x7fffffffu, wv[e] & 0x7fff0000u));
-    const int cmine = i < nitems ? i / per_col : -1;
-    const int ca = i0 / per_col, cb = min(i0 + 31, nitems - 1) / per_col;
+    const int cmine = i < nitems ? x_col(i, cdiv) : -1;
+    const int ca = x_col(i0, cdiv), cb = x_col(min(i0 + 31, nitems - 1), cdiv);
+#pragma unroll 1
     for (int c = ca; c <= cb; ++c) {
         const uint32_t mc = __reduce_max_sync(0xffffffffu, cmine == c ? m : 0u);
         if (lane == 0 && mc) atomicMax(&sh.xmax[c], mc);
@@ -1111,12 +1118,13 @@ __device__ __forceinline__ void x_max(Shared& sh, const uint4& v, int i0, int la
 
 // Scaled fp16 fragments and block sums of one item, for every gate/up format copy.
 __device__ __forceinline__ void x_put(const MoeParams& p, Shared& sh, uint8_t* xh, float* sx, int sxs, int nxc,
-                                      const uint4& v, int i0, int lane, int nitems, int per_col) {
+                                      const uint4& v, int i0, int lane, int nitems, int per_col, uint32_t cdiv) {
     const int i = i0 + lane;
     const bool in = i < nitems;
-    const int c = in ? i / per_col : 0, j = in ? i - c * per_col : 0;
+    const int c = in ? x_col(i, cdiv) : 0, j = in ? i - c * per_col : 0;
     const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
     const int step = j >> 1, half = j & 1;
+#pragma unroll 1
     for (int ci = 0; ci < nxc; ++ci) {
         const int fmt = p.xf[ci];
         const int sb = s_pos(fmt, j * 8, p.H);
@@ -1177,19 +1185,23 @@ __device__ void chain_rms(const MoeParams& p, Shared& sh, int sid, int nthr) {
 // rounded quotient; unless it lies within half an fp32 ulp (plus that margin)
 // of a bf16 rounding tie, or outside the normal bf16 range, its bf16 through
 // fp32 (two nearest-even steps) equals the quotient's.  Otherwise divide.
+// The division is out of line: it is rare, and inlined at every use it would
+// be most of the kernel's code.
+__device__ __noinline__ uint32_t chain_bf16_div(float y, double r) { return f64_to_bf16_rne((double)y / r); }
+
 __device__ __forceinline__ uint32_t chain_bf16(float y, double r, double ri) {
     const double q = (double)y * ri;
     const unsigned long long b = (unsigned long long)__double_as_longlong(q);
     const int e = (int)((b >> 52) & 0x7FF);
     const long long d = (long long)(b & ((1ull << 45) - 1ull)) - (1ll << 44);
     constexpr long long WIN = (1ll << 28) + 8;
-    if (e < 1023 - 126 || e == 0x7FF || (d < WIN && d > -WIN)) return f64_to_bf16_rne((double)y / r);
+    if (e < 1023 - 126 || e == 0x7FF || (d < WIN && d > -WIN)) return chain_bf16_div(y, r);
     return __bfloat16_as_ushort(__float2bfloat16_rn(__double2float_rn(q)));
 }
 
-// Item i (8 consecutive values of a column) of x as bf16 bits.
-__device__ __forceinline__ uint4 load_item(const MoeParams& p, const Shared& sh, int i, int per_col) {
-    if (!p.xc) return __ldg(reinterpret_cast<const uint4*>(p.x) + i);
+// Item i (8 consecutive values of a column) of the chained input as bf16
+// bits (out of line: one copy of the conversion code for every load site).
+__device__ __forceinline__ uint4 load_item_chained(const MoeParams& p, const Shared& sh, int i, int per_col) {
     const int c = i / per_col;
     const float4 a = __ldg(reinterpret_cast<const float4*>(p.xc) + 2 * i);
     const float4 b = __ldg(reinterpret_cast<const float4*>(p.xc) + 2 * i + 1);
@@ -1200,9 +1212,30 @@ __device__ __forceinline__ uint4 load_item(const MoeParams& p, const Shared& sh,
                       chain_bf16(b.z, r, ri) | (chain_bf16(b.w, r, ri) << 16));
 }
 
+// The items r0 + sid + k * nthr (k < XR) of x as bf16 bits, zero past the
+// end.  The test of the chained input is outside the loads: the plain path is
+// XR loads in flight and nothing else.
+__device__ __forceinline__ void load_round(const MoeParams& p, const Shared& sh, int r0, int sid, int nthr, int nitems,
+                                           int per_col, uint4 v[XR]) {
+    if (!p.xc) {
+#pragma unroll
+        for (int k = 0; k < XR; ++k) {
+            const int i = r0 + sid + k * nthr;
+            v[k] = i < nitems ? __ldg(reinterpret_cast<const uint4*>(p.x) + i) : make_uint4(0u, 0u, 0u, 0u);
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < XR; ++k) {
+            const int i = r0 + sid + k * nthr;
+            v[k] = i < nitems ? load_item_chained(p, sh, i, per_col) : make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
+}
+
 __device__ void stage_x(const MoeParams& p, Shared& sh, uint8_t* xh, int sid, int nthr) {
     const int lane = sid & 31;
     const int per_col = p.H / 8;
+    const uint32_t cdiv = 0xffffffffu / (uint32_t)per_col + 1u;
     const int nitems = p.T * per_col;
     if (p.xc) chain_rms(p, sh, sid, nthr);
     const int nxc = p.nxc;
@@ -1212,15 +1245,11 @@ __device__ void stage_x(const MoeParams& p, Shared& sh, uint8_t* xh, int sid, in
     uint4 v[XR];
     // pass 1: max |x| per column
     for (int r0 = 0; r0 < nitems; r0 += XR * nthr) {
-#pragma unroll
-        for (int k = 0; k < XR; ++k) {
-            const int i = r0 + sid + k * nthr;
-            v[k] = i < nitems ? load_item(p, sh, i, per_col) : make_uint4(0u, 0u, 0u, 0u);
-        }
+        load_round(p, sh, r0, sid, nthr, nitems, per_col, v);
 #pragma unroll
         for (int k = 0; k < XR; ++k) {
             const int i0 = r0 + k * nthr + sid - lane;
-            if (i0 < nitems) x_max(sh, v[k], i0, lane, nitems, per_col);
+            if (i0 < nitems) x_max(sh, v[k], i0, lane, nitems, cdiv);
         }
     }
     asm volatile("bar.sync 1, %0;" ::"r"(nthr) : "memory");
@@ -1232,17 +1261,11 @@ __device__ void stage_x(const MoeParams& p, Shared& sh, uint8_t* xh, int sid, in
     asm volatile("bar.sync 1, %0;" ::"r"(nthr) : "memory");
     // pass 2: scale, round to fp16, write fragments and block sums
     for (int r0 = 0; r0 < nitems; r0 += XR * nthr) {
-        if (!one_round) {
-#pragma unroll
-            for (int k = 0; k < XR; ++k) {
-                const int i = r0 + sid + k * nthr;
-                v[k] = i < nitems ? load_item(p, sh, i, per_col) : make_uint4(0u, 0u, 0u, 0u);
-            }
-        }
+        if (!one_round) load_round(p, sh, r0, sid, nthr, nitems, per_col, v);
 #pragma unroll
         for (int k = 0; k < XR; ++k) {
             const int i0 = r0 + k * nthr + sid - lane;
-            if (i0 < nitems) x_put(p, sh, xh, sx, sxs, nxc, v[k], i0, lane, nitems, per_col);
+            if (i0 < nitems) x_put(p, sh, xh, sx, sxs, nxc, v[k], i0, lane, nitems, per_col, cdiv);
         }
     }
 }
