@@ -155,24 +155,23 @@ __device__ void build_slots(const MoeParams& p, SlotTable& S, const Routing& rt)
     const int lane = threadIdx.x & 31;
     const int n = p.T * p.k;
     const int base = p.has_shared ? 1 : 0;
+    // entry i is (column i / k, choice i % k); the quotient as a multiply-shift
+    // (exact for i < 2^32 / k).  The passes below are loops of one copy with
+    // the entry's slot kept in the table: this code runs once per launch, with
+    // its instructions not yet in the cache.
+    const uint32_t kdiv = 0xffffffffu / (uint32_t)p.k + 1u;
     S.mask[lane] = 0u;
     for (int s = lane; s < MOE_MAXS; s += 32) S.colmask[s] = 0u;
-    if (lane < n) { S.idx[lane] = rt.e0; S.w[lane / p.k][lane % p.k] = rt.w0; }
-    if (lane + 32 < n) { S.idx[lane + 32] = rt.e1; S.w[(lane + 32) / p.k][(lane + 32) % p.k] = rt.w1; }
     __syncwarp();
-    bool ok[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int i = lane + 32 * h;
-        ok[h] = false;
-        if (i >= n) continue;
-        const int c = i / p.k, j = i - c * p.k;
-        const int e = S.idx[i];
-        const bool v = e >= 0 && e < p.E;
-        if (!v) set_error(p.ctrl, MOE_ERR_EXPERT);
-        ok[h] = v;
+#pragma unroll 1
+    for (int i = lane; i < n; i += 32) {
+        const int e = i < 32 ? rt.e0 : rt.e1;
+        const int c = (int)__umulhi((uint32_t)i, kdiv), j = i - c * p.k;
+        S.idx[i] = e;
+        S.w[c][j] = i < 32 ? rt.w0 : rt.w1;
         S.tslot[c][j] = -1;
-        if (v) atomicOr(&S.mask[e >> 5], 1u << (e & 31));
+        if (e >= 0 && e < p.E) atomicOr(&S.mask[e >> 5], 1u << (e & 31));
+        else set_error(p.ctrl, MOE_ERR_EXPERT);
     }
     __syncwarp();
     {
@@ -187,27 +186,25 @@ __device__ void build_slots(const MoeParams& p, SlotTable& S, const Routing& rt)
         if (lane == 31) S.nslots = base + incl;
     }
     __syncwarp();
-    int slot_of[2] = {-1, -1};
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        if (!ok[h]) continue;
-        const int i = lane + 32 * h;
+#pragma unroll 1
+    for (int i = lane; i < n; i += 32) {
         const int e = S.idx[i];
+        if (e < 0 || e >= p.E) continue;
+        const int c = (int)__umulhi((uint32_t)i, kdiv), j = i - c * p.k;
         const int s = base + S.prefix[e >> 5] + __popc(S.mask[e >> 5] & ((1u << (e & 31)) - 1u));
-        slot_of[h] = s;
         S.expert[s] = e;
-        atomicOr(&S.colmask[s], 1u << (i / p.k));
+        S.tslot[c][j] = (signed char)s;
+        atomicOr(&S.colmask[s], 1u << c);
     }
     __syncwarp();
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        if (slot_of[h] < 0) continue;
-        const int i = lane + 32 * h;
-        const int c = i / p.k, j = i - c * p.k, s = slot_of[h];
+#pragma unroll 1
+    for (int i = lane; i < n; i += 32) {
+        const int c = (int)__umulhi((uint32_t)i, kdiv), j = i - c * p.k;
+        const int s = S.tslot[c][j];
+        if (s < 0) continue;
         const unsigned cm = S.colmask[s];
         const int pos = __popc(cm & ((1u << c) - 1u));   // columns ascend within a slot
         S.cols[s][pos] = (signed char)c;
-        S.tslot[c][j] = (signed char)s;
         S.tpos[c][j] = (signed char)pos;
         if (pos == 0) S.ncols[s] = __popc(cm);   // several entries may write the same value
     }
@@ -1212,6 +1209,12 @@ __device__ __forceinline__ uint4 load_item_chained(const MoeParams& p, const Sha
                       chain_bf16(b.z, r, ri) | (chain_bf16(b.w, r, ri) << 16));
 }
 
+// Item i of x as bf16 bits.
+__device__ __forceinline__ uint4 load_item(const MoeParams& p, const Shared& sh, int i, int per_col) {
+    if (!p.xc) return __ldg(reinterpret_cast<const uint4*>(p.x) + i);
+    return load_item_chained(p, sh, i, per_col);
+}
+
 // The items r0 + sid + k * nthr (k < XR) of x as bf16 bits, zero past the
 // end.  The test of the chained input is outside the loads: the plain path is
 // XR loads in flight and nothing else.
@@ -1241,7 +1244,6 @@ __device__ void stage_x(const MoeParams& p, Shared& sh, uint8_t* xh, int sid, in
     const int nxc = p.nxc;
     float* sx = (float*)(xh + nxc * p.T * p.x_stride);
     const int sxs = moe_sxs(p.H);
-    const bool one_round = nitems <= XR * nthr;   // then pass 2 reuses the loaded items
     uint4 v[XR];
     // pass 1: max |x| per column
     for (int r0 = 0; r0 < nitems; r0 += XR * nthr) {
@@ -1259,14 +1261,18 @@ __device__ void stage_x(const MoeParams& p, Shared& sh, uint8_t* xh, int sid, in
         sh.xn[sid] = max(-100, min(100, n));
     }
     asm volatile("bar.sync 1, %0;" ::"r"(nthr) : "memory");
-    // pass 2: scale, round to fp16, write fragments and block sums
-    for (int r0 = 0; r0 < nitems; r0 += XR * nthr) {
-        if (!one_round) load_round(p, sh, r0, sid, nthr, nitems, per_col, v);
-#pragma unroll
-        for (int k = 0; k < XR; ++k) {
-            const int i0 = r0 + k * nthr + sid - lane;
-            if (i0 < nitems) x_put(p, sh, xh, sx, sxs, nxc, v[k], i0, lane, nitems, per_col, cdiv);
-        }
+    // pass 2: scale, round to fp16, write fragments and block sums.  One copy
+    // of the code (it runs once per launch, its instructions not yet cached):
+    // the items are read again (cache hits), each one item ahead of its use.
+    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+    int i0 = sid - lane;   // the warp's first item of the round
+    v[0] = i0 + lane < nitems ? load_item(p, sh, i0 + lane, per_col) : z;
+#pragma unroll 1
+    for (; i0 < nitems; i0 += nthr) {
+        const int in = i0 + nthr + lane;
+        v[1] = in < nitems ? load_item(p, sh, in, per_col) : z;
+        x_put(p, sh, xh, sx, sxs, nxc, v[0], i0, lane, nitems, per_col, cdiv);
+        v[0] = v[1];
     }
 }
 
