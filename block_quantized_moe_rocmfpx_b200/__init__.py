@@ -68,6 +68,7 @@ _ws_bytes = _proto("moe_ffn_workspace_bytes", _sz, [_vp, _i32])
 _ws_init = _proto("rfx_ws_init", _i32, [_vp, _sz, _vp])
 _ws_status = _proto("rfx_ws_status", _i32, [_vp, _vp])
 _forward = _proto("moe_ffn_forward", _i32, [_vp, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp])
+_forward_logits = _proto("moe_ffn_forward_logits", _i32, [_vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp])
 _host_scratch = _proto("moe_ffn_host_scratch_bytes", _sz, [_vp, _i32])
 _forward_host = _proto("moe_ffn_forward_host", _i32, [_vp, _vp, _vp, _i32, _vp, _vp, _sz, _vp])
 _forward_static = _proto("moe_ffn_forward_static", _i32, [_vp, _vp, _i32, _vp, _vp, _vp, _vp])
@@ -91,7 +92,7 @@ _pf_view = _proto("moe_prefill_view", _i32, [_vp, _i32, _vp, ctypes.POINTER(moe_
 
 EXPORTED = ["rfx_last_error", "rfx_packed_bytes", "rfx_pack", "rfx_unpack", "rfx_pack_device", "moe_router_topk",
             "rfx_gemv_q", "moe_layer_create", "moe_layer_create_mix", "moe_layer_destroy", "moe_ffn_workspace_bytes", "rfx_ws_init",
-            "rfx_ws_status", "moe_ffn_forward", "moe_ffn_forward_static", "moe_rms_norm_bf16",
+            "rfx_ws_status", "moe_ffn_forward", "moe_ffn_forward_logits", "moe_ffn_forward_static", "moe_rms_norm_bf16",
             "moe_stack_workspace_bytes", "moe_stack_forward", "moe_prefill_workspace_bytes", "moe_ffn_prefill",
             "moe_prefill_workspace_bytes_ex", "moe_ffn_prefill_ex",
             "moe_prefill_view", "moe_router_logits", "moe_router_project_topk",
@@ -229,6 +230,13 @@ def moe_ffn_forward(handle: int, x, T: int, idx, w, y, ws, stream=None):
                     _stream(stream)))
 
 
+def moe_ffn_forward_logits(handle: int, x, T: int, logits, idx, w, y, ws, stream=None):
+    """Router top-k of logits (fp32 [T][E]) into idx / w, then the MoE FFN
+    (moe_router_topk + moe_ffn_forward in one call)."""
+    _check(_forward_logits(handle, _ptr(x), T, _ptr(logits), _ptr(idx), _ptr(w), _ptr(y), _ptr(ws),
+                           ws.numel() * ws.element_size(), _stream(stream)))
+
+
 def moe_ffn_host_scratch_bytes(handle: int, T: int) -> int:
     return int(_host_scratch(handle, T))
 
@@ -353,6 +361,13 @@ class MoeLayer:
         if T > self.max_T:
             raise ValueError(f"T={T} > max_T={self.max_T}")
         moe_ffn_forward(self.handle, x, T, idx, w, y, self.ws, stream)
+
+    def forward_logits(self, x, logits, idx, w, y, stream=None):
+        """Routing from the logits, then the FFN (moe_ffn_forward_logits)."""
+        T = x.shape[0]
+        if T > self.max_T:
+            raise ValueError(f"T={T} > max_T={self.max_T}")
+        moe_ffn_forward_logits(self.handle, x, T, logits, idx, w, y, self.ws, stream)
 
     def forward_host(self, x, logits, y, stream=None):
         """Router + FFN from host buffers (see moe_ffn_forward_host); the device

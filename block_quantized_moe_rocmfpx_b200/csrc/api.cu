@@ -425,6 +425,20 @@ extern "C" int moe_ffn_forward(const moe_layer* layer, const void* x, int T, con
     return e == cudaSuccess ? RFX_OK : cuda_fail("moe_ffn_forward", e);
 }
 
+// The routed step from the logits: the router launch, then the FFN launch.
+// (Routing inside the FFN kernel, in its otherwise idle warps, was measured
+// slower: the selection runs once per launch from a cold instruction cache
+// and sits on the kernel's critical path.)
+extern "C" int moe_ffn_forward_logits(const moe_layer* layer, const void* x, int T, const float* logits, int32_t* idx,
+                                      float* w, float* y, void* ws, size_t ws_bytes, void* stream) {
+    if (!layer) return rfx_fail(RFX_EINVAL, "moe_ffn_forward_logits: null layer");
+    if (T == 0) return RFX_OK;   // no token columns: nothing to do
+    if (!logits || !idx || !w) return rfx_fail(RFX_EINVAL, "moe_ffn_forward_logits: null pointer");
+    int rc = moe_router_topk(logits, T, layer->d.E, layer->d.k, idx, w, stream);
+    if (rc != RFX_OK) return rc;
+    return moe_ffn_forward(layer, x, T, idx, w, y, ws, ws_bytes, stream);
+}
+
 // ------------------------------------------------------------ host buffers ---
 
 namespace {
@@ -511,8 +525,6 @@ extern "C" int moe_ffn_forward_host(const moe_layer* layer, const void* x, const
     if (side && e == cudaSuccess) e = cudaEventRecord(L->ev_ready[s], us);
     if (side && e == cudaSuccess) e = cudaStreamWaitEvent(st, L->ev_ready[s], 0);
     if (e != cudaSuccess) return cuda_fail("moe_ffn_forward_host", e);
-    int rc = moe_router_topk(ld, T, d.E, d.k, idx, w, stream);
-    if (rc != RFX_OK) return rc;
     // decode: pinned host y that the device can address (page-locked and
     // mapped, as cudaHostAlloc / cudaHostRegister memory is under unified
     // addressing) takes the kernel's combine stores directly, with no copy
@@ -524,7 +536,7 @@ extern "C" int moe_ffn_forward_host(const moe_layer* layer, const void* x, const
         else
             (void)cudaGetLastError();   // not an error: pageable memory takes the copy below
     }
-    rc = moe_ffn_forward(layer, xd, T, idx, w, ydev ? ydev : yd, b + S.ffn, S.x[0], stream);
+    int rc = moe_ffn_forward_logits(layer, xd, T, ld, idx, w, ydev ? ydev : yd, b + S.ffn, S.x[0], stream);
     if (rc != RFX_OK) return rc;
     if (side) {
         e = cudaEventRecord(L->ev_free[s], st);

@@ -287,6 +287,17 @@ int moe_ffn_forward(const moe_layer* layer, const void* x, int T, const int32_t*
                     float* y, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * The routed step from the router logits ([AI] "Lucebox 的优化三板斧": the
+ * top-k routing kernel in front of the expert FFN): moe_router_topk of
+ * logits (device fp32 [T][E]) into idx (device int32 [T][k]) and w (device
+ * fp32 [T][k]), caller-owned outputs, then moe_ffn_forward; two launches on
+ * `stream`.  Arguments, workspace and limits as moe_ffn_forward (T > 8: the
+ * prefill path, ws sized by moe_ffn_workspace_bytes).
+ */
+int moe_ffn_forward_logits(const moe_layer* layer, const void* x, int T, const float* logits, int32_t* idx,
+                           float* w, float* y, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * The same step from host buffers: x (bf16 bits [T][H]) and the router
  * logits (fp32 [T][E]) are copied host -> device, moe_router_topk and
  * moe_ffn_forward run, and y (fp32 [T][H]) is copied device -> host (one
