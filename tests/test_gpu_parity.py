@@ -292,6 +292,39 @@ def test_forward_host_pageable_buffers(full_layer):
     assert torch.equal(yh, y.cpu())
 
 
+def test_forward_host_mixed_paths(full_layer):
+    """Back-to-back host-buffer calls on one layer that alternate the buffer
+    kinds: all page-locked (y stored by the kernel straight into host memory),
+    page-locked inputs with pageable y (y copied back), all pageable; no
+    synchronisation between the calls, every y the device path's bits for its
+    own inputs."""
+    ml = full_layer.moe_layer()
+    T, n = 2, 6
+    Ls = [synth.logits(12, 0, 300 + 7 * i, T, 256, 1.1) for i in range(n)]
+    xbs = [synth.x_bf16(12, 300 + 7 * i, T, 4096) for i in range(n)]
+    ys = []
+    for i in range(n):
+        pin_in, pin_out = i % 3 != 2, i % 3 == 0
+        xh = torch.from_numpy(xbs[i]).view(torch.bfloat16)
+        lh = torch.from_numpy(Ls[i])
+        yh = torch.full((T, 4096), float("nan"), dtype=torch.float32)
+        if pin_in:
+            xh, lh = xh.pin_memory(), lh.pin_memory()
+        if pin_out:
+            yh = yh.pin_memory()
+        ml.forward_host(xh, lh, yh)
+        ys.append((yh, xh, lh))
+    torch.cuda.synchronize()
+    assert ml.host_status() == rfx.RFX_OK
+    for i in range(n):
+        idx = torch.empty((T, 6), dtype=torch.int32, device=DEV)
+        w = torch.empty((T, 6), dtype=torch.float32, device=DEV)
+        y = torch.empty((T, 4096), dtype=torch.float32, device=DEV)
+        rfx.moe_router_topk(to_dev(Ls[i]), 6, idx, w)
+        ml.forward(to_dev(xbs[i], torch.bfloat16), idx, w, y)
+        assert torch.equal(ys[i][0], y.cpu()), f"call {i}"
+
+
 def test_forward_host_prefill_path():
     H, I, E, k, T = 512, 256, 16, 4, 40
     lay = SynthLayer(29, 0, H, I, E, k)
