@@ -266,10 +266,17 @@ def test_zero_token_calls_are_noops():
         assert lib.moe_ffn_prefill(ctypes.c_void_p(h), None, 0, None, None, None, None, 0, None) == rfx.RFX_OK
         assert lib.moe_ffn_forward_static(ctypes.c_void_p(h), None, 0, None, None, None, None) == rfx.RFX_OK
         assert lib.moe_ffn_forward_host(ctypes.c_void_p(h), None, None, 0, None, None, 0, None) == rfx.RFX_OK
+        assert lib.moe_ffn_forward_logits(ctypes.c_void_p(h), None, 0, None, None, None, None, None, 0,
+                                          None) == rfx.RFX_OK
         arr = (ctypes.c_void_p * 1)(h)
         assert lib.moe_stack_forward(arr, 1, None, None, 0, None, None, 0, None) == rfx.RFX_OK
         # a null layer is still an error
         assert lib.moe_ffn_forward(None, None, 0, None, None, None, None, 0, None) == rfx.RFX_EINVAL
+        assert lib.moe_ffn_forward_logits(None, None, 1, None, None, None, None, None, 0, None) == rfx.RFX_EINVAL
+        # the call from the logits checks its routing buffers before any launch
+        assert lib.moe_ffn_forward_logits(ctypes.c_void_p(h), None, 1, None, None, None, None, None, 0,
+                                          None) == rfx.RFX_EINVAL
+        assert "null pointer" in rfx.rfx_last_error()
     finally:
         rfx.moe_layer_destroy(h)
 
