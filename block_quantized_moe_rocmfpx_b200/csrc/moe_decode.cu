@@ -1244,6 +1244,7 @@ __device__ void stage_x(const MoeParams& p, Shared& sh, uint8_t* xh, int sid, in
     const int nxc = p.nxc;
     float* sx = (float*)(xh + nxc * p.T * p.x_stride);
     const int sxs = moe_sxs(p.H);
+    const bool one_round = nitems <= XR * nthr;   // then pass 2 reuses the loaded items
     uint4 v[XR];
     // pass 1: max |x| per column
     for (int r0 = 0; r0 < nitems; r0 += XR * nthr) {
@@ -1263,16 +1264,21 @@ __device__ void stage_x(const MoeParams& p, Shared& sh, uint8_t* xh, int sid, in
     asm volatile("bar.sync 1, %0;" ::"r"(nthr) : "memory");
     // pass 2: scale, round to fp16, write fragments and block sums.  One copy
     // of the code (it runs once per launch, its instructions not yet cached):
-    // the items are read again (cache hits), each one item ahead of its use.
-    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-    int i0 = sid - lane;   // the warp's first item of the round
-    v[0] = i0 + lane < nitems ? load_item(p, sh, i0 + lane, per_col) : z;
+    // a rolled loop over the round's items.  With one round the items are
+    // still in registers from pass 1 (picked with static indices); else they
+    // are loaded again.
+    for (int r0 = 0; r0 < nitems; r0 += XR * nthr) {
+        if (!one_round) load_round(p, sh, r0, sid, nthr, nitems, per_col, v);
 #pragma unroll 1
-    for (; i0 < nitems; i0 += nthr) {
-        const int in = i0 + nthr + lane;
-        v[1] = in < nitems ? load_item(p, sh, in, per_col) : z;
-        x_put(p, sh, xh, sx, sxs, nxc, v[0], i0, lane, nitems, per_col, cdiv);
-        v[0] = v[1];
+        for (int k = 0; k < XR; ++k) {
+            const int i0 = r0 + k * nthr + sid - lane;   // warp-uniform
+            if (i0 >= nitems) break;
+            uint4 cur = v[0];
+#pragma unroll
+            for (int j = 1; j < XR; ++j)
+                if (k == j) cur = v[j];
+            x_put(p, sh, xh, sx, sxs, nxc, cur, i0, lane, nitems, per_col, cdiv);
+        }
     }
 }
 
