@@ -56,8 +56,8 @@ KERNEL_SOURCES = {
 # union of experts), and only while the sources still have that digest; after
 # any change the key reads null until the kernel is captured again.
 TRAFFIC = {
-    ("moe_decode", "q1"): ("4c1b402202f69b15", 67_081_728 + 926_208, 66_872_368),
-    ("moe_decode", "q4"): ("4c1b402202f69b15", 111_701_248 + 2_981_376, 111_513_792),
+    ("moe_decode", "q1"): ("557fce27bf9ab819", 67_082_240 + 866_816, 66_872_368),
+    ("moe_decode", "q4"): ("557fce27bf9ab819", 111_705_856 + 3_130_368, 111_513_792),
     # both pf_gemm launches of one T = 2048 step (gate/up + down), token batch 0
     ("prefill", "T2048"): ("ab522f207f7dd16d", 751_524_096 + 42_337_024 + 522_533_120 + 3_903_232, 1_070_858_240),
 }

@@ -1197,7 +1197,7 @@ __device__ __forceinline__ uint32_t chain_bf16(float y, double r, double ri) {
 }
 
 // Item i (8 consecutive values of a column) of the chained input as bf16
-// bits (out of line: one copy of the conversion code for every load site).
+// bits (inlined only in the chained branch of load_round).
 __device__ __forceinline__ uint4 load_item_chained(const MoeParams& p, const Shared& sh, int i, int per_col) {
     const int c = i / per_col;
     const float4 a = __ldg(reinterpret_cast<const float4*>(p.xc) + 2 * i);
@@ -1207,12 +1207,6 @@ __device__ __forceinline__ uint4 load_item_chained(const MoeParams& p, const Sha
                       chain_bf16(a.z, r, ri) | (chain_bf16(a.w, r, ri) << 16),
                       chain_bf16(b.x, r, ri) | (chain_bf16(b.y, r, ri) << 16),
                       chain_bf16(b.z, r, ri) | (chain_bf16(b.w, r, ri) << 16));
-}
-
-// Item i of x as bf16 bits.
-__device__ __forceinline__ uint4 load_item(const MoeParams& p, const Shared& sh, int i, int per_col) {
-    if (!p.xc) return __ldg(reinterpret_cast<const uint4*>(p.x) + i);
-    return load_item_chained(p, sh, i, per_col);
 }
 
 // The items r0 + sid + k * nthr (k < XR) of x as bf16 bits, zero past the
